@@ -1,0 +1,175 @@
+"""Seeded synthetic inputs and workload definitions.
+
+This module is shared by the tests, the smoke check and the benchmark. It
+holds only shapes, parameters and seeded random draws (numpy PCG64) -- none
+of the method's arithmetic -- so that the CUDA path and the CPU oracle can
+consume identical bytes while sharing no code.
+
+Distributions follow the workloads described on the pages: fp16 K/V drawn
+from N(0,1) with a few strongly scaled outlier channels (the channel-wise
+outliers that motivate the outlier-aware rotation of "RotateKV: Accurate and
+Robust 2-Bit KV Cache Quantization for LLMs via Outlier-Aware Adaptive
+Rotations", abstract), heavy-tailed Student-t vectors for the IsoQuant batch
+("KV缓存压缩技术：IsoQuant在大语言模型中的应用", §7: batch 8192, d = 128), and
+seeded unit quaternions for its 4-D blocks (§2.1). No dataset is used.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field, replace
+from typing import Optional
+
+import numpy as np
+
+_CHUNK = 1 << 24  # elements drawn per numpy call (bounds host memory)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    T: int  # tokens encoded (prefill) / cache slots for scoring
+    D: int = 128
+    rot: str = "fwht_head"  # none | fwht_head | fwht_group | iso
+    quant: str = "minmax"  # minmax | codebook
+    bits: int = 2
+    group: int = 128
+    group_heads: int = 1
+    rope_k: bool = True
+    n_sink: int = 0
+    perm: bool = False
+    dist: str = "normal_outliers"  # normal_outliers | student_t
+    outliers: tuple = ("pairs", 0.01, 10.0, 50.0)
+    seed: int = 0
+    Hq: int = 0  # query heads for scoring (0: no score)
+    append: int = 0  # tokens appended after the prefill (decode step)
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def n_vectors(self) -> int:
+        return self.B * self.H * self.T
+
+
+WORKLOADS = {
+    # 1 layer, batch 1, 8 heads x 128, 256 tokens; 4 outlier channels x20 per
+    # head; FWHT over head_dim; 4-bit min-max, group 128.
+    "tiny": Workload("tiny", B=1, H=8, T=256, bits=4, group=128, outliers=("per_head", 4, 20.0, 20.0),
+                     seed=1),
+    # Llama-2-7B-shaped MHA layer: batch 8, 32 heads, 4096 tokens; 1 % of the
+    # (head, channel) pairs scaled by U[10, 50]; abs-max permutation; 2-bit
+    # group 64; first 4 tokens kept in fp16.
+    "llama2_7b_mha": Workload("llama2_7b_mha", B=8, H=32, T=4096, bits=2, group=64, n_sink=4, perm=True,
+                              seed=2),
+    # Llama-3-8B-shaped GQA layer: batch 4, 8 KV heads, 32768 tokens; FWHT
+    # over the 8 heads x 128 = 1024 channels before RoPE; 2-bit group 128.
+    "llama3_8b_gqa": Workload("llama3_8b_gqa", B=4, H=8, T=32768, rot="fwht_group", group_heads=8, bits=2,
+                              group=128, seed=3),
+    # IsoQuant-style batch: 8192 x 2048 vectors of d = 128, Student-t(4);
+    # 3-bit Lloyd-Max codebook for N(0, 1/128).
+    "isoquant_batch": Workload("isoquant_batch", B=8192, H=1, T=2048, rot="iso", quant="codebook", bits=3,
+                               rope_k=False, dist="student_t", seed=4),
+    # Decode step: batch 64, 32 heads, 8192-token 2-bit cache encoded as in
+    # the Llama-2-7B workload, plus one appended token; fp32 scores.
+    "decode_score": Workload("decode_score", B=64, H=32, T=8192, bits=2, group=64, n_sink=4, perm=True,
+                             seed=5, Hq=32, append=1),
+    # Decode step at the Llama-3-8B shape: 8 KV heads, 32 query heads (GQA
+    # 4:1), 32768 cached tokens + 1 appended, head-dim FWHT, 2-bit group 128.
+    "llama3_8b_gqa_score": Workload("llama3_8b_gqa_score", B=4, H=8, T=32768, bits=2, group=128, n_sink=4,
+                                    seed=6, Hq=32, append=1),
+}
+
+
+def scaled(w: Workload, **kw) -> Workload:
+    """Same workload with some fields replaced (e.g. fewer tokens)."""
+    return replace(w, **kw)
+
+
+def _rng(seed: int, stream: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64([seed, stream]))
+
+
+def _normal_f16(rng, n: int) -> np.ndarray:
+    out = np.empty(n, np.float16)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        out[s:e] = rng.standard_normal(e - s, dtype=np.float32)
+    return out
+
+
+def _student_f16(rng, n: int, nu: float) -> np.ndarray:
+    out = np.empty(n, np.float16)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        out[s:e] = rng.standard_t(nu, e - s)
+    return out
+
+
+def outlier_scales(H: int, D: int, spec, rng) -> np.ndarray:
+    """[H][D] float32 multipliers (1 for ordinary channels)."""
+    sc = np.ones((H, D), np.float32)
+    kind = spec[0]
+    if kind == "per_head":  # k channels per head, fixed factor
+        _, k, lo, hi = spec
+        for h in range(H):
+            ch = rng.choice(D, size=k, replace=False)
+            sc[h, ch] = rng.uniform(lo, hi, size=k) if hi > lo else lo
+    elif kind == "pairs":  # a fraction of all (head, channel) pairs, U[lo, hi]
+        _, frac, lo, hi = spec
+        k = int(math.ceil(frac * H * D))
+        idx = rng.choice(H * D, size=k, replace=False)
+        sc.reshape(-1)[idx] = rng.uniform(lo, hi, size=k).astype(np.float32)
+    elif kind == "none":
+        pass
+    else:
+        raise ValueError(kind)
+    return sc
+
+
+def kv_tensor(w: Workload, which: str, T: Optional[int] = None, B: Optional[int] = None) -> np.ndarray:
+    """fp16 [B][H][T][D] tensor for K ('k'), V ('v') or the tokens appended
+    after a prefill ('k_append', 'v_append'; same outlier channels as K / V).
+    A smaller T or B draws a smaller tensor with the same recipe."""
+    T = w.T if T is None else T
+    B = w.B if B is None else B
+    stream = {"k": 1, "v": 2, "k_append": 3, "v_append": 4}[which]
+    rng = _rng(w.seed, stream)
+    n = B * w.H * T * w.D
+    if w.dist == "student_t":
+        x = _student_f16(rng, n, 4.0).reshape(B, w.H, T, w.D)
+        return x
+    x = _normal_f16(rng, n).reshape(B, w.H, T, w.D)
+    sc = outlier_scales(w.H, w.D, w.outliers, _rng(w.seed, 10 + stream % 2))
+    for h, c in zip(*np.nonzero(sc != 1.0)):
+        x[:, h, :, c] = (x[:, h, :, c].astype(np.float32) * sc[h, c]).astype(np.float16)
+    return x
+
+
+def queries(w: Workload, B: Optional[int] = None) -> np.ndarray:
+    """fp16 [B][Hq][D] query vectors, N(0,1) (taken as already RoPE'd)."""
+    B = w.B if B is None else B
+    rng = _rng(w.seed, 20)
+    return _normal_f16(rng, B * w.Hq * w.D).reshape(B, w.Hq, w.D)
+
+
+def unit_quaternions(n: int, seed: int, stream: int) -> np.ndarray:
+    """[n][4] float32 (real, i, j, k): 4 iid N(0,1) normalised in float64."""
+    g = _rng(seed, stream).standard_normal((n, 4))
+    g /= np.linalg.norm(g, axis=1, keepdims=True)
+    return g.astype(np.float32)
+
+
+def iso_tables(w: Workload):
+    """(qL, qR) for the IsoQuant rotation: one unit quaternion pair per 4-D block."""
+    return unit_quaternions(w.D // 4, w.seed, 30), unit_quaternions(w.D // 4, w.seed, 31)
+
+
+def random_perm(H: int, D: int, seed: int) -> np.ndarray:
+    """[H][D] int16, a seeded random permutation per head (any permutation
+    exercises the permutation step; calibrated ones are computed elsewhere)."""
+    rng = _rng(seed, 40)
+    return np.stack([rng.permutation(D) for _ in range(H)]).astype(np.int16)
+
+
+def positions(t0: int, T: int) -> np.ndarray:
+    return np.arange(t0, t0 + T, dtype=np.int64)
