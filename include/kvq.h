@@ -1,0 +1,179 @@
+/*
+ * kvq.h -- C ABI of libkvq: rotation + low-bit quantization of an LLM's fp16
+ * KV cache on one NVIDIA B200 (sm_100a), its inverse, and the fused
+ * decode-step q.K^T score.
+ *
+ * Pages the operations come from (title, section):
+ *   [RoPE-KV]  "RoPE启发的KV缓存压缩技术解析"
+ *   [EliteKV]  "EliteKV - RoPE频率选择与低秩投影"
+ *   [IsoQuant] "KV缓存压缩技术：IsoQuant在大语言模型中的应用"
+ *   [RotateKV] "RotateKV: Accurate and Robust 2-Bit KV Cache Quantization for
+ *              LLMs via Outlier-Aware Adaptive Rotations"
+ *
+ * Conventions for every entry point:
+ *  - Tensor pointers are DEVICE pointers owned by the caller unless a
+ *    parameter says "host". The library allocates no device memory, keeps
+ *    only a per-device error word (see kvq_check), never synchronises the
+ *    stream except in kvq_check, and is safe to call from several threads.
+ *  - Arguments are validated on the host before anything is launched; a bad
+ *    argument returns a status and launches nothing.
+ *  - Layouts are dense and row-major. fp16 is IEEE binary16.
+ *  - Inputs holding NaN/Inf, or whose rotated values exceed the fp16 range
+ *    (|v| > 65504, so the fp16 zero/scale overflow), give unspecified codes
+ *    but never out-of-bounds accesses.
+ *  - Output buffers must not overlap inputs.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* kvq_stream_t;
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID = 1,     /* null pointer, bad shape or range */
+  KVQ_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim, bits, combination) */
+  KVQ_ERR_ALIGN = 3,       /* a pointer is not aligned as required below */
+  KVQ_ERR_CUDA = 4,        /* a CUDA call or launch failed */
+  KVQ_ERR_TIMEOUT = 5      /* a kernel gave up waiting on a copy (from kvq_check) */
+} kvq_status;
+
+/* Rotation applied before quantization. */
+enum {
+  KVQ_ROT_NONE = 0,       /* quantize the (RoPE'd) vector as is */
+  KVQ_ROT_FWHT_HEAD = 1,  /* [RotateKV] RoPE -> channel permutation -> normalised FWHT over head_dim */
+  KVQ_ROT_FWHT_GROUP = 2, /* [RotateKV] pre-RoPE grouped-head rotation: permutation -> normalised FWHT
+                             over group_heads*head_dim channels (the heads of one token concatenated)
+                             -> RoPE on each head slice */
+  KVQ_ROT_ISO_SO4 = 3     /* [IsoQuant §2.2, §3.1] norm split rho = ||x||, x/(rho+1e-8), then
+                             w = qL (x) v (x) qR on each 4-D block v */
+};
+
+/* Scalar quantizer. */
+enum {
+  KVQ_Q_MINMAX = 0,  /* per-token per-group asymmetric min-max, fp16 (scale, zero); with
+                        rot in {NONE, FWHT_HEAD, FWHT_GROUP} */
+  KVQ_Q_CODEBOOK = 1 /* fixed scalar codebook (Lloyd-Max, [IsoQuant §3.1]); with rot = ISO_SO4 */
+};
+
+/* Which packed buffer kvq_packed_bytes sizes. */
+enum { KVQ_FIELD_CODES = 0, KVQ_FIELD_SCALE_ZERO = 1, KVQ_FIELD_SINK = 2, KVQ_FIELD_NORM = 3 };
+
+typedef struct {
+  int32_t batch;       /* B > 0 */
+  int32_t heads;       /* H > 0: KV heads */
+  int32_t head_dim;    /* D: 64 or 128 (128 only for FWHT_GROUP) */
+  int32_t tokens;      /* T >= 0: tokens in this call (T = 0 is a no-op) */
+  int32_t t0;          /* first cache slot written/read; also the RoPE position of token 0 */
+  int32_t t_cap;       /* cache capacity in slots; t0 + T <= t_cap */
+  int32_t bits;        /* 2, 3 or 4 */
+  int32_t group;       /* min-max group size in channels: 32, 64 or 128, dividing head_dim
+                          (at least head_dim*group_heads/128 channels for FWHT_GROUP) */
+  int32_t group_heads; /* FWHT_GROUP: 2, 4 or 8 consecutive heads per rotation, dividing heads */
+  int32_t rope;        /* 1: apply RoPE (keys), 0: not (values) */
+  int32_t n_sink;      /* positions 0..n_sink-1 are attention sinks kept verbatim in fp16 */
+  int32_t rot;         /* KVQ_ROT_* */
+  int32_t quant;       /* KVQ_Q_* */
+} kvq_desc;
+
+/* The compressed cache. Slot s of head (b, h) is record (b*H + h)*t_cap + s.
+ *   codes       u8   [B][H][t_cap][head_dim*bits/8]  code j of a record occupies bits
+ *                     [bits*j, bits*j+bits) of its little-endian byte stream (LSB first)
+ *   scale_zero  half [B][H][t_cap][head_dim/group][2]  (scale S, zero Z); min-max only
+ *   sink        half [B][H][n_sink][head_dim]          the first n_sink positions, verbatim
+ *   norm        f32  [B][H][t_cap]                      rho; ISO_SO4 only
+ * Slots of sink positions hold zero codes, zero scale/zero and zero norm.
+ * Alignment: codes, scale_zero and sink 16 bytes; norm 4 bytes. Unused fields may be NULL. */
+typedef struct {
+  uint8_t* codes;
+  void* scale_zero;
+  void* sink;
+  float* norm;
+} kvq_packed;
+
+/* Read-only tables (device pointers).
+ *   perm      int16 [H][head_dim] or NULL (identity): the permutation step gathers
+ *             p_j = y_perm[h][j] ([RotateKV] channel reordering); must be a permutation
+ *   rope_cs   f32 [rope_rows][head_dim/2][2] = (cos, sin) of position m times
+ *             theta_i = 10000^(-2i/head_dim) ([EliteKV §2.1]); fill it with kvq_rope_table.
+ *             16-byte aligned. Required when rope = 1 (and by kvq_score when n_sink > 0).
+ *   qL, qR    f32 [head_dim/4][4] unit quaternions (real, i, j, k), one pair per 4-D block
+ *   codebook  f32 [1 << bits] ascending levels (kvq_lloyd_max_codebook) */
+typedef struct {
+  const int16_t* perm;
+  const float* rope_cs;
+  int32_t rope_rows;
+  const float* qL;
+  const float* qR;
+  const float* codebook;
+} kvq_tables;
+
+/* Encode T tokens into cache slots t0..t0+T-1.
+ * x: half [B][H][T][head_dim], 16-byte aligned. Per token-head vector (or per token and head
+ * group for FWHT_GROUP): the rotation of d->rot, then the quantizer of d->quant, then bit
+ * packing. Min-max ([RotateKV] 2-bit KV quantization; the fp16 rounding reading): per group of
+ * `group` consecutive rotated channels, Z = largest fp16 <= min, S = smallest fp16 >=
+ * fp32((max - Z)/(2^bits - 1)), code = round-half-even(fp32(p - Z) * fp32(1/S)), so codes lie
+ * in [0, 2^bits - 1]. Codebook: code = number of fp32 midpoints 0.5*(l_k + l_{k+1}) below w.
+ * Sink positions (< n_sink) are copied to `sink` verbatim ([RotateKV] attention sinks). */
+kvq_status kvq_encode(const kvq_desc* d, const void* x, const kvq_tables* tb, const kvq_packed* out,
+                      kvq_stream_t stream);
+
+/* Decode slots t0..t0+T-1 back to the encoder's input basis (pre-RoPE keys, raw values):
+ * dequantize (Z + c*S, or the codebook level), then the inverse rotation in reverse order
+ * ([IsoQuant §3.1] step 3: inverse rotation, then restore the norm), then the inverse RoPE.
+ * x_out: [B][H][T][head_dim], fp32 if out_fp32 else fp16 (round to nearest), 16-byte
+ * aligned. Sink positions come back verbatim. */
+kvq_status kvq_decode(const kvq_desc* d, const kvq_packed* in, const kvq_tables* tb, void* x_out,
+                      int32_t out_fp32, kvq_stream_t stream);
+
+/* Decode-step attention scores ([EliteKV §2.2]: A_{m,n} = q_m^rot . k_n^rot / sqrt(d)):
+ *   scores[b][qh][n] = scale * <q[b][qh], khat[b][qh / (q_heads/H)][n]>,  n in [0, n_tokens)
+ * q: half [B][q_heads][head_dim] in attention space (RoPE'd at the query position); q_heads a
+ * multiple of H (grouped-query attention). khat_n is the key in attention space: RoPE_n(sink_n)
+ * for n < n_sink, else slot n decoded without the inverse RoPE. Supported for rot in
+ * {NONE, FWHT_HEAD} with min-max codes; the kernel rotates the query once instead of every key
+ * (q . P^T H y = (H P q) . y for the orthonormal H and permutation P).
+ * scores: f32 [B][q_heads][n_tokens]; n_tokens <= t_cap. d->tokens and d->t0 are ignored. */
+kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kvq_packed* cache,
+                     const kvq_tables* tb, int32_t n_tokens, float scale, float* scores,
+                     kvq_stream_t stream);
+
+/* Bytes of one packed buffer (KVQ_FIELD_*) for this descriptor; 0 if the field is unused or
+ * the descriptor is invalid. */
+size_t kvq_packed_bytes(const kvq_desc* d, int32_t field);
+
+/* Fill a HOST buffer cs[t_max][head_dim/2][2] with (float)cos(m*theta_i), (float)sin(m*theta_i),
+ * theta_i = base^(-2i/head_dim), the angle formed in double ([RoPE-KV §1], [EliteKV §2.1]).
+ * The caller copies it to the device. */
+kvq_status kvq_rope_table(float* cs_host, int32_t t_max, int32_t head_dim, double base);
+
+/* Fill a HOST buffer with the 2^bits Lloyd-Max levels of N(0, 1/head_dim), ascending: Lloyd's
+ * iteration on N(0,1) in double, scaled by 1/sqrt(head_dim), rounded to fp32 ([IsoQuant §3.1]). */
+kvq_status kvq_lloyd_max_codebook(float* levels_host, int32_t bits, int32_t head_dim);
+
+/* Synchronise `stream` and report (then clear) the device error word of the current device:
+ * KVQ_ERR_TIMEOUT if a kernel gave up on a bounded wait, KVQ_ERR_CUDA on a CUDA error. */
+kvq_status kvq_check(kvq_stream_t stream);
+
+/* Test hook for the bounded-wait path: launches one CTA that waits on a copy that is never
+ * issued, with the given limit in microseconds (1..1000000); the wait expires, the kernel sets
+ * the error word and returns, and kvq_check then reports KVQ_ERR_TIMEOUT. */
+kvq_status kvq_debug_expire_wait(uint32_t limit_us, kvq_stream_t stream);
+
+const char* kvq_status_str(kvq_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H */

@@ -1,0 +1,264 @@
+// Device-side building blocks shared by the libkvq kernels (sm_100a):
+// mbarrier + TMA (cp.async.bulk.tensor) staging with bounded waits, the
+// in-register FWHT, RoPE, the min-max quantizer and bit packing.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace kvq {
+
+// Error word bits, read and cleared by kvq_check. Kernels receive the
+// address of the per-device error word as an argument.
+constexpr uint32_t kErrTimeout = 1u;
+
+constexpr float kMagicRound = 12582912.0f;  // 1.5 * 2^23: fp32 ulp = 1 on [2^23, 2^24)
+constexpr uint32_t kMagicBits = 0x4B400000u;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait on an mbarrier phase: gives up after limit_ns of wall time
+// (and in any case after 2^30 polls), sets the error word, returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns, uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1; it < (1u << 30); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0 && global_ns() - t0 > limit_ns) break;
+  }
+  atomicOr(err, kErrTimeout);
+  return false;
+}
+
+// ---------------------------------------------------------------- TMA
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int y, int z, const void* src) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Make generic-proxy smem writes visible to the TMA (async proxy).
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- smem access
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float lds32f(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts32f(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ uint16_t lds16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+// Byte offset of 16-byte chunk c of row r in a TMA tile written with
+// CU_TENSOR_MAP_SWIZZLE_128B (128-byte rows, tile base 1024-byte aligned).
+__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }
+
+// ---------------------------------------------------------------- fp16
+__device__ __forceinline__ void h8_to_f32(uint4 raw, float* f) {
+  const __half2* h = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __half22float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ uint4 f32_to_h8(const float* f) {
+  uint4 raw;
+  __half2* h = reinterpret_cast<__half2*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+  return raw;
+}
+
+// ---------------------------------------------------------------- FWHT
+// Unnormalised Sylvester FWHT on a register array, strides 1, 2, ..., N/2
+// in ascending order; each pair (i, i+h), (i & h) == 0 becomes (a+b, a-b).
+template <int N>
+__device__ __forceinline__ void fwht_reg(float (&v)[N]) {
+#pragma unroll
+  for (int h = 1; h < N; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = __fadd_rn(a, b);
+        v[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- RoPE
+// Forward rotation of one pair with fp32 (c, s):
+//   y0 = fma(x0, c, -(x1*s)),  y1 = fma(x0, s, x1*c)
+__device__ __forceinline__ void rope_fwd(float& x0, float& x1, float c, float s) {
+  const float t1 = __fmul_rn(x1, s);
+  const float t2 = __fmul_rn(x1, c);
+  const float y0 = __fmaf_rn(x0, c, -t1);
+  const float y1 = __fmaf_rn(x0, s, t2);
+  x0 = y0;
+  x1 = y1;
+}
+// Inverse rotation (decode; tolerance-checked, any rounding order is fine).
+__device__ __forceinline__ void rope_inv(float& y0, float& y1, float c, float s) {
+  const float x0 = __fmaf_rn(y0, c, __fmul_rn(y1, s));
+  const float x1 = __fmaf_rn(y1, c, -__fmul_rn(y0, s));
+  y0 = x0;
+  y1 = x1;
+}
+
+// ---------------------------------------------------------------- min/max
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Min and max of v[off .. off+n) (n even, n >= 2).
+template <int N>
+__device__ __forceinline__ void minmax_range(const float (&v)[N], int off, int n, float& mn, float& mx) {
+  mn = fminf(v[off], v[off + 1]);
+  mx = fmaxf(v[off], v[off + 1]);
+#pragma unroll
+  for (int j = 2; j + 1 < n; j += 2) {
+    mn = min3f(mn, v[off + j], v[off + j + 1]);
+    mx = max3f(mx, v[off + j], v[off + j + 1]);
+  }
+}
+
+// Scale / zero of one min-max group from its (canonicalised) min and max:
+// Z = largest half <= mn, S = smallest half >= fp32((mx - Z)/L), R = 1/S.
+struct QParams {
+  float Z, R;
+  __half2 sz;  // (S, Z)
+};
+template <int BITS>
+__device__ __forceinline__ QParams minmax_params(float mn, float mx) {
+  mn = __fadd_rn(mn, 0.0f);
+  mx = __fadd_rn(mx, 0.0f);
+  const __half zh = __float2half_rd(mn);
+  const float Z = __half2float(zh);
+  const float w = __fsub_rn(mx, Z);
+  const float q = __fdiv_rn(w, static_cast<float>((1 << BITS) - 1));
+  const __half sh = __float2half_ru(q);
+  const float S = __half2float(sh);
+  QParams p;
+  p.Z = Z;
+  p.R = S > 0.0f ? __frcp_rn(S) : 0.0f;
+  p.sz = __halves2half2(sh, zh);
+  return p;
+}
+// code = round-half-even of the exact product fp32(p - Z) * R; the result's
+// fp32 bit pattern is kMagicBits + code (code in [0, 2^BITS - 1]).
+__device__ __forceinline__ uint32_t quant_code(float p, float Z, float R) {
+  const float d = __fsub_rn(p, Z);
+  return __float_as_uint(__fmaf_rn(d, R, kMagicRound)) - kMagicBits;
+}
+
+// ---------------------------------------------------------------- packing
+// Pack N codes (each < 2^BITS) LSB-first into N*BITS/32 words.
+template <int N, int BITS>
+__device__ __forceinline__ void pack_codes(const uint32_t (&c)[N], uint32_t (&w)[N * BITS / 32]) {
+#pragma unroll
+  for (int i = 0; i < N * BITS / 32; ++i) w[i] = 0u;
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const int p = j * BITS;
+    w[p >> 5] |= c[j] << (p & 31);
+    if ((p & 31) + BITS > 32) w[(p >> 5) + 1] |= c[j] >> (32 - (p & 31));
+  }
+}
+// Code j of a packed word array.
+template <int BITS, int NW>
+__device__ __forceinline__ uint32_t unpack_code(const uint32_t (&w)[NW], int j) {
+  const int p = j * BITS;
+  uint32_t c = w[p >> 5] >> (p & 31);
+  if ((p & 31) + BITS > 32) c |= w[(p >> 5) + 1] << (32 - (p & 31));
+  return c & ((1u << BITS) - 1u);
+}
+// Exact small integer -> float without the conversion pipe.
+__device__ __forceinline__ float code_to_float(uint32_t c) {
+  return __fsub_rn(__uint_as_float(0x4B000000u | c), 8388608.0f);
+}
+
+}  // namespace kvq

@@ -1,0 +1,53 @@
+// Host-side internals shared by the libkvq translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+// Per-call launch context prepared by the C-ABI layer.
+struct LaunchCtx {
+  uint32_t* err;     // device address of this device's error word
+  uint64_t wait_ns;  // bound on every in-kernel wait
+  int num_sms;
+};
+
+// Tensor-map construction (driver entry point resolved through the runtime).
+bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base, const uint64_t* dims,
+              const uint64_t* strides_bytes /* rank-1 entries */, const uint32_t* box, CUtensorMapSwizzle swz);
+
+// Heads per tile for the head-variant kernels: the largest power of two
+// <= 8 that divides H (so a tile never spans two batches).
+inline int heads_per_tile(int H) {
+  int ht = 8;
+  while (ht > 1 && H % ht) ht >>= 1;
+  return ht;
+}
+
+kvq_status launch_encode_head(const kvq_desc& d, const void* x, const kvq_tables& tb, const kvq_packed& out,
+                              cudaStream_t st, const LaunchCtx& ctx);
+kvq_status launch_decode_head(const kvq_desc& d, const kvq_packed& in, const kvq_tables& tb, void* x_out,
+                              int out_fp32, cudaStream_t st, const LaunchCtx& ctx);
+kvq_status launch_encode_group(const kvq_desc& d, const void* x, const kvq_tables& tb, const kvq_packed& out,
+                               cudaStream_t st, const LaunchCtx& ctx);
+kvq_status launch_decode_group(const kvq_desc& d, const kvq_packed& in, const kvq_tables& tb, void* x_out,
+                               int out_fp32, cudaStream_t st, const LaunchCtx& ctx);
+kvq_status launch_encode_iso(const kvq_desc& d, const void* x, const kvq_tables& tb, const kvq_packed& out,
+                             cudaStream_t st, const LaunchCtx& ctx);
+kvq_status launch_decode_iso(const kvq_desc& d, const kvq_packed& in, const kvq_tables& tb, void* x_out,
+                             int out_fp32, cudaStream_t st, const LaunchCtx& ctx);
+kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq_packed& cache,
+                        const kvq_tables& tb, int n_tokens, float scale, float* scores, cudaStream_t st,
+                        const LaunchCtx& ctx);
+kvq_status launch_debug_wait(uint64_t limit_ns, cudaStream_t st, const LaunchCtx& ctx);
+
+// Finish a launch: map a launch error to a status.
+inline kvq_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+}  // namespace kvq

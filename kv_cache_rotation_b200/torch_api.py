@@ -1,0 +1,119 @@
+"""Marshalling helpers between torch tensors and the libkvq C ABI.
+
+Nothing here computes: tensors are allocated with torch (device memory is
+PyTorch's job), their addresses are put into the ABI structs, and the C entry
+points run the CUDA kernels. Host-side tables (RoPE cos/sin, Lloyd-Max
+levels) are filled by the library's own host helpers and uploaded.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import (KVQ_FIELD_CODES, KVQ_FIELD_NORM, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_Q_CODEBOOK,
+               KVQ_Q_MINMAX, KVQ_ROT_FWHT_GROUP, KVQ_ROT_FWHT_HEAD, KVQ_ROT_ISO_SO4, KVQ_ROT_NONE, check,
+               kvq_decode, kvq_desc, kvq_encode, kvq_lloyd_max_codebook, kvq_packed, kvq_packed_bytes,
+               kvq_rope_table, kvq_score, kvq_tables)
+
+ROT = {"none": KVQ_ROT_NONE, "fwht_head": KVQ_ROT_FWHT_HEAD, "fwht_group": KVQ_ROT_FWHT_GROUP,
+       "iso": KVQ_ROT_ISO_SO4}
+QUANT = {"minmax": KVQ_Q_MINMAX, "codebook": KVQ_Q_CODEBOOK}
+
+
+def make_desc(*, batch, heads, head_dim=128, tokens, t0=0, t_cap=None, bits, group=128, group_heads=1, rope=0,
+              n_sink=0, rot="fwht_head", quant="minmax") -> kvq_desc:
+    d = kvq_desc()
+    d.batch, d.heads, d.head_dim, d.tokens, d.t0 = batch, heads, head_dim, tokens, t0
+    d.t_cap = t0 + tokens if t_cap is None else t_cap
+    d.bits, d.group, d.group_heads, d.rope, d.n_sink = bits, group, group_heads, int(rope), n_sink
+    d.rot = ROT[rot] if isinstance(rot, str) else rot
+    d.quant = QUANT[quant] if isinstance(quant, str) else quant
+    return d
+
+
+@dataclass
+class Packed:
+    codes: torch.Tensor
+    scale_zero: Optional[torch.Tensor]
+    sink: Optional[torch.Tensor]
+    norm: Optional[torch.Tensor]
+
+    def struct(self) -> kvq_packed:
+        p = kvq_packed()
+        p.codes = self.codes.data_ptr()
+        p.scale_zero = self.scale_zero.data_ptr() if self.scale_zero is not None else None
+        p.sink = self.sink.data_ptr() if self.sink is not None else None
+        p.norm = self.norm.data_ptr() if self.norm is not None else None
+        return p
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.scale_zero, self.sink, self.norm)
+                   if t is not None)
+
+
+def alloc_packed(d: kvq_desc, device="cuda", zero=True) -> Packed:
+    """Allocate the cache buffers of a descriptor (sizes from kvq_packed_bytes)."""
+    alloc = torch.zeros if zero else torch.empty
+
+    def buf(field, dtype, shape):
+        n = kvq_packed_bytes(d, field)
+        if n == 0:
+            return None
+        t = alloc(n, dtype=torch.uint8, device=device)
+        return t.view(dtype).view(shape)
+
+    B, H, C, D = d.batch, d.heads, d.t_cap, d.head_dim
+    codes = buf(KVQ_FIELD_CODES, torch.uint8, (B, H, C, D * d.bits // 8))
+    ng = D // d.group if d.quant == KVQ_Q_MINMAX else 0
+    sz = buf(KVQ_FIELD_SCALE_ZERO, torch.int16, (B, H, C, ng, 2)) if ng else None
+    sink = buf(KVQ_FIELD_SINK, torch.float16, (B, H, d.n_sink, D)) if d.n_sink else None
+    norm = buf(KVQ_FIELD_NORM, torch.float32, (B, H, C))
+    return Packed(codes, sz, sink, norm)
+
+
+def rope_table(t_max: int, head_dim: int, device="cuda", base: float = 10000.0) -> torch.Tensor:
+    """(cos, sin) table [t_max][head_dim/2][2] filled by kvq_rope_table."""
+    host = torch.empty((t_max, head_dim // 2, 2), dtype=torch.float32)
+    check(kvq_rope_table(host.data_ptr(), t_max, head_dim, base), "kvq_rope_table")
+    return host.to(device)
+
+
+def lloyd_max_codebook(bits: int, head_dim: int, device="cuda") -> torch.Tensor:
+    host = torch.empty(1 << bits, dtype=torch.float32)
+    check(kvq_lloyd_max_codebook(host.data_ptr(), bits, head_dim), "kvq_lloyd_max_codebook")
+    return host.to(device)
+
+
+def make_tables(perm=None, rope_cs=None, qL=None, qR=None, codebook=None) -> kvq_tables:
+    tb = kvq_tables()
+    tb.perm = perm.data_ptr() if perm is not None else None
+    tb.rope_cs = rope_cs.data_ptr() if rope_cs is not None else None
+    tb.rope_rows = rope_cs.shape[0] if rope_cs is not None else 0
+    tb.qL = qL.data_ptr() if qL is not None else None
+    tb.qR = qR.data_ptr() if qR is not None else None
+    tb.codebook = codebook.data_ptr() if codebook is not None else None
+    return tb
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def encode(d: kvq_desc, x: torch.Tensor, tables: kvq_tables, packed: Packed, stream=None) -> None:
+    check(kvq_encode(d, x.data_ptr(), tables, packed.struct(), _stream(stream)), "kvq_encode")
+
+
+def decode(d: kvq_desc, packed: Packed, tables: kvq_tables, out: torch.Tensor, stream=None) -> None:
+    fp32 = 1 if out.dtype == torch.float32 else 0
+    check(kvq_decode(d, packed.struct(), tables, out.data_ptr(), fp32, _stream(stream)), "kvq_decode")
+
+
+def score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: kvq_tables, n_tokens: int, scale: float,
+          out: torch.Tensor, stream=None) -> None:
+    check(kvq_score(d, q.data_ptr(), q.shape[1], packed.struct(), tables, n_tokens, scale, out.data_ptr(),
+                    _stream(stream)), "kvq_score")

@@ -81,7 +81,7 @@ def lib():
         L.orc_codebook.argtypes = [ci, ci, f32p]
         L.orc_encode.restype = ci
         L.orc_encode.argtypes = [ci, ci, ci, ci, i64p, ci, ci, ci, ci, ci, ci, ci, cd,
-                                 u16p, i16p, f32p, f32p, f32p, u8p, u16p, u16p, f32p]
+                                 u16p, i16p, f32p, f32p, f32p, u8p, u16p, u16p, f32p, f32p]
         L.orc_decode.restype = ci
         L.orc_decode.argtypes = [ci, ci, ci, ci, i64p, ci, ci, ci, ci, ci, ci, ci, cd,
                                  u8p, u16p, u16p, f32p, i16p, f32p, f32p, f32p, f64p]
@@ -208,10 +208,11 @@ def _packed_shapes(B, H, T, D, bits, group, n_sink):
 
 
 def encode(x, pos, *, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0, n_sink=0,
-           base=10000.0, perm=None, qL=None, qR=None, cb=None):
+           base=10000.0, perm=None, qL=None, qR=None, cb=None, want_pre=False):
     """x: uint16 (fp16 bits) [B][H][T][D]; pos: int64 [T]. Returns a dict of
     codes [B][H][T][D*bits/8], sz uint16 [B][H][T][D/G][2], sink uint16
-    [B][H][n_sink][D], norm f32 [B][H][T]."""
+    [B][H][n_sink][D], norm f32 [B][H][T], and with want_pre the rotated
+    pre-quantization values pre f32 [B][H][T][D]."""
     x = np.ascontiguousarray(x, np.uint16)
     B, H, T, D = x.shape
     pos = np.ascontiguousarray(pos, np.int64)
@@ -220,6 +221,7 @@ def encode(x, pos, *, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0,
     sz = np.zeros(zs, np.uint16)
     sink = np.zeros(ss if n_sink > 0 else (1,), np.uint16)
     norm = np.zeros(ns, np.float32)
+    pre = np.zeros((B, H, T, D), np.float32) if want_pre else None
     perm_a = None if perm is None else np.ascontiguousarray(perm, np.int16)
     qL_a = None if qL is None else np.ascontiguousarray(qL, np.float32)
     qR_a = None if qR is None else np.ascontiguousarray(qR, np.float32)
@@ -228,10 +230,10 @@ def encode(x, pos, *, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0,
                           rope, n_sink, base, _p(x, ctypes.c_uint16), _p(perm_a, ctypes.c_int16),
                           _p(qL_a, ctypes.c_float), _p(qR_a, ctypes.c_float), _p(cb_a, ctypes.c_float),
                           _p(codes, ctypes.c_uint8), _p(sz, ctypes.c_uint16), _p(sink, ctypes.c_uint16),
-                          _p(norm, ctypes.c_float))
+                          _p(norm, ctypes.c_float), _p(pre, ctypes.c_float))
     if rc:
         raise ValueError("oracle encode: unsupported parameters")
-    return {"codes": codes, "sz": sz, "sink": sink if n_sink > 0 else None, "norm": norm}
+    return {"codes": codes, "sz": sz, "sink": sink if n_sink > 0 else None, "norm": norm, "pre": pre}
 
 
 def decode(packed, pos, shape, *, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0,

@@ -193,7 +193,7 @@ float orc_fwht_scale_f32(int n) { return (float)(1.0 / sqrt((double)n)); }
  * Per-token per-group asymmetric min-max quantization with fp16 scale and
  * zero ([RotateKV] 2-bit KV quantization; the quantizer form is the reading
  * stated in the design notes).
- *   mn, mx   group minimum / maximum (fp32; -0 is folded to +0 by mn + 0.0f)
+ *   mn, mx   group minimum / maximum (fp32; -0 is folded to +0 by adding 0.0f)
  *   Z        = largest half <= mn                (zero, rounded down)
  *   S        = smallest half >= fp32((mx - Z) / L)  (scale, rounded up)
  *   R        = S > 0 ? fp32(1 / S) : 0
@@ -210,7 +210,8 @@ void orc_minmax_group(const float* p, int g, int bits, uint8_t* codes, uint16_t*
     if (p[j] < mn) mn = p[j];
     if (p[j] > mx) mx = p[j];
   }
-  mn = mn + 0.0f;
+  mn = mn + 0.0f; /* -0 -> +0: the stored zero and scale never depend on zero signs */
+  mx = mx + 0.0f;
   uint16_t zh = orc_float_to_half_rd(mn);
   float Z = orc_half_to_float(zh);
   float w = mx - Z;
@@ -356,6 +357,8 @@ static int codebook_code(float w, const float* cb, int bits) {
  *   norm  f32   [B][H][T]
  * Tokens with pos < n_sink are kept verbatim in sink ([RotateKV]: attention
  * sinks protected at high precision); their codes and sz entries are zero.
+ *   pre   f32   [B][H][T][D] or NULL: the rotated values that were quantized
+ *         (used by the tests to tell boundary ties from real mismatches)
  * ---------------------------------------------------------------------- */
 typedef struct {
   int B, H, T, D, rot, quant, bits, group, group_heads, rope, n_sink;
@@ -391,7 +394,7 @@ static int check_shape(const orc_shape* s) {
 int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quant, int bits, int group,
                int group_heads, int rope, int n_sink, double base, const uint16_t* x, const int16_t* perm,
                const float* qL, const float* qR, const float* codebook, uint8_t* codes, uint16_t* sz,
-               uint16_t* sink, float* norm) {
+               uint16_t* sink, float* norm, float* pre) {
   orc_shape s = {B, H, T, D, rot, quant, bits, group, group_heads, rope, n_sink, base};
   if (check_shape(&s)) return 1;
   size_t rb = rec_bytes(&s);
@@ -440,6 +443,7 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
           }
           uint8_t cds[256];
           for (int j = 0; j < D; ++j) cds[j] = (uint8_t)codebook_code(w[j], codebook, bits);
+          if (pre) memcpy(pre + v * D, w, sizeof(float) * D);
           orc_pack(cds, D, bits, codes + v * rb);
           norm[v] = rho;
           continue;
@@ -468,6 +472,7 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
               memcpy(ph, tmp, sizeof(float) * D);
             }
             size_t v = ((size_t)(b * H + h0 + hl) * T + t);
+            if (pre) memcpy(pre + v * D, ph, sizeof(float) * D);
             quantize_head(&s, ph, codes + v * rb, sz + v * ng * 2);
           }
           continue;
@@ -490,6 +495,7 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
             float r = orc_fwht_scale_f32(D);
             for (int j = 0; j < D; ++j) buf[j] = buf[j] * r;
           }
+          if (pre) memcpy(pre + v * D, buf, sizeof(float) * D);
           quantize_head(&s, buf, codes + v * rb, sz + v * ng * 2);
         }
       }

@@ -1,0 +1,141 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, validates arguments before launching anything, sizes the
+packed buffers, and its host helpers agree with the oracle's own tables."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import kv_cache_rotation_b200 as K
+from kv_cache_rotation_b200 import torch_api as TA
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert set(names) == set(K.EXPORTED)
+    lib = ctypes.CDLL(K.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings():
+    assert K.kvq_version() >= 100
+    for s in range(6):
+        assert K.kvq_status_str(s)
+
+
+def _desc(**kw):
+    base = dict(batch=2, heads=8, tokens=16, bits=2, group=64, rope=0)
+    base.update(kw)
+    return TA.make_desc(**base)
+
+
+def _packed(d, codes=256, sz=256, sink=0, norm=0):
+    p = K.kvq_packed()
+    p.codes, p.scale_zero, p.sink, p.norm = codes, sz, sink or None, norm or None
+    return p
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), K.KVQ_ERR_INVALID),
+    (dict(heads=-1), K.KVQ_ERR_INVALID),
+    (dict(tokens=-1), K.KVQ_ERR_INVALID),
+    (dict(t0=10, t_cap=20, tokens=16), K.KVQ_ERR_INVALID),
+    (dict(bits=5), K.KVQ_ERR_UNSUPPORTED),
+    (dict(bits=1), K.KVQ_ERR_UNSUPPORTED),
+    (dict(head_dim=96), K.KVQ_ERR_UNSUPPORTED),
+    (dict(group=48), K.KVQ_ERR_UNSUPPORTED),
+    (dict(head_dim=64, group=128), K.KVQ_ERR_INVALID),
+    (dict(rot="fwht_group", group_heads=3), K.KVQ_ERR_UNSUPPORTED),
+    (dict(rot="fwht_group", group_heads=8, heads=12), K.KVQ_ERR_INVALID),
+    (dict(rot="fwht_group", group_heads=8, head_dim=64), K.KVQ_ERR_UNSUPPORTED),
+    (dict(rot="iso", quant="minmax"), K.KVQ_ERR_UNSUPPORTED),
+    (dict(rot="fwht_head", quant="codebook"), K.KVQ_ERR_UNSUPPORTED),
+    (dict(rope=2), K.KVQ_ERR_INVALID),
+    (dict(rot=9), K.KVQ_ERR_INVALID),
+])
+def test_encode_rejects_bad_desc(kw, status):
+    d = _desc(**kw)
+    tb = K.kvq_tables()
+    assert K.kvq_encode(d, 256, tb, _packed(d), 0) == status
+    assert K.kvq_decode(d, _packed(d), tb, 256, 0, 0) == status
+
+
+def test_null_and_alignment_checks():
+    d = _desc()
+    tb = K.kvq_tables()
+    assert K.kvq_encode(d, None, tb, _packed(d), 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_encode(d, 258, tb, _packed(d), 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_encode(d, 256, tb, _packed(d, codes=0), 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_encode(d, 256, tb, _packed(d, codes=264), 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_encode(d, 256, tb, _packed(d, sz=0), 0) == K.KVQ_ERR_INVALID
+    assert K.lib.kvq_encode(None, 256, ctypes.byref(tb), ctypes.byref(_packed(d)), None) == K.KVQ_ERR_INVALID
+    ds = _desc(n_sink=4)
+    assert K.kvq_encode(ds, 256, tb, _packed(ds), 0) == K.KVQ_ERR_INVALID  # sinks need a buffer
+    dr = _desc(rope=1)
+    assert K.kvq_encode(dr, 256, tb, _packed(dr), 0) == K.KVQ_ERR_INVALID  # rope needs the table
+    tb.rope_cs, tb.rope_rows = 256, 8  # too few rows for t0 + T = 16
+    assert K.kvq_encode(dr, 256, tb, _packed(dr), 0) == K.KVQ_ERR_INVALID
+    tb.rope_cs, tb.rope_rows = 260, 64
+    assert K.kvq_encode(dr, 256, tb, _packed(dr), 0) == K.KVQ_ERR_ALIGN
+    di = _desc(rot="iso", quant="codebook", bits=3)
+    assert K.kvq_encode(di, 256, K.kvq_tables(), _packed(di, norm=256), 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_decode(d, _packed(d), K.kvq_tables(), 256, 2, 0) == K.KVQ_ERR_INVALID
+
+
+def test_score_argument_checks():
+    d = _desc(t_cap=32, tokens=0)
+    tb = K.kvq_tables()
+    p = _packed(d)
+    assert K.kvq_score(d, 256, 12, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_INVALID  # 12 % 8
+    assert K.kvq_score(d, 256, 8, p, tb, 33, 1.0, 256, 0) == K.KVQ_ERR_INVALID  # > t_cap
+    assert K.kvq_score(d, 258, 8, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_ALIGN
+    dg = _desc(t_cap=32, rot="fwht_group", group_heads=8, group=128)
+    assert K.kvq_score(dg, 256, 8, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_UNSUPPORTED
+    assert K.kvq_score(d, 256, 8, p, tb, 0, 1.0, 256, 0) == K.KVQ_OK  # empty: nothing to do
+
+
+def test_empty_call_is_a_noop():
+    d = _desc(tokens=0, t_cap=4)
+    assert K.kvq_encode(d, 256, K.kvq_tables(), _packed(d), 0) == K.KVQ_OK
+    assert K.kvq_decode(d, _packed(d), K.kvq_tables(), 256, 1, 0) == K.KVQ_OK
+
+
+def test_packed_bytes_and_compression_ratios():
+    """Bytes per 128-channel fp16 vector (256 B) of each format, and the
+    resulting compression ratios: 4-bit G128 68 B (3.76x), 2-bit G64 40 B
+    (6.4x), 2-bit G128 36 B (7.11x), 3-bit codebook + fp32 norm 52 B (4.92x)."""
+    for kw, per_vec in ((dict(bits=4, group=128), 68), (dict(bits=2, group=64), 40),
+                        (dict(bits=2, group=128), 36), (dict(bits=3, rot="iso", quant="codebook"), 52)):
+        d = _desc(batch=3, heads=5, tokens=7, t_cap=11, head_dim=128, **kw)
+        tot = sum(K.kvq_packed_bytes(d, f) for f in (0, 1, 3))
+        assert tot == 3 * 5 * 11 * per_vec
+    d = _desc(n_sink=4, t_cap=16)
+    assert K.kvq_packed_bytes(d, K.KVQ_FIELD_SINK) == 2 * 8 * 4 * 128 * 2
+    assert K.kvq_packed_bytes(d, 7) == 0
+    assert K.kvq_packed_bytes(_desc(bits=9), 0) == 0
+
+
+def test_rope_table_matches_oracle(orc):
+    import torch
+    cs = TA.rope_table(40000, 128, device="cpu").numpy()
+    for m in (0, 1, 777, 32768, 39999):
+        c, s = orc.rope_cs(m, 128)
+        assert np.array_equal(cs[m, :, 0], c) and np.array_equal(cs[m, :, 1], s)
+    assert K.kvq_rope_table(None, 4, 128, 10000.0) == K.KVQ_ERR_INVALID
+    assert K.kvq_rope_table(torch.empty(8).data_ptr(), 4, 127, 10000.0) == K.KVQ_ERR_INVALID
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_codebook_matches_oracle(orc, bits):
+    cb = TA.lloyd_max_codebook(bits, 128, device="cpu").numpy()
+    assert np.array_equal(cb, orc.codebook(bits, 128))
