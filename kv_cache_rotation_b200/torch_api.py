@@ -87,15 +87,29 @@ def lloyd_max_codebook(bits: int, head_dim: int, device="cuda") -> torch.Tensor:
     return host.to(device)
 
 
-def make_tables(perm=None, rope_cs=None, qL=None, qR=None, codebook=None) -> kvq_tables:
-    tb = kvq_tables()
-    tb.perm = perm.data_ptr() if perm is not None else None
-    tb.rope_cs = rope_cs.data_ptr() if rope_cs is not None else None
-    tb.rope_rows = rope_cs.shape[0] if rope_cs is not None else 0
-    tb.qL = qL.data_ptr() if qL is not None else None
-    tb.qR = qR.data_ptr() if qR is not None else None
-    tb.codebook = codebook.data_ptr() if codebook is not None else None
-    return tb
+@dataclass
+class Tables:
+    """Device tables of one call; holds the tensors so their memory stays
+    alive for as long as the struct built from them is in use."""
+    perm: Optional[torch.Tensor] = None
+    rope_cs: Optional[torch.Tensor] = None
+    qL: Optional[torch.Tensor] = None
+    qR: Optional[torch.Tensor] = None
+    codebook: Optional[torch.Tensor] = None
+
+    def struct(self) -> kvq_tables:
+        tb = kvq_tables()
+        tb.perm = self.perm.data_ptr() if self.perm is not None else None
+        tb.rope_cs = self.rope_cs.data_ptr() if self.rope_cs is not None else None
+        tb.rope_rows = self.rope_cs.shape[0] if self.rope_cs is not None else 0
+        tb.qL = self.qL.data_ptr() if self.qL is not None else None
+        tb.qR = self.qR.data_ptr() if self.qR is not None else None
+        tb.codebook = self.codebook.data_ptr() if self.codebook is not None else None
+        return tb
+
+
+def make_tables(perm=None, rope_cs=None, qL=None, qR=None, codebook=None) -> Tables:
+    return Tables(perm, rope_cs, qL, qR, codebook)
 
 
 def _stream(stream) -> int:
@@ -104,16 +118,16 @@ def _stream(stream) -> int:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def encode(d: kvq_desc, x: torch.Tensor, tables: kvq_tables, packed: Packed, stream=None) -> None:
-    check(kvq_encode(d, x.data_ptr(), tables, packed.struct(), _stream(stream)), "kvq_encode")
+def encode(d: kvq_desc, x: torch.Tensor, tables: Tables, packed: Packed, stream=None) -> None:
+    check(kvq_encode(d, x.data_ptr(), tables.struct(), packed.struct(), _stream(stream)), "kvq_encode")
 
 
-def decode(d: kvq_desc, packed: Packed, tables: kvq_tables, out: torch.Tensor, stream=None) -> None:
+def decode(d: kvq_desc, packed: Packed, tables: Tables, out: torch.Tensor, stream=None) -> None:
     fp32 = 1 if out.dtype == torch.float32 else 0
-    check(kvq_decode(d, packed.struct(), tables, out.data_ptr(), fp32, _stream(stream)), "kvq_decode")
+    check(kvq_decode(d, packed.struct(), tables.struct(), out.data_ptr(), fp32, _stream(stream)), "kvq_decode")
 
 
-def score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: kvq_tables, n_tokens: int, scale: float,
+def score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens: int, scale: float,
           out: torch.Tensor, stream=None) -> None:
-    check(kvq_score(d, q.data_ptr(), q.shape[1], packed.struct(), tables, n_tokens, scale, out.data_ptr(),
-                    _stream(stream)), "kvq_score")
+    check(kvq_score(d, q.data_ptr(), q.shape[1], packed.struct(), tables.struct(), n_tokens, scale,
+                    out.data_ptr(), _stream(stream)), "kvq_score")

@@ -21,6 +21,10 @@ import numpy as np
 EXCUSE_REL = 1e-5
 EXCUSE_FRAC = 1e-4
 RECON_ABS = 1e-3
+# Rows of extreme magnitude (edge-case tests only): fp32 rounding in the
+# inverse transform is ~2^-24 * sqrt(log2 N) * ||x_row||, so those rows get
+# RECON_ABS + RECON_ROW_REL * ||x_row||_2 instead of the plain 1e-3.
+RECON_ROW_REL = 2.0 ** -20
 SCORE_REL = 1e-3
 
 ORC_ROT = {"none": 0, "fwht_head": 1, "fwht_group": 2, "iso": 3}
@@ -87,6 +91,13 @@ def compare_codebook(gpu_codes, orc_codes, pre, cb, D, bits) -> CodeReport:
         ok = diff & (np.abs(cg - co) == 1) & near
         exc = int(ok.sum())
     return CodeReport(cg.size, n_mis, exc, n_mis - exc, 0)
+
+
+def recon_tolerance(ref, row_rel=0.0):
+    """Per-element decode tolerance broadcast over [..., D]."""
+    if not row_rel:
+        return RECON_ABS
+    return RECON_ABS + row_rel * np.linalg.norm(ref, axis=-1, keepdims=True)
 
 
 def score_tolerance(q, khat, scale):

@@ -3,11 +3,13 @@ head_dim -> min-max 2/3/4-bit -> packing, sinks; and the inverse) against the
 CPU oracle, through the C ABI. Shapes are small enough for the oracle to
 finish in seconds but span several tiles, a ragged tail, a nonzero first slot
 and every supported (head_dim, bits, group)."""
+import zlib
+
 import numpy as np
 import pytest
 
 import workloads as W
-from parity import RECON_ABS, compare_minmax
+from parity import RECON_ROW_REL, compare_minmax, recon_tolerance
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -44,7 +46,7 @@ def _inputs(name, B, H, T, D, seed):
     return W.kv_tensor(w, "k")
 
 
-def run_head_case(K, orc, x, *, t0, t_cap, bits, group, rope, perm, n_sink, rot):
+def run_head_case(K, orc, x, *, t0, t_cap, bits, group, rope, perm, n_sink, rot, row_rel=0.0):
     from kv_cache_rotation_b200 import torch_api as TA
     B, H, T, D = x.shape
     d = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, t0=t0, t_cap=t_cap, bits=bits, group=group,
@@ -83,7 +85,7 @@ def run_head_case(K, orc, x, *, t0, t_cap, bits, group, rope, perm, n_sink, rot)
     dec = orc.decode(packed_np, pos, x.shape, **okw)
     o32 = out32.cpu().numpy()
     err = np.abs(o32.astype(np.float64) - dec)
-    assert err.max() <= RECON_ABS, err.max()
+    assert np.all(err <= recon_tolerance(dec, row_rel)), err.max()
     assert np.array_equal(out16.cpu().numpy().view(np.uint16), o32.astype(np.float16).view(np.uint16))
     return rep, err.max()
 
@@ -91,7 +93,7 @@ def run_head_case(K, orc, x, *, t0, t_cap, bits, group, rope, perm, n_sink, rot)
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_head_parity(K, orc, case):
     name, B, H, T, D, t0, extra, bits, group, rope, use_perm, n_sink, rot = case
-    x = _inputs(name, B, H, T, D, seed=hash(name) % 1000)
+    x = _inputs(name, B, H, T, D, seed=zlib.crc32(name.encode()) % 1000)
     perm = W.random_perm(H, D, 7) if use_perm else None
     run_head_case(K, orc, x, t0=t0, t_cap=t0 + T + extra, bits=bits, group=group, rope=rope, perm=perm,
                   n_sink=n_sink, rot=rot)
@@ -109,8 +111,10 @@ def test_head_edge_values(K, orc):
     x[0, 3, :, ::2] = np.float16(-5000.0)  # large, still in range after the FWHT
     x[0, 4, :16] = np.float16(-0.0)
     x[0, 5, :, 7] = np.float16(60000.0)  # one huge channel: rotated values ~ 5300
-    run_head_case(K, orc, x, t0=0, t_cap=T, bits=2, group=64, rope=1, perm=None, n_sink=0, rot="fwht_head")
-    run_head_case(K, orc, x, t0=0, t_cap=T, bits=4, group=128, rope=0, perm=None, n_sink=0, rot="fwht_head")
+    run_head_case(K, orc, x, t0=0, t_cap=T, bits=2, group=64, rope=1, perm=None, n_sink=0, rot="fwht_head",
+                  row_rel=RECON_ROW_REL)
+    run_head_case(K, orc, x, t0=0, t_cap=T, bits=4, group=128, rope=0, perm=None, n_sink=0, rot="fwht_head",
+                  row_rel=RECON_ROW_REL)
 
 
 def test_head_deterministic(K):

@@ -1,0 +1,99 @@
+"""GPU parity of the decode-step score kernel: the cache is written by the
+GPU encoder (prefill + one appended token), and the GPU scores are compared
+with the oracle's fp64 scores computed from that same cache, within
+|s_gpu - s_orc| <= 1e-3 * scale * sum_j |q_j khat_j|."""
+import math
+
+import numpy as np
+import pytest
+
+import workloads as W
+from parity import SCORE_REL
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def K():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import kv_cache_rotation_b200 as K
+    return K
+
+
+def build_cache(K, w, x, x_app, perm, rot="fwht_head"):
+    from kv_cache_rotation_b200 import torch_api as TA
+    B, H, T, D = x.shape
+    t_cap = T + x_app.shape[2]
+    kw = dict(batch=B, heads=H, head_dim=D, t_cap=t_cap, bits=w.bits, group=w.group, rope=1, n_sink=w.n_sink,
+              rot=rot)
+    tb = TA.make_tables(perm=torch.from_numpy(perm).cuda() if perm is not None else None,
+                        rope_cs=TA.rope_table(t_cap, D))
+    d_pre = TA.make_desc(tokens=T, t0=0, **kw)
+    pk = TA.alloc_packed(d_pre)
+    TA.encode(d_pre, torch.from_numpy(x).cuda(), tb, pk)
+    d_app = TA.make_desc(tokens=x_app.shape[2], t0=T, **kw)
+    TA.encode(d_app, torch.from_numpy(x_app).cuda(), tb, pk)
+    assert K.kvq_check(0) == K.KVQ_OK
+    return d_pre, tb, pk
+
+
+def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None):
+    from kv_cache_rotation_b200 import torch_api as TA
+    x = W.kv_tensor(w, "k")
+    x_app = W.kv_tensor(w, "k_append", T=w.append)
+    d, tb, pk = build_cache(K, w, x, x_app, perm, rot)
+    q = W.queries(w)
+    n_tok = d.t_cap
+    scale = 1.0 / math.sqrt(w.D)
+    out = torch.full((w.B, w.Hq, n_tok), float("nan"), dtype=torch.float32, device="cuda")
+    TA.score(d, torch.from_numpy(q).cuda(), pk, tb, n_tok, scale, out)
+    assert K.kvq_check(0) == K.KVQ_OK
+    tok = np.arange(n_tok) if tokens is None else np.asarray(tokens)
+    cache = {"codes": pk.codes.cpu().numpy(), "sz": pk.scale_zero.cpu().numpy().view(np.uint16),
+             "sink": pk.sink.cpu().numpy().view(np.uint16) if w.n_sink else None}
+    okw = dict(rot={"none": 0, "fwht_head": 1}[rot], bits=w.bits, group=w.group, rope=1, n_sink=w.n_sink,
+               perm=perm)
+    ref = orc.score(q.view(np.uint16), cache, tok, H=w.H, t_cap=n_tok, scale=scale, **okw)
+    # attention-space keys (fp64) for the L1 bound
+    khat = orc.decode(cache, np.arange(n_tok), (w.B, w.H, n_tok, w.D), **okw)
+    got = out.cpu().numpy()[:, :, tok]
+    gq = w.Hq // w.H
+    worst = 0.0
+    for b in range(w.B):
+        for qh in range(w.Hq):
+            h = qh // gq
+            kk = np.stack([orc.rope_f64(khat[b, h, n], n) for n in tok])
+            bound = SCORE_REL * scale * (np.abs(kk) @ np.abs(q[b, qh].astype(np.float64)))
+            err = np.abs(got[b, qh] - ref[b, qh])
+            assert np.all(err <= bound), (b, qh, np.max(err / bound))
+            worst = max(worst, float(np.max(err / bound)))
+    assert np.isfinite(out.cpu().numpy()).all()
+    return worst
+
+
+def test_score_mha_perm_sinks(K, orc):
+    w = W.scaled(W.WORKLOADS["decode_score"], B=2, H=4, Hq=4, T=300)
+    run_score_case(K, orc, w, W.random_perm(w.H, w.D, 11))
+
+
+def test_score_gqa(K, orc):
+    w = W.scaled(W.WORKLOADS["llama3_8b_gqa_score"], B=2, H=2, Hq=8, T=257)
+    run_score_case(K, orc, w, None)
+
+
+@pytest.mark.parametrize("bits,group", [(3, 32), (4, 128), (3, 64)])
+def test_score_bits(K, orc, bits, group):
+    w = W.scaled(W.WORKLOADS["decode_score"], B=1, H=2, Hq=4, T=130, bits=bits, group=group, n_sink=1)
+    run_score_case(K, orc, w, W.random_perm(w.H, w.D, 2))
+
+
+def test_score_no_rotation(K, orc):
+    w = W.scaled(W.WORKLOADS["decode_score"], B=1, H=2, Hq=2, T=70, n_sink=0)
+    run_score_case(K, orc, w, None, rot="none")
+
+
+def test_score_d64(K, orc):
+    w = W.scaled(W.WORKLOADS["decode_score"], B=2, H=2, Hq=2, T=64, D=64, group=32)
+    run_score_case(K, orc, w, W.random_perm(2, 64, 5))
