@@ -1,0 +1,439 @@
+"""Benchmark: fp16-KV GB/s of encode / decode / score on the Llama-3-8B-shaped
+KV-cache layer, and the HBM roofline fraction of the dominant kernel.
+
+One step = one pass of the whole path over one layer's KV cache
+(batch 4, 8 KV heads x 128, 32768 tokens, fp16, synthetic):
+  encode K, encode V   grouped-head FWHT over 8 heads x 128 channels, RoPE on K,
+                       2-bit min-max, group 128
+  decode K, decode V   the exact inverse (fp16 out)
+  append               encode one new token per sequence into the decode cache
+                       (head-dim FWHT, 2-bit group 128, 4 fp16 sinks)
+  score                q . K^T for 32 query heads (GQA 4:1) over the 32769 cached
+                       tokens, straight from the packed cache
+value = fp16-equivalent KV bytes represented by the step's kernels / step time.
+
+Usage: python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+Under torchrun each rank runs its own copy of the workload on its own GPU
+(weak scaling, no collective on the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "fp16-KV GB/s for encode/decode/score and % of B200 HBM roofline"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def _config(n_gpus):
+    wg, ws = W.WORKLOADS["llama3_8b_gqa"], W.WORKLOADS["llama3_8b_gqa_score"]
+    return {
+        "workload": "llama3_8b_gqa",
+        "batch": wg.B, "kv_heads": wg.H, "head_dim": wg.D, "tokens": wg.T, "q_heads": ws.Hq,
+        "kv": "K and V fp16, N(0,1) + 1% outlier channels x U[10,50] (synthetic)",
+        "encode_decode": "fwht over 8 heads x 128, RoPE(K) after it, 2-bit min-max group 128",
+        "score_cache": "fwht over head_dim, 2-bit group 128, 4 fp16 sinks, 32768 + 1 appended tokens",
+        "l2": "no flush: every step streams ~1.4 GB (11x the 126 MB L2), so each kernel's inputs "
+              "were evicted by the kernels before it",
+        "parallelism": f"replicas x{n_gpus} (batch-sharded, no data-path collective)",
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+               0x10: "sync_boost"}
+
+    def __init__(self, dev_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- workload
+class Step:
+    """Device buffers and launches of one step (through the C ABI)."""
+
+    def __init__(self, device):
+        import torch
+        from kv_cache_rotation_b200 import torch_api as TA
+        self.torch, self.TA = torch, TA
+        wg, ws = W.WORKLOADS["llama3_8b_gqa"], W.WORKLOADS["llama3_8b_gqa_score"]
+        self.wg, self.ws = wg, ws
+        B, H, T, D = wg.B, wg.H, wg.T, wg.D
+        self.k_host = W.kv_tensor(wg, "k")
+        self.v_host = W.kv_tensor(wg, "v")
+        self.k = torch.from_numpy(self.k_host).to(device)
+        self.v = torch.from_numpy(self.v_host).to(device)
+        self.dk = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, bits=wg.bits, group=wg.group,
+                               group_heads=wg.group_heads, rope=1, rot="fwht_group")
+        self.dv = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, bits=wg.bits, group=wg.group,
+                               group_heads=wg.group_heads, rope=0, rot="fwht_group")
+        self.tk = TA.make_tables(rope_cs=TA.rope_table(T + 1, D, device=device))
+        self.tv = TA.make_tables()
+        self.pk, self.pv = TA.alloc_packed(self.dk, device), TA.alloc_packed(self.dv, device)
+        self.ok = torch.empty((B, H, T, D), dtype=torch.float16, device=device)
+        self.ov = torch.empty((B, H, T, D), dtype=torch.float16, device=device)
+        # decode-step cache: prefill (untimed) + one appended token per step
+        Ts = ws.T
+        self.n_tok = Ts + ws.append
+        cap = self.n_tok
+        self.ds_pre = TA.make_desc(batch=ws.B, heads=ws.H, head_dim=D, tokens=Ts, t0=0, t_cap=cap, bits=ws.bits,
+                                   group=ws.group, rope=1, n_sink=ws.n_sink, rot="fwht_head")
+        self.ds_app = TA.make_desc(batch=ws.B, heads=ws.H, head_dim=D, tokens=ws.append, t0=Ts, t_cap=cap,
+                                   bits=ws.bits, group=ws.group, rope=1, n_sink=ws.n_sink, rot="fwht_head")
+        self.ts = TA.make_tables(rope_cs=TA.rope_table(cap, D, device=device))
+        self.ps = TA.alloc_packed(self.ds_pre, device)
+        ks = torch.from_numpy(W.kv_tensor(ws, "k")).to(device)
+        TA.encode(self.ds_pre, ks, self.ts, self.ps)
+        del ks
+        self.app_host = W.kv_tensor(ws, "k_append", T=ws.append)
+        self.app = torch.from_numpy(self.app_host).to(device)
+        self.q_host = W.queries(ws)
+        self.q = torch.from_numpy(self.q_host).to(device)
+        self.scores = torch.empty((ws.B, ws.Hq, self.n_tok), dtype=torch.float32, device=device)
+        self.scale = 1.0 / math.sqrt(D)
+        torch.cuda.synchronize(device)
+        # accounting
+        rb, ng = D * wg.bits // 8, D // wg.group
+        nvec = B * H * T
+        self.alg = {
+            "encode_k": nvec * (2 * D + rb + 4 * ng),
+            "encode_v": nvec * (2 * D + rb + 4 * ng),
+            "decode_k": nvec * (rb + 4 * ng + 2 * D),
+            "decode_v": nvec * (rb + 4 * ng + 2 * D),
+            "append": ws.B * ws.H * ws.append * (2 * D + D * ws.bits // 8 + 4 * (D // ws.group)),
+            "score": (ws.B * ws.H * (self.n_tok - ws.n_sink) * (D * ws.bits // 8 + 4 * (D // ws.group))
+                      + ws.B * ws.H * ws.n_sink * D * 2 + ws.B * ws.Hq * D * 2 + ws.B * ws.Hq * self.n_tok * 4),
+        }
+        self.fp16_equiv = {
+            "encode_k": nvec * 2 * D, "encode_v": nvec * 2 * D, "decode_k": nvec * 2 * D, "decode_v": nvec * 2 * D,
+            "append": ws.B * ws.H * ws.append * 2 * D, "score": ws.B * ws.H * self.n_tok * 2 * D,
+        }
+        self.names = list(self.alg)
+
+    def launches(self):
+        TA = self.TA
+        return [
+            lambda: TA.encode(self.dk, self.k, self.tk, self.pk),
+            lambda: TA.encode(self.dv, self.v, self.tv, self.pv),
+            lambda: TA.decode(self.dk, self.pk, self.tk, self.ok),
+            lambda: TA.decode(self.dv, self.pv, self.tv, self.ov),
+            lambda: TA.encode(self.ds_app, self.app, self.ts, self.ps),
+            lambda: TA.score(self.ds_pre, self.q, self.ps, self.ts, self.n_tok, self.scale, self.scores),
+        ]
+
+
+def _kernel_sources_sha(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "kv_cache_rotation_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_for(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(kernel)
+    if not e:
+        return None
+    if e.get("source_sha") != _kernel_sources_sha(e.get("sources", [])):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+KERNEL_SOURCES = {
+    "encode_k": ("k_encode_group", ["kvq_group.cu", "kvq_device.cuh"]),
+    "encode_v": ("k_encode_group", ["kvq_group.cu", "kvq_device.cuh"]),
+    "decode_k": ("k_decode_group", ["kvq_group.cu", "kvq_device.cuh"]),
+    "decode_v": ("k_decode_group", ["kvq_group.cu", "kvq_device.cuh"]),
+    "append": ("k_encode_head", ["kvq_head.cu", "kvq_device.cuh"]),
+    "score": ("k_score", ["kvq_score.cu", "kvq_device.cuh"]),
+}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def cpu_sample(seconds_hint: float = 10.0, tokens: int = None, t_offset: int = 0):
+    """Time the oracle on a bounded sample of the same workload: batch 0 (all
+    8 KV heads) over `tokens` tokens for encode/decode of K and V, and the
+    score of batch 0's 32 query heads over as many cache slots. Returns
+    (fp16-equivalent bytes, seconds, description)."""
+    import oracle
+    wg, ws = W.WORKLOADS["llama3_8b_gqa"], W.WORKLOADS["llama3_8b_gqa_score"]
+    if tokens is None:
+        tokens = 4096 if seconds_hint >= 5 else 512
+    Tn = tokens
+    k = W.kv_tensor(W.scaled(wg, T=Tn, B=1, seed=wg.seed * 1000 + t_offset), "k").view(np.uint16)
+    v = W.kv_tensor(W.scaled(wg, T=Tn, B=1, seed=wg.seed * 1000 + t_offset), "v").view(np.uint16)
+    pos = np.arange(t_offset, t_offset + Tn)
+    kwk = dict(rot=oracle.ROT_FWHT_GROUP, bits=wg.bits, group=wg.group, group_heads=wg.group_heads, rope=1)
+    kwv = dict(kwk, rope=0)
+    ks = W.kv_tensor(W.scaled(ws, T=Tn, B=1, seed=ws.seed * 1000 + t_offset), "k").view(np.uint16)
+    q = W.queries(ws, B=1).view(np.uint16)
+    kws = dict(rot=oracle.ROT_FWHT_HEAD, bits=ws.bits, group=ws.group, rope=1, n_sink=ws.n_sink)
+    cache = oracle.encode(ks, np.arange(Tn), **kws)
+    t0 = time.perf_counter()
+    pk = oracle.encode(k, pos, **kwk)
+    pv = oracle.encode(v, pos, **kwv)
+    oracle.decode(pk, pos, k.shape, **kwk)
+    oracle.decode(pv, pos, v.shape, **kwv)
+    oracle.score(q, cache, np.arange(Tn), H=ws.H, t_cap=Tn, scale=1 / math.sqrt(ws.D), **kws)
+    dt = time.perf_counter() - t0
+    nbytes = 5 * wg.H * Tn * wg.D * 2  # 4 x (encode/decode of one tensor) + the score's key bytes
+    desc = (f"oracle (plain C, 1 thread): batch 1 of {wg.B}, {Tn} of {wg.T} tokens: encode+decode of K and V "
+            f"(grouped FWHT) and the score of 32 query heads over {Tn} cache slots")
+    return nbytes, dt, desc
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = _config(args.gpus)
+    for _ in range(args.warmup):
+        cpu_sample(tokens=256)
+    tot_b, tot_s = 0, 0.0
+    desc = ""
+    for i in range(args.steps):
+        b, s, desc = cpu_sample(tokens=args.ref_tokens, t_offset=(i * args.ref_tokens) % W.WORKLOADS["llama3_8b_gqa"].T)
+        tot_b += b
+        tot_s += s
+    value = tot_b / tot_s / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def run_ours(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import kv_cache_rotation_b200 as K
+    st = Step(dev)
+    launches = st.launches()
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        for f in launches:
+            f()
+    torch.cuda.synchronize(dev)
+    assert K.kvq_check(0) == K.KVQ_OK
+
+    nk = len(launches)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            for i, f in enumerate(launches):
+                f()
+                ev[s][i + 1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    per_kernel = {n: 0.0 for n in st.names}
+    for s in range(args.steps):
+        for i, n in enumerate(st.names):
+            per_kernel[n] += ev[s][i].elapsed_time(ev[s][i + 1])
+    status = K.kvq_check(0)
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    fp16_step = sum(st.fp16_equiv.values())
+    value = world * fp16_step * args.steps / (total_ms / 1e3) / 1e9
+    peak, peak_kind = _peaks()
+    kernels = {}
+    for n in st.names:
+        ms = per_kernel[n] / args.steps
+        kernels[n] = {"ms": ms, "fp16_gbs": st.fp16_equiv[n] / (ms / 1e3) / 1e9,
+                      "alg_gbs": st.alg[n] / (ms / 1e3) / 1e9,
+                      "frac_of_measured_hbm": st.alg[n] / (ms / 1e3) / 1e9 / peak}
+    dom = max(st.names, key=lambda n: per_kernel[n])
+    dom_ms = per_kernel[dom] / args.steps
+    achieved = st.alg[dom] / (dom_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": _traffic_for(KERNEL_SOURCES[dom][0]), "kernel": KERNEL_SOURCES[dom][0],
+                "kernel_step": dom, "alg_bytes_per_launch": st.alg[dom], "peak_kind": peak_kind}
+
+    e2e = run_e2e(st, launches, dev, stream, min(args.steps, args.e2e_steps), args.warmup_e2e)
+    if dist:
+        t = torch.tensor([e2e["ms_per_step"]], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms_per_step"] = float(t.item())
+    e2e_value = world * fp16_step / (e2e["ms_per_step"] / 1e3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        b, s, desc = cpu_sample()
+        cpu = {"value": b / s / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+               "seconds": s}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": _config(world), "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
+                    "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms_per_step"], "steps": e2e["steps"]},
+            "gpu_launches": nk * args.steps, "clocks": clk.summary(), "kernels": kernels,
+            "status": K.kvq_status_str(status),
+        }
+        print(json.dumps(line))
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if status == K.KVQ_OK else 1
+
+
+def run_e2e(st, launches, dev, stream, steps, warmup):
+    """Same step through host buffers: pinned K, V, the appended token and q
+    are copied in, and every result the step produces (packed K/V, decoded
+    K/V, scores) is copied back, inside the timed region."""
+    import torch
+    h_in = [torch.from_numpy(a).pin_memory() for a in (st.k_host, st.v_host, st.app_host, st.q_host)]
+    d_in = [st.k, st.v, st.app, st.q]
+    d_out = [st.pk.codes, st.pk.scale_zero, st.pv.codes, st.pv.scale_zero, st.ok, st.ov, st.scores]
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+
+    def one():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        for f in launches:
+            f()
+        for h, d in zip(h_out, d_out):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    return {"ms_per_step": a.elapsed_time(b) / steps, "h2d": h2d, "d2h": d2h, "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--warmup-e2e", type=int, default=3)
+    ap.add_argument("--ref-tokens", type=int, default=512, help="tokens per reference-arm step")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
