@@ -173,3 +173,31 @@ def random_perm(H: int, D: int, seed: int) -> np.ndarray:
 
 def positions(t0: int, T: int) -> np.ndarray:
     return np.arange(t0, t0 + T, dtype=np.int64)
+
+
+def kv_tensor_device(w: Workload, which: str, device, T: Optional[int] = None, B: Optional[int] = None):
+    """Large tensors drawn on the GPU with torch's seeded generator (same
+    recipe as kv_tensor, different stream): fp16 [B][H][T][D]. Student-t(4)
+    is z0 / sqrt((z1^2 + z2^2 + z3^2 + z4^2) / 4) with iid standard normals."""
+    import torch
+    T = w.T if T is None else T
+    B = w.B if B is None else B
+    stream = {"k": 1, "v": 2, "k_append": 3, "v_append": 4}[which]
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed * 1000 + stream)
+    n = B * w.H * T * w.D
+    out = torch.empty(n, dtype=torch.float16, device=device)
+    chunk = 1 << 25
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        if w.dist == "student_t":
+            z = torch.randn((5, e - s), generator=g, device=device)
+            out[s:e] = (z[0] / torch.sqrt((z[1:] ** 2).sum(0) / 4.0)).half()
+        else:
+            out[s:e] = torch.randn(e - s, generator=g, device=device).half()
+    out = out.view(B, w.H, T, w.D)
+    if w.dist != "student_t":
+        sc = outlier_scales(w.H, w.D, w.outliers, _rng(w.seed, 10 + stream % 2))
+        for h, c in zip(*np.nonzero(sc != 1.0)):
+            out[:, h, :, c] = (out[:, h, :, c].float() * float(sc[h, c])).half()
+    return out
