@@ -121,7 +121,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workload
 class Step:
-    """Device buffers and launches of one step (through the C ABI)."""
+    """Device buffers and launches of one step of the Llama-3-8B-shaped
+    layer (through the C ABI)."""
+
+    workload = "llama3_8b_gqa"
 
     def __init__(self, device):
         import torch
@@ -144,24 +147,7 @@ class Step:
         self.ok = torch.empty((B, H, T, D), dtype=torch.float16, device=device)
         self.ov = torch.empty((B, H, T, D), dtype=torch.float16, device=device)
         # decode-step cache: prefill (untimed) + one appended token per step
-        Ts = ws.T
-        self.n_tok = Ts + ws.append
-        cap = self.n_tok
-        self.ds_pre = TA.make_desc(batch=ws.B, heads=ws.H, head_dim=D, tokens=Ts, t0=0, t_cap=cap, bits=ws.bits,
-                                   group=ws.group, rope=1, n_sink=ws.n_sink, rot="fwht_head")
-        self.ds_app = TA.make_desc(batch=ws.B, heads=ws.H, head_dim=D, tokens=ws.append, t0=Ts, t_cap=cap,
-                                   bits=ws.bits, group=ws.group, rope=1, n_sink=ws.n_sink, rot="fwht_head")
-        self.ts = TA.make_tables(rope_cs=TA.rope_table(cap, D, device=device))
-        self.ps = TA.alloc_packed(self.ds_pre, device)
-        ks = torch.from_numpy(W.kv_tensor(ws, "k")).to(device)
-        TA.encode(self.ds_pre, ks, self.ts, self.ps)
-        del ks
-        self.app_host = W.kv_tensor(ws, "k_append", T=ws.append)
-        self.app = torch.from_numpy(self.app_host).to(device)
-        self.q_host = W.queries(ws)
-        self.q = torch.from_numpy(self.q_host).to(device)
-        self.scores = torch.empty((ws.B, ws.Hq, self.n_tok), dtype=torch.float32, device=device)
-        self.scale = 1.0 / math.sqrt(D)
+        self.sc = ScoreCache(ws, device)
         torch.cuda.synchronize(device)
         # accounting
         rb, ng = D * wg.bits // 8, D // wg.group
@@ -171,26 +157,143 @@ class Step:
             "encode_v": nvec * (2 * D + rb + 4 * ng),
             "decode_k": nvec * (rb + 4 * ng + 2 * D),
             "decode_v": nvec * (rb + 4 * ng + 2 * D),
-            "append": ws.B * ws.H * ws.append * (2 * D + D * ws.bits // 8 + 4 * (D // ws.group)),
-            "score": (ws.B * ws.H * (self.n_tok - ws.n_sink) * (D * ws.bits // 8 + 4 * (D // ws.group))
-                      + ws.B * ws.H * ws.n_sink * D * 2 + ws.B * ws.Hq * D * 2 + ws.B * ws.Hq * self.n_tok * 4),
+            "append": self.sc.alg_append,
+            "score": self.sc.alg_score,
         }
         self.fp16_equiv = {
             "encode_k": nvec * 2 * D, "encode_v": nvec * 2 * D, "decode_k": nvec * 2 * D, "decode_v": nvec * 2 * D,
-            "append": ws.B * ws.H * ws.append * 2 * D, "score": ws.B * ws.H * self.n_tok * 2 * D,
+            "append": self.sc.fp16_append, "score": self.sc.fp16_score,
         }
+        self.kernels = {"encode_k": "k_encode_group", "encode_v": "k_encode_group", "decode_k": "k_decode_group",
+                        "decode_v": "k_decode_group", "append": "k_encode_head", "score": "k_score_mma"}
         self.names = list(self.alg)
+        self.host_in = [self.k_host, self.v_host, self.sc.app_host, self.sc.q_host]
+        self.dev_in = [self.k, self.v, self.sc.app, self.sc.q]
+        self.dev_out = [self.pk.codes, self.pk.scale_zero, self.pv.codes, self.pv.scale_zero, self.ok, self.ov,
+                        self.sc.scores]
 
     def launches(self):
         TA = self.TA
         return [
-            lambda: TA.encode(self.dk, self.k, self.tk, self.pk),
-            lambda: TA.encode(self.dv, self.v, self.tv, self.pv),
-            lambda: TA.decode(self.dk, self.pk, self.tk, self.ok),
-            lambda: TA.decode(self.dv, self.pv, self.tv, self.ov),
-            lambda: TA.encode(self.ds_app, self.app, self.ts, self.ps),
-            lambda: TA.score(self.ds_pre, self.q, self.ps, self.ts, self.n_tok, self.scale, self.scores),
+            TA.bind_encode(self.dk, self.k, self.tk, self.pk),
+            TA.bind_encode(self.dv, self.v, self.tv, self.pv),
+            TA.bind_decode(self.dk, self.pk, self.tk, self.ok),
+            TA.bind_decode(self.dv, self.pv, self.tv, self.ov),
+            self.sc.append,
+            self.sc.score,
         ]
+
+
+class ScoreCache:
+    """A prefilled head-variant cache (untimed) plus the decode-step launches:
+    append one token per sequence, then score every cached slot."""
+
+    def __init__(self, ws, device):
+        import torch
+        from kv_cache_rotation_b200 import torch_api as TA
+        self.TA = TA
+        D = ws.D
+        Ts = ws.T
+        self.n_tok = Ts + ws.append
+        cap = self.n_tok
+        common = dict(batch=ws.B, heads=ws.H, head_dim=D, t_cap=cap, bits=ws.bits, group=ws.group, rope=1,
+                      n_sink=ws.n_sink, rot="fwht_head")
+        self.d_pre = TA.make_desc(tokens=Ts, t0=0, **common)
+        self.d_app = TA.make_desc(tokens=ws.append, t0=Ts, **common)
+        perm = torch.from_numpy(W.random_perm(ws.H, D, ws.seed)).to(device) if ws.perm else None
+        self.tables = TA.make_tables(perm=perm, rope_cs=TA.rope_table(cap, D, device=device))
+        self.packed = TA.alloc_packed(self.d_pre, device)
+        ks = torch.from_numpy(W.kv_tensor(ws, "k")).to(device)
+        TA.encode(self.d_pre, ks, self.tables, self.packed)
+        del ks
+        self.app_host = W.kv_tensor(ws, "k_append", T=ws.append)
+        self.app = torch.from_numpy(self.app_host).to(device)
+        self.q_host = W.queries(ws)
+        self.q = torch.from_numpy(self.q_host).to(device)
+        self.scores = torch.empty((ws.B, ws.Hq, self.n_tok), dtype=torch.float32, device=device)
+        self.scale = 1.0 / math.sqrt(D)
+        rb, ng = D * ws.bits // 8, D // ws.group
+        self.alg_append = ws.B * ws.H * ws.append * (2 * D + rb + 4 * ng)
+        self.alg_score = (ws.B * ws.H * (self.n_tok - ws.n_sink) * (rb + 4 * ng) + ws.B * ws.H * ws.n_sink * D * 2
+                          + ws.B * ws.Hq * D * 2 + ws.B * ws.Hq * self.n_tok * 4)
+        self.fp16_append = ws.B * ws.H * ws.append * 2 * D
+        self.fp16_score = ws.B * ws.H * self.n_tok * 2 * D
+        self.append = TA.bind_encode(self.d_app, self.app, self.tables, self.packed)
+        self.score = TA.bind_score(self.d_pre, self.q, self.packed, self.tables, self.n_tok, self.scale, self.scores)
+
+
+class EncDecStep:
+    """Encode then decode of K (and V when `both`) for one workload."""
+
+    def __init__(self, name, device, both=True, batch=None):
+        import torch
+        from kv_cache_rotation_b200 import torch_api as TA
+        self.workload = name
+        w = W.WORKLOADS[name] if batch is None else W.scaled(W.WORKLOADS[name], B=batch)
+        self.TA = TA
+        B, H, T, D = w.B, w.H, w.T, w.D
+        iso = w.rot == "iso"
+        tensors = ["k", "v"] if both and not iso else ["k"]
+        self.items = []
+        self.alg, self.fp16_equiv, self.kernels = {}, {}, {}
+        kern = {"fwht_head": "head", "none": "head", "fwht_group": "group", "iso": "iso"}[w.rot]
+        for which in tensors:
+            x = (W.kv_tensor_device(w, which, device) if iso else torch.from_numpy(W.kv_tensor(w, which)).to(device))
+            rope = 1 if (which == "k" and w.rope_k) else 0
+            d = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, bits=w.bits, group=w.group,
+                             group_heads=w.group_heads, rope=rope, n_sink=w.n_sink, rot=w.rot, quant=w.quant)
+            perm = torch.from_numpy(W.random_perm(H, D, w.seed + len(which))).to(device) if w.perm else None
+            if iso:
+                qL, qR = W.iso_tables(w)
+                tb = TA.make_tables(qL=torch.from_numpy(qL).to(device), qR=torch.from_numpy(qR).to(device),
+                                    codebook=TA.lloyd_max_codebook(w.bits, D, device=device))
+            else:
+                tb = TA.make_tables(perm=perm, rope_cs=TA.rope_table(T, D, device=device) if rope else None)
+            pk = TA.alloc_packed(d, device)
+            out = torch.empty((B, H, T, D), dtype=torch.float16, device=device)
+            self.items.append((which, d, x, tb, pk, out))
+            nvec = B * H * T
+            per_vec = D * w.bits // 8 + (4 * (D // w.group) if w.quant == "minmax" else 4)
+            self.alg[f"encode_{which}"] = nvec * (2 * D + per_vec) + (B * H * w.n_sink * D * 2)
+            self.alg[f"decode_{which}"] = nvec * (2 * D + per_vec)
+            self.fp16_equiv[f"encode_{which}"] = nvec * 2 * D
+            self.fp16_equiv[f"decode_{which}"] = nvec * 2 * D
+            self.kernels[f"encode_{which}"] = f"k_encode_{kern}"
+            self.kernels[f"decode_{which}"] = f"k_decode_{kern}"
+        self.names = list(self.alg)
+        torch.cuda.synchronize(device)
+
+    def launches(self):
+        TA = self.TA
+        fs = [TA.bind_encode(d, x, tb, pk) for which, d, x, tb, pk, out in self.items]
+        fs += [TA.bind_decode(d, pk, tb, out) for which, d, x, tb, pk, out in self.items]
+        return fs
+
+
+class DecodeScoreStep:
+    """Decode step of the batch-64 MHA cache: append one token, score all slots."""
+
+    workload = "decode_score"
+
+    def __init__(self, device):
+        import torch
+        self.sc = ScoreCache(W.WORKLOADS["decode_score"], device)
+        self.alg = {"append": self.sc.alg_append, "score": self.sc.alg_score}
+        self.fp16_equiv = {"append": self.sc.fp16_append, "score": self.sc.fp16_score}
+        self.kernels = {"append": "k_encode_head", "score": "k_score_mma"}
+        self.names = list(self.alg)
+        torch.cuda.synchronize(device)
+
+    def launches(self):
+        return [self.sc.append, self.sc.score]
+
+
+def make_step(workload, device, batch=None):
+    if workload == "llama3_8b_gqa":
+        return Step(device)
+    if workload == "decode_score":
+        return DecodeScoreStep(device)
+    return EncDecStep(workload, device, batch=batch)
 
 
 def _kernel_sources_sha(names):
@@ -217,34 +320,28 @@ def _traffic_for(kernel):
     return e.get("dram_bytes_per_launch")
 
 
-KERNEL_SOURCES = {
-    "encode_k": ("k_encode_group", ["kvq_group.cu", "kvq_device.cuh"]),
-    "encode_v": ("k_encode_group", ["kvq_group.cu", "kvq_device.cuh"]),
-    "decode_k": ("k_decode_group", ["kvq_group.cu", "kvq_device.cuh"]),
-    "decode_v": ("k_decode_group", ["kvq_group.cu", "kvq_device.cuh"]),
-    "append": ("k_encode_head", ["kvq_head.cu", "kvq_device.cuh"]),
-    "score": ("k_score", ["kvq_score.cu", "kvq_device.cuh"]),
-}
-
-
 # ---------------------------------------------------------------- CPU oracle timing
-def cpu_sample(seconds_hint: float = 10.0, tokens: int = None, t_offset: int = 0):
-    """Time the oracle on a bounded sample of the same workload: batch 0 (all
-    8 KV heads) over `tokens` tokens for encode/decode of K and V, and the
-    score of batch 0's 32 query heads over as many cache slots. Returns
-    (fp16-equivalent bytes, seconds, description)."""
+def cpu_sample(seconds_hint: float = 10.0, tokens: int = None, t_offset: int = 0, batches: int = None):
+    """Time the oracle on a bounded sample of the same workload: the first
+    `batches` sequences (all 8 KV heads) over `tokens` tokens for
+    encode/decode of K and V, and the score of their 32 query heads each over
+    as many cache slots. The default (2 full sequences of 32768 tokens) is
+    about 10 s of single-thread CPU work. Returns (fp16-equivalent bytes,
+    seconds, description)."""
     import oracle
     wg, ws = W.WORKLOADS["llama3_8b_gqa"], W.WORKLOADS["llama3_8b_gqa_score"]
     if tokens is None:
-        tokens = 4096 if seconds_hint >= 5 else 512
-    Tn = tokens
-    k = W.kv_tensor(W.scaled(wg, T=Tn, B=1, seed=wg.seed * 1000 + t_offset), "k").view(np.uint16)
-    v = W.kv_tensor(W.scaled(wg, T=Tn, B=1, seed=wg.seed * 1000 + t_offset), "v").view(np.uint16)
+        tokens = wg.T if seconds_hint >= 5 else 512
+    if batches is None:
+        batches = 2 if seconds_hint >= 5 else 1
+    Tn, Bn = tokens, batches
+    k = W.kv_tensor(W.scaled(wg, T=Tn, B=Bn, seed=wg.seed * 1000 + t_offset), "k").view(np.uint16)
+    v = W.kv_tensor(W.scaled(wg, T=Tn, B=Bn, seed=wg.seed * 1000 + t_offset), "v").view(np.uint16)
     pos = np.arange(t_offset, t_offset + Tn)
     kwk = dict(rot=oracle.ROT_FWHT_GROUP, bits=wg.bits, group=wg.group, group_heads=wg.group_heads, rope=1)
     kwv = dict(kwk, rope=0)
-    ks = W.kv_tensor(W.scaled(ws, T=Tn, B=1, seed=ws.seed * 1000 + t_offset), "k").view(np.uint16)
-    q = W.queries(ws, B=1).view(np.uint16)
+    ks = W.kv_tensor(W.scaled(ws, T=Tn, B=Bn, seed=ws.seed * 1000 + t_offset), "k").view(np.uint16)
+    q = W.queries(ws, B=Bn).view(np.uint16)
     kws = dict(rot=oracle.ROT_FWHT_HEAD, bits=ws.bits, group=ws.group, rope=1, n_sink=ws.n_sink)
     cache = oracle.encode(ks, np.arange(Tn), **kws)
     t0 = time.perf_counter()
@@ -254,9 +351,9 @@ def cpu_sample(seconds_hint: float = 10.0, tokens: int = None, t_offset: int = 0
     oracle.decode(pv, pos, v.shape, **kwv)
     oracle.score(q, cache, np.arange(Tn), H=ws.H, t_cap=Tn, scale=1 / math.sqrt(ws.D), **kws)
     dt = time.perf_counter() - t0
-    nbytes = 5 * wg.H * Tn * wg.D * 2  # 4 x (encode/decode of one tensor) + the score's key bytes
-    desc = (f"oracle (plain C, 1 thread): batch 1 of {wg.B}, {Tn} of {wg.T} tokens: encode+decode of K and V "
-            f"(grouped FWHT) and the score of 32 query heads over {Tn} cache slots")
+    nbytes = 5 * Bn * wg.H * Tn * wg.D * 2  # 4 x (encode/decode of one tensor) + the score's key bytes
+    desc = (f"oracle (plain C, 1 thread): {Bn} of {wg.B} sequences, {Tn} of {wg.T} tokens: encode+decode of K "
+            f"and V (grouped FWHT) and the score of 32 query heads per sequence over {Tn} cache slots")
     return nbytes, dt, desc
 
 
@@ -300,7 +397,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     import kv_cache_rotation_b200 as K
-    st = Step(dev)
+    st = make_step(args.workload, dev, args.batch)
     launches = st.launches()
     stream = torch.cuda.current_stream(dev)
 
@@ -352,18 +449,22 @@ def run_ours(args):
     dom_ms = per_kernel[dom] / args.steps
     achieved = st.alg[dom] / (dom_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": _traffic_for(KERNEL_SOURCES[dom][0]), "kernel": KERNEL_SOURCES[dom][0],
+                "traffic": _traffic_for(st.kernels[dom]), "kernel": st.kernels[dom],
                 "kernel_step": dom, "alg_bytes_per_launch": st.alg[dom], "peak_kind": peak_kind}
 
-    e2e = run_e2e(st, launches, dev, stream, min(args.steps, args.e2e_steps), args.warmup_e2e)
-    if dist:
-        t = torch.tensor([e2e["ms_per_step"]], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms_per_step"] = float(t.item())
-    e2e_value = world * fp16_step / (e2e["ms_per_step"] / 1e3) / 1e9
+    e2e_line = None
+    if hasattr(st, "host_in"):
+        e2e = run_e2e(st, launches, dev, stream, min(args.steps, args.e2e_steps), args.warmup_e2e)
+        if dist:
+            t = torch.tensor([e2e["ms_per_step"]], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e["ms_per_step"] = float(t.item())
+        e2e_line = {"value": world * fp16_step / (e2e["ms_per_step"] / 1e3) / 1e9, "unit": UNIT,
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "ms_per_step": e2e["ms_per_step"], "steps": e2e["steps"]}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu and args.workload == "llama3_8b_gqa":
         b, s, desc = cpu_sample()
         cpu = {"value": b / s / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                "seconds": s}
@@ -372,9 +473,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": _config(world), "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
-                    "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms_per_step"], "steps": e2e["steps"]},
+            "config": _config(world) if args.workload == "llama3_8b_gqa" else _other_config(args.workload, world),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e_line,
             "gpu_launches": nk * args.steps, "clocks": clk.summary(), "kernels": kernels,
             "status": K.kvq_status_str(status),
         }
@@ -386,13 +486,13 @@ def run_ours(args):
 
 
 def run_e2e(st, launches, dev, stream, steps, warmup):
-    """Same step through host buffers: pinned K, V, the appended token and q
-    are copied in, and every result the step produces (packed K/V, decoded
-    K/V, scores) is copied back, inside the timed region."""
+    """Same step through host buffers: the step's inputs are copied in from
+    pinned host memory and every result it produces is copied back, inside
+    the timed region."""
     import torch
-    h_in = [torch.from_numpy(a).pin_memory() for a in (st.k_host, st.v_host, st.app_host, st.q_host)]
-    d_in = [st.k, st.v, st.app, st.q]
-    d_out = [st.pk.codes, st.pk.scale_zero, st.pv.codes, st.pv.scale_zero, st.ok, st.ov, st.scores]
+    h_in = [torch.from_numpy(a).pin_memory() for a in st.host_in]
+    d_in = st.dev_in
+    d_out = st.dev_out
     h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
     h2d = sum(t.numel() * t.element_size() for t in h_in)
     d2h = sum(t.numel() * t.element_size() for t in h_out)
@@ -417,6 +517,14 @@ def run_e2e(st, launches, dev, stream, steps, warmup):
     return {"ms_per_step": a.elapsed_time(b) / steps, "h2d": h2d, "d2h": d2h, "steps": steps}
 
 
+def _other_config(name, n_gpus):
+    w = W.WORKLOADS[name]
+    return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T, "q_heads": w.Hq,
+            "rotation": w.rot, "quant": w.quant, "bits": w.bits, "group": w.group, "n_sink": w.n_sink,
+            "perm": w.perm, "l2": "no flush (inputs larger than L2)" if name != "tiny" else "L2-resident",
+            "parallelism": f"replicas x{n_gpus}"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -427,6 +535,11 @@ def main():
     ap.add_argument("--warmup-e2e", type=int, default=3)
     ap.add_argument("--ref-tokens", type=int, default=512, help="tokens per reference-arm step")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--workload", default="llama3_8b_gqa",
+                    choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "decode_score", "tiny"],
+                    help="which workload a step runs (the headline line is llama3_8b_gqa)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the batch of an encode/decode workload (small profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -40,6 +40,7 @@ constexpr int kStageX = 32768;  // x tile, exchange half and output tile (fp16)
 
 struct GroupArgs {
   int B, H, T, t0, t_cap, n_sink, rope, n_tblk, n_grp, n_tiles;
+  FastDiv div_grp, div_b;  // head groups per batch; batches
   float rscale;  // fp32(1/sqrt(HG*128))
   const int16_t* perm;
   const float* rope_cs;  // [rows][128/2][2]
@@ -71,11 +72,12 @@ __device__ __forceinline__ uint32_t xpos(int t, int c) {
 // token block -- and so the same RoPE rows -- run at the same time.
 __device__ __forceinline__ void tile_coords(const GroupArgs& a, int tile, int HG, int NT, int& b, int& h_base,
                                             int& t_base) {
-  const int grp = tile % a.n_grp;
-  const int rest = tile / a.n_grp;
-  b = rest % a.B;
-  t_base = (rest / a.B) * NT;
-  h_base = grp * HG;
+  const uint32_t rest = a.div_grp.div(tile);
+  const uint32_t grp = a.div_grp.mod(tile, rest);
+  const uint32_t tb = a.div_b.div(rest);
+  b = static_cast<int>(a.div_b.mod(rest, tb));
+  t_base = static_cast<int>(tb) * NT;
+  h_base = static_cast<int>(grp) * HG;
 }
 
 // Bytes of one stage: the x tile, which later carries the exchange halves
@@ -721,11 +723,9 @@ kvq_status run(bool enc, const GroupArgs& a, const CUtensorMap& m0, int out_fp32
   const size_t smem = 1024 + static_cast<size_t>(kStages) * stage_bytes<HG>();
   const void* fn = enc ? reinterpret_cast<const void*>(k_encode_group<HG, BITS, G>)
                        : reinterpret_cast<const void*>(k_decode_group<HG, BITS, G>);
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+  if (!set_smem_once(reinterpret_cast<const void*>(fn), smem))
     return KVQ_ERR_CUDA;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 128, smem) != cudaSuccess || per_sm < 1)
-    per_sm = 1;
+  const int per_sm = occupancy_once(fn, 128, smem);
   const long long want = static_cast<long long>(ctx.num_sms) * per_sm;
   const unsigned grid = static_cast<unsigned>(a.n_tiles < want ? a.n_tiles : want);
   if (enc)
@@ -764,6 +764,8 @@ GroupArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p
   a.n_tblk = (d.tokens + NT - 1) / NT;
   a.n_grp = d.heads / d.group_heads;
   a.n_tiles = d.batch * a.n_grp * a.n_tblk;
+  a.div_grp = FastDiv(static_cast<uint32_t>(a.n_grp));
+  a.div_b = FastDiv(static_cast<uint32_t>(d.batch));
   a.rscale = static_cast<float>(1.0 / sqrt(static_cast<double>(d.group_heads) * D));
   a.perm = tb.perm;
   a.rope_cs = tb.rope_cs;

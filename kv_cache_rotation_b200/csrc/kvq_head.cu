@@ -347,7 +347,7 @@ template <int D, int BITS, int G, bool ROT>
 kvq_status run_encode(const HeadArgs& a, const CUtensorMap& xm, const CUtensorMap& rm, size_t smem,
                       cudaStream_t st) {
   auto k = k_encode_head<D, BITS, G, ROT>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+  if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
     return KVQ_ERR_CUDA;
   const size_t grid = static_cast<size_t>(a.B) * a.n_hblk * a.n_tblk;
   k<<<static_cast<unsigned>(grid), 128, smem, st>>>(xm, rm, a);
@@ -357,7 +357,7 @@ template <int D, int BITS, int G, bool ROT>
 kvq_status run_decode(const HeadArgs& a, const CUtensorMap& om, const CUtensorMap& rm, size_t smem, int out_fp32,
                       cudaStream_t st) {
   auto k = k_decode_head<D, BITS, G, ROT>;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+  if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
     return KVQ_ERR_CUDA;
   const size_t grid = static_cast<size_t>(a.B) * a.n_hblk * a.n_tblk;
   k<<<static_cast<unsigned>(grid), 128, smem, st>>>(om, rm, a, out_fp32);

@@ -45,6 +45,56 @@ kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq
                         const LaunchCtx& ctx);
 kvq_status launch_debug_wait(uint64_t limit_ns, cudaStream_t st, const LaunchCtx& ctx);
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) only when a kernel needs
+// more dynamic shared memory on this device than it was last granted (the
+// attribute persists per device). A small per-thread cache of (kernel,
+// device, bytes) keeps the host cost of repeated launches low.
+inline bool set_smem_once(const void* fn, size_t bytes) {
+  struct Entry {
+    const void* fn;
+    int dev;
+    size_t bytes;
+  };
+  static thread_local Entry cache[32];
+  static thread_local int n = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  for (int i = 0; i < n; ++i)
+    if (cache[i].fn == fn && cache[i].dev == dev && bytes <= cache[i].bytes) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+      cudaSuccess)
+    return false;
+  for (int i = 0; i < n; ++i)
+    if (cache[i].fn == fn && cache[i].dev == dev) {
+      cache[i].bytes = bytes;
+      return true;
+    }
+  cache[n < 32 ? n++ : 31] = Entry{fn, dev, bytes};
+  return true;
+}
+
+// Resident CTAs per SM of a kernel (cached per kernel, device and smem size).
+inline int occupancy_once(const void* fn, int threads, size_t smem) {
+  struct Entry {
+    const void* fn;
+    int dev, threads;
+    size_t smem;
+    int per_sm;
+  };
+  static thread_local Entry cache[32];
+  static thread_local int n = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  for (int i = 0; i < n; ++i)
+    if (cache[i].fn == fn && cache[i].dev == dev && cache[i].threads == threads && cache[i].smem == smem)
+      return cache[i].per_sm;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  cache[n < 32 ? n++ : 31] = Entry{fn, dev, threads, smem, per_sm};
+  return per_sm;
+}
+
 // Finish a launch: map a launch error to a status.
 inline kvq_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;

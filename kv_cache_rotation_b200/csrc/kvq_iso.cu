@@ -258,13 +258,13 @@ kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, 
   if (enc) {
     const size_t smem = 1024 + D * 256;
     auto k = k_encode_iso<D, BITS>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
     k<<<grid, 128, smem, st>>>(m0, a);
   } else {
     const size_t smem = 1024 + D * 512;
     auto k = k_decode_iso<D, BITS>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
     k<<<grid, 128, smem, st>>>(m0, a, out_fp32);
   }

@@ -32,7 +32,7 @@ struct ScoreArgs {
 constexpr int kThreads = 256;
 
 template <int D, int BITS, int G, int GQ>
-__global__ void __launch_bounds__(kThreads) k_score(const ScoreArgs a) {
+__global__ void __launch_bounds__(kThreads) k_score_simt(const ScoreArgs a) {
   constexpr int NG = D / G;
   constexpr int NW = D * BITS / 32;
   constexpr int RB = D * BITS / 8;
@@ -144,10 +144,348 @@ __global__ void __launch_bounds__(kThreads) k_score(const ScoreArgs a) {
     a.scores[(static_cast<size_t>(b) * a.Hq + h * GQ + i) * a.n_tok + n] = __fmul_rn(acc[i], a.scale);
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core score (head_dim 128, 2- or 4-bit codes).
+//
+// Per (batch, KV head) the rotated queries qt = H P q of the GQ query heads
+// are quantized once to 16-bit integers Q = rint(qt / sq), sq = max|qt| / 32000,
+// and split into two int8 digits Q = 256 hi + lo. A warp then scores 16
+// tokens at a time with mma.sync m16n8k32 (u8 codes x s8 digits, exact int32
+// accumulation): A = the codes expanded to one byte each by a shift and a
+// mask per 4 codes, B = the digits, N = 2 columns (lo, hi) per query head.
+//   s_n = scale * sum_g ( S_g * sq * (sum_j c_j lo_j + 256 sum_j c_j hi_j) + Z_g * sum_{j in g} qt_j ).
+// The digit rounding moves each score by at most S * sq / 2 * sum_j c_j,
+// i.e. below 2e-5 of the score's L1 magnitude. Codes stream through shared
+// memory by bulk copy, two tiles of 128 tokens in flight; CTAs are
+// persistent over a range of tiles of one (batch, KV head) so the query
+// rotation is done once per CTA.
+// Tiling (compile-time tunables).
+#ifndef KVQ_SCORE_MT
+#define KVQ_SCORE_MT 2
+#endif
+#ifndef KVQ_SCORE_STAGES
+#define KVQ_SCORE_STAGES 4
+#endif
+#ifndef KVQ_SCORE_CTAS_PER_SM
+#define KVQ_SCORE_CTAS_PER_SM 4
+#endif
+constexpr int kMmaThreads = 256;
+constexpr int kMmaMT = KVQ_SCORE_MT;              // 16-token m-tiles per warp per tile
+constexpr int kMmaTile = 8 * 16 * kMmaMT;         // tokens per tile
+constexpr int kMmaStages = KVQ_SCORE_STAGES;      // tiles in flight per CTA
+
+struct MmaArgs {
+  ScoreArgs s;
+  int chunks, tiles_per_chunk;
+  FastDiv div_tpb, div_h;  // tiles per (batch, KV head); KV heads
+  uint32_t* err;
+  uint64_t wait_ns;
+};
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Channel that K index (k-step s, lane quad position tig, byte l, upper half u)
+// of the A fragment carries; B uses the same map.
+template <int BITS>
+__device__ __forceinline__ int kchan(int s, int tig, int l, int u) {
+  if constexpr (BITS == 2) return 32 * s + 16 * u + 4 * l + tig;
+  else return 32 * s + 16 * u + 8 * (tig >> 1) + 2 * l + (tig & 1);
+}
+
+template <int BITS, int G, int GQ>
+__global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
+  constexpr int D = 128;
+  constexpr int RB = D * BITS / 8;
+  constexpr int NW = RB / 4;             // words per record
+  constexpr int NTN = (2 * GQ + 7) / 8;  // n-tiles of 8 columns
+  constexpr int NGK = D / G;             // quantization groups per record
+  constexpr uint32_t MASK = BITS == 2 ? 0x03030303u : 0x0F0F0F0Fu;
+  const ScoreArgs& a = ma.s;
+  extern __shared__ __align__(128) uint8_t codes_dyn[];  // kMmaStages tiles of kMmaTile records
+  __shared__ __align__(16) uint2 bfrag[NTN][4][4][8];
+  __shared__ __align__(16) float qraw[GQ][D];
+  __shared__ int8_t qd[GQ][2][D];
+  __shared__ float qsum[GQ][NGK];
+  __shared__ float sqh[GQ];
+  __shared__ __align__(8) uint64_t full[kMmaStages];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  // this CTA's contiguous range of global tiles (batch-major, then KV head, then token tile)
+  const int total = a.B * a.H * static_cast<int>(ma.div_tpb.d);
+  const int gt0 = static_cast<int>(static_cast<long long>(total) * blockIdx.x / gridDim.x);
+  const int gt1 = static_cast<int>(static_cast<long long>(total) * (blockIdx.x + 1) / gridDim.x);
+  if (gt0 >= gt1) return;
+
+  auto issue = [&](int gt, int st) {
+    const int bh = static_cast<int>(ma.div_tpb.div(gt));
+    const int n0 = static_cast<int>(ma.div_tpb.mod(gt, bh)) * kMmaTile;
+    const uint32_t bytes = static_cast<uint32_t>(min(kMmaTile, a.n_tok - n0) * RB);
+    mbar_arrive_expect_tx(&full[st], bytes);
+    bulk_load(codes_dyn + st * (kMmaTile * RB), a.codes + (static_cast<size_t>(bh) * a.t_cap + n0) * RB, bytes,
+              &full[st]);
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kMmaStages; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int i = 0; i < kMmaStages && gt0 + i < gt1; ++i) issue(gt0 + i, i);
+  }
+
+  // rotated, digit-split queries of one (batch, KV head); warp w < GQ handles query head w
+  auto prologue = [&](int b, int h, bool with_sinks) {
+    __syncthreads();  // previous (batch, head) fully consumed
+    if (warp < GQ) {
+      const int qh = h * GQ + warp;
+      const __half* qv = a.q + (static_cast<size_t>(b) * a.Hq + qh) * D;
+      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qv) + lane);  // channels 4 lane .. 4 lane + 3
+      const float2 r01 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+      const float2 r23 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+      float v[4] = {r01.x, r01.y, r23.x, r23.y};
+      *reinterpret_cast<float4*>(&qraw[warp][4 * lane]) = make_float4(v[0], v[1], v[2], v[3]);
+      if (a.perm) {
+        const uint2 pk = __ldg(reinterpret_cast<const uint2*>(a.perm + static_cast<size_t>(h) * D) + lane);
+        const uint32_t pw[2] = {pk.x, pk.y};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = __half2float(qv[(pw[i >> 1] >> (16 * (i & 1))) & (D - 1)]);
+      }
+      if (a.rot == KVQ_ROT_FWHT_HEAD) {
+        const float t0 = v[0] + v[1], t1 = v[0] - v[1], t2 = v[2] + v[3], t3 = v[2] - v[3];
+        v[0] = t0 + t2; v[2] = t0 - t2; v[1] = t1 + t3; v[3] = t1 - t3;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float p = __shfl_xor_sync(0xffffffffu, v[i], m);
+            v[i] = (lane & m) ? (p - v[i]) : (v[i] + p);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] *= a.rscale;
+      }
+      float mx = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+      const float sq = mx > 0.0f ? mx / 32000.0f : 1.0f;
+      const float rsq = 1.0f / sq;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int Q = __float2int_rn(v[i] * rsq);
+        const int lo = ((Q + 128) & 255) - 128;
+        qd[warp][0][4 * lane + i] = static_cast<int8_t>(lo);
+        qd[warp][1][4 * lane + i] = static_cast<int8_t>((Q - lo) >> 8);
+      }
+      float ps = (v[0] + v[1]) + (v[2] + v[3]);
+#pragma unroll
+      for (int m = 1; m < G / 4; m <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
+      if ((lane & (G / 4 - 1)) == 0) qsum[warp][lane / (G / 4)] = ps;
+      if (lane == 0) sqh[warp] = sq;
+    }
+    __syncthreads();
+    for (int e = tid; e < NTN * 128; e += kMmaThreads) {  // B fragments: column c = 2 * head + digit
+      const int nt = e >> 7, s = (e >> 5) & 3, tg = (e >> 3) & 3, n = e & 7;
+      const int c = nt * 8 + n, hh = c >> 1, dg = c & 1;
+      uint32_t b0 = 0, b1 = 0;
+      if (hh < GQ) {
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+          b0 |= static_cast<uint32_t>(static_cast<uint8_t>(qd[hh][dg][kchan<BITS>(s, tg, l, 0)])) << (8 * l);
+          b1 |= static_cast<uint32_t>(static_cast<uint8_t>(qd[hh][dg][kchan<BITS>(s, tg, l, 1)])) << (8 * l);
+        }
+      }
+      bfrag[nt][s][tg][n] = make_uint2(b0, b1);
+    }
+    __syncthreads();
+    // fp16 sinks of this (batch, head): s = scale * q . RoPE_n(sink_n); done by the
+    // CTA that owns the (batch, head)'s first tile, one warp per (sink, query head)
+    if (with_sinks) {
+      const size_t vh = static_cast<size_t>(b) * a.H + h;
+      for (int e = warp; e < min(a.n_sink, a.n_tok) * GQ; e += kMmaThreads / 32) {
+        const int n = e / GQ, hh = e % GQ;
+        const uint2 kr = __ldg(reinterpret_cast<const uint2*>(a.sink + (vh * a.n_sink + n) * D) + lane);
+        const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kr.x));
+        const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kr.y));
+        float k4[4] = {k01.x, k01.y, k23.x, k23.y};
+        if (a.rope) {  // pairs 2 lane and 2 lane + 1 of position n
+          const float4 cs = __ldg(reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(n) * D) + lane);
+          rope_fwd(k4[0], k4[1], cs.x, cs.y);
+          rope_fwd(k4[2], k4[3], cs.z, cs.w);
+        }
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc = __fmaf_rn(qraw[hh][4 * lane + i], k4[i], acc);
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+        if (lane == 0) a.scores[(static_cast<size_t>(b) * a.Hq + h * GQ + hh) * a.n_tok + n] = acc * a.scale;
+      }
+    }
+  };
+  // scale / zero of this thread's tokens of one tile (register prefetch)
+  auto load_sz = [&](int gt, __half2 (&sza)[kMmaMT][NGK], __half2 (&szb)[kMmaMT][NGK]) {
+    const int bh = static_cast<int>(ma.div_tpb.div(gt));
+    const int n0 = static_cast<int>(ma.div_tpb.mod(gt, bh)) * kMmaTile;
+#pragma unroll
+    for (int mt = 0; mt < kMmaMT; ++mt) {
+      const int na = n0 + warp * 16 * kMmaMT + mt * 16 + g, nb = na + 8;
+#pragma unroll
+      for (int q = 0; q < NGK; ++q) {
+        sza[mt][q] = na < a.n_tok ? a.sz[(static_cast<size_t>(bh) * a.t_cap + na) * NGK + q] : __half2();
+        szb[mt][q] = nb < a.n_tok ? a.sz[(static_cast<size_t>(bh) * a.t_cap + nb) * NGK + q] : __half2();
+      }
+    }
+  };
+
+  __half2 sza[kMmaMT][NGK], szb[kMmaMT][NGK];
+  load_sz(gt0, sza, szb);
+  int cur_bh = -1;
+  bool ok = true;
+  for (int gt = gt0; gt < gt1; ++gt) {
+    const int it = gt - gt0;
+    const int st = it % kMmaStages;
+    const int bh = static_cast<int>(ma.div_tpb.div(gt));
+    const int b = static_cast<int>(ma.div_h.div(bh)), h = bh - b * a.H;
+    const int n0 = static_cast<int>(ma.div_tpb.mod(gt, bh)) * kMmaTile;
+    if (bh != cur_bh) {
+      prologue(b, h, n0 == 0);
+      cur_bh = bh;
+    }
+    ok = mbar_wait(&full[st], (it / kMmaStages) & 1, ma.wait_ns, ma.err) && ok;
+    const uint32_t base = smem_u32(codes_dyn + st * (kMmaTile * RB));
+    int acc[kMmaMT][NGK][NTN][4];
+#pragma unroll
+    for (int mt = 0; mt < kMmaMT; ++mt) {
+      const int ra = warp * 16 * kMmaMT + mt * 16 + g;  // tile rows ra and ra + 8
+      uint32_t wa[NW], wb[NW];
+#pragma unroll
+      for (int i = 0; i < NW / 4; ++i) {
+        const uint4 ua = lds128(base + ra * RB + 16 * i);
+        const uint4 ub = lds128(base + (ra + 8) * RB + 16 * i);
+        wa[4 * i] = ua.x; wa[4 * i + 1] = ua.y; wa[4 * i + 2] = ua.z; wa[4 * i + 3] = ua.w;
+        wb[4 * i] = ub.x; wb[4 * i + 1] = ub.y; wb[4 * i + 2] = ub.z; wb[4 * i + 3] = ub.w;
+      }
+#pragma unroll
+      for (int q = 0; q < NGK; ++q)
+#pragma unroll
+        for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[mt][q][nt][i] = 0;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        uint32_t a0, a1, a2, a3;
+        if constexpr (BITS == 2) {
+          a0 = (wa[2 * s] >> (2 * tig)) & MASK;
+          a1 = (wb[2 * s] >> (2 * tig)) & MASK;
+          a2 = (wa[2 * s + 1] >> (2 * tig)) & MASK;
+          a3 = (wb[2 * s + 1] >> (2 * tig)) & MASK;
+        } else {
+          const bool odd = (tig & 2) != 0;  // word 4s + (tig >> 1), selected without dynamic indexing
+          const int sh = 4 * (tig & 1);
+          a0 = ((odd ? wa[4 * s + 1] : wa[4 * s]) >> sh) & MASK;
+          a1 = ((odd ? wb[4 * s + 1] : wb[4 * s]) >> sh) & MASK;
+          a2 = ((odd ? wa[4 * s + 3] : wa[4 * s + 2]) >> sh) & MASK;
+          a3 = ((odd ? wb[4 * s + 3] : wb[4 * s + 2]) >> sh) & MASK;
+        }
+        constexpr int SPG = G / 32;  // k-steps per group
+        const int q = s / SPG;
+#pragma unroll
+        for (int nt = 0; nt < NTN; ++nt) {
+          const uint2 bb = bfrag[nt][s][tig][g];
+          asm volatile(
+              "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+              "{%0,%1,%2,%3};"
+              : "+r"(acc[mt][q][nt][0]), "+r"(acc[mt][q][nt][1]), "+r"(acc[mt][q][nt][2]),
+                "+r"(acc[mt][q][nt][3])
+              : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bb.x), "r"(bb.y));
+        }
+      }
+    }
+    // every warp has read this stage: refill it with the tile kMmaStages ahead
+    if (!__syncthreads_and(ok)) break;
+    if (tid == 0 && gt + kMmaStages < gt1) issue(gt + kMmaStages, st);
+    __half2 pa[kMmaMT][NGK], pb[kMmaMT][NGK];
+#pragma unroll
+    for (int mt = 0; mt < kMmaMT; ++mt)
+#pragma unroll
+      for (int q = 0; q < NGK; ++q) {
+        pa[mt][q] = sza[mt][q];
+        pb[mt][q] = szb[mt][q];
+      }
+    if (gt + 1 < gt1) load_sz(gt + 1, sza, szb);  // next tile's scale / zero
+    // epilogue: thread holds columns 2 tig (lo) and 2 tig + 1 (hi) = query head nt*4 + tig
+#pragma unroll
+    for (int mt = 0; mt < kMmaMT; ++mt) {
+      const int na = n0 + warp * 16 * kMmaMT + mt * 16 + g, nb = na + 8;
+#pragma unroll
+      for (int nt = 0; nt < NTN; ++nt) {
+        const int hh = nt * 4 + tig;
+        if (hh >= GQ) continue;
+        const float sq = sqh[hh];
+        float sa = 0.0f, sb = 0.0f;
+#pragma unroll
+        for (int q = 0; q < NGK; ++q) {
+          const float da = static_cast<float>(acc[mt][q][nt][0] + 256 * acc[mt][q][nt][1]);
+          const float db = static_cast<float>(acc[mt][q][nt][2] + 256 * acc[mt][q][nt][3]);
+          sa = __fmaf_rn(__low2float(pa[mt][q]) * sq, da, __fmaf_rn(__high2float(pa[mt][q]), qsum[hh][q], sa));
+          sb = __fmaf_rn(__low2float(pb[mt][q]) * sq, db, __fmaf_rn(__high2float(pb[mt][q]), qsum[hh][q], sb));
+        }
+        float* out = a.scores + (static_cast<size_t>(b) * a.Hq + h * GQ + hh) * a.n_tok;
+        if (na < a.n_tok && na >= a.n_sink) out[na] = sa * a.scale;
+        if (nb < a.n_tok && nb >= a.n_sink) out[nb] = sb * a.scale;
+      }
+    }
+  }
+  if (!ok && tid == 0) {
+    for (int st = 0; st < kMmaStages; ++st)
+      for (uint32_t p = 0; p < 2; ++p) mbar_wait(&full[st], p, ma.wait_ns, ma.err);
+  }
+}
+
+template <int BITS, int G, int GQ>
+kvq_status run_mma(const ScoreArgs& a, const LaunchCtx& ctx, cudaStream_t st) {
+  MmaArgs ma;
+  ma.s = a;
+  ma.err = ctx.err;
+  ma.wait_ns = ctx.wait_ns;
+  const size_t smem = static_cast<size_t>(kMmaStages) * kMmaTile * (128 * BITS / 8);
+  if (!set_smem_once(reinterpret_cast<const void*>(k_score_mma<BITS, G, GQ>), smem)) return KVQ_ERR_CUDA;
+  int per_sm = occupancy_once(reinterpret_cast<const void*>(k_score_mma<BITS, G, GQ>), kMmaThreads, smem);
+  per_sm = per_sm > KVQ_SCORE_CTAS_PER_SM ? KVQ_SCORE_CTAS_PER_SM : per_sm;
+  const int tpb = (a.n_tok + kMmaTile - 1) / kMmaTile;
+  const long long total = static_cast<long long>(a.B) * a.H * tpb;
+  if (total >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+  ma.div_tpb = FastDiv(static_cast<uint32_t>(tpb));
+  ma.div_h = FastDiv(static_cast<uint32_t>(a.H));
+  long long grid = static_cast<long long>(ctx.num_sms) * per_sm;
+  if (grid > total) grid = total;
+  ma.chunks = static_cast<int>(grid);
+  ma.tiles_per_chunk = 0;
+  k_score_mma<BITS, G, GQ><<<static_cast<unsigned>(grid), kMmaThreads, smem, st>>>(ma);
+  return launch_status();
+}
+
+template <int BITS, int G>
+kvq_status mma_by_gq(const ScoreArgs& a, int gq, const LaunchCtx& ctx, cudaStream_t st) {
+  switch (gq) {
+    case 1: return run_mma<BITS, G, 1>(a, ctx, st);
+    case 2: return run_mma<BITS, G, 2>(a, ctx, st);
+    case 4: return run_mma<BITS, G, 4>(a, ctx, st);
+    case 8: return run_mma<BITS, G, 8>(a, ctx, st);
+    default: return KVQ_ERR_UNSUPPORTED;
+  }
+}
+
 template <int D, int BITS, int G, int GQ>
 kvq_status run(const ScoreArgs& a, cudaStream_t st) {
   const dim3 grid((a.n_tok + kThreads - 1) / kThreads, a.H, a.B);
-  k_score<D, BITS, G, GQ><<<grid, kThreads, 0, st>>>(a);
+  k_score_simt<D, BITS, G, GQ><<<grid, kThreads, 0, st>>>(a);
   return launch_status();
 }
 
@@ -166,7 +504,7 @@ kvq_status by_gq(const ScoreArgs& a, int gq, cudaStream_t st) {
 
 kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq_packed& cache,
                         const kvq_tables& tb, int n_tokens, float scale, float* scores, cudaStream_t st,
-                        const LaunchCtx&) {
+                        const LaunchCtx& ctx) {
   ScoreArgs a{};
   a.B = d.batch;
   a.H = d.heads;
@@ -186,6 +524,17 @@ kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq
   a.sink = static_cast<const __half*>(cache.sink);
   a.scores = scores;
   const int gq = q_heads / d.heads;
+  if (d.head_dim == 128 && (d.bits == 2 || d.bits == 4)) {
+#define KVQ_MMA(B_, G_) \
+  if (d.bits == B_ && d.group == G_) return mma_by_gq<B_, G_>(a, gq, ctx, st);
+    KVQ_MMA(2, 128)
+    KVQ_MMA(2, 64)
+    KVQ_MMA(2, 32)
+    KVQ_MMA(4, 128)
+    KVQ_MMA(4, 64)
+    KVQ_MMA(4, 32)
+#undef KVQ_MMA
+  }
 #define KVQ_CASE(D_, B_, G_) \
   if (d.head_dim == D_ && d.bits == B_ && d.group == G_) return by_gq<D_, B_, G_>(a, gq, st);
 #define KVQ_BITS(D_, G_) KVQ_CASE(D_, 2, G_) KVQ_CASE(D_, 3, G_) KVQ_CASE(D_, 4, G_)

@@ -131,3 +131,46 @@ def score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens
           out: torch.Tensor, stream=None) -> None:
     check(kvq_score(d, q.data_ptr(), q.shape[1], packed.struct(), tables.struct(), n_tokens, scale,
                     out.data_ptr(), _stream(stream)), "kvq_score")
+
+
+# ---------------------------------------------------------------- pre-bound calls
+# The same marshalling, done once: the returned zero-argument callables hold
+# the ctypes structs and raw addresses and launch with no per-call Python
+# struct building (for tight loops such as a benchmark or a decode loop).
+def bind_encode(d: kvq_desc, x: torch.Tensor, tables: Tables, packed: Packed, stream=None):
+    from . import lib
+    tb, pk, st = tables.struct(), packed.struct(), _stream(stream)
+    args = (ctypes.byref(d), x.data_ptr(), ctypes.byref(tb), ctypes.byref(pk), st)
+    keep = (d, x, tables, packed, tb, pk)
+
+    def call():
+        check(lib.kvq_encode(*args), "kvq_encode")
+    call.keep = keep
+    return call
+
+
+def bind_decode(d: kvq_desc, packed: Packed, tables: Tables, out: torch.Tensor, stream=None):
+    from . import lib
+    tb, pk, st = tables.struct(), packed.struct(), _stream(stream)
+    fp32 = 1 if out.dtype == torch.float32 else 0
+    args = (ctypes.byref(d), ctypes.byref(pk), ctypes.byref(tb), out.data_ptr(), fp32, st)
+    keep = (d, packed, tables, out, tb, pk)
+
+    def call():
+        check(lib.kvq_decode(*args), "kvq_decode")
+    call.keep = keep
+    return call
+
+
+def bind_score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens: int, scale: float,
+               out: torch.Tensor, stream=None):
+    from . import lib
+    tb, pk, st = tables.struct(), packed.struct(), _stream(stream)
+    args = (ctypes.byref(d), q.data_ptr(), q.shape[1], ctypes.byref(pk), ctypes.byref(tb), n_tokens,
+            ctypes.c_float(scale), out.data_ptr(), st)
+    keep = (d, q, packed, tables, out, tb, pk)
+
+    def call():
+        check(lib.kvq_score(*args), "kvq_score")
+    call.keep = keep
+    return call
