@@ -7,22 +7,26 @@
 // strides -- and only then rotated by RoPE head slice by head slice; each
 // head slice is quantized with per-group min-max and packed.
 //
-// Persistent CTAs of 128 threads walk tiles of HG heads x NT tokens
-// (HG * NT = 128) of one batch. Each tile's fp16 rows and RoPE rows arrive
-// by TMA into one of two shared-memory stages, so the next tile streams in
-// while the current one is computed.
-//   phase 1: thread (head, token) holds one 128-channel row in registers and
-//            runs the 7 in-head FWHT strides;
-//   exchange: the rows go through the stage's buffer in two halves of 64
-//            channels (fp32, XOR-swizzled: conflict-free row writes and
-//            column reads);
-//   phase 2: thread (token, k) holds channels [k*C, (k+1)*C), C = 128/HG, of
-//            all HG heads, runs the cross-head strides, RoPE, the group
-//            min/max (a transpose-reduce across the lanes sharing a group,
-//            so each lane derives one head's fp16 scale/zero), quantizes and
-//            stores its slice of each head's packed record.
-// Decode runs the phases in reverse, staging its output through the same
-// buffers and writing it back by TMA.
+// Persistent CTAs of kThreads threads walk tiles of HG heads x NT tokens
+// (HG * NT = kThreads / 2 head rows) of one batch. Every thread holds 64
+// values:
+//   phase 1: thread (half s, head, token) holds channels [64s, 64s + 64) of
+//            one head row (loaded straight from global memory, the next
+//            tile's row prefetched into registers) and runs the strides
+//            1 .. 32;
+//   exchange: the rows go through shared memory as fp32 in 16-byte chunks of
+//            four channels (rows padded to 17 chunks: every access is a base
+//            address plus a constant, and conflict-free);
+//   phase 2: thread (token, k) holds, for every head of the group and both
+//            halves, the 4Q channels [4kQ, 4kQ + 4Q) (Q = 8/HG), runs the
+//            stride 64 and the cross-head strides, RoPE, the group min/max (a
+//            transpose-reduce over the 2*HG lanes of the token; one lane per
+//            group derives its fp16 scale/zero and publishes (Z, 1/S) in
+//            shared memory), quantizes and packs.
+// Decode streams the packed codes in by TMA and the scales by cp.async, runs
+// the phases in reverse and stores its output rows straight to global memory.
+// The kernels are bound by the fp32 pipe and shared-memory bandwidth, not by
+// HBM: the exchange is the one transpose the stride order forces.
 //
 // Arithmetic is fp32 with the oracle's operation order, two lanes at a time
 // (sm_100 packed fp32 add / mul / fma). The FWHT normalisation 1/sqrt(HG*128)
@@ -35,15 +39,34 @@ namespace kvq {
 namespace {
 
 constexpr int D = 128;
-constexpr int kStages = 2;
-constexpr int kStageX = 32768;  // x tile, exchange half and output tile (fp16)
+#ifndef KVQ_GROUP_CT
+#define KVQ_GROUP_CT 64
+#endif
+constexpr int kThreads = KVQ_GROUP_CT;  // threads per CTA (64, 128 or 256)
+constexpr int kRows = kThreads / 2;     // head rows per tile
+constexpr int kPitch = 272;             // exchange row: 16 chunks of 16 bytes + one pad chunk
+constexpr int kXch = kRows * kPitch;    // fp32 exchange of one 64-channel half
+constexpr int kCodes = kRows * 64;      // packed codes of one tile (at most 64 bytes a row)
+constexpr int kStage = 264;             // row pitch of the fp16 staging used by the permutation
+constexpr int kHalf = kRows * 128;      // decode: one 64-channel half of the fp16 output tile (one TMA box)
+constexpr int kXchS = kRows * 256;      // decode: XOR-swizzled fp32 exchange of one 64-channel half
+static_assert(kRows >= 32 && kRows <= 128 && (kRows & (kRows - 1)) == 0, "unsupported CTA size");
+#ifndef KVQ_GROUP_PRELOAD
+#define KVQ_GROUP_PRELOAD 0
+#endif
+// 1: encode loads the next tile's rows into registers during phase 2 (more
+// registers); 0: each tile's rows are loaded when the tile starts.
+constexpr bool kPreload = KVQ_GROUP_PRELOAD != 0;
 
 struct GroupArgs {
   int B, H, T, t0, t_cap, n_sink, rope, n_tblk, n_grp, n_tiles;
+  int v8;                  // the fp16 / fp32 rows may be moved with 32-byte accesses
   FastDiv div_grp, div_b;  // head groups per batch; batches
-  float rscale;  // fp32(1/sqrt(HG*128))
+  float rscale;            // fp32(1/sqrt(HG*128))
+  const __half* x;         // encode input [B][H][T][128]
+  void* out;               // decode output [B][H][T][128], fp16 or fp32
   const int16_t* perm;
-  const float* rope_cs;  // [rows][128/2][2]
+  const float* rope_cs;    // [rows][128/2][2]
   uint8_t* codes;
   __half2* sz;
   __half* sink;
@@ -62,10 +85,62 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ void bfly(float2& a, float2& b) {
+  const float2 p = a, q = b;
+  a = add2(p, q);
+  b = sub2(p, q);
+}
 
-// 16-byte chunk c (0..15) of the 64-channel exchange row (t, h) -> position.
-__device__ __forceinline__ uint32_t xpos(int t, int c) {
-  return (static_cast<uint32_t>(c & 1) << 3) | ((static_cast<uint32_t>(c >> 1) ^ static_cast<uint32_t>(t)) & 7u);
+// Byte offset of 16-byte chunk g (0..15) inside a padded exchange row. Rows
+// are kPitch = 17 chunks apart and chunks 8..15 skip one slot, so 8
+// consecutive rows at one chunk, or one row at chunks 0..7, 8..15 or at every
+// other chunk, fall on 8 distinct bank groups.
+__host__ __device__ constexpr uint32_t xoff(int g) { return 16u * static_cast<uint32_t>(g + (g >> 3)); }
+
+// Decode's exchange: byte offset of 16-byte chunk g (0..15) of row rho of an
+// unpadded 256-byte-row buffer (it later holds the TMA output tile); r = head *
+// NT + token. The chunk index is XOR-swizzled by a rotation of r's low 3 bits:
+// 8 consecutive r at one chunk, or consecutive chunks of one or two tokens,
+// fall on 8 distinct bank groups.
+__device__ __forceinline__ uint32_t xaddr(uint32_t rho, uint32_t r, uint32_t g) {
+  const uint32_t sig = ((r << 1) | ((r >> 2) & 1u)) & 7u;
+  return rho * 256u + 16u * ((g & 8u) | ((g ^ (g >> 3) ^ sig) & 7u));
+}
+
+// 128 contiguous bytes of global memory <-> 32 registers.
+__device__ __forceinline__ void ld_row128(const void* p, bool v8, uint32_t (&w)[32]) {
+  if (v8) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                   : "=r"(w[8 * i]), "=r"(w[8 * i + 1]), "=r"(w[8 * i + 2]), "=r"(w[8 * i + 3]),
+                     "=r"(w[8 * i + 4]), "=r"(w[8 * i + 5]), "=r"(w[8 * i + 6]), "=r"(w[8 * i + 7])
+                   : "l"(static_cast<const uint8_t*>(p) + 32 * i));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 v = __ldg(static_cast<const uint4*>(p) + i);
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+  }
+}
+template <int N>  // N words (a multiple of 8)
+__device__ __forceinline__ void st_row(void* p, bool v8, const uint32_t* w) {
+  if (v8) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i)
+      asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(static_cast<uint8_t*>(p) + 32 * i),
+                   "r"(w[8 * i]), "r"(w[8 * i + 1]), "r"(w[8 * i + 2]), "r"(w[8 * i + 3]), "r"(w[8 * i + 4]),
+                   "r"(w[8 * i + 5]), "r"(w[8 * i + 6]), "r"(w[8 * i + 7])
+                   : "memory");
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i)
+      static_cast<uint4*>(p)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  }
 }
 
 // Tiles are ordered (token block, batch, head group): the tiles that share a
@@ -80,665 +155,718 @@ __device__ __forceinline__ void tile_coords(const GroupArgs& a, int tile, int HG
   h_base = static_cast<int>(grp) * HG;
 }
 
-// Bytes of one stage: the x tile, which later carries the exchange halves
-// and (decode) the output tile.
-template <int HG>
-__host__ __device__ constexpr int stage_bytes() {
-  return kStageX;
-}
-
-// Sum over the codes of one packed word of (kMagicBits << bit position):
-// the packer adds each code's raw fp32 pattern (kMagicBits + code) at its
-// shift and subtracts this once per word.
-template <int BITS>
-__host__ __device__ constexpr uint32_t magic_word_offset() {
+// Sum of kMagicBits << (BITS * j) over the N codes of one packed word: the
+// packer adds each code's raw fp32 pattern (kMagicBits + code) at its shift
+// and subtracts this once per word. The constant only touches bits 22 and
+// up, so runs of at most 22 bits need no correction.
+template <int BITS, int N>
+__host__ __device__ constexpr uint32_t magic_offset() {
   uint32_t k = 0;
-  for (int j = 0; j < 32 / BITS; ++j) k += kMagicBits << (BITS * j);
+  for (int j = 0; j < N; ++j) k += kMagicBits << (BITS * j);
   return k;
 }
 
-template <int NB>
-__device__ __forceinline__ void st_bytes(uint8_t* dst, const uint32_t* w) {
-  if constexpr (NB % 16 == 0) {
+// Phase-1 register layout: P[2g + e] = (x[4g + e], x[4g + 2 + e]), g = 0..15,
+// over 64 consecutive channels. FWHT strides 1, 2, 4, ..., 32 in ascending
+// order (stride 2 falls inside a pair).
+__device__ __forceinline__ void fwht64_pairs(float2 (&P)[32]) {
 #pragma unroll
-    for (int i = 0; i < NB / 16; ++i)
-      reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-  } else if constexpr (NB % 8 == 0) {
+  for (int g = 0; g < 16; ++g) bfly(P[2 * g], P[2 * g + 1]);  // stride 1
 #pragma unroll
-    for (int i = 0; i < NB / 8; ++i) reinterpret_cast<uint2*>(dst)[i] = make_uint2(w[2 * i], w[2 * i + 1]);
-  } else if constexpr (NB % 4 == 0) {
-#pragma unroll
-    for (int i = 0; i < NB / 4; ++i) reinterpret_cast<uint32_t*>(dst)[i] = w[i];
-  } else {
-#pragma unroll
-    for (int i = 0; i < NB / 2; ++i)
-      reinterpret_cast<uint16_t*>(dst)[i] = static_cast<uint16_t>(w[i >> 1] >> (16 * (i & 1)));
-  }
-}
-template <int NB>
-__device__ __forceinline__ void ld_bytes(const uint8_t* src, uint32_t* w) {
-  if constexpr (NB % 16 == 0) {
-#pragma unroll
-    for (int i = 0; i < NB / 16; ++i) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
-      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-    }
-  } else if constexpr (NB % 8 == 0) {
-#pragma unroll
-    for (int i = 0; i < NB / 8; ++i) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + i);
-      w[2 * i] = v.x; w[2 * i + 1] = v.y;
-    }
-  } else if constexpr (NB % 4 == 0) {
-#pragma unroll
-    for (int i = 0; i < NB / 4; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t*>(src) + i);
-  } else {
-#pragma unroll
-    for (int i = 0; i < (NB + 3) / 4; ++i) w[i] = 0u;
-#pragma unroll
-    for (int i = 0; i < NB / 2; ++i)
-      w[i >> 1] |= static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(src) + i)) << (16 * (i & 1));
-  }
-}
-
-// Phase-1 register layout: P[2g + e] = (x[4g + e], x[4g + 2 + e]), g = 0..31.
-// In-head FWHT strides 1, 2, 4, ..., 64 in ascending order.
-__device__ __forceinline__ void fwht128_pairs(float2 (&P)[64]) {
-#pragma unroll
-  for (int g = 0; g < 32; ++g) {  // stride 1: x[4g] <-> x[4g+1], x[4g+2] <-> x[4g+3]
-    const float2 a = P[2 * g], b = P[2 * g + 1];
-    P[2 * g] = add2(a, b);
-    P[2 * g + 1] = sub2(a, b);
-  }
-#pragma unroll
-  for (int k = 0; k < 64; ++k) {  // stride 2: inside each pair
+  for (int k = 0; k < 32; ++k) {  // stride 2
     const float a = P[k].x, b = P[k].y;
     P[k] = f2(__fadd_rn(a, b), __fsub_rn(a, b));
   }
 #pragma unroll
-  for (int hs = 1; hs < 32; hs <<= 1) {  // strides 4 .. 64 = group strides 1 .. 16
+  for (int hs = 1; hs < 16; hs <<= 1) {  // strides 4 .. 32
 #pragma unroll
-    for (int g = 0; g < 32; ++g) {
+    for (int g = 0; g < 16; ++g) {
       if ((g & hs) == 0) {
+        bfly(P[2 * g], P[2 * (g + hs)]);
+        bfly(P[2 * g + 1], P[2 * (g + hs) + 1]);
+      }
+    }
+  }
+}
+
+// fp16 words (h[2j], h[2j+1]) of 64 consecutive channels -> phase-1 pairs.
+__device__ __forceinline__ void halves_to_pairs(const uint32_t (&w)[32], float2 (&P)[32]) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float2 a = P[2 * g + e], b = P[2 * (g + hs) + e];
-          P[2 * g + e] = add2(a, b);
-          P[2 * (g + hs) + e] = sub2(a, b);
+  for (int g = 0; g < 16; ++g) {
+    const float2 h01 = __half22float2(*reinterpret_cast<const __half2*>(&w[2 * g]));
+    const float2 h23 = __half22float2(*reinterpret_cast<const __half2*>(&w[2 * g + 1]));
+    P[2 * g] = f2(h01.x, h23.x);
+    P[2 * g + 1] = f2(h01.y, h23.y);
+  }
+}
+
+// Min/max of NGP groups, each spread over the TPT lanes of one token (an
+// aligned lane group). Halving exchanges (upper lanes keep the upper half of
+// the groups) and, when TPT > NGP, a final butterfly: lane k ends with the
+// totals of group k >> log2(TPT / NGP) in slot 0.
+template <int NGP, int TPT>
+__device__ __forceinline__ void group_reduce(float (&mn)[NGP], float (&mx)[NGP], int lane) {
+#pragma unroll
+  for (int i = 0; (TPT >> (i + 1)) >= 1; ++i) {
+    const int o = TPT >> (i + 1);
+    const int L = NGP >> i;  // groups held before this round
+    if (L >= 2) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int j = 0; j < L / 2; ++j) {
+        const float send_mn = upper ? mn[j] : mn[j + L / 2];
+        const float send_mx = upper ? mx[j] : mx[j + L / 2];
+        const float keep_mn = upper ? mn[j + L / 2] : mn[j];
+        const float keep_mx = upper ? mx[j + L / 2] : mx[j];
+        mn[j] = fminf(keep_mn, __shfl_xor_sync(0xffffffffu, send_mn, o));
+        mx[j] = fmaxf(keep_mx, __shfl_xor_sync(0xffffffffu, send_mx, o));
+      }
+    } else {
+      mn[0] = fminf(mn[0], __shfl_xor_sync(0xffffffffu, mn[0], o));
+      mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
+    }
+  }
+}
+
+// Store / load NBY bytes of packed codes (little-endian words w). The
+// callers' offsets are multiples of the access width used.
+template <int NBY>
+__device__ __forceinline__ void st_code(uint8_t* p, const uint32_t* w) {
+  if constexpr (NBY == 1) {
+    *p = static_cast<uint8_t>(w[0]);
+  } else if constexpr (NBY == 2) {
+    *reinterpret_cast<uint16_t*>(p) = static_cast<uint16_t>(w[0]);
+  } else if constexpr (NBY == 3) {
+    p[0] = static_cast<uint8_t>(w[0]);
+    p[1] = static_cast<uint8_t>(w[0] >> 8);
+    p[2] = static_cast<uint8_t>(w[0] >> 16);
+  } else if constexpr (NBY == 4) {
+    *reinterpret_cast<uint32_t*>(p) = w[0];
+  } else if constexpr (NBY == 6) {
+    reinterpret_cast<uint16_t*>(p)[0] = static_cast<uint16_t>(w[0]);
+    reinterpret_cast<uint16_t*>(p)[1] = static_cast<uint16_t>(w[0] >> 16);
+    reinterpret_cast<uint16_t*>(p)[2] = static_cast<uint16_t>(w[1]);
+  } else {
+    static_assert(NBY == 8, "unsupported code run");
+    *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+  }
+}
+template <int NBY>
+__device__ __forceinline__ void ld_code(const uint8_t* p, uint32_t* w) {
+  if constexpr (NBY == 1) {
+    w[0] = *p;
+  } else if constexpr (NBY == 2) {
+    w[0] = *reinterpret_cast<const uint16_t*>(p);
+  } else if constexpr (NBY == 3) {
+    w[0] = static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[1]) << 8) | (static_cast<uint32_t>(p[2]) << 16);
+  } else if constexpr (NBY == 4) {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  } else if constexpr (NBY == 6) {
+    const uint16_t* q = reinterpret_cast<const uint16_t*>(p);
+    w[0] = static_cast<uint32_t>(q[0]) | (static_cast<uint32_t>(q[1]) << 16);
+    w[1] = q[2];
+  } else {
+    static_assert(NBY == 8, "unsupported code run");
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x;
+    w[1] = v.y;
+  }
+}
+
+template <int HG, int BITS, int G>
+__global__ void __launch_bounds__(kThreads, 512 / kThreads) k_encode_group(const GroupArgs a) {
+  constexpr int NT = kRows / HG;     // tokens per tile
+  constexpr int Q = 8 / HG;          // channel quads per phase-2 thread, head and half
+  constexpr int TPT = 2 * HG;        // phase-2 threads per token
+  constexpr int NG = D / G;          // min-max groups per head
+  constexpr int NGP = HG * NG;       // groups per token
+  constexpr int SH = TPT > NGP ? 1 : 0;
+  constexpr int RB = D * BITS / 8;   // packed bytes per head row
+  constexpr int NCB = 4 * Q * BITS;  // code bits per phase-2 thread, head and half
+  constexpr int NWC = (NCB + 31) / 32;
+  constexpr bool FOLD = (HG != 4);   // 1/sqrt(HG*128) is a power of two
+  constexpr bool PRE_CS = (Q == 1);  // the thread's RoPE rows fit in registers early
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(16) float2 prm[NT * NGP];  // (Z, R) of every group of the tile
+  const uint32_t x0_u = smem_u32(align1024(smem_raw));  // exchange, lower half
+  const uint32_t x1_u = x0_u + kXch;                    // exchange, upper half
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int s1 = tid / kRows, r1 = tid % kRows, h1 = r1 / NT, t1 = r1 % NT;  // phase-1 role
+  const int t2 = tid / TPT, k2 = tid % TPT;                                    // phase-2 role
+  const float r = a.rscale;
+  const bool v8 = a.v8 != 0;
+
+  // this thread's half row of a tile (zeros past the last token)
+  uint32_t raw[32];
+  auto load_raw = [&](int tile) {
+    int b, h_base, t_base;
+    tile_coords(a, tile, HG, NT, b, h_base, t_base);
+    const int tt = t_base + t1;
+    if (tt < a.T) {
+      ld_row128(a.x + ((static_cast<size_t>(b) * a.H + h_base + h1) * a.T + tt) * D + 64 * s1, v8, raw);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) raw[i] = 0u;
+    }
+  };
+  if (kPreload && blockIdx.x < a.n_tiles) load_raw(blockIdx.x);
+
+  for (int it = 0;; ++it) {
+    const int tile = blockIdx.x + it * gridDim.x;
+    if (tile >= a.n_tiles) break;
+    int b, h_base, t_base;
+    tile_coords(a, tile, HG, NT, b, h_base, t_base);
+    if (!kPreload) load_raw(tile);
+
+    // RoPE rows of this thread's phase-2 channels (from L2)
+    const uint4* rp =
+        a.rope ? reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(min(a.t0 + t_base + t2,
+                                                                                    a.t0 + a.T - 1)) * D)
+               : nullptr;
+    uint4 cs_pre[2];
+    if (PRE_CS && a.rope) {
+      cs_pre[0] = __ldg(rp + k2);
+      cs_pre[1] = __ldg(rp + 16 + k2);
+    }
+
+    // ---------------- phase 1: 64 channels of one head row, strides 1 .. 32
+    float2 P[32];
+    {
+      const int tt = t_base + t1, m = a.t0 + tt;
+      if (tt < a.T && m < a.n_sink) {
+        uint4* dst = reinterpret_cast<uint4*>(
+            a.sink + ((static_cast<size_t>(b) * a.H + h_base + h1) * a.n_sink + m) * D + 64 * s1);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(raw[4 * c], raw[4 * c + 1], raw[4 * c + 2], raw[4 * c + 3]);
+      }
+      if (a.perm) {  // the gather reads the whole row: stage the tile in shared memory
+        __syncthreads();  // the previous tile's exchange reads are done
+        const uint32_t row_u = x0_u + r1 * kStage;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sts64(row_u + 128 * s1 + 8 * i, raw[2 * i], raw[2 * i + 1]);
+        __syncthreads();
+        const int16_t* pr = a.perm + static_cast<size_t>(h_base + h1) * D + 64 * s1;
+        float xv[64];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 pk = __ldg(reinterpret_cast<const uint4*>(pr) + c);
+          const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t e = (pw[i >> 1] >> (16 * (i & 1))) & (D - 1);
+            xv[8 * c + i] = __half2float(__ushort_as_half(lds16(row_u + 2 * e)));
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < 16; ++g) {
+          P[2 * g] = f2(xv[4 * g], xv[4 * g + 2]);
+          P[2 * g + 1] = f2(xv[4 * g + 1], xv[4 * g + 3]);
+        }
+      } else {
+        halves_to_pairs(raw, P);
+      }
+      fwht64_pairs(P);
+    }
+    __syncthreads();  // the previous tile's exchange reads (and the gathers) are done
+    {
+      const uint32_t rowp = (s1 == 0 ? x0_u : x1_u) + r1 * kPitch;
+#pragma unroll
+      for (int g = 0; g < 16; ++g)
+        sts128(rowp + xoff(g), make_uint4(__float_as_uint(P[2 * g].x), __float_as_uint(P[2 * g].y),
+                                          __float_as_uint(P[2 * g + 1].x), __float_as_uint(P[2 * g + 1].y)));
+    }
+    __syncthreads();
+    // A[h][half][q][e] = (x[c + e], x[c + 2 + e]) of head h, c = 64 half + 4 (k2 Q + q)
+    float2 A[HG][2][Q][2];
+    {
+      const uint32_t base = x0_u + t2 * kPitch + xoff(k2 * Q);
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs)
+#pragma unroll
+        for (int h = 0; h < HG; ++h)
+#pragma unroll
+          for (int q = 0; q < Q; ++q) {
+            const uint4 u = lds128(base + hs * kXch + h * NT * kPitch + 16 * q);
+            A[h][hs][q][0] = f2(__uint_as_float(u.x), __uint_as_float(u.y));
+            A[h][hs][q][1] = f2(__uint_as_float(u.z), __uint_as_float(u.w));
+          }
+    }
+    if (kPreload) {  // the next tile's rows arrive while this one finishes
+      const int next = tile + gridDim.x;
+      if (next < a.n_tiles) load_raw(next);
+    }
+
+    // ---------------- phase 2: stride 64, cross-head strides
+#pragma unroll
+    for (int h = 0; h < HG; ++h)
+#pragma unroll
+      for (int q = 0; q < Q; ++q)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) bfly(A[h][0][q][e], A[h][1][q][e]);
+#pragma unroll
+    for (int sh = 1; sh < HG; sh <<= 1)
+#pragma unroll
+      for (int h = 0; h < HG; ++h)
+        if ((h & sh) == 0)
+#pragma unroll
+          for (int hs = 0; hs < 2; ++hs)
+#pragma unroll
+            for (int q = 0; q < Q; ++q)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) bfly(A[h][hs][q][e], A[h + sh][hs][q][e]);
+    if (!FOLD) {
+#pragma unroll
+      for (int h = 0; h < HG; ++h)
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs)
+#pragma unroll
+          for (int q = 0; q < Q; ++q)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) A[h][hs][q][e] = mul2(A[h][hs][q][e], f2(r, r));
+    }
+    if (a.rope) {  // y0 = fma(x0, c, -(x1*s)), y1 = fma(x0, s, x1*c), two pairs at a time
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+          // table chunk = (c_i, s_i, c_i+1, s_i+1) for channels c .. c+3; scaled by r when folding (exact)
+          const uint4 cv = PRE_CS ? cs_pre[hs] : __ldg(rp + 16 * hs + k2 * Q + q);
+          float2 cc = f2(__uint_as_float(cv.x), __uint_as_float(cv.z));
+          float2 ss = f2(__uint_as_float(cv.y), __uint_as_float(cv.w));
+          if (FOLD) {
+            cc = mul2(cc, f2(r, r));
+            ss = mul2(ss, f2(r, r));
+          }
+          const float2 nss = f2(-ss.x, -ss.y);
+#pragma unroll
+          for (int h = 0; h < HG; ++h) {
+            const float2 x0 = A[h][hs][q][0], x1 = A[h][hs][q][1];
+            A[h][hs][q][0] = fma2(x0, cc, mul2(x1, nss));
+            A[h][hs][q][1] = fma2(x0, ss, mul2(x1, cc));
+          }
+        }
+      }
+    }
+    // values are now p (keys, or every HG = 4 tensor) or p / r (values when folding)
+    const bool unscaled = FOLD && !a.rope;
+    float mn[NGP], mx[NGP];
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+#pragma unroll
+      for (int grp = 0; grp < NG; ++grp) {
+        float lo = 0.0f, hi = 0.0f;
+        bool first = true;
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+          if (NG == 2 && hs != grp) continue;
+#pragma unroll
+          for (int q = 0; q < Q; ++q) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float2 v = A[h][hs][q][e];
+              if (first) {
+                lo = fminf(v.x, v.y);
+                hi = fmaxf(v.x, v.y);
+                first = false;
+              } else {
+                lo = min3f(lo, v.x, v.y);
+                hi = max3f(hi, v.x, v.y);
+              }
+            }
+          }
+        }
+        mn[h * NG + grp] = lo;
+        mx[h * NG + grp] = hi;
+      }
+    }
+    group_reduce<NGP, TPT>(mn, mx, lane);
+    const int tt2 = t_base + t2, m2 = a.t0 + tt2;
+    const bool store = tt2 < a.T;
+    const bool sink_tok = m2 < a.n_sink;
+    {
+      const int gi = k2 >> SH;  // the group whose totals this lane holds
+      float lo = mn[0], hi = mx[0];
+      if (unscaled) {
+        lo = __fmul_rn(lo, r);
+        hi = __fmul_rn(hi, r);
+      }
+      const QParams p = minmax_params<BITS>(lo, hi);
+      if ((k2 & ((1 << SH) - 1)) == 0) {
+        // Z / r is exact (power of two). A sink slot quantizes with Z = R = 0:
+        // every code of it comes out 0.
+        prm[t2 * NGP + gi] = sink_tok ? f2(0.0f, 0.0f)
+                                      : f2(unscaled ? __fdiv_rn(p.Z, r) : p.Z, unscaled ? __fmul_rn(p.R, r) : p.R);
+        if (store) {
+          const size_t slot = (static_cast<size_t>(b) * a.H + h_base + gi / NG) * a.t_cap + m2;
+          a.sz[slot * NG + gi % NG] = sink_tok ? __halves2half2(__ushort_as_half(0), __ushort_as_half(0)) : p.sz;
+        }
+      }
+    }
+    __syncwarp();
+    float4 zr4[NGP / 2];  // (Z, R) of groups 2j and 2j + 1
+#pragma unroll
+    for (int j = 0; j < NGP / 2; ++j) zr4[j] = *reinterpret_cast<const float4*>(&prm[t2 * NGP + 2 * j]);
+
+    // ---------------- quantize and pack this thread's runs of 4Q channels
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      const size_t slot = (static_cast<size_t>(b) * a.H + h_base + h) * a.t_cap + m2;
+      uint8_t* rec = a.codes + slot * RB;
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        const int gi = h * NG + (NG == 2 ? hs : 0);
+        const float Z = (gi & 1) ? zr4[gi >> 1].z : zr4[gi >> 1].x;
+        const float R = (gi & 1) ? zr4[gi >> 1].w : zr4[gi >> 1].y;
+        const float2 nZ = f2(-Z, -Z), R2 = f2(R, R), M2 = f2(kMagicRound, kMagicRound);
+        // raw fp32 patterns kMagicBits + code of local channels 0 .. 4Q-1
+        uint32_t t[4 * Q];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+          const float2 ua = fma2(add2(A[h][hs][q][0], nZ), R2, M2);
+          const float2 ub = fma2(add2(A[h][hs][q][1], nZ), R2, M2);
+          t[4 * q + 0] = __float_as_uint(ua.x);
+          t[4 * q + 1] = __float_as_uint(ub.x);
+          t[4 * q + 2] = __float_as_uint(ua.y);
+          t[4 * q + 3] = __float_as_uint(ub.y);
+        }
+        uint32_t w[NWC];
+        if constexpr (32 % BITS == 0) {
+          constexpr int PER = 32 / BITS;  // codes per word
+#pragma unroll
+          for (int i = 0; i < NWC; ++i) {
+            const int lo_c = i * PER;
+            const int n_c = (4 * Q - lo_c) < PER ? (4 * Q - lo_c) : PER;
+            uint32_t v = t[lo_c + n_c - 1];
+#pragma unroll
+            for (int j = n_c - 2; j >= 0; --j) v = (v << BITS) + t[lo_c + j];  // codes never straddle a word
+            w[i] = v;
+          }
+          if constexpr (NCB > 22) {
+#pragma unroll
+            for (int i = 0; i < NWC; ++i)
+              w[i] -= (NCB - 32 * i >= 32) ? magic_offset<BITS, PER>() : magic_offset<BITS, (NCB % 32) / BITS>();
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < NWC; ++i) w[i] = 0u;
+#pragma unroll
+          for (int j = 0; j < 4 * Q; ++j) {
+            const int pos = j * BITS;
+            const uint32_t c = t[j] - kMagicBits;
+            w[pos >> 5] |= c << (pos & 31);
+            if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= c >> (32 - (pos & 31));
+          }
+        }
+        if constexpr (NCB % 8 != 0) {
+          // 12-bit runs (HG = 8, 3 bits): even lanes append their odd neighbour's run
+          const uint32_t nb = __shfl_down_sync(0xffffffffu, w[0], 1);
+          if (store && (k2 & 1) == 0) {
+            const uint32_t v = w[0] | (nb << NCB);
+            st_code<2 * NCB / 8>(rec + (64 * hs + 4 * k2 * Q) * BITS / 8, &v);
+          }
+        } else {
+          if (store) st_code<NCB / 8>(rec + (64 * hs + 4 * k2 * Q) * BITS / 8, w);
         }
       }
     }
   }
 }
 
-// Transpose-reduce of per-head (min, max) across the TPG lanes that share a
-// group: afterwards lane k (within its aligned TPG-lane group) holds the
-// totals of heads [k*HG/TPG, (k+1)*HG/TPG).
-template <int HG, int TPG>
-__device__ __forceinline__ void transpose_reduce(float (&mn)[HG], float (&mx)[HG], int lane) {
-  constexpr int L0 = HG;
-#pragma unroll
-  for (int o = TPG / 2, L = L0; o >= 1; o >>= 1, L >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < L / 2; ++i) {
-      const float send_mn = upper ? mn[i] : mn[i + L / 2];
-      const float send_mx = upper ? mx[i] : mx[i + L / 2];
-      const float keep_mn = upper ? mn[i + L / 2] : mn[i];
-      const float keep_mx = upper ? mx[i + L / 2] : mx[i];
-      mn[i] = fminf(keep_mn, __shfl_xor_sync(0xffffffffu, send_mn, o));
-      mx[i] = fmaxf(keep_mx, __shfl_xor_sync(0xffffffffu, send_mx, o));
-    }
-  }
-}
-
-template <int HG, int BITS, int G>
-__global__ void __launch_bounds__(128) k_encode_group(const __grid_constant__ CUtensorMap xmap, const GroupArgs a) {
-  constexpr int NT = 128 / HG;      // tokens per tile
-  constexpr int C = D / HG;         // channels per phase-2 thread
-  constexpr int NGL = C / 4;        // 4-channel groups per phase-2 thread
-  constexpr int TPG = G / C;        // phase-2 lanes sharing one min-max group
-  constexpr int HPL = HG / TPG;     // heads whose scale/zero one lane derives
-  constexpr int NB = C * BITS / 8;  // packed bytes per phase-2 thread and head
-  constexpr int RB = D * BITS / 8;
+template <int HG, int BITS, int G, bool F32>
+__global__ void __launch_bounds__(kThreads, 512 / kThreads) k_decode_group(const __grid_constant__ CUtensorMap cmap,
+                                                               const __grid_constant__ CUtensorMap omap,
+                                                               const GroupArgs a) {
+  constexpr int NT = kRows / HG;
+  constexpr int Q = 8 / HG;
+  constexpr int TPT = 2 * HG;
   constexpr int NG = D / G;
-  constexpr int SB = stage_bytes<HG>();
-  constexpr bool FOLD = (HG != 4);  // 1/sqrt(HG*128) is a power of two
-  constexpr int L = (1 << BITS) - 1;
+  constexpr int RB = D * BITS / 8;
+  constexpr int NCB = 4 * Q * BITS;
+  constexpr int NWC = (NCB + 31) / 32;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  constexpr bool PRE_CS = (Q == 1);
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ __align__(8) uint64_t full[2];
+  __shared__ __half2 szs[2][kRows * NG];  // scale/zero of the tile's rows, by cp.async
   uint8_t* sm = align1024(smem_raw);
+  uint8_t* xr = sm + 2 * kCodes;  // exchange (two halves), then the output tile
+  const uint32_t xr_u = smem_u32(xr);
   const int tid = threadIdx.x;
-  const int hl = tid / NT, t = tid % NT;   // phase-1 role
-  const int t2 = tid / HG, k = tid % HG;   // phase-2 role
-  const int lane = tid & 31;
+  const int s1 = tid / kRows, r1 = tid % kRows, h1 = r1 / NT, t1 = r1 % NT;
+  const int t2 = tid / TPT, k2 = tid % TPT;
+  const float r = a.rscale;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
   }
-  __syncthreads();
   auto issue = [&](int tile, int s) {
     int b, h_base, t_base;
     tile_coords(a, tile, HG, NT, b, h_base, t_base);
-    uint8_t* st = sm + s * SB;
-    mbar_arrive_expect_tx(&full[s], kStageX);
-    tma_load_3d(st, &xmap, 0, t_base, b * a.H + h_base, &full[s]);
-    tma_load_3d(st + 16384, &xmap, 64, t_base, b * a.H + h_base, &full[s]);
+    mbar_arrive_expect_tx(&full[s], kRows * RB);
+    tma_load_3d(sm + s * kCodes, &cmap, 0, a.t0 + t_base, b * a.H + h_base, &full[s]);
+  };
+  // scale/zero of one tile's rows (zero-filled past the last token)
+  auto fetch_sz = [&](int tile, int buf) {
+    if (tid < kRows * NG) {
+      int b, h_base, t_base;
+      tile_coords(a, tile, HG, NT, b, h_base, t_base);
+      const int rr = tid % kRows, grp = tid / kRows;
+      const int h = rr / NT, t = rr % NT;
+      const bool live = t_base + t < a.T;
+      const size_t slot = (static_cast<size_t>(b) * a.H + h_base + h) * a.t_cap + a.t0 + t_base + t;
+      cp_async4(smem_u32(&szs[buf][tid]), live ? static_cast<const void*>(a.sz + slot * NG + grp) : a.sz,
+                live ? 4u : 0u);
+    }
+    cp_async_commit();
   };
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < 2; ++s) {
       const int tile = blockIdx.x + s * gridDim.x;
       if (tile < a.n_tiles) issue(tile, s);
     }
   }
-  const float r = a.rscale;
+  if (blockIdx.x < a.n_tiles) fetch_sz(blockIdx.x, 0);
+  cp_async_wait_all();
+  __syncthreads();
   bool ok = true;
 
   for (int it = 0;; ++it) {
     const int tile = blockIdx.x + it * gridDim.x;
     if (tile >= a.n_tiles) break;
     const int s = it & 1;
-    const uint32_t parity = (it >> 1) & 1;
     int b, h_base, t_base;
     tile_coords(a, tile, HG, NT, b, h_base, t_base);
-    uint8_t* st = sm + s * SB;
-    const uint32_t st_u = smem_u32(st);
-    ok = mbar_wait(&full[s], parity, a.wait_ns, a.err);  // on a timeout the tile is garbage; see below
-
-
-    // ---------------- phase 1
-    const int tt = t_base + t, m = a.t0 + tt;
-    float2 P[64];
     {
-      if (tt < a.T && m < a.n_sink) {
-        uint4* dst = reinterpret_cast<uint4*>(a.sink + ((static_cast<size_t>(b) * a.H + h_base + hl) * a.n_sink + m) * D);
+      const int next = tile + gridDim.x;
+      if (next < a.n_tiles) fetch_sz(next, s ^ 1);
+    }
+    const uint4* rp =
+        a.rope ? reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(min(a.t0 + t_base + t2,
+                                                                                    a.t0 + a.T - 1)) * D)
+               : nullptr;
+    uint4 cs_pre[2];
+    if (PRE_CS && a.rope) {
+      cs_pre[0] = __ldg(rp + k2);
+      cs_pre[1] = __ldg(rp + 16 + k2);
+    }
+    ok = mbar_wait(&full[s], (it >> 1) & 1, a.wait_ns, a.err);
+
+    // ---------------- phase 2 (reverse): dequantize (normalisation folded in), inverse RoPE, strides
+    float2 A[HG][2][Q][2];
+    const uint8_t* cst = sm + s * kCodes;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) dst[c] = lds128(st_u + (c >> 3) * 16384 + sw128(tid, c & 7));
+    for (int h = 0; h < HG; ++h) {
+      const uint8_t* rec = cst + (h * NT + t2) * RB;
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        const float2 szf = __half22float2(szs[s][(NG == 2 ? hs : 0) * kRows + h * NT + t2]);
+        const float S = __fmul_rn(szf.x, r), Z = __fmul_rn(szf.y, r);
+        uint32_t w[NWC];
+        if constexpr (NCB % 8 != 0) {  // 12-bit runs start half a byte in for odd k2
+          const int bit = (64 * hs + 4 * k2 * Q) * BITS;
+          const uint8_t* p = rec + (bit >> 3);
+          w[0] = ((static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[1]) << 8)) >> (bit & 7)) & 0xfffu;
+        } else {
+          ld_code<NCB / 8>(rec + (64 * hs + 4 * k2 * Q) * BITS / 8, w);
+        }
+        // Codes 0 and 2 of a quad are masked in place at bit 0, codes 1 and 3
+        // at bit BITS; read through the fp32 pattern 2^23 + v they give
+        // code * 2^p, and the power of two 2^p is folded exactly into the scale.
+        const float2 S0 = f2(S, S), S1 = f2(S * (1.0f / (1 << BITS)), S * (1.0f / (1 << BITS)));
+        const float2 Z2 = f2(Z, Z), nM = f2(-8388608.0f, -8388608.0f);
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+          const int pos = 4 * q * BITS;
+          const uint32_t lo = w[pos >> 5] >> (pos & 31);
+          const uint32_t w0 = (32 - (pos & 31) >= 4 * BITS || (pos >> 5) + 1 >= NWC)
+                                  ? lo
+                                  : (lo | (w[(pos >> 5) + 1] << (32 - (pos & 31))));
+          const uint32_t w1 = w0 >> (2 * BITS);
+          const float2 c02 =
+              f2(__uint_as_float(0x4B000000u | (w0 & MASK)), __uint_as_float(0x4B000000u | (w1 & MASK)));
+          const float2 c13 = f2(__uint_as_float(0x4B000000u | (w0 & (MASK << BITS))),
+                                __uint_as_float(0x4B000000u | (w1 & (MASK << BITS))));
+          A[h][hs][q][0] = fma2(add2(c02, nM), S0, Z2);
+          A[h][hs][q][1] = fma2(add2(c13, nM), S1, Z2);
+        }
       }
-      if (a.perm) {
-        const int16_t* pr = a.perm + static_cast<size_t>(h_base + hl) * D;
-        float xv[D];
+    }
+    if (a.rope) {
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 pk = __ldg(reinterpret_cast<const uint4*>(pr) + c);
-          const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
+      for (int hs = 0; hs < 2; ++hs) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t e = (pw[i >> 1] >> (16 * (i & 1))) & (D - 1);
-            const uint32_t addr = st_u + (e >> 6) * 16384 + sw128(tid, (e & 63) >> 3) + (e & 7) * 2;
-            xv[8 * c + i] = __half2float(__ushort_as_half(lds16(addr)));
+        for (int q = 0; q < Q; ++q) {
+          const uint4 cv = PRE_CS ? cs_pre[hs] : __ldg(rp + 16 * hs + k2 * Q + q);
+          const float2 cc = f2(__uint_as_float(cv.x), __uint_as_float(cv.z));
+          const float2 ss = f2(__uint_as_float(cv.y), __uint_as_float(cv.w));
+          const float2 nss = f2(-ss.x, -ss.y);
+#pragma unroll
+          for (int h = 0; h < HG; ++h) {  // x0 = y0 c + y1 s, x1 = y1 c - y0 s
+            const float2 y0 = A[h][hs][q][0], y1 = A[h][hs][q][1];
+            A[h][hs][q][0] = fma2(y0, cc, mul2(y1, ss));
+            A[h][hs][q][1] = fma2(y1, cc, mul2(y0, nss));
           }
         }
-#pragma unroll
-        for (int g = 0; g < 32; ++g) {
-          P[2 * g] = f2(xv[4 * g], xv[4 * g + 2]);
-          P[2 * g + 1] = f2(xv[4 * g + 1], xv[4 * g + 3]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint4 raw = lds128(st_u + (c >> 3) * 16384 + sw128(tid, c & 7));
-          const __half2* hp = reinterpret_cast<const __half2*>(&raw);
-          const float2 h01 = __half22float2(hp[0]), h23 = __half22float2(hp[1]);
-          const float2 h45 = __half22float2(hp[2]), h67 = __half22float2(hp[3]);
-          P[4 * c + 0] = f2(h01.x, h23.x);
-          P[4 * c + 1] = f2(h01.y, h23.y);
-          P[4 * c + 2] = f2(h45.x, h67.x);
-          P[4 * c + 3] = f2(h45.y, h67.y);
-        }
       }
-      fwht128_pairs(P);
     }
-    // the x tile is consumed; its space carries the exchange. A timed-out wait
-    // in any thread ends the CTA's work uniformly here.
+#pragma unroll
+    for (int sh = 1; sh < HG; sh <<= 1)
+#pragma unroll
+      for (int h = 0; h < HG; ++h)
+        if ((h & sh) == 0)
+#pragma unroll
+          for (int hs = 0; hs < 2; ++hs)
+#pragma unroll
+            for (int q = 0; q < Q; ++q)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) bfly(A[h][hs][q][e], A[h + sh][hs][q][e]);
+#pragma unroll
+    for (int h = 0; h < HG; ++h)
+#pragma unroll
+      for (int q = 0; q < Q; ++q)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) bfly(A[h][0][q][e], A[h][1][q][e]);
+
+    // The previous tile's output store has read the exchange region, and the
+    // codes stage is consumed. A timed-out wait ends the CTA's work uniformly.
+    if (tid == 0) bulk_wait_read<0>();
     if (!__syncthreads_and(ok)) {
       ok = false;
       break;
     }
+    if (tid == 0 && tile + 2 * static_cast<int>(gridDim.x) < a.n_tiles) issue(tile + 2 * gridDim.x, s);
 
-    // ---------------- exchange (two halves of 64 channels) -> phase-2 registers
-    float2 A[HG][NGL], Bv[HG][NGL];  // A = (ch 4g, 4g+2), Bv = (ch 4g+1, 4g+3) of head h
+    // ---------------- exchange -> phase-1 registers
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      const uint32_t row1 = st_u + (t * HG + hl) * 256;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {  // 8-channel chunk q8 = 2q + h2 = groups 2*q8, 2*q8+1
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int g = 2 * (2 * q + h2) + e;
-          sts128(row1 + xpos(t, 2 * q + e) * 16,
-                 make_uint4(__float_as_uint(P[2 * g].x), __float_as_uint(P[2 * g].y), __float_as_uint(P[2 * g + 1].x),
-                            __float_as_uint(P[2 * g + 1].y)));
-        }
-      }
-      __syncthreads();
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const uint32_t row2 = st_u + (t2 * HG + h) * 256;
-#pragma unroll
-        for (int qq = 0; qq < C / 16; ++qq) {  // this thread's chunks of the half
-          const int q8 = k * (C / 8) + 2 * qq + h2;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const uint4 u = lds128(row2 + xpos(t2, 2 * (q8 >> 1) + e) * 16);
-            const int gl = 2 * (2 * qq + h2) + e;  // static: keeps A / Bv in registers
-            A[h][gl] = f2(__uint_as_float(u.x), __uint_as_float(u.y));
-            Bv[h][gl] = f2(__uint_as_float(u.z), __uint_as_float(u.w));
-          }
-        }
-      }
-      __syncthreads();
-    }
-    // the stage is free again: stream in the tile after next
-    if (tid == 0 && tile + kStages * gridDim.x < a.n_tiles) issue(tile + kStages * gridDim.x, s);
-    // RoPE (cos, sin) of this thread's phase-2 channels, straight from L2
-    // (the tiles of one token block run together, so the rows stay hot)
-    uint4 csr[NGL];
-    if (a.rope) {
-      const int mr = min(a.t0 + t_base + t2, a.t0 + a.T - 1);
-      const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(mr) * D) + k * NGL;
-#pragma unroll
-      for (int gl = 0; gl < NGL; ++gl) csr[gl] = __ldg(rp + gl);
-    }
-
-    // ---------------- phase 2
-#pragma unroll
-    for (int sh = 1; sh < HG; sh <<= 1) {  // cross-head strides
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        if ((h & sh) == 0) {
-#pragma unroll
-          for (int gl = 0; gl < NGL; ++gl) {
-            const float2 pa = A[h][gl], qa = A[h + sh][gl];
-            A[h][gl] = add2(pa, qa);
-            A[h + sh][gl] = sub2(pa, qa);
-            const float2 pb = Bv[h][gl], qb = Bv[h + sh][gl];
-            Bv[h][gl] = add2(pb, qb);
-            Bv[h + sh][gl] = sub2(pb, qb);
-          }
-        }
-      }
-    }
-    if (!FOLD) {
+    for (int hs = 0; hs < 2; ++hs)
 #pragma unroll
       for (int h = 0; h < HG; ++h)
 #pragma unroll
-        for (int gl = 0; gl < NGL; ++gl) {
-          A[h][gl] = mul2(A[h][gl], f2(r, r));
-          Bv[h][gl] = mul2(Bv[h][gl], f2(r, r));
-        }
-    }
-    if (a.rope) {  // y0 = fma(x0, c, -(x1*s)), y1 = fma(x0, s, x1*c), two pairs at a time
+        for (int q = 0; q < Q; ++q)
+          sts128(xr_u + hs * kXchS + xaddr(t2 * HG + h, h * NT + t2, k2 * Q + q),
+                 make_uint4(__float_as_uint(A[h][hs][q][0].x), __float_as_uint(A[h][hs][q][0].y),
+                            __float_as_uint(A[h][hs][q][1].x), __float_as_uint(A[h][hs][q][1].y)));
+    __syncthreads();
+    float2 P[32];
+    {
+      const uint32_t xb = xr_u + s1 * kXchS;
+      const uint32_t rho = t1 * HG + h1;
 #pragma unroll
-      for (int gl = 0; gl < NGL; ++gl) {
-        // table chunk g = (c_2g, s_2g, c_2g+1, s_2g+1); scaled by r when folding (exact)
-        float2 cc = f2(__uint_as_float(csr[gl].x), __uint_as_float(csr[gl].z));
-        float2 ss = f2(__uint_as_float(csr[gl].y), __uint_as_float(csr[gl].w));
-        if (FOLD) {
-          cc = mul2(cc, f2(r, r));
-          ss = mul2(ss, f2(r, r));
-        }
-        const float2 nss = f2(-ss.x, -ss.y);
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          const float2 x0 = A[h][gl], x1 = Bv[h][gl];
-          const float2 t1n = mul2(x1, nss);
-          const float2 t2c = mul2(x1, cc);
-          A[h][gl] = fma2(x0, cc, t1n);
-          Bv[h][gl] = fma2(x0, ss, t2c);
-        }
+      for (int g = 0; g < 16; ++g) {
+        const uint4 u = lds128(xb + xaddr(rho, r1, g));
+        P[2 * g] = f2(__uint_as_float(u.x), __uint_as_float(u.y));
+        P[2 * g + 1] = f2(__uint_as_float(u.z), __uint_as_float(u.w));
       }
     }
-    // values are now p (keys, or every HG = 4 tensor) or p / r (values when folding)
-    const bool unscaled = FOLD && !a.rope;
-    float mn[HG], mx[HG];
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      float lo = fminf(A[h][0].x, A[h][0].y), hi = fmaxf(A[h][0].x, A[h][0].y);
-      lo = min3f(lo, Bv[h][0].x, Bv[h][0].y);
-      hi = max3f(hi, Bv[h][0].x, Bv[h][0].y);
-#pragma unroll
-      for (int gl = 1; gl < NGL; ++gl) {
-        lo = min3f(lo, A[h][gl].x, A[h][gl].y);
-        hi = max3f(hi, A[h][gl].x, A[h][gl].y);
-        lo = min3f(lo, Bv[h][gl].x, Bv[h][gl].y);
-        hi = max3f(hi, Bv[h][gl].x, Bv[h][gl].y);
-      }
-      mn[h] = lo;
-      mx[h] = hi;
-    }
-    transpose_reduce<HG, TPG>(mn, mx, lane);
-    const int kg = lane & (TPG - 1);  // this lane's rank among the lanes of its group
-    float Zq[HPL], Rq[HPL];
-    __half2 szo[HPL];
-#pragma unroll
-    for (int i = 0; i < HPL; ++i) {
-      float lo = mn[i], hi = mx[i];
-      if (unscaled) {
-        lo = __fmul_rn(lo, r);
-        hi = __fmul_rn(hi, r);
-      }
-      const QParams p = minmax_params<BITS>(lo, hi);
-      szo[i] = p.sz;
-      Zq[i] = unscaled ? __fdiv_rn(p.Z, r) : p.Z;  // Z / r is exact (power of two)
-      Rq[i] = unscaled ? __fmul_rn(p.R, r) : p.R;
-    }
-    const int tt2 = t_base + t2, m2 = a.t0 + tt2;
-    const bool store = tt2 < a.T;
-    const bool sink_tok = m2 < a.n_sink;
-    const int lane0 = lane - kg;  // first lane of this thread's group
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      // (Z, R) of head h live in lane (lane0 + h / HPL), slot h % HPL
-      const float Z = __shfl_sync(0xffffffffu, Zq[h % HPL], lane0 + h / HPL);
-      const float R = __shfl_sync(0xffffffffu, Rq[h % HPL], lane0 + h / HPL);
-      const float2 nZ = f2(-Z, -Z), R2 = f2(R, R), M2 = f2(kMagicRound, kMagicRound);
-      constexpr int NWC = (C * BITS + 31) / 32;
-      uint32_t w[NWC];
-#pragma unroll
-      for (int i = 0; i < NWC; ++i) w[i] = 0u;
-#pragma unroll
-      for (int gl = 0; gl < NGL; ++gl) {
-        const float2 ua = fma2(add2(A[h][gl], nZ), R2, M2);
-        const float2 ub = fma2(add2(Bv[h][gl], nZ), R2, M2);
-        // raw fp32 patterns kMagicBits + code of local channels 4gl + 0, 1, 2, 3
-        const uint32_t t4[4] = {__float_as_uint(ua.x), __float_as_uint(ub.x), __float_as_uint(ua.y),
-                                __float_as_uint(ub.y)};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int pos = (4 * gl + e) * BITS;
-          if constexpr (32 % BITS == 0) {
-            w[pos >> 5] += t4[e] << (pos & 31);  // codes never straddle a word
-          } else {
-            const uint32_t c = t4[e] - kMagicBits;
-            w[pos >> 5] |= c << (pos & 31);
-            if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= c >> (32 - (pos & 31));
-          }
-        }
-      }
-      if constexpr (32 % BITS == 0) {
-#pragma unroll
-        for (int i = 0; i < NWC; ++i) w[i] -= magic_word_offset<BITS>();
-      }
-#pragma unroll
-      for (int i = 0; i < NWC; ++i) w[i] = sink_tok ? 0u : w[i];
-      if (store) {
-        const size_t slot = (static_cast<size_t>(b) * a.H + h_base + h) * a.t_cap + m2;
-        st_bytes<NB>(a.codes + slot * RB + k * NB, w);
-      }
-    }
-    if (store) {
-      const __half2 zero2 = __halves2half2(__ushort_as_half(0), __ushort_as_half(0));
-#pragma unroll
-      for (int i = 0; i < HPL; ++i) {
-        const int h = kg * HPL + i;
-        const size_t slot = (static_cast<size_t>(b) * a.H + h_base + h) * a.t_cap + m2;
-        a.sz[slot * NG + (k * C) / G] = sink_tok ? zero2 : szo[i];
-      }
-    }
-    (void)L;
-  }
-  if (!ok && tid == 0) {  // let copies in flight land (bounded) before the CTA exits
-    for (int s = 0; s < kStages; ++s)
-      for (uint32_t p = 0; p < 2; ++p) mbar_wait(&full[s], p, a.wait_ns, a.err);
-  }
-}
-
-template <int HG, int BITS, int G>
-__global__ void __launch_bounds__(128) k_decode_group(const __grid_constant__ CUtensorMap omap, const GroupArgs a,
-                                                       int out_fp32) {
-  constexpr int NT = 128 / HG;
-  constexpr int C = D / HG;
-  constexpr int NGL = C / 4;
-  constexpr int NB = C * BITS / 8;
-  constexpr int NW = (C * BITS + 31) / 32;
-  constexpr int RB = D * BITS / 8;
-  constexpr int NG = D / G;
-  constexpr int SB = stage_bytes<HG>();
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = align1024(smem_raw);
-  const int tid = threadIdx.x;
-  const int hl = tid / NT, t = tid % NT;
-  const int t2 = tid / HG, k = tid % HG;
-  const float r = a.rscale;
-
-  // this thread's packed codes, (S, Z) and RoPE (cos, sin) of one tile
-  auto load_tile = [&](int tile, uint32_t (&cw)[HG][NW], __half2 (&szv)[HG], uint4 (&csr)[NGL]) {
-    int b, h_base, t_base;
-    tile_coords(a, tile, HG, NT, b, h_base, t_base);
-    const int tt2 = t_base + t2, m2 = a.t0 + tt2;
-    const bool live = tt2 < a.T && m2 >= a.n_sink;
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      if (live) {
-        const size_t slot = (static_cast<size_t>(b) * a.H + h_base + h) * a.t_cap + m2;
-        ld_bytes<NB>(a.codes + slot * RB + k * NB, cw[h]);
-        szv[h] = a.sz[slot * NG + (k * C) / G];
-      } else {
-#pragma unroll
-        for (int i = 0; i < NW; ++i) cw[h][i] = 0u;
-        szv[h] = __halves2half2(__ushort_as_half(0), __ushort_as_half(0));
-      }
-    }
-    if (a.rope) {
-      const int mr = min(m2, a.t0 + a.T - 1);
-      const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(mr) * D) + k * NGL;
-#pragma unroll
-      for (int gl = 0; gl < NGL; ++gl) csr[gl] = __ldg(rp + gl);
-    }
-  };
-  uint32_t cw[HG][NW];
-  __half2 szv[HG];
-  uint4 csr[NGL];
-  if (blockIdx.x < a.n_tiles) load_tile(blockIdx.x, cw, szv, csr);
-
-  for (int it = 0;; ++it) {
-    const int tile = blockIdx.x + it * gridDim.x;
-    if (tile >= a.n_tiles) break;
-    const int s = it & 1;
-    int b, h_base, t_base;
-    tile_coords(a, tile, HG, NT, b, h_base, t_base);
-    uint8_t* st = sm + s * SB;
-    const uint32_t st_u = smem_u32(st);
-
-    // ---------------- phase 2 (reverse): dequantize (normalisation folded in), inverse RoPE, cross-head
-    float2 A[HG][NGL], Bv[HG][NGL];
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      const float S = __fmul_rn(__low2float(szv[h]), r), Z = __fmul_rn(__high2float(szv[h]), r);
-      const float2 S2 = f2(S, S), Z2 = f2(Z, Z);
-#pragma unroll
-      for (int gl = 0; gl < NGL; ++gl) {
-        const float2 ca = f2(code_to_float(unpack_code<BITS, NW>(cw[h], 4 * gl + 0)),
-                             code_to_float(unpack_code<BITS, NW>(cw[h], 4 * gl + 2)));
-        const float2 cb = f2(code_to_float(unpack_code<BITS, NW>(cw[h], 4 * gl + 1)),
-                             code_to_float(unpack_code<BITS, NW>(cw[h], 4 * gl + 3)));
-        A[h][gl] = fma2(ca, S2, Z2);
-        Bv[h][gl] = fma2(cb, S2, Z2);
-      }
-    }
-    if (a.rope) {
-#pragma unroll
-      for (int gl = 0; gl < NGL; ++gl) {
-        const float2 cc = f2(__uint_as_float(csr[gl].x), __uint_as_float(csr[gl].z));
-        const float2 ss = f2(__uint_as_float(csr[gl].y), __uint_as_float(csr[gl].w));
-        const float2 nss = f2(-ss.x, -ss.y);
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {  // x0 = y0 c + y1 s, x1 = y1 c - y0 s
-          const float2 y0 = A[h][gl], y1 = Bv[h][gl];
-          A[h][gl] = fma2(y0, cc, mul2(y1, ss));
-          Bv[h][gl] = fma2(y1, cc, mul2(y0, nss));
-        }
-      }
-    }
-#pragma unroll
-    for (int sh = 1; sh < HG; sh <<= 1) {
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        if ((h & sh) == 0) {
-#pragma unroll
-          for (int gl = 0; gl < NGL; ++gl) {
-            const float2 pa = A[h][gl], qa = A[h + sh][gl];
-            A[h][gl] = add2(pa, qa);
-            A[h + sh][gl] = sub2(pa, qa);
-            const float2 pb = Bv[h][gl], qb = Bv[h + sh][gl];
-            Bv[h][gl] = add2(pb, qb);
-            Bv[h + sh][gl] = sub2(pb, qb);
-          }
-        }
-      }
-    }
-    // the output store of two tiles ago must have read this stage
-    if (tid == 0) bulk_wait_read<1>();
     __syncthreads();
 
-    // ---------------- exchange (two halves) -> phase-1 registers
-    float2 P[64];
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const uint32_t row2 = st_u + (t2 * HG + h) * 256;
-#pragma unroll
-        for (int qq = 0; qq < C / 16; ++qq) {
-          const int q8 = k * (C / 8) + 2 * qq + h2;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int gl = 2 * (2 * qq + h2) + e;  // static: keeps A / Bv in registers
-            sts128(row2 + xpos(t2, 2 * (q8 >> 1) + e) * 16,
-                   make_uint4(__float_as_uint(A[h][gl].x), __float_as_uint(A[h][gl].y),
-                              __float_as_uint(Bv[h][gl].x), __float_as_uint(Bv[h][gl].y)));
-          }
-        }
-      }
-      __syncthreads();
-      const uint32_t row1 = st_u + (t * HG + hl) * 256;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int g = 2 * (2 * q + h2) + e;
-          const uint4 u = lds128(row1 + xpos(t, 2 * q + e) * 16);
-          P[2 * g] = f2(__uint_as_float(u.x), __uint_as_float(u.y));
-          P[2 * g + 1] = f2(__uint_as_float(u.z), __uint_as_float(u.w));
-        }
-      }
-      __syncthreads();
-    }
-
-    // prefetch the next tile's codes, scales and RoPE rows while this one finishes
-    const int next = tile + gridDim.x;
-    if (next < a.n_tiles) load_tile(next, cw, szv, csr);
-
     // ---------------- phase 1 (reverse): in-head strides, inverse permutation, output
-    fwht128_pairs(P);
-    const int tt = t_base + t, m = a.t0 + tt;
-    float x[D];
+    fwht64_pairs(P);
+    const int tt = t_base + t1, m = a.t0 + tt;
+    const bool sink_tok = tt < a.T && m < a.n_sink;
+    const bool permute = a.perm != nullptr && !sink_tok;
+    const int16_t* pr = a.perm ? a.perm + static_cast<size_t>(h_base + h1) * D + 64 * s1 : nullptr;
+    float x[64];
 #pragma unroll
-    for (int g = 0; g < 32; ++g) {
+    for (int g = 0; g < 16; ++g) {
       x[4 * g] = P[2 * g].x;
       x[4 * g + 2] = P[2 * g].y;
       x[4 * g + 1] = P[2 * g + 1].x;
       x[4 * g + 3] = P[2 * g + 1].y;
     }
-    const bool sink_tok = tt < a.T && m < a.n_sink;
-    if (sink_tok) {
+    if (sink_tok) {  // sink positions come back verbatim
       const uint4* src = reinterpret_cast<const uint4*>(
-          a.sink + ((static_cast<size_t>(b) * a.H + h_base + hl) * a.n_sink + m) * D);
+          a.sink + ((static_cast<size_t>(b) * a.H + h_base + h1) * a.n_sink + m) * D + 64 * s1);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) h8_to_f32(__ldg(src + c), &x[8 * c]);
+      for (int c = 0; c < 8; ++c) h8_to_f32(__ldg(src + c), &x[8 * c]);
     }
-    const bool permute = a.perm != nullptr && !sink_tok;
-    const int16_t* pr = a.perm ? a.perm + static_cast<size_t>(h_base + hl) * D : nullptr;
-    if (!out_fp32) {
-      if (permute) {  // x'[perm[j]] = x[j], written straight into this thread's output row
+    if constexpr (!F32) {
+      if (permute) {  // x'[perm[j]] = x[j], written straight into the output row
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
+        for (int c = 0; c < 8; ++c) {
           const uint4 pk = __ldg(reinterpret_cast<const uint4*>(pr) + c);
           const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const uint32_t e = (pw[i >> 1] >> (16 * (i & 1))) & (D - 1);
-            sts16(st_u + (e >> 6) * 16384 + sw128(tid, (e & 63) >> 3) + (e & 7) * 2,
+            sts16(xr_u + (e >> 6) * kHalf + sw128(r1, (e & 63) >> 3) + (e & 7) * 2,
                   __half_as_ushort(__float2half_rn(x[8 * c + i])));
           }
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) sts128(st_u + (c >> 3) * 16384 + sw128(tid, c & 7), f32_to_h8(&x[8 * c]));
+        for (int c = 0; c < 8; ++c) sts128(xr_u + s1 * kHalf + sw128(r1, c), f32_to_h8(&x[8 * c]));
       }
-      fence_async_smem();
-      __syncthreads();
-      if (tid == 0) {
-        tma_store_3d(&omap, 0, t_base, b * a.H + h_base, st);
-        tma_store_3d(&omap, 64, t_base, b * a.H + h_base, st + 16384);
-        bulk_commit();
-      }
-    } else {
-      // fp32 tile = 64 KB: two passes of 64 channels through the 32 KB stage
+    } else {  // fp32: four 32-channel boxes of 16 KB
+      if (permute) {
 #pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        if (pass == 1) {
-          if (tid == 0) bulk_wait_read<0>();
-          __syncthreads();
-        }
-        if (permute) {
+        for (int c = 0; c < 8; ++c) {
+          const uint4 pk = __ldg(reinterpret_cast<const uint4*>(pr) + c);
+          const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
-            const uint4 pk = __ldg(reinterpret_cast<const uint4*>(pr) + c);
-            const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t e = (pw[i >> 1] >> (16 * (i & 1))) & (D - 1);
-              if ((e >> 6) == static_cast<uint32_t>(pass))
-                sts32f(st_u + ((e & 63) >> 5) * 16384 + sw128(tid, (e & 31) >> 2) + (e & 3) * 4, x[8 * c + i]);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int cc = pass * 16 + c;
-            sts128(st_u + (c >> 3) * 16384 + sw128(tid, c & 7),
-                   make_uint4(__float_as_uint(x[4 * cc]), __float_as_uint(x[4 * cc + 1]),
-                              __float_as_uint(x[4 * cc + 2]), __float_as_uint(x[4 * cc + 3])));
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t e = (pw[i >> 1] >> (16 * (i & 1))) & (D - 1);
+            sts32f(xr_u + (e >> 5) * kHalf + sw128(r1, (e & 31) >> 2) + (e & 3) * 4, x[8 * c + i]);
           }
         }
-        fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-          tma_store_3d(&omap, pass * 64, t_base, b * a.H + h_base, st);
-          tma_store_3d(&omap, pass * 64 + 32, t_base, b * a.H + h_base, st + 16384);
-          bulk_commit();
-        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          sts128(xr_u + (2 * s1 + (c >> 3)) * kHalf + sw128(r1, c & 7),
+                 make_uint4(__float_as_uint(x[4 * c]), __float_as_uint(x[4 * c + 1]), __float_as_uint(x[4 * c + 2]),
+                            __float_as_uint(x[4 * c + 3])));
       }
     }
+    cp_async_wait_all();  // the next tile's scale/zero rows, published by the barrier below
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      if constexpr (!F32) {
+        tma_store_3d(&omap, 0, t_base, b * a.H + h_base, xr);
+        tma_store_3d(&omap, 64, t_base, b * a.H + h_base, xr + kHalf);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tma_store_3d(&omap, 32 * j, t_base, b * a.H + h_base, xr + j * kHalf);
+      }
+      bulk_commit();
+    }
   }
-  if (tid == 0) bulk_wait_read<0>();  // the last stores have read shared memory
+  if (tid == 0) {
+    bulk_wait_read<0>();  // the last stores have read shared memory
+    if (!ok)              // let copies in flight land (bounded) before the CTA exits
+      for (int s = 0; s < 2; ++s)
+        for (uint32_t p = 0; p < 2; ++p) mbar_wait(&full[s], p, a.wait_ns, a.err);
+  }
+  cp_async_wait_all();
 }
 
 template <int HG, int BITS, int G>
-kvq_status run(bool enc, const GroupArgs& a, const CUtensorMap& m0, int out_fp32,
+kvq_status run(bool enc, const GroupArgs& a, const CUtensorMap& cm, const CUtensorMap& om, int out_fp32,
                const LaunchCtx& ctx, cudaStream_t st) {
-  const size_t smem = 1024 + static_cast<size_t>(kStages) * stage_bytes<HG>();
-  const void* fn = enc ? reinterpret_cast<const void*>(k_encode_group<HG, BITS, G>)
-                       : reinterpret_cast<const void*>(k_decode_group<HG, BITS, G>);
-  if (!set_smem_once(reinterpret_cast<const void*>(fn), smem))
-    return KVQ_ERR_CUDA;
-  const int per_sm = occupancy_once(fn, 128, smem);
+  const size_t smem =
+      enc ? 1024 + 2 * static_cast<size_t>(kXch) : 1024 + 2 * static_cast<size_t>(kCodes) + 2 * kXchS;
+  const void* fn = enc        ? reinterpret_cast<const void*>(k_encode_group<HG, BITS, G>)
+                   : out_fp32 ? reinterpret_cast<const void*>(k_decode_group<HG, BITS, G, true>)
+                              : reinterpret_cast<const void*>(k_decode_group<HG, BITS, G, false>);
+  if (!set_smem_once(fn, smem)) return KVQ_ERR_CUDA;
+  const int per_sm = occupancy_once(fn, kThreads, smem);
   const long long want = static_cast<long long>(ctx.num_sms) * per_sm;
   const unsigned grid = static_cast<unsigned>(a.n_tiles < want ? a.n_tiles : want);
   if (enc)
-    k_encode_group<HG, BITS, G><<<grid, 128, smem, st>>>(m0, a);
+    k_encode_group<HG, BITS, G><<<grid, kThreads, smem, st>>>(a);
+  else if (out_fp32)
+    k_decode_group<HG, BITS, G, true><<<grid, kThreads, smem, st>>>(cm, om, a);
   else
-    k_decode_group<HG, BITS, G><<<grid, 128, smem, st>>>(m0, a, out_fp32);
+    k_decode_group<HG, BITS, G, false><<<grid, kThreads, smem, st>>>(cm, om, a);
   return launch_status();
 }
 
-kvq_status dispatch(bool enc, const kvq_desc& d, const GroupArgs& a, const CUtensorMap& m0, int out_fp32,
-                    const LaunchCtx& ctx, cudaStream_t st) {
-#define KVQ_CASE(HG_, B_, G_) \
-  if (d.group_heads == HG_ && d.bits == B_ && d.group == G_) return run<HG_, B_, G_>(enc, a, m0, out_fp32, ctx, st);
+kvq_status dispatch(bool enc, const kvq_desc& d, const GroupArgs& a, const CUtensorMap& cm, const CUtensorMap& om,
+                    int out_fp32, const LaunchCtx& ctx, cudaStream_t st) {
+#define KVQ_CASE(HG_, B_, G_)                                    \
+  if (d.group_heads == HG_ && d.bits == B_ && d.group == G_) \
+    return run<HG_, B_, G_>(enc, a, cm, om, out_fp32, ctx, st);
 #define KVQ_BITS(HG_, G_) KVQ_CASE(HG_, 2, G_) KVQ_CASE(HG_, 3, G_) KVQ_CASE(HG_, 4, G_)
   KVQ_BITS(8, 128)
   KVQ_BITS(8, 64)
@@ -760,7 +888,7 @@ GroupArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p
   a.t_cap = d.t_cap;
   a.n_sink = d.n_sink;
   a.rope = d.rope;
-  const int NT = 128 / d.group_heads;
+  const int NT = kRows / d.group_heads;
   a.n_tblk = (d.tokens + NT - 1) / NT;
   a.n_grp = d.heads / d.group_heads;
   a.n_tiles = d.batch * a.n_grp * a.n_tblk;
@@ -777,25 +905,33 @@ GroupArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p
   return a;
 }
 
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
 }  // namespace
 
 kvq_status launch_encode_group(const kvq_desc& d, const void* x, const kvq_tables& tb, const kvq_packed& out,
                                cudaStream_t st, const LaunchCtx& ctx) {
-  const GroupArgs a = make_args(d, tb, out, ctx);
-  const int NT = 128 / d.group_heads;
-  CUtensorMap xm;
-  const uint64_t dims[3] = {D, static_cast<uint64_t>(d.tokens), static_cast<uint64_t>(d.batch) * d.heads};
-  const uint64_t strides[2] = {D * 2, static_cast<uint64_t>(d.tokens) * D * 2};
-  const uint32_t box[3] = {64, static_cast<uint32_t>(NT), static_cast<uint32_t>(d.group_heads)};
-  if (!make_map(&xm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-    return KVQ_ERR_CUDA;
-  return dispatch(true, d, a, xm, 0, ctx, st);
+  GroupArgs a = make_args(d, tb, out, ctx);
+  a.x = static_cast<const __half*>(x);
+  a.v8 = aligned32(x);
+  CUtensorMap unused{};
+  return dispatch(true, d, a, unused, unused, 0, ctx, st);
 }
 
 kvq_status launch_decode_group(const kvq_desc& d, const kvq_packed& in, const kvq_tables& tb, void* x_out,
                                int out_fp32, cudaStream_t st, const LaunchCtx& ctx) {
   const GroupArgs a = make_args(d, tb, in, ctx);
-  const int NT = 128 / d.group_heads;
+  const int NT = kRows / d.group_heads;
+  // packed codes: [B*H][t_cap][RB] bytes; one box = the tile's records
+  CUtensorMap cm;
+  const uint64_t rb = static_cast<uint64_t>(D) * d.bits / 8;
+  const uint64_t cdims[3] = {rb, static_cast<uint64_t>(d.t_cap), static_cast<uint64_t>(d.batch) * d.heads};
+  const uint64_t cstrides[2] = {rb, static_cast<uint64_t>(d.t_cap) * rb};
+  const uint32_t cbox[3] = {static_cast<uint32_t>(rb), static_cast<uint32_t>(NT),
+                            static_cast<uint32_t>(d.group_heads)};
+  if (!make_map(&cm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, in.codes, cdims, cstrides, cbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return KVQ_ERR_CUDA;
+  // output tile: boxes of 64 fp16 or 32 fp32 channels x NT tokens x HG heads
   CUtensorMap om;
   const uint64_t es = out_fp32 ? 4 : 2;
   const uint64_t dims[3] = {D, static_cast<uint64_t>(d.tokens), static_cast<uint64_t>(d.batch) * d.heads};
@@ -804,7 +940,7 @@ kvq_status launch_decode_group(const kvq_desc& d, const kvq_packed& in, const kv
   if (!make_map(&om, out_fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, x_out, dims,
                 strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
     return KVQ_ERR_CUDA;
-  return dispatch(false, d, a, om, out_fp32, ctx, st);
+  return dispatch(false, d, a, cm, om, out_fp32, ctx, st);
 }
 
 }  // namespace kvq
