@@ -166,6 +166,8 @@ class Step:
         }
         self.kernels = {"encode_k": "k_encode_group", "encode_v": "k_encode_group", "decode_k": "k_decode_group",
                         "decode_v": "k_decode_group", "append": "k_encode_head", "score": "k_score_mma"}
+        self.fp32_ops = {n: nvec * D * fp32_ops_per_element("fwht_group", n, wg.group_heads, D)
+                         for n in ("encode_k", "encode_v", "decode_k", "decode_v")}
         self.names = list(self.alg)
         self.host_in = [self.k_host, self.v_host, self.sc.app_host, self.sc.q_host]
         self.dev_in = [self.k, self.v, self.sc.app, self.sc.q]
@@ -235,7 +237,7 @@ class EncDecStep:
         iso = w.rot == "iso"
         tensors = ["k", "v"] if both and not iso else ["k"]
         self.items = []
-        self.alg, self.fp16_equiv, self.kernels = {}, {}, {}
+        self.alg, self.fp16_equiv, self.kernels, self.fp32_ops = {}, {}, {}, {}
         kern = {"fwht_head": "head", "none": "head", "fwht_group": "group", "iso": "iso"}[w.rot]
         for which in tensors:
             x = (W.kv_tensor_device(w, which, device) if iso else torch.from_numpy(W.kv_tensor(w, which)).to(device))
@@ -260,6 +262,10 @@ class EncDecStep:
             self.fp16_equiv[f"decode_{which}"] = nvec * 2 * D
             self.kernels[f"encode_{which}"] = f"k_encode_{kern}"
             self.kernels[f"decode_{which}"] = f"k_decode_{kern}"
+            for n in (f"encode_{which}", f"decode_{which}"):
+                ops = fp32_ops_per_element(w.rot, n, w.group_heads, D, rope=rope)
+                if ops:
+                    self.fp32_ops[n] = nvec * D * ops
         self.names = list(self.alg)
         torch.cuda.synchronize(device)
 
@@ -281,11 +287,28 @@ class DecodeScoreStep:
         self.alg = {"append": self.sc.alg_append, "score": self.sc.alg_score}
         self.fp16_equiv = {"append": self.sc.fp16_append, "score": self.sc.fp16_score}
         self.kernels = {"append": "k_encode_head", "score": "k_score_mma"}
+        self.fp32_ops = {}
         self.names = list(self.alg)
         torch.cuda.synchronize(device)
 
     def launches(self):
         return [self.sc.append, self.sc.score]
+
+
+def fp32_ops_per_element(rot, step, group_heads, D, rope=None):
+    """Algorithmic fp32 operations per element of an encode/decode launch, in
+    the oracle's order: FWHT log2(N) add/sub (N = D, or group_heads * D), RoPE
+    2 (one mul and one fma per output, keys only), the quantizer 2 (sub + fma)
+    or the dequantizer 2 (fma + the folded normalisation). Min/max compares run
+    on the ALU pipe and are not counted. None for IsoQuant (norm, 4x4 blocks,
+    codebook search)."""
+    if rot == "iso":
+        return None
+    n = D * (group_heads if rot == "fwht_group" else 1)
+    fwht = 0 if rot == "none" else int(math.log2(n))
+    if rope is None:
+        rope = 1 if step.endswith("_k") else 0
+    return fwht + 2 * rope + 2
 
 
 def make_step(workload, device, batch=None):
@@ -451,6 +474,15 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": _traffic_for(st.kernels[dom]), "kernel": st.kernels[dom],
                 "kernel_step": dom, "alg_bytes_per_launch": st.alg[dom], "peak_kind": peak_kind}
+    clocks = clk.summary()
+    if dom in st.fp32_ops:
+        # the same launch against the fp32 pipe: SMs x 128 fp32 lanes x max SM clock
+        mhz = clocks.get("sm_max_mhz") or 1965
+        alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * mhz * 1e6
+        alu_ach = st.fp32_ops[dom] / (dom_ms / 1e3)
+        roofline["alu"] = {"achieved": alu_ach / 1e12, "peak": alu_peak / 1e12, "unit": "T fp32-op/s",
+                           "frac": alu_ach / alu_peak, "ops_per_launch": st.fp32_ops[dom]}
+        roofline["alu_frac"] = alu_ach / alu_peak
 
     e2e_line = None
     if hasattr(st, "host_in"):
@@ -475,7 +507,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": _config(world) if args.workload == "llama3_8b_gqa" else _other_config(args.workload, world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e_line,
-            "gpu_launches": nk * args.steps, "clocks": clk.summary(), "kernels": kernels,
+            "gpu_launches": nk * args.steps, "clocks": clocks, "kernels": kernels,
             "status": K.kvq_status_str(status),
         }
         print(json.dumps(line))
