@@ -270,9 +270,13 @@ class EncDecStep:
         torch.cuda.synchronize(device)
 
     def launches(self):
+        """One launch per entry of self.names, in the same order (encode then
+        decode of each tensor)."""
         TA = self.TA
-        fs = [TA.bind_encode(d, x, tb, pk) for which, d, x, tb, pk, out in self.items]
-        fs += [TA.bind_decode(d, pk, tb, out) for which, d, x, tb, pk, out in self.items]
+        fs = []
+        for which, d, x, tb, pk, out in self.items:
+            fs += [TA.bind_encode(d, x, tb, pk), TA.bind_decode(d, pk, tb, out)]
+        assert len(fs) == len(self.names)
         return fs
 
 

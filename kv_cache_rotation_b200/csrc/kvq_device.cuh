@@ -214,6 +214,95 @@ __device__ __forceinline__ void fwht_reg(float (&v)[N]) {
   }
 }
 
+// ---------------------------------------------------------------- packed fp32 (sm_100 FADD2 / FFMA2 / FMUL2)
+// Same IEEE rounding per lane as the scalar operations.
+__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// a - b as one packed fma: fma(b, -1, a) rounds a - b exactly once, like a subtraction.
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ void bfly(float2& a, float2& b) {
+  const float2 p = a, q = b;
+  a = add2(p, q);
+  b = sub2(p, q);
+}
+
+// Register-pair layout of V consecutive channels: P[2g + e] = (x[4g + e],
+// x[4g + 2 + e]), g < V/4. Unnormalised Sylvester FWHT strides 1, 2, 4, ...,
+// V/2 in ascending order; stride 2 falls inside a pair (scalar ops), every
+// other stride is one packed add and one packed subtract per two pairs.
+template <int V>
+__device__ __forceinline__ void fwht_pairs(float2 (&P)[V / 2]) {
+#pragma unroll
+  for (int g = 0; g < V / 4; ++g) bfly(P[2 * g], P[2 * g + 1]);  // stride 1
+#pragma unroll
+  for (int k = 0; k < V / 2; ++k) {  // stride 2
+    const float a = P[k].x, b = P[k].y;
+    P[k] = f2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+#pragma unroll
+  for (int hs = 1; hs < V / 4; hs <<= 1) {  // strides 4 .. V/2
+#pragma unroll
+    for (int g = 0; g < V / 4; ++g) {
+      if ((g & hs) == 0) {
+        bfly(P[2 * g], P[2 * (g + hs)]);
+        bfly(P[2 * g + 1], P[2 * (g + hs) + 1]);
+      }
+    }
+  }
+}
+
+// N words (N a multiple of 8) of global memory <-> registers: 256-bit accesses
+// when the address is 32-byte aligned, 128-bit ones otherwise. Loads use the
+// read-only path and do not allocate in L1.
+template <int N>
+__device__ __forceinline__ void ld_row(const void* p, bool v8, uint32_t* w) {
+  if (v8) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i)
+      asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                   : "=r"(w[8 * i]), "=r"(w[8 * i + 1]), "=r"(w[8 * i + 2]), "=r"(w[8 * i + 3]),
+                     "=r"(w[8 * i + 4]), "=r"(w[8 * i + 5]), "=r"(w[8 * i + 6]), "=r"(w[8 * i + 7])
+                   : "l"(static_cast<const uint8_t*>(p) + 32 * i));
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const uint4 v = __ldg(static_cast<const uint4*>(p) + i);
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+  }
+}
+template <int N>
+__device__ __forceinline__ void st_row(void* p, bool v8, const uint32_t* w) {
+  if (v8) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i)
+      asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(static_cast<uint8_t*>(p) + 32 * i),
+                   "r"(w[8 * i]), "r"(w[8 * i + 1]), "r"(w[8 * i + 2]), "r"(w[8 * i + 3]), "r"(w[8 * i + 4]),
+                   "r"(w[8 * i + 5]), "r"(w[8 * i + 6]), "r"(w[8 * i + 7])
+                   : "memory");
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i)
+      static_cast<uint4*>(p)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  }
+}
+
+// Sum of kMagicBits << (BITS * j) over the N codes of one packed word: a packer
+// that adds each code's raw fp32 pattern (kMagicBits + code) at its shift
+// subtracts this once per word. The constant only touches bits 22 and up, so
+// runs of at most 22 bits need no correction.
+template <int BITS, int N>
+__host__ __device__ constexpr uint32_t magic_offset() {
+  uint32_t k = 0;
+  for (int j = 0; j < N; ++j) k += kMagicBits << (BITS * j);
+  return k;
+}
+
 // ---------------------------------------------------------------- RoPE
 // Forward rotation of one pair with fp32 (c, s):
 //   y0 = fma(x0, c, -(x1*s)),  y1 = fma(x0, s, x1*c)

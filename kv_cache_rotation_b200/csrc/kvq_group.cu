@@ -79,18 +79,6 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return p + (((a + 1023u) & ~1023u) - a);
 }
 
-__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-// a - b as one packed fma: fma(b, -1, a) rounds a - b exactly once, like a subtraction.
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ void bfly(float2& a, float2& b) {
-  const float2 p = a, q = b;
-  a = add2(p, q);
-  b = sub2(p, q);
-}
-
 // Byte offset of 16-byte chunk g (0..15) inside a padded exchange row. Rows
 // are kPitch = 17 chunks apart and chunks 8..15 skip one slot, so 8
 // consecutive rows at one chunk, or one row at chunks 0..7, 8..15 or at every
@@ -107,42 +95,6 @@ __device__ __forceinline__ uint32_t xaddr(uint32_t rho, uint32_t r, uint32_t g) 
   return rho * 256u + 16u * ((g & 8u) | ((g ^ (g >> 3) ^ sig) & 7u));
 }
 
-// 128 contiguous bytes of global memory <-> 32 registers.
-__device__ __forceinline__ void ld_row128(const void* p, bool v8, uint32_t (&w)[32]) {
-  if (v8) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                   : "=r"(w[8 * i]), "=r"(w[8 * i + 1]), "=r"(w[8 * i + 2]), "=r"(w[8 * i + 3]),
-                     "=r"(w[8 * i + 4]), "=r"(w[8 * i + 5]), "=r"(w[8 * i + 6]), "=r"(w[8 * i + 7])
-                   : "l"(static_cast<const uint8_t*>(p) + 32 * i));
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint4 v = __ldg(static_cast<const uint4*>(p) + i);
-      w[4 * i] = v.x;
-      w[4 * i + 1] = v.y;
-      w[4 * i + 2] = v.z;
-      w[4 * i + 3] = v.w;
-    }
-  }
-}
-template <int N>  // N words (a multiple of 8)
-__device__ __forceinline__ void st_row(void* p, bool v8, const uint32_t* w) {
-  if (v8) {
-#pragma unroll
-    for (int i = 0; i < N / 8; ++i)
-      asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(static_cast<uint8_t*>(p) + 32 * i),
-                   "r"(w[8 * i]), "r"(w[8 * i + 1]), "r"(w[8 * i + 2]), "r"(w[8 * i + 3]), "r"(w[8 * i + 4]),
-                   "r"(w[8 * i + 5]), "r"(w[8 * i + 6]), "r"(w[8 * i + 7])
-                   : "memory");
-  } else {
-#pragma unroll
-    for (int i = 0; i < N / 4; ++i)
-      static_cast<uint4*>(p)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-  }
-}
-
 // Tiles are ordered (token block, batch, head group): the tiles that share a
 // token block -- and so the same RoPE rows -- run at the same time.
 __device__ __forceinline__ void tile_coords(const GroupArgs& a, int tile, int HG, int NT, int& b, int& h_base,
@@ -153,40 +105,6 @@ __device__ __forceinline__ void tile_coords(const GroupArgs& a, int tile, int HG
   b = static_cast<int>(a.div_b.mod(rest, tb));
   t_base = static_cast<int>(tb) * NT;
   h_base = static_cast<int>(grp) * HG;
-}
-
-// Sum of kMagicBits << (BITS * j) over the N codes of one packed word: the
-// packer adds each code's raw fp32 pattern (kMagicBits + code) at its shift
-// and subtracts this once per word. The constant only touches bits 22 and
-// up, so runs of at most 22 bits need no correction.
-template <int BITS, int N>
-__host__ __device__ constexpr uint32_t magic_offset() {
-  uint32_t k = 0;
-  for (int j = 0; j < N; ++j) k += kMagicBits << (BITS * j);
-  return k;
-}
-
-// Phase-1 register layout: P[2g + e] = (x[4g + e], x[4g + 2 + e]), g = 0..15,
-// over 64 consecutive channels. FWHT strides 1, 2, 4, ..., 32 in ascending
-// order (stride 2 falls inside a pair).
-__device__ __forceinline__ void fwht64_pairs(float2 (&P)[32]) {
-#pragma unroll
-  for (int g = 0; g < 16; ++g) bfly(P[2 * g], P[2 * g + 1]);  // stride 1
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {  // stride 2
-    const float a = P[k].x, b = P[k].y;
-    P[k] = f2(__fadd_rn(a, b), __fsub_rn(a, b));
-  }
-#pragma unroll
-  for (int hs = 1; hs < 16; hs <<= 1) {  // strides 4 .. 32
-#pragma unroll
-    for (int g = 0; g < 16; ++g) {
-      if ((g & hs) == 0) {
-        bfly(P[2 * g], P[2 * (g + hs)]);
-        bfly(P[2 * g + 1], P[2 * (g + hs) + 1]);
-      }
-    }
-  }
 }
 
 // fp16 words (h[2j], h[2j+1]) of 64 consecutive channels -> phase-1 pairs.
@@ -303,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) k_encode_group(const
     tile_coords(a, tile, HG, NT, b, h_base, t_base);
     const int tt = t_base + t1;
     if (tt < a.T) {
-      ld_row128(a.x + ((static_cast<size_t>(b) * a.H + h_base + h1) * a.T + tt) * D + 64 * s1, v8, raw);
+      ld_row<32>(a.x + ((static_cast<size_t>(b) * a.H + h_base + h1) * a.T + tt) * D + 64 * s1, v8, raw);
     } else {
 #pragma unroll
       for (int i = 0; i < 32; ++i) raw[i] = 0u;
@@ -365,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) k_encode_group(const
       } else {
         halves_to_pairs(raw, P);
       }
-      fwht64_pairs(P);
+      fwht_pairs<64>(P);
     }
     __syncthreads();  // the previous tile's exchange reads (and the gathers) are done
     {
@@ -762,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 512 / kThreads) k_decode_group(const
     __syncthreads();
 
     // ---------------- phase 1 (reverse): in-head strides, inverse permutation, output
-    fwht64_pairs(P);
+    fwht_pairs<64>(P);
     const int tt = t_base + t1, m = a.t0 + tt;
     const bool sink_tok = tt < a.T && m < a.n_sink;
     const bool permute = a.perm != nullptr && !sink_tok;

@@ -1,384 +1,445 @@
-// Head-variant encode / decode: one thread per token-head vector, the whole
-// vector in registers.
-//
-// Encode ("RotateKV: Accurate and Robust 2-Bit KV Cache Quantization for LLMs
-// via Outlier-Aware Adaptive Rotations", abstract and 关键设计: channel
-// reordering followed by the FWHT; 2-bit KV quantization; attention sinks):
+// Head-variant encode / decode ("RotateKV: Accurate and Robust 2-Bit KV Cache
+// Quantization for LLMs via Outlier-Aware Adaptive Rotations", abstract and
+// 关键设计: channel reordering followed by the FWHT; 2-bit KV quantization;
+// attention sinks):
 //   RoPE (keys) -> channel permutation -> normalised FWHT over head_dim
 //   -> per-group min-max quantization with fp16 (scale, zero) -> LSB-first packing.
-// Decode is the exact inverse.
+// Decode is the inverse.
 //
-// A CTA owns a tile of HT heads x NT tokens of one batch (HT * NT = 128).
-// The fp16 rows arrive in shared memory by one 3-D TMA copy per 64-channel
-// half (128-byte swizzle, so the per-thread row reads are bank-conflict
-// free); the RoPE cos/sin rows of the tile's NT positions arrive by 2-D TMA
-// copies and are shared by the HT heads.
+// Two lanes of a warp share one token-head vector: lane 2i + s holds channels
+// [sV, sV + V), V = D/2, loaded straight from global memory (256-bit loads).
+// Warps work independently (no barriers): each takes 16 consecutive vectors.
+// Without RoPE the order is (batch, head, token): 4 KB of contiguous rows of
+// one head, which share that head's permutation. With RoPE it is (batch,
+// token, head): the heads of a token share its cos/sin row in L1, which costs
+// more than the permutation's bank conflicts. The FWHT strides 1 .. V/2 run in registers; the last stride V pairs
+// the two lanes: each lane computes fma(own, +-1, partner), i.e. exactly
+// a + b (lower lane) or a - b (upper lane), and so keeps final values of its
+// own channels. Groups of G <= V channels are then whole inside one lane; a
+// group of D channels takes one min/max exchange with the partner.
+// The permutation gathers (decode: scatters) through a per-warp buffer of rows
+// in shared memory; with one permutation per warp and rows 130 words apart,
+// the 16 rows read at one channel fall on 16 distinct banks.
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
 namespace {
 
+constexpr int kThreads = 128;  // 4 independent warps per CTA
+constexpr int kVecW = 16;      // vectors per warp step
+
 struct HeadArgs {
-  int B, H, T, t0, t_cap, n_sink, rope, HT, NT, n_tblk, n_hblk;
-  float rscale;  // fp32(1/sqrt(D))
+  int B, H, T, t0, t_cap, n_sink, rope, v8;
+  uint32_t n_vec;        // B * H * T
+  FastDiv div_t, div_h;  // tokens; heads
+  float rscale;          // fp32(1/sqrt(D))
+  const __half* x;       // encode input  [B][H][T][D]
+  void* out;             // decode output [B][H][T][D], fp16 or fp32
   const int16_t* perm;
+  const float* rope_cs;  // [rows][D/2][2]
   uint8_t* codes;
   __half2* sz;
   __half* sink;
-  uint32_t* err;
-  uint64_t wait_ns;
 };
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  const uint32_t a = smem_u32(p);
-  return p + (((a + 1023u) & ~1023u) - a);
+// Rows of the per-warp permutation buffer: D floats plus two pad words (an
+// odd number of 8-byte units, so row k starts 2k words into the banks);
+// element e of a row is at row + 4e.
+template <int D>
+__host__ __device__ constexpr uint32_t row_pitch() {
+  return D * 4 + 8;
 }
 
-template <int BYTES>
-__device__ __forceinline__ void store_words(uint8_t* dst, const uint32_t* w) {
-  if constexpr (BYTES % 16 == 0) {
+// Store / load this lane's run of NBY packed bytes; ALN = the run's alignment.
+template <int NBY, int ALN>
+__device__ __forceinline__ void st_run(uint8_t* p, const uint32_t* w) {
+  if constexpr (ALN >= 16) {
 #pragma unroll
-    for (int i = 0; i < BYTES / 16; ++i)
-      reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    for (int i = 0; i < NBY / 16; ++i)
+      reinterpret_cast<uint4*>(p)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  } else if constexpr (ALN == 8) {
+#pragma unroll
+    for (int i = 0; i < NBY / 8; ++i) reinterpret_cast<uint2*>(p)[i] = make_uint2(w[2 * i], w[2 * i + 1]);
   } else {
 #pragma unroll
-    for (int i = 0; i < BYTES / 8; ++i) reinterpret_cast<uint2*>(dst)[i] = make_uint2(w[2 * i], w[2 * i + 1]);
+    for (int i = 0; i < NBY / 4; ++i) reinterpret_cast<uint32_t*>(p)[i] = w[i];
   }
 }
-template <int BYTES>
-__device__ __forceinline__ void load_words(const uint8_t* src, uint32_t* w) {
-  if constexpr (BYTES % 16 == 0) {
+template <int NBY, int ALN>
+__device__ __forceinline__ void ld_run(const uint8_t* p, uint32_t* w) {
+  if constexpr (ALN >= 16) {
 #pragma unroll
-    for (int i = 0; i < BYTES / 16; ++i) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
-      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    for (int i = 0; i < NBY / 16; ++i) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + i);
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+  } else if constexpr (ALN == 8) {
+#pragma unroll
+    for (int i = 0; i < NBY / 8; ++i) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p) + i);
+      w[2 * i] = v.x;
+      w[2 * i + 1] = v.y;
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < BYTES / 8; ++i) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + i);
-      w[2 * i] = v.x; w[2 * i + 1] = v.y;
-    }
+    for (int i = 0; i < NBY / 4; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t*>(p) + i);
   }
 }
-template <int NG>
-__device__ __forceinline__ void store_sz(__half2* dst, const __half2* v) {
-  if constexpr (NG == 1) {
-    *dst = v[0];
-  } else if constexpr (NG == 2) {
-    uint2 u;
-    u.x = *reinterpret_cast<const uint32_t*>(&v[0]);
-    u.y = *reinterpret_cast<const uint32_t*>(&v[1]);
-    *reinterpret_cast<uint2*>(dst) = u;
-  } else {
-#pragma unroll
-    for (int i = 0; i < NG; i += 4) {
-      uint4 u;
-      u.x = *reinterpret_cast<const uint32_t*>(&v[i]);
-      u.y = *reinterpret_cast<const uint32_t*>(&v[i + 1]);
-      u.z = *reinterpret_cast<const uint32_t*>(&v[i + 2]);
-      u.w = *reinterpret_cast<const uint32_t*>(&v[i + 3]);
-      *reinterpret_cast<uint4*>(dst + i) = u;
-    }
-  }
-}
+__host__ __device__ constexpr int pow2_align(int n) { return (n & 15) == 0 ? 16 : (n & 7) == 0 ? 8 : 4; }
 
-// Permutation through a thread-private shared-memory row of D floats
-// (16-byte chunks XOR-swizzled by the thread index).
-template <int D>
-__device__ __forceinline__ uint32_t perm_addr(uint32_t row, int e, int tid) {
-  return row + ((((e >> 2) ^ (tid & 7)) << 4) | ((e & 3) << 2));
-}
-// gather: v[j] <- v[perm[j]]
-template <int D>
-__device__ __forceinline__ void perm_gather(float (&v)[D], const int16_t* perm_row, uint32_t row, int tid) {
-#pragma unroll
-  for (int c = 0; c < D / 4; ++c)
-    sts128(row + ((c ^ (tid & 7)) << 4), make_uint4(__float_as_uint(v[4 * c]), __float_as_uint(v[4 * c + 1]),
-                                                    __float_as_uint(v[4 * c + 2]), __float_as_uint(v[4 * c + 3])));
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
-    const uint4 pk = __ldg(reinterpret_cast<const uint4*>(perm_row) + c);
-    const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = static_cast<int>((pw[i >> 1] >> (16 * (i & 1))) & (D - 1));
-      v[8 * c + i] = lds32f(perm_addr<D>(row, e, tid));
-    }
+// (b * H + h, h, token) of vector v, ordered (batch, head, token) without RoPE
+// and (batch, token, head) with it.
+__device__ __forceinline__ void vec_coords(const HeadArgs& a, uint32_t v, uint32_t& bh, int& h, int& tt) {
+  if (a.rope) {
+    const uint32_t bt = a.div_h.div(v);
+    h = static_cast<int>(a.div_h.mod(v, bt));
+    const uint32_t b = a.div_t.div(bt);
+    tt = static_cast<int>(a.div_t.mod(bt, b));
+    bh = b * static_cast<uint32_t>(a.H) + static_cast<uint32_t>(h);
+  } else {
+    bh = a.div_t.div(v);
+    tt = static_cast<int>(a.div_t.mod(v, bh));
+    h = static_cast<int>(a.div_h.mod(bh, a.div_h.div(bh)));
   }
-}
-// scatter: v'[perm[j]] <- v[j]
-template <int D>
-__device__ __forceinline__ void perm_scatter(float (&v)[D], const int16_t* perm_row, uint32_t row, int tid) {
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
-    const uint4 pk = __ldg(reinterpret_cast<const uint4*>(perm_row) + c);
-    const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = static_cast<int>((pw[i >> 1] >> (16 * (i & 1))) & (D - 1));
-      sts32f(perm_addr<D>(row, e, tid), v[8 * c + i]);
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < D / 4; ++c) {
-    const uint4 u = lds128(row + ((c ^ (tid & 7)) << 4));
-    v[4 * c] = __uint_as_float(u.x);
-    v[4 * c + 1] = __uint_as_float(u.y);
-    v[4 * c + 2] = __uint_as_float(u.z);
-    v[4 * c + 3] = __uint_as_float(u.w);
-  }
-}
-
-// Tile index -> (b, head base, token base).
-__device__ __forceinline__ void tile_coords(const HeadArgs& a, int& b, int& h_base, int& t_base) {
-  int blk = blockIdx.x;
-  const int tb = blk % a.n_tblk;
-  blk /= a.n_tblk;
-  const int hb = blk % a.n_hblk;
-  b = blk / a.n_hblk;
-  h_base = hb * a.HT;
-  t_base = tb * a.NT;
 }
 
 template <int D, int BITS, int G, bool ROT>
-__global__ void __launch_bounds__(128) k_encode_head(const __grid_constant__ CUtensorMap xmap,
-                                                      const __grid_constant__ CUtensorMap rmap, const HeadArgs a) {
-  constexpr int RB = D * BITS / 8;  // record bytes
-  constexpr int NG = D / G;
-  constexpr int NW = D * BITS / 32;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar;
-  uint8_t* xs = align1024(smem_raw);   // D/64 swizzled halves of 128 rows x 128 B
-  uint8_t* rs = xs + D * 256;          // D/32 quarters of NT rows x 128 B
-  uint8_t* ps = rs + a.NT * D * 4;     // permutation rows (128 x D floats)
-  const int tid = threadIdx.x;
-  int b, h_base, t_base;
-  tile_coords(a, b, h_base, t_base);
+__global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
+  constexpr int V = D / 2;            // channels per lane
+  constexpr int RB = D * BITS / 8;    // record bytes
+  constexpr int NG = D / G;           // groups per record
+  constexpr bool SHARED = G > V;      // one group spans both lanes
+  constexpr int GS = SHARED ? V : G;  // channels of a group inside this lane
+  constexpr int NGT = V / GS;         // groups inside this lane
+  constexpr int NBY = V * BITS / 8;   // this lane's packed bytes
+  constexpr int NW = NBY / 4;
+  extern __shared__ uint8_t smem_raw[];  // permutation rows: 16 x D floats per warp
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int s = lane & 1, slot = lane >> 1;
+  const uint32_t row = smem_u32(smem_raw) + (warp * kVecW + slot) * row_pitch<D>();
+  const float r = a.rscale;
+  const bool v8 = a.v8 != 0;
+  const uint32_t gw = blockIdx.x * (kThreads / 32) + warp, nw = gridDim.x * (kThreads / 32);
 
-  if (tid == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t bytes = D * 256 + (a.rope ? a.NT * D * 4 : 0);
-    mbar_arrive_expect_tx(&bar, bytes);
-#pragma unroll
-    for (int hh = 0; hh < D / 64; ++hh) tma_load_3d(xs + hh * 16384, &xmap, hh * 64, t_base, b * a.H + h_base, &bar);
-    if (a.rope)
-      for (int q = 0; q < D / 32; ++q) tma_load_2d(rs + q * a.NT * 128, &rmap, q * 32, a.t0 + t_base, &bar);
-  }
-  if (!mbar_wait(&bar, 0, a.wait_ns, a.err)) {
-    if (tid == 0) mbar_wait(&bar, 0, a.wait_ns, a.err);  // let an in-flight copy land before exiting
-    return;
-  }
+  for (uint32_t base = gw * kVecW; base < a.n_vec; base += nw * kVecW) {
+    const uint32_t v = base + slot;
+    const bool live = v < a.n_vec;
+    uint32_t bh;
+    int h, tt;
+    vec_coords(a, live ? v : a.n_vec - 1, bh, h, tt);
+    const int m = a.t0 + tt;
+    const size_t vec = bh;
+    const bool sink_tok = m < a.n_sink;
 
-  const int hl = tid / a.NT, t = tid % a.NT;
-  const int h = h_base + hl, tt = t_base + t;
-  if (h >= a.H || tt >= a.T) return;
-  const int m = a.t0 + tt;
-  const size_t v = static_cast<size_t>(b) * a.H + h;
-  const size_t slot = v * a.t_cap + m;
-  const uint32_t xs_u = smem_u32(xs);
-
-  if (m < a.n_sink) {  // attention sink: verbatim fp16, zero codes / scale / zero
-    uint4* dst = reinterpret_cast<uint4*>(a.sink + (v * a.n_sink + m) * D);
+    uint32_t raw[V / 2];
+    ld_row<V / 2>(a.x + (vec * a.T + tt) * D + V * s, v8, raw);
+    if (live && sink_tok) {  // attention sink: this lane's half row, verbatim
+      uint4* dst = reinterpret_cast<uint4*>(a.sink + (vec * a.n_sink + m) * D + V * s);
 #pragma unroll
-    for (int hh = 0; hh < D / 64; ++hh)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) dst[hh * 8 + c] = lds128(xs_u + hh * 16384 + sw128(tid, c));
-    uint32_t z[NW];
-#pragma unroll
-    for (int i = 0; i < NW; ++i) z[i] = 0u;
-    store_words<RB>(a.codes + slot * RB, z);
-    __half2 zs[NG];
-#pragma unroll
-    for (int g = 0; g < NG; ++g) zs[g] = __half2(__ushort_as_half(0), __ushort_as_half(0));
-    store_sz<NG>(a.sz + slot * NG, zs);
-    return;
-  }
-
-  float x[D];
-#pragma unroll
-  for (int hh = 0; hh < D / 64; ++hh)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) h8_to_f32(lds128(xs_u + hh * 16384 + sw128(tid, c)), &x[hh * 64 + c * 8]);
-
-  if (a.rope) {
-    const uint32_t rs_u = smem_u32(rs);
-#pragma unroll
-    for (int k = 0; k < D / 4; ++k) {  // chunk k = pairs 2k, 2k+1 = channels 4k..4k+3
-      const uint4 cs = lds128(rs_u + (k >> 3) * a.NT * 128 + sw128(t, k & 7));
-      rope_fwd(x[4 * k], x[4 * k + 1], __uint_as_float(cs.x), __uint_as_float(cs.y));
-      rope_fwd(x[4 * k + 2], x[4 * k + 3], __uint_as_float(cs.z), __uint_as_float(cs.w));
+      for (int c = 0; c < V / 8; ++c) dst[c] = make_uint4(raw[4 * c], raw[4 * c + 1], raw[4 * c + 2], raw[4 * c + 3]);
     }
-  }
-  if (a.perm) perm_gather<D>(x, a.perm + static_cast<size_t>(h) * D, smem_u32(ps) + tid * D * 4, tid);
-  if constexpr (ROT) {
-    fwht_reg<D>(x);
+    // P[2g + e] = (x[4g + e], x[4g + 2 + e]) over this lane's channels
+    float2 P[V / 2];
 #pragma unroll
-    for (int j = 0; j < D; ++j) x[j] = __fmul_rn(x[j], a.rscale);
-  }
-
-  uint32_t w[NW];
-#pragma unroll
-  for (int i = 0; i < NW; ++i) w[i] = 0u;
-  __half2 szv[NG];
-#pragma unroll
-  for (int g = 0; g < NG; ++g) {
-    float mn, mx;
-    minmax_range<D>(x, g * G, G, mn, mx);
-    const QParams p = minmax_params<BITS>(mn, mx);
-    szv[g] = p.sz;
-#pragma unroll
-    for (int jj = 0; jj < G; ++jj) {
-      const int j = g * G + jj;
-      const uint32_t c = quant_code(x[j], p.Z, p.R);
-      const int pos = j * BITS;
-      w[pos >> 5] |= c << (pos & 31);
-      if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= c >> (32 - (pos & 31));
+    for (int g = 0; g < V / 4; ++g) {
+      const float2 h01 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * g]));
+      const float2 h23 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * g + 1]));
+      P[2 * g] = f2(h01.x, h23.x);
+      P[2 * g + 1] = f2(h01.y, h23.y);
     }
-  }
-  store_words<RB>(a.codes + slot * RB, w);
-  store_sz<NG>(a.sz + slot * NG, szv);
-}
-
-template <int D, int BITS, int G, bool ROT>
-__global__ void __launch_bounds__(128) k_decode_head(const __grid_constant__ CUtensorMap omap,
-                                                      const __grid_constant__ CUtensorMap rmap, const HeadArgs a,
-                                                      int out_fp32) {
-  constexpr int RB = D * BITS / 8;
-  constexpr int NG = D / G;
-  constexpr int NW = D * BITS / 32;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar;
-  uint8_t* os = align1024(smem_raw);                   // output tile: fp16 D*256 B or fp32 D*512 B
-  uint8_t* rs = os + D * 512;                          // rope rows
-  uint8_t* ps = rs + a.NT * D * 4;                     // permutation rows
-  const int tid = threadIdx.x;
-  int b, h_base, t_base;
-  tile_coords(a, b, h_base, t_base);
-
-  if (a.rope) {
-    if (tid == 0) {
-      mbar_init(&bar, 1);
-      fence_mbar_init();
+    if (a.rope) {  // pairs (2i, 2i+1): y0 = fma(x0, c, -(x1*s)), y1 = fma(x0, s, x1*c)
+      const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D) + (V / 4) * s;
+#pragma unroll
+      for (int g = 0; g < V / 4; ++g) {
+        const uint4 cv = __ldg(rp + g);  // (c, s) of pairs 2g and 2g+1 of this lane
+        const float2 cc = f2(__uint_as_float(cv.x), __uint_as_float(cv.z));
+        const float2 ss = f2(__uint_as_float(cv.y), __uint_as_float(cv.w));
+        const float2 x0 = P[2 * g], x1 = P[2 * g + 1];
+        P[2 * g] = fma2(x0, cc, mul2(x1, f2(-ss.x, -ss.y)));
+        P[2 * g + 1] = fma2(x0, ss, mul2(x1, cc));
+      }
     }
-    __syncthreads();
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&bar, a.NT * D * 4);
-      for (int q = 0; q < D / 32; ++q) tma_load_2d(rs + q * a.NT * 128, &rmap, q * 32, a.t0 + t_base, &bar);
-    }
-  }
-
-  const int hl = tid / a.NT, t = tid % a.NT;
-  const int h = h_base + hl, tt = t_base + t;
-  const bool active = (h < a.H) && (tt < a.T);
-  const int m = a.t0 + tt;
-  const size_t v = static_cast<size_t>(b) * a.H + h;
-  const size_t slot = v * a.t_cap + m;
-  float x[D];
-
-  if (active && m < a.n_sink) {
-    const uint4* src = reinterpret_cast<const uint4*>(a.sink + (v * a.n_sink + m) * D);
+    if (a.perm) {  // p_j = y_perm[h][j]: stage the row, gather
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) h8_to_f32(__ldg(src + c), &x[8 * c]);
-  } else if (active) {
-    uint32_t w[NW];
-    load_words<RB>(a.codes + slot * RB, w);
-    __half2 szv[NG];
+      for (int g = 0; g < V / 4; ++g) {
+        sts64(row + 4 * (V * s + 4 * g), __float_as_uint(P[2 * g].x), __float_as_uint(P[2 * g + 1].x));
+        sts64(row + 4 * (V * s + 4 * g + 2), __float_as_uint(P[2 * g].y), __float_as_uint(P[2 * g + 1].y));
+      }
+      __syncwarp();
+      const int16_t* pr = a.perm + static_cast<size_t>(h) * D + V * s;
+      float xv[V];
 #pragma unroll
-    for (int g = 0; g < NG; ++g) szv[g] = a.sz[slot * NG + g];
+      for (int c = 0; c < V / 8; ++c) {
+        const uint4 pk = __ldg(reinterpret_cast<const uint4*>(pr) + c);
+        const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
-    for (int j = 0; j < D; ++j) {
-      const float S = __low2float(szv[j / G]), Z = __high2float(szv[j / G]);
-      x[j] = __fmaf_rn(code_to_float(unpack_code<BITS, NW>(w, j)), S, Z);
+        for (int i = 0; i < 8; ++i)
+          xv[8 * c + i] = lds32f(row + 4 * ((pw[i >> 1] >> (16 * (i & 1))) & (D - 1)));
+      }
+      __syncwarp();  // the row buffer is free for the next step
+#pragma unroll
+      for (int g = 0; g < V / 4; ++g) {
+        P[2 * g] = f2(xv[4 * g], xv[4 * g + 2]);
+        P[2 * g + 1] = f2(xv[4 * g + 1], xv[4 * g + 3]);
+      }
     }
     if constexpr (ROT) {
-      fwht_reg<D>(x);
+      fwht_pairs<V>(P);
+      // stride V across the lane pair: lower lane a + b, upper lane a - b
+      const float sg = s ? -1.0f : 1.0f;
 #pragma unroll
-      for (int j = 0; j < D; ++j) x[j] = __fmul_rn(x[j], a.rscale);
+      for (int k = 0; k < V / 2; ++k) {
+        const float2 o = P[k];
+        const float2 p = f2(__shfl_xor_sync(0xffffffffu, o.x, 1), __shfl_xor_sync(0xffffffffu, o.y, 1));
+        P[k] = fma2(o, f2(sg, sg), p);
+      }
+#pragma unroll
+      for (int k = 0; k < V / 2; ++k) P[k] = mul2(P[k], f2(r, r));
     }
-    if (a.perm) perm_scatter<D>(x, a.perm + static_cast<size_t>(h) * D, smem_u32(ps) + tid * D * 4, tid);
-  }
-  // Every thread waits for the RoPE rows (so no copy is in flight when the
-  // CTA exits); on a timeout the kernel still reaches its barrier and exits.
-  const bool rope_ok = a.rope ? mbar_wait(&bar, 0, a.wait_ns, a.err) : true;
-  if (active && m >= a.n_sink && a.rope && rope_ok) {
-    {
-      const uint32_t rs_u = smem_u32(rs);
+
+    // min-max per group, fp16 (scale, zero); a sink slot quantizes with Z = R = 0
+    float Zg[NGT], Rg[NGT];
+    __half2 szg[NGT];
 #pragma unroll
-      for (int k = 0; k < D / 4; ++k) {
-        const uint4 cs = lds128(rs_u + (k >> 3) * a.NT * 128 + sw128(t, k & 7));
-        rope_inv(x[4 * k], x[4 * k + 1], __uint_as_float(cs.x), __uint_as_float(cs.y));
-        rope_inv(x[4 * k + 2], x[4 * k + 3], __uint_as_float(cs.z), __uint_as_float(cs.w));
+    for (int gg = 0; gg < NGT; ++gg) {
+      constexpr int QG = GS / 4;  // channel quads per group
+      float lo = fminf(P[2 * QG * gg].x, P[2 * QG * gg].y), hi = fmaxf(P[2 * QG * gg].x, P[2 * QG * gg].y);
+      lo = min3f(lo, P[2 * QG * gg + 1].x, P[2 * QG * gg + 1].y);
+      hi = max3f(hi, P[2 * QG * gg + 1].x, P[2 * QG * gg + 1].y);
+#pragma unroll
+      for (int q = 1; q < QG; ++q) {
+        const float2 e0 = P[2 * (QG * gg + q)], e1 = P[2 * (QG * gg + q) + 1];
+        lo = min3f(lo, e0.x, e0.y);
+        hi = max3f(hi, e0.x, e0.y);
+        lo = min3f(lo, e1.x, e1.y);
+        hi = max3f(hi, e1.x, e1.y);
+      }
+      if constexpr (SHARED) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, 1));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, 1));
+      }
+      const QParams p = minmax_params<BITS>(lo, hi);
+      Zg[gg] = sink_tok ? 0.0f : p.Z;
+      Rg[gg] = sink_tok ? 0.0f : p.R;
+      szg[gg] = sink_tok ? __halves2half2(__ushort_as_half(0), __ushort_as_half(0)) : p.sz;
+    }
+
+    // quantize and pack this lane's V codes (LSB first)
+    uint32_t w[NW];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) w[i] = 0u;
+#pragma unroll
+    for (int g = 0; g < V / 4; ++g) {
+      const int gg = (4 * g) / GS;
+      const float2 nZ = f2(-Zg[gg], -Zg[gg]), R2 = f2(Rg[gg], Rg[gg]), M2 = f2(kMagicRound, kMagicRound);
+      const float2 ua = fma2(add2(P[2 * g], nZ), R2, M2);
+      const float2 ub = fma2(add2(P[2 * g + 1], nZ), R2, M2);
+      const uint32_t t4[4] = {__float_as_uint(ua.x), __float_as_uint(ub.x), __float_as_uint(ua.y),
+                              __float_as_uint(ub.y)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int pos = (4 * g + e) * BITS;
+        if constexpr (32 % BITS == 0) {
+          w[pos >> 5] += t4[e] << (pos & 31);  // codes never straddle a word
+        } else {
+          const uint32_t c = t4[e] - kMagicBits;
+          w[pos >> 5] |= c << (pos & 31);
+          if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= c >> (32 - (pos & 31));
+        }
+      }
+    }
+    if constexpr (32 % BITS == 0) {
+#pragma unroll
+      for (int i = 0; i < NW; ++i) w[i] -= magic_offset<BITS, 32 / BITS>();
+    }
+    if (live) {
+      const size_t slot_i = vec * a.t_cap + m;
+      st_run<NBY, pow2_align(NBY)>(a.codes + slot_i * RB + NBY * s, w);
+      if constexpr (SHARED) {
+        if (s == 0) a.sz[slot_i] = szg[0];
+      } else if constexpr (NGT == 1) {
+        a.sz[slot_i * NG + s] = szg[0];
+      } else {
+        static_assert(NGT == 2, "at most two groups per lane");
+        *reinterpret_cast<uint2*>(a.sz + slot_i * NG + 2 * s) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&szg[0]), *reinterpret_cast<const uint32_t*>(&szg[1]));
       }
     }
   }
+}
 
-  const uint32_t os_u = smem_u32(os);
-  if (active) {
-    if (out_fp32) {
+template <int D, int BITS, int G, bool ROT, bool F32>
+__global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
+  constexpr int V = D / 2;
+  constexpr int RB = D * BITS / 8;
+  constexpr int NG = D / G;
+  constexpr bool SHARED = G > V;
+  constexpr int GS = SHARED ? V : G;
+  constexpr int NGT = V / GS;
+  constexpr int NBY = V * BITS / 8;
+  constexpr int NW = NBY / 4;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  constexpr int ES = F32 ? 4 : 2;
+  extern __shared__ uint8_t smem_raw[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int s = lane & 1, slot = lane >> 1;
+  const uint32_t row = smem_u32(smem_raw) + (warp * kVecW + slot) * row_pitch<D>();
+  const float r = a.rscale;
+  const bool v8 = a.v8 != 0;
+  const uint32_t gw = blockIdx.x * (kThreads / 32) + warp, nw = gridDim.x * (kThreads / 32);
+
+  for (uint32_t base = gw * kVecW; base < a.n_vec; base += nw * kVecW) {
+    const uint32_t v = base + slot;
+    const bool live = v < a.n_vec;
+    uint32_t bh;
+    int h, tt;
+    vec_coords(a, live ? v : a.n_vec - 1, bh, h, tt);
+    const int m = a.t0 + tt;
+    const size_t vec = bh;
+    const size_t slot_i = vec * a.t_cap + m;
+    const bool sink_tok = m < a.n_sink;
+
+    uint32_t w[NW];
+    ld_run<NBY, pow2_align(NBY)>(a.codes + slot_i * RB + NBY * s, w);
+    float Sg[NGT], Zg[NGT];
 #pragma unroll
-      for (int c = 0; c < D / 4; ++c)
-        sts128(os_u + (c >> 3) * 16384 + sw128(tid, c & 7),
-               make_uint4(__float_as_uint(x[4 * c]), __float_as_uint(x[4 * c + 1]), __float_as_uint(x[4 * c + 2]),
-                          __float_as_uint(x[4 * c + 3])));
+    for (int gg = 0; gg < NGT; ++gg) {
+      const float2 sz = __half22float2(a.sz[slot_i * NG + (SHARED ? 0 : NGT * s + gg)]);
+      Sg[gg] = ROT ? __fmul_rn(sz.x, r) : sz.x;  // the normalisation folds into S and Z
+      Zg[gg] = ROT ? __fmul_rn(sz.y, r) : sz.y;
+    }
+    // dequantize: codes 0 and 2 of a quad are masked in place at bit 0, codes
+    // 1 and 3 at bit BITS; read through the fp32 pattern 2^23 + v they give
+    // code * 2^p, and the power of two 2^p folds exactly into the scale.
+    float2 P[V / 2];
+#pragma unroll
+    for (int g = 0; g < V / 4; ++g) {
+      const int gg = (4 * g) / GS;
+      const int pos = 4 * g * BITS;
+      const uint32_t lo = w[pos >> 5] >> (pos & 31);
+      const uint32_t w0 =
+          (32 - (pos & 31) >= 4 * BITS || (pos >> 5) + 1 >= NW) ? lo : (lo | (w[(pos >> 5) + 1] << (32 - (pos & 31))));
+      const uint32_t w1 = w0 >> (2 * BITS);
+      const float2 c02 = f2(__uint_as_float(0x4B000000u | (w0 & MASK)), __uint_as_float(0x4B000000u | (w1 & MASK)));
+      const float2 c13 = f2(__uint_as_float(0x4B000000u | (w0 & (MASK << BITS))),
+                            __uint_as_float(0x4B000000u | (w1 & (MASK << BITS))));
+      const float2 nM = f2(-8388608.0f, -8388608.0f), Z2 = f2(Zg[gg], Zg[gg]);
+      const float S1 = Sg[gg] * (1.0f / (1 << BITS));
+      P[2 * g] = fma2(add2(c02, nM), f2(Sg[gg], Sg[gg]), Z2);
+      P[2 * g + 1] = fma2(add2(c13, nM), f2(S1, S1), Z2);
+    }
+    if constexpr (ROT) {  // the transform is its own inverse: stride V across the pair, then 1 .. V/2
+      const float sg = s ? -1.0f : 1.0f;
+#pragma unroll
+      for (int k = 0; k < V / 2; ++k) {
+        const float2 o = P[k];
+        const float2 p = f2(__shfl_xor_sync(0xffffffffu, o.x, 1), __shfl_xor_sync(0xffffffffu, o.y, 1));
+        P[k] = fma2(o, f2(sg, sg), p);
+      }
+      fwht_pairs<V>(P);
+    }
+    if (a.perm) {  // x[perm[h][j]] = p_j: scatter into the row, read this lane's half back
+      const int16_t* pr = a.perm + static_cast<size_t>(h) * D + V * s;
+#pragma unroll
+      for (int c = 0; c < V / 8; ++c) {
+        const uint4 pk = __ldg(reinterpret_cast<const uint4*>(pr) + c);
+        const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = 8 * c + i;  // local channel: P[2(j/4) + (j&1)], lane (j>>1)&1
+          const float xv = ((j >> 1) & 1) ? P[2 * (j >> 2) + (j & 1)].y : P[2 * (j >> 2) + (j & 1)].x;
+          sts32f(row + 4 * ((pw[i >> 1] >> (16 * (i & 1))) & (D - 1)), xv);
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int g = 0; g < V / 4; ++g) {
+        const uint2 u = lds64(row + 4 * (V * s + 4 * g)), w2 = lds64(row + 4 * (V * s + 4 * g + 2));
+        P[2 * g] = f2(__uint_as_float(u.x), __uint_as_float(w2.x));
+        P[2 * g + 1] = f2(__uint_as_float(u.y), __uint_as_float(w2.y));
+      }
+      __syncwarp();  // the row buffer is free for the next step
+    }
+    if (a.rope) {  // inverse pairs: x0 = y0 c + y1 s, x1 = y1 c - y0 s
+      const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D) + (V / 4) * s;
+#pragma unroll
+      for (int g = 0; g < V / 4; ++g) {
+        const uint4 cv = __ldg(rp + g);
+        const float2 cc = f2(__uint_as_float(cv.x), __uint_as_float(cv.z));
+        const float2 ss = f2(__uint_as_float(cv.y), __uint_as_float(cv.w));
+        const float2 y0 = P[2 * g], y1 = P[2 * g + 1];
+        P[2 * g] = fma2(y0, cc, mul2(y1, ss));
+        P[2 * g + 1] = fma2(y1, cc, mul2(y0, f2(-ss.x, -ss.y)));
+      }
+    }
+    // output words of this lane's half row (a sink slot comes back verbatim)
+    uint32_t ow[V * ES / 4];
+    if (sink_tok) {
+      uint32_t hv[V / 2];
+      ld_row<V / 2>(a.sink + (vec * a.n_sink + m) * D + V * s, false, hv);
+      if constexpr (F32) {
+#pragma unroll
+        for (int j = 0; j < V / 2; ++j) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hv[j]));
+          ow[2 * j] = __float_as_uint(f.x);
+          ow[2 * j + 1] = __float_as_uint(f.y);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < V / 2; ++j) ow[j] = hv[j];
+      }
+    } else if constexpr (F32) {
+#pragma unroll
+      for (int g = 0; g < V / 4; ++g) {
+        ow[4 * g] = __float_as_uint(P[2 * g].x);
+        ow[4 * g + 1] = __float_as_uint(P[2 * g + 1].x);
+        ow[4 * g + 2] = __float_as_uint(P[2 * g].y);
+        ow[4 * g + 3] = __float_as_uint(P[2 * g + 1].y);
+      }
     } else {
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) sts128(os_u + (c >> 3) * 16384 + sw128(tid, c & 7), f32_to_h8(&x[8 * c]));
+      for (int g = 0; g < V / 4; ++g) {
+        const __half2 h01 = __floats2half2_rn(P[2 * g].x, P[2 * g + 1].x);
+        const __half2 h23 = __floats2half2_rn(P[2 * g].y, P[2 * g + 1].y);
+        ow[2 * g] = *reinterpret_cast<const uint32_t*>(&h01);
+        ow[2 * g + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+      }
     }
-  }
-  fence_async_smem();
-  __syncthreads();
-  if (tid == 0 && a.rope && !rope_ok) mbar_wait(&bar, 0, a.wait_ns, a.err);
-  if (tid == 0) {
-    const int nbox = out_fp32 ? D / 32 : D / 64;
-    const int step = out_fp32 ? 32 : 64;
-    for (int i = 0; i < nbox; ++i) tma_store_3d(&omap, i * step, t_base, b * a.H + h_base, os + i * 16384);
-    bulk_commit();
-    bulk_wait_read0();
+    if (live) st_row<V * ES / 4>(static_cast<uint8_t*>(a.out) + ((vec * a.T + tt) * D + V * s) * ES, v8, ow);
   }
 }
 
 template <int D, int BITS, int G, bool ROT>
-kvq_status run_encode(const HeadArgs& a, const CUtensorMap& xm, const CUtensorMap& rm, size_t smem,
-                      cudaStream_t st) {
-  auto k = k_encode_head<D, BITS, G, ROT>;
-  if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
-    return KVQ_ERR_CUDA;
-  const size_t grid = static_cast<size_t>(a.B) * a.n_hblk * a.n_tblk;
-  k<<<static_cast<unsigned>(grid), 128, smem, st>>>(xm, rm, a);
-  return launch_status();
-}
-template <int D, int BITS, int G, bool ROT>
-kvq_status run_decode(const HeadArgs& a, const CUtensorMap& om, const CUtensorMap& rm, size_t smem, int out_fp32,
-                      cudaStream_t st) {
-  auto k = k_decode_head<D, BITS, G, ROT>;
-  if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
-    return KVQ_ERR_CUDA;
-  const size_t grid = static_cast<size_t>(a.B) * a.n_hblk * a.n_tblk;
-  k<<<static_cast<unsigned>(grid), 128, smem, st>>>(om, rm, a, out_fp32);
+kvq_status run(bool enc, const HeadArgs& a, int out_fp32, const LaunchCtx& ctx, cudaStream_t st) {
+  const size_t smem = a.perm ? static_cast<size_t>(kThreads / 32) * kVecW * row_pitch<D>() : 0;
+  const void* fn = enc        ? reinterpret_cast<const void*>(k_encode_head<D, BITS, G, ROT>)
+                   : out_fp32 ? reinterpret_cast<const void*>(k_decode_head<D, BITS, G, ROT, true>)
+                              : reinterpret_cast<const void*>(k_decode_head<D, BITS, G, ROT, false>);
+  if (smem && !set_smem_once(fn, smem)) return KVQ_ERR_CUDA;
+  const int per_sm = occupancy_once(fn, kThreads, smem);
+  const long long steps = (static_cast<long long>(a.n_vec) + kVecW * (kThreads / 32) - 1) / (kVecW * (kThreads / 32));
+  const long long want = static_cast<long long>(ctx.num_sms) * per_sm;
+  const unsigned grid = static_cast<unsigned>(steps < want ? steps : want);
+  if (enc)
+    k_encode_head<D, BITS, G, ROT><<<grid, kThreads, smem, st>>>(a);
+  else if (out_fp32)
+    k_decode_head<D, BITS, G, ROT, true><<<grid, kThreads, smem, st>>>(a);
+  else
+    k_decode_head<D, BITS, G, ROT, false><<<grid, kThreads, smem, st>>>(a);
   return launch_status();
 }
 
-// Dispatch over (D, BITS, G, ROT).
-template <bool ENC>
-kvq_status dispatch(const kvq_desc& d, const HeadArgs& a, const CUtensorMap& m0, const CUtensorMap& rm, size_t smem,
-                    int out_fp32, cudaStream_t st) {
+kvq_status dispatch(bool enc, const kvq_desc& d, const HeadArgs& a, int out_fp32, const LaunchCtx& ctx,
+                    cudaStream_t st) {
   const bool rot = d.rot == KVQ_ROT_FWHT_HEAD;
-#define KVQ_CASE(D_, B_, G_)                                                                     \
-  if (d.head_dim == D_ && d.bits == B_ && d.group == G_) {                                      \
-    if constexpr (ENC) {                                                                        \
-      return rot ? run_encode<D_, B_, G_, true>(a, m0, rm, smem, st)                            \
-                 : run_encode<D_, B_, G_, false>(a, m0, rm, smem, st);                          \
-    } else {                                                                                    \
-      return rot ? run_decode<D_, B_, G_, true>(a, m0, rm, smem, out_fp32, st)                  \
-                 : run_decode<D_, B_, G_, false>(a, m0, rm, smem, out_fp32, st);                \
-    }                                                                                           \
-  }
+#define KVQ_CASE(D_, B_, G_)                                                  \
+  if (d.head_dim == D_ && d.bits == B_ && d.group == G_)                     \
+    return rot ? run<D_, B_, G_, true>(enc, a, out_fp32, ctx, st)            \
+               : run<D_, B_, G_, false>(enc, a, out_fp32, ctx, st);
 #define KVQ_BITS(D_, G_) KVQ_CASE(D_, 2, G_) KVQ_CASE(D_, 3, G_) KVQ_CASE(D_, 4, G_)
   KVQ_BITS(128, 128)
   KVQ_BITS(128, 64)
@@ -390,8 +451,10 @@ kvq_status dispatch(const kvq_desc& d, const HeadArgs& a, const CUtensorMap& m0,
   return KVQ_ERR_UNSUPPORTED;
 }
 
-HeadArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p, const LaunchCtx& ctx) {
-  HeadArgs a{};
+bool make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p, HeadArgs& a) {
+  const unsigned long long n = static_cast<unsigned long long>(d.batch) * d.heads * d.tokens;
+  if (n >= (1ull << 31)) return false;  // vector indices are 31-bit
+  a = HeadArgs{};
   a.B = d.batch;
   a.H = d.heads;
   a.T = d.tokens;
@@ -399,68 +462,38 @@ HeadArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p,
   a.t_cap = d.t_cap;
   a.n_sink = d.n_sink;
   a.rope = d.rope;
-  a.HT = heads_per_tile(d.heads);
-  a.NT = 128 / a.HT;
-  a.n_tblk = (d.tokens + a.NT - 1) / a.NT;
-  a.n_hblk = d.heads / a.HT;
+  a.n_vec = static_cast<uint32_t>(n);
+  a.div_t = FastDiv(static_cast<uint32_t>(d.tokens));
+  a.div_h = FastDiv(static_cast<uint32_t>(d.heads));
   a.rscale = static_cast<float>(1.0 / sqrt(static_cast<double>(d.head_dim)));
   a.perm = tb.perm;
+  a.rope_cs = tb.rope_cs;
   a.codes = p.codes;
   a.sz = static_cast<__half2*>(p.scale_zero);
   a.sink = static_cast<__half*>(p.sink);
-  a.err = ctx.err;
-  a.wait_ns = ctx.wait_ns;
-  return a;
+  return true;
 }
 
-bool rope_map(CUtensorMap* m, const kvq_desc& d, const kvq_tables& tb, int NT) {
-  if (!d.rope) {
-    *m = CUtensorMap{};
-    return true;
-  }
-  const uint64_t dims[2] = {static_cast<uint64_t>(d.head_dim), static_cast<uint64_t>(tb.rope_rows)};
-  const uint64_t strides[1] = {static_cast<uint64_t>(d.head_dim) * 4};
-  const uint32_t box[2] = {32, static_cast<uint32_t>(NT)};
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, tb.rope_cs, dims, strides, box,
-                  CU_TENSOR_MAP_SWIZZLE_128B);
-}
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 }  // namespace
 
 kvq_status launch_encode_head(const kvq_desc& d, const void* x, const kvq_tables& tb, const kvq_packed& out,
                               cudaStream_t st, const LaunchCtx& ctx) {
-  const HeadArgs a = make_args(d, tb, out, ctx);
-  CUtensorMap xm, rm;
-  const uint64_t dims[3] = {static_cast<uint64_t>(d.head_dim), static_cast<uint64_t>(d.tokens),
-                            static_cast<uint64_t>(d.batch) * d.heads};
-  const uint64_t strides[2] = {static_cast<uint64_t>(d.head_dim) * 2,
-                               static_cast<uint64_t>(d.tokens) * d.head_dim * 2};
-  const uint32_t box[3] = {64, static_cast<uint32_t>(a.NT), static_cast<uint32_t>(a.HT)};
-  if (!make_map(&xm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-    return KVQ_ERR_CUDA;
-  if (!rope_map(&rm, d, tb, a.NT)) return KVQ_ERR_CUDA;
-  const size_t smem = 1024 + static_cast<size_t>(d.head_dim) * 256 + static_cast<size_t>(a.NT) * d.head_dim * 4 +
-                      (tb.perm ? static_cast<size_t>(128) * d.head_dim * 4 : 0);
-  return dispatch<true>(d, a, xm, rm, smem, 0, st);
+  HeadArgs a;
+  if (!make_args(d, tb, out, a)) return KVQ_ERR_UNSUPPORTED;
+  a.x = static_cast<const __half*>(x);
+  a.v8 = aligned32(x);
+  return dispatch(true, d, a, 0, ctx, st);
 }
 
 kvq_status launch_decode_head(const kvq_desc& d, const kvq_packed& in, const kvq_tables& tb, void* x_out,
                               int out_fp32, cudaStream_t st, const LaunchCtx& ctx) {
-  HeadArgs a = make_args(d, tb, in, ctx);
-  CUtensorMap om, rm;
-  const uint64_t es = out_fp32 ? 4 : 2;
-  const uint64_t dims[3] = {static_cast<uint64_t>(d.head_dim), static_cast<uint64_t>(d.tokens),
-                            static_cast<uint64_t>(d.batch) * d.heads};
-  const uint64_t strides[2] = {static_cast<uint64_t>(d.head_dim) * es,
-                               static_cast<uint64_t>(d.tokens) * d.head_dim * es};
-  const uint32_t box[3] = {out_fp32 ? 32u : 64u, static_cast<uint32_t>(a.NT), static_cast<uint32_t>(a.HT)};
-  if (!make_map(&om, out_fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, x_out, dims,
-                strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-    return KVQ_ERR_CUDA;
-  if (!rope_map(&rm, d, tb, a.NT)) return KVQ_ERR_CUDA;
-  const size_t smem = 1024 + static_cast<size_t>(d.head_dim) * 512 + static_cast<size_t>(a.NT) * d.head_dim * 4 +
-                      (tb.perm ? static_cast<size_t>(128) * d.head_dim * 4 : 0);
-  return dispatch<false>(d, a, om, rm, smem, out_fp32, st);
+  HeadArgs a;
+  if (!make_args(d, tb, in, a)) return KVQ_ERR_UNSUPPORTED;
+  a.out = x_out;
+  a.v8 = aligned32(x_out);
+  return dispatch(false, d, a, out_fp32, ctx, st);
 }
 
 }  // namespace kvq
