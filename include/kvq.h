@@ -146,6 +146,29 @@ kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kv
                      const kvq_tables* tb, int32_t n_tokens, float scale, float* scores,
                      kvq_stream_t stream);
 
+/* Decode-step attention over the compressed cache ([EliteKV §2.2] scores; [EliteKV §7.1] the
+ * softmax of the scaled scores weights the values):
+ *   out[b][qh] = sum_n p_n vhat[b][h][n],  p = softmax_n(scale * <q[b][qh], khat[b][h][n]>),
+ *   n in [0, n_tokens), h = qh / (q_heads/H).
+ * khat_n is the kvq_score key (K cache: dk, k_cache, tk); vhat_n is value slot n decoded as by
+ * kvq_decode (V cache: dv, v_cache, tv), the sink rows verbatim. dk and dv must agree in batch,
+ * heads, head_dim (= 128), t_cap, bits, group, n_sink, rot (NONE or FWHT_HEAD) and quant
+ * (MINMAX); dv->rope must be 0 and q_heads/H in {1, 2, 4, 8} (else KVQ_ERR_UNSUPPORTED).
+ * The value decode is linear in the dequantized codes y_n, so sum_n p_n vhat_n =
+ * P^T H_norm (sum_n p_n y_n): the inverse rotation runs once per output, not per token.
+ * q: half [B][q_heads][head_dim] in attention space, 16-byte aligned. out: f32
+ * [B][q_heads][head_dim], 16-byte aligned. workspace: caller-owned device memory, 256-byte
+ * aligned, at least kvq_attend_workspace_bytes() bytes; it holds the scores and per-chunk
+ * partial sums, needs no initialisation and must not be shared by calls in flight at the same
+ * time. d->tokens and d->t0 are ignored. Launches three kernels on `stream`. */
+kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int32_t q_heads,
+                      const kvq_packed* k_cache, const kvq_tables* tk, const kvq_packed* v_cache,
+                      const kvq_tables* tv, int32_t n_tokens, float scale, float* out, void* workspace,
+                      size_t workspace_bytes, kvq_stream_t stream);
+
+/* Workspace bytes kvq_attend needs for these arguments; 0 if they are invalid or unsupported. */
+size_t kvq_attend_workspace_bytes(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads, int32_t n_tokens);
+
 /* Bytes of one packed buffer (KVQ_FIELD_*) for this descriptor; 0 if the field is unused or
  * the descriptor is invalid. */
 size_t kvq_packed_bytes(const kvq_desc* d, int32_t field);

@@ -248,6 +248,57 @@ kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kv
                       ctx);
 }
 
+namespace {
+// Shapes kvq_attend accepts: dk / dv valid, head-variant (or unrotated) min-max
+// caches of the same record shape, head_dim 128, values without RoPE.
+kvq_status check_attend(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads, int32_t n_tokens,
+                        kvq_desc* k_out, kvq_desc* v_out) {
+  if (!dk || !dv) return KVQ_ERR_INVALID;
+  kvq_desc k = *dk, v = *dv;
+  k.tokens = v.tokens = 0;
+  k.t0 = v.t0 = 0;
+  kvq_status s;
+  if ((s = check_desc(&k)) != KVQ_OK || (s = check_desc(&v)) != KVQ_OK) return s;
+  if (k.rot != KVQ_ROT_NONE && k.rot != KVQ_ROT_FWHT_HEAD) return KVQ_ERR_UNSUPPORTED;
+  if (k.quant != KVQ_Q_MINMAX || k.head_dim != 128 || v.rope) return KVQ_ERR_UNSUPPORTED;
+  if (k.batch != v.batch || k.heads != v.heads || k.head_dim != v.head_dim || k.t_cap != v.t_cap ||
+      k.bits != v.bits || k.group != v.group || k.n_sink != v.n_sink || k.rot != v.rot || k.quant != v.quant)
+    return KVQ_ERR_INVALID;
+  if (q_heads <= 0 || q_heads % k.heads) return KVQ_ERR_INVALID;
+  const int gq = q_heads / k.heads;
+  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KVQ_ERR_UNSUPPORTED;
+  if (n_tokens < 1 || n_tokens > k.t_cap) return KVQ_ERR_INVALID;
+  *k_out = k;
+  *v_out = v;
+  return KVQ_OK;
+}
+}  // namespace
+
+size_t kvq_attend_workspace_bytes(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads, int32_t n_tokens) {
+  kvq_desc k, v;
+  if (check_attend(dk, dv, q_heads, n_tokens, &k, &v) != KVQ_OK) return 0;
+  return attend_workspace_bytes(k.batch, q_heads, n_tokens);
+}
+
+kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int32_t q_heads,
+                      const kvq_packed* k_cache, const kvq_tables* tk, const kvq_packed* v_cache,
+                      const kvq_tables* tv, int32_t n_tokens, float scale, float* out, void* workspace,
+                      size_t workspace_bytes, kvq_stream_t stream) {
+  kvq_desc k, v;
+  kvq_status s = check_attend(dk, dv, q_heads, n_tokens, &k, &v);
+  if (s != KVQ_OK) return s;
+  if (!q || !out || !workspace) return KVQ_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_ALIGN;
+  if (workspace_bytes < attend_workspace_bytes(k.batch, q_heads, n_tokens)) return KVQ_ERR_INVALID;
+  if ((s = check_tables(&k, tk, k.rope ? (n_tokens < k.n_sink ? n_tokens : k.n_sink) : 0)) != KVQ_OK) return s;
+  if ((s = check_tables(&v, tv, 0)) != KVQ_OK) return s;
+  if ((s = check_packed(&k, k_cache)) != KVQ_OK || (s = check_packed(&v, v_cache)) != KVQ_OK) return s;
+  LaunchCtx ctx;
+  if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
+  return launch_attend(k, v, q, q_heads, *k_cache, *tk, *v_cache, *tv, n_tokens, scale, out, workspace,
+                       reinterpret_cast<cudaStream_t>(stream), ctx);
+}
+
 size_t kvq_packed_bytes(const kvq_desc* d, int32_t field) {
   if (!d) return 0;
   kvq_desc dd = *d;

@@ -133,6 +133,38 @@ def score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens
                     out.data_ptr(), _stream(stream)), "kvq_score")
 
 
+def attend_workspace(dk: kvq_desc, dv: kvq_desc, q_heads: int, n_tokens: int, device="cuda") -> torch.Tensor:
+    """A workspace tensor for kvq_attend (256-byte aligned, as torch allocates)."""
+    from . import kvq_attend_workspace_bytes
+    nb = kvq_attend_workspace_bytes(dk, dv, q_heads, n_tokens)
+    if nb == 0:
+        raise ValueError("kvq_attend: invalid or unsupported shapes")
+    return torch.empty(nb, dtype=torch.uint8, device=device)
+
+
+def attend(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, tk: Tables, v_packed: Packed, tv: Tables,
+           n_tokens: int, scale: float, out: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    from . import kvq_attend
+    check(kvq_attend(dk, dv, q.data_ptr(), q.shape[1], k_packed.struct(), tk.struct(), v_packed.struct(),
+                     tv.struct(), n_tokens, scale, out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                     _stream(stream)), "kvq_attend")
+
+
+def bind_attend(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, tk: Tables, v_packed: Packed,
+                tv: Tables, n_tokens: int, scale: float, out: torch.Tensor, workspace: torch.Tensor, stream=None):
+    from . import lib
+    tks, kps, tvs, vps, st = tk.struct(), k_packed.struct(), tv.struct(), v_packed.struct(), _stream(stream)
+    args = (ctypes.byref(dk), ctypes.byref(dv), q.data_ptr(), q.shape[1], ctypes.byref(kps), ctypes.byref(tks),
+            ctypes.byref(vps), ctypes.byref(tvs), n_tokens, ctypes.c_float(scale), out.data_ptr(),
+            workspace.data_ptr(), workspace.numel(), st)
+    keep = (dk, dv, q, k_packed, tk, v_packed, tv, out, workspace, tks, kps, tvs, vps)
+
+    def call():
+        check(lib.kvq_attend(*args), "kvq_attend")
+    call.keep = keep
+    return call
+
+
 # ---------------------------------------------------------------- pre-bound calls
 # The same marshalling, done once: the returned zero-argument callables hold
 # the ctypes structs and raw addresses and launch with no per-call Python

@@ -88,6 +88,9 @@ def lib():
         L.orc_score.restype = ci
         L.orc_score.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, cd,
                                 u16p, u8p, u16p, u16p, f32p, i16p, f32p, f32p, f32p, i64p, ci, cd, f64p]
+        L.orc_attend.restype = ci
+        L.orc_attend.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, cd, u16p,
+                                 u8p, u16p, u16p, i16p, ci, u8p, u16p, u16p, i16p, ci, cd, f64p]
         L.orc_calibrate_perm.restype = ci
         L.orc_calibrate_perm.argtypes = [ci, ci, ci, ci, i64p, ci, ci, cd, u16p, i16p]
         _lib = L
@@ -285,6 +288,34 @@ def score(q, cache, tokens, *, H, t_cap, rot, quant=Q_MINMAX, bits, group=0, gro
                          _p(tok, ctypes.c_int64), tok.size, float(scale), _p(out, ctypes.c_double))
     if rc:
         raise ValueError("oracle score: unsupported parameters")
+    return out
+
+
+def attend(q, kcache, vcache, n_tok, *, H, t_cap, rot, bits, group, n_sink=0, base=10000.0, scale,
+           kperm=None, vperm=None, krope=1, vrope=0):
+    """Decode-step attention (orc_attend). q: uint16 [B][Hq][D] in attention
+    space; kcache / vcache: dicts of codes, sz and sink laid out over t_cap
+    slots. Returns float64 [B][Hq][D]."""
+    q = np.ascontiguousarray(q, np.uint16)
+    B, Hq, D = q.shape
+    out = np.zeros((B, Hq, D), np.float64)
+
+    def arrs(c, perm):
+        codes = np.ascontiguousarray(c["codes"], np.uint8)
+        sz = np.ascontiguousarray(c["sz"], np.uint16)
+        sink = np.ascontiguousarray(c["sink"], np.uint16) if c.get("sink") is not None else None
+        pm = None if perm is None else np.ascontiguousarray(perm, np.int16)
+        return codes, sz, sink, pm
+
+    kc, kz, ks, kp = arrs(kcache, kperm)
+    vc, vz, vs, vp = arrs(vcache, vperm)
+    rc = lib().orc_attend(B, H, Hq, D, t_cap, int(n_tok), rot, bits, group, n_sink, base, _p(q, ctypes.c_uint16),
+                          _p(kc, ctypes.c_uint8), _p(kz, ctypes.c_uint16), _p(ks, ctypes.c_uint16),
+                          _p(kp, ctypes.c_int16), int(krope), _p(vc, ctypes.c_uint8), _p(vz, ctypes.c_uint16),
+                          _p(vs, ctypes.c_uint16), _p(vp, ctypes.c_int16), int(vrope), float(scale),
+                          _p(out, ctypes.c_double))
+    if rc:
+        raise ValueError("oracle attend: unsupported parameters")
     return out
 
 

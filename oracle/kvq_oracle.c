@@ -688,6 +688,57 @@ int orc_score(int B, int H, int Hq, int D, int t_cap, int rot, int quant, int bi
 }
 
 /* ------------------------------------------------------------------------
+ * Decode-step attention ("EliteKV - RoPE频率选择与低秩投影" §2.2: the score
+ * of query m and key n is q_m^rot . k_n^rot / sqrt(d); §7.1: the softmax of
+ * the scaled scores over the cached tokens weights the values). For query
+ * head qh of batch b (KV head h = qh / (Hq/H)) over cache slots n < n_tok:
+ *   s_n   = scale * q . khat_n          (as orc_score: attention-space keys)
+ *   p_n   = exp(s_n - max s) / sum exp(s - max s)
+ *   out   = sum_n p_n * vhat_n          (vhat_n: decoded V slot n; sinks verbatim)
+ * K and V caches share the record shape (rot, bits, group, n_sink) and have
+ * their own RoPE flag and permutation. fp64 throughout.
+ * ---------------------------------------------------------------------- */
+int orc_attend(int B, int H, int Hq, int D, int t_cap, int n_tok, int rot, int bits, int group, int n_sink,
+               double base, const uint16_t* q, const uint8_t* kcodes, const uint16_t* ksz,
+               const uint16_t* ksink, const int16_t* kperm, int krope, const uint8_t* vcodes,
+               const uint16_t* vsz, const uint16_t* vsink, const int16_t* vperm, int vrope, double scale,
+               double* out) {
+  if (Hq % H || n_tok < 1 || n_tok > t_cap) return 1;
+  if (rot != ORC_ROT_NONE && rot != ORC_ROT_FWHT_HEAD) return 1;
+  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)t_cap);
+  for (int n = 0; n < t_cap; ++n) tok[n] = n;
+  double* s = (double*)malloc(sizeof(double) * (size_t)B * Hq * n_tok);
+  double* vh = (double*)malloc(sizeof(double) * (size_t)B * H * t_cap * D);
+  int rc = orc_score(B, H, Hq, D, t_cap, rot, ORC_Q_MINMAX, bits, group, 1, krope, n_sink, base, q, kcodes, ksz,
+                     ksink, NULL, kperm, NULL, NULL, NULL, tok, n_tok, scale, s);
+  if (!rc)
+    rc = orc_decode(B, H, t_cap, D, tok, rot, ORC_Q_MINMAX, bits, group, 1, vrope, n_sink, base, vcodes, vsz,
+                    vsink, NULL, vperm, NULL, NULL, NULL, vh);
+  if (!rc) {
+    for (int b = 0; b < B; ++b)
+      for (int qh = 0; qh < Hq; ++qh) {
+        const double* sv = s + ((size_t)b * Hq + qh) * n_tok;
+        double mx = sv[0];
+        for (int n = 1; n < n_tok; ++n) mx = sv[n] > mx ? sv[n] : mx;
+        double den = 0.0;
+        for (int n = 0; n < n_tok; ++n) den += exp(sv[n] - mx);
+        double* o = out + ((size_t)b * Hq + qh) * D;
+        for (int j = 0; j < D; ++j) o[j] = 0.0;
+        int h = qh / (Hq / H);
+        for (int n = 0; n < n_tok; ++n) {
+          double p = exp(sv[n] - mx) / den;
+          const double* v = vh + (((size_t)b * H + h) * t_cap + n) * D;
+          for (int j = 0; j < D; ++j) o[j] += p * v[j];
+        }
+      }
+  }
+  free(tok);
+  free(s);
+  free(vh);
+  return rc;
+}
+
+/* ------------------------------------------------------------------------
  * Channel permutation by abs-max ([RotateKV] outlier-aware rotation:
  * channel reordering before the FWHT). For each head, a_j = max over
  * batches and non-sink tokens of |y_j|, y = the fp32 input to the

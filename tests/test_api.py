@@ -104,6 +104,25 @@ def test_score_argument_checks():
     assert K.kvq_score(d, 256, 8, p, tb, 0, 1.0, 256, 0) == K.KVQ_OK  # empty: nothing to do
 
 
+def test_attend_argument_checks():
+    dk = _desc(t_cap=32, tokens=0, rope=1)
+    dv = _desc(t_cap=32, tokens=0, rope=0)
+    tb = K.kvq_tables()
+    p = _packed(dk)
+    ws = K.kvq_attend_workspace_bytes(dk, dv, 16, 20)
+    assert ws > 0
+    assert K.kvq_attend_workspace_bytes(dk, dv, 12, 20) == 0  # 12 % 8
+    assert K.kvq_attend_workspace_bytes(dk, dv, 8 * 16, 20) == 0  # 16 query heads per KV head
+    assert K.kvq_attend(dk, dv, 256, 16, p, tb, p, tb, 33, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_INVALID  # > t_cap
+    assert K.kvq_attend(dk, dv, 256, 16, p, tb, p, tb, 0, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_INVALID  # no token
+    assert K.kvq_attend(dk, dv, 256, 16, p, tb, p, tb, 20, 1.0, 256, 256, ws - 1, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_attend(dk, dv, 256, 16, p, tb, p, tb, 20, 1.0, 256, 512 + 16, ws, 0) == K.KVQ_ERR_ALIGN
+    dvr = _desc(t_cap=32, tokens=0, rope=1)
+    assert K.kvq_attend(dk, dvr, 256, 16, p, tb, p, tb, 20, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_UNSUPPORTED
+    dv4 = _desc(t_cap=32, tokens=0, rope=0, bits=4)
+    assert K.kvq_attend(dk, dv4, 256, 16, p, tb, p, tb, 20, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_INVALID
+
+
 def test_empty_call_is_a_noop():
     d = _desc(tokens=0, t_cap=4)
     assert K.kvq_encode(d, 256, K.kvq_tables(), _packed(d), 0) == K.KVQ_OK

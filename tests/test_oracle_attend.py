@@ -1,0 +1,65 @@
+"""Pins of the oracle's decode-step attention ("EliteKV - RoPE频率选择与低秩投影"
+§2.2 scores, §7.1 softmax-weighted values) by closed forms that do not
+repeat its arithmetic: one cached token gives that token's value exactly; a
+zero scale gives the plain mean of the values; every output lies in the
+values' convex hull; a large scale selects the value of the top-scoring key."""
+import numpy as np
+import pytest
+
+import workloads as W
+
+B, H, HQ, T, D = 2, 2, 8, 24, 128
+
+
+@pytest.fixture(scope="module")
+def caches(orc):
+    w = W.Workload("attn_pin", B=B, H=H, Hq=HQ, T=T, D=D, bits=2, group=64, n_sink=3, perm=True)
+    k = W.kv_tensor(w, "k").view(np.uint16)
+    v = W.kv_tensor(w, "v").view(np.uint16)
+    pos = np.arange(T)
+    kp, vp = W.random_perm(H, D, 3), W.random_perm(H, D, 4)
+    common = dict(rot=orc.ROT_FWHT_HEAD, bits=2, group=64, n_sink=3)
+    kc = orc.encode(k, pos, rope=1, perm=kp, **common)
+    vc = orc.encode(v, pos, rope=0, perm=vp, **common)
+    vhat = orc.decode(vc, pos, (B, H, T, D), rope=0, perm=vp, **common)
+    q = W.queries(w).view(np.uint16)
+    return dict(kc=kc, vc=vc, vhat=vhat, q=q, kp=kp, vp=vp, common=common)
+
+
+def _attend(orc, c, n_tok, scale):
+    return orc.attend(c["q"], c["kc"], c["vc"], n_tok, H=H, t_cap=T, scale=scale, kperm=c["kp"], vperm=c["vp"],
+                      **c["common"])
+
+
+def test_single_token_is_its_value(orc, caches):
+    out = _attend(orc, caches, 1, 0.3)
+    for qh in range(HQ):
+        assert np.array_equal(out[:, qh], caches["vhat"][:, qh // (HQ // H), 0])
+
+
+def test_zero_scale_is_the_mean(orc, caches):
+    out = _attend(orc, caches, T, 0.0)
+    mean = caches["vhat"].mean(axis=2)
+    for qh in range(HQ):
+        np.testing.assert_allclose(out[:, qh], mean[:, qh // (HQ // H)], rtol=0, atol=1e-12)
+
+
+def test_inside_convex_hull(orc, caches):
+    out = _attend(orc, caches, T, 1.0 / np.sqrt(D))
+    v = caches["vhat"]
+    for qh in range(HQ):
+        h = qh // (HQ // H)
+        assert np.all(out[:, qh] <= v[:, h].max(axis=1) + 1e-12)
+        assert np.all(out[:, qh] >= v[:, h].min(axis=1) - 1e-12)
+
+
+def test_large_scale_selects_the_top_key(orc, caches):
+    s = orc.score(caches["q"], caches["kc"], np.arange(T), H=H, t_cap=T, scale=1.0, rope=1, perm=caches["kp"],
+                  **caches["common"])
+    out = _attend(orc, caches, T, 1e4)
+    for b in range(B):
+        for qh in range(HQ):
+            top = int(np.argmax(s[b, qh]))
+            gap = np.sort(s[b, qh])[-1] - np.sort(s[b, qh])[-2]
+            assert gap * 1e4 > 50  # the runner-up's weight is below e^-50
+            np.testing.assert_allclose(out[b, qh], caches["vhat"][b, qh // (HQ // H), top], rtol=0, atol=1e-9)

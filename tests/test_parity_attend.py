@@ -1,0 +1,101 @@
+"""GPU parity of the decode-step attention (kvq_attend: "EliteKV -
+RoPE频率选择与低秩投影" §2.2 scores, §7.1 softmax-weighted values). K and V
+caches are written by the GPU encoder; the oracle reads those same caches.
+
+Two checks per case:
+  * tight: given the scores the GPU computes (kvq_score, same inputs), the
+    softmax, the value accumulation in the rotated basis, the inverse rotation
+    and the sink rows must match fp64 within 2e-5 * max|vhat| (fp32
+    accumulation over at most a few thousand tokens);
+  * end to end, against the oracle's scores: softmax weights move by at most
+    a factor e^(2 * max|ds|), so |out - out_orc| <= (e^(2*ds_max) - 1) * max|vhat|
+    + the tight bound, with ds_max the score contract's bound
+    1e-3 * scale * sum_j |q_j khat_j|."""
+import math
+
+import numpy as np
+import pytest
+
+import workloads as W
+from parity import SCORE_REL
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # name, B, H, Hq, t_cap, n_tok, bits, group, n_sink, perm, rot
+    ("gqa4_bits2_g128_sinks", 2, 2, 8, 300, 300, 2, 128, 4, False, "fwht_head"),
+    ("mha_perm_g64_ragged", 1, 4, 4, 260, 257, 2, 64, 4, True, "fwht_head"),
+    ("gqa2_bits3_g32", 1, 2, 4, 140, 130, 3, 32, 0, True, "fwht_head"),
+    ("gqa8_bits4", 1, 1, 8, 129, 129, 4, 64, 2, False, "fwht_head"),
+    ("no_rotation", 1, 2, 2, 64, 64, 2, 64, 2, True, "none"),
+    ("single_token", 2, 2, 8, 16, 1, 2, 128, 0, False, "fwht_head"),
+    ("sinks_only", 1, 2, 4, 16, 3, 2, 64, 4, True, "fwht_head"),
+]
+
+
+@pytest.fixture(scope="module")
+def K():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import kv_cache_rotation_b200 as K
+    return K
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_attend_parity(K, orc, case):
+    from kv_cache_rotation_b200 import torch_api as TA
+    name, B, H, Hq, t_cap, n_tok, bits, group, n_sink, use_perm, rot = case
+    D = 128
+    w = W.Workload(name, B=B, H=H, Hq=Hq, T=t_cap, D=D, bits=bits, group=group, n_sink=n_sink,
+                   outliers=("pairs", 0.02, 10.0, 50.0))
+    k, v, q = W.kv_tensor(w, "k"), W.kv_tensor(w, "v"), W.queries(w)
+    kp = W.random_perm(H, D, 5) if use_perm else None
+    vp = W.random_perm(H, D, 6) if use_perm else None
+    common = dict(batch=B, heads=H, head_dim=D, tokens=t_cap, t_cap=t_cap, bits=bits, group=group,
+                  n_sink=n_sink, rot=rot)
+    dk, dv = TA.make_desc(rope=1, **common), TA.make_desc(rope=0, **common)
+    tk = TA.make_tables(perm=torch.from_numpy(kp).cuda() if use_perm else None, rope_cs=TA.rope_table(t_cap, D))
+    tv = TA.make_tables(perm=torch.from_numpy(vp).cuda() if use_perm else None)
+    pk, pv = TA.alloc_packed(dk), TA.alloc_packed(dv)
+    TA.encode(dk, torch.from_numpy(k).cuda(), tk, pk)
+    TA.encode(dv, torch.from_numpy(v).cuda(), tv, pv)
+    scale = 1.0 / math.sqrt(D)
+    qg = torch.from_numpy(q).cuda()
+    out = torch.full((B, Hq, D), float("nan"), dtype=torch.float32, device="cuda")
+    ws = TA.attend_workspace(dk, dv, Hq, n_tok)
+    TA.attend(dk, dv, qg, pk, tk, pv, tv, n_tok, scale, out, ws)
+    s_gpu = torch.empty((B, Hq, n_tok), dtype=torch.float32, device="cuda")
+    TA.score(dk, qg, pk, tk, n_tok, scale, s_gpu)
+    assert K.kvq_check(0) == K.KVQ_OK
+    got, s_gpu = out.cpu().numpy().astype(np.float64), s_gpu.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+
+    rotv = {"none": 0, "fwht_head": 1}[rot]
+    okw = dict(rot=rotv, bits=bits, group=group, n_sink=n_sink)
+    kc = {"codes": pk.codes.cpu().numpy(), "sz": pk.scale_zero.cpu().numpy().view(np.uint16),
+          "sink": pk.sink.cpu().numpy().view(np.uint16) if n_sink else None}
+    vc = {"codes": pv.codes.cpu().numpy(), "sz": pv.scale_zero.cpu().numpy().view(np.uint16),
+          "sink": pv.sink.cpu().numpy().view(np.uint16) if n_sink else None}
+    pos = np.arange(t_cap)
+    vhat = orc.decode(vc, pos, (B, H, t_cap, D), rope=0, perm=vp, **okw)[:, :, :n_tok]
+    khat = orc.decode(kc, pos, (B, H, t_cap, D), rope=1, perm=kp, **okw)
+    ref = orc.attend(q.view(np.uint16), kc, vc, n_tok, H=H, t_cap=t_cap, scale=scale, kperm=kp, vperm=vp,
+                     krope=1, vrope=0, **okw)
+    gq = Hq // H
+    for b in range(B):
+        for qh in range(Hq):
+            h = qh // gq
+            vmax = np.abs(vhat[b, h]).max()
+            # tight: the GPU's own scores through fp64 softmax and values
+            sv = s_gpu[b, qh]
+            p = np.exp(sv - sv.max())
+            p /= p.sum()
+            want = p @ vhat[b, h]
+            tight = 2e-5 * vmax
+            assert np.all(np.abs(got[b, qh] - want) <= tight), (b, qh, np.abs(got[b, qh] - want).max() / vmax)
+            # end to end against the oracle
+            kk = np.stack([orc.rope_f64(khat[b, h, n], n) for n in range(n_tok)])
+            ds = SCORE_REL * scale * (np.abs(kk) @ np.abs(q[b, qh].astype(np.float64)))
+            bound = (math.exp(2 * ds.max()) - 1) * vmax + tight
+            assert np.all(np.abs(got[b, qh] - ref[b, qh]) <= bound), (b, qh, np.abs(got[b, qh] - ref[b, qh]).max())
