@@ -188,9 +188,10 @@ class Step:
 
 class ScoreCache:
     """A prefilled head-variant cache (untimed) plus the decode-step launches:
-    append one token per sequence, then score every cached slot."""
+    append one token per sequence, then score every cached slot. `which` =
+    "v" builds the value cache of the same shape (no RoPE)."""
 
-    def __init__(self, ws, device):
+    def __init__(self, ws, device, which="k"):
         import torch
         from kv_cache_rotation_b200 import torch_api as TA
         self.TA = TA
@@ -198,17 +199,19 @@ class ScoreCache:
         Ts = ws.T
         self.n_tok = Ts + ws.append
         cap = self.n_tok
-        common = dict(batch=ws.B, heads=ws.H, head_dim=D, t_cap=cap, bits=ws.bits, group=ws.group, rope=1,
+        rope = 1 if which == "k" else 0
+        common = dict(batch=ws.B, heads=ws.H, head_dim=D, t_cap=cap, bits=ws.bits, group=ws.group, rope=rope,
                       n_sink=ws.n_sink, rot="fwht_head")
         self.d_pre = TA.make_desc(tokens=Ts, t0=0, **common)
         self.d_app = TA.make_desc(tokens=ws.append, t0=Ts, **common)
-        perm = torch.from_numpy(W.random_perm(ws.H, D, ws.seed)).to(device) if ws.perm else None
-        self.tables = TA.make_tables(perm=perm, rope_cs=TA.rope_table(cap, D, device=device))
+        perm = (torch.from_numpy(W.random_perm(ws.H, D, ws.seed + (which == "v"))).to(device) if ws.perm
+                else None)
+        self.tables = TA.make_tables(perm=perm, rope_cs=TA.rope_table(cap, D, device=device) if rope else None)
         self.packed = TA.alloc_packed(self.d_pre, device)
-        ks = torch.from_numpy(W.kv_tensor(ws, "k")).to(device)
+        ks = torch.from_numpy(W.kv_tensor(ws, which)).to(device)
         TA.encode(self.d_pre, ks, self.tables, self.packed)
         del ks
-        self.app_host = W.kv_tensor(ws, "k_append", T=ws.append)
+        self.app_host = W.kv_tensor(ws, which + "_append", T=ws.append)
         self.app = torch.from_numpy(self.app_host).to(device)
         self.q_host = W.queries(ws)
         self.q = torch.from_numpy(self.q_host).to(device)
@@ -222,6 +225,38 @@ class ScoreCache:
         self.fp16_score = ws.B * ws.H * self.n_tok * 2 * D
         self.append = TA.bind_encode(self.d_app, self.app, self.tables, self.packed)
         self.score = TA.bind_score(self.d_pre, self.q, self.packed, self.tables, self.n_tok, self.scale, self.scores)
+        self.alg_cache = (ws.B * ws.H * (self.n_tok - ws.n_sink) * (rb + 4 * ng) + ws.B * ws.H * ws.n_sink * D * 2)
+
+
+class AttendStep:
+    """Decode-step attention at the Llama-3-8B shape: append one token to the
+    K and the V cache, then out = softmax(q . k) . v over every slot."""
+
+    workload = "llama3_8b_gqa_attend"
+
+    def __init__(self, device):
+        import torch
+        from kv_cache_rotation_b200 import torch_api as TA
+        ws = W.WORKLOADS[self.workload]
+        self.k = ScoreCache(ws, device, "k")
+        self.v = ScoreCache(ws, device, "v")
+        n = self.k.n_tok
+        self.out = torch.empty((ws.B, ws.Hq, ws.D), dtype=torch.float32, device=device)
+        self.ws = TA.attend_workspace(self.k.d_pre, self.v.d_pre, ws.Hq, n, device=device)
+        self.attend = TA.bind_attend(self.k.d_pre, self.v.d_pre, self.k.q, self.k.packed, self.k.tables,
+                                     self.v.packed, self.v.tables, n, self.k.scale, self.out, self.ws)
+        q_out = ws.B * ws.Hq * ws.D * (2 + 4)
+        self.alg = {"append_k": self.k.alg_append, "append_v": self.v.alg_append,
+                    "attend": self.k.alg_cache + self.v.alg_cache + q_out}
+        self.fp16_equiv = {"append_k": self.k.fp16_append, "append_v": self.v.fp16_append,
+                           "attend": 2 * self.k.fp16_score}
+        self.kernels = {"append_k": "k_encode_head", "append_v": "k_encode_head", "attend": "k_attend_part"}
+        self.fp32_ops = {}
+        self.names = list(self.alg)
+        torch.cuda.synchronize(device)
+
+    def launches(self):
+        return [self.k.append, self.v.append, self.attend]
 
 
 class EncDecStep:
@@ -320,6 +355,8 @@ def make_step(workload, device, batch=None):
         return Step(device)
     if workload == "decode_score":
         return DecodeScoreStep(device)
+    if workload == "llama3_8b_gqa_attend":
+        return AttendStep(device)
     return EncDecStep(workload, device, batch=batch)
 
 
@@ -572,7 +609,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=512, help="tokens per reference-arm step")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--workload", default="llama3_8b_gqa",
-                    choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "decode_score", "tiny"],
+                    choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "decode_score",
+                             "llama3_8b_gqa_attend", "tiny"],
                     help="which workload a step runs (the headline line is llama3_8b_gqa)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch of an encode/decode workload (small profiling captures)")

@@ -8,12 +8,14 @@
 // the inverse rotation runs once per output instead of once per token.
 //
 // Three launches on the caller's stream: the scores (kvq_score's kernel) into
-// the workspace; k_attend_part, one CTA per (chunk of 128 tokens, batch, KV
-// head), writes the chunk's softmax statistics (max m, sum l) and
-// sum_n e^(s_n - m) y_n per query head of the group; k_attend_combine, one CTA
+// the workspace; k_attend_part, one CTA per (chunk of 1024 tokens, batch, KV
+// head), walks the chunk in sub-chunks of 128 with a running (online) softmax
+// and writes the chunk's statistics (max m, sum l) and sum_n e^(s_n - m) y_n
+// per query head of the group; k_attend_combine, one CTA
 // per (batch, query head), merges the chunks (log-sum-exp), applies the
 // inverse rotation and permutation and adds the sink rows.
 #include <math.h>
+
 
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -22,7 +24,8 @@ namespace kvq {
 namespace {
 
 constexpr int D = 128;
-constexpr int kCh = 128;       // tokens per chunk
+constexpr int kCh = 128;       // tokens per sub-chunk (one per thread in the score pass)
+constexpr int kSub = 8;        // sub-chunks per chunk: a chunk is 1024 tokens
 constexpr int kThreads = 128;  // part: one token each, then 32 channel quads x 4 token phases;
                                // combine: one thread per channel
 
@@ -55,111 +58,104 @@ __global__ void __launch_bounds__(kThreads) k_attend_part(const AttnArgs a) {
   constexpr int NG = D / G;
   constexpr int RB = D * BITS / 8;
   constexpr uint32_t MASK = (1u << BITS) - 1u;
-  constexpr int TPT = kCh / kThreads;  // tokens per thread in the score pass
-  __shared__ __align__(16) float wsm[kCh][NG][GQ];  // p_n * S_ng
+  __shared__ __align__(16) float wsm[kCh][NG][GQ];  // p_n * S_ng of the sub-chunk
   __shared__ __align__(16) uint32_t csm[kCh][RB / 4];
   __shared__ float red[4][GQ * (1 + NG)];
   __shared__ float mx_s[4][GQ];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int n0 = c * kCh, nn = min(kCh, a.n_tok - n0);
-
-  // the chunk's packed value records (zero past the last token)
-  const uint4* vsrc = reinterpret_cast<const uint4*>(a.vcodes + (static_cast<size_t>(bh) * a.t_cap + n0) * RB);
-  for (int i = tid; i < kCh * RB / 16; i += kThreads) {
-    const int n = i / (RB / 16);
-    const uint4 v = n < nn ? __ldg(vsrc + i) : make_uint4(0, 0, 0, 0);
-    reinterpret_cast<uint4*>(&csm[0][0])[i] = v;
-  }
-
-  // scores of the chunk, per query head of this KV head
-  float s[GQ][TPT];
-#pragma unroll
-  for (int r = 0; r < GQ; ++r) {
-    const float* sp = a.scores + (static_cast<size_t>(b) * a.Hq + h * GQ + r) * a.n_tok + n0;
-#pragma unroll
-    for (int i = 0; i < TPT; ++i) {
-      const int n = tid + i * kThreads;
-      s[r][i] = n < nn ? __ldg(sp + n) : -INFINITY;
-    }
-  }
-  float m[GQ];
-#pragma unroll
-  for (int r = 0; r < GQ; ++r) {
-    float v = s[r][0];
-#pragma unroll
-    for (int i = 1; i < TPT; ++i) v = fmaxf(v, s[r][i]);
-    v = warp_max(v);
-    if (lane == 0) mx_s[warp][r] = v;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < GQ; ++r) m[r] = fmaxf(fmaxf(mx_s[0][r], mx_s[1][r]), fmaxf(mx_s[2][r], mx_s[3][r]));
-
-  // p_n = e^(s_n - m); w_n = p_n * S_g, and the chunk sums of p_n and p_n * Z_g
-  float lsum[GQ], zsum[GQ][NG];
-#pragma unroll
-  for (int r = 0; r < GQ; ++r) {
-    lsum[r] = 0.0f;
-#pragma unroll
-    for (int g = 0; g < NG; ++g) zsum[r][g] = 0.0f;
-  }
-#pragma unroll
-  for (int i = 0; i < TPT; ++i) {
-    const int n = tid + i * kThreads;
-    float2 sz[NG];
-#pragma unroll
-    for (int g = 0; g < NG; ++g)
-      sz[g] = n < nn ? __half22float2(a.vsz[(static_cast<size_t>(bh) * a.t_cap + n0 + n) * NG + g])
-                     : make_float2(0.0f, 0.0f);
-#pragma unroll
-    for (int r = 0; r < GQ; ++r) {
-      const float p = n < nn ? __expf(s[r][i] - m[r]) : 0.0f;
-      lsum[r] += p;
-#pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        wsm[n][g][r] = p * sz[g].x;
-        zsum[r][g] = fmaf(p, sz[g].y, zsum[r][g]);
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < GQ; ++r) {
-    const float l = warp_sum(lsum[r]);
-    if (lane == 0) red[warp][r] = l;
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      const float z = warp_sum(zsum[r][g]);
-      if (lane == 0) red[warp][GQ + r * NG + g] = z;
-    }
-  }
-  __syncthreads();
-
-  // sum_n w_n c_n per channel: thread (quad, phase) takes channels 4q..4q+3 of tokens n = phase mod 4
+  // accumulation role: thread (quad, phase) takes channels 4q..4q+3 of tokens n = phase mod 4
   const int q = tid >> 2, ph = tid & 3;
   const int g = (4 * q) / G;
-  float acc[GQ][4];
+  const int bit = 4 * q * BITS, wi = bit >> 5, sh = bit & 31;
+
+  // running (online-softmax) state over the chunk's sub-chunks
+  float m_run[GQ], l_run[GQ], z_run[GQ], acc[GQ][4];
 #pragma unroll
-  for (int r = 0; r < GQ; ++r)
+  for (int r = 0; r < GQ; ++r) {
+    m_run[r] = -INFINITY;
+    l_run[r] = 0.0f;
+    z_run[r] = 0.0f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[r][e] = 0.0f;
-  const int bit = 4 * q * BITS, wi = bit >> 5, sh = bit & 31;
-  for (int n = ph; n < nn; n += 4) {
-    uint32_t v = csm[n][wi] >> sh;
-    if constexpr ((4 * BITS) % 8 != 0 || 32 % (4 * BITS) != 0) {
-      if (sh + 4 * BITS > 32) v |= csm[n][wi + 1] << (32 - sh);
+  }
+
+  for (int sub = 0; sub < kSub; ++sub) {
+    const int n0 = (c * kSub + sub) * kCh;
+    if (n0 >= a.n_tok) break;  // uniform over the CTA
+    const int nn = min(kCh, a.n_tok - n0);
+    __syncthreads();  // the previous sub-chunk's csm / wsm / red readers are done
+
+    // packed value records (zero past the last token)
+    const uint4* vsrc = reinterpret_cast<const uint4*>(a.vcodes + (static_cast<size_t>(bh) * a.t_cap + n0) * RB);
+    for (int i = tid; i < kCh * RB / 16; i += kThreads) {
+      const int n = i / (RB / 16);
+      reinterpret_cast<uint4*>(&csm[0][0])[i] = n < nn ? __ldg(vsrc + i) : make_uint4(0, 0, 0, 0);
     }
-    float cf[4];
+    // scores (thread = token), the sub-chunk max per query head
+    float sv[GQ];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) cf[e] = __uint_as_float(0x4B000000u | ((v >> (BITS * e)) & MASK)) - 8388608.0f;
-    float w[GQ];
+    for (int r = 0; r < GQ; ++r) {
+      const float* sp = a.scores + (static_cast<size_t>(b) * a.Hq + h * GQ + r) * a.n_tok + n0;
+      sv[r] = tid < nn ? __ldg(sp + tid) : -INFINITY;
+      const float v = warp_max(sv[r]);
+      if (lane == 0) mx_s[warp][r] = v;
+    }
+    __syncthreads();
+    float m_new[GQ], f_old[GQ];
 #pragma unroll
-    for (int r = 0; r < GQ; ++r) w[r] = wsm[n][g][r];
+    for (int r = 0; r < GQ; ++r) {
+      m_new[r] = fmaxf(m_run[r], fmaxf(fmaxf(mx_s[0][r], mx_s[1][r]), fmaxf(mx_s[2][r], mx_s[3][r])));
+      f_old[r] = __expf(m_run[r] - m_new[r]);  // 0 on the first sub-chunk
+    }
+    // p_n = e^(s_n - m); w_n = p_n S_g; sub-chunk sums of p_n and p_n Z_g
+    {
+      float2 sz[NG];
 #pragma unroll
-    for (int r = 0; r < GQ; ++r)
+      for (int gg = 0; gg < NG; ++gg)
+        sz[gg] = tid < nn ? __half22float2(a.vsz[(static_cast<size_t>(bh) * a.t_cap + n0 + tid) * NG + gg])
+                          : make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(w[r], cf[e], acc[r][e]);
+      for (int r = 0; r < GQ; ++r) {
+        const float p = tid < nn ? __expf(sv[r] - m_new[r]) : 0.0f;
+        const float l = warp_sum(p);
+        if (lane == 0) red[warp][r] = l;
+#pragma unroll
+        for (int gg = 0; gg < NG; ++gg) {
+          wsm[tid][gg][r] = p * sz[gg].x;
+          const float z = warp_sum(p * sz[gg].y);
+          if (lane == 0) red[warp][GQ + r * NG + gg] = z;
+        }
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < GQ; ++r) {
+      const int zi = GQ + r * NG + g;
+      l_run[r] = fmaf(l_run[r], f_old[r], red[0][r] + red[1][r] + red[2][r] + red[3][r]);
+      z_run[r] = fmaf(z_run[r], f_old[r], red[0][zi] + red[1][zi] + red[2][zi] + red[3][zi]);
+      m_run[r] = m_new[r];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[r][e] *= f_old[r];
+    }
+    // sum_n w_n c_n for this thread's channels and token phase
+    for (int n = ph; n < nn; n += 4) {
+      uint32_t v = csm[n][wi] >> sh;
+      if constexpr ((4 * BITS) % 8 != 0 || 32 % (4 * BITS) != 0) {
+        if (sh + 4 * BITS > 32) v |= csm[n][wi + 1] << (32 - sh);
+      }
+      float cf[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cf[e] = __uint_as_float(0x4B000000u | ((v >> (BITS * e)) & MASK)) - 8388608.0f;
+      float w[GQ];
+#pragma unroll
+      for (int r = 0; r < GQ; ++r) w[r] = wsm[n][g][r];
+#pragma unroll
+      for (int r = 0; r < GQ; ++r)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[r][e] = fmaf(w[r], cf[e], acc[r][e]);
+    }
   }
   // the four token phases of a quad sit in adjacent lanes
 #pragma unroll
@@ -169,21 +165,17 @@ __global__ void __launch_bounds__(kThreads) k_attend_part(const AttnArgs a) {
       acc[r][e] += __shfl_xor_sync(0xffffffffu, acc[r][e], 1);
       acc[r][e] += __shfl_xor_sync(0xffffffffu, acc[r][e], 2);
     }
-
   // add sum_n p_n Z_g; write the chunk's partials
   const size_t pc = static_cast<size_t>(a.n_chunks);
 #pragma unroll
   for (int r = 0; r < GQ; ++r) {
     const size_t row = (static_cast<size_t>(b) * a.Hq + h * GQ + r) * pc + c;
-    if (ph == 0) {
-      const int zi = GQ + r * NG + g;
-      const float z = red[0][zi] + red[1][zi] + red[2][zi] + red[3][zi];
+    if (ph == 0)
       *reinterpret_cast<float4*>(a.part_acc + row * D + 4 * q) =
-          make_float4(acc[r][0] + z, acc[r][1] + z, acc[r][2] + z, acc[r][3] + z);
-    }
+          make_float4(acc[r][0] + z_run[r], acc[r][1] + z_run[r], acc[r][2] + z_run[r], acc[r][3] + z_run[r]);
     if (tid == 0) {
-      a.part_ml[row * 2] = m[r];
-      a.part_ml[row * 2 + 1] = red[0][r] + red[1][r] + red[2][r] + red[3][r];
+      a.part_ml[row * 2] = m_run[r];
+      a.part_ml[row * 2 + 1] = l_run[r];
     }
   }
 }
@@ -262,7 +254,7 @@ size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
 size_t attend_workspace_bytes(int B, int q_heads, int n_tokens) {
   const size_t bq = static_cast<size_t>(B) * q_heads;
-  const size_t n_chunks = (static_cast<size_t>(n_tokens) + kCh - 1) / kCh;
+  const size_t n_chunks = (static_cast<size_t>(n_tokens) + kCh * kSub - 1) / (kCh * kSub);
   return align256(bq * n_tokens * 4) + align256(bq * n_chunks * D * 4) + align256(bq * n_chunks * 2 * 4);
 }
 
@@ -277,7 +269,7 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
   a.GQ = q_heads / dk.heads;
   a.t_cap = dk.t_cap;
   a.n_tok = n_tokens;
-  a.n_chunks = (n_tokens + kCh - 1) / kCh;
+  a.n_chunks = (n_tokens + kCh * kSub - 1) / (kCh * kSub);
   a.n_sink = dv.n_sink;
   a.rot = dv.rot;
   a.rscale = static_cast<float>(1.0 / sqrt(static_cast<double>(D)));

@@ -77,6 +77,10 @@ WORKLOADS = {
     # 4:1), 32768 cached tokens + 1 appended, head-dim FWHT, 2-bit group 128.
     "llama3_8b_gqa_score": Workload("llama3_8b_gqa_score", B=4, H=8, T=32768, bits=2, group=128, n_sink=4,
                                     seed=6, Hq=32, append=1),
+    # Decode-step attention at the same shape: K and V caches (values without
+    # RoPE), one token appended to each, then softmax(q . k) . v.
+    "llama3_8b_gqa_attend": Workload("llama3_8b_gqa_attend", B=4, H=8, T=32768, bits=2, group=128, n_sink=4,
+                                     seed=7, Hq=32, append=1),
 }
 
 
