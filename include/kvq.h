@@ -166,6 +166,23 @@ kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int
                       const kvq_tables* tv, int32_t n_tokens, float scale, float* out, void* workspace,
                       size_t workspace_bytes, kvq_stream_t stream);
 
+/* kvq_attend without a workspace argument, for callers that cannot allocate device memory
+ * when they call (a fixed-budget serving loop, host code without a device allocator, a caller
+ * whose workspace would have to stay put between repeated launches of the same work). The
+ * pages have no counterpart: it is a variant of kvq_attend with the same arguments and
+ * results, whose scores and chunk partials live in a fixed 40 MiB device array of the library
+ * (enough for 4 sequences x 32 query heads x 32769 cached tokens); it allocates nothing.
+ * Returns KVQ_ERR_UNSUPPORTED when kvq_attend_workspace_bytes() exceeds 40 MiB. The array's
+ * device address is looked up on the first call made with each device current: make that
+ * first call outside any stream capture. The array is shared by every call on a device: two
+ * calls that can run at the same time (different streams, or host threads without ordering)
+ * race on it and corrupt each other's results; calls in order on one stream are safe. Nothing
+ * in it needs to start at zero. */
+kvq_status kvq_attend_noalloc(const kvq_desc* dk, const kvq_desc* dv, const void* q, int32_t q_heads,
+                              const kvq_packed* k_cache, const kvq_tables* tk, const kvq_packed* v_cache,
+                              const kvq_tables* tv, int32_t n_tokens, float scale, float* out,
+                              kvq_stream_t stream);
+
 /* Workspace bytes kvq_attend needs for these arguments; 0 if they are invalid or unsupported. */
 size_t kvq_attend_workspace_bytes(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads, int32_t n_tokens);
 

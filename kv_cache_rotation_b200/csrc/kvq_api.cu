@@ -299,6 +299,27 @@ kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int
                        reinterpret_cast<cudaStream_t>(stream), ctx);
 }
 
+kvq_status kvq_attend_noalloc(const kvq_desc* dk, const kvq_desc* dv, const void* q, int32_t q_heads,
+                              const kvq_packed* k_cache, const kvq_tables* tk, const kvq_packed* v_cache,
+                              const kvq_tables* tv, int32_t n_tokens, float scale, float* out,
+                              kvq_stream_t stream) {
+  kvq_desc k, v;
+  kvq_status s = check_attend(dk, dv, q_heads, n_tokens, &k, &v);
+  if (s != KVQ_OK) return s;
+  if (!q || !out) return KVQ_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_ALIGN;
+  if (attend_workspace_bytes(k.batch, q_heads, n_tokens) > attend_scratch_bytes()) return KVQ_ERR_UNSUPPORTED;
+  if ((s = check_tables(&k, tk, k.rope ? (n_tokens < k.n_sink ? n_tokens : k.n_sink) : 0)) != KVQ_OK) return s;
+  if ((s = check_tables(&v, tv, 0)) != KVQ_OK) return s;
+  if ((s = check_packed(&k, k_cache)) != KVQ_OK || (s = check_packed(&v, v_cache)) != KVQ_OK) return s;
+  LaunchCtx ctx;
+  if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
+  void* ws = attend_scratch();
+  if (!ws) return KVQ_ERR_CUDA;
+  return launch_attend(k, v, q, q_heads, *k_cache, *tk, *v_cache, *tv, n_tokens, scale, out, ws,
+                       reinterpret_cast<cudaStream_t>(stream), ctx);
+}
+
 size_t kvq_packed_bytes(const kvq_desc* d, int32_t field) {
   if (!d) return 0;
   kvq_desc dd = *d;

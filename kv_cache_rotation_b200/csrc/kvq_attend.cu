@@ -16,6 +16,7 @@
 // inverse rotation and permutation and adds the sink rows.
 #include <math.h>
 
+#include <mutex>
 
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -250,7 +251,35 @@ kvq_status dispatch_part(int bits, int group, const AttnArgs& a, cudaStream_t st
 
 size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
+// Fixed scratch of kvq_attend_noalloc: a file-scope device array, reserved when
+// the module is loaded, so that entry point never allocates. 40 MiB holds the
+// scores and chunk partials of about 9 M (query head x cached token) pairs
+// (4 bytes of score + 0.5 byte of chunk partials each), e.g. 4 sequences x 32
+// query heads x 32769 tokens (19 MB). Nothing in it has
+// to start at zero: every byte a call reads was written earlier in that call.
+constexpr size_t kAttendScratchBytes = size_t{40} << 20;
+__device__ __align__(256) uint8_t g_attend_scratch[kAttendScratchBytes];
+
 }  // namespace
+
+size_t attend_scratch_bytes() { return kAttendScratchBytes; }
+
+// Device address of the fixed scratch on the current device, looked up once
+// per device (with that device current) and cached; nullptr on a CUDA error.
+void* attend_scratch() {
+  constexpr int kDevices = 64;
+  static std::mutex mu;
+  static void* ptr[kDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_attend_scratch) != cudaSuccess) return nullptr;
+    ptr[dev] = p;
+  }
+  return ptr[dev];
+}
 
 size_t attend_workspace_bytes(int B, int q_heads, int n_tokens) {
   const size_t bq = static_cast<size_t>(B) * q_heads;

@@ -45,6 +45,8 @@ kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq
                         const LaunchCtx& ctx);
 kvq_status launch_debug_wait(uint64_t limit_ns, cudaStream_t st, const LaunchCtx& ctx);
 size_t attend_workspace_bytes(int B, int q_heads, int n_tokens);
+size_t attend_scratch_bytes();
+void* attend_scratch();
 kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, int q_heads,
                          const kvq_packed& kc, const kvq_tables& tk, const kvq_packed& vc, const kvq_tables& tv,
                          int n_tokens, float scale, float* out, void* ws, cudaStream_t st, const LaunchCtx& ctx);

@@ -150,6 +150,14 @@ def attend(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, tk: Ta
                      _stream(stream)), "kvq_attend")
 
 
+def attend_noalloc(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, tk: Tables, v_packed: Packed,
+                   tv: Tables, n_tokens: int, scale: float, out: torch.Tensor, stream=None) -> None:
+    """kvq_attend through the library's fixed scratch (no workspace tensor)."""
+    from . import kvq_attend_noalloc
+    check(kvq_attend_noalloc(dk, dv, q.data_ptr(), q.shape[1], k_packed.struct(), tk.struct(), v_packed.struct(),
+                             tv.struct(), n_tokens, scale, out.data_ptr(), _stream(stream)), "kvq_attend_noalloc")
+
+
 def bind_attend(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, tk: Tables, v_packed: Packed,
                 tv: Tables, n_tokens: int, scale: float, out: torch.Tensor, workspace: torch.Tensor, stream=None):
     from . import lib

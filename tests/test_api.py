@@ -123,6 +123,16 @@ def test_attend_argument_checks():
     assert K.kvq_attend(dk, dv4, 256, 16, p, tb, p, tb, 20, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_INVALID
 
 
+def test_attend_noalloc_rejects_oversize():
+    # 8 sequences x 64 query heads x 32768 tokens: 67 MB of scores alone, more than the 40 MiB scratch
+    dk = _desc(batch=8, heads=8, t_cap=32768, tokens=0, rope=0)
+    dv = _desc(batch=8, heads=8, t_cap=32768, tokens=0, rope=0)
+    assert K.kvq_attend_workspace_bytes(dk, dv, 64, 32768) > (40 << 20)
+    p, tb = _packed(dk), K.kvq_tables()
+    assert K.kvq_attend_noalloc(dk, dv, 256, 64, p, tb, p, tb, 32768, 1.0, 256, 0) == K.KVQ_ERR_UNSUPPORTED
+    assert K.kvq_attend_noalloc(dk, dv, 258, 64, p, tb, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_ALIGN
+
+
 def test_empty_call_is_a_noop():
     d = _desc(tokens=0, t_cap=4)
     assert K.kvq_encode(d, 256, K.kvq_tables(), _packed(d), 0) == K.KVQ_OK
