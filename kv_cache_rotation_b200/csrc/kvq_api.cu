@@ -277,7 +277,7 @@ kvq_status check_attend(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads,
 size_t kvq_attend_workspace_bytes(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads, int32_t n_tokens) {
   kvq_desc k, v;
   if (check_attend(dk, dv, q_heads, n_tokens, &k, &v) != KVQ_OK) return 0;
-  return attend_workspace_bytes(k.batch, q_heads, n_tokens);
+  return attend_workspace_bytes(k, q_heads, n_tokens);
 }
 
 kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int32_t q_heads,
@@ -289,7 +289,7 @@ kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int
   if (s != KVQ_OK) return s;
   if (!q || !out || !workspace) return KVQ_ERR_INVALID;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_ALIGN;
-  if (workspace_bytes < attend_workspace_bytes(k.batch, q_heads, n_tokens)) return KVQ_ERR_INVALID;
+  if (workspace_bytes < attend_workspace_bytes(k, q_heads, n_tokens)) return KVQ_ERR_INVALID;
   if ((s = check_tables(&k, tk, k.rope ? (n_tokens < k.n_sink ? n_tokens : k.n_sink) : 0)) != KVQ_OK) return s;
   if ((s = check_tables(&v, tv, 0)) != KVQ_OK) return s;
   if ((s = check_packed(&k, k_cache)) != KVQ_OK || (s = check_packed(&v, v_cache)) != KVQ_OK) return s;
@@ -308,7 +308,7 @@ kvq_status kvq_attend_noalloc(const kvq_desc* dk, const kvq_desc* dv, const void
   if (s != KVQ_OK) return s;
   if (!q || !out) return KVQ_ERR_INVALID;
   if (!aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_ALIGN;
-  if (attend_workspace_bytes(k.batch, q_heads, n_tokens) > attend_scratch_bytes()) return KVQ_ERR_UNSUPPORTED;
+  if (attend_workspace_bytes(k, q_heads, n_tokens) > attend_scratch_bytes()) return KVQ_ERR_UNSUPPORTED;
   if ((s = check_tables(&k, tk, k.rope ? (n_tokens < k.n_sink ? n_tokens : k.n_sink) : 0)) != KVQ_OK) return s;
   if ((s = check_tables(&v, tv, 0)) != KVQ_OK) return s;
   if ((s = check_packed(&k, k_cache)) != KVQ_OK || (s = check_packed(&v, v_cache)) != KVQ_OK) return s;

@@ -20,6 +20,7 @@
 
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
+#include "kvq_qdigits.cuh"
 
 namespace kvq {
 namespace {
@@ -251,6 +252,483 @@ kvq_status dispatch_part(int bits, int group, const AttnArgs& a, cudaStream_t st
 
 size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
+// ---------------------------------------------------------------------------
+// Fused path (head_dim 128, one quantization group per record, 2- or 4-bit
+// codes): one pass over the K and V records of a chunk of tokens forms the
+// scores, the running softmax statistics and sum_n p_n y_n, all products on
+// the tensor cores; a small merge kernel then combines the chunks.
+//
+// Scores: exactly the score kernel's arithmetic (u8 codes x s8 query digits,
+// mma.sync m16n8k32, same fp32 epilogue), so they match kvq_score bit for bit.
+//
+// Values: out_rot = sum_n p_n (S_n c_n + Z_n) = sum_n w_n c_n + sum_n p_n Z_n
+// with w_n = p_n S_n. sum_n w_n c_n runs on mma.sync m16n8k16 (fp16 in, fp32
+// accumulate) with A = codes (channels x tokens; small integers, exact in
+// fp16) and B = weights (tokens x columns). Each weight is carried as two fp16
+// terms w = hi + lo (hi = fp16(w), lo = fp16(w - hi)), one column each, so the
+// product keeps about 22 bits of w: with N = 8 columns a group of four query
+// heads fills one n-tile.
+//
+// Range: the running reference m tracks the largest key lambda_n = s_n log2(e)
+// + log2(S_n) (S_n clamped to >= 2^-30), and p'_n = 2^(s_n log2(e) - m), so
+// w'_n = p'_n S_n <= 2^8 (m is raised, and the sums rescaled, only when a key
+// exceeds it by more than 2^8); p'_n and every sum stay in fp32 range. The
+// partial of a chunk is (m, l = sum p'_n, sum_n p'_n y_n) in the log2 domain.
+//
+// A operand without a shift per m-tile: a lane's rows g and g + 8 of m-tile t
+// are two channels whose codes sit at the same bit offset in the low and high
+// 16-bit halves of one record word; the two tokens of a register are paired
+// with one byte permute per word pair, and the code is masked in place:
+// (y & (3 << 2t)) | 0x6400 is the fp16 1024 + c 4^t, minus 1024 exactly c 4^t
+// (kept below 1024 by taking t >= 5 from y >> 10). The 4^t is undone once on
+// the accumulators.
+constexpr int kFWarps = 8;
+constexpr int kFThreads = 32 * kFWarps;
+constexpr int kFTile = 16 * kFWarps;  // tokens per stage: one 16-token block per warp
+constexpr int kFStages = 4;
+constexpr int kFMaxChunks = 256;
+constexpr int kFMaxSinks = 1024;        // merge keeps the sink scores in shared memory
+constexpr float kFLazy = 8.0f;          // log2 headroom before the reference is raised
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kMinS = 9.3132257e-10f;  // 2^-30: floor of S in the reference key
+
+struct FusedArgs {
+  int B, H, Hq, t_cap, n_tok, n_sink, rot, tiles, tiles_per_chunk, n_chunks;
+  float scale, rscale;
+  const __half* q;
+  const int16_t* kperm;
+  const uint8_t* kcodes;
+  const uint32_t* ksz;  // (S, Z) fp16 pair per token
+  const uint8_t* vcodes;
+  const uint32_t* vsz;
+  float* part_acc;  // [B*Hq][n_chunks][D]
+  float* part_ml;   // [B*Hq][n_chunks][2]: (m, l), log2 domain
+  uint32_t* err;
+  uint64_t wait_ns;
+};
+
+__device__ __forceinline__ void bulk_load_f(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// w as the fp16 pair (hi, lo) = (fp16(w), fp16(w - hi)): hi in the low half.
+__device__ __forceinline__ uint32_t split_hi_lo(float w) {
+  const __half hi = __float2half_rn(w);
+  const __half lo = __float2half_rn(w - __half2float(hi));
+  return static_cast<uint32_t>(__half_as_ushort(hi)) | (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
+}
+
+// ((y & msk) | 0x6400 per half) as fp16 pairs, minus 1024: the masked code values.
+__device__ __forceinline__ uint32_t code_pair(uint32_t y, uint32_t msk) {
+  const uint32_t x = (y & msk) | 0x64006400u;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&x), __halves2half2(__ushort_as_half(0x6400),
+                                                                                  __ushort_as_half(0x6400)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float2 h2f(uint32_t w) { return __half22float2(*reinterpret_cast<const __half2*>(&w)); }
+
+template <int BITS, int GQ>
+__global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(const FusedArgs a) {
+  constexpr int D = 128;
+  constexpr int RB = D * BITS / 8;
+  constexpr int NW = RB / 4;
+  constexpr int NTN = (2 * GQ + 7) / 8;
+  constexpr uint32_t STAGE = kFTile * (2 * RB + 8);
+  extern __shared__ __align__(128) uint8_t fdyn[];  // kFStages x {K codes, V codes, K sz, V sz}
+  __shared__ __align__(16) uint2 bfrag[NTN][4][4][8];
+  __shared__ __align__(16) float qraw[GQ][D];
+  __shared__ int8_t qd[GQ][2][D];
+  __shared__ float qsum[GQ][1];
+  __shared__ float sqh[GQ];
+  __shared__ float mw[kFWarps][GQ], lw[kFWarps][GQ], zw[kFWarps][GQ];
+  __shared__ __align__(8) uint64_t full[kFStages];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh - b * a.H;
+  const int t_begin = c * a.tiles_per_chunk;
+  const int n_tiles = min(a.tiles_per_chunk, a.tiles - t_begin);
+  const size_t rec0 = static_cast<size_t>(bh) * a.t_cap;
+  const uint32_t base = smem_u32(fdyn);
+
+  auto issue = [&](int i, int st) {
+    const int n0 = (t_begin + i) * kFTile;
+    const int nn = min(kFTile, a.n_tok - n0);
+    const uint32_t sb = base + st * STAGE;
+    if (tid == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(nn * RB);
+      mbar_arrive_expect_tx(&full[st], 2 * bytes);
+      bulk_load_f(fdyn + st * STAGE, a.kcodes + (rec0 + n0) * RB, bytes, &full[st]);
+      bulk_load_f(fdyn + st * STAGE + kFTile * RB, a.vcodes + (rec0 + n0) * RB, bytes, &full[st]);
+    }
+    // scale / zero words, one per thread: K for tid < kFTile, V above (zero past the last token)
+    const int tok = tid & (kFTile - 1);
+    const uint32_t* src = (tid < kFTile ? a.ksz : a.vsz) + rec0 + n0 + min(tok, nn - 1);
+    cp_async4(sb + 2 * kFTile * RB + 4 * tid, src, tok < nn ? 4u : 0u);
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kFStages; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < kFStages; ++i) {
+    if (i < n_tiles) issue(i, i);
+    cp_async_commit();
+  }
+
+  // the GQ query heads of this KV head, rotated and split into int8 digits
+  if (warp < GQ)
+    query_digits<128>(a.q + (static_cast<size_t>(b) * a.Hq + h * GQ + warp) * D,
+                      a.kperm ? a.kperm + static_cast<size_t>(h) * D : nullptr, a.rot, a.rscale, lane, qraw[warp],
+                      qd[warp][0], qd[warp][1], qsum[warp], &sqh[warp]);
+  __syncthreads();
+  build_score_bfrag<BITS, GQ, NTN>(bfrag, qd, tid, kFThreads);
+  cp_async_wait_group<kFStages - 1>();  // this thread's scale / zero words of tile 0
+  __syncthreads();
+  uint2 bq[4][NTN];
+  float sq[NTN], qs[NTN];
+#pragma unroll
+  for (int nt = 0; nt < NTN; ++nt) {
+    const int qh = 4 * nt + tig;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) bq[s][nt] = bfrag[nt][s][tig][g];
+    sq[nt] = qh < GQ ? sqh[qh] : 0.0f;
+    qs[nt] = qh < GQ ? qsum[qh][0] : 0.0f;
+  }
+
+  float acc[8][NTN][4];
+  float m_run[NTN], l_run[NTN], z_run[NTN];
+#pragma unroll
+  for (int nt = 0; nt < NTN; ++nt) {
+    m_run[nt] = -INFINITY;
+    l_run[nt] = 0.0f;
+    z_run[nt] = 0.0f;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.0f;
+  }
+  // value B fragments come from the score lanes of rows 2 tig (+8) and 2 tig + 1 (+9)
+  const int srcA = 8 * tig + (g >> 1), srcB = srcA + 4;
+  const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;  // column g: digit hi (low halves) or lo
+
+  bool ok = true;
+  for (int i = 0; i < n_tiles; ++i) {
+    const int st = i % kFStages;
+    ok = mbar_wait(&full[st], (i / kFStages) & 1, a.wait_ns, a.err) && ok;
+    const int n0 = (t_begin + i) * kFTile;
+    const uint32_t kcb = base + st * STAGE, vcb = kcb + kFTile * RB;
+    const uint32_t kzb = vcb + kFTile * RB, vzb = kzb + 4 * kFTile;
+
+    // ---- scores of rows ra = 16 warp + g and rb = ra + 8
+    const int ra = 16 * warp + g, rb = ra + 8;
+    uint32_t wa[NW], wb[NW];
+#pragma unroll
+    for (int k = 0; k < NW / 4; ++k) {
+      const uint4 ua = lds128(kcb + ra * RB + 16 * k), ub = lds128(kcb + rb * RB + 16 * k);
+      wa[4 * k] = ua.x; wa[4 * k + 1] = ua.y; wa[4 * k + 2] = ua.z; wa[4 * k + 3] = ua.w;
+      wb[4 * k] = ub.x; wb[4 * k + 1] = ub.y; wb[4 * k + 2] = ub.z; wb[4 * k + 3] = ub.w;
+    }
+    int sacc[NTN][4];
+#pragma unroll
+    for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      uint32_t a0, a1, a2, a3;
+      score_afrag<BITS, NW>(wa, wb, s, tig, a0, a1, a2, a3);
+#pragma unroll
+      for (int nt = 0; nt < NTN; ++nt) mma_u8s8(sacc[nt], a0, a1, a2, a3, bq[s][nt]);
+    }
+    const int na = n0 + ra, nb = n0 + rb;
+    const bool va = na >= a.n_sink && na < a.n_tok, vb = nb >= a.n_sink && nb < a.n_tok;
+    const float2 kza = h2f(lds32(kzb + 4 * ra)), kzb2 = h2f(lds32(kzb + 4 * rb));
+    float2 vza = h2f(lds32(vzb + 4 * ra)), vzb2 = h2f(lds32(vzb + 4 * rb));
+    if (!va) vza = make_float2(0.0f, 0.0f);
+    if (!vb) vzb2 = make_float2(0.0f, 0.0f);
+    const float lga = __log2f(fmaxf(vza.x, kMinS)), lgb = __log2f(fmaxf(vzb2.x, kMinS));
+    uint32_t hla[NTN], hlb[NTN];
+#pragma unroll
+    for (int nt = 0; nt < NTN; ++nt) {
+      const bool qv = 4 * nt + tig < GQ;
+      const float da = static_cast<float>(sacc[nt][0] + 256 * sacc[nt][1]);
+      const float db = static_cast<float>(sacc[nt][2] + 256 * sacc[nt][3]);
+      const float sa = __fmaf_rn(kza.x * sq[nt], da, __fmaf_rn(kza.y, qs[nt], 0.0f)) * a.scale;
+      const float sb = __fmaf_rn(kzb2.x * sq[nt], db, __fmaf_rn(kzb2.y, qs[nt], 0.0f)) * a.scale;
+      const bool oka = va && qv, okb = vb && qv;
+      float blk = fmaxf(oka ? __fmaf_rn(sa, kLog2e, lga) : -INFINITY, okb ? __fmaf_rn(sb, kLog2e, lgb) : -INFINITY);
+      blk = fmaxf(blk, __shfl_xor_sync(0xffffffffu, blk, 4));
+      blk = fmaxf(blk, __shfl_xor_sync(0xffffffffu, blk, 8));
+      blk = fmaxf(blk, __shfl_xor_sync(0xffffffffu, blk, 16));
+      if (blk > m_run[nt] + kFLazy) {  // uniform over the lanes of this query head
+        const float f = exp2f(m_run[nt] - blk);
+        m_run[nt] = blk;
+        l_run[nt] *= f;
+        z_run[nt] *= f;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[mt][nt][e] *= f;
+      }
+      const float pa = oka ? exp2f(__fmaf_rn(sa, kLog2e, -m_run[nt])) : 0.0f;
+      const float pb = okb ? exp2f(__fmaf_rn(sb, kLog2e, -m_run[nt])) : 0.0f;
+      l_run[nt] += pa + pb;
+      z_run[nt] = __fmaf_rn(pa, vza.y, __fmaf_rn(pb, vzb2.y, z_run[nt]));
+      hla[nt] = split_hi_lo(pa * vza.x);
+      hlb[nt] = split_hi_lo(pb * vzb2.x);
+    }
+    // ---- value B fragments: tokens 2 tig, 2 tig + 1 (b0 b1) and + 8 (b2 b3), column g
+    uint32_t bv0[NTN], bv1[NTN];
+#pragma unroll
+    for (int nt = 0; nt < NTN; ++nt) {
+      const uint32_t x0 = __shfl_sync(0xffffffffu, hla[nt], srcA), x1 = __shfl_sync(0xffffffffu, hla[nt], srcB);
+      const uint32_t x2 = __shfl_sync(0xffffffffu, hlb[nt], srcA), x3 = __shfl_sync(0xffffffffu, hlb[nt], srcB);
+      bv0[nt] = __byte_perm(x0, x1, sel);
+      bv1[nt] = __byte_perm(x2, x3, sel);
+    }
+    // ---- value A fragments and products
+    const uint32_t t0 = vcb + (16 * warp + 2 * tig) * RB;
+    if constexpr (BITS == 2) {
+      const uint32_t u0 = lds32(t0 + 4 * g), u1 = lds32(t0 + RB + 4 * g);
+      const uint32_t u8 = lds32(t0 + 8 * RB + 4 * g), u9 = lds32(t0 + 9 * RB + 4 * g);
+      uint32_t y[2][4];
+      y[0][0] = __byte_perm(u0, u1, 0x5410);  // channel 16 g + t, tokens 2 tig, 2 tig + 1
+      y[0][1] = __byte_perm(u0, u1, 0x7632);  // channel 16 g + 8 + t
+      y[0][2] = __byte_perm(u8, u9, 0x5410);
+      y[0][3] = __byte_perm(u8, u9, 0x7632);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) y[1][r] = y[0][r] >> 10;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int hs = mt < 5 ? 0 : 1;
+        const uint32_t msk = 0x00030003u << (2 * (mt < 5 ? mt : mt - 5));
+        const uint32_t a0 = code_pair(y[hs][0], msk), a1 = code_pair(y[hs][1], msk);
+        const uint32_t a2 = code_pair(y[hs][2], msk), a3 = code_pair(y[hs][3], msk);
+#pragma unroll
+        for (int nt = 0; nt < NTN; ++nt) mma_f16(acc[mt][nt], a0, a1, a2, a3, bv0[nt], bv1[nt]);
+      }
+    } else {
+      uint32_t y[2][2][4];  // [word g / g + 8][shift 0 / 8][register]
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const uint32_t o = 4 * (g + 8 * w);
+        const uint32_t u0 = lds32(t0 + o), u1 = lds32(t0 + RB + o);
+        const uint32_t u8 = lds32(t0 + 8 * RB + o), u9 = lds32(t0 + 9 * RB + o);
+        y[w][0][0] = __byte_perm(u0, u1, 0x5410);
+        y[w][0][1] = __byte_perm(u0, u1, 0x7632);
+        y[w][0][2] = __byte_perm(u8, u9, 0x5410);
+        y[w][0][3] = __byte_perm(u8, u9, 0x7632);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) y[w][1][r] = y[w][0][r] >> 8;
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int w = mt >> 2, p = mt & 3, hs = p >> 1;
+        const uint32_t msk = 0x000F000Fu << (4 * (p & 1));
+        const uint32_t a0 = code_pair(y[w][hs][0], msk), a1 = code_pair(y[w][hs][1], msk);
+        const uint32_t a2 = code_pair(y[w][hs][2], msk), a3 = code_pair(y[w][hs][3], msk);
+#pragma unroll
+        for (int nt = 0; nt < NTN; ++nt) mma_f16(acc[mt][nt], a0, a1, a2, a3, bv0[nt], bv1[nt]);
+      }
+    }
+    cp_async_wait_group<kFStages - 2>();  // this thread's scale / zero words of the next tile
+    if (!__syncthreads_and(ok)) break;
+    if (i + kFStages < n_tiles) issue(i + kFStages, st);
+    cp_async_commit();
+  }
+  if (!ok) {
+    if (tid == 0)
+      for (int st = 0; st < kFStages; ++st)
+        for (uint32_t p = 0; p < 2; ++p) mbar_wait(&full[st], p, a.wait_ns, a.err);
+  }
+  cp_async_wait_all();
+#pragma unroll
+  for (int nt = 0; nt < NTN; ++nt) {
+#pragma unroll
+    for (int o = 4; o <= 16; o <<= 1) {
+      l_run[nt] += __shfl_xor_sync(0xffffffffu, l_run[nt], o);
+      z_run[nt] += __shfl_xor_sync(0xffffffffu, z_run[nt], o);
+    }
+  }
+  __syncthreads();  // every stage consumed: the stage memory now holds the per-warp sums
+  float* accw = reinterpret_cast<float*>(fdyn);  // [kFWarps][GQ][D]
+#pragma unroll
+  for (int nt = 0; nt < NTN; ++nt) {
+    const int qh = 4 * nt + tig;
+    if (qh >= GQ) continue;
+    float* dst = accw + (warp * GQ + qh) * D;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      int cha, chb;
+      float sc;
+      if constexpr (BITS == 2) {
+        cha = 16 * g + mt;
+        chb = cha + 8;
+        sc = 1.0f / static_cast<float>(1 << (2 * (mt < 5 ? mt : mt - 5)));
+      } else {
+        const int j = g + 8 * (mt >> 2), p = mt & 3;
+        cha = 8 * j + p;
+        chb = cha + 4;
+        sc = (p & 1) ? 0.0625f : 1.0f;
+      }
+      dst[cha] = (acc[mt][nt][0] + acc[mt][nt][1]) * sc;
+      dst[chb] = (acc[mt][nt][2] + acc[mt][nt][3]) * sc;
+    }
+    if (g == 0) {
+      mw[warp][qh] = m_run[nt];
+      lw[warp][qh] = l_run[nt];
+      zw[warp][qh] = z_run[nt];
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < GQ * D; e += kFThreads) {
+    const int qh = e / D, j = e - qh * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kFWarps; ++w) M = fmaxf(M, mw[w][qh]);
+    float s = 0.0f, L = 0.0f, Z = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kFWarps; ++w) {
+      const float f = mw[w][qh] == -INFINITY ? 0.0f : exp2f(mw[w][qh] - M);
+      s = __fmaf_rn(f, accw[(w * GQ + qh) * D + j], s);
+      L = __fmaf_rn(f, lw[w][qh], L);
+      Z = __fmaf_rn(f, zw[w][qh], Z);
+    }
+    const size_t row = (static_cast<size_t>(b) * a.Hq + h * GQ + qh) * a.n_chunks + c;
+    a.part_acc[row * D + j] = s + Z;
+    if (j == 0) {
+      a.part_ml[2 * row] = M;
+      a.part_ml[2 * row + 1] = L;
+    }
+  }
+}
+
+struct MergeArgs {
+  int B, H, Hq, GQ, n_tok, n_sink, n_chunks, rot, krope;
+  float scale, rscale;
+  const __half* q;
+  const __half* ksink;
+  const float* rope_cs;
+  const __half* vsink;
+  const int16_t* vperm;
+  const float* part_acc;
+  const float* part_ml;
+  float* out;
+};
+
+// One CTA per (batch, query head): sink scores (fp16 keys, exactly as the
+// score kernel forms them), the log-sum-exp merge of the chunks and sinks, the
+// inverse rotation and permutation, and the sink values.
+__global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
+  __shared__ __align__(16) float qraw[D];
+  __shared__ float ts[kFMaxSinks];
+  __shared__ float ys[2][D];
+  __shared__ float nat[D];
+  __shared__ float red[4];
+  const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
+  const int bq = blockIdx.x;
+  const int b = bq / a.Hq, qh = bq % a.Hq, h = qh / a.GQ;
+  const int ns = min(a.n_sink, a.n_tok);
+  const size_t vh = static_cast<size_t>(b) * a.H + h;
+  qraw[j] = __half2float(a.q[static_cast<size_t>(bq) * D + j]);
+  __syncthreads();
+  float mloc = -INFINITY;
+  for (int n = warp; n < ns; n += kThreads / 32) {
+    const float s = sink_dot(qraw, a.ksink + (vh * a.n_sink + n) * D,
+                             a.krope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane) *
+                    a.scale;
+    const float t = s * kLog2e;
+    if (lane == 0) ts[n] = s;
+    mloc = fmaxf(mloc, t);
+  }
+  const float* ml = a.part_ml + static_cast<size_t>(bq) * a.n_chunks * 2;
+  const float* pa = a.part_acc + static_cast<size_t>(bq) * a.n_chunks * D;
+  for (int c = 0; c < a.n_chunks; ++c) mloc = fmaxf(mloc, ml[2 * c]);
+  if (lane == 0) red[warp] = mloc;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float L = 0.0f, acc = 0.0f;
+  for (int c = 0; c < a.n_chunks; ++c) {
+    const float f = ml[2 * c] == -INFINITY ? 0.0f : exp2f(ml[2 * c] - M);
+    L = __fmaf_rn(ml[2 * c + 1], f, L);
+    acc = __fmaf_rn(pa[static_cast<size_t>(c) * D + j], f, acc);
+  }
+  for (int n = 0; n < ns; ++n) L += exp2f(__fmaf_rn(ts[n], kLog2e, -M));
+  const float invL = 1.0f / L;
+  float y = acc * invL;  // sum_n p_n y_n, channel j of the rotated basis
+  if (a.rot == KVQ_ROT_FWHT_HEAD) {  // x = H y / sqrt(D), Sylvester order, strides 1 .. 64
+    int cur = 0;
+    ys[0][j] = y;
+    __syncthreads();
+#pragma unroll
+    for (int st = 1; st < D; st <<= 1) {
+      const float u = ys[cur][j], w = ys[cur][j ^ st];
+      ys[cur ^ 1][j] = (j & st) ? w - u : u + w;
+      cur ^= 1;
+      __syncthreads();
+    }
+    y = ys[cur][j] * a.rscale;
+  }
+  nat[a.vperm ? a.vperm[static_cast<size_t>(h) * D + j] & (D - 1) : j] = y;  // x[perm[j]] = y_j
+  __syncthreads();
+  float o = nat[j];
+  for (int n = 0; n < ns; ++n) {
+    const float p = exp2f(__fmaf_rn(ts[n], kLog2e, -M)) * invL;
+    o = __fmaf_rn(p, __half2float(a.vsink[(vh * a.n_sink + n) * D + j]), o);
+  }
+  a.out[static_cast<size_t>(bq) * D + j] = o;
+}
+
+template <int BITS, int GQ>
+kvq_status run_fused(FusedArgs& fa, const LaunchCtx& ctx, cudaStream_t st) {
+  constexpr size_t smem = static_cast<size_t>(kFStages) * kFTile * (2 * (128 * BITS / 8) + 8);
+  const void* fn = reinterpret_cast<const void*>(k_attend_fused<BITS, GQ>);
+  if (!set_smem_once(fn, smem)) return KVQ_ERR_CUDA;
+  const int per_sm = occupancy_once(fn, kFThreads, smem);
+  const int bh = fa.B * fa.H;
+  int want = ctx.num_sms * per_sm / bh;  // chunks per (batch, KV head) for about one wave
+  want = want < 1 ? 1 : (want > kFMaxChunks ? kFMaxChunks : want);
+  fa.tiles_per_chunk = (fa.tiles + want - 1) / want;
+  fa.n_chunks = (fa.tiles + fa.tiles_per_chunk - 1) / fa.tiles_per_chunk;
+  k_attend_fused<BITS, GQ><<<dim3(static_cast<unsigned>(fa.n_chunks), static_cast<unsigned>(bh)), kFThreads,
+                             smem, st>>>(fa);
+  return launch_status();
+}
+
+template <int BITS>
+kvq_status fused_by_gq(FusedArgs& fa, int gq, const LaunchCtx& ctx, cudaStream_t st) {
+  switch (gq) {
+    case 1: return run_fused<BITS, 1>(fa, ctx, st);
+    case 2: return run_fused<BITS, 2>(fa, ctx, st);
+    case 4: return run_fused<BITS, 4>(fa, ctx, st);
+    case 8: return run_fused<BITS, 8>(fa, ctx, st);
+    default: return KVQ_ERR_UNSUPPORTED;
+  }
+}
+
+bool fused_path(int bits, int group, int n_sink) {
+  return (bits == 2 || bits == 4) && group == 128 && n_sink <= kFMaxSinks;
+}
+
+int fused_tiles(int n_tokens) { return (n_tokens + kFTile - 1) / kFTile; }
+
 // Fixed scratch of kvq_attend_noalloc: a file-scope device array, reserved when
 // the module is loaded, so that entry point never allocates. 40 MiB holds the
 // scores and chunk partials of about 9 M (query head x cached token) pairs
@@ -281,8 +759,13 @@ void* attend_scratch() {
   return ptr[dev];
 }
 
-size_t attend_workspace_bytes(int B, int q_heads, int n_tokens) {
-  const size_t bq = static_cast<size_t>(B) * q_heads;
+size_t attend_workspace_bytes(const kvq_desc& dk, int q_heads, int n_tokens) {
+  const size_t bq = static_cast<size_t>(dk.batch) * q_heads;
+  if (fused_path(dk.bits, dk.group, dk.n_sink)) {  // chunk partials only; chunks <= min(tiles, kFMaxChunks)
+    const int tiles = fused_tiles(n_tokens);
+    const size_t n_chunks = static_cast<size_t>(tiles < kFMaxChunks ? tiles : kFMaxChunks);
+    return align256(bq * n_chunks * D * 4) + align256(bq * n_chunks * 2 * 4);
+  }
   const size_t n_chunks = (static_cast<size_t>(n_tokens) + kCh * kSub - 1) / (kCh * kSub);
   return align256(bq * n_tokens * 4) + align256(bq * n_chunks * D * 4) + align256(bq * n_chunks * 2 * 4);
 }
@@ -291,6 +774,57 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
                          const kvq_packed& kc, const kvq_tables& tk, const kvq_packed& vc, const kvq_tables& tv,
                          int n_tokens, float scale, float* out, void* ws, cudaStream_t st, const LaunchCtx& ctx) {
   const size_t bq = static_cast<size_t>(dk.batch) * q_heads;
+  if (fused_path(dk.bits, dk.group, dk.n_sink)) {
+    const int tiles = fused_tiles(n_tokens);
+    const int max_chunks = tiles < kFMaxChunks ? tiles : kFMaxChunks;
+    FusedArgs fa{};
+    fa.B = dk.batch;
+    fa.H = dk.heads;
+    fa.Hq = q_heads;
+    fa.t_cap = dk.t_cap;
+    fa.n_tok = n_tokens;
+    fa.n_sink = dk.n_sink;
+    fa.rot = dk.rot;
+    fa.tiles = tiles;
+    fa.scale = scale;
+    fa.rscale = static_cast<float>(1.0 / sqrt(static_cast<double>(D)));
+    fa.q = static_cast<const __half*>(q);
+    fa.kperm = tk.perm;
+    fa.kcodes = kc.codes;
+    fa.ksz = static_cast<const uint32_t*>(kc.scale_zero);
+    fa.vcodes = vc.codes;
+    fa.vsz = static_cast<const uint32_t*>(vc.scale_zero);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    fa.part_acc = reinterpret_cast<float*>(w);
+    fa.part_ml = reinterpret_cast<float*>(w + align256(bq * max_chunks * D * 4));
+    fa.err = ctx.err;
+    fa.wait_ns = ctx.wait_ns;
+    const int gq = q_heads / dk.heads;
+    kvq_status s = dk.bits == 2 ? fused_by_gq<2>(fa, gq, ctx, st) : fused_by_gq<4>(fa, gq, ctx, st);
+    if (s != KVQ_OK) return s;
+    MergeArgs ma{};
+    ma.B = dk.batch;
+    ma.H = dk.heads;
+    ma.Hq = q_heads;
+    ma.GQ = gq;
+    ma.n_tok = n_tokens;
+    ma.n_sink = dk.n_sink;
+    ma.n_chunks = fa.n_chunks;
+    ma.rot = dv.rot;
+    ma.krope = dk.rope;
+    ma.scale = scale;
+    ma.rscale = fa.rscale;
+    ma.q = fa.q;
+    ma.ksink = static_cast<const __half*>(kc.sink);
+    ma.rope_cs = tk.rope_cs;
+    ma.vsink = static_cast<const __half*>(vc.sink);
+    ma.vperm = tv.perm;
+    ma.part_acc = fa.part_acc;
+    ma.part_ml = fa.part_ml;
+    ma.out = out;
+    k_attend_merge<<<static_cast<unsigned>(bq), kThreads, 0, st>>>(ma);
+    return launch_status();
+  }
   AttnArgs a{};
   a.B = dk.batch;
   a.H = dk.heads;

@@ -44,7 +44,7 @@ kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq
                         const kvq_tables& tb, int n_tokens, float scale, float* scores, cudaStream_t st,
                         const LaunchCtx& ctx);
 kvq_status launch_debug_wait(uint64_t limit_ns, cudaStream_t st, const LaunchCtx& ctx);
-size_t attend_workspace_bytes(int B, int q_heads, int n_tokens);
+size_t attend_workspace_bytes(const kvq_desc& dk, int q_heads, int n_tokens);
 size_t attend_scratch_bytes();
 void* attend_scratch();
 kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, int q_heads,

@@ -13,6 +13,7 @@
 // thread, fp32 accumulation.
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
+#include "kvq_qdigits.cuh"
 
 namespace kvq {
 namespace {
@@ -190,14 +191,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// Channel that K index (k-step s, lane quad position tig, byte l, upper half u)
-// of the A fragment carries; B uses the same map.
-template <int BITS>
-__device__ __forceinline__ int kchan(int s, int tig, int l, int u) {
-  if constexpr (BITS == 2) return 32 * s + 16 * u + 4 * l + tig;
-  else return 32 * s + 16 * u + 8 * (tig >> 1) + 2 * l + (tig & 1);
-}
-
 template <int BITS, int G, int GQ>
 __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
   constexpr int D = 128;
@@ -205,7 +198,6 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
   constexpr int NW = RB / 4;             // words per record
   constexpr int NTN = (2 * GQ + 7) / 8;  // n-tiles of 8 columns
   constexpr int NGK = D / G;             // quantization groups per record
-  constexpr uint32_t MASK = BITS == 2 ? 0x03030303u : 0x0F0F0F0Fu;
   const ScoreArgs& a = ma.s;
   extern __shared__ __align__(128) uint8_t codes_dyn[];  // kMmaStages tiles of kMmaTile records
   __shared__ __align__(16) uint2 bfrag[NTN][4][4][8];
@@ -245,64 +237,12 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
     __syncthreads();  // previous (batch, head) fully consumed
     if (warp < GQ) {
       const int qh = h * GQ + warp;
-      const __half* qv = a.q + (static_cast<size_t>(b) * a.Hq + qh) * D;
-      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qv) + lane);  // channels 4 lane .. 4 lane + 3
-      const float2 r01 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-      const float2 r23 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      float v[4] = {r01.x, r01.y, r23.x, r23.y};
-      *reinterpret_cast<float4*>(&qraw[warp][4 * lane]) = make_float4(v[0], v[1], v[2], v[3]);
-      if (a.perm) {
-        const uint2 pk = __ldg(reinterpret_cast<const uint2*>(a.perm + static_cast<size_t>(h) * D) + lane);
-        const uint32_t pw[2] = {pk.x, pk.y};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = __half2float(qv[(pw[i >> 1] >> (16 * (i & 1))) & (D - 1)]);
-      }
-      if (a.rot == KVQ_ROT_FWHT_HEAD) {
-        const float t0 = v[0] + v[1], t1 = v[0] - v[1], t2 = v[2] + v[3], t3 = v[2] - v[3];
-        v[0] = t0 + t2; v[2] = t0 - t2; v[1] = t1 + t3; v[3] = t1 - t3;
-#pragma unroll
-        for (int m = 1; m < 32; m <<= 1) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float p = __shfl_xor_sync(0xffffffffu, v[i], m);
-            v[i] = (lane & m) ? (p - v[i]) : (v[i] + p);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] *= a.rscale;
-      }
-      float mx = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-#pragma unroll
-      for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-      const float sq = mx > 0.0f ? mx / 32000.0f : 1.0f;
-      const float rsq = 1.0f / sq;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int Q = __float2int_rn(v[i] * rsq);
-        const int lo = ((Q + 128) & 255) - 128;
-        qd[warp][0][4 * lane + i] = static_cast<int8_t>(lo);
-        qd[warp][1][4 * lane + i] = static_cast<int8_t>((Q - lo) >> 8);
-      }
-      float ps = (v[0] + v[1]) + (v[2] + v[3]);
-#pragma unroll
-      for (int m = 1; m < G / 4; m <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, m);
-      if ((lane & (G / 4 - 1)) == 0) qsum[warp][lane / (G / 4)] = ps;
-      if (lane == 0) sqh[warp] = sq;
+      query_digits<G>(a.q + (static_cast<size_t>(b) * a.Hq + qh) * D,
+                      a.perm ? a.perm + static_cast<size_t>(h) * D : nullptr, a.rot, a.rscale, lane, qraw[warp],
+                      qd[warp][0], qd[warp][1], qsum[warp], &sqh[warp]);
     }
     __syncthreads();
-    for (int e = tid; e < NTN * 128; e += kMmaThreads) {  // B fragments: column c = 2 * head + digit
-      const int nt = e >> 7, s = (e >> 5) & 3, tg = (e >> 3) & 3, n = e & 7;
-      const int c = nt * 8 + n, hh = c >> 1, dg = c & 1;
-      uint32_t b0 = 0, b1 = 0;
-      if (hh < GQ) {
-#pragma unroll
-        for (int l = 0; l < 4; ++l) {
-          b0 |= static_cast<uint32_t>(static_cast<uint8_t>(qd[hh][dg][kchan<BITS>(s, tg, l, 0)])) << (8 * l);
-          b1 |= static_cast<uint32_t>(static_cast<uint8_t>(qd[hh][dg][kchan<BITS>(s, tg, l, 1)])) << (8 * l);
-        }
-      }
-      bfrag[nt][s][tg][n] = make_uint2(b0, b1);
-    }
+    build_score_bfrag<BITS, GQ, NTN>(bfrag, qd, tid, kMmaThreads);  // column c = 2 * head + digit
     __syncthreads();
     // fp16 sinks of this (batch, head): s = scale * q . RoPE_n(sink_n); done by the
     // CTA that owns the (batch, head)'s first tile, one warp per (sink, query head)
@@ -310,20 +250,8 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
       const size_t vh = static_cast<size_t>(b) * a.H + h;
       for (int e = warp; e < min(a.n_sink, a.n_tok) * GQ; e += kMmaThreads / 32) {
         const int n = e / GQ, hh = e % GQ;
-        const uint2 kr = __ldg(reinterpret_cast<const uint2*>(a.sink + (vh * a.n_sink + n) * D) + lane);
-        const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kr.x));
-        const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kr.y));
-        float k4[4] = {k01.x, k01.y, k23.x, k23.y};
-        if (a.rope) {  // pairs 2 lane and 2 lane + 1 of position n
-          const float4 cs = __ldg(reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(n) * D) + lane);
-          rope_fwd(k4[0], k4[1], cs.x, cs.y);
-          rope_fwd(k4[2], k4[3], cs.z, cs.w);
-        }
-        float acc = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc = __fmaf_rn(qraw[hh][4 * lane + i], k4[i], acc);
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+        const float acc = sink_dot(qraw[hh], a.sink + (vh * a.n_sink + n) * D,
+                                   a.rope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane);
         if (lane == 0) a.scores[(static_cast<size_t>(b) * a.Hq + h * GQ + hh) * a.n_tok + n] = acc * a.scale;
       }
     }
@@ -380,31 +308,11 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         uint32_t a0, a1, a2, a3;
-        if constexpr (BITS == 2) {
-          a0 = (wa[2 * s] >> (2 * tig)) & MASK;
-          a1 = (wb[2 * s] >> (2 * tig)) & MASK;
-          a2 = (wa[2 * s + 1] >> (2 * tig)) & MASK;
-          a3 = (wb[2 * s + 1] >> (2 * tig)) & MASK;
-        } else {
-          const bool odd = (tig & 2) != 0;  // word 4s + (tig >> 1), selected without dynamic indexing
-          const int sh = 4 * (tig & 1);
-          a0 = ((odd ? wa[4 * s + 1] : wa[4 * s]) >> sh) & MASK;
-          a1 = ((odd ? wb[4 * s + 1] : wb[4 * s]) >> sh) & MASK;
-          a2 = ((odd ? wa[4 * s + 3] : wa[4 * s + 2]) >> sh) & MASK;
-          a3 = ((odd ? wb[4 * s + 3] : wb[4 * s + 2]) >> sh) & MASK;
-        }
+        score_afrag<BITS, NW>(wa, wb, s, tig, a0, a1, a2, a3);
         constexpr int SPG = G / 32;  // k-steps per group
         const int q = s / SPG;
 #pragma unroll
-        for (int nt = 0; nt < NTN; ++nt) {
-          const uint2 bb = bfrag[nt][s][tig][g];
-          asm volatile(
-              "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-              "{%0,%1,%2,%3};"
-              : "+r"(acc[mt][q][nt][0]), "+r"(acc[mt][q][nt][1]), "+r"(acc[mt][q][nt][2]),
-                "+r"(acc[mt][q][nt][3])
-              : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bb.x), "r"(bb.y));
-        }
+        for (int nt = 0; nt < NTN; ++nt) mma_u8s8(acc[mt][q][nt], a0, a1, a2, a3, bfrag[nt][s][tig][g]);
       }
     }
     // every warp has read this stage: refill it with the tile kMmaStages ahead
