@@ -38,6 +38,7 @@ import workloads as W  # noqa: E402
 METRIC = "fp16-KV GB/s for encode/decode/score and % of B200 HBM roofline"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 512 << 20
 
 
 def _peaks():
@@ -233,6 +234,8 @@ class AttendStep:
     K and the V cache, then out = softmax(q . k) . v over every slot."""
 
     workload = "llama3_8b_gqa_attend"
+    # K and V caches are 75 MB, less than the 126 MB L2: flush it before every step
+    l2_flush = True
 
     def __init__(self, device):
         import torch
@@ -250,7 +253,7 @@ class AttendStep:
                     "attend": self.k.alg_cache + self.v.alg_cache + q_out}
         self.fp16_equiv = {"append_k": self.k.fp16_append, "append_v": self.v.fp16_append,
                            "attend": 2 * self.k.fp16_score}
-        self.kernels = {"append_k": "k_encode_head", "append_v": "k_encode_head", "attend": "k_attend_part"}
+        self.kernels = {"append_k": "k_encode_head", "append_v": "k_encode_head", "attend": "k_attend_fused"}
         self.fp32_ops = {}
         self.names = list(self.alg)
         torch.cuda.synchronize(device)
@@ -473,6 +476,9 @@ def run_ours(args):
 
     nk = len(launches)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    flush = getattr(st, "l2_flush", False)
+    # read-based flush (a clean 512 MB sweep, 4x the L2): leaves no dirty lines for the next kernel to write back
+    fbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -481,6 +487,8 @@ def run_ours(args):
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record(stream)
         for s in range(args.steps):
+            if flush:
+                fbuf.sum()
             ev[s][0].record(stream)
             for i, f in enumerate(launches):
                 f()
@@ -489,7 +497,9 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
-    total_ms = t_start.elapsed_time(t_end)
+    # with a flush the timed region is the steps alone (each step bracketed by its own events)
+    total_ms = (sum(ev[s][0].elapsed_time(ev[s][nk]) for s in range(args.steps)) if flush
+                else t_start.elapsed_time(t_end))
     per_kernel = {n: 0.0 for n in st.names}
     for s in range(args.steps):
         for i, n in enumerate(st.names):
@@ -594,7 +604,9 @@ def _other_config(name, n_gpus):
     w = W.WORKLOADS[name]
     return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T, "q_heads": w.Hq,
             "rotation": w.rot, "quant": w.quant, "bits": w.bits, "group": w.group, "n_sink": w.n_sink,
-            "perm": w.perm, "l2": "no flush (inputs larger than L2)" if name != "tiny" else "L2-resident",
+            "perm": w.perm, "l2": ("flushed before every step by a 512 MB read (outside the timed steps)"
+                                   if name == "llama3_8b_gqa_attend" else
+                                   "no flush (inputs larger than L2)" if name != "tiny" else "L2-resident"),
             "parallelism": f"replicas x{n_gpus}"}
 
 

@@ -17,6 +17,7 @@
 #include <math.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -258,16 +259,20 @@ size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 // scores, the running softmax statistics and sum_n p_n y_n, all products on
 // the tensor cores; a small merge kernel then combines the chunks.
 //
+// Work split: CTA = (chunk of 16-token blocks, batch x KV head); its 8 warps
+// take the chunk's blocks in turn and each streams its own blocks through a
+// private ring of shared-memory stages filled by cp.async (no CTA barrier in
+// the loop); the warps' running sums are merged once at the end.
+//
 // Scores: exactly the score kernel's arithmetic (u8 codes x s8 query digits,
 // mma.sync m16n8k32, same fp32 epilogue), so they match kvq_score bit for bit.
 //
 // Values: out_rot = sum_n p_n (S_n c_n + Z_n) = sum_n w_n c_n + sum_n p_n Z_n
 // with w_n = p_n S_n. sum_n w_n c_n runs on mma.sync m16n8k16 (fp16 in, fp32
-// accumulate) with A = codes (channels x tokens; small integers, exact in
-// fp16) and B = weights (tokens x columns). Each weight is carried as two fp16
-// terms w = hi + lo (hi = fp16(w), lo = fp16(w - hi)), one column each, so the
-// product keeps about 22 bits of w: with N = 8 columns a group of four query
-// heads fills one n-tile.
+// accumulate) with A = codes (channels x tokens) and B = weights (tokens x
+// columns). Each weight is carried as two fp16 terms w = hi + lo (hi =
+// fp16(w), lo = fp16(w - hi)), one column each, so the product keeps about 22
+// bits of w; with N = 8 columns a group of four query heads fills one n-tile.
 //
 // Range: the running reference m tracks the largest key lambda_n = s_n log2(e)
 // + log2(S_n) (S_n clamped to >= 2^-30), and p'_n = 2^(s_n log2(e) - m), so
@@ -277,23 +282,44 @@ size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 //
 // A operand without a shift per m-tile: a lane's rows g and g + 8 of m-tile t
 // are two channels whose codes sit at the same bit offset in the low and high
-// 16-bit halves of one record word; the two tokens of a register are paired
-// with one byte permute per word pair, and the code is masked in place:
+// 16-bit halves of one record word, and the two tokens of a register are
+// paired by one byte permute per word pair. The code is masked in place:
 // (y & (3 << 2t)) | 0x6400 is the fp16 1024 + c 4^t, minus 1024 exactly c 4^t
-// (kept below 1024 by taking t >= 5 from y >> 10). The 4^t is undone once on
-// the accumulators.
+// (kept below 1024 by taking t >= 5 from y >> 10); 4^-t is applied once to the
+// accumulators. (Leaving the masked field as an fp16 subnormal, c 4^t 2^-24,
+// would save the subtraction, but its products with subnormal lo halves of
+// small weights lost precision on the tensor cores.)
+#ifndef KVQ_ATTEND_MINB
+#define KVQ_ATTEND_MINB 2  // resident CTAs per SM the register budget is sized for (GQ <= 4)
+#endif
+#ifndef KVQ_ATTEND_WAVES_NUM  // CTAs launched = resident slots x NUM / DEN (rounded to whole chunks)
+#define KVQ_ATTEND_WAVES_NUM 1
+#endif
+#ifndef KVQ_ATTEND_WAVES_DEN
+#define KVQ_ATTEND_WAVES_DEN 1
+#endif
+#ifndef KVQ_ATTEND_IMAD_SHIFT
+#define KVQ_ATTEND_IMAD_SHIFT 0  // 2-bit score operand: lane shift as an integer multiply
+#endif
 constexpr int kFWarps = 8;
 constexpr int kFThreads = 32 * kFWarps;
-constexpr int kFTile = 16 * kFWarps;  // tokens per stage: one 16-token block per warp
-constexpr int kFStages = 4;
+constexpr int kFBlock = 16;           // tokens per warp step (one m16 tile of the score MMA)
 constexpr int kFMaxChunks = 256;
-constexpr int kFMaxSinks = 1024;        // merge keeps the sink scores in shared memory
-constexpr float kFLazy = 8.0f;          // log2 headroom before the reference is raised
+constexpr int kFMaxSinks = 1024;      // merge keeps the sink scores in shared memory
+constexpr float kFLazy = 8.0f;        // log2 headroom before the reference is raised
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kMinS = 9.3132257e-10f;  // 2^-30: floor of S in the reference key
 
+template <int BITS>
+struct FusedCfg {
+  static constexpr int RB = 128 * BITS / 8;
+  static constexpr int STAGES = BITS == 2 ? 6 : 4;                    // per warp
+  static constexpr int STAGE = 2 * kFBlock * RB + 2 * kFBlock * 4;    // K codes, V codes, K sz, V sz
+  static constexpr int SMEM = kFWarps * STAGES * STAGE;
+};
+
 struct FusedArgs {
-  int B, H, Hq, t_cap, n_tok, n_sink, rot, tiles, tiles_per_chunk, n_chunks;
+  int B, H, Hq, t_cap, n_tok, n_sink, rot, blocks, blocks_per_chunk, n_chunks;
   float scale, rscale;
   const __half* q;
   const int16_t* kperm;
@@ -303,16 +329,17 @@ struct FusedArgs {
   const uint32_t* vsz;
   float* part_acc;  // [B*Hq][n_chunks][D]
   float* part_ml;   // [B*Hq][n_chunks][2]: (m, l), log2 domain
-  uint32_t* err;
-  uint64_t wait_ns;
 };
 
-__device__ __forceinline__ void bulk_load_f(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // w as the fp16 pair (hi, lo) = (fp16(w), fp16(w - hi)): hi in the low half.
@@ -322,73 +349,74 @@ __device__ __forceinline__ uint32_t split_hi_lo(float w) {
   return static_cast<uint32_t>(__half_as_ushort(hi)) | (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
 }
 
-// ((y & msk) | 0x6400 per half) as fp16 pairs, minus 1024: the masked code values.
-__device__ __forceinline__ uint32_t code_pair(uint32_t y, uint32_t msk) {
-  const uint32_t x = (y & msk) | 0x64006400u;
-  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&x), __halves2half2(__ushort_as_half(0x6400),
-                                                                                  __ushort_as_half(0x6400)));
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-
 __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// ((y & msk) | 0x6400 per half) as fp16 pairs, minus 1024: the masked code values.
+__device__ __forceinline__ uint32_t code_pair(uint32_t y, uint32_t msk) {
+  const uint32_t x = (y & msk) | 0x64006400u;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&x),
+                            __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 __device__ __forceinline__ float2 h2f(uint32_t w) { return __half22float2(*reinterpret_cast<const __half2*>(&w)); }
 
 template <int BITS, int GQ>
-__global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(const FusedArgs a) {
+__global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 2) k_attend_fused(const FusedArgs a) {
+  using C = FusedCfg<BITS>;
   constexpr int D = 128;
-  constexpr int RB = D * BITS / 8;
+  constexpr int RB = C::RB;
   constexpr int NW = RB / 4;
   constexpr int NTN = (2 * GQ + 7) / 8;
-  constexpr uint32_t STAGE = kFTile * (2 * RB + 8);
-  extern __shared__ __align__(128) uint8_t fdyn[];  // kFStages x {K codes, V codes, K sz, V sz}
+  constexpr int S = C::STAGES;
+  constexpr int CPL = kFBlock * RB / (32 * 16);  // 16-byte code copies per lane and tensor
+  constexpr bool ALLQ = GQ % 4 == 0;             // every lane's query head exists
+  constexpr bool IMAD_SHIFT = KVQ_ATTEND_IMAD_SHIFT && BITS == 2;
+  extern __shared__ __align__(128) uint8_t fdyn[];  // per warp: S stages of {K codes, V codes, K sz, V sz}
   __shared__ __align__(16) uint2 bfrag[NTN][4][4][8];
   __shared__ __align__(16) float qraw[GQ][D];
   __shared__ int8_t qd[GQ][2][D];
   __shared__ float qsum[GQ][1];
   __shared__ float sqh[GQ];
   __shared__ float mw[kFWarps][GQ], lw[kFWarps][GQ], zw[kFWarps][GQ];
-  __shared__ __align__(8) uint64_t full[kFStages];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tig = lane & 3;
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh - b * a.H;
-  const int t_begin = c * a.tiles_per_chunk;
-  const int n_tiles = min(a.tiles_per_chunk, a.tiles - t_begin);
+  const int k_begin = c * a.blocks_per_chunk;
+  const int nk = min(a.blocks_per_chunk, a.blocks - k_begin);
+  const int my_n = nk > warp ? (nk - warp + kFWarps - 1) / kFWarps : 0;  // blocks k_begin + warp + 8 i
   const size_t rec0 = static_cast<size_t>(bh) * a.t_cap;
-  const uint32_t base = smem_u32(fdyn);
+  const uint32_t wbase = smem_u32(fdyn) + warp * (S * C::STAGE);
 
+  // block i of this warp into stage st: codes 16 bytes per lane, scale / zero 4 bytes (zero past n_tok)
   auto issue = [&](int i, int st) {
-    const int n0 = (t_begin + i) * kFTile;
-    const int nn = min(kFTile, a.n_tok - n0);
-    const uint32_t sb = base + st * STAGE;
-    if (tid == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(nn * RB);
-      mbar_arrive_expect_tx(&full[st], 2 * bytes);
-      bulk_load_f(fdyn + st * STAGE, a.kcodes + (rec0 + n0) * RB, bytes, &full[st]);
-      bulk_load_f(fdyn + st * STAGE + kFTile * RB, a.vcodes + (rec0 + n0) * RB, bytes, &full[st]);
-    }
-    // scale / zero words, one per thread: K for tid < kFTile, V above (zero past the last token)
-    const int tok = tid & (kFTile - 1);
-    const uint32_t* src = (tid < kFTile ? a.ksz : a.vsz) + rec0 + n0 + min(tok, nn - 1);
-    cp_async4(sb + 2 * kFTile * RB + 4 * tid, src, tok < nn ? 4u : 0u);
-  };
-  if (tid == 0) {
-    for (int i = 0; i < kFStages; ++i) mbar_init(&full[i], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
+    const int n0 = (k_begin + warp + i * kFWarps) * kFBlock;
+    const uint32_t sb = wbase + st * C::STAGE;
 #pragma unroll
-  for (int i = 0; i < kFStages; ++i) {
-    if (i < n_tiles) issue(i, i);
+    for (int r = 0; r < CPL; ++r) {
+      const int off = 16 * (lane + 32 * r);
+      const bool live = n0 + off / RB < a.n_tok;
+      const size_t src = (rec0 + n0) * RB + (live ? off : 0);
+      cp_async16(sb + off, a.kcodes + src, live ? 16u : 0u);
+      cp_async16(sb + kFBlock * RB + off, a.vcodes + src, live ? 16u : 0u);
+    }
+    const int tok = lane & (kFBlock - 1);
+    const bool live = n0 + tok < a.n_tok;
+    cp_async4(sb + 2 * kFBlock * RB + 4 * lane, (lane < kFBlock ? a.ksz : a.vsz) + rec0 + n0 + (live ? tok : 0),
+              live ? 4u : 0u);
+  };
+#pragma unroll
+  for (int i = 0; i < S; ++i) {
+    if (i < my_n) issue(i, i);
     cp_async_commit();
   }
 
@@ -399,7 +427,6 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
                       qd[warp][0], qd[warp][1], qsum[warp], &sqh[warp]);
   __syncthreads();
   build_score_bfrag<BITS, GQ, NTN>(bfrag, qd, tid, kFThreads);
-  cp_async_wait_group<kFStages - 1>();  // this thread's scale / zero words of tile 0
   __syncthreads();
   uint2 bq[4][NTN];
   float sq[NTN], qs[NTN];
@@ -426,22 +453,23 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
   }
   // value B fragments come from the score lanes of rows 2 tig (+8) and 2 tig + 1 (+9)
   const int srcA = 8 * tig + (g >> 1), srcB = srcA + 4;
+  const uint32_t lmul = 1u << (6 - 2 * tig);  // multiply variant: bits 2 tig .. 2 tig + 1 of a byte to 6 .. 7
   const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;  // column g: digit hi (low halves) or lo
 
-  bool ok = true;
-  for (int i = 0; i < n_tiles; ++i) {
-    const int st = i % kFStages;
-    ok = mbar_wait(&full[st], (i / kFStages) & 1, a.wait_ns, a.err) && ok;
-    const int n0 = (t_begin + i) * kFTile;
-    const uint32_t kcb = base + st * STAGE, vcb = kcb + kFTile * RB;
-    const uint32_t kzb = vcb + kFTile * RB, vzb = kzb + 4 * kFTile;
-
-    // ---- scores of rows ra = 16 warp + g and rb = ra + 8
-    const int ra = 16 * warp + g, rb = ra + 8;
+  // one 16-token block; INTERIOR: no sink and no position past n_tok in it
+  // shared-memory reads as plain loads, so the compiler may schedule them around the products
+  auto ld4 = [](const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); };
+  auto block = [&](auto interior, int n0, const uint8_t* kcb) {
+    constexpr bool INTERIOR = decltype(interior)::value;
+    const uint8_t* vcb = kcb + kFBlock * RB;
+    const uint8_t* kzb = vcb + kFBlock * RB;
+    const uint8_t* vzb = kzb + 4 * kFBlock;
+    // ---- scores of rows g and g + 8
     uint32_t wa[NW], wb[NW];
 #pragma unroll
     for (int k = 0; k < NW / 4; ++k) {
-      const uint4 ua = lds128(kcb + ra * RB + 16 * k), ub = lds128(kcb + rb * RB + 16 * k);
+      const uint4 ua = *reinterpret_cast<const uint4*>(kcb + g * RB + 16 * k);
+      const uint4 ub = *reinterpret_cast<const uint4*>(kcb + (g + 8) * RB + 16 * k);
       wa[4 * k] = ua.x; wa[4 * k + 1] = ua.y; wa[4 * k + 2] = ua.z; wa[4 * k + 3] = ua.w;
       wb[4 * k] = ub.x; wb[4 * k + 1] = ub.y; wb[4 * k + 2] = ub.z; wb[4 * k + 3] = ub.w;
     }
@@ -453,23 +481,36 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
       uint32_t a0, a1, a2, a3;
-      score_afrag<BITS, NW>(wa, wb, s, tig, a0, a1, a2, a3);
+      if constexpr (IMAD_SHIFT) {  // code tig of every byte moved to bits 6..7 by a multiply: 64 c per byte
+        a0 = (wa[2 * s] * lmul) & 0xC0C0C0C0u;
+        a1 = (wb[2 * s] * lmul) & 0xC0C0C0C0u;
+        a2 = (wa[2 * s + 1] * lmul) & 0xC0C0C0C0u;
+        a3 = (wb[2 * s + 1] * lmul) & 0xC0C0C0C0u;
+      } else {
+        score_afrag<BITS, NW>(wa, wb, s, tig, a0, a1, a2, a3);
+      }
 #pragma unroll
       for (int nt = 0; nt < NTN; ++nt) mma_u8s8(sacc[nt], a0, a1, a2, a3, bq[s][nt]);
     }
-    const int na = n0 + ra, nb = n0 + rb;
-    const bool va = na >= a.n_sink && na < a.n_tok, vb = nb >= a.n_sink && nb < a.n_tok;
-    const float2 kza = h2f(lds32(kzb + 4 * ra)), kzb2 = h2f(lds32(kzb + 4 * rb));
-    float2 vza = h2f(lds32(vzb + 4 * ra)), vzb2 = h2f(lds32(vzb + 4 * rb));
-    if (!va) vza = make_float2(0.0f, 0.0f);
-    if (!vb) vzb2 = make_float2(0.0f, 0.0f);
-    const float lga = __log2f(fmaxf(vza.x, kMinS)), lgb = __log2f(fmaxf(vzb2.x, kMinS));
+    bool va = true, vb = true;
+    if constexpr (!INTERIOR) {
+      va = n0 + g >= a.n_sink && n0 + g < a.n_tok;
+      vb = n0 + g + 8 >= a.n_sink && n0 + g + 8 < a.n_tok;
+    }
+    const float2 kza = h2f(ld4(kzb + 4 * g)), kzb2 = h2f(ld4(kzb + 4 * (g + 8)));
+    float2 vza = h2f(ld4(vzb + 4 * g)), vzb2 = h2f(ld4(vzb + 4 * (g + 8)));
+    if constexpr (!INTERIOR) {
+      if (!va) vza = make_float2(0.0f, 0.0f);
+      if (!vb) vzb2 = make_float2(0.0f, 0.0f);
+    }
+    const float lga = lg2_approx(fmaxf(vza.x, kMinS)), lgb = lg2_approx(fmaxf(vzb2.x, kMinS));
     uint32_t hla[NTN], hlb[NTN];
 #pragma unroll
     for (int nt = 0; nt < NTN; ++nt) {
-      const bool qv = 4 * nt + tig < GQ;
-      const float da = static_cast<float>(sacc[nt][0] + 256 * sacc[nt][1]);
-      const float db = static_cast<float>(sacc[nt][2] + 256 * sacc[nt][3]);
+      const bool qv = ALLQ || 4 * nt + tig < GQ;
+      // (the multiply variant's sums are 64x: exact multiples of 64, shifted back exactly)
+      const float da = static_cast<float>((sacc[nt][0] + 256 * sacc[nt][1]) >> (IMAD_SHIFT ? 6 : 0));
+      const float db = static_cast<float>((sacc[nt][2] + 256 * sacc[nt][3]) >> (IMAD_SHIFT ? 6 : 0));
       const float sa = __fmaf_rn(kza.x * sq[nt], da, __fmaf_rn(kza.y, qs[nt], 0.0f)) * a.scale;
       const float sb = __fmaf_rn(kzb2.x * sq[nt], db, __fmaf_rn(kzb2.y, qs[nt], 0.0f)) * a.scale;
       const bool oka = va && qv, okb = vb && qv;
@@ -478,7 +519,7 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
       blk = fmaxf(blk, __shfl_xor_sync(0xffffffffu, blk, 8));
       blk = fmaxf(blk, __shfl_xor_sync(0xffffffffu, blk, 16));
       if (blk > m_run[nt] + kFLazy) {  // uniform over the lanes of this query head
-        const float f = exp2f(m_run[nt] - blk);
+        const float f = ex2_approx(m_run[nt] - blk);
         m_run[nt] = blk;
         l_run[nt] *= f;
         z_run[nt] *= f;
@@ -487,8 +528,8 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[mt][nt][e] *= f;
       }
-      const float pa = oka ? exp2f(__fmaf_rn(sa, kLog2e, -m_run[nt])) : 0.0f;
-      const float pb = okb ? exp2f(__fmaf_rn(sb, kLog2e, -m_run[nt])) : 0.0f;
+      const float pa = oka ? ex2_approx(__fmaf_rn(sa, kLog2e, -m_run[nt])) : 0.0f;
+      const float pb = okb ? ex2_approx(__fmaf_rn(sb, kLog2e, -m_run[nt])) : 0.0f;
       l_run[nt] += pa + pb;
       z_run[nt] = __fmaf_rn(pa, vza.y, __fmaf_rn(pb, vzb2.y, z_run[nt]));
       hla[nt] = split_hi_lo(pa * vza.x);
@@ -504,10 +545,10 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
       bv1[nt] = __byte_perm(x2, x3, sel);
     }
     // ---- value A fragments and products
-    const uint32_t t0 = vcb + (16 * warp + 2 * tig) * RB;
+    const uint8_t* t0 = vcb + 2 * tig * RB;
     if constexpr (BITS == 2) {
-      const uint32_t u0 = lds32(t0 + 4 * g), u1 = lds32(t0 + RB + 4 * g);
-      const uint32_t u8 = lds32(t0 + 8 * RB + 4 * g), u9 = lds32(t0 + 9 * RB + 4 * g);
+      const uint32_t u0 = ld4(t0 + 4 * g), u1 = ld4(t0 + RB + 4 * g);
+      const uint32_t u8 = ld4(t0 + 8 * RB + 4 * g), u9 = ld4(t0 + 9 * RB + 4 * g);
       uint32_t y[2][4];
       y[0][0] = __byte_perm(u0, u1, 0x5410);  // channel 16 g + t, tokens 2 tig, 2 tig + 1
       y[0][1] = __byte_perm(u0, u1, 0x7632);  // channel 16 g + 8 + t
@@ -528,9 +569,9 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
       uint32_t y[2][2][4];  // [word g / g + 8][shift 0 / 8][register]
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
-        const uint32_t o = 4 * (g + 8 * w);
-        const uint32_t u0 = lds32(t0 + o), u1 = lds32(t0 + RB + o);
-        const uint32_t u8 = lds32(t0 + 8 * RB + o), u9 = lds32(t0 + 9 * RB + o);
+        const int o = 4 * (g + 8 * w);
+        const uint32_t u0 = ld4(t0 + o), u1 = ld4(t0 + RB + o);
+        const uint32_t u8 = ld4(t0 + 8 * RB + o), u9 = ld4(t0 + 9 * RB + o);
         y[w][0][0] = __byte_perm(u0, u1, 0x5410);
         y[w][0][1] = __byte_perm(u0, u1, 0x7632);
         y[w][0][2] = __byte_perm(u8, u9, 0x5410);
@@ -548,17 +589,23 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
         for (int nt = 0; nt < NTN; ++nt) mma_f16(acc[mt][nt], a0, a1, a2, a3, bv0[nt], bv1[nt]);
       }
     }
-    cp_async_wait_group<kFStages - 2>();  // this thread's scale / zero words of the next tile
-    if (!__syncthreads_and(ok)) break;
-    if (i + kFStages < n_tiles) issue(i + kFStages, st);
+  };
+
+  for (int i = 0; i < my_n; ++i) {
+    const int st = i % S;
+    cp_async_wait_group<S - 1>();  // this lane's copies of block i
+    __syncwarp();                  // ... and every other lane's
+    const int n0 = (k_begin + warp + i * kFWarps) * kFBlock;
+    const uint8_t* kcb = fdyn + (warp * S + st) * C::STAGE;
+    if (n0 >= a.n_sink && n0 + kFBlock <= a.n_tok) block(std::true_type{}, n0, kcb);
+    else block(std::false_type{}, n0, kcb);
+    __syncwarp();  // every lane has read the stage
+    if (i + S < my_n) issue(i + S, st);
     cp_async_commit();
   }
-  if (!ok) {
-    if (tid == 0)
-      for (int st = 0; st < kFStages; ++st)
-        for (uint32_t p = 0; p < 2; ++p) mbar_wait(&full[st], p, a.wait_ns, a.err);
-  }
   cp_async_wait_all();
+  // let the merge kernel start its independent prologue (it waits for this grid before reading partials)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #pragma unroll
   for (int nt = 0; nt < NTN; ++nt) {
 #pragma unroll
@@ -567,7 +614,7 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
       z_run[nt] += __shfl_xor_sync(0xffffffffu, z_run[nt], o);
     }
   }
-  __syncthreads();  // every stage consumed: the stage memory now holds the per-warp sums
+  __syncthreads();  // every warp is done with its stages: the stage memory now holds the per-warp sums
   float* accw = reinterpret_cast<float*>(fdyn);  // [kFWarps][GQ][D]
 #pragma unroll
   for (int nt = 0; nt < NTN; ++nt) {
@@ -598,25 +645,31 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? 2 : 1) k_attend_fused(con
     }
   }
   __syncthreads();
-  for (int e = tid; e < GQ * D; e += kFThreads) {
-    const int qh = e / D, j = e - qh * D;
+  if (tid < GQ) {  // per query head: the chunk's reference, each warp's factor, l and the Z term
+    const int qh = tid;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kFWarps; ++w) M = fmaxf(M, mw[w][qh]);
-    float s = 0.0f, L = 0.0f, Z = 0.0f;
+    float L = 0.0f, Z = 0.0f;
 #pragma unroll
     for (int w = 0; w < kFWarps; ++w) {
-      const float f = mw[w][qh] == -INFINITY ? 0.0f : exp2f(mw[w][qh] - M);
-      s = __fmaf_rn(f, accw[(w * GQ + qh) * D + j], s);
+      const float f = mw[w][qh] == -INFINITY ? 0.0f : ex2_approx(mw[w][qh] - M);
+      mw[w][qh] = f;
       L = __fmaf_rn(f, lw[w][qh], L);
       Z = __fmaf_rn(f, zw[w][qh], Z);
     }
+    zw[0][qh] = Z;
     const size_t row = (static_cast<size_t>(b) * a.Hq + h * GQ + qh) * a.n_chunks + c;
-    a.part_acc[row * D + j] = s + Z;
-    if (j == 0) {
-      a.part_ml[2 * row] = M;
-      a.part_ml[2 * row + 1] = L;
-    }
+    *reinterpret_cast<float2*>(a.part_ml + 2 * row) = make_float2(M, L);
+  }
+  __syncthreads();
+  for (int e = tid; e < GQ * D; e += kFThreads) {
+    const int qh = e / D, j = e - qh * D;
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kFWarps; ++w) s = __fmaf_rn(mw[w][qh], accw[(w * GQ + qh) * D + j], s);
+    const size_t row = (static_cast<size_t>(b) * a.Hq + h * GQ + qh) * a.n_chunks + c;
+    a.part_acc[row * D + j] = s + zw[0][qh];
   }
 }
 
@@ -635,10 +688,13 @@ struct MergeArgs {
 
 // One CTA per (batch, query head): sink scores (fp16 keys, exactly as the
 // score kernel forms them), the log-sum-exp merge of the chunks and sinks, the
-// inverse rotation and permutation, and the sink values.
+// inverse rotation and permutation, and the sink values. Launched as a
+// programmatic dependent of the fused kernel: everything up to the grid
+// dependency wait reads only the caller's inputs.
 __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
   __shared__ __align__(16) float qraw[D];
   __shared__ float ts[kFMaxSinks];
+  __shared__ float2 mls[kFMaxChunks];
   __shared__ float ys[2][D];
   __shared__ float nat[D];
   __shared__ float red[4];
@@ -647,6 +703,7 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
   const int b = bq / a.Hq, qh = bq % a.Hq, h = qh / a.GQ;
   const int ns = min(a.n_sink, a.n_tok);
   const size_t vh = static_cast<size_t>(b) * a.H + h;
+  const int pj = a.vperm ? a.vperm[static_cast<size_t>(h) * D + j] & (D - 1) : j;
   qraw[j] = __half2float(a.q[static_cast<size_t>(bq) * D + j]);
   __syncthreads();
   float mloc = -INFINITY;
@@ -654,23 +711,42 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
     const float s = sink_dot(qraw, a.ksink + (vh * a.n_sink + n) * D,
                              a.krope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane) *
                     a.scale;
-    const float t = s * kLog2e;
     if (lane == 0) ts[n] = s;
-    mloc = fmaxf(mloc, t);
+    mloc = fmaxf(mloc, s * kLog2e);
   }
-  const float* ml = a.part_ml + static_cast<size_t>(bq) * a.n_chunks * 2;
+  constexpr int kPre = 4;  // sink values held in registers from before the wait
+  float sv[kPre];
+#pragma unroll
+  for (int n = 0; n < kPre; ++n)
+    sv[n] = n < ns ? __half2float(a.vsink[(vh * a.n_sink + n) * D + j]) : 0.0f;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the fused kernel's partials are complete
+  const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + static_cast<size_t>(bq) * a.n_chunks;
   const float* pa = a.part_acc + static_cast<size_t>(bq) * a.n_chunks * D;
-  for (int c = 0; c < a.n_chunks; ++c) mloc = fmaxf(mloc, ml[2 * c]);
+  for (int c = j; c < a.n_chunks; c += kThreads) {
+    const float2 v = ml[c];
+    mls[c] = v;
+    mloc = fmaxf(mloc, v.x);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
   if (lane == 0) red[warp] = mloc;
   __syncthreads();
   const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
   float L = 0.0f, acc = 0.0f;
-  for (int c = 0; c < a.n_chunks; ++c) {
-    const float f = ml[2 * c] == -INFINITY ? 0.0f : exp2f(ml[2 * c] - M);
-    L = __fmaf_rn(ml[2 * c + 1], f, L);
-    acc = __fmaf_rn(pa[static_cast<size_t>(c) * D + j], f, acc);
+  for (int c0 = 0; c0 < a.n_chunks; c0 += 8) {  // eight loads in flight, then their weights
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = c0 + u < a.n_chunks ? pa[static_cast<size_t>(c0 + u) * D + j] : 0.0f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (c0 + u >= a.n_chunks) break;
+      const float2 m = mls[c0 + u];
+      const float f = m.x == -INFINITY ? 0.0f : ex2_approx(m.x - M);
+      L = __fmaf_rn(m.y, f, L);
+      acc = __fmaf_rn(v[u], f, acc);
+    }
   }
-  for (int n = 0; n < ns; ++n) L += exp2f(__fmaf_rn(ts[n], kLog2e, -M));
+  for (int n = 0; n < ns; ++n) L += ex2_approx(__fmaf_rn(ts[n], kLog2e, -M));
   const float invL = 1.0f / L;
   float y = acc * invL;  // sum_n p_n y_n, channel j of the rotated basis
   if (a.rot == KVQ_ROT_FWHT_HEAD) {  // x = H y / sqrt(D), Sylvester order, strides 1 .. 64
@@ -686,11 +762,14 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
     }
     y = ys[cur][j] * a.rscale;
   }
-  nat[a.vperm ? a.vperm[static_cast<size_t>(h) * D + j] & (D - 1) : j] = y;  // x[perm[j]] = y_j
+  nat[pj] = y;  // x[perm[j]] = y_j
   __syncthreads();
   float o = nat[j];
-  for (int n = 0; n < ns; ++n) {
-    const float p = exp2f(__fmaf_rn(ts[n], kLog2e, -M)) * invL;
+#pragma unroll
+  for (int n = 0; n < kPre; ++n)
+    if (n < ns) o = __fmaf_rn(ex2_approx(__fmaf_rn(ts[n], kLog2e, -M)) * invL, sv[n], o);
+  for (int n = kPre; n < ns; ++n) {
+    const float p = ex2_approx(__fmaf_rn(ts[n], kLog2e, -M)) * invL;
     o = __fmaf_rn(p, __half2float(a.vsink[(vh * a.n_sink + n) * D + j]), o);
   }
   a.out[static_cast<size_t>(bq) * D + j] = o;
@@ -698,15 +777,15 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
 
 template <int BITS, int GQ>
 kvq_status run_fused(FusedArgs& fa, const LaunchCtx& ctx, cudaStream_t st) {
-  constexpr size_t smem = static_cast<size_t>(kFStages) * kFTile * (2 * (128 * BITS / 8) + 8);
+  constexpr size_t smem = FusedCfg<BITS>::SMEM;
   const void* fn = reinterpret_cast<const void*>(k_attend_fused<BITS, GQ>);
   if (!set_smem_once(fn, smem)) return KVQ_ERR_CUDA;
   const int per_sm = occupancy_once(fn, kFThreads, smem);
   const int bh = fa.B * fa.H;
-  int want = ctx.num_sms * per_sm / bh;  // chunks per (batch, KV head) for about one wave
+  int want = ctx.num_sms * per_sm * KVQ_ATTEND_WAVES_NUM / (KVQ_ATTEND_WAVES_DEN * bh);  // chunks per (batch, KV head)
   want = want < 1 ? 1 : (want > kFMaxChunks ? kFMaxChunks : want);
-  fa.tiles_per_chunk = (fa.tiles + want - 1) / want;
-  fa.n_chunks = (fa.tiles + fa.tiles_per_chunk - 1) / fa.tiles_per_chunk;
+  fa.blocks_per_chunk = (fa.blocks + want - 1) / want;
+  fa.n_chunks = (fa.blocks + fa.blocks_per_chunk - 1) / fa.blocks_per_chunk;
   k_attend_fused<BITS, GQ><<<dim3(static_cast<unsigned>(fa.n_chunks), static_cast<unsigned>(bh)), kFThreads,
                              smem, st>>>(fa);
   return launch_status();
@@ -723,11 +802,27 @@ kvq_status fused_by_gq(FusedArgs& fa, int gq, const LaunchCtx& ctx, cudaStream_t
   }
 }
 
+// The merge as a programmatic dependent launch of the fused kernel.
+kvq_status launch_merge(const MergeArgs& ma, unsigned grid, cudaStream_t st) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_attend_merge, ma) != cudaSuccess) return KVQ_ERR_CUDA;
+  return launch_status();
+}
+
 bool fused_path(int bits, int group, int n_sink) {
   return (bits == 2 || bits == 4) && group == 128 && n_sink <= kFMaxSinks;
 }
 
-int fused_tiles(int n_tokens) { return (n_tokens + kFTile - 1) / kFTile; }
+int fused_tiles(int n_tokens) { return (n_tokens + kFBlock - 1) / kFBlock; }
 
 // Fixed scratch of kvq_attend_noalloc: a file-scope device array, reserved when
 // the module is loaded, so that entry point never allocates. 40 MiB holds the
@@ -785,7 +880,7 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
     fa.n_tok = n_tokens;
     fa.n_sink = dk.n_sink;
     fa.rot = dk.rot;
-    fa.tiles = tiles;
+    fa.blocks = tiles;
     fa.scale = scale;
     fa.rscale = static_cast<float>(1.0 / sqrt(static_cast<double>(D)));
     fa.q = static_cast<const __half*>(q);
@@ -797,8 +892,6 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
     uint8_t* w = static_cast<uint8_t*>(ws);
     fa.part_acc = reinterpret_cast<float*>(w);
     fa.part_ml = reinterpret_cast<float*>(w + align256(bq * max_chunks * D * 4));
-    fa.err = ctx.err;
-    fa.wait_ns = ctx.wait_ns;
     const int gq = q_heads / dk.heads;
     kvq_status s = dk.bits == 2 ? fused_by_gq<2>(fa, gq, ctx, st) : fused_by_gq<4>(fa, gq, ctx, st);
     if (s != KVQ_OK) return s;
@@ -822,8 +915,7 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
     ma.part_acc = fa.part_acc;
     ma.part_ml = fa.part_ml;
     ma.out = out;
-    k_attend_merge<<<static_cast<unsigned>(bq), kThreads, 0, st>>>(ma);
-    return launch_status();
+    return launch_merge(ma, static_cast<unsigned>(bq), st);
   }
   AttnArgs a{};
   a.B = dk.batch;

@@ -133,6 +133,10 @@ __device__ __forceinline__ void fence_async_smem() {
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t n) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
+// 16-byte async copy through L2 only; n < 16 fills the rest with zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t n) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 template <int N>
