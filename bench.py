@@ -234,6 +234,7 @@ class AttendStep:
     K and the V cache, then out = softmax(q . k) . v over every slot."""
 
     workload = "llama3_8b_gqa_attend"
+    kernels_per_step = 4  # two appends, the fused attention kernel and its merge
     # K and V caches are 75 MB, less than the 126 MB L2: flush it before every step
     l2_flush = True
 
@@ -260,6 +261,36 @@ class AttendStep:
 
     def launches(self):
         return [self.k.append, self.v.append, self.attend]
+
+
+class CalibrateStep:
+    """Channel-permutation calibration of the Llama-3-8B GQA keys (head-dim
+    variant: RoPE, then the abs-max over 4 x 32768 positions per head)."""
+
+    workload = "llama3_8b_calibrate"
+    kernels_per_step = 2  # abs-max and rank (plus a memset of the maxima)
+
+    def __init__(self, device):
+        import torch
+        from kv_cache_rotation_b200 import torch_api as TA
+        w = W.WORKLOADS["llama3_8b_gqa_score"]
+        self.x = torch.from_numpy(W.kv_tensor(w, "k")).to(device)
+        self.d = TA.make_desc(batch=w.B, heads=w.H, head_dim=w.D, tokens=w.T, bits=w.bits, group=w.group,
+                              rope=1, n_sink=w.n_sink, rot="fwht_head")
+        self.tb = TA.make_tables(rope_cs=TA.rope_table(w.T, w.D, device=device))
+        self.perm = torch.empty((w.H, w.D), dtype=torch.int16, device=device)
+        self.ws = TA.calibrate_workspace(self.d, device)
+        self.call = TA.bind_calibrate(self.d, self.x, self.tb, self.perm, self.ws)
+        nbytes = self.x.numel() * 2
+        self.alg = {"calibrate": nbytes + self.perm.numel() * 2}
+        self.fp16_equiv = {"calibrate": nbytes}
+        self.kernels = {"calibrate": "k_absmax"}
+        self.fp32_ops = {}
+        self.names = list(self.alg)
+        torch.cuda.synchronize(device)
+
+    def launches(self):
+        return [self.call]
 
 
 class EncDecStep:
@@ -360,6 +391,8 @@ def make_step(workload, device, batch=None):
         return DecodeScoreStep(device)
     if workload == "llama3_8b_gqa_attend":
         return AttendStep(device)
+    if workload == "llama3_8b_calibrate":
+        return CalibrateStep(device)
     return EncDecStep(workload, device, batch=batch)
 
 
@@ -558,7 +591,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": _config(world) if args.workload == "llama3_8b_gqa" else _other_config(args.workload, world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e_line,
-            "gpu_launches": nk * args.steps, "clocks": clocks, "kernels": kernels,
+            "gpu_launches": getattr(st, "kernels_per_step", nk) * args.steps, "clocks": clocks, "kernels": kernels,
             "status": K.kvq_status_str(status),
         }
         print(json.dumps(line))
@@ -601,6 +634,11 @@ def run_e2e(st, launches, dev, stream, steps, warmup):
 
 
 def _other_config(name, n_gpus):
+    if name == "llama3_8b_calibrate":
+        w = W.WORKLOADS["llama3_8b_gqa_score"]
+        return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T,
+                "input": "keys fp16, RoPE'd before the abs-max (head-dim variant)", "n_sink": w.n_sink,
+                "l2": "no flush (the 268 MB input is larger than L2)", "parallelism": f"replicas x{n_gpus}"}
     w = W.WORKLOADS[name]
     return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T, "q_heads": w.Hq,
             "rotation": w.rot, "quant": w.quant, "bits": w.bits, "group": w.group, "n_sink": w.n_sink,
@@ -622,7 +660,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--workload", default="llama3_8b_gqa",
                     choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "decode_score",
-                             "llama3_8b_gqa_attend", "tiny"],
+                             "llama3_8b_gqa_attend", "llama3_8b_calibrate", "tiny"],
                     help="which workload a step runs (the headline line is llama3_8b_gqa)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch of an encode/decode workload (small profiling captures)")

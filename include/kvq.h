@@ -186,6 +186,27 @@ kvq_status kvq_attend_noalloc(const kvq_desc* dk, const kvq_desc* dv, const void
 /* Workspace bytes kvq_attend needs for these arguments; 0 if they are invalid or unsupported. */
 size_t kvq_attend_workspace_bytes(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads, int32_t n_tokens);
 
+/* Channel permutation by abs-max ([RotateKV] outlier-aware rotation: channel reordering before
+ * the FWHT). For each head h, a_j = max over the B batches and the positions t0..t0+T-1 that are
+ * not sinks (position >= n_sink) of |y_j|, where y is the fp32 input of the permutation step:
+ * RoPE_m(x), with kvq_encode's fp32 arithmetic, for rope = 1 and rot NONE or FWHT_HEAD (RoPE comes
+ * before the permutation there); x itself otherwise (values; FWHT_GROUP permutes the raw input).
+ * perm_out[h] lists the channels by descending a_j, equal a_j in ascending channel order: a table
+ * for kvq_tables.perm.
+ *   x          half [B][H][T][head_dim], 16-byte aligned (the tensor kvq_encode would take)
+ *   tb         rope_cs as for kvq_encode when RoPE applies (other fields unused)
+ *   perm_out   int16 [H][head_dim], 16-byte aligned, overwritten
+ *   workspace  device memory of at least kvq_calibrate_workspace_bytes(d) bytes (H * head_dim * 4),
+ *              256-byte aligned; its contents do not matter (the call zeroes it on the stream first),
+ *              the caller owns it
+ * The result is integer and exact: it does not depend on scheduling. KVQ_ERR_UNSUPPORTED for
+ * ISO_SO4 (no permutation there) and for B*T >= 2^31. */
+kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables* tb, int16_t* perm_out,
+                              void* workspace, size_t workspace_bytes, kvq_stream_t stream);
+
+/* Workspace bytes kvq_calibrate_perm needs for d; 0 if d is invalid or unsupported. */
+size_t kvq_calibrate_workspace_bytes(const kvq_desc* d);
+
 /* Bytes of one packed buffer (KVQ_FIELD_*) for this descriptor; 0 if the field is unused or
  * the descriptor is invalid. */
 size_t kvq_packed_bytes(const kvq_desc* d, int32_t field);

@@ -23,6 +23,7 @@ KVQ_Q_MINMAX, KVQ_Q_CODEBOOK = 0, 1
 KVQ_FIELD_CODES, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_FIELD_NORM = range(4)
 
 EXPORTED = ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_attend_workspace_bytes",
+            "kvq_calibrate_perm", "kvq_calibrate_workspace_bytes",
             "kvq_packed_bytes", "kvq_rope_table", "kvq_lloyd_max_codebook", "kvq_check", "kvq_debug_expire_wait",
             "kvq_status_str", "kvq_version")
 
@@ -63,6 +64,9 @@ def _load():
                              P(kvq_tables), i32, ctypes.c_float, vp, vp, ctypes.c_size_t, st]
     L.kvq_attend_noalloc.argtypes = [P(kvq_desc), P(kvq_desc), vp, i32, P(kvq_packed), P(kvq_tables),
                                      P(kvq_packed), P(kvq_tables), i32, ctypes.c_float, vp, st]
+    L.kvq_calibrate_perm.argtypes = [P(kvq_desc), vp, P(kvq_tables), vp, vp, ctypes.c_size_t, st]
+    L.kvq_calibrate_workspace_bytes.argtypes = [P(kvq_desc)]
+    L.kvq_calibrate_workspace_bytes.restype = ctypes.c_size_t
     L.kvq_attend_workspace_bytes.argtypes = [P(kvq_desc), P(kvq_desc), i32, i32]
     L.kvq_attend_workspace_bytes.restype = ctypes.c_size_t
     L.kvq_packed_bytes.argtypes = [P(kvq_desc), i32]
@@ -74,7 +78,8 @@ def _load():
     L.kvq_status_str.argtypes = [i32]
     L.kvq_status_str.restype = ctypes.c_char_p
     L.kvq_version.restype = i32
-    for n in ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_rope_table",
+    for n in ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_calibrate_perm",
+              "kvq_rope_table",
               "kvq_lloyd_max_codebook",
               "kvq_check", "kvq_debug_expire_wait"):
         getattr(L, n).restype = i32
@@ -115,6 +120,15 @@ def kvq_attend_noalloc(dk: kvq_desc, dv: kvq_desc, q: int, q_heads: int, k_cache
     return lib.kvq_attend_noalloc(ctypes.byref(dk), ctypes.byref(dv), q, q_heads, ctypes.byref(k_cache),
                                   ctypes.byref(tk), ctypes.byref(v_cache), ctypes.byref(tv), n_tokens, scale, out,
                                   stream)
+
+
+def kvq_calibrate_perm(d: kvq_desc, x: int, tb: kvq_tables, perm_out: int, workspace: int, workspace_bytes: int,
+                       stream: int = 0) -> int:
+    return lib.kvq_calibrate_perm(ctypes.byref(d), x, ctypes.byref(tb), perm_out, workspace, workspace_bytes, stream)
+
+
+def kvq_calibrate_workspace_bytes(d: kvq_desc) -> int:
+    return lib.kvq_calibrate_workspace_bytes(ctypes.byref(d))
 
 
 def kvq_attend_workspace_bytes(dk: kvq_desc, dv: kvq_desc, q_heads: int, n_tokens: int) -> int:

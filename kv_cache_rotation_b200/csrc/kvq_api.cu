@@ -320,6 +320,30 @@ kvq_status kvq_attend_noalloc(const kvq_desc* dk, const kvq_desc* dv, const void
                        reinterpret_cast<cudaStream_t>(stream), ctx);
 }
 
+size_t kvq_calibrate_workspace_bytes(const kvq_desc* d) {
+  if (check_desc(d) != KVQ_OK || d->rot == KVQ_ROT_ISO_SO4) return 0;
+  return calibrate_workspace_bytes(*d);
+}
+
+kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables* tb, int16_t* perm_out,
+                              void* workspace, size_t workspace_bytes, kvq_stream_t stream) {
+  kvq_status s = check_desc(d);
+  if (s != KVQ_OK) return s;
+  if (d->rot == KVQ_ROT_ISO_SO4) return KVQ_ERR_UNSUPPORTED;  // no permutation in that variant
+  if (!x || !perm_out || !workspace || !tb) return KVQ_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(perm_out, 16) || !aligned(workspace, 256)) return KVQ_ERR_ALIGN;
+  if (workspace_bytes < calibrate_workspace_bytes(*d)) return KVQ_ERR_INVALID;
+  if (calibrate_rope(*d)) {
+    if (!tb->rope_cs) return KVQ_ERR_INVALID;
+    if (!aligned(tb->rope_cs, 16)) return KVQ_ERR_ALIGN;
+    if (tb->rope_rows < static_cast<int64_t>(d->t0) + d->tokens || tb->rope_rows <= 0) return KVQ_ERR_INVALID;
+  }
+  if (static_cast<int64_t>(d->batch) * d->tokens >= (int64_t(1) << 31)) return KVQ_ERR_UNSUPPORTED;
+  LaunchCtx ctx;
+  if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
+  return launch_calibrate(*d, x, *tb, perm_out, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t kvq_packed_bytes(const kvq_desc* d, int32_t field) {
   if (!d) return 0;
   kvq_desc dd = *d;

@@ -369,7 +369,7 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t y, uint32_t msk) {
 __device__ __forceinline__ float2 h2f(uint32_t w) { return __half22float2(*reinterpret_cast<const __half2*>(&w)); }
 
 template <int BITS, int GQ>
-__global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 2) k_attend_fused(const FusedArgs a) {
+__global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 1) k_attend_fused(const FusedArgs a) {
   using C = FusedCfg<BITS>;
   constexpr int D = 128;
   constexpr int RB = C::RB;
@@ -396,23 +396,44 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 2) k_at
   const int my_n = nk > warp ? (nk - warp + kFWarps - 1) / kFWarps : 0;  // blocks k_begin + warp + 8 i
   const size_t rec0 = static_cast<size_t>(bh) * a.t_cap;
   const uint32_t wbase = smem_u32(fdyn) + warp * (S * C::STAGE);
+  // The merge kernel may launch once every CTA of this grid has started (all are resident by then, so its
+  // CTAs never hold slots this grid still needs); it runs its input-only prologue beside this grid and
+  // waits for this grid's completion before reading any partial.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // block i of this warp into stage st: codes 16 bytes per lane, scale / zero 4 bytes (zero past n_tok)
+  // per-lane sources of this warp's first block; consecutive blocks of a warp are kFWarps blocks apart
+  constexpr size_t kStep = static_cast<size_t>(kFWarps) * kFBlock;  // records between a warp's blocks
+  const int n_first = (k_begin + warp) * kFBlock;
+  const size_t rec_first = rec0 + n_first;
+  const uint8_t* kc_src = a.kcodes + rec_first * RB + 16 * lane;
+  const uint8_t* vc_src = a.vcodes + rec_first * RB + 16 * lane;
+  const uint32_t* sz_src = (lane < kFBlock ? a.ksz : a.vsz) + rec_first + (lane & (kFBlock - 1));
+  const uint32_t sz_dst = 2 * kFBlock * RB + 4 * lane;
   auto issue = [&](int i, int st) {
-    const int n0 = (k_begin + warp + i * kFWarps) * kFBlock;
+    const int n0 = n_first + i * static_cast<int>(kStep);
+    const size_t roff = static_cast<size_t>(i) * kStep;
     const uint32_t sb = wbase + st * C::STAGE;
+    if (n0 + kFBlock <= a.n_tok) {  // the whole block exists (uniform over the warp)
 #pragma unroll
-    for (int r = 0; r < CPL; ++r) {
-      const int off = 16 * (lane + 32 * r);
-      const bool live = n0 + off / RB < a.n_tok;
-      const size_t src = (rec0 + n0) * RB + (live ? off : 0);
-      cp_async16(sb + off, a.kcodes + src, live ? 16u : 0u);
-      cp_async16(sb + kFBlock * RB + off, a.vcodes + src, live ? 16u : 0u);
+      for (int r = 0; r < CPL; ++r) {
+        cp_async16(sb + 512 * r + 16 * lane, kc_src + roff * RB + 512 * r, 16u);
+        cp_async16(sb + kFBlock * RB + 512 * r + 16 * lane, vc_src + roff * RB + 512 * r, 16u);
+      }
+      cp_async4(sb + sz_dst, sz_src + roff, 4u);
+    } else {  // last block: zero past n_tok, sources kept inside the cache
+#pragma unroll
+      for (int r = 0; r < CPL; ++r) {
+        const int off = 16 * (lane + 32 * r);
+        const bool live = n0 + off / RB < a.n_tok;
+        const size_t src = (rec0 + n0) * RB + (live ? off : 0);
+        cp_async16(sb + off, a.kcodes + src, live ? 16u : 0u);
+        cp_async16(sb + kFBlock * RB + off, a.vcodes + src, live ? 16u : 0u);
+      }
+      const int tok = lane & (kFBlock - 1);
+      const bool live = n0 + tok < a.n_tok;
+      cp_async4(sb + sz_dst, (lane < kFBlock ? a.ksz : a.vsz) + rec0 + n0 + (live ? tok : 0), live ? 4u : 0u);
     }
-    const int tok = lane & (kFBlock - 1);
-    const bool live = n0 + tok < a.n_tok;
-    cp_async4(sb + 2 * kFBlock * RB + 4 * lane, (lane < kFBlock ? a.ksz : a.vsz) + rec0 + n0 + (live ? tok : 0),
-              live ? 4u : 0u);
   };
 #pragma unroll
   for (int i = 0; i < S; ++i) {
@@ -473,11 +494,11 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 2) k_at
       wa[4 * k] = ua.x; wa[4 * k + 1] = ua.y; wa[4 * k + 2] = ua.z; wa[4 * k + 3] = ua.w;
       wb[4 * k] = ub.x; wb[4 * k + 1] = ub.y; wb[4 * k + 2] = ub.z; wb[4 * k + 3] = ub.w;
     }
-    int sacc[NTN][4];
+    int sacc[NTN][4], sacc2[NTN][4];  // k-steps 0, 2 and 1, 3: two independent product chains
 #pragma unroll
     for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0;
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
       uint32_t a0, a1, a2, a3;
@@ -490,8 +511,12 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 2) k_at
         score_afrag<BITS, NW>(wa, wb, s, tig, a0, a1, a2, a3);
       }
 #pragma unroll
-      for (int nt = 0; nt < NTN; ++nt) mma_u8s8(sacc[nt], a0, a1, a2, a3, bq[s][nt]);
+      for (int nt = 0; nt < NTN; ++nt) mma_u8s8((s & 1) ? sacc2[nt] : sacc[nt], a0, a1, a2, a3, bq[s][nt]);
     }
+#pragma unroll
+    for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
     bool va = true, vb = true;
     if constexpr (!INTERIOR) {
       va = n0 + g >= a.n_sink && n0 + g < a.n_tok;
@@ -591,21 +616,20 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 2) k_at
     }
   };
 
+  int st = 0;
   for (int i = 0; i < my_n; ++i) {
-    const int st = i % S;
     cp_async_wait_group<S - 1>();  // this lane's copies of block i
     __syncwarp();                  // ... and every other lane's
-    const int n0 = (k_begin + warp + i * kFWarps) * kFBlock;
+    const int n0 = n_first + i * static_cast<int>(kStep);
     const uint8_t* kcb = fdyn + (warp * S + st) * C::STAGE;
     if (n0 >= a.n_sink && n0 + kFBlock <= a.n_tok) block(std::true_type{}, n0, kcb);
     else block(std::false_type{}, n0, kcb);
     __syncwarp();  // every lane has read the stage
     if (i + S < my_n) issue(i + S, st);
     cp_async_commit();
+    st = st + 1 == S ? 0 : st + 1;
   }
   cp_async_wait_all();
-  // let the merge kernel start its independent prologue (it waits for this grid before reading partials)
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #pragma unroll
   for (int nt = 0; nt < NTN; ++nt) {
 #pragma unroll
@@ -733,12 +757,12 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
   __syncthreads();
   const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
   float L = 0.0f, acc = 0.0f;
-  for (int c0 = 0; c0 < a.n_chunks; c0 += 8) {  // eight loads in flight, then their weights
-    float v[8];
+  for (int c0 = 0; c0 < a.n_chunks; c0 += 16) {  // sixteen loads in flight, then their weights
+    float v[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = c0 + u < a.n_chunks ? pa[static_cast<size_t>(c0 + u) * D + j] : 0.0f;
+    for (int u = 0; u < 16; ++u) v[u] = c0 + u < a.n_chunks ? pa[static_cast<size_t>(c0 + u) * D + j] : 0.0f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       if (c0 + u >= a.n_chunks) break;
       const float2 m = mls[c0 + u];
       const float f = m.x == -INFINITY ? 0.0f : ex2_approx(m.x - M);

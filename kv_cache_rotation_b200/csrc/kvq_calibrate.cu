@@ -1,0 +1,160 @@
+// Channel permutation by abs-max ("RotateKV: Accurate and Robust 2-Bit KV Cache
+// Quantization for LLMs via Outlier-Aware Adaptive Rotations": outlier-aware
+// rotation, channel reordering before the FWHT). For each head h,
+//   a_j = max over the batches and the non-sink positions of |y_j|,
+// y = the fp32 input of the permutation step: RoPE_m(x) for keys of the
+// head-dim variants (the permutation follows RoPE there), x itself otherwise
+// (values, and the grouped variant, whose permutation acts on the raw input).
+// perm[h] lists the channels by descending a_j; equal a_j keep ascending
+// channel order.
+//
+// A memset and two launches. k_absmax: CTA = (chunk of token rows, head);
+// each thread owns 8 channels of a row (16-byte loads, four rows in flight),
+// applies RoPE in registers with the encoder's fp32 order, and keeps a running
+// |y| maximum; the CTA's maxima go to the zeroed [H][D] workspace by atomicMax
+// on the fp32 bit patterns (for non-negative floats the unsigned order is the
+// numeric order, and a maximum does not depend on the order of the updates).
+// k_perm_rank: one CTA per head ranks the channels,
+// rank_j = #{k : a_k > a_j or (a_k = a_j and k < j)}, perm[rank_j] = j.
+#include "kvq_device.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxChunks = 64;
+constexpr int kMinRows = 256;  // token rows per chunk, at least
+
+struct CalArgs {
+  int H, T, t0, n_sink, rope, rows, rows_per_chunk;
+  FastDiv div_t;
+  const __half* x;
+  const float* rope_cs;
+  uint32_t* amax;  // [H][D]: fp32 bit patterns of the running maxima (zeroed before k_absmax)
+  int16_t* perm;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
+  constexpr int TPR = D / 8;           // threads per row
+  constexpr int RPI = kThreads / TPR;  // rows in flight per CTA iteration
+  __shared__ float red[RPI][D];
+  const int tid = threadIdx.x, cg = tid % TPR, rl = tid / TPR;
+  const int h = blockIdx.y;
+  const int r0 = blockIdx.x * a.rows_per_chunk;
+  const int r1 = min(r0 + a.rows_per_chunk, a.rows);
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+  constexpr int U = 4;  // rows per thread in flight
+  for (int r = r0 + rl; r < r1; r += U * RPI) {  // row r = (batch b, token t)
+    uint4 raw[U];
+    float4 c0[U], c1[U];
+    bool live[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int rr = r + u * RPI;
+      const int b = static_cast<int>(a.div_t.div(static_cast<uint32_t>(rr)));
+      const int t = rr - b * a.T;
+      const int pos = a.t0 + t;
+      live[u] = rr < r1 && pos >= a.n_sink;
+      raw[u] = live[u] ? __ldg(reinterpret_cast<const uint4*>(
+                             a.x + ((static_cast<size_t>(b) * a.H + h) * a.T + t) * D) + cg)
+                       : make_uint4(0, 0, 0, 0);
+      if (a.rope && live[u]) {  // pairs 4 cg .. 4 cg + 3 of position pos
+        const float4* cs = reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(pos) * D) + 2 * cg;
+        c0[u] = __ldg(cs);
+        c1[u] = __ldg(cs + 1);
+      } else {
+        c0[u] = c1[u] = make_float4(1.0f, 0.0f, 1.0f, 0.0f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float v[8];
+      h8_to_f32(raw[u], v);
+      if (a.rope) {
+        rope_fwd(v[0], v[1], c0[u].x, c0[u].y);
+        rope_fwd(v[2], v[3], c0[u].z, c0[u].w);
+        rope_fwd(v[4], v[5], c1[u].x, c1[u].y);
+        rope_fwd(v[6], v[7], c1[u].z, c1[u].w);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(v[i]));  // rows not live hold zeros
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[rl][8 * cg + i] = m[i];
+  __syncthreads();
+  if (tid < D) {
+    float mx = 0.0f;
+#pragma unroll 8
+    for (int k = 0; k < RPI; ++k) mx = fmaxf(mx, red[k][tid]);
+    atomicMax(a.amax + static_cast<size_t>(h) * D + tid, __float_as_uint(mx));
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) k_perm_rank(const CalArgs a) {
+  __shared__ float s_a[D];
+  const int j = threadIdx.x, h = blockIdx.x;
+  const float aj = __uint_as_float(a.amax[static_cast<size_t>(h) * D + j]);
+  s_a[j] = aj;
+  __syncthreads();
+  int rank = 0;
+#pragma unroll 8
+  for (int k = 0; k < D; ++k) {
+    const float ak = s_a[k];
+    rank += (ak > aj || (ak == aj && k < j)) ? 1 : 0;
+  }
+  a.perm[static_cast<size_t>(h) * D + rank] = static_cast<int16_t>(j);
+}
+
+int chunks_for(int64_t rows) {
+  int64_t c = (rows + kMinRows - 1) / kMinRows;
+  if (c < 1) c = 1;
+  return static_cast<int>(c < kMaxChunks ? c : kMaxChunks);
+}
+
+template <int D>
+kvq_status run(CalArgs& a, int chunks, cudaStream_t st) {
+  if (cudaMemsetAsync(a.amax, 0, static_cast<size_t>(a.H) * D * sizeof(uint32_t), st) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  k_absmax<D><<<dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(a.H)), kThreads, 0, st>>>(a);
+  kvq_status s = launch_status();
+  if (s != KVQ_OK) return s;
+  k_perm_rank<D><<<static_cast<unsigned>(a.H), D, 0, st>>>(a);
+  return launch_status();
+}
+
+}  // namespace
+
+bool calibrate_rope(const kvq_desc& d) {
+  return d.rope != 0 && (d.rot == KVQ_ROT_NONE || d.rot == KVQ_ROT_FWHT_HEAD);
+}
+
+size_t calibrate_workspace_bytes(const kvq_desc& d) { return static_cast<size_t>(d.heads) * d.head_dim * 4; }
+
+kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& tb, int16_t* perm, void* ws,
+                            cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(d.batch) * d.tokens;
+  if (rows >= (int64_t(1) << 31)) return KVQ_ERR_UNSUPPORTED;
+  CalArgs a{};
+  a.H = d.heads;
+  a.T = d.tokens;
+  a.t0 = d.t0;
+  a.n_sink = d.n_sink;
+  a.rope = calibrate_rope(d) ? 1 : 0;
+  a.rows = static_cast<int>(rows);
+  const int chunks = chunks_for(rows);
+  a.rows_per_chunk = static_cast<int>((rows + chunks - 1) / chunks);
+  a.div_t = FastDiv(static_cast<uint32_t>(d.tokens > 0 ? d.tokens : 1));
+  a.x = static_cast<const __half*>(x);
+  a.rope_cs = tb.rope_cs;
+  a.amax = static_cast<uint32_t*>(ws);
+  a.perm = perm;
+  return d.head_dim == 128 ? run<128>(a, chunks, st) : run<64>(a, chunks, st);
+}
+
+}  // namespace kvq

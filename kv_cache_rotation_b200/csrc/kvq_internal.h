@@ -46,6 +46,10 @@ kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq
 kvq_status launch_debug_wait(uint64_t limit_ns, cudaStream_t st, const LaunchCtx& ctx);
 size_t attend_workspace_bytes(const kvq_desc& dk, int q_heads, int n_tokens);
 size_t attend_scratch_bytes();
+bool calibrate_rope(const kvq_desc& d);
+size_t calibrate_workspace_bytes(const kvq_desc& d);
+kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& tb, int16_t* perm, void* ws,
+                            cudaStream_t st);
 void* attend_scratch();
 kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, int q_heads,
                          const kvq_packed& kc, const kvq_tables& tk, const kvq_packed& vc, const kvq_tables& tv,

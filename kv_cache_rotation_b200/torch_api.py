@@ -158,6 +158,42 @@ def attend_noalloc(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed
                              tv.struct(), n_tokens, scale, out.data_ptr(), _stream(stream)), "kvq_attend_noalloc")
 
 
+def calibrate_workspace(d: kvq_desc, device="cuda") -> torch.Tensor:
+    """A workspace tensor for kvq_calibrate_perm."""
+    from . import kvq_calibrate_workspace_bytes
+    nb = kvq_calibrate_workspace_bytes(d)
+    if nb == 0:
+        raise ValueError("kvq_calibrate_perm: invalid or unsupported descriptor")
+    return torch.empty(nb, dtype=torch.uint8, device=device)
+
+
+def calibrate_perm(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Tensor = None,
+                   workspace: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """Channel permutation by abs-max (int16 [H][head_dim]) for kvq_tables.perm."""
+    from . import kvq_calibrate_perm
+    if perm_out is None:
+        perm_out = torch.empty((d.heads, d.head_dim), dtype=torch.int16, device=x.device)
+    if workspace is None:
+        workspace = calibrate_workspace(d, x.device)
+    check(kvq_calibrate_perm(d, x.data_ptr(), tb.struct(), perm_out.data_ptr(), workspace.data_ptr(),
+                             workspace.numel(), _stream(stream)), "kvq_calibrate_perm")
+    return perm_out
+
+
+def bind_calibrate(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Tensor, workspace: torch.Tensor,
+                   stream=None):
+    from . import lib
+    tbs, st = tb.struct(), _stream(stream)
+    args = (ctypes.byref(d), x.data_ptr(), ctypes.byref(tbs), perm_out.data_ptr(), workspace.data_ptr(),
+            workspace.numel(), st)
+    keep = (d, x, tb, tbs, perm_out, workspace)
+
+    def call():
+        check(lib.kvq_calibrate_perm(*args), "kvq_calibrate_perm")
+    call.keep = keep
+    return call
+
+
 def bind_attend(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, tk: Tables, v_packed: Packed,
                 tv: Tables, n_tokens: int, scale: float, out: torch.Tensor, workspace: torch.Tensor, stream=None):
     from . import lib

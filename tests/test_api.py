@@ -168,3 +168,27 @@ def test_rope_table_matches_oracle(orc):
 def test_codebook_matches_oracle(orc, bits):
     cb = TA.lloyd_max_codebook(bits, 128, device="cpu").numpy()
     assert np.array_equal(cb, orc.codebook(bits, 128))
+
+
+def test_calibrate_argument_checks():
+    d = _desc(tokens=40, rope=1)
+    nb = K.kvq_calibrate_workspace_bytes(d)
+    assert nb == 8 * 128 * 4  # the fp32 maxima of 8 heads x 128 channels
+    tb = K.kvq_tables()
+    tb.rope_cs, tb.rope_rows = 256, 40
+    ok = (256, tb, 512, 1024, nb, 0)
+    assert K.kvq_calibrate_perm(_desc(batch=0), *ok) == K.KVQ_ERR_INVALID
+    assert K.kvq_calibrate_perm(d, 0, tb, 512, 1024, nb, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_calibrate_perm(d, 258, tb, 512, 1024, nb, 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_calibrate_perm(d, 256, tb, 514, 1024, nb, 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_calibrate_perm(d, 256, tb, 512, 1040, nb, 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_calibrate_perm(d, 256, tb, 512, 1024, nb - 4, 0) == K.KVQ_ERR_INVALID
+    short = K.kvq_tables()
+    short.rope_cs, short.rope_rows = 256, 39  # positions 0..39 need 40 rows
+    assert K.kvq_calibrate_perm(d, 256, short, 512, 1024, nb, 0) == K.KVQ_ERR_INVALID
+    iso = _desc(rot="iso", quant="codebook", bits=3, group=128)
+    assert K.kvq_calibrate_workspace_bytes(iso) == 0
+    assert K.kvq_calibrate_perm(iso, 256, tb, 512, 1024, nb, 0) == K.KVQ_ERR_UNSUPPORTED
+    # grouped keys permute the raw input: no RoPE table needed
+    g = _desc(tokens=40, rope=1, rot="fwht_group", group_heads=8, group=128)
+    assert K.kvq_calibrate_workspace_bytes(g) == nb
