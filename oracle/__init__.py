@@ -93,6 +93,8 @@ def lib():
                                  u8p, u16p, u16p, i16p, ci, u8p, u16p, u16p, i16p, ci, cd, f64p]
         L.orc_calibrate_perm.restype = ci
         L.orc_calibrate_perm.argtypes = [ci, ci, ci, ci, i64p, ci, ci, cd, u16p, i16p]
+        L.orc_pair_energy.restype = ci
+        L.orc_pair_energy.argtypes = [ci, ci, ci, ci, u16p, ctypes.POINTER(ctypes.c_uint64), i16p]
         _lib = L
     return _lib
 
@@ -327,3 +329,21 @@ def calibrate_perm(x, pos, *, rope=0, n_sink=0, base=10000.0):
     lib().orc_calibrate_perm(B, H, T, D, _p(pos, ctypes.c_int64), rope, n_sink, base,
                              _p(x, ctypes.c_uint16), _p(perm, ctypes.c_int16))
     return perm
+
+
+def pair_energy(x):
+    """orc_pair_energy: per head, the exact energy of each RoPE pair summed over
+    batches and tokens, as Python ints in units of 2^-48, and the pairs ranked
+    by descending energy (ties in ascending pair order). x: uint16 [B][H][T][D]."""
+    x = np.ascontiguousarray(x, np.uint16)
+    B, H, T, D = x.shape
+    e = np.zeros((H, D // 2, 2), np.uint64)
+    rank = np.zeros((H, D // 2), np.int16)
+    if lib().orc_pair_energy(B, H, T, D, _p(x, ctypes.c_uint16), _p(e, ctypes.c_uint64), _p(rank, ctypes.c_int16)):
+        raise MemoryError("oracle pair energy")
+    return e, rank
+
+
+def energy_ints(e):
+    """(lo, hi) uint64 pairs -> Python ints."""
+    return [[int(p[0]) | (int(p[1]) << 64) for p in row] for row in e]

@@ -778,3 +778,48 @@ int orc_calibrate_perm(int B, int H, int T, int D, const int64_t* pos, int rope,
   free(a);
   return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Energy of each RoPE frequency pair ([EliteKV] §3.1 frequency energy
+ * analysis): E_i = sum over the cached keys of |K_{2i}|^2 + |K_{2i+1}|^2,
+ * here per head, summed over batches and tokens of the fp16 keys. A pair's
+ * norm is what RoPE preserves, so the energy is taken on the keys as given.
+ * Exact: an fp16 value is M 2^(e) with an 11-bit M, so its square is an
+ * integer multiple of 2^-48 below 2^80; the sum is kept as an unsigned
+ * 128-bit integer in units of 2^-48 (energy[2k] = low 64 bits, energy[2k+1]
+ * = high 64 bits). rank lists the pairs by descending energy, equal
+ * energies in ascending pair order.
+ * ---------------------------------------------------------------------- */
+static unsigned __int128 half_square_units(uint16_t h) {
+  unsigned e = (h >> 10) & 31u, m = h & 1023u;
+  if (e == 31) return 0; /* inf / nan: not a finite key, contributes nothing */
+  uint64_t M = e ? (m | 1024u) : m;
+  unsigned shift = e ? 2 * e - 2 : 0; /* v = M 2^(e-25) (normal) or M 2^-24 */
+  return ((unsigned __int128)(M * M)) << shift;
+}
+
+int orc_pair_energy(int B, int H, int T, int D, const uint16_t* x, uint64_t* energy, int16_t* rank) {
+  int P = D / 2;
+  unsigned __int128* acc = (unsigned __int128*)calloc((size_t)H * P, sizeof(unsigned __int128));
+  if (!acc) return 1;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int t = 0; t < T; ++t) {
+        const uint16_t* xv = x + ((size_t)(b * H + h) * T + t) * D;
+        for (int i = 0; i < P; ++i) acc[h * P + i] += half_square_units(xv[2 * i]) + half_square_units(xv[2 * i + 1]);
+      }
+  for (int h = 0; h < H; ++h)
+    for (int i = 0; i < P; ++i) {
+      unsigned __int128 v = acc[h * P + i];
+      energy[2 * (h * P + i)] = (uint64_t)v;
+      energy[2 * (h * P + i) + 1] = (uint64_t)(v >> 64);
+      int r = 0;
+      for (int k = 0; k < P; ++k) {
+        unsigned __int128 w = acc[h * P + k];
+        if (w > v || (w == v && k < i)) ++r;
+      }
+      rank[h * P + r] = (int16_t)i;
+    }
+  free(acc);
+  return 0;
+}
