@@ -63,10 +63,10 @@ def lib():
             getattr(L, n).restype = ctypes.c_uint16
             getattr(L, n).argtypes = [ctypes.c_float]
         L.orc_rope_theta.restype = cd
-        L.orc_rope_theta.argtypes = [ci, ci, cd]
-        L.orc_rope_cs.argtypes = [ctypes.c_int64, ci, cd, f32p, f32p]
+        L.orc_rope_theta.argtypes = [ci, ci, cd, ci]
+        L.orc_rope_cs.argtypes = [ctypes.c_int64, ci, cd, ci, f32p, f32p]
         L.orc_rope_apply_f32.argtypes = [f32p, f32p, f32p, f32p, ci]
-        L.orc_rope_apply_f64.argtypes = [f64p, f64p, ctypes.c_int64, ci, cd, ci]
+        L.orc_rope_apply_f64.argtypes = [f64p, f64p, ctypes.c_int64, ci, cd, ci, ci]
         L.orc_fwht_f32.argtypes = [f32p, ci]
         L.orc_fwht_f64.argtypes = [f64p, ci]
         L.orc_fwht_scale_f32.restype = ctypes.c_float
@@ -108,14 +108,19 @@ def float_to_half(f: float, mode: str = "rn") -> int:
     return getattr(lib(), f"orc_float_to_half_{mode}")(float(f))
 
 
-def rope_theta(i: int, d: int, base: float = 10000.0) -> float:
-    return lib().orc_rope_theta(i, d, base)
+# RoPE frequency tables, passed where a rope flag goes: ROPE_STD (1) the
+# standard theta_i = base^(-2i/d), ROPE_FREQ_AWARE (2) the frequency-aware table.
+ROPE_STD, ROPE_FREQ_AWARE = 1, 2
 
 
-def rope_cs(m: int, d: int, base: float = 10000.0):
+def rope_theta(i: int, d: int, base: float = 10000.0, mode: int = ROPE_STD) -> float:
+    return lib().orc_rope_theta(i, d, base, mode)
+
+
+def rope_cs(m: int, d: int, base: float = 10000.0, mode: int = ROPE_STD):
     c = np.zeros(d // 2, np.float32)
     s = np.zeros(d // 2, np.float32)
-    lib().orc_rope_cs(int(m), d, base, _p(c, ctypes.c_float), _p(s, ctypes.c_float))
+    lib().orc_rope_cs(int(m), d, base, mode, _p(c, ctypes.c_float), _p(s, ctypes.c_float))
     return c, s
 
 
@@ -128,10 +133,10 @@ def rope_f32(x, c, s):
     return y
 
 
-def rope_f64(x, m: int, base: float = 10000.0, inverse: bool = False):
+def rope_f64(x, m: int, base: float = 10000.0, inverse: bool = False, mode: int = ROPE_STD):
     x = np.ascontiguousarray(x, np.float64)
     y = np.empty_like(x)
-    lib().orc_rope_apply_f64(_p(y, ctypes.c_double), _p(x, ctypes.c_double), int(m), x.size, base,
+    lib().orc_rope_apply_f64(_p(y, ctypes.c_double), _p(x, ctypes.c_double), int(m), x.size, base, mode,
                              int(inverse))
     return y
 

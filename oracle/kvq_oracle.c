@@ -127,11 +127,20 @@ uint16_t orc_float_to_half_ru(float f) {
  * Pins: R(a)R(b) = R(a+b) ([RoPE-KV §7.1]); the score depends only on m-n
  * ([EliteKV §2.2]).
  * ---------------------------------------------------------------------- */
-double orc_rope_theta(int i, int d, double base) { return pow(base, -(2.0 * i) / d); }
+/* Frequency of pair i (0-based; the pages' j = i + 1). mode (the rope flag):
+ * 1: the standard table theta_i = base^(-2i/d) ([EliteKV §2.1]);
+ * 2: frequency-aware RoPE ([KV-Latent], frequency-aware RoPE): the first half
+ *    of the pairs (i < d/4) take base^(-2(i + d/8)/d), the second half
+ *    base^(-(i + 3d/4)/d): the highest frequencies are skipped and the low
+ *    ones sampled twice as densely. */
+double orc_rope_theta(int i, int d, double base, int mode) {
+  if (mode == 2) return i < d / 4 ? pow(base, -2.0 * (i + d / 8) / d) : pow(base, -(double)(i + 3 * d / 4) / d);
+  return pow(base, -(2.0 * i) / d);
+}
 
-void orc_rope_cs(int64_t m, int d, double base, float* c, float* s) {
+void orc_rope_cs(int64_t m, int d, double base, int mode, float* c, float* s) {
   for (int i = 0; i < d / 2; ++i) {
-    double ang = (double)m * orc_rope_theta(i, d, base);
+    double ang = (double)m * orc_rope_theta(i, d, base, mode);
     c[i] = (float)cos(ang);
     s[i] = (float)sin(ang);
   }
@@ -148,9 +157,9 @@ void orc_rope_apply_f32(float* y, const float* x, const float* c, const float* s
 }
 
 /* exact-angle rotation in fp64; inverse != 0 rotates by -m*theta */
-void orc_rope_apply_f64(double* y, const double* x, int64_t m, int d, double base, int inverse) {
+void orc_rope_apply_f64(double* y, const double* x, int64_t m, int d, double base, int mode, int inverse) {
   for (int i = 0; i < d / 2; ++i) {
-    double ang = (double)m * orc_rope_theta(i, d, base);
+    double ang = (double)m * orc_rope_theta(i, d, base, mode);
     double c = cos(ang), s = inverse ? -sin(ang) : sin(ang);
     double x0 = x[2 * i], x1 = x[2 * i + 1];
     y[2 * i] = x0 * c - x1 * s;
@@ -406,7 +415,7 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
     for (int h0 = 0; h0 < H; h0 += hg)
       for (int t = 0; t < T; ++t) {
         int64_t m = pos[t];
-        if (rope) orc_rope_cs(m, D, base, c, sn);
+        if (rope) orc_rope_cs(m, D, base, rope, c, sn);
         for (int hl = 0; hl < hg; ++hl) {
           size_t v = ((size_t)(b * H + h0 + hl) * T + t);
           const uint16_t* xv = x + v * D;
@@ -549,7 +558,7 @@ static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* co
             const uint16_t* sv = sink + ((size_t)(b * H + h0 + hl) * s->n_sink + m) * D;
             for (int j = 0; j < D; ++j) y[j] = orc_half_to_float(sv[j]);
             if (attn_space && s->rope)
-              orc_rope_apply_f64(out + v * D, y, m, D, s->base, 0);
+              orc_rope_apply_f64(out + v * D, y, m, D, s->base, s->rope, 0);
             else
               memcpy(out + v * D, y, sizeof(double) * D);
           }
@@ -577,7 +586,7 @@ static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* co
             size_t v = ((size_t)(b * H + h0 + hl) * T + t);
             dequant_head(s, codes + v * rb, sz + v * ng * 2, y);
             if (s->rope)
-              orc_rope_apply_f64(buf + hl * D, y, m, D, s->base, 1);
+              orc_rope_apply_f64(buf + hl * D, y, m, D, s->base, s->rope, 1);
             else
               memcpy(buf + hl * D, y, sizeof(double) * D);
           }
@@ -591,7 +600,7 @@ static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* co
               x[dst] = buf[hl * D + j] * r;
             }
             if (attn_space && s->rope)
-              orc_rope_apply_f64(out + v * D, x, m, D, s->base, 0);
+              orc_rope_apply_f64(out + v * D, x, m, D, s->base, s->rope, 0);
             else
               memcpy(out + v * D, x, sizeof(double) * D);
           }
@@ -607,7 +616,7 @@ static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* co
           }
           for (int j = 0; j < D; ++j) y[perm ? perm[h0 * D + j] : j] = buf[j];
           if (s->rope && !attn_space)
-            orc_rope_apply_f64(out + v * D, y, m, D, s->base, 1);
+            orc_rope_apply_f64(out + v * D, y, m, D, s->base, s->rope, 1);
           else
             memcpy(out + v * D, y, sizeof(double) * D);
         }
@@ -756,7 +765,7 @@ int orc_calibrate_perm(int B, int H, int T, int D, const int64_t* pos, int rope,
         const uint16_t* xv = x + ((size_t)(b * H + h) * T + t) * D;
         for (int j = 0; j < D; ++j) xf[j] = orc_half_to_float(xv[j]);
         if (rope) {
-          orc_rope_cs(pos[t], D, base, c, sn);
+          orc_rope_cs(pos[t], D, base, rope, c, sn);
           orc_rope_apply_f32(y, xf, c, sn, D);
         } else {
           memcpy(y, xf, sizeof(float) * D);
