@@ -293,6 +293,34 @@ class CalibrateStep:
         return [self.call]
 
 
+class PairEnergyStep:
+    """Exact per-pair RoPE energies and their ranking over the Llama-3-8B GQA
+    keys (4 x 8 x 32768 x 128)."""
+
+    workload = "llama3_8b_pair_energy"
+    kernels_per_step = 2  # energy and rank (plus a memset of the sums)
+
+    def __init__(self, device):
+        import torch
+        from kv_cache_rotation_b200 import torch_api as TA
+        w = W.WORKLOADS["llama3_8b_gqa_score"]
+        self.x = torch.from_numpy(W.kv_tensor(w, "k")).to(device)
+        self.d = TA.make_desc(batch=w.B, heads=w.H, head_dim=w.D, tokens=w.T, bits=w.bits, group=w.group)
+        self.e = torch.empty((w.H, w.D // 2, 2), dtype=torch.uint64, device=device)
+        self.r = torch.empty((w.H, w.D // 2), dtype=torch.int16, device=device)
+        self.call = TA.bind_pair_energy(self.d, self.x, self.e, self.r)
+        nbytes = self.x.numel() * 2
+        self.alg = {"pair_energy": nbytes + self.e.numel() * 8 + self.r.numel() * 2}
+        self.fp16_equiv = {"pair_energy": nbytes}
+        self.kernels = {"pair_energy": "k_pair_energy"}
+        self.fp32_ops = {}
+        self.names = list(self.alg)
+        torch.cuda.synchronize(device)
+
+    def launches(self):
+        return [self.call]
+
+
 class EncDecStep:
     """Encode then decode of K (and V when `both`) for one workload."""
 
@@ -393,6 +421,8 @@ def make_step(workload, device, batch=None):
         return AttendStep(device)
     if workload == "llama3_8b_calibrate":
         return CalibrateStep(device)
+    if workload == "llama3_8b_pair_energy":
+        return PairEnergyStep(device)
     return EncDecStep(workload, device, batch=batch)
 
 
@@ -634,6 +664,11 @@ def run_e2e(st, launches, dev, stream, steps, warmup):
 
 
 def _other_config(name, n_gpus):
+    if name == "llama3_8b_pair_energy":
+        w = W.WORKLOADS["llama3_8b_gqa_score"]
+        return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T,
+                "input": "keys fp16; exact 128-bit sums of each RoPE pair's squared norm, then the pair ranking",
+                "l2": "no flush (the 268 MB input is larger than L2)", "parallelism": f"replicas x{n_gpus}"}
     if name == "llama3_8b_calibrate":
         w = W.WORKLOADS["llama3_8b_gqa_score"]
         return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T,
@@ -660,7 +695,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--workload", default="llama3_8b_gqa",
                     choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "decode_score",
-                             "llama3_8b_gqa_attend", "llama3_8b_calibrate", "tiny"],
+                             "llama3_8b_gqa_attend", "llama3_8b_calibrate", "llama3_8b_pair_energy", "tiny"],
                     help="which workload a step runs (the headline line is llama3_8b_gqa)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch of an encode/decode workload (small profiling captures)")

@@ -207,6 +207,22 @@ kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables
 /* Workspace bytes kvq_calibrate_perm needs for d; 0 if d is invalid or unsupported. */
 size_t kvq_calibrate_workspace_bytes(const kvq_desc* d);
 
+/* Energy of each RoPE frequency pair ([EliteKV] §3.1, frequency energy analysis): per head h,
+ *   E[h][i] = sum over the B batches and the T tokens of x[..][2i]^2 + x[..][2i+1]^2,
+ * on the keys as given (RoPE rotates each pair without changing its norm), exactly: every fp16
+ * square is an integer multiple of 2^-48, and E is returned as an unsigned 128-bit count of 2^-48
+ * (energy_out[h][i][0] = low 64 bits, [1] = high 64 bits; E = (lo + hi * 2^64) * 2^-48).
+ * rank_out[h] lists the pairs by descending E, equal E in ascending pair order (the elite
+ * frequencies are its first entries). Infinite or NaN inputs contribute nothing.
+ *   x           half [B][H][T][head_dim], 16-byte aligned (only batch, heads, head_dim, tokens of d
+ *               are used)
+ *   energy_out  uint64 [H][head_dim/2][2], 16-byte aligned, zeroed and filled by the call
+ *   rank_out    int16 [H][head_dim/2], 16-byte aligned
+ * The results are integers and exact: they do not depend on scheduling. KVQ_ERR_UNSUPPORTED for
+ * B*T >= 2^31. */
+kvq_status kvq_pair_energy(const kvq_desc* d, const void* x, uint64_t* energy_out, int16_t* rank_out,
+                           kvq_stream_t stream);
+
 /* Bytes of one packed buffer (KVQ_FIELD_*) for this descriptor; 0 if the field is unused or
  * the descriptor is invalid. */
 size_t kvq_packed_bytes(const kvq_desc* d, int32_t field);
@@ -215,6 +231,19 @@ size_t kvq_packed_bytes(const kvq_desc* d, int32_t field);
  * theta_i = base^(-2i/head_dim), the angle formed in double ([RoPE-KV §1], [EliteKV §2.1]).
  * The caller copies it to the device. */
 kvq_status kvq_rope_table(float* cs_host, int32_t t_max, int32_t head_dim, double base);
+
+/* Frequency tables for kvq_rope_table_ex. Every kernel takes whatever table it is given. */
+enum {
+  KVQ_ROPE_STANDARD = 0,   /* theta_i = base^(-2i/head_dim): the kvq_rope_table table */
+  KVQ_ROPE_FREQ_AWARE = 1  /* [KV-Latent] frequency-aware RoPE: pairs i < head_dim/4 take
+                              base^(-2(i + head_dim/8)/head_dim), the others
+                              base^(-(i + 3 head_dim/4)/head_dim): the highest frequencies are
+                              skipped and the low ones sampled twice as densely */
+};
+
+/* kvq_rope_table with a choice of frequencies (KVQ_ROPE_*); head_dim a multiple of 8 for
+ * KVQ_ROPE_FREQ_AWARE. Same layout and rounding: (float)cos / (float)sin of the double angle. */
+kvq_status kvq_rope_table_ex(float* cs_host, int32_t t_max, int32_t head_dim, double base, int32_t freq);
 
 /* Fill a HOST buffer with the 2^bits Lloyd-Max levels of N(0, 1/head_dim), ascending: Lloyd's
  * iteration on N(0,1) in double, scaled by 1/sqrt(head_dim), rounded to fp32 ([IsoQuant §3.1]). */

@@ -23,8 +23,8 @@ KVQ_Q_MINMAX, KVQ_Q_CODEBOOK = 0, 1
 KVQ_FIELD_CODES, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_FIELD_NORM = range(4)
 
 EXPORTED = ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_attend_workspace_bytes",
-            "kvq_calibrate_perm", "kvq_calibrate_workspace_bytes",
-            "kvq_packed_bytes", "kvq_rope_table", "kvq_lloyd_max_codebook", "kvq_check", "kvq_debug_expire_wait",
+            "kvq_calibrate_perm", "kvq_calibrate_workspace_bytes", "kvq_pair_energy",
+            "kvq_packed_bytes", "kvq_rope_table", "kvq_rope_table_ex", "kvq_lloyd_max_codebook", "kvq_check", "kvq_debug_expire_wait",
             "kvq_status_str", "kvq_version")
 
 
@@ -65,6 +65,7 @@ def _load():
     L.kvq_attend_noalloc.argtypes = [P(kvq_desc), P(kvq_desc), vp, i32, P(kvq_packed), P(kvq_tables),
                                      P(kvq_packed), P(kvq_tables), i32, ctypes.c_float, vp, st]
     L.kvq_calibrate_perm.argtypes = [P(kvq_desc), vp, P(kvq_tables), vp, vp, ctypes.c_size_t, st]
+    L.kvq_pair_energy.argtypes = [P(kvq_desc), vp, vp, vp, st]
     L.kvq_calibrate_workspace_bytes.argtypes = [P(kvq_desc)]
     L.kvq_calibrate_workspace_bytes.restype = ctypes.c_size_t
     L.kvq_attend_workspace_bytes.argtypes = [P(kvq_desc), P(kvq_desc), i32, i32]
@@ -72,6 +73,7 @@ def _load():
     L.kvq_packed_bytes.argtypes = [P(kvq_desc), i32]
     L.kvq_packed_bytes.restype = ctypes.c_size_t
     L.kvq_rope_table.argtypes = [vp, i32, i32, ctypes.c_double]
+    L.kvq_rope_table_ex.argtypes = [vp, i32, i32, ctypes.c_double, i32]
     L.kvq_lloyd_max_codebook.argtypes = [vp, i32, i32]
     L.kvq_check.argtypes = [st]
     L.kvq_debug_expire_wait.argtypes = [ctypes.c_uint32, st]
@@ -79,7 +81,8 @@ def _load():
     L.kvq_status_str.restype = ctypes.c_char_p
     L.kvq_version.restype = i32
     for n in ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_calibrate_perm",
-              "kvq_rope_table",
+              "kvq_pair_energy",
+              "kvq_rope_table", "kvq_rope_table_ex",
               "kvq_lloyd_max_codebook",
               "kvq_check", "kvq_debug_expire_wait"):
         getattr(L, n).restype = i32
@@ -127,6 +130,10 @@ def kvq_calibrate_perm(d: kvq_desc, x: int, tb: kvq_tables, perm_out: int, works
     return lib.kvq_calibrate_perm(ctypes.byref(d), x, ctypes.byref(tb), perm_out, workspace, workspace_bytes, stream)
 
 
+def kvq_pair_energy(d: kvq_desc, x: int, energy_out: int, rank_out: int, stream: int = 0) -> int:
+    return lib.kvq_pair_energy(ctypes.byref(d), x, energy_out, rank_out, stream)
+
+
 def kvq_calibrate_workspace_bytes(d: kvq_desc) -> int:
     return lib.kvq_calibrate_workspace_bytes(ctypes.byref(d))
 
@@ -141,6 +148,14 @@ def kvq_packed_bytes(desc: kvq_desc, field: int) -> int:
 
 def kvq_rope_table(cs_host: int, t_max: int, head_dim: int, base: float = 10000.0) -> int:
     return lib.kvq_rope_table(cs_host, t_max, head_dim, base)
+
+
+KVQ_ROPE_STANDARD, KVQ_ROPE_FREQ_AWARE = 0, 1
+
+
+def kvq_rope_table_ex(cs_host: int, t_max: int, head_dim: int, base: float = 10000.0,
+                      freq: int = KVQ_ROPE_STANDARD) -> int:
+    return lib.kvq_rope_table_ex(cs_host, t_max, head_dim, base, freq)
 
 
 def kvq_lloyd_max_codebook(levels_host: int, bits: int, head_dim: int) -> int:

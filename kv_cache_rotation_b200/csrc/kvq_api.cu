@@ -320,6 +320,18 @@ kvq_status kvq_attend_noalloc(const kvq_desc* dk, const kvq_desc* dv, const void
                        reinterpret_cast<cudaStream_t>(stream), ctx);
 }
 
+kvq_status kvq_pair_energy(const kvq_desc* d, const void* x, uint64_t* energy_out, int16_t* rank_out,
+                           kvq_stream_t stream) {
+  kvq_status s = check_desc(d);
+  if (s != KVQ_OK) return s;
+  if (!x || !energy_out || !rank_out) return KVQ_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(energy_out, 16) || !aligned(rank_out, 16)) return KVQ_ERR_ALIGN;
+  if (static_cast<int64_t>(d->batch) * d->tokens >= (int64_t(1) << 31)) return KVQ_ERR_UNSUPPORTED;
+  LaunchCtx ctx;
+  if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
+  return launch_pair_energy(*d, x, energy_out, rank_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t kvq_calibrate_workspace_bytes(const kvq_desc* d) {
   if (check_desc(d) != KVQ_OK || d->rot == KVQ_ROT_ISO_SO4) return 0;
   return calibrate_workspace_bytes(*d);
@@ -366,10 +378,21 @@ size_t kvq_packed_bytes(const kvq_desc* d, int32_t field) {
 }
 
 kvq_status kvq_rope_table(float* cs_host, int32_t t_max, int32_t head_dim, double base) {
+  return kvq_rope_table_ex(cs_host, t_max, head_dim, base, KVQ_ROPE_STANDARD);
+}
+
+kvq_status kvq_rope_table_ex(float* cs_host, int32_t t_max, int32_t head_dim, double base, int32_t freq) {
   if (!cs_host || t_max <= 0 || head_dim <= 0 || head_dim % 2 || !(base > 1.0)) return KVQ_ERR_INVALID;
+  if (freq != KVQ_ROPE_STANDARD && freq != KVQ_ROPE_FREQ_AWARE) return KVQ_ERR_INVALID;
+  if (freq == KVQ_ROPE_FREQ_AWARE && head_dim % 8) return KVQ_ERR_INVALID;
   const int half = head_dim / 2;
   for (int i = 0; i < half; ++i) {
-    const double theta = pow(base, -(2.0 * i) / head_dim);
+    double theta;
+    if (freq == KVQ_ROPE_FREQ_AWARE)  // two samplings: the upper half of the pairs twice as dense
+      theta = i < head_dim / 4 ? pow(base, -2.0 * (i + head_dim / 8) / head_dim)
+                               : pow(base, -static_cast<double>(i + 3 * head_dim / 4) / head_dim);
+    else
+      theta = pow(base, -(2.0 * i) / head_dim);
     for (int64_t m = 0; m < t_max; ++m) {
       const double ang = static_cast<double>(m) * theta;
       cs_host[(m * half + i) * 2] = static_cast<float>(cos(ang));

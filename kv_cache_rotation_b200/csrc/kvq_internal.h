@@ -46,6 +46,7 @@ kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq
 kvq_status launch_debug_wait(uint64_t limit_ns, cudaStream_t st, const LaunchCtx& ctx);
 size_t attend_workspace_bytes(const kvq_desc& dk, int q_heads, int n_tokens);
 size_t attend_scratch_bytes();
+kvq_status launch_pair_energy(const kvq_desc& d, const void* x, uint64_t* energy, int16_t* rank, cudaStream_t st);
 bool calibrate_rope(const kvq_desc& d);
 size_t calibrate_workspace_bytes(const kvq_desc& d);
 kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& tb, int16_t* perm, void* ws,

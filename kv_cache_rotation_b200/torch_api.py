@@ -74,10 +74,11 @@ def alloc_packed(d: kvq_desc, device="cuda", zero=True) -> Packed:
     return Packed(codes, sz, sink, norm)
 
 
-def rope_table(t_max: int, head_dim: int, device="cuda", base: float = 10000.0) -> torch.Tensor:
-    """(cos, sin) table [t_max][head_dim/2][2] filled by kvq_rope_table."""
+def rope_table(t_max: int, head_dim: int, device="cuda", base: float = 10000.0, freq: int = 0) -> torch.Tensor:
+    """(cos, sin) table [t_max][head_dim/2][2] filled by kvq_rope_table_ex (freq: KVQ_ROPE_*)."""
+    from . import kvq_rope_table_ex
     host = torch.empty((t_max, head_dim // 2, 2), dtype=torch.float32)
-    check(kvq_rope_table(host.data_ptr(), t_max, head_dim, base), "kvq_rope_table")
+    check(kvq_rope_table_ex(host.data_ptr(), t_max, head_dim, base, freq), "kvq_rope_table_ex")
     return host.to(device)
 
 
@@ -178,6 +179,28 @@ def calibrate_perm(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Ten
     check(kvq_calibrate_perm(d, x.data_ptr(), tb.struct(), perm_out.data_ptr(), workspace.data_ptr(),
                              workspace.numel(), _stream(stream)), "kvq_calibrate_perm")
     return perm_out
+
+
+def pair_energy(d: kvq_desc, x: torch.Tensor, stream=None):
+    """Exact RoPE-pair energies (uint64 [H][head_dim/2][2]: low, high words of the count of
+    2^-48) and the pairs ranked by descending energy (int16 [H][head_dim/2])."""
+    from . import kvq_pair_energy
+    energy = torch.empty((d.heads, d.head_dim // 2, 2), dtype=torch.uint64, device=x.device)
+    rank = torch.empty((d.heads, d.head_dim // 2), dtype=torch.int16, device=x.device)
+    check(kvq_pair_energy(d, x.data_ptr(), energy.data_ptr(), rank.data_ptr(), _stream(stream)), "kvq_pair_energy")
+    return energy, rank
+
+
+def bind_pair_energy(d: kvq_desc, x: torch.Tensor, energy: torch.Tensor, rank: torch.Tensor, stream=None):
+    from . import lib
+    st = _stream(stream)
+    args = (ctypes.byref(d), x.data_ptr(), energy.data_ptr(), rank.data_ptr(), st)
+    keep = (d, x, energy, rank)
+
+    def call():
+        check(lib.kvq_pair_energy(*args), "kvq_pair_energy")
+    call.keep = keep
+    return call
 
 
 def bind_calibrate(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Tensor, workspace: torch.Tensor,

@@ -192,3 +192,24 @@ def test_calibrate_argument_checks():
     # grouped keys permute the raw input: no RoPE table needed
     g = _desc(tokens=40, rope=1, rot="fwht_group", group_heads=8, group=128)
     assert K.kvq_calibrate_workspace_bytes(g) == nb
+
+
+def test_pair_energy_argument_checks():
+    d = _desc(tokens=40)
+    assert K.kvq_pair_energy(_desc(batch=0), 256, 512, 1024, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_pair_energy(d, 0, 512, 1024, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_pair_energy(d, 264, 512, 1024, 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_pair_energy(d, 256, 520, 1024, 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_pair_energy(d, 256, 512, 1032, 0) == K.KVQ_ERR_ALIGN
+
+
+@pytest.mark.parametrize("d", [16, 64, 128])
+def test_freq_aware_rope_table_matches_oracle(orc, d):
+    import torch
+    cs = TA.rope_table(40000, d, device="cpu", freq=K.KVQ_ROPE_FREQ_AWARE).numpy()
+    for m in (0, 1, 777, 32768, 39999):
+        c, s = orc.rope_cs(m, d, mode=orc.ROPE_FREQ_AWARE)
+        assert np.array_equal(cs[m, :, 0], c) and np.array_equal(cs[m, :, 1], s)
+    buf = torch.empty(4 * 12).data_ptr()
+    assert K.kvq_rope_table_ex(buf, 4, 12, 10000.0, K.KVQ_ROPE_FREQ_AWARE) == K.KVQ_ERR_INVALID  # not a multiple of 8
+    assert K.kvq_rope_table_ex(buf, 4, 8, 10000.0, 7) == K.KVQ_ERR_INVALID

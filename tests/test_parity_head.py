@@ -46,20 +46,22 @@ def _inputs(name, B, H, T, D, seed):
     return W.kv_tensor(w, "k")
 
 
-def run_head_case(K, orc, x, *, t0, t_cap, bits, group, rope, perm, n_sink, rot, row_rel=0.0):
+def run_head_case(K, orc, x, *, t0, t_cap, bits, group, rope, perm, n_sink, rot, row_rel=0.0, freq=0):
     from kv_cache_rotation_b200 import torch_api as TA
     B, H, T, D = x.shape
     d = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, t0=t0, t_cap=t_cap, bits=bits, group=group,
                      rope=rope, n_sink=n_sink, rot=rot)
     xg = torch.from_numpy(x).cuda()
-    cs = TA.rope_table(t_cap + 3, D) if rope else None
+    cs = TA.rope_table(t_cap + 3, D, freq=freq) if rope else None
     pg = torch.from_numpy(perm).cuda() if perm is not None else None
     tb = TA.make_tables(perm=pg, rope_cs=cs)
     pk = TA.alloc_packed(d)
     TA.encode(d, xg, tb, pk)
     assert K.kvq_check(0) == K.KVQ_OK
     pos = np.arange(t0, t0 + T)
-    okw = dict(rot={"none": 0, "fwht_head": 1}[rot], bits=bits, group=group, rope=rope, n_sink=n_sink, perm=perm)
+    # the oracle's rope flag names its table: 1 standard, 2 frequency-aware
+    orope = rope * (orc.ROPE_FREQ_AWARE if freq == K.KVQ_ROPE_FREQ_AWARE else orc.ROPE_STD)
+    okw = dict(rot={"none": 0, "fwht_head": 1}[rot], bits=bits, group=group, rope=orope, n_sink=n_sink, perm=perm)
     ref = orc.encode(x.view(np.uint16), pos, want_pre=True, **okw)
     gc = pk.codes[:, :, t0:t0 + T].cpu().numpy()
     gs = pk.scale_zero[:, :, t0:t0 + T].cpu().numpy()
@@ -128,3 +130,12 @@ def test_head_deterministic(K):
     TA.encode(d, xg, tb, a)
     TA.encode(d, xg, tb, b)
     assert torch.equal(a.codes, b.codes) and torch.equal(a.scale_zero, b.scale_zero)
+
+
+@pytest.mark.parametrize("D,group", [(128, 64), (64, 32)])
+def test_head_freq_aware_rope_table(K, orc, D, group):
+    """KV-Latent frequency-aware RoPE: the kernels take the table they are given;
+    codes stay bit-exact against the oracle rotating with the same frequencies."""
+    x = _inputs("freq_aware", 2, 4, 70, D, 21)
+    run_head_case(K, orc, x, t0=3, t_cap=80, bits=2, group=group, rope=1, perm=W.random_perm(4, D, 8), n_sink=4,
+                  rot="fwht_head", freq=K.KVQ_ROPE_FREQ_AWARE)
