@@ -14,8 +14,9 @@
 //
 // A memset and two launches: k_pair_energy, CTA = (chunk of token rows,
 // head), each thread owns 4 pairs of a row with four rows' 16-byte loads in
-// flight, then adds its CTA's sums into the zeroed output with 64-bit
-// atomics (low word, then high word plus the low word's carry);
+// flight (two carry chains per pair), then adds its CTA's sums into the
+// zeroed output with 64-bit atomics (low word, then high word plus the low
+// word's carry);
 // k_pair_rank, one CTA per head, ranks the pairs.
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -63,7 +64,8 @@ __global__ void __launch_bounds__(kThreads) k_pair_energy(const EnergyArgs a) {
   const int h = blockIdx.y;
   const int r0 = blockIdx.x * a.rows_per_chunk;
   const int r1 = min(r0 + a.rows_per_chunk, a.rows);
-  uint64_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
+  // two independent 128-bit sums per pair (its even and its odd channel): shorter carry chains
+  uint64_t lo[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, hi[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
   for (int r = r0 + rl; r < r1; r += U * RPI) {  // row r = (batch b, token t)
     uint4 raw[U];
 #pragma unroll
@@ -80,15 +82,16 @@ __global__ void __launch_bounds__(kThreads) k_pair_energy(const EnergyArgs a) {
       const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};  // word k = pair 4 cg + k
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        add_square(lo[k], hi[k], w[k] & 0xFFFFu);
-        add_square(lo[k], hi[k], w[k] >> 16);
+        add_square(lo[0][k], hi[0][k], w[k] & 0xFFFFu);
+        add_square(lo[1][k], hi[1][k], w[k] >> 16);
       }
     }
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    red[rl][4 * cg + k][0] = lo[k];
-    red[rl][4 * cg + k][1] = hi[k];
+    add128(lo[0][k], hi[0][k], lo[1][k], hi[1][k]);
+    red[rl][4 * cg + k][0] = lo[0][k];
+    red[rl][4 * cg + k][1] = hi[0][k];
   }
   __syncthreads();
   if (tid < P) {
