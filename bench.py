@@ -514,6 +514,23 @@ def run_reference(args):
     return 0
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest x over all ranks (every rank receives it); x itself without a
+    process group. Each rank times its own device; the job takes as long as the
+    slowest rank."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step_per_rank: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the bytes all ranks processed over the slowest rank's time."""
+    return world * bytes_per_step_per_rank * steps / (max_ms / 1e3) / 1e9
+
+
 def run_ours(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -568,13 +585,10 @@ def run_ours(args):
         for i, n in enumerate(st.names):
             per_kernel[n] += ev[s][i].elapsed_time(ev[s][i + 1])
     status = K.kvq_check(0)
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     fp16_step = sum(st.fp16_equiv.values())
-    value = world * fp16_step * args.steps / (total_ms / 1e3) / 1e9
+    value = whole_job_gbs(world, fp16_step, args.steps, total_ms)
     peak, peak_kind = _peaks()
     kernels = {}
     for n in st.names:
@@ -601,11 +615,8 @@ def run_ours(args):
     e2e_line = None
     if hasattr(st, "host_in"):
         e2e = run_e2e(st, launches, dev, stream, min(args.steps, args.e2e_steps), args.warmup_e2e)
-        if dist:
-            t = torch.tensor([e2e["ms_per_step"]], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e["ms_per_step"] = float(t.item())
-        e2e_line = {"value": world * fp16_step / (e2e["ms_per_step"] / 1e3) / 1e9, "unit": UNIT,
+        e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, dev)
+        e2e_line = {"value": whole_job_gbs(world, fp16_step, 1, e2e["ms_per_step"]), "unit": UNIT,
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                     "ms_per_step": e2e["ms_per_step"], "steps": e2e["steps"]}
 
