@@ -289,18 +289,9 @@ size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 // accumulators. (Leaving the masked field as an fp16 subnormal, c 4^t 2^-24,
 // would save the subtraction, but its products with subnormal lo halves of
 // small weights lost precision on the tensor cores.)
-#ifndef KVQ_ATTEND_MINB
-#define KVQ_ATTEND_MINB 2  // resident CTAs per SM the register budget is sized for (GQ <= 4)
-#endif
-#ifndef KVQ_ATTEND_WAVES_NUM  // CTAs launched = resident slots x NUM / DEN (rounded to whole chunks)
-#define KVQ_ATTEND_WAVES_NUM 1
-#endif
-#ifndef KVQ_ATTEND_WAVES_DEN
-#define KVQ_ATTEND_WAVES_DEN 1
-#endif
-#ifndef KVQ_ATTEND_IMAD_SHIFT
-#define KVQ_ATTEND_IMAD_SHIFT 0  // 2-bit score operand: lane shift as an integer multiply
-#endif
+// Resident CTAs per SM the register budget of the fused kernel is sized for
+// (GQ <= 4): 2 (<= 128 registers) measured faster than 3 (<= 80).
+constexpr int kFMinBlocks = 2;
 constexpr int kFWarps = 8;
 constexpr int kFThreads = 32 * kFWarps;
 constexpr int kFBlock = 16;           // tokens per warp step (one m16 tile of the score MMA)
@@ -369,7 +360,7 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t y, uint32_t msk) {
 __device__ __forceinline__ float2 h2f(uint32_t w) { return __half22float2(*reinterpret_cast<const __half2*>(&w)); }
 
 template <int BITS, int GQ>
-__global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 1) k_attend_fused(const FusedArgs a) {
+__global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend_fused(const FusedArgs a) {
   using C = FusedCfg<BITS>;
   constexpr int D = 128;
   constexpr int RB = C::RB;
@@ -378,7 +369,6 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 1) k_at
   constexpr int S = C::STAGES;
   constexpr int CPL = kFBlock * RB / (32 * 16);  // 16-byte code copies per lane and tensor
   constexpr bool ALLQ = GQ % 4 == 0;             // every lane's query head exists
-  constexpr bool IMAD_SHIFT = KVQ_ATTEND_IMAD_SHIFT && BITS == 2;
   extern __shared__ __align__(128) uint8_t fdyn[];  // per warp: S stages of {K codes, V codes, K sz, V sz}
   __shared__ __align__(16) uint2 bfrag[NTN][4][4][8];
   __shared__ __align__(16) float qraw[GQ][D];
@@ -474,7 +464,6 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 1) k_at
   }
   // value B fragments come from the score lanes of rows 2 tig (+8) and 2 tig + 1 (+9)
   const int srcA = 8 * tig + (g >> 1), srcB = srcA + 4;
-  const uint32_t lmul = 1u << (6 - 2 * tig);  // multiply variant: bits 2 tig .. 2 tig + 1 of a byte to 6 .. 7
   const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;  // column g: digit hi (low halves) or lo
 
   // one 16-token block; INTERIOR: no sink and no position past n_tok in it
@@ -502,14 +491,7 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 1) k_at
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
       uint32_t a0, a1, a2, a3;
-      if constexpr (IMAD_SHIFT) {  // code tig of every byte moved to bits 6..7 by a multiply: 64 c per byte
-        a0 = (wa[2 * s] * lmul) & 0xC0C0C0C0u;
-        a1 = (wb[2 * s] * lmul) & 0xC0C0C0C0u;
-        a2 = (wa[2 * s + 1] * lmul) & 0xC0C0C0C0u;
-        a3 = (wb[2 * s + 1] * lmul) & 0xC0C0C0C0u;
-      } else {
-        score_afrag<BITS, NW>(wa, wb, s, tig, a0, a1, a2, a3);
-      }
+      score_afrag<BITS, NW>(wa, wb, s, tig, a0, a1, a2, a3);
 #pragma unroll
       for (int nt = 0; nt < NTN; ++nt) mma_u8s8((s & 1) ? sacc2[nt] : sacc[nt], a0, a1, a2, a3, bq[s][nt]);
     }
@@ -533,9 +515,8 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? KVQ_ATTEND_MINB : 1) k_at
 #pragma unroll
     for (int nt = 0; nt < NTN; ++nt) {
       const bool qv = ALLQ || 4 * nt + tig < GQ;
-      // (the multiply variant's sums are 64x: exact multiples of 64, shifted back exactly)
-      const float da = static_cast<float>((sacc[nt][0] + 256 * sacc[nt][1]) >> (IMAD_SHIFT ? 6 : 0));
-      const float db = static_cast<float>((sacc[nt][2] + 256 * sacc[nt][3]) >> (IMAD_SHIFT ? 6 : 0));
+      const float da = static_cast<float>(sacc[nt][0] + 256 * sacc[nt][1]);
+      const float db = static_cast<float>(sacc[nt][2] + 256 * sacc[nt][3]);
       const float sa = __fmaf_rn(kza.x * sq[nt], da, __fmaf_rn(kza.y, qs[nt], 0.0f)) * a.scale;
       const float sb = __fmaf_rn(kzb2.x * sq[nt], db, __fmaf_rn(kzb2.y, qs[nt], 0.0f)) * a.scale;
       const bool oka = va && qv, okb = vb && qv;
@@ -806,7 +787,7 @@ kvq_status run_fused(FusedArgs& fa, const LaunchCtx& ctx, cudaStream_t st) {
   if (!set_smem_once(fn, smem)) return KVQ_ERR_CUDA;
   const int per_sm = occupancy_once(fn, kFThreads, smem);
   const int bh = fa.B * fa.H;
-  int want = ctx.num_sms * per_sm * KVQ_ATTEND_WAVES_NUM / (KVQ_ATTEND_WAVES_DEN * bh);  // chunks per (batch, KV head)
+  int want = ctx.num_sms * per_sm / bh;  // chunks per (batch, KV head) for about one wave
   want = want < 1 ? 1 : (want > kFMaxChunks ? kFMaxChunks : want);
   fa.blocks_per_chunk = (fa.blocks + want - 1) / want;
   fa.n_chunks = (fa.blocks + fa.blocks_per_chunk - 1) / fa.blocks_per_chunk;
