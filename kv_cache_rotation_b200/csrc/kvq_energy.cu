@@ -7,16 +7,17 @@
 //
 // Exact integer arithmetic: an fp16 value is M 2^(e - 25) (M = 1024 + the
 // 10-bit fraction, biased exponent e >= 1) or M 2^-24 (subnormal), so its
-// square is M^2 2^(2e - 2) (or M^2) units of 2^-48, below 2^80. Sums are
-// unsigned 128-bit integers (two 64-bit words with carries), so the result
-// does not depend on the order of the additions and the ranking is decided
-// on exact values.
+// square is M^2 2^s units of 2^-48 with s = 2e - 2 (or 0), below 2^80. Each
+// square is one 32x32 -> 64-bit product M^2 2^(s mod 32) (< 2^53) added to one
+// of two 64-bit windows (weights 1 and 2^32), which are folded into the
+// unsigned 128-bit sums (two words with carries) every 64 row steps, long
+// before a window could overflow. The result does not depend on the order of
+// the additions, and the ranking is decided on exact values.
 //
 // A memset and two launches: k_pair_energy, CTA = (chunk of token rows,
 // head), each thread owns 4 pairs of a row with four rows' 16-byte loads in
-// flight (two carry chains per pair), then adds its CTA's sums into the
-// zeroed output with 64-bit atomics (low word, then high word plus the low
-// word's carry);
+// flight, then adds its CTA's sums into the zeroed output with 64-bit atomics
+// (low word, then high word plus the low word's carry);
 // k_pair_rank, one CTA per head, ranks the pairs.
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -36,16 +37,15 @@ struct EnergyArgs {
   int16_t* rank;               // [H][D/2]
 };
 
-// (lo, hi) += square of the fp16 value h in units of 2^-48 (inf / nan add nothing).
-__device__ __forceinline__ void add_square(uint64_t& lo, uint64_t& hi, uint32_t h) {
+// (a0, a1) += square of the fp16 value h: a0 in units of 2^-48, a1 in units of 2^-16 (inf / nan add nothing).
+__device__ __forceinline__ void add_square(uint64_t& a0, uint64_t& a1, uint32_t h) {
   const uint32_t e = (h >> 10) & 31u, f = h & 1023u;
   const uint32_t M = e == 31u ? 0u : (e ? (f | 1024u) : f);
-  const uint32_t sh = e ? 2u * e - 2u : 0u;  // 0 .. 60; M^2 < 2^22
-  const uint64_t sq = static_cast<uint64_t>(M * M);
-  const uint64_t vlo = sq << sh;
-  const uint64_t vhi = sh > 42u ? sq >> (64u - sh) : 0u;
-  lo += vlo;
-  hi += vhi + (lo < vlo ? 1u : 0u);
+  const uint32_t s = e ? 2u * e - 2u : 0u;  // 0 .. 58
+  const uint64_t t = static_cast<uint64_t>(M * M) * static_cast<uint64_t>(1u << (s & 31u));  // < 2^53
+  const uint64_t m = s >= 32u ? ~0ull : 0ull;
+  a1 += t & m;
+  a0 += t & ~m;
 }
 
 __device__ __forceinline__ void add128(uint64_t& lo, uint64_t& hi, uint64_t blo, uint64_t bhi) {
@@ -64,8 +64,9 @@ __global__ void __launch_bounds__(kThreads) k_pair_energy(const EnergyArgs a) {
   const int h = blockIdx.y;
   const int r0 = blockIdx.x * a.rows_per_chunk;
   const int r1 = min(r0 + a.rows_per_chunk, a.rows);
-  // two independent 128-bit sums per pair (its even and its odd channel): shorter carry chains
-  uint64_t lo[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, hi[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+  uint64_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};  // 128-bit sums per pair
+  uint64_t a0[4] = {0, 0, 0, 0}, a1[4] = {0, 0, 0, 0};  // windows of weight 1 and 2^32
+  int n_it = 0;
   for (int r = r0 + rl; r < r1; r += U * RPI) {  // row r = (batch b, token t)
     uint4 raw[U];
 #pragma unroll
@@ -82,16 +83,29 @@ __global__ void __launch_bounds__(kThreads) k_pair_energy(const EnergyArgs a) {
       const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};  // word k = pair 4 cg + k
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        add_square(lo[0][k], hi[0][k], w[k] & 0xFFFFu);
-        add_square(lo[1][k], hi[1][k], w[k] >> 16);
+        add_square(a0[k], a1[k], w[k] & 0xFFFFu);
+        add_square(a0[k], a1[k], w[k] >> 16);
       }
+    }
+    if (++n_it == 64) {  // fold before a window could overflow (64 x 8 terms < 2^53 each)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        add128(lo[k], hi[k], a0[k], 0);
+        add128(lo[k], hi[k], a1[k] << 32, a1[k] >> 32);
+        a0[k] = a1[k] = 0;
+      }
+      n_it = 0;
     }
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    add128(lo[0][k], hi[0][k], lo[1][k], hi[1][k]);
-    red[rl][4 * cg + k][0] = lo[0][k];
-    red[rl][4 * cg + k][1] = hi[0][k];
+    add128(lo[k], hi[k], a0[k], 0);
+    add128(lo[k], hi[k], a1[k] << 32, a1[k] >> 32);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    red[rl][4 * cg + k][0] = lo[k];
+    red[rl][4 * cg + k][1] = hi[k];
   }
   __syncthreads();
   if (tid < P) {
