@@ -158,9 +158,14 @@ kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kv
  * P^T H_norm (sum_n p_n y_n): the inverse rotation runs once per output, not per token.
  * q: half [B][q_heads][head_dim] in attention space, 16-byte aligned. out: f32
  * [B][q_heads][head_dim], 16-byte aligned. workspace: caller-owned device memory, 256-byte
- * aligned, at least kvq_attend_workspace_bytes() bytes; it holds the scores and per-chunk
- * partial sums, needs no initialisation and must not be shared by calls in flight at the same
- * time. d->tokens and d->t0 are ignored. Launches three kernels on `stream`. */
+ * aligned, at least kvq_attend_workspace_bytes() bytes; it holds per-chunk partial sums (and,
+ * outside the fused form, the scores), needs no initialisation and must not be shared by calls
+ * in flight at the same time. d->tokens and d->t0 are ignored. With 2- or 4-bit codes and one
+ * group per record (group = 128) two kernels run on `stream`: a fused pass over the K and V
+ * records (scores, running softmax and value sums on the tensor cores) and a merge launched as
+ * its programmatic dependent; other shapes run three (scores, chunked softmax-weighted sums,
+ * merge). Results agree with kvq_score's scores through an exact fp64 softmax within
+ * 2e-5 * max|vhat|. */
 kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int32_t q_heads,
                       const kvq_packed* k_cache, const kvq_tables* tk, const kvq_packed* v_cache,
                       const kvq_tables* tv, int32_t n_tokens, float scale, float* out, void* workspace,
