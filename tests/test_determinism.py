@@ -1,0 +1,78 @@
+"""Race check by repetition: every kernel family run twice on the same inputs
+must produce the same bytes. The kernels are deterministic by construction
+(no floating-point atomics; the integer and max atomics of the calibration
+and pair-energy reductions are order-independent), so a difference would
+point at a read-before-write race on shared or global memory."""
+import numpy as np
+import pytest
+
+import workloads as W
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def TA():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from kv_cache_rotation_b200 import torch_api as TA
+    return TA
+
+
+def _twice(f):
+    a = f()
+    b = f()
+    torch.cuda.synchronize()
+    return a, b
+
+
+def test_grouped_encode_decode_repeat(TA):
+    w = W.Workload("det_group", B=1, H=8, T=300, D=128, rot="fwht_group", group_heads=8, bits=2, group=128)
+    x = torch.from_numpy(W.kv_tensor(w, "k")).cuda()
+    d = TA.make_desc(batch=1, heads=8, head_dim=128, tokens=300, bits=2, group=128, group_heads=8, rope=1,
+                     rot="fwht_group")
+    tb = TA.make_tables(rope_cs=TA.rope_table(300, 128))
+
+    def enc():
+        pk = TA.alloc_packed(d)
+        TA.encode(d, x, tb, pk)
+        out = torch.empty((1, 8, 300, 128), dtype=torch.float16, device="cuda")
+        TA.decode(d, pk, tb, out)
+        return pk.codes.clone(), pk.scale_zero.clone(), out
+    (c1, s1, o1), (c2, s2, o2) = _twice(enc)
+    assert torch.equal(c1, c2) and torch.equal(s1, s2) and torch.equal(o1, o2)
+
+
+def test_score_and_attention_repeat(TA):
+    B, H, Hq, T, D = 2, 2, 8, 700, 128
+    w = W.Workload("det_attend", B=B, H=H, Hq=Hq, T=T, D=D, bits=2, group=128, n_sink=4, seed=3)
+    common = dict(batch=B, heads=H, head_dim=D, tokens=T, t_cap=T, bits=2, group=128, n_sink=4, rot="fwht_head")
+    dk, dv = TA.make_desc(rope=1, **common), TA.make_desc(rope=0, **common)
+    tk = TA.make_tables(rope_cs=TA.rope_table(T, D))
+    tv = TA.make_tables()
+    pk, pv = TA.alloc_packed(dk), TA.alloc_packed(dv)
+    TA.encode(dk, torch.from_numpy(W.kv_tensor(w, "k")).cuda(), tk, pk)
+    TA.encode(dv, torch.from_numpy(W.kv_tensor(w, "v")).cuda(), tv, pv)
+    q = torch.from_numpy(W.queries(w)).cuda()
+    ws = TA.attend_workspace(dk, dv, Hq, T)
+
+    def run():
+        s = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
+        TA.score(dk, q, pk, tk, T, 0.088, s)
+        o = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+        TA.attend(dk, dv, q, pk, tk, pv, tv, T, 0.088, o, ws)
+        return s, o
+    (s1, o1), (s2, o2) = _twice(run)
+    assert torch.equal(s1, s2) and torch.equal(o1, o2)
+
+
+def test_calibration_and_energy_repeat(TA):
+    w = W.Workload("det_cal", B=2, H=4, T=3000, D=128, outliers=("pairs", 0.02, 10.0, 50.0))
+    x = torch.from_numpy(W.kv_tensor(w, "k")).cuda()
+    d = TA.make_desc(batch=2, heads=4, head_dim=128, tokens=3000, bits=2, group=128, rope=1, n_sink=4)
+    tb = TA.make_tables(rope_cs=TA.rope_table(3000, 128))
+    (p1, p2) = _twice(lambda: TA.calibrate_perm(d, x, tb).clone())
+    assert torch.equal(p1, p2)
+    (e1, e2) = _twice(lambda: tuple(t.cpu() for t in TA.pair_energy(d, x)))
+    assert np.array_equal(e1[0].numpy(), e2[0].numpy()) and torch.equal(e1[1], e2[1])
