@@ -63,3 +63,29 @@ def test_large_scale_selects_the_top_key(orc, caches):
             gap = np.sort(s[b, qh])[-1] - np.sort(s[b, qh])[-2]
             assert gap * 1e4 > 50  # the runner-up's weight is below e^-50
             np.testing.assert_allclose(out[b, qh], caches["vhat"][b, qh // (HQ // H), top], rtol=0, atol=1e-9)
+
+
+def test_sinks_are_verbatim_values(orc, caches):
+    # with three cached tokens, all sinks, the output is a convex mix of the fp16 sink rows themselves
+    out = _attend(orc, caches, 3, 1.0 / np.sqrt(D))
+    sink_v = caches["vc"]["sink"].view(np.float16).astype(np.float64)  # [B][H][n_sink][D]
+    for qh in range(HQ):
+        h = qh // (HQ // H)
+        lo, hi = sink_v[:, h].min(axis=1), sink_v[:, h].max(axis=1)
+        assert np.all(out[:, qh] >= lo - 1e-12) and np.all(out[:, qh] <= hi + 1e-12)
+    # and a single sink token returns its row exactly
+    one = _attend(orc, caches, 1, 0.7)
+    for qh in range(HQ):
+        assert np.array_equal(one[:, qh], sink_v[:, qh // (HQ // H), 0])
+
+
+def test_query_heads_share_their_kv_head(orc, caches):
+    # two query heads of the same KV head with the same query give the same output; the GQA grouping is
+    # contiguous (query head qh reads KV head qh // (HQ / H))
+    q = caches["q"].copy()
+    q[:, 1] = q[:, 0]          # same group (KV head 0)
+    q[:, HQ // H] = q[:, 0]    # first query head of KV head 1
+    out = orc.attend(q, caches["kc"], caches["vc"], T, H=H, t_cap=T, scale=0.2, kperm=caches["kp"],
+                     vperm=caches["vp"], **caches["common"])
+    assert np.array_equal(out[:, 1], out[:, 0])
+    assert not np.allclose(out[:, HQ // H], out[:, 0])  # a different cache gives a different result
