@@ -175,8 +175,9 @@ kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int
  * when they call (a fixed-budget serving loop, host code without a device allocator, a caller
  * whose workspace would have to stay put between repeated launches of the same work). The
  * pages have no counterpart: it is a variant of kvq_attend with the same arguments and
- * results, whose scores and chunk partials live in a fixed 40 MiB device array of the library
- * (enough for 4 sequences x 32 query heads x 32769 cached tokens); it allocates nothing.
+ * results, whose workspace (chunk partials, and the scores outside the fused form) lives in a
+ * fixed 40 MiB device array of the library (enough for 4 sequences x 32 query heads x 32769
+ * cached tokens in either form); it allocates nothing.
  * Returns KVQ_ERR_UNSUPPORTED when kvq_attend_workspace_bytes() exceeds 40 MiB. The array's
  * device address is looked up on the first call made with each device current: make that
  * first call outside any stream capture. The array is shared by every call on a device: two

@@ -831,10 +831,11 @@ int fused_tiles(int n_tokens) { return (n_tokens + kFBlock - 1) / kFBlock; }
 
 // Fixed scratch of kvq_attend_noalloc: a file-scope device array, reserved when
 // the module is loaded, so that entry point never allocates. 40 MiB holds the
-// scores and chunk partials of about 9 M (query head x cached token) pairs
-// (4 bytes of score + 0.5 byte of chunk partials each), e.g. 4 sequences x 32
-// query heads x 32769 tokens (19 MB). Nothing in it has
-// to start at zero: every byte a call reads was written earlier in that call.
+// workspace of either form: chunk partials (at most 256 chunks per query head
+// in the fused form: 4 sequences x 32 query heads x 32769 tokens take 17 MB),
+// or scores plus partials (about 4.5 bytes per query head and cached token,
+// 19 MB for the same shape). Nothing in it has to start at zero: every byte a
+// call reads was written earlier in that call.
 constexpr size_t kAttendScratchBytes = size_t{40} << 20;
 __device__ __align__(256) uint8_t g_attend_scratch[kAttendScratchBytes];
 
