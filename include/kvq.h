@@ -179,8 +179,12 @@ kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int
  * fixed 40 MiB device array of the library (enough for 4 sequences x 32 query heads x 32769
  * cached tokens in either form); it allocates nothing.
  * Returns KVQ_ERR_UNSUPPORTED when kvq_attend_workspace_bytes() exceeds 40 MiB. The array's
- * device address is looked up on the first call made with each device current: make that
- * first call outside any stream capture. The array is shared by every call on a device: two
+ * device address is looked up once per device, by the first call of ANY libkvq entry point that
+ * launches work with that device current; with CUDA's lazy module loading (the default) that
+ * lookup is also when the driver reserves the array, so make one library call that launches
+ * work on each device (an encode, a decode, a score) before the serving loop, and outside any
+ * stream capture; a kvq_attend_noalloc that is itself that first call reserves the array then. If the array could not be reserved, this entry point returns KVQ_ERR_CUDA; the
+ * others are unaffected. The array is shared by every call on a device: two
  * calls that can run at the same time (different streams, or host threads without ordering)
  * race on it and corrupt each other's results; calls in order on one stream are safe. Nothing
  * in it needs to start at zero. */

@@ -48,6 +48,12 @@ kvq_status get_ctx(LaunchCtx* ctx) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return KVQ_ERR_CUDA;
     g_err_addr[dev] = static_cast<uint32_t*>(p);
     g_num_sms[dev] = sms;
+    // Resolve kvq_attend_noalloc's fixed scratch now, on the first call of any
+    // entry point on this device: under lazy module loading this is when the
+    // array is reserved, so a later kvq_attend_noalloc call finds it ready and
+    // reserves nothing. A failure here is reported by kvq_attend_noalloc alone
+    // (it returns KVQ_ERR_CUDA); every other entry point keeps working.
+    (void)attend_scratch();
   }
   ctx->err = g_err_addr[dev];
   ctx->num_sms = g_num_sms[dev];
@@ -265,6 +271,8 @@ kvq_status check_attend(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads,
       k.bits != v.bits || k.group != v.group || k.n_sink != v.n_sink || k.rot != v.rot || k.quant != v.quant)
     return KVQ_ERR_INVALID;
   if (q_heads <= 0 || q_heads % k.heads) return KVQ_ERR_INVALID;
+  // the attention kernels put batch x KV head (and batch x query head) on one grid axis
+  if (static_cast<int64_t>(k.batch) * q_heads > 65535) return KVQ_ERR_UNSUPPORTED;
   const int gq = q_heads / k.heads;
   if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KVQ_ERR_UNSUPPORTED;
   if (n_tokens < 1 || n_tokens > k.t_cap) return KVQ_ERR_INVALID;

@@ -160,20 +160,13 @@ __global__ void __launch_bounds__(kThreads) k_score_simt(const ScoreArgs a) {
 // memory by bulk copy, two tiles of 128 tokens in flight; CTAs are
 // persistent over a range of tiles of one (batch, KV head) so the query
 // rotation is done once per CTA.
-// Tiling (compile-time tunables).
-#ifndef KVQ_SCORE_MT
-#define KVQ_SCORE_MT 2
-#endif
-#ifndef KVQ_SCORE_STAGES
-#define KVQ_SCORE_STAGES 4
-#endif
-#ifndef KVQ_SCORE_CTAS_PER_SM
-#define KVQ_SCORE_CTAS_PER_SM 4
-#endif
+// Tiling: 2 m-tiles of 16 tokens per warp (256-token tiles), 4 tiles in
+// flight per CTA, at most 4 CTAs per SM.
 constexpr int kMmaThreads = 256;
-constexpr int kMmaMT = KVQ_SCORE_MT;              // 16-token m-tiles per warp per tile
-constexpr int kMmaTile = 8 * 16 * kMmaMT;         // tokens per tile
-constexpr int kMmaStages = KVQ_SCORE_STAGES;      // tiles in flight per CTA
+constexpr int kMmaMT = 2;                  // 16-token m-tiles per warp per tile
+constexpr int kMmaTile = 8 * 16 * kMmaMT;  // tokens per tile
+constexpr int kMmaStages = 4;              // tiles in flight per CTA
+constexpr int kMmaCtasPerSm = 4;
 
 struct MmaArgs {
   ScoreArgs s;
@@ -275,6 +268,7 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
   load_sz(gt0, sza, szb);
   int cur_bh = -1;
   bool ok = true;
+  int gt_fail = gt1;  // first tile whose copy was not seen to land
   for (int gt = gt0; gt < gt1; ++gt) {
     const int it = gt - gt0;
     const int st = it % kMmaStages;
@@ -316,7 +310,10 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
       }
     }
     // every warp has read this stage: refill it with the tile kMmaStages ahead
-    if (!__syncthreads_and(ok)) break;
+    if (!__syncthreads_and(ok)) {
+      gt_fail = gt;
+      break;
+    }
     if (tid == 0 && gt + kMmaStages < gt1) issue(gt + kMmaStages, st);
     __half2 pa[kMmaMT][NGK], pb[kMmaMT][NGK];
 #pragma unroll
@@ -350,9 +347,14 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
       }
     }
   }
-  if (!ok && tid == 0) {
-    for (int st = 0; st < kMmaStages; ++st)
-      for (uint32_t p = 0; p < 2; ++p) mbar_wait(&full[st], p, ma.wait_ns, ma.err);
+  // After a timed-out wait, let the copies still in flight land (bounded)
+  // before the CTA exits: tiles gt_fail .. gt_fail + kMmaStages - 1 were
+  // issued and not consumed; each is waited on once, at its stage and phase.
+  if (gt_fail < gt1 && tid == 0) {
+    for (int gt = gt_fail; gt < gt1 && gt < gt_fail + kMmaStages; ++gt) {
+      const int it = gt - gt0;
+      mbar_wait(&full[it % kMmaStages], (it / kMmaStages) & 1, ma.wait_ns, ma.err);
+    }
   }
 }
 
@@ -365,7 +367,7 @@ kvq_status run_mma(const ScoreArgs& a, const LaunchCtx& ctx, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(kMmaStages) * kMmaTile * (128 * BITS / 8);
   if (!set_smem_once(reinterpret_cast<const void*>(k_score_mma<BITS, G, GQ>), smem)) return KVQ_ERR_CUDA;
   int per_sm = occupancy_once(reinterpret_cast<const void*>(k_score_mma<BITS, G, GQ>), kMmaThreads, smem);
-  per_sm = per_sm > KVQ_SCORE_CTAS_PER_SM ? KVQ_SCORE_CTAS_PER_SM : per_sm;
+  per_sm = per_sm > kMmaCtasPerSm ? kMmaCtasPerSm : per_sm;
   const int tpb = (a.n_tok + kMmaTile - 1) / kMmaTile;
   const long long total = static_cast<long long>(a.B) * a.H * tpb;
   if (total >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;

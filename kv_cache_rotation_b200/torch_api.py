@@ -113,6 +113,32 @@ def make_tables(perm=None, rope_cs=None, qL=None, qR=None, codebook=None) -> Tab
     return Tables(perm, rope_cs, qL, qR, codebook)
 
 
+def _req(t: torch.Tensor, name: str, dtypes, shape=None) -> None:
+    """Reject a tensor the C ABI would misread: it must be a contiguous CUDA
+    tensor of one of `dtypes`, shaped `shape` when given."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _kv_shape(d: kvq_desc):
+    return (d.batch, d.heads, d.tokens, d.head_dim)
+
+
+def _q_heads(d: kvq_desc, q: torch.Tensor) -> int:
+    _req(q, "q", (torch.float16,))
+    if q.dim() != 3 or q.shape[0] != d.batch or q.shape[2] != d.head_dim:
+        raise ValueError(f"q: shape {tuple(q.shape)}, expected ({d.batch}, q_heads, {d.head_dim})")
+    return int(q.shape[1])
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -120,17 +146,21 @@ def _stream(stream) -> int:
 
 
 def encode(d: kvq_desc, x: torch.Tensor, tables: Tables, packed: Packed, stream=None) -> None:
+    _req(x, "x", (torch.float16,), _kv_shape(d))
     check(kvq_encode(d, x.data_ptr(), tables.struct(), packed.struct(), _stream(stream)), "kvq_encode")
 
 
 def decode(d: kvq_desc, packed: Packed, tables: Tables, out: torch.Tensor, stream=None) -> None:
+    _req(out, "out", (torch.float16, torch.float32), _kv_shape(d))
     fp32 = 1 if out.dtype == torch.float32 else 0
     check(kvq_decode(d, packed.struct(), tables.struct(), out.data_ptr(), fp32, _stream(stream)), "kvq_decode")
 
 
 def score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens: int, scale: float,
           out: torch.Tensor, stream=None) -> None:
-    check(kvq_score(d, q.data_ptr(), q.shape[1], packed.struct(), tables.struct(), n_tokens, scale,
+    hq = _q_heads(d, q)
+    _req(out, "scores", (torch.float32,), (d.batch, hq, n_tokens))
+    check(kvq_score(d, q.data_ptr(), hq, packed.struct(), tables.struct(), n_tokens, scale,
                     out.data_ptr(), _stream(stream)), "kvq_score")
 
 
@@ -146,7 +176,10 @@ def attend_workspace(dk: kvq_desc, dv: kvq_desc, q_heads: int, n_tokens: int, de
 def attend(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, tk: Tables, v_packed: Packed, tv: Tables,
            n_tokens: int, scale: float, out: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
     from . import kvq_attend
-    check(kvq_attend(dk, dv, q.data_ptr(), q.shape[1], k_packed.struct(), tk.struct(), v_packed.struct(),
+    hq = _q_heads(dk, q)
+    _req(out, "out", (torch.float32,), (dk.batch, hq, dk.head_dim))
+    _req(workspace, "workspace", (torch.uint8,))
+    check(kvq_attend(dk, dv, q.data_ptr(), hq, k_packed.struct(), tk.struct(), v_packed.struct(),
                      tv.struct(), n_tokens, scale, out.data_ptr(), workspace.data_ptr(), workspace.numel(),
                      _stream(stream)), "kvq_attend")
 
@@ -155,7 +188,9 @@ def attend_noalloc(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed
                    tv: Tables, n_tokens: int, scale: float, out: torch.Tensor, stream=None) -> None:
     """kvq_attend through the library's fixed scratch (no workspace tensor)."""
     from . import kvq_attend_noalloc
-    check(kvq_attend_noalloc(dk, dv, q.data_ptr(), q.shape[1], k_packed.struct(), tk.struct(), v_packed.struct(),
+    hq = _q_heads(dk, q)
+    _req(out, "out", (torch.float32,), (dk.batch, hq, dk.head_dim))
+    check(kvq_attend_noalloc(dk, dv, q.data_ptr(), hq, k_packed.struct(), tk.struct(), v_packed.struct(),
                              tv.struct(), n_tokens, scale, out.data_ptr(), _stream(stream)), "kvq_attend_noalloc")
 
 
@@ -172,10 +207,12 @@ def calibrate_perm(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Ten
                    workspace: torch.Tensor = None, stream=None) -> torch.Tensor:
     """Channel permutation by abs-max (int16 [H][head_dim]) for kvq_tables.perm."""
     from . import kvq_calibrate_perm
+    _req(x, "x", (torch.float16,), _kv_shape(d))
     if perm_out is None:
         perm_out = torch.empty((d.heads, d.head_dim), dtype=torch.int16, device=x.device)
     if workspace is None:
         workspace = calibrate_workspace(d, x.device)
+    _req(perm_out, "perm_out", (torch.int16,), (d.heads, d.head_dim))
     check(kvq_calibrate_perm(d, x.data_ptr(), tb.struct(), perm_out.data_ptr(), workspace.data_ptr(),
                              workspace.numel(), _stream(stream)), "kvq_calibrate_perm")
     return perm_out
@@ -185,6 +222,7 @@ def pair_energy(d: kvq_desc, x: torch.Tensor, stream=None):
     """Exact RoPE-pair energies (uint64 [H][head_dim/2][2]: low, high words of the count of
     2^-48) and the pairs ranked by descending energy (int16 [H][head_dim/2])."""
     from . import kvq_pair_energy
+    _req(x, "x", (torch.float16,), _kv_shape(d))
     energy = torch.empty((d.heads, d.head_dim // 2, 2), dtype=torch.uint64, device=x.device)
     rank = torch.empty((d.heads, d.head_dim // 2), dtype=torch.int16, device=x.device)
     check(kvq_pair_energy(d, x.data_ptr(), energy.data_ptr(), rank.data_ptr(), _stream(stream)), "kvq_pair_energy")
@@ -193,6 +231,9 @@ def pair_energy(d: kvq_desc, x: torch.Tensor, stream=None):
 
 def bind_pair_energy(d: kvq_desc, x: torch.Tensor, energy: torch.Tensor, rank: torch.Tensor, stream=None):
     from . import lib
+    _req(x, "x", (torch.float16,), _kv_shape(d))
+    _req(energy, "energy", (torch.uint64,), (d.heads, d.head_dim // 2, 2))
+    _req(rank, "rank", (torch.int16,), (d.heads, d.head_dim // 2))
     st = _stream(stream)
     args = (ctypes.byref(d), x.data_ptr(), energy.data_ptr(), rank.data_ptr(), st)
     keep = (d, x, energy, rank)
@@ -206,6 +247,8 @@ def bind_pair_energy(d: kvq_desc, x: torch.Tensor, energy: torch.Tensor, rank: t
 def bind_calibrate(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Tensor, workspace: torch.Tensor,
                    stream=None):
     from . import lib
+    _req(x, "x", (torch.float16,), _kv_shape(d))
+    _req(perm_out, "perm_out", (torch.int16,), (d.heads, d.head_dim))
     tbs, st = tb.struct(), _stream(stream)
     args = (ctypes.byref(d), x.data_ptr(), ctypes.byref(tbs), perm_out.data_ptr(), workspace.data_ptr(),
             workspace.numel(), st)
@@ -220,8 +263,11 @@ def bind_calibrate(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Ten
 def bind_attend(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, tk: Tables, v_packed: Packed,
                 tv: Tables, n_tokens: int, scale: float, out: torch.Tensor, workspace: torch.Tensor, stream=None):
     from . import lib
+    hq = _q_heads(dk, q)
+    _req(out, "out", (torch.float32,), (dk.batch, hq, dk.head_dim))
+    _req(workspace, "workspace", (torch.uint8,))
     tks, kps, tvs, vps, st = tk.struct(), k_packed.struct(), tv.struct(), v_packed.struct(), _stream(stream)
-    args = (ctypes.byref(dk), ctypes.byref(dv), q.data_ptr(), q.shape[1], ctypes.byref(kps), ctypes.byref(tks),
+    args = (ctypes.byref(dk), ctypes.byref(dv), q.data_ptr(), hq, ctypes.byref(kps), ctypes.byref(tks),
             ctypes.byref(vps), ctypes.byref(tvs), n_tokens, ctypes.c_float(scale), out.data_ptr(),
             workspace.data_ptr(), workspace.numel(), st)
     keep = (dk, dv, q, k_packed, tk, v_packed, tv, out, workspace, tks, kps, tvs, vps)
@@ -238,6 +284,7 @@ def bind_attend(dk: kvq_desc, dv: kvq_desc, q: torch.Tensor, k_packed: Packed, t
 # struct building (for tight loops such as a benchmark or a decode loop).
 def bind_encode(d: kvq_desc, x: torch.Tensor, tables: Tables, packed: Packed, stream=None):
     from . import lib
+    _req(x, "x", (torch.float16,), _kv_shape(d))
     tb, pk, st = tables.struct(), packed.struct(), _stream(stream)
     args = (ctypes.byref(d), x.data_ptr(), ctypes.byref(tb), ctypes.byref(pk), st)
     keep = (d, x, tables, packed, tb, pk)
@@ -250,6 +297,7 @@ def bind_encode(d: kvq_desc, x: torch.Tensor, tables: Tables, packed: Packed, st
 
 def bind_decode(d: kvq_desc, packed: Packed, tables: Tables, out: torch.Tensor, stream=None):
     from . import lib
+    _req(out, "out", (torch.float16, torch.float32), _kv_shape(d))
     tb, pk, st = tables.struct(), packed.struct(), _stream(stream)
     fp32 = 1 if out.dtype == torch.float32 else 0
     args = (ctypes.byref(d), ctypes.byref(pk), ctypes.byref(tb), out.data_ptr(), fp32, st)
@@ -264,8 +312,10 @@ def bind_decode(d: kvq_desc, packed: Packed, tables: Tables, out: torch.Tensor, 
 def bind_score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens: int, scale: float,
                out: torch.Tensor, stream=None):
     from . import lib
+    hq = _q_heads(d, q)
+    _req(out, "scores", (torch.float32,), (d.batch, hq, n_tokens))
     tb, pk, st = tables.struct(), packed.struct(), _stream(stream)
-    args = (ctypes.byref(d), q.data_ptr(), q.shape[1], ctypes.byref(pk), ctypes.byref(tb), n_tokens,
+    args = (ctypes.byref(d), q.data_ptr(), hq, ctypes.byref(pk), ctypes.byref(tb), n_tokens,
             ctypes.c_float(scale), out.data_ptr(), st)
     keep = (d, q, packed, tables, out, tb, pk)
 

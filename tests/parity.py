@@ -14,6 +14,7 @@ in the L1 magnitude of the dot product; fp32 accumulation on the GPU).
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass
 
 import numpy as np
@@ -44,6 +45,17 @@ class CodeReport:
         return self.unexcused == 0 and self.sz_mismatch == 0 and self.excused <= EXCUSE_FRAC * self.n
 
 
+# Every code comparison made in this process, as (test id, CodeReport): the
+# session summary (conftest.py) prints the mismatched and excused counts per
+# test, so the excused fraction is reported, not only bounded.
+REPORTS = []
+
+
+def _record(rep: "CodeReport") -> "CodeReport":
+    REPORTS.append((os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], rep))
+    return rep
+
+
 def unpack_all(codes: np.ndarray, D: int, bits: int) -> np.ndarray:
     """[..., D*bits/8] bytes -> [..., D] codes (LSB-first bit stream)."""
     flat = codes.reshape(-1, D * bits // 8)
@@ -72,7 +84,7 @@ def compare_minmax(gpu_codes, orc_codes, gpu_sz, orc_sz, pre, D, bits, group) ->
         near = np.abs(v - beta) <= EXCUSE_REL * np.maximum(np.abs(v), S)
         ok = diff & (np.abs(cg - co) == 1) & near
         exc = int(ok.sum())
-    return CodeReport(cg.size, n_mis, exc, n_mis - exc, szm)
+    return _record(CodeReport(cg.size, n_mis, exc, n_mis - exc, szm))
 
 
 def compare_codebook(gpu_codes, orc_codes, pre, cb, D, bits) -> CodeReport:
@@ -90,7 +102,7 @@ def compare_codebook(gpu_codes, orc_codes, pre, cb, D, bits) -> CodeReport:
         near = np.abs(v - beta[kk]) <= EXCUSE_REL * np.maximum(np.abs(v), sigma)
         ok = diff & (np.abs(cg - co) == 1) & near
         exc = int(ok.sum())
-    return CodeReport(cg.size, n_mis, exc, n_mis - exc, 0)
+    return _record(CodeReport(cg.size, n_mis, exc, n_mis - exc, 0))
 
 
 def recon_tolerance(ref, row_rel=0.0):

@@ -67,22 +67,32 @@ def test_full_llama3_8b_gqa(K, orc, which):
     assert np.all(np.abs(got - dec) <= 1e-3 + np.abs(dec) * 2.0 ** -11), np.abs(got - dec).max()
 
 
-def test_full_llama2_7b_mha(K, orc):
+@pytest.mark.parametrize("which", ["k", "v"])
+def test_full_llama2_7b_mha(K, orc, which):
+    """The Llama-2-7B MHA layer (8 x 32 x 4096 x 128) with its own channel
+    permutation: kvq_calibrate_perm on the tensor itself (abs-max per channel,
+    RoPE'd for the keys, sinks excluded), equal to the oracle's calibration,
+    then encode / decode with it; 2-bit groups of 64, 4 fp16 sinks."""
     from kv_cache_rotation_b200 import torch_api as TA
     w = W.WORKLOADS["llama2_7b_mha"]
-    x = W.kv_tensor(w, "k")
-    perm = W.random_perm(w.H, w.D, 17)
-    d = TA.make_desc(batch=w.B, heads=w.H, head_dim=w.D, tokens=w.T, bits=w.bits, group=w.group, rope=1,
+    rope = 1 if which == "k" else 0
+    x = W.kv_tensor(w, which)
+    d = TA.make_desc(batch=w.B, heads=w.H, head_dim=w.D, tokens=w.T, bits=w.bits, group=w.group, rope=rope,
                      n_sink=w.n_sink, rot="fwht_head")
-    tb = TA.make_tables(perm=torch.from_numpy(perm).cuda(), rope_cs=TA.rope_table(w.T, w.D))
-    pk = TA.alloc_packed(d)
     xg = torch.from_numpy(x).cuda()
+    cs = TA.rope_table(w.T, w.D) if rope else None
+    perm_g = TA.calibrate_perm(d, xg, TA.make_tables(rope_cs=cs))
+    perm = perm_g.cpu().numpy()
+    want = orc.calibrate_perm(x.view(np.uint16), W.positions(0, w.T), rope=rope, n_sink=w.n_sink)
+    assert np.array_equal(perm, want)
+    tb = TA.make_tables(perm=perm_g, rope_cs=cs)
+    pk = TA.alloc_packed(d)
     TA.encode(d, xg, tb, pk)
     out = torch.empty(xg.shape, dtype=torch.float32, device="cuda")
     TA.decode(d, pk, tb, out)
     assert K.kvq_check(0) == K.KVQ_OK
-    tok = _sample(w.T, 24, 5, always=(0, 1, 2, 3, 4, w.T - 1))
-    okw = dict(rot=orc.ROT_FWHT_HEAD, bits=w.bits, group=w.group, rope=1, n_sink=w.n_sink, perm=perm)
+    tok = _sample(w.T, 24, 5 + rope, always=(0, 1, 2, 3, 4, w.T - 1))
+    okw = dict(rot=orc.ROT_FWHT_HEAD, bits=w.bits, group=w.group, rope=rope, n_sink=w.n_sink, perm=perm)
     gc, gs = _check_minmax_sample(orc, x, pk, tok, okw, w.D, w.bits, w.group, w.n_sink)
     dec = orc.decode({"codes": gc, "sz": gs.view(np.uint16), "sink": pk.sink.cpu().numpy().view(np.uint16)},
                      tok, (w.B, w.H, tok.size, w.D), **okw)

@@ -101,6 +101,19 @@ def test_head_parity(K, orc, case):
                   n_sink=n_sink, rot=rot)
 
 
+@pytest.mark.parametrize("which", ["k", "v"])
+def test_tiny_workload_own_inputs(K, orc, which):
+    """The tiny configuration on its own input recipe (1 sequence x 8 heads x
+    256 tokens, N(0,1) with 4 channels per head scaled by 20): RoPE on the
+    keys, FWHT over head_dim, 4-bit min-max with groups of 128, K and V."""
+    w = W.WORKLOADS["tiny"]
+    x = W.kv_tensor(w, which)
+    assert x.shape == (1, 8, 256, 128)
+    rep, _ = run_head_case(K, orc, x, t0=0, t_cap=w.T, bits=w.bits, group=w.group,
+                           rope=1 if which == "k" else 0, perm=None, n_sink=w.n_sink, rot=w.rot)
+    assert rep.n == x.size
+
+
 def test_head_edge_values(K, orc):
     """Zero vectors, constant vectors, fp16 extremes that stay in range after
     the rotation, subnormals, and a mix in one batch."""
