@@ -321,6 +321,39 @@ class PairEnergyStep:
         return [self.call]
 
 
+class GroupScoreStep:
+    """Decode-step scores over the headline layer's own grouped-head key cache
+    (4 x 8 KV heads x 32768 slots, FWHT over the 8 heads before RoPE, 2-bit
+    group 128) for 32 query heads (GQA 4:1): every slot is decoded, turned by
+    RoPE and dotted with its query heads."""
+
+    workload = "llama3_8b_gqa_group_score"
+
+    def __init__(self, device):
+        import torch
+        from kv_cache_rotation_b200 import torch_api as TA
+        wg, ws = W.WORKLOADS["llama3_8b_gqa"], W.WORKLOADS["llama3_8b_gqa_score"]
+        B, H, T, D = wg.B, wg.H, wg.T, wg.D
+        self.d = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, bits=wg.bits, group=wg.group,
+                              group_heads=wg.group_heads, rope=1, rot="fwht_group")
+        self.tb = TA.make_tables(rope_cs=TA.rope_table(T, D, device=device))
+        self.pk = TA.alloc_packed(self.d, device)
+        TA.encode(self.d, torch.from_numpy(W.kv_tensor(wg, "k")).to(device), self.tb, self.pk)
+        self.q = torch.from_numpy(W.queries(ws)).to(device)
+        self.scores = torch.empty((B, ws.Hq, T), dtype=torch.float32, device=device)
+        self.call = TA.bind_score(self.d, self.q, self.pk, self.tb, T, 1.0 / math.sqrt(D), self.scores)
+        rb, ng = D * wg.bits // 8, D // wg.group
+        self.alg = {"score": B * H * T * (rb + 4 * ng) + B * ws.Hq * D * 2 + B * ws.Hq * T * 4}
+        self.fp16_equiv = {"score": B * H * T * D * 2}
+        self.kernels = {"score": "k_score_group"}
+        self.fp32_ops = {}
+        self.names = list(self.alg)
+        torch.cuda.synchronize(device)
+
+    def launches(self):
+        return [self.call]
+
+
 class EncDecStep:
     """Encode then decode of K (and V when `both`) for one workload."""
 
@@ -331,11 +364,11 @@ class EncDecStep:
         w = W.WORKLOADS[name] if batch is None else W.scaled(W.WORKLOADS[name], B=batch)
         self.TA = TA
         B, H, T, D = w.B, w.H, w.T, w.D
-        iso = w.rot == "iso"
+        iso = w.rot in ("iso", "iso3")
         tensors = ["k", "v"] if both and not iso else ["k"]
         self.items = []
         self.alg, self.fp16_equiv, self.kernels, self.fp32_ops = {}, {}, {}, {}
-        kern = {"fwht_head": "head", "none": "head", "fwht_group": "group", "iso": "iso"}[w.rot]
+        kern = {"fwht_head": "head", "none": "head", "fwht_group": "group", "iso": "iso", "iso3": "iso"}[w.rot]
         for which in tensors:
             x = (W.kv_tensor_device(w, which, device) if iso else torch.from_numpy(W.kv_tensor(w, which)).to(device))
             rope = 1 if (which == "k" and w.rope_k) else 0
@@ -343,8 +376,9 @@ class EncDecStep:
                              group_heads=w.group_heads, rope=rope, n_sink=w.n_sink, rot=w.rot, quant=w.quant)
             perm = torch.from_numpy(W.random_perm(H, D, w.seed + len(which))).to(device) if w.perm else None
             if iso:
-                qL, qR = W.iso_tables(w)
-                tb = TA.make_tables(qL=torch.from_numpy(qL).to(device), qR=torch.from_numpy(qR).to(device),
+                qL, qR = W.iso_tables(w) if w.rot == "iso" else (W.iso3_tables(D, w.seed), None)
+                tb = TA.make_tables(qL=torch.from_numpy(qL).to(device),
+                                    qR=torch.from_numpy(qR).to(device) if qR is not None else None,
                                     codebook=TA.lloyd_max_codebook(w.bits, D, device=device))
             else:
                 tb = TA.make_tables(perm=perm, rope_cs=TA.rope_table(T, D, device=device) if rope else None)
@@ -403,7 +437,7 @@ def fp32_ops_per_element(rot, step, group_heads, D, rope=None):
     or the dequantizer 2 (fma + the folded normalisation). Min/max compares run
     on the ALU pipe and are not counted. None for IsoQuant (norm, 4x4 blocks,
     codebook search)."""
-    if rot == "iso":
+    if rot in ("iso", "iso3"):
         return None
     n = D * (group_heads if rot == "fwht_group" else 1)
     fwht = 0 if rot == "none" else int(math.log2(n))
@@ -423,6 +457,8 @@ def make_step(workload, device, batch=None):
         return CalibrateStep(device)
     if workload == "llama3_8b_pair_energy":
         return PairEnergyStep(device)
+    if workload == "llama3_8b_gqa_group_score":
+        return GroupScoreStep(device)
     return EncDecStep(workload, device, batch=batch)
 
 
@@ -734,6 +770,12 @@ def _other_config(name, n_gpus):
         return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T,
                 "input": "keys fp16; exact 128-bit sums of each RoPE pair's squared norm, then the pair ranking",
                 "l2": "no flush (the 268 MB input is larger than L2)", "parallelism": f"replicas x{n_gpus}"}
+    if name == "llama3_8b_gqa_group_score":
+        w = W.WORKLOADS["llama3_8b_gqa"]
+        return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T, "q_heads": 32,
+                "cache": "grouped-head FWHT over 8 heads x 128 before RoPE, 2-bit group 128 (the headline K cache)",
+                "l2": "no flush (the 38 MB cache and 17 MB of scores are read / written once per step)",
+                "parallelism": f"replicas x{n_gpus}"}
     if name == "llama3_8b_calibrate":
         w = W.WORKLOADS["llama3_8b_gqa_score"]
         return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T,
@@ -760,7 +802,8 @@ def main():
                     help="token positions (of each of the 4 sequences) per reference-arm step")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--workload", default="llama3_8b_gqa",
-                    choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "decode_score",
+                    choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "isoquant_so3_batch", "decode_score",
+                             "llama3_8b_gqa_group_score",
                              "llama3_8b_gqa_attend", "llama3_8b_calibrate", "llama3_8b_pair_energy", "tiny"],
                     help="which workload a step runs (the headline line is llama3_8b_gqa)")
     ap.add_argument("--batch", type=int, default=None,

@@ -52,15 +52,20 @@ enum {
   KVQ_ROT_FWHT_GROUP = 2, /* [RotateKV] pre-RoPE grouped-head rotation: permutation -> normalised FWHT
                              over group_heads*head_dim channels (the heads of one token concatenated)
                              -> RoPE on each head slice */
-  KVQ_ROT_ISO_SO4 = 3     /* [IsoQuant §2.2, §3.1] norm split rho = ||x||, x/(rho+1e-8), then
+  KVQ_ROT_ISO_SO4 = 3,    /* [IsoQuant §2.2, §3.1] norm split rho = ||x||, x/(rho+1e-8), then
                              w = qL (x) v (x) qR on each 4-D block v */
+  KVQ_ROT_ISO_SO3 = 4     /* [IsoQuant §2.1, §1] the same norm split, then the 3-D sandwich
+                             w = q v q* on each block of 3 channels taken as a pure quaternion; a
+                             2-channel tail (head_dim 128: 42 blocks + 2) is turned in its plane by
+                             the same sandwich, a 1-channel tail (64, 256) is kept as it is */
 };
 
 /* Scalar quantizer. */
 enum {
   KVQ_Q_MINMAX = 0,  /* per-token per-group asymmetric min-max, fp16 (scale, zero); with
                         rot in {NONE, FWHT_HEAD, FWHT_GROUP} */
-  KVQ_Q_CODEBOOK = 1 /* fixed scalar codebook (Lloyd-Max, [IsoQuant §3.1]); with rot = ISO_SO4 */
+  KVQ_Q_CODEBOOK = 1 /* fixed scalar codebook (Lloyd-Max, [IsoQuant §3.1]); with rot = ISO_SO4
+                        or ISO_SO3 */
 };
 
 /* Which packed buffer kvq_packed_bytes sizes. */
@@ -77,7 +82,10 @@ typedef struct {
   int32_t group;       /* min-max group size in channels: 32, 64 or 128, dividing head_dim
                           (at least head_dim*group_heads/128 channels for FWHT_GROUP) */
   int32_t group_heads; /* FWHT_GROUP: 2, 4 or 8 consecutive heads per rotation, dividing heads */
-  int32_t rope;        /* 1: apply RoPE (keys), 0: not (values) */
+  int32_t rope;        /* 0: no RoPE (values); 1: RoPE on the interleaved pairs (2i, 2i+1) of the
+                          rotation matrix ([EliteKV §2.1]); 2: RoPE on the half-split pairs
+                          (i, i + head_dim/2) of the page's apply_rope code ([EliteKV §7.1]);
+                          pair i turns by m*theta_i either way, from the same table */
   int32_t n_sink;      /* positions 0..n_sink-1 are attention sinks kept verbatim in fp16 */
   int32_t rot;         /* KVQ_ROT_* */
   int32_t quant;       /* KVQ_Q_* */
@@ -88,7 +96,7 @@ typedef struct {
  *                     [bits*j, bits*j+bits) of its little-endian byte stream (LSB first)
  *   scale_zero  half [B][H][t_cap][head_dim/group][2]  (scale S, zero Z); min-max only
  *   sink        half [B][H][n_sink][head_dim]          the first n_sink positions, verbatim
- *   norm        f32  [B][H][t_cap]                      rho; ISO_SO4 only
+ *   norm        f32  [B][H][t_cap]                      rho; ISO_SO4 and ISO_SO3 only
  * Slots of sink positions hold zero codes, zero scale/zero and zero norm.
  * Alignment: codes, scale_zero and sink 16 bytes; norm 4 bytes. Unused fields may be NULL. */
 typedef struct {
@@ -105,6 +113,9 @@ typedef struct {
  *             theta_i = 10000^(-2i/head_dim) ([EliteKV §2.1]); fill it with kvq_rope_table.
  *             16-byte aligned. Required when rope = 1 (and by kvq_score when n_sink > 0).
  *   qL, qR    f32 [head_dim/4][4] unit quaternions (real, i, j, k), one pair per 4-D block
+ *             (ISO_SO4). ISO_SO3 reads qL only: f32 [ceil(head_dim/3)][4], one unit quaternion
+ *             per 3-channel block and, when head_dim mod 3 = 2, one for the 2-channel tail whose
+ *             i and j parts must be zero (otherwise the tail's output is not a rotation)
  *   codebook  f32 [1 << bits] ascending levels (kvq_lloyd_max_codebook) */
 typedef struct {
   const int16_t* perm;

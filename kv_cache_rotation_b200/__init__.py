@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 KVQ_OK, KVQ_ERR_INVALID, KVQ_ERR_UNSUPPORTED, KVQ_ERR_ALIGN, KVQ_ERR_CUDA, KVQ_ERR_TIMEOUT = range(6)
-KVQ_ROT_NONE, KVQ_ROT_FWHT_HEAD, KVQ_ROT_FWHT_GROUP, KVQ_ROT_ISO_SO4 = range(4)
+KVQ_ROT_NONE, KVQ_ROT_FWHT_HEAD, KVQ_ROT_FWHT_GROUP, KVQ_ROT_ISO_SO4, KVQ_ROT_ISO_SO3 = range(5)
 KVQ_Q_MINMAX, KVQ_Q_CODEBOOK = 0, 1
 KVQ_FIELD_CODES, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_FIELD_NORM = range(4)
 

@@ -70,7 +70,7 @@ kvq_status check_desc(const kvq_desc* d) {
   if (d->batch <= 0 || d->heads <= 0 || d->tokens < 0 || d->t0 < 0 || d->t_cap <= 0 || d->n_sink < 0)
     return KVQ_ERR_INVALID;
   if (static_cast<int64_t>(d->t0) + d->tokens > d->t_cap) return KVQ_ERR_INVALID;
-  if (d->rope != 0 && d->rope != 1) return KVQ_ERR_INVALID;
+  if (d->rope < 0 || d->rope > 2) return KVQ_ERR_INVALID;
   if (d->bits < 2 || d->bits > 4) return KVQ_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->batch) * d->heads * d->t_cap * d->head_dim > (int64_t(1) << 40))
@@ -91,6 +91,7 @@ kvq_status check_desc(const kvq_desc* d) {
       if (d->group < 128 / d->group_heads) return KVQ_ERR_UNSUPPORTED;
       break;
     case KVQ_ROT_ISO_SO4:
+    case KVQ_ROT_ISO_SO3:
       if (d->quant != KVQ_Q_CODEBOOK) return KVQ_ERR_UNSUPPORTED;
       if (d->rope) return KVQ_ERR_UNSUPPORTED;
       break;
@@ -113,6 +114,10 @@ kvq_status check_tables(const kvq_desc* d, const kvq_tables* tb, int64_t rope_ro
     if (!tb->qL || !tb->qR || !tb->codebook) return KVQ_ERR_INVALID;
     if (!aligned(tb->qL, 16) || !aligned(tb->qR, 16) || !aligned(tb->codebook, 4)) return KVQ_ERR_ALIGN;
   }
+  if (d->rot == KVQ_ROT_ISO_SO3) {
+    if (!tb->qL || !tb->codebook) return KVQ_ERR_INVALID;
+    if (!aligned(tb->qL, 16) || !aligned(tb->codebook, 4)) return KVQ_ERR_ALIGN;
+  }
   return KVQ_OK;
 }
 
@@ -123,7 +128,7 @@ kvq_status check_packed(const kvq_desc* d, const kvq_packed* p) {
     if (!p->scale_zero) return KVQ_ERR_INVALID;
     if (!aligned(p->scale_zero, 16)) return KVQ_ERR_ALIGN;
   }
-  if (d->rot == KVQ_ROT_ISO_SO4) {
+  if (d->rot == KVQ_ROT_ISO_SO4 || d->rot == KVQ_ROT_ISO_SO3) {
     if (!p->norm) return KVQ_ERR_INVALID;
     if (!aligned(p->norm, 4)) return KVQ_ERR_ALIGN;
   }
@@ -203,6 +208,7 @@ kvq_status kvq_encode(const kvq_desc* d, const void* x, const kvq_tables* tb, co
     case KVQ_ROT_FWHT_GROUP:
       return launch_encode_group(*d, x, *tb, *out, st, ctx);
     case KVQ_ROT_ISO_SO4:
+    case KVQ_ROT_ISO_SO3:
       return launch_encode_iso(*d, x, *tb, *out, st, ctx);
     default:
       return launch_encode_head(*d, x, *tb, *out, st, ctx);
@@ -226,6 +232,7 @@ kvq_status kvq_decode(const kvq_desc* d, const kvq_packed* in, const kvq_tables*
     case KVQ_ROT_FWHT_GROUP:
       return launch_decode_group(*d, *in, *tb, x_out, out_fp32, st, ctx);
     case KVQ_ROT_ISO_SO4:
+    case KVQ_ROT_ISO_SO3:
       return launch_decode_iso(*d, *in, *tb, x_out, out_fp32, st, ctx);
     default:
       return launch_decode_head(*d, *in, *tb, x_out, out_fp32, st, ctx);
@@ -240,16 +247,26 @@ kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kv
   dd.t0 = 0;
   kvq_status s = check_desc(&dd);
   if (s != KVQ_OK) return s;
-  if (dd.rot != KVQ_ROT_NONE && dd.rot != KVQ_ROT_FWHT_HEAD) return KVQ_ERR_UNSUPPORTED;
+  const bool grouped = dd.rot == KVQ_ROT_FWHT_GROUP;
+  if (dd.rot != KVQ_ROT_NONE && dd.rot != KVQ_ROT_FWHT_HEAD && !grouped) return KVQ_ERR_UNSUPPORTED;
   if (!q || !scores) return KVQ_ERR_INVALID;
   if (!aligned(q, 16) || !aligned(scores, 16)) return KVQ_ERR_ALIGN;
   if (q_heads <= 0 || q_heads % dd.heads || q_heads / dd.heads > 16) return KVQ_ERR_INVALID;
   if (n_tokens < 0 || n_tokens > dd.t_cap) return KVQ_ERR_INVALID;
-  if ((s = check_tables(&dd, tb, dd.rope ? (n_tokens < dd.n_sink ? n_tokens : dd.n_sink) : 0)) != KVQ_OK) return s;
+  if (grouped) {  // keys with RoPE, no permutation, up to 8 query heads per KV head
+    if (!dd.rope || (tb && tb->perm)) return KVQ_ERR_UNSUPPORTED;
+    const int gq = q_heads / dd.heads;
+    if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KVQ_ERR_UNSUPPORTED;
+  }
+  const int64_t rows = grouped ? n_tokens : (dd.rope ? (n_tokens < dd.n_sink ? n_tokens : dd.n_sink) : 0);
+  if ((s = check_tables(&dd, tb, rows)) != KVQ_OK) return s;
   if ((s = check_packed(&dd, cache)) != KVQ_OK) return s;
   if (n_tokens == 0) return KVQ_OK;
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
+  if (grouped)
+    return launch_score_group(dd, q, q_heads, *cache, *tb, n_tokens, scale, scores,
+                              reinterpret_cast<cudaStream_t>(stream), ctx);
   return launch_score(dd, q, q_heads, *cache, *tb, n_tokens, scale, scores, reinterpret_cast<cudaStream_t>(stream),
                       ctx);
 }
@@ -341,7 +358,7 @@ kvq_status kvq_pair_energy(const kvq_desc* d, const void* x, uint64_t* energy_ou
 }
 
 size_t kvq_calibrate_workspace_bytes(const kvq_desc* d) {
-  if (check_desc(d) != KVQ_OK || d->rot == KVQ_ROT_ISO_SO4) return 0;
+  if (check_desc(d) != KVQ_OK || d->rot == KVQ_ROT_ISO_SO4 || d->rot == KVQ_ROT_ISO_SO3) return 0;
   return calibrate_workspace_bytes(*d);
 }
 
@@ -349,7 +366,8 @@ kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables
                               void* workspace, size_t workspace_bytes, kvq_stream_t stream) {
   kvq_status s = check_desc(d);
   if (s != KVQ_OK) return s;
-  if (d->rot == KVQ_ROT_ISO_SO4) return KVQ_ERR_UNSUPPORTED;  // no permutation in that variant
+  if (d->rot == KVQ_ROT_ISO_SO4 || d->rot == KVQ_ROT_ISO_SO3)
+    return KVQ_ERR_UNSUPPORTED;  // no permutation in those variants
   if (!x || !perm_out || !workspace || !tb) return KVQ_ERR_INVALID;
   if (!aligned(x, 16) || !aligned(perm_out, 16) || !aligned(workspace, 256)) return KVQ_ERR_ALIGN;
   if (workspace_bytes < calibrate_workspace_bytes(*d)) return KVQ_ERR_INVALID;
@@ -379,7 +397,7 @@ size_t kvq_packed_bytes(const kvq_desc* d, int32_t field) {
     case KVQ_FIELD_SINK:
       return static_cast<size_t>(d->batch) * d->heads * d->n_sink * d->head_dim * 2;
     case KVQ_FIELD_NORM:
-      return d->rot == KVQ_ROT_ISO_SO4 ? vecs * 4 : 0;
+      return (d->rot == KVQ_ROT_ISO_SO4 || d->rot == KVQ_ROT_ISO_SO3) ? vecs * 4 : 0;
     default:
       return 0;
   }

@@ -714,7 +714,7 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
   float mloc = -INFINITY;
   for (int n = warp; n < ns; n += kThreads / 32) {
     const float s = sink_dot(qraw, a.ksink + (vh * a.n_sink + n) * D,
-                             a.krope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane) *
+                             a.krope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane, a.krope == 2) *
                     a.scale;
     if (lane == 0) ts[n] = s;
     mloc = fmaxf(mloc, s * kLog2e);

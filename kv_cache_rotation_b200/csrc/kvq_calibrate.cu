@@ -48,21 +48,26 @@ __global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = 0.0f;
   constexpr int U = 4;  // rows per thread in flight
-  for (int r = r0 + rl; r < r1; r += U * RPI) {  // row r = (batch b, token t)
+  // the trip count is the same for every thread (rows past r1 are not live),
+  // so the half-split pairs may exchange channels between threads
+  for (int rb = r0; rb < r1; rb += U * RPI) {  // row r = (batch b, token t)
+    const int r = rb + rl;
     uint4 raw[U];
     float4 c0[U], c1[U];
+    int posu[U];
     bool live[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int rr = r + u * RPI;
-      const int b = static_cast<int>(a.div_t.div(static_cast<uint32_t>(rr)));
-      const int t = rr - b * a.T;
+      const int b = static_cast<int>(a.div_t.div(static_cast<uint32_t>(min(rr, r1 - 1))));
+      const int t = min(rr, r1 - 1) - b * a.T;
       const int pos = a.t0 + t;
+      posu[u] = pos;
       live[u] = rr < r1 && pos >= a.n_sink;
       raw[u] = live[u] ? __ldg(reinterpret_cast<const uint4*>(
                              a.x + ((static_cast<size_t>(b) * a.H + h) * a.T + t) * D) + cg)
                        : make_uint4(0, 0, 0, 0);
-      if (a.rope && live[u]) {  // pairs 4 cg .. 4 cg + 3 of position pos
+      if (a.rope == 1 && live[u]) {  // pairs 4 cg .. 4 cg + 3 of position pos
         const float4* cs = reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(pos) * D) + 2 * cg;
         c0[u] = __ldg(cs);
         c1[u] = __ldg(cs + 1);
@@ -74,11 +79,24 @@ __global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
     for (int u = 0; u < U; ++u) {
       float v[8];
       h8_to_f32(raw[u], v);
-      if (a.rope) {
+      if (a.rope == 1) {
         rope_fwd(v[0], v[1], c0[u].x, c0[u].y);
         rope_fwd(v[2], v[3], c0[u].z, c0[u].w);
         rope_fwd(v[4], v[5], c1[u].x, c1[u].y);
         rope_fwd(v[6], v[7], c1[u].z, c1[u].w);
+      } else if (a.rope == 2) {
+        // half-split pairs (c, c + D/2): this thread's channel 8 (cg mod TPR/2) + i pairs with the same
+        // channel of thread cg ^ TPR/2 (the other half of the row), angle 8 (cg mod TPR/2) + i
+        const float4* cs = reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(posu[u]) * D) +
+                           4 * (cg & (TPR / 2 - 1));
+        const bool upper = (cg & (TPR / 2)) != 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {  // channels 2k, 2k + 1 of the eight: angles +2k, +2k + 1
+          const float4 c = live[u] ? __ldg(cs + k) : make_float4(1.0f, 0.0f, 1.0f, 0.0f);
+          const float2 y = rope_half_fwd2(f2(v[2 * k], v[2 * k + 1]), f2(c.x, c.z), f2(c.y, c.w), upper, TPR / 2);
+          v[2 * k] = y.x;
+          v[2 * k + 1] = y.y;
+        }
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(v[i]));  // rows not live hold zeros
@@ -145,7 +163,7 @@ kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& 
   a.T = d.tokens;
   a.t0 = d.t0;
   a.n_sink = d.n_sink;
-  a.rope = calibrate_rope(d) ? 1 : 0;
+  a.rope = calibrate_rope(d) ? d.rope : 0;  // 1 interleaved pairs, 2 half-split pairs
   a.rows = static_cast<int>(rows);
   const int chunks = chunks_for(rows);
   a.rows_per_chunk = static_cast<int>((rows + chunks - 1) / chunks);

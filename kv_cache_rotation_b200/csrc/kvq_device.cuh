@@ -94,6 +94,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
 // Pull a tensor tile into L2 ahead of its TMA load (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
@@ -113,6 +121,13 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int 
                "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, int x, int y, int z, int w, const void* src) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
@@ -121,6 +136,12 @@ __device__ __forceinline__ void bulk_wait_read0() {
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N committed bulk-store groups are still incomplete
+// (their global writes done, not only their shared-memory reads).
+template <int N>
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 // Make generic-proxy smem writes visible to the TMA (async proxy).
 __device__ __forceinline__ void fence_async_smem() {
@@ -241,6 +262,21 @@ __device__ __forceinline__ void bfly(float2& a, float2& b) {
   b = sub2(p, q);
 }
 
+// Stride-1 butterfly of the two fp16 channels held in one word w = (x0 | x1 << 16):
+// s = x0 + x1 and d = x0 - x1, each rounded once to fp32. The sm_100 mixed-
+// precision add / sub take x0 as fp16 (its conversion is exact), so only x1 is
+// converted: the same fp32 results as converting both and adding, in one
+// conversion fewer.
+__device__ __forceinline__ void bfly_h2(uint32_t w, float& s, float& d) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t.reg .f32 f1;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.f32.f16 f1, hi;\n\t"
+      "add.rn.f32.f16 %0, lo, f1;\n\t"
+      "sub.rn.f32.f16 %1, lo, f1;\n\t}"
+      : "=f"(s), "=f"(d)
+      : "r"(w));
+}
+
 // Register-pair layout of V consecutive channels: P[2g + e] = (x[4g + e],
 // x[4g + 2 + e]), g < V/4. Unnormalised Sylvester FWHT strides 1, 2, 4, ...,
 // V/2 in ascending order; stride 2 falls inside a pair (scalar ops), every
@@ -256,6 +292,22 @@ __device__ __forceinline__ void fwht_pairs(float2 (&P)[V / 2]) {
   }
 #pragma unroll
   for (int hs = 1; hs < V / 4; hs <<= 1) {  // strides 4 .. V/2
+#pragma unroll
+    for (int g = 0; g < V / 4; ++g) {
+      if ((g & hs) == 0) {
+        bfly(P[2 * g], P[2 * (g + hs)]);
+        bfly(P[2 * g + 1], P[2 * (g + hs) + 1]);
+      }
+    }
+  }
+}
+
+// Strides 4 .. V/2 of the FWHT on the register-pair layout above (strides 1
+// and 2 already applied).
+template <int V>
+__device__ __forceinline__ void fwht_pairs_from4(float2 (&P)[V / 2]) {
+#pragma unroll
+  for (int hs = 1; hs < V / 4; hs <<= 1) {
 #pragma unroll
     for (int g = 0; g < V / 4; ++g) {
       if ((g & hs) == 0) {
@@ -327,6 +379,21 @@ __device__ __forceinline__ void rope_fwd(float& x0, float& x1, float c, float s)
   x0 = y0;
   x1 = y1;
 }
+// Half-split RoPE pairs (i, i + D/2) held by two lanes (partner = lane ^ pm):
+// this lane holds two channels of the lower half (upper == false) or of the
+// upper half, and (cc, ss) are the cosines and sines of their pairs' angles.
+// Forward, the encoder's fp32 order: lower y0 = fma(x0, c, -(x1*s)), upper
+// y1 = fma(x0, s, x1*c), x0 / x1 the lower / upper channel of the pair.
+__device__ __forceinline__ float2 rope_half_fwd2(float2 own, float2 cc, float2 ss, bool upper, int pm) {
+  const float2 oth = f2(__shfl_xor_sync(0xffffffffu, own.x, pm), __shfl_xor_sync(0xffffffffu, own.y, pm));
+  return upper ? fma2(oth, ss, mul2(own, cc)) : fma2(own, cc, mul2(oth, f2(-ss.x, -ss.y)));
+}
+// Inverse: lower x0 = y0 c + y1 s, upper x1 = y1 c - y0 s.
+__device__ __forceinline__ float2 rope_half_inv2(float2 own, float2 cc, float2 ss, bool upper, int pm) {
+  const float2 oth = f2(__shfl_xor_sync(0xffffffffu, own.x, pm), __shfl_xor_sync(0xffffffffu, own.y, pm));
+  return upper ? fma2(own, cc, mul2(oth, f2(-ss.x, -ss.y))) : fma2(own, cc, mul2(oth, ss));
+}
+
 // Inverse rotation (decode; tolerance-checked, any rounding order is fine).
 __device__ __forceinline__ void rope_inv(float& y0, float& y1, float c, float s) {
   const float x0 = __fmaf_rn(y0, c, __fmul_rn(y1, s));

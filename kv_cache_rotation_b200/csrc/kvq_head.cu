@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
       P[2 * g] = f2(h01.x, h23.x);
       P[2 * g + 1] = f2(h01.y, h23.y);
     }
-    if (a.rope) {  // pairs (2i, 2i+1): y0 = fma(x0, c, -(x1*s)), y1 = fma(x0, s, x1*c)
+    if (a.rope == 1) {  // pairs (2i, 2i+1): y0 = fma(x0, c, -(x1*s)), y1 = fma(x0, s, x1*c)
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D) + (V / 4) * s;
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
@@ -161,6 +161,17 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
         const float2 x0 = P[2 * g], x1 = P[2 * g + 1];
         P[2 * g] = fma2(x0, cc, mul2(x1, f2(-ss.x, -ss.y)));
         P[2 * g + 1] = fma2(x0, ss, mul2(x1, cc));
+      }
+    } else if (a.rope == 2) {  // half-split pairs (i, i + V): local channel j of both lanes, angle j
+      const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D);
+#pragma unroll
+      for (int g = 0; g < V / 4; ++g) {
+        const uint4 c0 = __ldg(rp + 2 * g), c1 = __ldg(rp + 2 * g + 1);  // angles 4g .. 4g+1, 4g+2 .. 4g+3
+        // P[2g] holds local channels 4g, 4g+2; P[2g+1] holds 4g+1, 4g+3
+        P[2 * g] = rope_half_fwd2(P[2 * g], f2(__uint_as_float(c0.x), __uint_as_float(c1.x)),
+                                  f2(__uint_as_float(c0.y), __uint_as_float(c1.y)), s != 0, 1);
+        P[2 * g + 1] = rope_half_fwd2(P[2 * g + 1], f2(__uint_as_float(c0.z), __uint_as_float(c1.z)),
+                                      f2(__uint_as_float(c0.w), __uint_as_float(c1.w)), s != 0, 1);
       }
     }
     if (a.perm) {  // p_j = y_perm[h][j]: stage the row, gather
@@ -364,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
       }
       __syncwarp();  // the row buffer is free for the next step
     }
-    if (a.rope) {  // inverse pairs: x0 = y0 c + y1 s, x1 = y1 c - y0 s
+    if (a.rope == 1) {  // inverse pairs: x0 = y0 c + y1 s, x1 = y1 c - y0 s
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D) + (V / 4) * s;
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
@@ -374,6 +385,16 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
         const float2 y0 = P[2 * g], y1 = P[2 * g + 1];
         P[2 * g] = fma2(y0, cc, mul2(y1, ss));
         P[2 * g + 1] = fma2(y1, cc, mul2(y0, f2(-ss.x, -ss.y)));
+      }
+    } else if (a.rope == 2) {  // half-split pairs across the lane pair
+      const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D);
+#pragma unroll
+      for (int g = 0; g < V / 4; ++g) {
+        const uint4 c0 = __ldg(rp + 2 * g), c1 = __ldg(rp + 2 * g + 1);
+        P[2 * g] = rope_half_inv2(P[2 * g], f2(__uint_as_float(c0.x), __uint_as_float(c1.x)),
+                                  f2(__uint_as_float(c0.y), __uint_as_float(c1.y)), s != 0, 1);
+        P[2 * g + 1] = rope_half_inv2(P[2 * g + 1], f2(__uint_as_float(c0.z), __uint_as_float(c1.z)),
+                                      f2(__uint_as_float(c0.w), __uint_as_float(c1.w)), s != 0, 1);
       }
     }
     // output words of this lane's half row (a sink slot comes back verbatim)

@@ -3,12 +3,17 @@
 //   rho = ||x||, u = x / (rho + 1e-8), per 4-D block v: w = qL (x) v (x) qR,
 //   scalar Lloyd-Max codes against a fixed codebook, LSB-first packing, and
 //   rho stored as fp32. Decode applies the inverse rotation and restores rho.
+// The 3-D variant (§2.1: T(v) = q v q* on pure quaternions; §1: 3-channel
+// blocks leave 42 blocks and a 2-D tail at d = 128) rotates blocks of three
+// channels, turns a 2-channel tail in its own plane with the same sandwich
+// and keeps a 1-channel tail.
 //
 // One thread per vector. The quaternion sandwich of block k is applied as
-// the 4x4 matrix M_k = L(qL_k) R(qR_k) (left / right multiplication
-// matrices of the Hamilton product), built once per CTA in shared memory:
-// 16 multiply-adds per block instead of two quaternion products. M_k is
-// orthogonal, so the inverse is M_k^T. The division by rho + eps is a
+// its matrix, built once per CTA in shared memory: M_k = L(qL_k) R(qR_k)
+// (left / right multiplication matrices of the Hamilton product), 16
+// multiply-adds per 4-D block instead of two quaternion products, or the 3x3
+// vector part of L(q_k) R(q_k*) for the 3-D sandwich. The matrices are
+// orthogonal, so the inverse is the transpose. The division by rho + eps is a
 // multiplication by its reciprocal. Both reorder fp32 rounding relative to
 // the literal sandwich, so a code can differ by one level where w sits
 // within a few ulps of a decision boundary.
@@ -57,15 +62,55 @@ __device__ __forceinline__ void build_m(const float* qL, const float* qR, float*
   }
 }
 
-template <int D, int BITS>
+// The 3-D sandwich's matrix of entry k (k < nblk = ceil(D/3)): rows / columns
+// i, j channels (i, j, k parts) of L(q) R(q*), row-major 3x3.
+__device__ __forceinline__ void build_m3(const float* q, float* M, int nblk) {
+  for (int k = threadIdx.x; k < nblk; k += blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(q)[k];
+    const float4 b = make_float4(a.x, -a.y, -a.z, -a.w);  // q*
+    const float L[4][4] = {{a.x, -a.y, -a.z, -a.w}, {a.y, a.x, -a.w, a.z}, {a.z, a.w, a.x, -a.y},
+                           {a.w, -a.z, a.y, a.x}};
+    const float R[4][4] = {{b.x, -b.y, -b.z, -b.w}, {b.y, b.x, b.w, -b.z}, {b.z, -b.w, b.x, b.y},
+                           {b.w, b.z, -b.y, b.x}};
+#pragma unroll
+    for (int i = 1; i < 4; ++i)
+#pragma unroll
+      for (int j = 1; j < 4; ++j) {
+        float s = __fmul_rn(L[i][0], R[0][j]);
+#pragma unroll
+        for (int t = 1; t < 4; ++t) s = __fmaf_rn(L[i][t], R[t][j], s);
+        M[k * 9 + (i - 1) * 3 + (j - 1)] = s;
+      }
+  }
+}
+
+// code = number of midpoints strictly below w (binary search)
+template <int NL>
+__device__ __forceinline__ uint32_t cb_code(float w, const float* beta) {
+  uint32_t c = 0;
+#pragma unroll
+  for (int s = NL / 2; s >= 1; s >>= 1)
+    if (w > beta[c + s - 1]) c += s;
+  return c;
+}
+
+template <int BITS, int NW>
+__device__ __forceinline__ void put_code(uint32_t (&w)[NW], int j, uint32_t c) {
+  const int pos = j * BITS;
+  w[pos >> 5] |= c << (pos & 31);
+  if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= c >> (32 - (pos & 31));
+}
+
+template <int D, int BITS, bool SO3>
 __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUtensorMap xmap, const IsoArgs a) {
   constexpr int NB = D / 4;
+  constexpr int NB3 = D / 3, TAIL = D % 3;  // 3-D sandwich blocks, tail channels
   constexpr int NL = 1 << BITS;
   constexpr int NW = D * BITS / 32;
   constexpr int RB = D * BITS / 8;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar;
-  __shared__ __align__(16) float Ms[NB * 16];
+  __shared__ __align__(16) float Ms[NB * 16];  // holds the 3x3 matrices too (9 * ceil(D/3) < 4 D)
   __shared__ float beta[NL];
   uint8_t* xs = align1024(smem_raw);
   const int tid = threadIdx.x;
@@ -81,7 +126,10 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
 #pragma unroll
     for (int hh = 0; hh < D / 64; ++hh) tma_load_2d(xs + hh * 16384, &xmap, hh * 64, static_cast<int>(r0), &bar);
   }
-  build_m(a.qL, a.qR, Ms, NB);
+  if constexpr (SO3)
+    build_m3(a.qL, Ms, NB3 + (TAIL ? 1 : 0));
+  else
+    build_m(a.qL, a.qR, Ms, NB);
   if (tid < NL - 1) beta[tid] = __fmul_rn(0.5f, __fadd_rn(a.codebook[tid], a.codebook[tid + 1]));
   __syncthreads();
   if (!mbar_wait(&bar, 0, a.wait_ns, a.err)) {
@@ -116,27 +164,48 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
   uint32_t w[NW];
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
+  if constexpr (!SO3) {
 #pragma unroll
-  for (int k = 0; k < NB; ++k) {
-    float u[4];
+    for (int k = 0; k < NB; ++k) {
+      float u[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) u[e] = __fmul_rn(x[4 * k + e], inv);
-    const float4* Mk = reinterpret_cast<const float4*>(Ms + k * 16);
+      for (int e = 0; e < 4; ++e) u[e] = __fmul_rn(x[4 * k + e], inv);
+      const float4* Mk = reinterpret_cast<const float4*>(Ms + k * 16);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 row = Mk[i];
-      float wi = __fmul_rn(row.x, u[0]);
-      wi = __fmaf_rn(row.y, u[1], wi);
-      wi = __fmaf_rn(row.z, u[2], wi);
-      wi = __fmaf_rn(row.w, u[3], wi);
-      // code = number of midpoints strictly below wi (binary search)
-      uint32_t c = 0;
+      for (int i = 0; i < 4; ++i) {
+        const float4 row = Mk[i];
+        float wi = __fmul_rn(row.x, u[0]);
+        wi = __fmaf_rn(row.y, u[1], wi);
+        wi = __fmaf_rn(row.z, u[2], wi);
+        wi = __fmaf_rn(row.w, u[3], wi);
+        put_code<BITS, NW>(w, 4 * k + i, cb_code<NL>(wi, beta));
+      }
+    }
+  } else {
 #pragma unroll
-      for (int s = NL / 2; s >= 1; s >>= 1)
-        if (wi > beta[c + s - 1]) c += s;
-      const int j = 4 * k + i, pos = j * BITS;
-      w[pos >> 5] |= c << (pos & 31);
-      if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= c >> (32 - (pos & 31));
+    for (int k = 0; k < NB3; ++k) {
+      float u[3];
+#pragma unroll
+      for (int e = 0; e < 3; ++e) u[e] = __fmul_rn(x[3 * k + e], inv);
+      const float* Mk = Ms + k * 9;
+#pragma unroll
+      for (int i = 0; i < 3; ++i) {
+        float wi = __fmul_rn(Mk[3 * i], u[0]);
+        wi = __fmaf_rn(Mk[3 * i + 1], u[1], wi);
+        wi = __fmaf_rn(Mk[3 * i + 2], u[2], wi);
+        put_code<BITS, NW>(w, 3 * k + i, cb_code<NL>(wi, beta));
+      }
+    }
+    if constexpr (TAIL == 2) {  // the tail in its own plane: the matrix's upper-left 2x2 block
+      const float u0 = __fmul_rn(x[D - 2], inv), u1 = __fmul_rn(x[D - 1], inv);
+      const float* Mk = Ms + NB3 * 9;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float wi = __fmaf_rn(Mk[3 * i + 1], u1, __fmul_rn(Mk[3 * i], u0));
+        put_code<BITS, NW>(w, D - 2 + i, cb_code<NL>(wi, beta));
+      }
+    } else if constexpr (TAIL == 1) {  // a single channel is kept
+      put_code<BITS, NW>(w, D - 1, cb_code<NL>(__fmul_rn(x[D - 1], inv), beta));
     }
   }
   uint8_t* dst = a.codes + slot * RB;
@@ -151,10 +220,11 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
   a.norm[slot] = rho;
 }
 
-template <int D, int BITS>
+template <int D, int BITS, bool SO3>
 __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUtensorMap omap, const IsoArgs a,
                                                      int out_fp32) {
   constexpr int NB = D / 4;
+  constexpr int NB3 = D / 3, TAIL = D % 3;
   constexpr int NL = 1 << BITS;
   constexpr int NW = D * BITS / 32;
   constexpr int RB = D * BITS / 8;
@@ -164,7 +234,10 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
   uint8_t* os = align1024(smem_raw);
   const int tid = threadIdx.x;
   const long long r0 = static_cast<long long>(blockIdx.x) * 128;
-  build_m(a.qL, a.qR, Ms, NB);
+  if constexpr (SO3)
+    build_m3(a.qL, Ms, NB3 + (TAIL ? 1 : 0));
+  else
+    build_m(a.qL, a.qR, Ms, NB);
   if (tid < NL) lv[tid] = a.codebook[tid];
   __syncthreads();
   const long long vid = r0 + tid;
@@ -195,19 +268,45 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
         }
       }
       const float rho = a.norm[slot];
+      if constexpr (!SO3) {
 #pragma unroll
-      for (int k = 0; k < NB; ++k) {
-        float wh[4];
+        for (int k = 0; k < NB; ++k) {
+          float wh[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) wh[e] = lv[unpack_code<BITS, NW>(w, 4 * k + e)];
-        const float* Mk = Ms + k * 16;
+          for (int e = 0; e < 4; ++e) wh[e] = lv[unpack_code<BITS, NW>(w, 4 * k + e)];
+          const float* Mk = Ms + k * 16;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // v = M^T w
-          float vi = __fmul_rn(Mk[i], wh[0]);
-          vi = __fmaf_rn(Mk[4 + i], wh[1], vi);
-          vi = __fmaf_rn(Mk[8 + i], wh[2], vi);
-          vi = __fmaf_rn(Mk[12 + i], wh[3], vi);
-          x[4 * k + i] = __fmul_rn(vi, rho);
+          for (int i = 0; i < 4; ++i) {  // v = M^T w
+            float vi = __fmul_rn(Mk[i], wh[0]);
+            vi = __fmaf_rn(Mk[4 + i], wh[1], vi);
+            vi = __fmaf_rn(Mk[8 + i], wh[2], vi);
+            vi = __fmaf_rn(Mk[12 + i], wh[3], vi);
+            x[4 * k + i] = __fmul_rn(vi, rho);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < NB3; ++k) {
+          float wh[3];
+#pragma unroll
+          for (int e = 0; e < 3; ++e) wh[e] = lv[unpack_code<BITS, NW>(w, 3 * k + e)];
+          const float* Mk = Ms + k * 9;
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {  // v = M^T w
+            float vi = __fmul_rn(Mk[i], wh[0]);
+            vi = __fmaf_rn(Mk[3 + i], wh[1], vi);
+            vi = __fmaf_rn(Mk[6 + i], wh[2], vi);
+            x[3 * k + i] = __fmul_rn(vi, rho);
+          }
+        }
+        if constexpr (TAIL == 2) {
+          const float w0 = lv[unpack_code<BITS, NW>(w, D - 2)], w1 = lv[unpack_code<BITS, NW>(w, D - 1)];
+          const float* Mk = Ms + NB3 * 9;
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+            x[D - 2 + i] = __fmul_rn(__fmaf_rn(Mk[3 + i], w1, __fmul_rn(Mk[i], w0)), rho);
+        } else if constexpr (TAIL == 1) {
+          x[D - 1] = __fmul_rn(lv[unpack_code<BITS, NW>(w, D - 1)], rho);
         }
       }
     }
@@ -252,18 +351,18 @@ IsoArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p, 
   return a;
 }
 
-template <int D, int BITS>
+template <int D, int BITS, bool SO3>
 kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((a.rows + 127) / 128);
   if (enc) {
     const size_t smem = 1024 + D * 256;
-    auto k = k_encode_iso<D, BITS>;
+    auto k = k_encode_iso<D, BITS, SO3>;
     if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
     k<<<grid, 128, smem, st>>>(m0, a);
   } else {
     const size_t smem = 1024 + D * 512;
-    auto k = k_decode_iso<D, BITS>;
+    auto k = k_decode_iso<D, BITS, SO3>;
     if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
     k<<<grid, 128, smem, st>>>(m0, a, out_fp32);
@@ -273,8 +372,10 @@ kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, 
 
 kvq_status dispatch(bool enc, const kvq_desc& d, const IsoArgs& a, const CUtensorMap& m0, int out_fp32,
                     cudaStream_t st) {
-#define KVQ_CASE(D_, B_) \
-  if (d.head_dim == D_ && d.bits == B_) return run<D_, B_>(enc, a, m0, out_fp32, st);
+#define KVQ_CASE(D_, B_)                                                                  \
+  if (d.head_dim == D_ && d.bits == B_)                                                   \
+    return d.rot == KVQ_ROT_ISO_SO3 ? run<D_, B_, true>(enc, a, m0, out_fp32, st)         \
+                                    : run<D_, B_, false>(enc, a, m0, out_fp32, st);
   KVQ_CASE(128, 2)
   KVQ_CASE(128, 3)
   KVQ_CASE(128, 4)

@@ -125,17 +125,28 @@ __device__ __forceinline__ void score_afrag(const uint32_t (&wa)[NW], const uint
 
 // q . RoPE_n(sink_n) for an fp16 sink key by one warp (fp32; every lane gets
 // the sum): lane takes channels 4 lane .. 4 lane + 3, the lane sums are added
-// by an xor butterfly. rope_row: the position's (cos, sin) pairs, or nullptr.
+// by an xor butterfly. rope_row: the position's (cos, sin) pairs, or nullptr;
+// half: the half-split pairs (c, c + 64) (lane ^ 16 holds the partner
+// channels) instead of the interleaved (2i, 2i + 1).
 __device__ __forceinline__ float sink_dot(const float* qraw, const __half* sink_row, const float* rope_row,
-                                          int lane) {
+                                          int lane, bool half = false) {
   const uint2 kr = __ldg(reinterpret_cast<const uint2*>(sink_row) + lane);
   const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kr.x));
   const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kr.y));
   float k4[4] = {k01.x, k01.y, k23.x, k23.y};
-  if (rope_row) {  // pairs 2 lane and 2 lane + 1 of the sink's position
+  if (rope_row && !half) {  // pairs 2 lane and 2 lane + 1 of the sink's position
     const float4 cs = __ldg(reinterpret_cast<const float4*>(rope_row) + lane);
     rope_fwd(k4[0], k4[1], cs.x, cs.y);
     rope_fwd(k4[2], k4[3], cs.z, cs.w);
+  } else if (rope_row) {  // angles 4 (lane mod 16) .. + 3
+    const float4 c0 = __ldg(reinterpret_cast<const float4*>(rope_row) + 2 * (lane & 15));
+    const float4 c1 = __ldg(reinterpret_cast<const float4*>(rope_row) + 2 * (lane & 15) + 1);
+    const float2 y01 = rope_half_fwd2(f2(k4[0], k4[1]), f2(c0.x, c0.z), f2(c0.y, c0.w), lane >= 16, 16);
+    const float2 y23 = rope_half_fwd2(f2(k4[2], k4[3]), f2(c1.x, c1.z), f2(c1.y, c1.w), lane >= 16, 16);
+    k4[0] = y01.x;
+    k4[1] = y01.y;
+    k4[2] = y23.x;
+    k4[3] = y23.y;
   }
   float acc = 0.0f;
 #pragma unroll

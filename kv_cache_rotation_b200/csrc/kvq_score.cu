@@ -86,7 +86,29 @@ __global__ void __launch_bounds__(kThreads) k_score_simt(const ScoreArgs a) {
   for (int i = 0; i < GQ; ++i) acc[i] = 0.0f;
   const size_t vh = static_cast<size_t>(b) * a.H + h;
 
-  if (n < a.n_sink) {
+  if (n < a.n_sink && a.rope == 2) {  // half-split pairs (c, c + D/2): chunks c and c + D/16 together
+    const uint4* src = reinterpret_cast<const uint4*>(a.sink + (vh * a.n_sink + n) * D);
+    const float4* cs = reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(n) * D);
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      float lo[8], hi[8];
+      h8_to_f32(__ldg(src + c), lo);
+      h8_to_f32(__ldg(src + c + D / 16), hi);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {  // angles 8c + 2k, 8c + 2k + 1
+        const float4 t = __ldg(cs + 4 * c + k);
+        rope_fwd(lo[2 * k], hi[2 * k], t.x, t.y);
+        rope_fwd(lo[2 * k + 1], hi[2 * k + 1], t.z, t.w);
+      }
+#pragma unroll
+      for (int i = 0; i < GQ; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          acc[i] = __fmaf_rn(qr[i][8 * c + e], lo[e], acc[i]);
+          acc[i] = __fmaf_rn(qr[i][D / 2 + 8 * c + e], hi[e], acc[i]);
+        }
+    }
+  } else if (n < a.n_sink) {
     const uint4* src = reinterpret_cast<const uint4*>(a.sink + (vh * a.n_sink + n) * D);
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
@@ -156,22 +178,23 @@ __global__ void __launch_bounds__(kThreads) k_score_simt(const ScoreArgs a) {
 // mask per 4 codes, B = the digits, N = 2 columns (lo, hi) per query head.
 //   s_n = scale * sum_g ( S_g * sq * (sum_j c_j lo_j + 256 sum_j c_j hi_j) + Z_g * sum_{j in g} qt_j ).
 // The digit rounding moves each score by at most S * sq / 2 * sum_j c_j,
-// i.e. below 2e-5 of the score's L1 magnitude. Codes stream through shared
-// memory by bulk copy, two tiles of 128 tokens in flight; CTAs are
-// persistent over a range of tiles of one (batch, KV head) so the query
-// rotation is done once per CTA.
-// Tiling: 2 m-tiles of 16 tokens per warp (256-token tiles), 4 tiles in
-// flight per CTA, at most 4 CTAs per SM.
+// i.e. below 2e-5 of the score's L1 magnitude.
+// A CTA owns a contiguous range of 64-token blocks of one (batch, KV head):
+// it rotates and splits the queries once, then its 8 warps work independently
+// (no CTA barrier in the loop), each streaming every 8th block through its
+// own ring of kMmaStages stages: the records by one bulk copy (one mbarrier
+// per stage), the scale/zero words by 4-byte cp.async spread over the lanes.
+// A block is four m-tiles of 16 tokens.
 constexpr int kMmaThreads = 256;
-constexpr int kMmaMT = 2;                  // 16-token m-tiles per warp per tile
-constexpr int kMmaTile = 8 * 16 * kMmaMT;  // tokens per tile
-constexpr int kMmaStages = 4;              // tiles in flight per CTA
+constexpr int kMmaWarps = kMmaThreads / 32;
+constexpr int kMmaStages = 3;     // blocks in flight per warp
 constexpr int kMmaCtasPerSm = 4;
+constexpr int kMmaBlk = 64;       // tokens per block
 
 struct MmaArgs {
   ScoreArgs s;
-  int chunks, tiles_per_chunk;
-  FastDiv div_tpb, div_h;  // tiles per (batch, KV head); KV heads
+  int splits;  // CTAs per (batch, KV head)
+  int n_blk;   // 64-token blocks per (batch, KV head)
   uint32_t* err;
   uint64_t wait_ns;
 };
@@ -184,6 +207,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+template <int BITS, int G>
+__host__ __device__ constexpr int mma_stage_bytes() {
+  return kMmaBlk * (128 * BITS / 8) + kMmaBlk * (128 / G) * 4;  // records + scale/zero words of a block
+}
+
 template <int BITS, int G, int GQ>
 __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
   constexpr int D = 128;
@@ -191,114 +219,125 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
   constexpr int NW = RB / 4;             // words per record
   constexpr int NTN = (2 * GQ + 7) / 8;  // n-tiles of 8 columns
   constexpr int NGK = D / G;             // quantization groups per record
+  constexpr int CB = kMmaBlk * RB;       // records of one block
+  constexpr int NSZ = kMmaBlk * NGK;     // scale/zero words of one block
+  constexpr int STB = mma_stage_bytes<BITS, G>();
   const ScoreArgs& a = ma.s;
-  extern __shared__ __align__(128) uint8_t codes_dyn[];  // kMmaStages tiles of kMmaTile records
+  extern __shared__ __align__(128) uint8_t ring[];  // [warp][stage][STB]
   __shared__ __align__(16) uint2 bfrag[NTN][4][4][8];
   __shared__ __align__(16) float qraw[GQ][D];
   __shared__ int8_t qd[GQ][2][D];
   __shared__ float qsum[GQ][NGK];
   __shared__ float sqh[GQ];
-  __shared__ __align__(8) uint64_t full[kMmaStages];
+  __shared__ __align__(8) uint64_t full[kMmaWarps][kMmaStages];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tig = lane & 3;
-  // this CTA's contiguous range of global tiles (batch-major, then KV head, then token tile)
-  const int total = a.B * a.H * static_cast<int>(ma.div_tpb.d);
-  const int gt0 = static_cast<int>(static_cast<long long>(total) * blockIdx.x / gridDim.x);
-  const int gt1 = static_cast<int>(static_cast<long long>(total) * (blockIdx.x + 1) / gridDim.x);
-  if (gt0 >= gt1) return;
+  const int bh = static_cast<int>(blockIdx.x) / ma.splits, part = static_cast<int>(blockIdx.x) % ma.splits;
+  const int b = bh / a.H, h = bh - b * a.H;
+  const int blk0 = static_cast<int>(static_cast<long long>(ma.n_blk) * part / ma.splits);
+  const int blk1 = static_cast<int>(static_cast<long long>(ma.n_blk) * (part + 1) / ma.splits);
+  const int n_my = blk1 - blk0 > warp ? (blk1 - blk0 - warp + kMmaWarps - 1) / kMmaWarps : 0;  // this warp's blocks
+  uint8_t* const wring = ring + warp * (kMmaStages * STB);
+  const size_t rec0 = static_cast<size_t>(bh) * a.t_cap;  // slot of token 0 of this stream
 
-  auto issue = [&](int gt, int st) {
-    const int bh = static_cast<int>(ma.div_tpb.div(gt));
-    const int n0 = static_cast<int>(ma.div_tpb.mod(gt, bh)) * kMmaTile;
-    const uint32_t bytes = static_cast<uint32_t>(min(kMmaTile, a.n_tok - n0) * RB);
-    mbar_arrive_expect_tx(&full[st], bytes);
-    bulk_load(codes_dyn + st * (kMmaTile * RB), a.codes + (static_cast<size_t>(bh) * a.t_cap + n0) * RB, bytes,
-              &full[st]);
+  // this warp's i-th block -> stage i % kMmaStages (records by bulk copy, words by cp.async)
+  auto issue = [&](int i) {
+    uint8_t* dst = wring + (i % kMmaStages) * STB;
+    const int n0 = (blk0 + warp + i * kMmaWarps) * kMmaBlk;
+    const int nv = i < n_my ? min(kMmaBlk, a.n_tok - n0) : 0;
+    if (nv > 0 && lane == 0) {
+      fence_async_smem();
+      mbar_arrive_expect_tx(&full[warp][i % kMmaStages], static_cast<uint32_t>(nv * RB));
+      bulk_load(dst, a.codes + (rec0 + n0) * RB, static_cast<uint32_t>(nv * RB), &full[warp][i % kMmaStages]);
+    }
+#pragma unroll
+    for (int e = lane; e < NSZ; e += 32) {
+      const bool live = e / NGK < nv;
+      cp_async4(smem_u32(dst + CB + e * 4), live ? static_cast<const void*>(a.sz + (rec0 + n0) * NGK + e) : a.sz,
+                live ? 4u : 0u);
+    }
+    cp_async_commit();
   };
-  if (tid == 0) {
-    for (int i = 0; i < kMmaStages; ++i) mbar_init(&full[i], 1);
+  if (lane == 0) {
+    for (int i = 0; i < kMmaStages; ++i) mbar_init(&full[warp][i], 1);
     fence_mbar_init();
   }
-  __syncthreads();
-  if (tid == 0) {
-    for (int i = 0; i < kMmaStages && gt0 + i < gt1; ++i) issue(gt0 + i, i);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < kMmaStages; ++i) issue(i);
+
+  // rotated, digit-split queries of this (batch, KV head); warp w < GQ handles query head w
+  if (warp < GQ) {
+    const int qh = h * GQ + warp;
+    query_digits<G>(a.q + (static_cast<size_t>(b) * a.Hq + qh) * D, a.perm ? a.perm + static_cast<size_t>(h) * D : nullptr,
+                    a.rot, a.rscale, lane, qraw[warp], qd[warp][0], qd[warp][1], qsum[warp], &sqh[warp]);
   }
+  __syncthreads();
+  build_score_bfrag<BITS, GQ, NTN>(bfrag, qd, tid, kMmaThreads);  // column c = 2 * head + digit
+  __syncthreads();
+  // fp16 sinks: s = scale * q . RoPE_n(sink_n), by the CTA that owns the stream's first block
+  if (part == 0) {
+    for (int e = warp; e < min(a.n_sink, a.n_tok) * GQ; e += kMmaWarps) {
+      const int n = e / GQ, hh = e % GQ;
+      const float acc = sink_dot(qraw[hh], a.sink + (static_cast<size_t>(bh) * a.n_sink + n) * D,
+                                 a.rope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane, a.rope == 2);
+      if (lane == 0) a.scores[(static_cast<size_t>(b) * a.Hq + h * GQ + hh) * a.n_tok + n] = acc * a.scale;
+    }
+  }
+  uint2 bq[4][NTN];  // this lane's B fragments, kept in registers
+#pragma unroll
+  for (int nt = 0; nt < NTN; ++nt)
+#pragma unroll
+    for (int s = 0; s < 4; ++s) bq[s][nt] = bfrag[nt][s][tig][g];
+  float sqv[NTN], qsv[NTN][NGK];  // sq and the group sums of this lane's query head per n-tile
+#pragma unroll
+  for (int nt = 0; nt < NTN; ++nt) {
+    const int hh = min(nt * 4 + tig, GQ - 1);
+    sqv[nt] = sqh[hh];
+#pragma unroll
+    for (int q = 0; q < NGK; ++q) qsv[nt][q] = qsum[hh][q];
+  }
+  float* const out_h = a.scores + (static_cast<size_t>(b) * a.Hq + h * GQ) * a.n_tok;  // query head h*GQ
 
-  // rotated, digit-split queries of one (batch, KV head); warp w < GQ handles query head w
-  auto prologue = [&](int b, int h, bool with_sinks) {
-    __syncthreads();  // previous (batch, head) fully consumed
-    if (warp < GQ) {
-      const int qh = h * GQ + warp;
-      query_digits<G>(a.q + (static_cast<size_t>(b) * a.Hq + qh) * D,
-                      a.perm ? a.perm + static_cast<size_t>(h) * D : nullptr, a.rot, a.rscale, lane, qraw[warp],
-                      qd[warp][0], qd[warp][1], qsum[warp], &sqh[warp]);
+  int i_fail = -1;
+  for (int i = 0; i < n_my; ++i) {
+    const int st = i % kMmaStages;
+    const bool ok = mbar_wait(&full[warp][st], (i / kMmaStages) & 1, ma.wait_ns, ma.err);
+    if (!__all_sync(0xffffffffu, ok)) {
+      i_fail = i;
+      break;
     }
-    __syncthreads();
-    build_score_bfrag<BITS, GQ, NTN>(bfrag, qd, tid, kMmaThreads);  // column c = 2 * head + digit
-    __syncthreads();
-    // fp16 sinks of this (batch, head): s = scale * q . RoPE_n(sink_n); done by the
-    // CTA that owns the (batch, head)'s first tile, one warp per (sink, query head)
-    if (with_sinks) {
-      const size_t vh = static_cast<size_t>(b) * a.H + h;
-      for (int e = warp; e < min(a.n_sink, a.n_tok) * GQ; e += kMmaThreads / 32) {
-        const int n = e / GQ, hh = e % GQ;
-        const float acc = sink_dot(qraw[hh], a.sink + (vh * a.n_sink + n) * D,
-                                   a.rope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane);
-        if (lane == 0) a.scores[(static_cast<size_t>(b) * a.Hq + h * GQ + hh) * a.n_tok + n] = acc * a.scale;
-      }
-    }
-  };
-  // scale / zero of this thread's tokens of one tile (register prefetch)
-  auto load_sz = [&](int gt, __half2 (&sza)[kMmaMT][NGK], __half2 (&szb)[kMmaMT][NGK]) {
-    const int bh = static_cast<int>(ma.div_tpb.div(gt));
-    const int n0 = static_cast<int>(ma.div_tpb.mod(gt, bh)) * kMmaTile;
+    cp_async_wait_group<kMmaStages - 1>();
+    __syncwarp();  // the stage's records and words are visible to the whole warp
+    const uint8_t* sb = wring + st * STB;
+    const int n0 = (blk0 + warp + i * kMmaWarps) * kMmaBlk;
+    const int nv = min(kMmaBlk, a.n_tok - n0);
 #pragma unroll
-    for (int mt = 0; mt < kMmaMT; ++mt) {
-      const int na = n0 + warp * 16 * kMmaMT + mt * 16 + g, nb = na + 8;
-#pragma unroll
-      for (int q = 0; q < NGK; ++q) {
-        sza[mt][q] = na < a.n_tok ? a.sz[(static_cast<size_t>(bh) * a.t_cap + na) * NGK + q] : __half2();
-        szb[mt][q] = nb < a.n_tok ? a.sz[(static_cast<size_t>(bh) * a.t_cap + nb) * NGK + q] : __half2();
-      }
-    }
-  };
-
-  __half2 sza[kMmaMT][NGK], szb[kMmaMT][NGK];
-  load_sz(gt0, sza, szb);
-  int cur_bh = -1;
-  bool ok = true;
-  int gt_fail = gt1;  // first tile whose copy was not seen to land
-  for (int gt = gt0; gt < gt1; ++gt) {
-    const int it = gt - gt0;
-    const int st = it % kMmaStages;
-    const int bh = static_cast<int>(ma.div_tpb.div(gt));
-    const int b = static_cast<int>(ma.div_h.div(bh)), h = bh - b * a.H;
-    const int n0 = static_cast<int>(ma.div_tpb.mod(gt, bh)) * kMmaTile;
-    if (bh != cur_bh) {
-      prologue(b, h, n0 == 0);
-      cur_bh = bh;
-    }
-    ok = mbar_wait(&full[st], (it / kMmaStages) & 1, ma.wait_ns, ma.err) && ok;
-    const uint32_t base = smem_u32(codes_dyn + st * (kMmaTile * RB));
-    int acc[kMmaMT][NGK][NTN][4];
-#pragma unroll
-    for (int mt = 0; mt < kMmaMT; ++mt) {
-      const int ra = warp * 16 * kMmaMT + mt * 16 + g;  // tile rows ra and ra + 8
+    for (int mt = 0; mt < kMmaBlk / 16; ++mt) {
+      if (mt * 16 >= nv) break;
+      const int ra = mt * 16 + g;  // block rows ra and ra + 8
       uint32_t wa[NW], wb[NW];
 #pragma unroll
-      for (int i = 0; i < NW / 4; ++i) {
-        const uint4 ua = lds128(base + ra * RB + 16 * i);
-        const uint4 ub = lds128(base + (ra + 8) * RB + 16 * i);
-        wa[4 * i] = ua.x; wa[4 * i + 1] = ua.y; wa[4 * i + 2] = ua.z; wa[4 * i + 3] = ua.w;
-        wb[4 * i] = ub.x; wb[4 * i + 1] = ub.y; wb[4 * i + 2] = ub.z; wb[4 * i + 3] = ub.w;
+      for (int k = 0; k < NW / 4; ++k) {
+        const uint4 ua = *reinterpret_cast<const uint4*>(sb + ra * RB + 16 * k);
+        const uint4 ub = *reinterpret_cast<const uint4*>(sb + (ra + 8) * RB + 16 * k);
+        wa[4 * k] = ua.x; wa[4 * k + 1] = ua.y; wa[4 * k + 2] = ua.z; wa[4 * k + 3] = ua.w;
+        wb[4 * k] = ub.x; wb[4 * k + 1] = ub.y; wb[4 * k + 2] = ub.z; wb[4 * k + 3] = ub.w;
       }
+      float2 sza[NGK], szb[NGK];  // (S, Z) of rows ra and ra + 8
+#pragma unroll
+      for (int q = 0; q < NGK; ++q) {
+        sza[q] = __half22float2(*reinterpret_cast<const __half2*>(sb + CB + (ra * NGK + q) * 4));
+        szb[q] = __half22float2(*reinterpret_cast<const __half2*>(sb + CB + ((ra + 8) * NGK + q) * 4));
+      }
+      int acc[NGK][NTN][4];
 #pragma unroll
       for (int q = 0; q < NGK; ++q)
 #pragma unroll
         for (int nt = 0; nt < NTN; ++nt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) acc[mt][q][nt][i] = 0;
+          for (int e = 0; e < 4; ++e) acc[q][nt][e] = 0;
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         uint32_t a0, a1, a2, a3;
@@ -306,56 +345,46 @@ __global__ void __launch_bounds__(kMmaThreads) k_score_mma(const MmaArgs ma) {
         constexpr int SPG = G / 32;  // k-steps per group
         const int q = s / SPG;
 #pragma unroll
-        for (int nt = 0; nt < NTN; ++nt) mma_u8s8(acc[mt][q][nt], a0, a1, a2, a3, bfrag[nt][s][tig][g]);
+        for (int nt = 0; nt < NTN; ++nt) mma_u8s8(acc[q][nt], a0, a1, a2, a3, bq[s][nt]);
       }
-    }
-    // every warp has read this stage: refill it with the tile kMmaStages ahead
-    if (!__syncthreads_and(ok)) {
-      gt_fail = gt;
-      break;
-    }
-    if (tid == 0 && gt + kMmaStages < gt1) issue(gt + kMmaStages, st);
-    __half2 pa[kMmaMT][NGK], pb[kMmaMT][NGK];
-#pragma unroll
-    for (int mt = 0; mt < kMmaMT; ++mt)
-#pragma unroll
-      for (int q = 0; q < NGK; ++q) {
-        pa[mt][q] = sza[mt][q];
-        pb[mt][q] = szb[mt][q];
-      }
-    if (gt + 1 < gt1) load_sz(gt + 1, sza, szb);  // next tile's scale / zero
-    // epilogue: thread holds columns 2 tig (lo) and 2 tig + 1 (hi) = query head nt*4 + tig
-#pragma unroll
-    for (int mt = 0; mt < kMmaMT; ++mt) {
-      const int na = n0 + warp * 16 * kMmaMT + mt * 16 + g, nb = na + 8;
+      // epilogue: lane holds columns 2 tig (lo) and 2 tig + 1 (hi) = query head nt*4 + tig
+      const int na = n0 + ra, nb = na + 8;
+      const bool full_tile = n0 + mt * 16 >= a.n_sink && n0 + mt * 16 + 16 <= a.n_tok;
 #pragma unroll
       for (int nt = 0; nt < NTN; ++nt) {
         const int hh = nt * 4 + tig;
         if (hh >= GQ) continue;
-        const float sq = sqh[hh];
-        float sa = 0.0f, sb = 0.0f;
+        float sa = 0.0f, sbv = 0.0f;
 #pragma unroll
         for (int q = 0; q < NGK; ++q) {
-          const float da = static_cast<float>(acc[mt][q][nt][0] + 256 * acc[mt][q][nt][1]);
-          const float db = static_cast<float>(acc[mt][q][nt][2] + 256 * acc[mt][q][nt][3]);
-          sa = __fmaf_rn(__low2float(pa[mt][q]) * sq, da, __fmaf_rn(__high2float(pa[mt][q]), qsum[hh][q], sa));
-          sb = __fmaf_rn(__low2float(pb[mt][q]) * sq, db, __fmaf_rn(__high2float(pb[mt][q]), qsum[hh][q], sb));
+          const float da = static_cast<float>(acc[q][nt][0] + 256 * acc[q][nt][1]);
+          const float db = static_cast<float>(acc[q][nt][2] + 256 * acc[q][nt][3]);
+          sa = __fmaf_rn(sza[q].x * sqv[nt], da, __fmaf_rn(sza[q].y, qsv[nt][q], sa));
+          sbv = __fmaf_rn(szb[q].x * sqv[nt], db, __fmaf_rn(szb[q].y, qsv[nt][q], sbv));
         }
-        float* out = a.scores + (static_cast<size_t>(b) * a.Hq + h * GQ + hh) * a.n_tok;
-        if (na < a.n_tok && na >= a.n_sink) out[na] = sa * a.scale;
-        if (nb < a.n_tok && nb >= a.n_sink) out[nb] = sb * a.scale;
+        float* out = out_h + static_cast<size_t>(hh) * a.n_tok;
+        sa = sa * a.scale;
+        sbv = sbv * a.scale;
+        if (full_tile) {
+          out[na] = sa;
+          out[nb] = sbv;
+        } else {
+          if (na < a.n_tok && na >= a.n_sink) out[na] = sa;
+          if (nb < a.n_tok && nb >= a.n_sink) out[nb] = sbv;
+        }
       }
     }
+    __syncwarp();  // every lane has read the stage: refill it with the block kMmaStages ahead
+    issue(i + kMmaStages);
   }
-  // After a timed-out wait, let the copies still in flight land (bounded)
-  // before the CTA exits: tiles gt_fail .. gt_fail + kMmaStages - 1 were
-  // issued and not consumed; each is waited on once, at its stage and phase.
-  if (gt_fail < gt1 && tid == 0) {
-    for (int gt = gt_fail; gt < gt1 && gt < gt_fail + kMmaStages; ++gt) {
-      const int it = gt - gt0;
-      mbar_wait(&full[it % kMmaStages], (it / kMmaStages) & 1, ma.wait_ns, ma.err);
-    }
+  // After a timed-out wait, let this warp's copies still in flight land
+  // (bounded) before the CTA exits: blocks i_fail .. i_fail + kMmaStages - 1
+  // were issued and not consumed; each is waited on once, at its stage and phase.
+  if (i_fail >= 0 && lane == 0) {
+    for (int i = i_fail; i < n_my && i < i_fail + kMmaStages; ++i)
+      mbar_wait(&full[warp][i % kMmaStages], (i / kMmaStages) & 1, ma.wait_ns, ma.err);
   }
+  cp_async_wait_all();
 }
 
 template <int BITS, int G, int GQ>
@@ -364,20 +393,22 @@ kvq_status run_mma(const ScoreArgs& a, const LaunchCtx& ctx, cudaStream_t st) {
   ma.s = a;
   ma.err = ctx.err;
   ma.wait_ns = ctx.wait_ns;
-  const size_t smem = static_cast<size_t>(kMmaStages) * kMmaTile * (128 * BITS / 8);
-  if (!set_smem_once(reinterpret_cast<const void*>(k_score_mma<BITS, G, GQ>), smem)) return KVQ_ERR_CUDA;
-  int per_sm = occupancy_once(reinterpret_cast<const void*>(k_score_mma<BITS, G, GQ>), kMmaThreads, smem);
+  const size_t smem = static_cast<size_t>(kMmaWarps) * kMmaStages * mma_stage_bytes<BITS, G>();
+  const void* fn = reinterpret_cast<const void*>(k_score_mma<BITS, G, GQ>);
+  if (!set_smem_once(fn, smem)) return KVQ_ERR_CUDA;
+  int per_sm = occupancy_once(fn, kMmaThreads, smem);
   per_sm = per_sm > kMmaCtasPerSm ? kMmaCtasPerSm : per_sm;
-  const int tpb = (a.n_tok + kMmaTile - 1) / kMmaTile;
-  const long long total = static_cast<long long>(a.B) * a.H * tpb;
-  if (total >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
-  ma.div_tpb = FastDiv(static_cast<uint32_t>(tpb));
-  ma.div_h = FastDiv(static_cast<uint32_t>(a.H));
-  long long grid = static_cast<long long>(ctx.num_sms) * per_sm;
-  if (grid > total) grid = total;
-  ma.chunks = static_cast<int>(grid);
-  ma.tiles_per_chunk = 0;
-  k_score_mma<BITS, G, GQ><<<static_cast<unsigned>(grid), kMmaThreads, smem, st>>>(ma);
+  ma.n_blk = (a.n_tok + kMmaBlk - 1) / kMmaBlk;
+  const long long streams = static_cast<long long>(a.B) * a.H;
+  // as many CTAs per stream as one wave holds (rounded down: a partial second
+  // wave would double the tail); each of a stream's CTAs takes at least one block per warp
+  long long splits = static_cast<long long>(ctx.num_sms) * per_sm / streams;
+  const long long max_splits = (ma.n_blk + kMmaWarps - 1) / kMmaWarps;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  if (streams * splits >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+  ma.splits = static_cast<int>(splits);
+  k_score_mma<BITS, G, GQ><<<static_cast<unsigned>(streams * splits), kMmaThreads, smem, st>>>(ma);
   return launch_status();
 }
 

@@ -14,12 +14,13 @@ from typing import Optional
 import torch
 
 from . import (KVQ_FIELD_CODES, KVQ_FIELD_NORM, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_Q_CODEBOOK,
-               KVQ_Q_MINMAX, KVQ_ROT_FWHT_GROUP, KVQ_ROT_FWHT_HEAD, KVQ_ROT_ISO_SO4, KVQ_ROT_NONE, check,
+               KVQ_Q_MINMAX, KVQ_ROT_FWHT_GROUP, KVQ_ROT_FWHT_HEAD, KVQ_ROT_ISO_SO3, KVQ_ROT_ISO_SO4, KVQ_ROT_NONE,
+               check,
                kvq_decode, kvq_desc, kvq_encode, kvq_lloyd_max_codebook, kvq_packed, kvq_packed_bytes,
                kvq_rope_table, kvq_score, kvq_tables)
 
 ROT = {"none": KVQ_ROT_NONE, "fwht_head": KVQ_ROT_FWHT_HEAD, "fwht_group": KVQ_ROT_FWHT_GROUP,
-       "iso": KVQ_ROT_ISO_SO4}
+       "iso": KVQ_ROT_ISO_SO4, "iso3": KVQ_ROT_ISO_SO3}
 QUANT = {"minmax": KVQ_Q_MINMAX, "codebook": KVQ_Q_CODEBOOK}
 
 

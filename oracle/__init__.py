@@ -25,7 +25,7 @@ _LIB_PATH = os.path.join(_HERE, "libkvq_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-ROT_NONE, ROT_FWHT_HEAD, ROT_FWHT_GROUP, ROT_ISO = 0, 1, 2, 3
+ROT_NONE, ROT_FWHT_HEAD, ROT_FWHT_GROUP, ROT_ISO, ROT_ISO3 = 0, 1, 2, 3, 4
 Q_MINMAX, Q_CODEBOOK = 0, 1
 
 CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
@@ -66,6 +66,7 @@ def lib():
         L.orc_rope_theta.argtypes = [ci, ci, cd, ci]
         L.orc_rope_cs.argtypes = [ctypes.c_int64, ci, cd, ci, f32p, f32p]
         L.orc_rope_apply_f32.argtypes = [f32p, f32p, f32p, f32p, ci]
+        L.orc_rope_apply_f32_mode.argtypes = [f32p, f32p, f32p, f32p, ci, ci]
         L.orc_rope_apply_f64.argtypes = [f64p, f64p, ctypes.c_int64, ci, cd, ci, ci]
         L.orc_fwht_f32.argtypes = [f32p, ci]
         L.orc_fwht_f64.argtypes = [f64p, ci]
@@ -111,6 +112,8 @@ def float_to_half(f: float, mode: str = "rn") -> int:
 # RoPE frequency tables, passed where a rope flag goes: ROPE_STD (1) the
 # standard theta_i = base^(-2i/d), ROPE_FREQ_AWARE (2) the frequency-aware table.
 ROPE_STD, ROPE_FREQ_AWARE = 1, 2
+# added to either: the half-split pairing (i, i + d/2) instead of the interleaved (2i, 2i + 1)
+ROPE_HALF = 4
 
 
 def rope_theta(i: int, d: int, base: float = 10000.0, mode: int = ROPE_STD) -> float:
@@ -124,12 +127,14 @@ def rope_cs(m: int, d: int, base: float = 10000.0, mode: int = ROPE_STD):
     return c, s
 
 
-def rope_f32(x, c, s):
+def rope_f32(x, c, s, mode: int = ROPE_STD):
+    """fp32 RoPE of one vector with the given (cos, sin); mode's ROPE_HALF bit
+    chooses the half-split pairs."""
     x = np.ascontiguousarray(x, np.float32)
     y = np.empty_like(x)
-    lib().orc_rope_apply_f32(_p(y, ctypes.c_float), _p(x, ctypes.c_float),
-                             _p(np.ascontiguousarray(c, np.float32), ctypes.c_float),
-                             _p(np.ascontiguousarray(s, np.float32), ctypes.c_float), x.size)
+    lib().orc_rope_apply_f32_mode(_p(y, ctypes.c_float), _p(x, ctypes.c_float),
+                                  _p(np.ascontiguousarray(c, np.float32), ctypes.c_float),
+                                  _p(np.ascontiguousarray(s, np.float32), ctypes.c_float), x.size, int(mode))
     return y
 
 
@@ -226,7 +231,7 @@ def encode(x, pos, *, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0,
     x = np.ascontiguousarray(x, np.uint16)
     B, H, T, D = x.shape
     pos = np.ascontiguousarray(pos, np.int64)
-    cs, zs, ss, ns = _packed_shapes(B, H, T, D, bits, group if rot != ROT_ISO else 0, n_sink)
+    cs, zs, ss, ns = _packed_shapes(B, H, T, D, bits, group if rot not in (ROT_ISO, ROT_ISO3) else 0, n_sink)
     codes = np.zeros(cs, np.uint8)
     sz = np.zeros(zs, np.uint16)
     sink = np.zeros(ss if n_sink > 0 else (1,), np.uint16)

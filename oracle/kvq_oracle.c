@@ -38,6 +38,7 @@
 #define ORC_ROT_FWHT_HEAD 1
 #define ORC_ROT_FWHT_GROUP 2
 #define ORC_ROT_ISO 3
+#define ORC_ROT_ISO3 4
 #define ORC_Q_MINMAX 0
 #define ORC_Q_CODEBOOK 1
 
@@ -127,14 +128,32 @@ uint16_t orc_float_to_half_ru(float f) {
  * Pins: R(a)R(b) = R(a+b) ([RoPE-KV §7.1]); the score depends only on m-n
  * ([EliteKV §2.2]).
  * ---------------------------------------------------------------------- */
-/* Frequency of pair i (0-based; the pages' j = i + 1). mode (the rope flag):
+/* Frequency of pair i (0-based; the pages' j = i + 1). mode (the rope flag),
+ * low two bits:
  * 1: the standard table theta_i = base^(-2i/d) ([EliteKV §2.1]);
  * 2: frequency-aware RoPE ([KV-Latent], frequency-aware RoPE): the first half
  *    of the pairs (i < d/4) take base^(-2(i + d/8)/d), the second half
  *    base^(-(i + 3d/4)/d): the highest frequencies are skipped and the low
- *    ones sampled twice as densely. */
+ *    ones sampled twice as densely.
+ * Bit 4 of the flag chooses the channel pairs: clear, pair i is the
+ * interleaved (2i, 2i+1) of the rotation matrix ([EliteKV §2.1]); set, it is
+ * the half-split (i, i + d/2) of the page's apply_rope code ([EliteKV §7.1]).
+ * Pins: both pairings rotate by the same angles, the half-split one is the
+ * interleaved one with the channels reordered, R(a)R(b) = R(a+b). */
+#define ORC_ROPE_HALF 4
+static void rope_pair(int i, int d, int mode, int* j0, int* j1) {
+  if (mode & ORC_ROPE_HALF) {
+    *j0 = i;
+    *j1 = i + d / 2;
+  } else {
+    *j0 = 2 * i;
+    *j1 = 2 * i + 1;
+  }
+}
+
 double orc_rope_theta(int i, int d, double base, int mode) {
-  if (mode == 2) return i < d / 4 ? pow(base, -2.0 * (i + d / 8) / d) : pow(base, -(double)(i + 3 * d / 4) / d);
+  if ((mode & 3) == 2)
+    return i < d / 4 ? pow(base, -2.0 * (i + d / 8) / d) : pow(base, -(double)(i + 3 * d / 4) / d);
   return pow(base, -(2.0 * i) / d);
 }
 
@@ -146,24 +165,33 @@ void orc_rope_cs(int64_t m, int d, double base, int mode, float* c, float* s) {
   }
 }
 
-void orc_rope_apply_f32(float* y, const float* x, const float* c, const float* s, int d) {
+/* the fp32 rotation on the pairs chosen by mode (see above) */
+void orc_rope_apply_f32_mode(float* y, const float* x, const float* c, const float* s, int d, int mode) {
   for (int i = 0; i < d / 2; ++i) {
-    float x0 = x[2 * i], x1 = x[2 * i + 1];
+    int j0, j1;
+    rope_pair(i, d, mode, &j0, &j1);
+    float x0 = x[j0], x1 = x[j1];
     float t1 = x1 * s[i];
     float t2 = x1 * c[i];
-    y[2 * i] = fmaf(x0, c[i], -t1);
-    y[2 * i + 1] = fmaf(x0, s[i], t2);
+    y[j0] = fmaf(x0, c[i], -t1);
+    y[j1] = fmaf(x0, s[i], t2);
   }
+}
+
+void orc_rope_apply_f32(float* y, const float* x, const float* c, const float* s, int d) {
+  orc_rope_apply_f32_mode(y, x, c, s, d, 1);
 }
 
 /* exact-angle rotation in fp64; inverse != 0 rotates by -m*theta */
 void orc_rope_apply_f64(double* y, const double* x, int64_t m, int d, double base, int mode, int inverse) {
   for (int i = 0; i < d / 2; ++i) {
+    int j0, j1;
+    rope_pair(i, d, mode, &j0, &j1);
     double ang = (double)m * orc_rope_theta(i, d, base, mode);
     double c = cos(ang), s = inverse ? -sin(ang) : sin(ang);
-    double x0 = x[2 * i], x1 = x[2 * i + 1];
-    y[2 * i] = x0 * c - x1 * s;
-    y[2 * i + 1] = x0 * s + x1 * c;
+    double x0 = x[j0], x1 = x[j1];
+    y[j0] = x0 * c - x1 * s;
+    y[j1] = x0 * s + x1 * c;
   }
 }
 
@@ -390,6 +418,8 @@ static int check_shape(const orc_shape* s) {
   if (s->bits < 2 || s->bits > 4) return 1;
   if (s->rot == ORC_ROT_ISO) {
     if (s->quant != ORC_Q_CODEBOOK || s->D % 4) return 1;
+  } else if (s->rot == ORC_ROT_ISO3) {
+    if (s->quant != ORC_Q_CODEBOOK) return 1;
   } else {
     if (s->quant != ORC_Q_MINMAX || s->group <= 0 || s->D % s->group) return 1;
   }
@@ -398,6 +428,58 @@ static int check_shape(const orc_shape* s) {
     if (hg <= 0 || (hg & (hg - 1)) || s->H % hg || hg * s->D > 2048) return 1;
   }
   return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * 3-D sandwich ([IsoQuant §2.1]: a unit quaternion q rotates a vector v,
+ * taken as the pure quaternion (0, v), by T(v) = q v q*; [IsoQuant §1]: with
+ * 3-channel blocks, d = 128 gives 42 whole blocks and a 2-D tail).
+ * Block k < D/3 is channels 3k .. 3k+2: w = q_k (x) ((0, u) (x) q_k*), the
+ * same association as the 4-D sandwich's listing, and the block's output is
+ * the vector part (w_i, w_j, w_k). A 2-channel tail (D mod 3 = 2) is the
+ * pure quaternion (0, u_{D-2}, u_{D-1}, 0) rotated by the next table entry,
+ * whose i and j parts are zero, so the sandwich turns the tail in its own
+ * plane; its output is (w_i, w_j). A 1-channel tail is left as it is. q holds
+ * ceil(D/3) unit quaternions (real, i, j, k).
+ * Pins: scipy's rotation of each block, the planar rotation of the tail,
+ * norm preservation, the block counts printed on the page.
+ * ---------------------------------------------------------------------- */
+static void iso3_rotate_f32(const float* u, const float* q, int D, float* w) {
+  int nb = D / 3;
+  for (int k = 0; k <= nb; ++k) {
+    int c = 3 * k, n = D - c < 3 ? D - c : 3;
+    if (n == 1) {
+      w[c] = u[c];
+      break;
+    }
+    if (n <= 0) break;
+    float v4[4] = {0.0f, u[c], u[c + 1], n == 3 ? u[c + 2] : 0.0f};
+    float qc[4] = {q[4 * k], -q[4 * k + 1], -q[4 * k + 2], -q[4 * k + 3]};
+    float t4[4], w4[4];
+    orc_quat_mul_f32(v4, qc, t4);
+    orc_quat_mul_f32(q + 4 * k, t4, w4);
+    for (int e = 0; e < n; ++e) w[c + e] = w4[1 + e];
+  }
+}
+
+/* inverse in fp64: v = q* (x) (w (x) q) on each block (q unit) */
+static void iso3_unrotate_f64(const double* w, const float* q, int D, double* v) {
+  int nb = D / 3;
+  for (int k = 0; k <= nb; ++k) {
+    int c = 3 * k, n = D - c < 3 ? D - c : 3;
+    if (n == 1) {
+      v[c] = w[c];
+      break;
+    }
+    if (n <= 0) break;
+    double w4[4] = {0.0, w[c], w[c + 1], n == 3 ? w[c + 2] : 0.0};
+    double qd[4] = {q[4 * k], q[4 * k + 1], q[4 * k + 2], q[4 * k + 3]};
+    double qc[4] = {qd[0], -qd[1], -qd[2], -qd[3]};
+    double t4[4], v4[4];
+    orc_quat_mul_f64(w4, qd, t4);
+    orc_quat_mul_f64(qc, t4, v4);
+    for (int e = 0; e < n; ++e) v[c + e] = v4[1 + e];
+  }
 }
 
 int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quant, int bits, int group,
@@ -423,13 +505,36 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
           if (m < n_sink) {
             memcpy(sink + ((size_t)(b * H + h0 + hl) * n_sink + m) * D, xv, sizeof(uint16_t) * D);
             memset(rec, 0, rb);
-            if (rot == ORC_ROT_ISO)
+            if (rot == ORC_ROT_ISO || rot == ORC_ROT_ISO3)
               norm[v] = 0.0f;
             else
               memset(sz + v * ng * 2, 0, sizeof(uint16_t) * ng * 2);
           }
         }
         if (m < n_sink) continue;
+
+        if (rot == ORC_ROT_ISO3) {
+          /* the norm split of [IsoQuant §3.1], then the 3-D sandwich on
+             3-channel blocks ([IsoQuant §2.1]); Lloyd-Max codes */
+          size_t v = ((size_t)(b * H + h0) * T + t);
+          const uint16_t* xv = x + v * D;
+          double acc = 0.0;
+          for (int j = 0; j < D; ++j) {
+            float f = orc_half_to_float(xv[j]);
+            acc += (double)f * (double)f;
+          }
+          float rho = (float)sqrt(acc);
+          float den = rho + 1e-8f;
+          float u[256], w[256];
+          for (int j = 0; j < D; ++j) u[j] = orc_half_to_float(xv[j]) / den;
+          iso3_rotate_f32(u, qL, D, w);
+          uint8_t cds[256];
+          for (int j = 0; j < D; ++j) cds[j] = (uint8_t)codebook_code(w[j], codebook, bits);
+          if (pre) memcpy(pre + v * D, w, sizeof(float) * D);
+          orc_pack(cds, D, bits, codes + v * rb);
+          norm[v] = rho;
+          continue;
+        }
 
         if (rot == ORC_ROT_ISO) {
           /* [IsoQuant §3.1]: rho = ||x||, x_hat = x / (rho + eps); 4-D blocks
@@ -477,7 +582,7 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
           for (int hl = 0; hl < hg; ++hl) {
             float* ph = buf + hl * D;
             if (rope) {
-              orc_rope_apply_f32(tmp, ph, c, sn, D);
+              orc_rope_apply_f32_mode(tmp, ph, c, sn, D, rope);
               memcpy(ph, tmp, sizeof(float) * D);
             }
             size_t v = ((size_t)(b * H + h0 + hl) * T + t);
@@ -495,7 +600,7 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
           for (int j = 0; j < D; ++j) tmp[j] = orc_half_to_float(xv[j]);
           float y[256];
           if (rope)
-            orc_rope_apply_f32(y, tmp, c, sn, D);
+            orc_rope_apply_f32_mode(y, tmp, c, sn, D, rope);
           else
             memcpy(y, tmp, sizeof(float) * D);
           for (int j = 0; j < D; ++j) buf[j] = y[perm ? perm[h0 * D + j] : j];
@@ -562,6 +667,16 @@ static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* co
             else
               memcpy(out + v * D, y, sizeof(double) * D);
           }
+          continue;
+        }
+        if (s->rot == ORC_ROT_ISO3) {
+          size_t v = ((size_t)(b * H + h0) * T + t);
+          uint8_t cds[256];
+          orc_unpack(codes + v * rb, D, s->bits, cds);
+          double w[256], u[256];
+          for (int j = 0; j < D; ++j) w[j] = codebook[cds[j]];
+          iso3_unrotate_f64(w, qL, D, u);
+          for (int j = 0; j < D; ++j) out[v * D + j] = u[j] * (double)norm[v];
           continue;
         }
         if (s->rot == ORC_ROT_ISO) {
@@ -766,7 +881,7 @@ int orc_calibrate_perm(int B, int H, int T, int D, const int64_t* pos, int rope,
         for (int j = 0; j < D; ++j) xf[j] = orc_half_to_float(xv[j]);
         if (rope) {
           orc_rope_cs(pos[t], D, base, rope, c, sn);
-          orc_rope_apply_f32(y, xf, c, sn, D);
+          orc_rope_apply_f32_mode(y, xf, c, sn, D, rope);
         } else {
           memcpy(y, xf, sizeof(float) * D);
         }

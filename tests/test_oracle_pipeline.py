@@ -181,6 +181,33 @@ def test_score_matches_decode(orc):
     assert math.isclose(s5[1, 3, 3], orc.rope_f64(xr[1, 1, 7], 7)[5], rel_tol=1e-12, abs_tol=1e-12)
 
 
+def test_score_grouped_cache_matches_decode(orc):
+    """Grouped-head cache ([RotateKV] pre-RoPE grouped-head rotation): the score
+    of query head qh at slot n is scale * q . RoPE_n(k), k = head qh // (Hq/H)
+    of the group decode (inverse RoPE, FWHT over the group, the head's slice);
+    sinks give RoPE_n(sink)."""
+    B, H, Hq, T, D, hg = 1, 4, 8, 10, 128, 4
+    n_sink = 2
+    x = _kv(23, B, H, T, D)
+    kw = dict(rot=orc.ROT_FWHT_GROUP, bits=2, group=128, group_heads=hg, rope=1, n_sink=n_sink)
+    pos = np.arange(T)
+    pk = orc.encode(x.view(np.uint16), pos, **kw)
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    scale = 1 / math.sqrt(D)
+    tok = np.array([0, 1, 2, 5, 9])
+    s = orc.score(q.view(np.uint16), pk, tok, H=H, t_cap=T, scale=scale, **kw)
+    xr = orc.decode(pk, pos, x.shape, **kw)
+    for qh in range(Hq):
+        h = qh // (Hq // H)
+        for i, n in enumerate(tok):
+            k = orc.rope_f64(xr[0, h, n], n)
+            assert math.isclose(s[0, qh, i], scale * (q[0, qh].astype(np.float64) @ k), rel_tol=1e-9,
+                                abs_tol=1e-9)
+    # the sink slots return the stored fp16 key itself
+    assert np.array_equal(xr[0, :, :n_sink], x[0, :, :n_sink].astype(np.float64))
+
+
 def test_calibrate_perm(orc):
     B, H, T, D = 2, 3, 17, 128
     x = _kv(31, B, H, T, D)

@@ -100,15 +100,18 @@ def test_full_llama2_7b_mha(K, orc, which):
     assert np.all(err <= recon_tolerance(dec)), err.max()
 
 
-def test_full_isoquant_batch(K, orc):
+@pytest.mark.parametrize("name", ["isoquant_batch", "isoquant_so3_batch"])
+def test_full_isoquant_batch(K, orc, name):
     from kv_cache_rotation_b200 import torch_api as TA
-    w = W.WORKLOADS["isoquant_batch"]
+    w = W.WORKLOADS[name]
+    so3 = w.rot == "iso3"
     xg = W.kv_tensor_device(w, "k", "cuda")
-    qL, qR = W.iso_tables(w)
-    d = TA.make_desc(batch=w.B, heads=w.H, head_dim=w.D, tokens=w.T, bits=w.bits, rope=0, rot="iso",
+    qL, qR = (W.iso3_tables(w.D, w.seed), None) if so3 else W.iso_tables(w)
+    d = TA.make_desc(batch=w.B, heads=w.H, head_dim=w.D, tokens=w.T, bits=w.bits, rope=0, rot=w.rot,
                      quant="codebook")
     cb = TA.lloyd_max_codebook(w.bits, w.D)
-    tb = TA.make_tables(qL=torch.from_numpy(qL).cuda(), qR=torch.from_numpy(qR).cuda(), codebook=cb)
+    tb = TA.make_tables(qL=torch.from_numpy(qL).cuda(), qR=torch.from_numpy(qR).cuda() if qR is not None else None,
+                        codebook=cb)
     pk = TA.alloc_packed(d)
     TA.encode(d, xg, tb, pk)
     out = torch.empty_like(xg)
@@ -119,7 +122,7 @@ def test_full_isoquant_batch(K, orc):
     tok = _sample(w.T, 16, 9, always=(0, w.T - 1))
     x = xg[bs][:, :, tok].cpu().numpy()  # [48, 1, n, 128]
     ocb = orc.codebook(w.bits, w.D)
-    okw = dict(rot=orc.ROT_ISO, quant=orc.Q_CODEBOOK, bits=w.bits, qL=qL, qR=qR, cb=ocb)
+    okw = dict(rot=orc.ROT_ISO3 if so3 else orc.ROT_ISO, quant=orc.Q_CODEBOOK, bits=w.bits, qL=qL, qR=qR, cb=ocb)
     ref = orc.encode(x.view(np.uint16), tok, want_pre=True, **okw)
     gc = pk.codes[bs][:, :, tok].cpu().numpy()
     rep = compare_codebook(gc, ref["codes"], ref["pre"], ocb, w.D, w.bits)

@@ -27,7 +27,7 @@ def build_cache(K, w, x, x_app, perm, rot="fwht_head"):
     B, H, T, D = x.shape
     t_cap = T + x_app.shape[2]
     kw = dict(batch=B, heads=H, head_dim=D, t_cap=t_cap, bits=w.bits, group=w.group, rope=1, n_sink=w.n_sink,
-              rot=rot)
+              rot=rot, group_heads=w.group_heads)
     tb = TA.make_tables(perm=torch.from_numpy(perm).cuda() if perm is not None else None,
                         rope_cs=TA.rope_table(t_cap, D))
     d_pre = TA.make_desc(tokens=T, t0=0, **kw)
@@ -53,8 +53,8 @@ def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None):
     tok = np.arange(n_tok) if tokens is None else np.asarray(tokens)
     cache = {"codes": pk.codes.cpu().numpy(), "sz": pk.scale_zero.cpu().numpy().view(np.uint16),
              "sink": pk.sink.cpu().numpy().view(np.uint16) if w.n_sink else None}
-    okw = dict(rot={"none": 0, "fwht_head": 1}[rot], bits=w.bits, group=w.group, rope=1, n_sink=w.n_sink,
-               perm=perm)
+    okw = dict(rot={"none": 0, "fwht_head": 1, "fwht_group": 2}[rot], bits=w.bits, group=w.group,
+               group_heads=w.group_heads, rope=1, n_sink=w.n_sink, perm=perm)
     ref = orc.score(q.view(np.uint16), cache, tok, H=w.H, t_cap=n_tok, scale=scale, **okw)
     # attention-space keys (fp64) for the L1 bound
     khat = orc.decode(cache, np.arange(n_tok), (w.B, w.H, n_tok, w.D), **okw)
@@ -97,3 +97,13 @@ def test_score_no_rotation(K, orc):
 def test_score_d64(K, orc):
     w = W.scaled(W.WORKLOADS["decode_score"], B=2, H=2, Hq=2, T=64, D=64, group=32)
     run_score_case(K, orc, w, W.random_perm(2, 64, 5))
+
+
+@pytest.mark.parametrize("hg,gq,bits,group,n_sink,T", [(8, 4, 2, 128, 0, 300), (8, 1, 4, 128, 2, 97),
+                                                       (4, 2, 2, 128, 3, 150), (8, 8, 2, 64, 0, 61)])
+def test_score_grouped_cache(K, orc, hg, gq, bits, group, n_sink, T):
+    """A grouped-head cache (FWHT over hg heads x 128 before RoPE): every slot is
+    decoded, turned by RoPE_n and dotted with the query heads of its KV head."""
+    w = W.Workload("score_group", B=2, H=hg, T=T, rot="fwht_group", group_heads=hg, bits=bits, group=group,
+                   n_sink=n_sink, Hq=hg * gq, append=1, seed=70 + hg + gq)
+    run_score_case(K, orc, w, None, rot="fwht_group")

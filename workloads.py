@@ -69,6 +69,10 @@ WORKLOADS = {
     # 3-bit Lloyd-Max codebook for N(0, 1/128).
     "isoquant_batch": Workload("isoquant_batch", B=8192, H=1, T=2048, rot="iso", quant="codebook", bits=3,
                                rope_k=False, dist="student_t", seed=4),
+    # The same batch through the 3-D sandwich q v q* (3-channel blocks, a
+    # 2-channel tail turned in its plane).
+    "isoquant_so3_batch": Workload("isoquant_so3_batch", B=8192, H=1, T=2048, rot="iso3", quant="codebook",
+                                   bits=3, rope_k=False, dist="student_t", seed=4),
     # Decode step: batch 64, 32 heads, 8192-token 2-bit cache encoded as in
     # the Llama-2-7B workload, plus one appended token; fp32 scores.
     "decode_score": Workload("decode_score", B=64, H=32, T=8192, bits=2, group=64, n_sink=4, perm=True,
@@ -166,6 +170,20 @@ def unit_quaternions(n: int, seed: int, stream: int) -> np.ndarray:
 def iso_tables(w: Workload):
     """(qL, qR) for the IsoQuant rotation: one unit quaternion pair per 4-D block."""
     return unit_quaternions(w.D // 4, w.seed, 30), unit_quaternions(w.D // 4, w.seed, 31)
+
+
+def iso3_tables(D: int, seed: int) -> np.ndarray:
+    """[ceil(D/3)][4] float32 unit quaternions (real, i, j, k) for the 3-D
+    sandwich: one per 3-channel block, drawn like unit_quaternions; when D mod
+    3 = 2 the last entry, for the 2-channel tail, has zero i and j parts
+    (real and k drawn N(0,1), normalised in float64)."""
+    nb = D // 3
+    n = nb + (1 if D % 3 else 0)
+    g = _rng(seed, 32).standard_normal((n, 4))
+    if D % 3 == 2:
+        g[nb, 1:3] = 0.0
+    g /= np.linalg.norm(g, axis=1, keepdims=True)
+    return g.astype(np.float32)
 
 
 def random_perm(H: int, D: int, seed: int) -> np.ndarray:
