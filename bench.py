@@ -321,6 +321,40 @@ class PairEnergyStep:
         return [self.call]
 
 
+class SinkDetectStep:
+    """Attention-sink detection over the Llama-2-7B-shaped key prefill (8 x 32
+    heads x 4096 tokens x 128, with massive activations planted on 4 tokens
+    per sequence): per-token maxima over all heads and channels, then the
+    median, threshold tau = 8 and a list of at most 8 sinks per sequence."""
+
+    workload = "llama2_7b_sink_detect"
+    kernels_per_step = 2  # per-token maxima, then one selection CTA per sequence
+
+    def __init__(self, device):
+        import torch
+        from kv_cache_rotation_b200 import torch_api as TA
+        w = W.WORKLOADS["llama2_7b_mha"]
+        x = W.kv_tensor(w, "k")
+        W.plant_massive(x, 4, 11)
+        self.x = torch.from_numpy(x).to(device)
+        self.d = TA.make_desc(batch=w.B, heads=w.H, head_dim=w.D, tokens=w.T, bits=w.bits, group=w.group)
+        self.sp = torch.empty((w.B, 8), dtype=torch.int32, device=device)
+        self.cnt = torch.empty((w.B,), dtype=torch.int32, device=device)
+        self.ws = TA.detect_sinks_workspace(self.d, device)
+        self.call = TA.bind_detect_sinks(self.d, self.x, 8.0, self.sp, self.cnt, self.ws)
+        nbytes = self.x.numel() * 2
+        # x once, the per-token keys written and read back, the lists and counts
+        self.alg = {"detect": nbytes + 2 * (w.B * w.T * 2) + self.sp.numel() * 4 + w.B * 4}
+        self.fp16_equiv = {"detect": nbytes}
+        self.kernels = {"detect": "k_token_absmax"}
+        self.fp32_ops = {}
+        self.names = list(self.alg)
+        torch.cuda.synchronize(device)
+
+    def launches(self):
+        return [self.call]
+
+
 class GroupScoreStep:
     """Decode-step scores over the headline layer's own grouped-head key cache
     (4 x 8 KV heads x 32768 slots, FWHT over the 8 heads before RoPE, 2-bit
@@ -459,6 +493,8 @@ def make_step(workload, device, batch=None):
         return PairEnergyStep(device)
     if workload == "llama3_8b_gqa_group_score":
         return GroupScoreStep(device)
+    if workload == "llama2_7b_sink_detect":
+        return SinkDetectStep(device)
     return EncDecStep(workload, device, batch=batch)
 
 
@@ -803,7 +839,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--workload", default="llama3_8b_gqa",
                     choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "isoquant_so3_batch", "decode_score",
-                             "llama3_8b_gqa_group_score",
+                             "llama3_8b_gqa_group_score", "llama2_7b_sink_detect",
                              "llama3_8b_gqa_attend", "llama3_8b_calibrate", "llama3_8b_pair_energy", "tiny"],
                     help="which workload a step runs (the headline line is llama3_8b_gqa)")
     ap.add_argument("--batch", type=int, default=None,

@@ -86,7 +86,8 @@ typedef struct {
                           rotation matrix ([EliteKV §2.1]); 2: RoPE on the half-split pairs
                           (i, i + head_dim/2) of the page's apply_rope code ([EliteKV §7.1]);
                           pair i turns by m*theta_i either way, from the same table */
-  int32_t n_sink;      /* positions 0..n_sink-1 are attention sinks kept verbatim in fp16 */
+  int32_t n_sink;      /* attention sinks kept verbatim in fp16: positions 0..n_sink-1, or the
+                          n_sink entries of kvq_tables.sink_pos when that is given */
   int32_t rot;         /* KVQ_ROT_* */
   int32_t quant;       /* KVQ_Q_* */
 } kvq_desc;
@@ -95,7 +96,8 @@ typedef struct {
  *   codes       u8   [B][H][t_cap][head_dim*bits/8]  code j of a record occupies bits
  *                     [bits*j, bits*j+bits) of its little-endian byte stream (LSB first)
  *   scale_zero  half [B][H][t_cap][head_dim/group][2]  (scale S, zero Z); min-max only
- *   sink        half [B][H][n_sink][head_dim]          the first n_sink positions, verbatim
+ *   sink        half [B][H][n_sink][head_dim]          the sink positions, verbatim (row k: position
+ *                                                     k, or the list's entry k)
  *   norm        f32  [B][H][t_cap]                      rho; ISO_SO4 and ISO_SO3 only
  * Slots of sink positions hold zero codes, zero scale/zero and zero norm.
  * Alignment: codes, scale_zero and sink 16 bytes; norm 4 bytes. Unused fields may be NULL. */
@@ -111,12 +113,20 @@ typedef struct {
  *             p_j = y_perm[h][j] ([RotateKV] channel reordering); must be a permutation
  *   rope_cs   f32 [rope_rows][head_dim/2][2] = (cos, sin) of position m times
  *             theta_i = 10000^(-2i/head_dim) ([EliteKV §2.1]); fill it with kvq_rope_table.
- *             16-byte aligned. Required when rope = 1 (and by kvq_score when n_sink > 0).
+ *             16-byte aligned. Required when rope != 0.
  *   qL, qR    f32 [head_dim/4][4] unit quaternions (real, i, j, k), one pair per 4-D block
  *             (ISO_SO4). ISO_SO3 reads qL only: f32 [ceil(head_dim/3)][4], one unit quaternion
  *             per 3-channel block and, when head_dim mod 3 = 2, one for the 2-channel tail whose
  *             i and j parts must be zero (otherwise the tail's output is not a rotation)
- *   codebook  f32 [1 << bits] ascending levels (kvq_lloyd_max_codebook) */
+ *   codebook  f32 [1 << bits] ascending levels (kvq_lloyd_max_codebook)
+ *   sink_pos  int32 [B][n_sink] or NULL (the sinks are positions 0..n_sink-1): the list form
+ *             of the sink set ([RotateKV] attention sinks found from the activations, e.g. by
+ *             kvq_detect_sinks). Entry k of sequence b is the position (cache slot) whose fp16
+ *             row is sink row k, or -1 for an unused entry; entries must be distinct. 4-byte
+ *             aligned. Read by kvq_encode, kvq_decode, kvq_score and kvq_calibrate_perm;
+ *             kvq_attend returns KVQ_ERR_UNSUPPORTED for it. With a list, encode, decode and
+ *             score run their kernels on every slot and one more small kernel then writes the
+ *             sink entries; kvq_score then needs rope_rows >= n_tokens when rope != 0. */
 typedef struct {
   const int16_t* perm;
   const float* rope_cs;
@@ -124,6 +134,7 @@ typedef struct {
   const float* qL;
   const float* qR;
   const float* codebook;
+  const int32_t* sink_pos;
 } kvq_tables;
 
 /* Encode T tokens into cache slots t0..t0+T-1.
@@ -133,7 +144,8 @@ typedef struct {
  * `group` consecutive rotated channels, Z = largest fp16 <= min, S = smallest fp16 >=
  * fp32((max - Z)/(2^bits - 1)), code = round-half-even(fp32(p - Z) * fp32(1/S)), so codes lie
  * in [0, 2^bits - 1]. Codebook: code = number of fp32 midpoints 0.5*(l_k + l_{k+1}) below w.
- * Sink positions (< n_sink) are copied to `sink` verbatim ([RotateKV] attention sinks). */
+ * Sink positions (< n_sink, or those listed in tb->sink_pos) are copied to `sink` verbatim
+ * ([RotateKV] attention sinks). */
 kvq_status kvq_encode(const kvq_desc* d, const void* x, const kvq_tables* tb, const kvq_packed* out,
                       kvq_stream_t stream);
 
@@ -149,9 +161,12 @@ kvq_status kvq_decode(const kvq_desc* d, const kvq_packed* in, const kvq_tables*
  *   scores[b][qh][n] = scale * <q[b][qh], khat[b][qh / (q_heads/H)][n]>,  n in [0, n_tokens)
  * q: half [B][q_heads][head_dim] in attention space (RoPE'd at the query position); q_heads a
  * multiple of H (grouped-query attention). khat_n is the key in attention space: RoPE_n(sink_n)
- * for n < n_sink, else slot n decoded without the inverse RoPE. Supported for rot in
+ * for a sink position n, else slot n decoded without the inverse RoPE. Supported for rot in
  * {NONE, FWHT_HEAD} with min-max codes; the kernel rotates the query once instead of every key
- * (q . P^T H y = (H P q) . y for the orthonormal H and permutation P).
+ * (q . P^T H y = (H P q) . y for the orthonormal H and permutation P). Also for FWHT_GROUP
+ * (the grouped-head rotation) with rope != 0, no permutation, q_heads/H in {1, 2, 4, 8} and
+ * rope_rows >= n_tokens: RoPE comes after the rotation there, so each key is decoded (inverse
+ * FWHT over its head group) and turned to its position before the dot product.
  * scores: f32 [B][q_heads][n_tokens]; n_tokens <= t_cap. d->tokens and d->t0 are ignored. */
 kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kvq_packed* cache,
                      const kvq_tables* tb, int32_t n_tokens, float scale, float* scores,
@@ -209,7 +224,7 @@ size_t kvq_attend_workspace_bytes(const kvq_desc* dk, const kvq_desc* dv, int32_
 
 /* Channel permutation by abs-max ([RotateKV] outlier-aware rotation: channel reordering before
  * the FWHT). For each head h, a_j = max over the B batches and the positions t0..t0+T-1 that are
- * not sinks (position >= n_sink) of |y_j|, where y is the fp32 input of the permutation step:
+ * not sinks (position >= n_sink, or not in tb->sink_pos) of |y_j|, where y is the fp32 input of the permutation step:
  * RoPE_m(x), with kvq_encode's fp32 arithmetic, for rope = 1 and rot NONE or FWHT_HEAD (RoPE comes
  * before the permutation there); x itself otherwise (values; FWHT_GROUP permutes the raw input).
  * perm_out[h] lists the channels by descending a_j, equal a_j in ascending channel order: a table
@@ -227,6 +242,30 @@ kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables
 
 /* Workspace bytes kvq_calibrate_perm needs for d; 0 if d is invalid or unsupported. */
 size_t kvq_calibrate_workspace_bytes(const kvq_desc* d);
+
+/* Attention sinks by massive activations ([RotateKV] abstract (iii) and 关键设计: the sink
+ * tokens carry activations far above the rest and are found from them). Per sequence b of the
+ * T tokens x[b][:, t] at positions t0 + t:
+ *   a_t  = max over heads and channels of |x[b][h][t][j]| (exact: fp16 magnitudes),
+ *   med  = the lower median of a_0 .. a_{T-1} (ascending rank floor((T-1)/2)),
+ *   sinks: the tokens with a_t > tau * med, the product and the comparison in fp64; at most
+ *          max_sinks of them, the largest a_t first, equal a_t to the earlier token.
+ *   x          half [B][H][T][head_dim], 16-byte aligned (only batch, heads, head_dim, tokens, t0
+ *              of d are used, but d must be valid as a whole)
+ *   sink_pos   int32 [B][max_sinks], overwritten: the sinks' positions ascending, then -1; it is
+ *              kvq_tables.sink_pos for a descriptor with n_sink = max_sinks
+ *   count      int32 [B] or NULL: how many sinks each sequence has
+ *   workspace  device memory of at least kvq_detect_sinks_workspace_bytes(d) bytes, 16-byte
+ *              aligned, caller-owned, contents irrelevant
+ * tau must be finite, max_sinks in 1..65536, tokens > 0 (else KVQ_ERR_INVALID). Two kernels run
+ * on `stream`: one pass over x (the per-token maxima), then one CTA per sequence. NaN inputs
+ * give an unspecified list. */
+kvq_status kvq_detect_sinks(const kvq_desc* d, const void* x, double tau, int32_t max_sinks, int32_t* sink_pos,
+                            int32_t* count, void* workspace, size_t workspace_bytes, kvq_stream_t stream);
+
+/* Workspace bytes kvq_detect_sinks needs for d (2 bytes per token, rounded up to 16); 0 if d is
+ * invalid. */
+size_t kvq_detect_sinks_workspace_bytes(const kvq_desc* d);
 
 /* Energy of each RoPE frequency pair ([EliteKV] §3.1, frequency energy analysis): per head h,
  *   E[h][i] = sum over the B batches and the T tokens of x[..][2i]^2 + x[..][2i+1]^2,

@@ -24,6 +24,7 @@ KVQ_FIELD_CODES, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_FIELD_NORM = range(4)
 
 EXPORTED = ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_attend_workspace_bytes",
             "kvq_calibrate_perm", "kvq_calibrate_workspace_bytes", "kvq_pair_energy",
+            "kvq_detect_sinks", "kvq_detect_sinks_workspace_bytes",
             "kvq_packed_bytes", "kvq_rope_table", "kvq_rope_table_ex", "kvq_lloyd_max_codebook", "kvq_check", "kvq_debug_expire_wait",
             "kvq_status_str", "kvq_version")
 
@@ -41,7 +42,8 @@ class kvq_packed(ctypes.Structure):
 
 class kvq_tables(ctypes.Structure):
     _fields_ = [("perm", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p), ("rope_rows", ctypes.c_int32),
-                ("qL", ctypes.c_void_p), ("qR", ctypes.c_void_p), ("codebook", ctypes.c_void_p)]
+                ("qL", ctypes.c_void_p), ("qR", ctypes.c_void_p), ("codebook", ctypes.c_void_p),
+                ("sink_pos", ctypes.c_void_p)]
 
 
 class KvqError(RuntimeError):
@@ -66,6 +68,9 @@ def _load():
                                      P(kvq_packed), P(kvq_tables), i32, ctypes.c_float, vp, st]
     L.kvq_calibrate_perm.argtypes = [P(kvq_desc), vp, P(kvq_tables), vp, vp, ctypes.c_size_t, st]
     L.kvq_pair_energy.argtypes = [P(kvq_desc), vp, vp, vp, st]
+    L.kvq_detect_sinks.argtypes = [P(kvq_desc), vp, ctypes.c_double, i32, vp, vp, vp, ctypes.c_size_t, st]
+    L.kvq_detect_sinks_workspace_bytes.argtypes = [P(kvq_desc)]
+    L.kvq_detect_sinks_workspace_bytes.restype = ctypes.c_size_t
     L.kvq_calibrate_workspace_bytes.argtypes = [P(kvq_desc)]
     L.kvq_calibrate_workspace_bytes.restype = ctypes.c_size_t
     L.kvq_attend_workspace_bytes.argtypes = [P(kvq_desc), P(kvq_desc), i32, i32]
@@ -81,7 +86,7 @@ def _load():
     L.kvq_status_str.restype = ctypes.c_char_p
     L.kvq_version.restype = i32
     for n in ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_calibrate_perm",
-              "kvq_pair_energy",
+              "kvq_pair_energy", "kvq_detect_sinks",
               "kvq_rope_table", "kvq_rope_table_ex",
               "kvq_lloyd_max_codebook",
               "kvq_check", "kvq_debug_expire_wait"):
@@ -132,6 +137,16 @@ def kvq_calibrate_perm(d: kvq_desc, x: int, tb: kvq_tables, perm_out: int, works
 
 def kvq_pair_energy(d: kvq_desc, x: int, energy_out: int, rank_out: int, stream: int = 0) -> int:
     return lib.kvq_pair_energy(ctypes.byref(d), x, energy_out, rank_out, stream)
+
+
+def kvq_detect_sinks(d: kvq_desc, x: int, tau: float, max_sinks: int, sink_pos: int, count: int, workspace: int,
+                     workspace_bytes: int, stream: int = 0) -> int:
+    return lib.kvq_detect_sinks(ctypes.byref(d), x, tau, max_sinks, sink_pos, count, workspace, workspace_bytes,
+                                stream)
+
+
+def kvq_detect_sinks_workspace_bytes(d: kvq_desc) -> int:
+    return lib.kvq_detect_sinks_workspace_bytes(ctypes.byref(d))
 
 
 def kvq_calibrate_workspace_bytes(d: kvq_desc) -> int:

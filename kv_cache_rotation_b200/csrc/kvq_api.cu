@@ -110,6 +110,7 @@ kvq_status check_tables(const kvq_desc* d, const kvq_tables* tb, int64_t rope_ro
     if (tb->rope_rows < rope_rows_needed || tb->rope_rows <= 0) return KVQ_ERR_INVALID;
   }
   if (tb->perm && !aligned(tb->perm, 16)) return KVQ_ERR_ALIGN;
+  if (tb->sink_pos && !aligned(tb->sink_pos, 4)) return KVQ_ERR_ALIGN;
   if (d->rot == KVQ_ROT_ISO_SO4) {
     if (!tb->qL || !tb->qR || !tb->codebook) return KVQ_ERR_INVALID;
     if (!aligned(tb->qL, 16) || !aligned(tb->qR, 16) || !aligned(tb->codebook, 4)) return KVQ_ERR_ALIGN;
@@ -204,15 +205,22 @@ kvq_status kvq_encode(const kvq_desc* d, const void* x, const kvq_tables* tb, co
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  switch (d->rot) {
+  const bool listed = tb->sink_pos && d->n_sink > 0;
+  kvq_desc dd = *d;
+  if (listed) dd.n_sink = 0;  // every slot is coded first; the listed sinks are written after
+  switch (dd.rot) {
     case KVQ_ROT_FWHT_GROUP:
-      return launch_encode_group(*d, x, *tb, *out, st, ctx);
+      s = launch_encode_group(dd, x, *tb, *out, st, ctx);
+      break;
     case KVQ_ROT_ISO_SO4:
     case KVQ_ROT_ISO_SO3:
-      return launch_encode_iso(*d, x, *tb, *out, st, ctx);
+      s = launch_encode_iso(dd, x, *tb, *out, st, ctx);
+      break;
     default:
-      return launch_encode_head(*d, x, *tb, *out, st, ctx);
+      s = launch_encode_head(dd, x, *tb, *out, st, ctx);
   }
+  if (s != KVQ_OK || !listed) return s;
+  return launch_sink_fix_encode(*d, x, *tb, *out, st);
 }
 
 kvq_status kvq_decode(const kvq_desc* d, const kvq_packed* in, const kvq_tables* tb, void* x_out,
@@ -228,15 +236,22 @@ kvq_status kvq_decode(const kvq_desc* d, const kvq_packed* in, const kvq_tables*
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  switch (d->rot) {
+  const bool listed = tb->sink_pos && d->n_sink > 0;
+  kvq_desc dd = *d;
+  if (listed) dd.n_sink = 0;  // every slot is decoded first; the listed sinks are written after
+  switch (dd.rot) {
     case KVQ_ROT_FWHT_GROUP:
-      return launch_decode_group(*d, *in, *tb, x_out, out_fp32, st, ctx);
+      s = launch_decode_group(dd, *in, *tb, x_out, out_fp32, st, ctx);
+      break;
     case KVQ_ROT_ISO_SO4:
     case KVQ_ROT_ISO_SO3:
-      return launch_decode_iso(*d, *in, *tb, x_out, out_fp32, st, ctx);
+      s = launch_decode_iso(dd, *in, *tb, x_out, out_fp32, st, ctx);
+      break;
     default:
-      return launch_decode_head(*d, *in, *tb, x_out, out_fp32, st, ctx);
+      s = launch_decode_head(dd, *in, *tb, x_out, out_fp32, st, ctx);
   }
+  if (s != KVQ_OK || !listed) return s;
+  return launch_sink_fix_decode(*d, *in, *tb, x_out, out_fp32, st);
 }
 
 kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kvq_packed* cache,
@@ -258,17 +273,21 @@ kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kv
     const int gq = q_heads / dd.heads;
     if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KVQ_ERR_UNSUPPORTED;
   }
-  const int64_t rows = grouped ? n_tokens : (dd.rope ? (n_tokens < dd.n_sink ? n_tokens : dd.n_sink) : 0);
+  const bool listed = tb && tb->sink_pos && dd.n_sink > 0;
+  const int64_t rows = grouped || listed ? n_tokens
+                                         : (dd.rope ? (n_tokens < dd.n_sink ? n_tokens : dd.n_sink) : 0);
   if ((s = check_tables(&dd, tb, rows)) != KVQ_OK) return s;
   if ((s = check_packed(&dd, cache)) != KVQ_OK) return s;
   if (n_tokens == 0) return KVQ_OK;
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
-  if (grouped)
-    return launch_score_group(dd, q, q_heads, *cache, *tb, n_tokens, scale, scores,
-                              reinterpret_cast<cudaStream_t>(stream), ctx);
-  return launch_score(dd, q, q_heads, *cache, *tb, n_tokens, scale, scores, reinterpret_cast<cudaStream_t>(stream),
-                      ctx);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  kvq_desc dm = dd;
+  if (listed) dm.n_sink = 0;  // every slot is scored from its codes first; the listed sinks after
+  s = grouped ? launch_score_group(dm, q, q_heads, *cache, *tb, n_tokens, scale, scores, st, ctx)
+              : launch_score(dm, q, q_heads, *cache, *tb, n_tokens, scale, scores, st, ctx);
+  if (s != KVQ_OK || !listed) return s;
+  return launch_sink_fix_score(dd, q, q_heads, *cache, *tb, n_tokens, scale, scores, st);
 }
 
 namespace {
@@ -317,6 +336,7 @@ kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int
   if (workspace_bytes < attend_workspace_bytes(k, q_heads, n_tokens)) return KVQ_ERR_INVALID;
   if ((s = check_tables(&k, tk, k.rope ? (n_tokens < k.n_sink ? n_tokens : k.n_sink) : 0)) != KVQ_OK) return s;
   if ((s = check_tables(&v, tv, 0)) != KVQ_OK) return s;
+  if (tk->sink_pos || tv->sink_pos) return KVQ_ERR_UNSUPPORTED;  // sinks as a prefix only
   if ((s = check_packed(&k, k_cache)) != KVQ_OK || (s = check_packed(&v, v_cache)) != KVQ_OK) return s;
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
@@ -336,6 +356,7 @@ kvq_status kvq_attend_noalloc(const kvq_desc* dk, const kvq_desc* dv, const void
   if (attend_workspace_bytes(k, q_heads, n_tokens) > attend_scratch_bytes()) return KVQ_ERR_UNSUPPORTED;
   if ((s = check_tables(&k, tk, k.rope ? (n_tokens < k.n_sink ? n_tokens : k.n_sink) : 0)) != KVQ_OK) return s;
   if ((s = check_tables(&v, tv, 0)) != KVQ_OK) return s;
+  if (tk->sink_pos || tv->sink_pos) return KVQ_ERR_UNSUPPORTED;  // sinks as a prefix only
   if ((s = check_packed(&k, k_cache)) != KVQ_OK || (s = check_packed(&v, v_cache)) != KVQ_OK) return s;
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
@@ -376,10 +397,32 @@ kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables
     if (!aligned(tb->rope_cs, 16)) return KVQ_ERR_ALIGN;
     if (tb->rope_rows < static_cast<int64_t>(d->t0) + d->tokens || tb->rope_rows <= 0) return KVQ_ERR_INVALID;
   }
+  if (tb->sink_pos && !aligned(tb->sink_pos, 4)) return KVQ_ERR_ALIGN;
   if (static_cast<int64_t>(d->batch) * d->tokens >= (int64_t(1) << 31)) return KVQ_ERR_UNSUPPORTED;
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
   return launch_calibrate(*d, x, *tb, perm_out, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t kvq_detect_sinks_workspace_bytes(const kvq_desc* d) {
+  if (check_desc(d) != KVQ_OK) return 0;
+  return detect_sinks_workspace_bytes(*d);
+}
+
+kvq_status kvq_detect_sinks(const kvq_desc* d, const void* x, double tau, int32_t max_sinks, int32_t* sink_pos,
+                            int32_t* count, void* workspace, size_t workspace_bytes, kvq_stream_t stream) {
+  kvq_status s = check_desc(d);
+  if (s != KVQ_OK) return s;
+  if (!x || !sink_pos || !workspace || d->tokens <= 0) return KVQ_ERR_INVALID;
+  if (!isfinite(tau) || max_sinks < 1 || max_sinks > 65536) return KVQ_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(workspace, 16) || !aligned(sink_pos, 4) || (count && !aligned(count, 4)))
+    return KVQ_ERR_ALIGN;
+  if (workspace_bytes < detect_sinks_workspace_bytes(*d)) return KVQ_ERR_INVALID;
+  if (d->batch > 65535) return KVQ_ERR_UNSUPPORTED;  // one CTA per sequence on a grid axis
+  LaunchCtx ctx;
+  if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
+  return launch_detect_sinks(*d, x, tau, max_sinks, sink_pos, count, workspace,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t kvq_packed_bytes(const kvq_desc* d, int32_t field) {

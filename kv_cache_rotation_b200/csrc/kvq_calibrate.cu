@@ -28,12 +28,20 @@ constexpr int kMinRows = 256;  // token rows per chunk, at least
 
 struct CalArgs {
   int H, T, t0, n_sink, rope, rows, rows_per_chunk;
+  const int32_t* sink_pos;  // [B][n_sink] listed sink positions, or nullptr: positions < n_sink
   FastDiv div_t;
   const __half* x;
   const float* rope_cs;
   uint32_t* amax;  // [H][D]: fp32 bit patterns of the running maxima (zeroed before k_absmax)
   int16_t* perm;
 };
+
+__device__ __forceinline__ bool is_sink(const CalArgs& a, int b, int pos) {
+  if (!a.sink_pos) return pos < a.n_sink;
+  bool hit = false;
+  for (int k = 0; k < a.n_sink; ++k) hit |= __ldg(a.sink_pos + static_cast<size_t>(b) * a.n_sink + k) == pos;
+  return hit;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
@@ -63,7 +71,7 @@ __global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
       const int t = min(rr, r1 - 1) - b * a.T;
       const int pos = a.t0 + t;
       posu[u] = pos;
-      live[u] = rr < r1 && pos >= a.n_sink;
+      live[u] = rr < r1 && !is_sink(a, b, pos);
       raw[u] = live[u] ? __ldg(reinterpret_cast<const uint4*>(
                              a.x + ((static_cast<size_t>(b) * a.H + h) * a.T + t) * D) + cg)
                        : make_uint4(0, 0, 0, 0);
@@ -163,6 +171,7 @@ kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& 
   a.T = d.tokens;
   a.t0 = d.t0;
   a.n_sink = d.n_sink;
+  a.sink_pos = tb.sink_pos;
   a.rope = calibrate_rope(d) ? d.rope : 0;  // 1 interleaved pairs, 2 half-split pairs
   a.rows = static_cast<int>(rows);
   const int chunks = chunks_for(rows);

@@ -55,6 +55,17 @@ size_t calibrate_workspace_bytes(const kvq_desc& d);
 kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& tb, int16_t* perm, void* ws,
                             cudaStream_t st);
 void* attend_scratch();
+size_t detect_sinks_workspace_bytes(const kvq_desc& d);
+kvq_status launch_detect_sinks(const kvq_desc& d, const void* x, double tau, int max_sinks, int32_t* sink_pos,
+                               int32_t* count, void* ws, cudaStream_t st);
+// The list form of the sink set (kvq_tables.sink_pos): run after the kernels of
+// encode / decode / score were launched with n_sink = 0.
+kvq_status launch_sink_fix_encode(const kvq_desc& d, const void* x, const kvq_tables& tb, const kvq_packed& out,
+                                  cudaStream_t st);
+kvq_status launch_sink_fix_decode(const kvq_desc& d, const kvq_packed& in, const kvq_tables& tb, void* x_out,
+                                  int out_fp32, cudaStream_t st);
+kvq_status launch_sink_fix_score(const kvq_desc& d, const void* q, int q_heads, const kvq_packed& cache,
+                                 const kvq_tables& tb, int n_tokens, float scale, float* scores, cudaStream_t st);
 kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, int q_heads,
                          const kvq_packed& kc, const kvq_tables& tk, const kvq_packed& vc, const kvq_tables& tv,
                          int n_tokens, float scale, float* out, void* ws, cudaStream_t st, const LaunchCtx& ctx);

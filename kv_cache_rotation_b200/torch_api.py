@@ -98,6 +98,7 @@ class Tables:
     qL: Optional[torch.Tensor] = None
     qR: Optional[torch.Tensor] = None
     codebook: Optional[torch.Tensor] = None
+    sink_pos: Optional[torch.Tensor] = None  # int32 [B][n_sink]: the list form of the sink set
 
     def struct(self) -> kvq_tables:
         tb = kvq_tables()
@@ -107,11 +108,14 @@ class Tables:
         tb.qL = self.qL.data_ptr() if self.qL is not None else None
         tb.qR = self.qR.data_ptr() if self.qR is not None else None
         tb.codebook = self.codebook.data_ptr() if self.codebook is not None else None
+        if self.sink_pos is not None:
+            _req(self.sink_pos, "sink_pos", (torch.int32,))
+            tb.sink_pos = self.sink_pos.data_ptr()
         return tb
 
 
-def make_tables(perm=None, rope_cs=None, qL=None, qR=None, codebook=None) -> Tables:
-    return Tables(perm, rope_cs, qL, qR, codebook)
+def make_tables(perm=None, rope_cs=None, qL=None, qR=None, codebook=None, sink_pos=None) -> Tables:
+    return Tables(perm, rope_cs, qL, qR, codebook, sink_pos)
 
 
 def _req(t: torch.Tensor, name: str, dtypes, shape=None) -> None:
@@ -217,6 +221,53 @@ def calibrate_perm(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Ten
     check(kvq_calibrate_perm(d, x.data_ptr(), tb.struct(), perm_out.data_ptr(), workspace.data_ptr(),
                              workspace.numel(), _stream(stream)), "kvq_calibrate_perm")
     return perm_out
+
+
+def detect_sinks_workspace(d: kvq_desc, device="cuda") -> torch.Tensor:
+    """A workspace tensor for kvq_detect_sinks."""
+    from . import kvq_detect_sinks_workspace_bytes
+    nb = kvq_detect_sinks_workspace_bytes(d)
+    if nb == 0:
+        raise ValueError("kvq_detect_sinks: invalid descriptor")
+    return torch.empty(nb, dtype=torch.uint8, device=device)
+
+
+def detect_sinks(d: kvq_desc, x: torch.Tensor, *, tau: float, max_sinks: int, sink_pos: torch.Tensor = None,
+                 count: torch.Tensor = None, workspace: torch.Tensor = None, stream=None):
+    """Attention sinks by massive activations: (sink_pos int32 [B][max_sinks], ascending
+    positions padded with -1, for Tables.sink_pos with n_sink = max_sinks; count int32 [B])."""
+    from . import kvq_detect_sinks
+    _req(x, "x", (torch.float16,), _kv_shape(d))
+    if sink_pos is None:
+        sink_pos = torch.empty((d.batch, max_sinks), dtype=torch.int32, device=x.device)
+    if count is None:
+        count = torch.empty((d.batch,), dtype=torch.int32, device=x.device)
+    if workspace is None:
+        workspace = detect_sinks_workspace(d, x.device)
+    _req(sink_pos, "sink_pos", (torch.int32,), (d.batch, max_sinks))
+    _req(count, "count", (torch.int32,), (d.batch,))
+    check(kvq_detect_sinks(d, x.data_ptr(), float(tau), int(max_sinks), sink_pos.data_ptr(), count.data_ptr(),
+                           workspace.data_ptr(), workspace.numel(), _stream(stream)), "kvq_detect_sinks")
+    return sink_pos, count
+
+
+def bind_detect_sinks(d: kvq_desc, x: torch.Tensor, tau: float, sink_pos: torch.Tensor, count: torch.Tensor,
+                      workspace: torch.Tensor, stream=None):
+    from . import lib
+    _req(x, "x", (torch.float16,), _kv_shape(d))
+    _req(sink_pos, "sink_pos", (torch.int32,))
+    _req(count, "count", (torch.int32,), (d.batch,))
+    if sink_pos.dim() != 2 or sink_pos.shape[0] != d.batch:
+        raise ValueError(f"sink_pos: shape {tuple(sink_pos.shape)}, expected ({d.batch}, max_sinks)")
+    st = _stream(stream)
+    args = (ctypes.byref(d), x.data_ptr(), float(tau), int(sink_pos.shape[1]), sink_pos.data_ptr(),
+            count.data_ptr(), workspace.data_ptr(), workspace.numel(), st)
+    keep = (d, x, sink_pos, count, workspace)
+
+    def call():
+        check(lib.kvq_detect_sinks(*args), "kvq_detect_sinks")
+    call.keep = keep
+    return call
 
 
 def pair_energy(d: kvq_desc, x: torch.Tensor, stream=None):

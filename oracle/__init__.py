@@ -81,19 +81,22 @@ def lib():
         L.orc_lloyd_max_normal.argtypes = [ci, f64p, f64p]
         L.orc_codebook.argtypes = [ci, ci, f32p]
         L.orc_encode.restype = ci
+        i32p = ctypes.POINTER(ctypes.c_int32)
         L.orc_encode.argtypes = [ci, ci, ci, ci, i64p, ci, ci, ci, ci, ci, ci, ci, cd,
-                                 u16p, i16p, f32p, f32p, f32p, u8p, u16p, u16p, f32p, f32p]
+                                 u16p, i16p, f32p, f32p, f32p, u8p, u16p, u16p, f32p, f32p, i32p]
         L.orc_decode.restype = ci
         L.orc_decode.argtypes = [ci, ci, ci, ci, i64p, ci, ci, ci, ci, ci, ci, ci, cd,
-                                 u8p, u16p, u16p, f32p, i16p, f32p, f32p, f32p, f64p]
+                                 u8p, u16p, u16p, f32p, i16p, f32p, f32p, f32p, f64p, i32p]
         L.orc_score.restype = ci
         L.orc_score.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, cd,
-                                u16p, u8p, u16p, u16p, f32p, i16p, f32p, f32p, f32p, i64p, ci, cd, f64p]
+                                u16p, u8p, u16p, u16p, f32p, i16p, f32p, f32p, f32p, i64p, ci, cd, f64p, i32p]
         L.orc_attend.restype = ci
         L.orc_attend.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, cd, u16p,
                                  u8p, u16p, u16p, i16p, ci, u8p, u16p, u16p, i16p, ci, cd, f64p]
         L.orc_calibrate_perm.restype = ci
-        L.orc_calibrate_perm.argtypes = [ci, ci, ci, ci, i64p, ci, ci, cd, u16p, i16p]
+        L.orc_calibrate_perm.argtypes = [ci, ci, ci, ci, i64p, ci, ci, cd, u16p, i16p, i32p]
+        L.orc_detect_sinks.restype = ci
+        L.orc_detect_sinks.argtypes = [ci, ci, ci, ci, i64p, u16p, cd, ci, i32p, i32p]
         L.orc_pair_energy.restype = ci
         L.orc_pair_energy.argtypes = [ci, ci, ci, ci, u16p, ctypes.POINTER(ctypes.c_uint64), i16p]
         _lib = L
@@ -223,11 +226,12 @@ def _packed_shapes(B, H, T, D, bits, group, n_sink):
 
 
 def encode(x, pos, *, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0, n_sink=0,
-           base=10000.0, perm=None, qL=None, qR=None, cb=None, want_pre=False):
+           base=10000.0, perm=None, qL=None, qR=None, cb=None, want_pre=False, sink_pos=None):
     """x: uint16 (fp16 bits) [B][H][T][D]; pos: int64 [T]. Returns a dict of
     codes [B][H][T][D*bits/8], sz uint16 [B][H][T][D/G][2], sink uint16
     [B][H][n_sink][D], norm f32 [B][H][T], and with want_pre the rotated
-    pre-quantization values pre f32 [B][H][T][D]."""
+    pre-quantization values pre f32 [B][H][T][D]. sink_pos: int32 [B][n_sink]
+    sink positions (-1 unused), or None for positions 0 .. n_sink-1."""
     x = np.ascontiguousarray(x, np.uint16)
     B, H, T, D = x.shape
     pos = np.ascontiguousarray(pos, np.int64)
@@ -241,18 +245,19 @@ def encode(x, pos, *, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0,
     qL_a = None if qL is None else np.ascontiguousarray(qL, np.float32)
     qR_a = None if qR is None else np.ascontiguousarray(qR, np.float32)
     cb_a = None if cb is None else np.ascontiguousarray(cb, np.float32)
+    sp_a = None if sink_pos is None else np.ascontiguousarray(sink_pos, np.int32)
     rc = lib().orc_encode(B, H, T, D, _p(pos, ctypes.c_int64), rot, quant, bits, group, group_heads,
                           rope, n_sink, base, _p(x, ctypes.c_uint16), _p(perm_a, ctypes.c_int16),
                           _p(qL_a, ctypes.c_float), _p(qR_a, ctypes.c_float), _p(cb_a, ctypes.c_float),
                           _p(codes, ctypes.c_uint8), _p(sz, ctypes.c_uint16), _p(sink, ctypes.c_uint16),
-                          _p(norm, ctypes.c_float), _p(pre, ctypes.c_float))
+                          _p(norm, ctypes.c_float), _p(pre, ctypes.c_float), _p(sp_a, ctypes.c_int32))
     if rc:
         raise ValueError("oracle encode: unsupported parameters")
     return {"codes": codes, "sz": sz, "sink": sink if n_sink > 0 else None, "norm": norm, "pre": pre}
 
 
 def decode(packed, pos, shape, *, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0,
-           n_sink=0, base=10000.0, perm=None, qL=None, qR=None, cb=None):
+           n_sink=0, base=10000.0, perm=None, qL=None, qR=None, cb=None, sink_pos=None):
     """Inverse of encode, in fp64. shape = (B, H, T, D); packed arrays are
     dense over the same T tokens. Returns float64 [B][H][T][D]."""
     B, H, T, D = shape
@@ -266,18 +271,19 @@ def decode(packed, pos, shape, *, rot, quant=Q_MINMAX, bits, group=0, group_head
     qL_a = None if qL is None else np.ascontiguousarray(qL, np.float32)
     qR_a = None if qR is None else np.ascontiguousarray(qR, np.float32)
     cb_a = None if cb is None else np.ascontiguousarray(cb, np.float32)
+    sp_a = None if sink_pos is None else np.ascontiguousarray(sink_pos, np.int32)
     rc = lib().orc_decode(B, H, T, D, _p(pos, ctypes.c_int64), rot, quant, bits, group, group_heads,
                           rope, n_sink, base, _p(codes, ctypes.c_uint8), _p(sz, ctypes.c_uint16),
                           _p(sink, ctypes.c_uint16), _p(norm, ctypes.c_float), _p(perm_a, ctypes.c_int16),
                           _p(qL_a, ctypes.c_float), _p(qR_a, ctypes.c_float), _p(cb_a, ctypes.c_float),
-                          _p(out, ctypes.c_double))
+                          _p(out, ctypes.c_double), _p(sp_a, ctypes.c_int32))
     if rc:
         raise ValueError("oracle decode: unsupported parameters")
     return out
 
 
 def score(q, cache, tokens, *, H, t_cap, rot, quant=Q_MINMAX, bits, group=0, group_heads=1, rope=0,
-          n_sink=0, base=10000.0, scale, perm=None, qL=None, qR=None, cb=None):
+          n_sink=0, base=10000.0, scale, perm=None, qL=None, qR=None, cb=None, sink_pos=None):
     """q: uint16 [B][Hq][D] (attention space); cache arrays laid out over
     t_cap slots; tokens: int64 positions to score. Returns float64
     [B][Hq][len(tokens)]."""
@@ -293,11 +299,13 @@ def score(q, cache, tokens, *, H, t_cap, rot, quant=Q_MINMAX, bits, group=0, gro
     qL_a = None if qL is None else np.ascontiguousarray(qL, np.float32)
     qR_a = None if qR is None else np.ascontiguousarray(qR, np.float32)
     cb_a = None if cb is None else np.ascontiguousarray(cb, np.float32)
+    sp_a = None if sink_pos is None else np.ascontiguousarray(sink_pos, np.int32)
     rc = lib().orc_score(B, H, Hq, D, t_cap, rot, quant, bits, group, group_heads, rope, n_sink, base,
                          _p(q, ctypes.c_uint16), _p(codes, ctypes.c_uint8), _p(sz, ctypes.c_uint16),
                          _p(sink, ctypes.c_uint16), _p(norm, ctypes.c_float), _p(perm_a, ctypes.c_int16),
                          _p(qL_a, ctypes.c_float), _p(qR_a, ctypes.c_float), _p(cb_a, ctypes.c_float),
-                         _p(tok, ctypes.c_int64), tok.size, float(scale), _p(out, ctypes.c_double))
+                         _p(tok, ctypes.c_int64), tok.size, float(scale), _p(out, ctypes.c_double),
+                         _p(sp_a, ctypes.c_int32))
     if rc:
         raise ValueError("oracle score: unsupported parameters")
     return out
@@ -331,14 +339,30 @@ def attend(q, kcache, vcache, n_tok, *, H, t_cap, rot, bits, group, n_sink=0, ba
     return out
 
 
-def calibrate_perm(x, pos, *, rope=0, n_sink=0, base=10000.0):
+def calibrate_perm(x, pos, *, rope=0, n_sink=0, base=10000.0, sink_pos=None):
     x = np.ascontiguousarray(x, np.uint16)
     B, H, T, D = x.shape
     pos = np.ascontiguousarray(pos, np.int64)
     perm = np.zeros((H, D), np.int16)
+    sp_a = None if sink_pos is None else np.ascontiguousarray(sink_pos, np.int32)
     lib().orc_calibrate_perm(B, H, T, D, _p(pos, ctypes.c_int64), rope, n_sink, base,
-                             _p(x, ctypes.c_uint16), _p(perm, ctypes.c_int16))
+                             _p(x, ctypes.c_uint16), _p(perm, ctypes.c_int16), _p(sp_a, ctypes.c_int32))
     return perm
+
+
+def detect_sinks(x, pos, *, tau, max_sinks):
+    """Sinks by massive activations (orc_detect_sinks): x uint16 [B][H][T][D];
+    returns (int32 [B][max_sinks] ascending positions padded with -1, int32 [B] counts)."""
+    x = np.ascontiguousarray(x, np.uint16)
+    B, H, T, D = x.shape
+    pos = np.ascontiguousarray(pos, np.int64)
+    sp = np.zeros((B, max_sinks), np.int32)
+    cnt = np.zeros(B, np.int32)
+    rc = lib().orc_detect_sinks(B, H, T, D, _p(pos, ctypes.c_int64), _p(x, ctypes.c_uint16), float(tau),
+                                int(max_sinks), _p(sp, ctypes.c_int32), _p(cnt, ctypes.c_int32))
+    if rc:
+        raise ValueError("oracle detect_sinks: unsupported parameters")
+    return sp, cnt
 
 
 def pair_energy(x):

@@ -390,7 +390,7 @@ static int codebook_code(float w, const float* cb, int bits) {
  *   x     half  [B][H][T][D]      pos[T] = RoPE position m of each token
  *   codes u8    [B][H][T][D*bits/8]
  *   sz    half  [B][H][T][D/G][2]  (scale, zero)
- *   sink  half  [B][H][n_sink][D]  indexed by position
+ *   sink  half  [B][H][n_sink][D]  indexed by sink slot (= position without a list)
  *   norm  f32   [B][H][T]
  * Tokens with pos < n_sink are kept verbatim in sink ([RotateKV]: attention
  * sinks protected at high precision); their codes and sz entries are zero.
@@ -400,7 +400,17 @@ static int codebook_code(float w, const float* cb, int bits) {
 typedef struct {
   int B, H, T, D, rot, quant, bits, group, group_heads, rope, n_sink;
   double base;
+  const int32_t* sink_pos; /* [B][n_sink] positions of the sinks, or NULL: positions 0 .. n_sink-1 */
 } orc_shape;
+
+/* Sink slot of position m of sequence b: its index in the sequence's sink
+ * list (the stored fp16 row), or -1 when m is not a sink. */
+static int sink_slot(const int32_t* sink_pos, int n_sink, int b, int64_t m) {
+  if (!sink_pos) return m < n_sink ? (int)m : -1;
+  for (int k = 0; k < n_sink; ++k)
+    if (sink_pos[(size_t)b * n_sink + k] == m) return k;
+  return -1;
+}
 
 static size_t rec_bytes(const orc_shape* s) { return (size_t)s->D * s->bits / 8; }
 
@@ -485,8 +495,8 @@ static void iso3_unrotate_f64(const double* w, const float* q, int D, double* v)
 int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quant, int bits, int group,
                int group_heads, int rope, int n_sink, double base, const uint16_t* x, const int16_t* perm,
                const float* qL, const float* qR, const float* codebook, uint8_t* codes, uint16_t* sz,
-               uint16_t* sink, float* norm, float* pre) {
-  orc_shape s = {B, H, T, D, rot, quant, bits, group, group_heads, rope, n_sink, base};
+               uint16_t* sink, float* norm, float* pre, const int32_t* sink_pos) {
+  orc_shape s = {B, H, T, D, rot, quant, bits, group, group_heads, rope, n_sink, base, sink_pos};
   if (check_shape(&s)) return 1;
   size_t rb = rec_bytes(&s);
   int ng = D / (group > 0 ? group : D);
@@ -498,12 +508,13 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
       for (int t = 0; t < T; ++t) {
         int64_t m = pos[t];
         if (rope) orc_rope_cs(m, D, base, rope, c, sn);
+        const int ks = sink_slot(sink_pos, n_sink, b, m);
         for (int hl = 0; hl < hg; ++hl) {
           size_t v = ((size_t)(b * H + h0 + hl) * T + t);
           const uint16_t* xv = x + v * D;
           uint8_t* rec = codes + v * rb;
-          if (m < n_sink) {
-            memcpy(sink + ((size_t)(b * H + h0 + hl) * n_sink + m) * D, xv, sizeof(uint16_t) * D);
+          if (ks >= 0) {
+            memcpy(sink + ((size_t)(b * H + h0 + hl) * n_sink + ks) * D, xv, sizeof(uint16_t) * D);
             memset(rec, 0, rb);
             if (rot == ORC_ROT_ISO || rot == ORC_ROT_ISO3)
               norm[v] = 0.0f;
@@ -511,7 +522,7 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
               memset(sz + v * ng * 2, 0, sizeof(uint16_t) * ng * 2);
           }
         }
-        if (m < n_sink) continue;
+        if (ks >= 0) continue;
 
         if (rot == ORC_ROT_ISO3) {
           /* the norm split of [IsoQuant §3.1], then the 3-D sandwich on
@@ -657,10 +668,11 @@ static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* co
     for (int h0 = 0; h0 < H; h0 += hg)
       for (int t = 0; t < T; ++t) {
         int64_t m = pos[t];
-        if (m < s->n_sink) {
+        const int ks = sink_slot(s->sink_pos, s->n_sink, b, m);
+        if (ks >= 0) {
           for (int hl = 0; hl < hg; ++hl) {
             size_t v = ((size_t)(b * H + h0 + hl) * T + t);
-            const uint16_t* sv = sink + ((size_t)(b * H + h0 + hl) * s->n_sink + m) * D;
+            const uint16_t* sv = sink + ((size_t)(b * H + h0 + hl) * s->n_sink + ks) * D;
             for (int j = 0; j < D; ++j) y[j] = orc_half_to_float(sv[j]);
             if (attn_space && s->rope)
               orc_rope_apply_f64(out + v * D, y, m, D, s->base, s->rope, 0);
@@ -742,8 +754,8 @@ static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* co
 int orc_decode(int B, int H, int T, int D, const int64_t* pos, int rot, int quant, int bits, int group,
                int group_heads, int rope, int n_sink, double base, const uint8_t* codes, const uint16_t* sz,
                const uint16_t* sink, const float* norm, const int16_t* perm, const float* qL, const float* qR,
-               const float* codebook, double* out) {
-  orc_shape s = {B, H, T, D, rot, quant, bits, group, group_heads, rope, n_sink, base};
+               const float* codebook, double* out, const int32_t* sink_pos) {
+  orc_shape s = {B, H, T, D, rot, quant, bits, group, group_heads, rope, n_sink, base, sink_pos};
   return decode_impl(&s, pos, codes, sz, sink, norm, perm, qL, qR, codebook, out, 0);
 }
 
@@ -760,9 +772,10 @@ int orc_decode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
 int orc_score(int B, int H, int Hq, int D, int t_cap, int rot, int quant, int bits, int group, int group_heads,
               int rope, int n_sink, double base, const uint16_t* q, const uint8_t* codes, const uint16_t* sz,
               const uint16_t* sink, const float* norm, const int16_t* perm, const float* qL, const float* qR,
-              const float* codebook, const int64_t* tok, int n_idx, double scale, double* out) {
+              const float* codebook, const int64_t* tok, int n_idx, double scale, double* out,
+              const int32_t* sink_pos) {
   if (Hq % H) return 1;
-  orc_shape s = {B, H, 1, D, rot, quant, bits, group, group_heads, rope, n_sink, base};
+  orc_shape s = {B, H, 1, D, rot, quant, bits, group, group_heads, rope, n_sink, base, NULL};
   if (check_shape(&s)) return 1;
   int hg = rot == ORC_ROT_FWHT_GROUP ? group_heads : 1;
   int ng = D / (group > 0 ? group : D);
@@ -778,6 +791,7 @@ int orc_score(int B, int H, int Hq, int D, int t_cap, int rot, int quant, int bi
         s1.B = 1;
         s1.H = hg;
         s1.T = 1;
+        s1.sink_pos = sink_pos ? sink_pos + (size_t)b * n_sink : NULL;  /* the one-sequence view's list */
         uint8_t* c1 = (uint8_t*)malloc(rb * hg + 1);
         uint16_t* z1 = (uint16_t*)malloc(sizeof(uint16_t) * 2 * ng * hg + 2);
         uint16_t* k1 = (uint16_t*)malloc(sizeof(uint16_t) * ((size_t)hg * (n_sink > 0 ? n_sink : 1) * D));
@@ -834,10 +848,10 @@ int orc_attend(int B, int H, int Hq, int D, int t_cap, int n_tok, int rot, int b
   double* s = (double*)malloc(sizeof(double) * (size_t)B * Hq * n_tok);
   double* vh = (double*)malloc(sizeof(double) * (size_t)B * H * t_cap * D);
   int rc = orc_score(B, H, Hq, D, t_cap, rot, ORC_Q_MINMAX, bits, group, 1, krope, n_sink, base, q, kcodes, ksz,
-                     ksink, NULL, kperm, NULL, NULL, NULL, tok, n_tok, scale, s);
+                     ksink, NULL, kperm, NULL, NULL, NULL, tok, n_tok, scale, s, NULL);
   if (!rc)
     rc = orc_decode(B, H, t_cap, D, tok, rot, ORC_Q_MINMAX, bits, group, 1, vrope, n_sink, base, vcodes, vsz,
-                    vsink, NULL, vperm, NULL, NULL, NULL, vh);
+                    vsink, NULL, vperm, NULL, NULL, NULL, vh, NULL);
   if (!rc) {
     for (int b = 0; b < B; ++b)
       for (int qh = 0; qh < Hq; ++qh) {
@@ -870,13 +884,13 @@ int orc_attend(int B, int H, int Hq, int D, int t_cap, int n_tok, int rot, int b
  * descending a_j; equal a_j keep ascending channel order.
  * ---------------------------------------------------------------------- */
 int orc_calibrate_perm(int B, int H, int T, int D, const int64_t* pos, int rope, int n_sink, double base,
-                       const uint16_t* x, int16_t* perm) {
+                       const uint16_t* x, int16_t* perm, const int32_t* sink_pos) {
   float* a = (float*)calloc((size_t)H * D, sizeof(float));
   float c[128], sn[128], xf[256], y[256];
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < H; ++h)
       for (int t = 0; t < T; ++t) {
-        if (pos[t] < n_sink) continue;
+        if (sink_slot(sink_pos, n_sink, b, pos[t]) >= 0) continue;
         const uint16_t* xv = x + ((size_t)(b * H + h) * T + t) * D;
         for (int j = 0; j < D; ++j) xf[j] = orc_half_to_float(xv[j]);
         if (rope) {
@@ -945,5 +959,72 @@ int orc_pair_energy(int B, int H, int T, int D, const uint16_t* x, uint64_t* ene
       rank[h * P + r] = (int16_t)i;
     }
   free(acc);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Sink detection by massive activations ([RotateKV] abstract (iii) and
+ * 关键设计: attention sinks are identified from the activations, by their
+ * massive magnitude, and protected). Per sequence b:
+ *   a_t = max over heads h and channels j of |x[b][h][t][j]| (exact fp16),
+ *   med = the lower median of a_0 .. a_{T-1} (rank floor((T-1)/2), ascending),
+ *   sinks = the tokens with a_t > tau * med (exact: both sides in fp64),
+ * at most max_sinks of them, the largest a_t first, equal a_t to the earlier
+ * token; sink_pos[b] lists their positions pos[t] in ascending order, padded
+ * with -1, and count[b] how many there are.
+ * Pins: constructed sequences with known massive tokens, the median by
+ * numpy, the cap, ties, the strict threshold.
+ * ---------------------------------------------------------------------- */
+static int cmp_f32(const void* pa, const void* pb) {
+  float a = *(const float*)pa, b = *(const float*)pb;
+  return a < b ? -1 : a > b ? 1 : 0;
+}
+
+int orc_detect_sinks(int B, int H, int T, int D, const int64_t* pos, const uint16_t* x, double tau, int max_sinks,
+                     int32_t* sink_pos, int32_t* count) {
+  if (T <= 0 || max_sinks < 1) return 1;
+  float* a = (float*)malloc(sizeof(float) * (size_t)T);
+  float* srt = (float*)malloc(sizeof(float) * (size_t)T);
+  int* pick = (int*)malloc(sizeof(int) * (size_t)max_sinks);
+  for (int b = 0; b < B; ++b) {
+    for (int t = 0; t < T; ++t) {
+      float m = 0.0f;
+      for (int h = 0; h < H; ++h) {
+        const uint16_t* xv = x + ((size_t)(b * H + h) * T + t) * D;
+        for (int j = 0; j < D; ++j) {
+          float v = fabsf(orc_half_to_float(xv[j]));
+          if (v > m) m = v;
+        }
+      }
+      a[t] = m;
+    }
+    memcpy(srt, a, sizeof(float) * (size_t)T);
+    qsort(srt, (size_t)T, sizeof(float), cmp_f32);
+    double thr = tau * (double)srt[(T - 1) / 2];
+    int n = 0;
+    for (int k = 0; k < max_sinks; ++k) {  /* the next largest a_t above the threshold */
+      int best = -1;
+      for (int t = 0; t < T; ++t) {
+        if (!((double)a[t] > thr)) continue;
+        int taken = 0;
+        for (int i = 0; i < n; ++i) taken |= pick[i] == t;
+        if (taken) continue;
+        if (best < 0 || a[t] > a[best]) best = t;  /* equal a_t: the earlier t stays */
+      }
+      if (best < 0) break;
+      pick[n++] = best;
+    }
+    for (int i = 1; i < n; ++i)  /* ascending positions */
+      for (int j = i; j > 0 && pick[j] < pick[j - 1]; --j) {
+        int tmp = pick[j];
+        pick[j] = pick[j - 1];
+        pick[j - 1] = tmp;
+      }
+    for (int k = 0; k < max_sinks; ++k) sink_pos[(size_t)b * max_sinks + k] = k < n ? (int32_t)pos[pick[k]] : -1;
+    count[b] = n;
+  }
+  free(a);
+  free(srt);
+  free(pick);
   return 0;
 }

@@ -39,6 +39,9 @@ CASES = [
     ("fused_gqa2_bits4_ragged", 1, 2, 4, 200, 131, 4, 128, 2, False, "fwht_head"),
     ("fused_sinks_only", 1, 2, 8, 16, 3, 2, 128, 4, True, "fwht_head"),
     ("fused_single_token_no_sinks", 1, 1, 1, 8, 1, 4, 128, 0, False, "fwht_head"),
+    # keys with half-split RoPE pairs (the fp16 sinks are turned on (i, i + 64))
+    ("half_split_fused_sinks", 2, 2, 8, 300, 300, 2, 128, 4, True, "fwht_head"),
+    ("half_split_three_kernel_sinks", 1, 2, 4, 260, 257, 2, 64, 4, True, "fwht_head"),
 ]
 E2E_PAIRS = 8  # (batch, query head) pairs checked end to end on the larger cases
 
@@ -63,7 +66,9 @@ def test_attend_parity(K, orc, case):
     vp = W.random_perm(H, D, 6) if use_perm else None
     common = dict(batch=B, heads=H, head_dim=D, tokens=t_cap, t_cap=t_cap, bits=bits, group=group,
                   n_sink=n_sink, rot=rot)
-    dk, dv = TA.make_desc(rope=1, **common), TA.make_desc(rope=0, **common)
+    krope = 2 if name.startswith("half_split") else 1  # 2: half-split RoPE pairs on the keys
+    okrope = orc.ROPE_STD + (orc.ROPE_HALF if krope == 2 else 0)
+    dk, dv = TA.make_desc(rope=krope, **common), TA.make_desc(rope=0, **common)
     tk = TA.make_tables(perm=torch.from_numpy(kp).cuda() if use_perm else None, rope_cs=TA.rope_table(t_cap, D))
     tv = TA.make_tables(perm=torch.from_numpy(vp).cuda() if use_perm else None)
     pk, pv = TA.alloc_packed(dk), TA.alloc_packed(dv)
@@ -88,9 +93,9 @@ def test_attend_parity(K, orc, case):
           "sink": pv.sink.cpu().numpy().view(np.uint16) if n_sink else None}
     pos = np.arange(t_cap)
     vhat = orc.decode(vc, pos, (B, H, t_cap, D), rope=0, perm=vp, **okw)[:, :, :n_tok]
-    khat = orc.decode(kc, pos, (B, H, t_cap, D), rope=1, perm=kp, **okw)
+    khat = orc.decode(kc, pos, (B, H, t_cap, D), rope=okrope, perm=kp, **okw)
     ref = orc.attend(q.view(np.uint16), kc, vc, n_tok, H=H, t_cap=t_cap, scale=scale, kperm=kp, vperm=vp,
-                     krope=1, vrope=0, **okw)
+                     krope=okrope, vrope=0, **okw)
     gq = Hq // H
     pairs = [(b, qh) for b in range(B) for qh in range(Hq)]
     e2e = set(pairs if len(pairs) <= E2E_PAIRS else
@@ -110,7 +115,7 @@ def test_attend_parity(K, orc, case):
             continue
         # end to end against the oracle
         if (b, h) not in krot:
-            krot[b, h] = np.stack([orc.rope_f64(khat[b, h, n], n) for n in range(n_tok)])
+            krot[b, h] = np.stack([orc.rope_f64(khat[b, h, n], n, mode=okrope) for n in range(n_tok)])
         ds = SCORE_REL * scale * (np.abs(krot[b, h]) @ np.abs(q[b, qh].astype(np.float64)))
         bound = (math.exp(2 * ds.max()) - 1) * vmax + tight
         assert np.all(np.abs(got[b, qh] - ref[b, qh]) <= bound), (b, qh, np.abs(got[b, qh] - ref[b, qh]).max())

@@ -21,6 +21,9 @@ CASES = [
     ("single_token", 3, 2, 1, 128, 7, 1, 0, "fwht_head", 1),
     ("all_positions_are_sinks", 1, 2, 3, 128, 0, 1, 4, "fwht_head", 1),
     ("many_chunks", 4, 2, 9000, 128, 0, 1, 4, "fwht_head", 1),
+    # rope 2: keys turned on half-split pairs (i, i + D/2) before the abs-max
+    ("keys_half_split", 2, 3, 300, 128, 0, 2, 4, "fwht_head", 1),
+    ("keys_half_split_d64_ragged", 1, 4, 77, 64, 9, 2, 10, "none", 1),
 ]
 
 
@@ -50,6 +53,7 @@ def test_calibrate_parity(K, orc, case):
     got = _run(x, B, H, T, D, t0, rope, n_sink, rot, gh)
     # the permutation's input is RoPE'd only where RoPE precedes it (head-dim variants)
     orope = rope if rot in ("none", "fwht_head") else 0
+    orope = {0: 0, 1: orc.ROPE_STD, 2: orc.ROPE_STD + orc.ROPE_HALF}[orope]
     want = orc.calibrate_perm(x.view(np.uint16), W.positions(t0, T), rope=orope, n_sink=n_sink)
     assert got.dtype == np.int16 and got.shape == (H, D)
     assert np.array_equal(got, want), (np.argwhere(got != want)[:5])

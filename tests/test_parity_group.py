@@ -20,6 +20,10 @@ CASES = [
     ("hg2_ragged", 1, 4, 130, 2, 2, 128, 1, True, 0, 0),
     ("hg2_bits4_g64", 2, 2, 65, 2, 4, 64, 0, False, 1, 0),
     ("append_one", 2, 8, 1, 8, 2, 128, 1, False, 4, 77),
+    # rope 2: half-split pairs (i, i + 64)
+    ("half_split_hg8_sinks", 2, 8, 70, 8, 2, 128, 2, False, 2, 0),
+    ("half_split_hg4_perm", 1, 4, 90, 4, 2, 128, 2, True, 0, 3),
+    ("half_split_hg2_g64", 1, 4, 130, 2, 3, 64, 2, True, 0, 0),
 ]
 
 
@@ -42,7 +46,8 @@ def run_group_case(K, orc, x, *, t0, t_cap, hg, bits, group, rope, perm, n_sink,
     TA.encode(d, torch.from_numpy(x).cuda(), tb, pk)
     assert K.kvq_check(0) == K.KVQ_OK
     pos = np.arange(t0, t0 + T)
-    okw = dict(rot=orc.ROT_FWHT_GROUP, bits=bits, group=group, group_heads=hg, rope=rope, n_sink=n_sink, perm=perm)
+    orope = {0: 0, 1: orc.ROPE_STD, 2: orc.ROPE_STD + orc.ROPE_HALF}[rope]
+    okw = dict(rot=orc.ROT_FWHT_GROUP, bits=bits, group=group, group_heads=hg, rope=orope, n_sink=n_sink, perm=perm)
     ref = orc.encode(x.view(np.uint16), pos, want_pre=True, **okw)
     gc = pk.codes[:, :, t0:t0 + T].cpu().numpy()
     gs = pk.scale_zero[:, :, t0:t0 + T].cpu().numpy()

@@ -30,6 +30,10 @@ CASES = [
     ("bits4_g64", 1, 8, 64, 128, 0, 0, 4, 64, 1, True, 0, "fwht_head"),
     ("bits2_g32", 1, 8, 64, 128, 0, 0, 2, 32, 1, False, 0, "fwht_head"),
     ("bits3_g128", 1, 8, 64, 128, 0, 0, 3, 128, 0, False, 0, "fwht_head"),
+    # rope 2: half-split pairs (i, i + D/2)
+    ("half_split_perm_sink", 2, 4, 37, 128, 5, 2, 2, 64, 2, True, 4, "fwht_head"),
+    ("half_split_d64", 1, 8, 40, 64, 2, 1, 3, 32, 2, True, 1, "fwht_head"),
+    ("half_split_no_rotation", 1, 8, 50, 128, 0, 0, 4, 128, 2, False, 2, "none"),
 ]
 
 
@@ -59,8 +63,10 @@ def run_head_case(K, orc, x, *, t0, t_cap, bits, group, rope, perm, n_sink, rot,
     TA.encode(d, xg, tb, pk)
     assert K.kvq_check(0) == K.KVQ_OK
     pos = np.arange(t0, t0 + T)
-    # the oracle's rope flag names its table: 1 standard, 2 frequency-aware
-    orope = rope * (orc.ROPE_FREQ_AWARE if freq == K.KVQ_ROPE_FREQ_AWARE else orc.ROPE_STD)
+    # the oracle's rope flag names its table (1 standard, 2 frequency-aware) plus
+    # ROPE_HALF for the half-split pairs the descriptor's rope = 2 selects
+    table = orc.ROPE_FREQ_AWARE if freq == K.KVQ_ROPE_FREQ_AWARE else orc.ROPE_STD
+    orope = 0 if not rope else table + (orc.ROPE_HALF if rope == 2 else 0)
     okw = dict(rot={"none": 0, "fwht_head": 1}[rot], bits=bits, group=group, rope=orope, n_sink=n_sink, perm=perm)
     ref = orc.encode(x.view(np.uint16), pos, want_pre=True, **okw)
     gc = pk.codes[:, :, t0:t0 + T].cpu().numpy()
@@ -145,10 +151,11 @@ def test_head_deterministic(K):
     assert torch.equal(a.codes, b.codes) and torch.equal(a.scale_zero, b.scale_zero)
 
 
-@pytest.mark.parametrize("D,group", [(128, 64), (64, 32)])
-def test_head_freq_aware_rope_table(K, orc, D, group):
+@pytest.mark.parametrize("D,group,rope", [(128, 64, 1), (64, 32, 1), (128, 64, 2)])
+def test_head_freq_aware_rope_table(K, orc, D, group, rope):
     """KV-Latent frequency-aware RoPE: the kernels take the table they are given;
-    codes stay bit-exact against the oracle rotating with the same frequencies."""
+    codes stay bit-exact against the oracle rotating with the same frequencies
+    (on interleaved or half-split pairs)."""
     x = _inputs("freq_aware", 2, 4, 70, D, 21)
-    run_head_case(K, orc, x, t0=3, t_cap=80, bits=2, group=group, rope=1, perm=W.random_perm(4, D, 8), n_sink=4,
+    run_head_case(K, orc, x, t0=3, t_cap=80, bits=2, group=group, rope=rope, perm=W.random_perm(4, D, 8), n_sink=4,
                   rot="fwht_head", freq=K.KVQ_ROPE_FREQ_AWARE)

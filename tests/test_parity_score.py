@@ -22,11 +22,11 @@ def K():
     return K
 
 
-def build_cache(K, w, x, x_app, perm, rot="fwht_head"):
+def build_cache(K, w, x, x_app, perm, rot="fwht_head", rope=1):
     from kv_cache_rotation_b200 import torch_api as TA
     B, H, T, D = x.shape
     t_cap = T + x_app.shape[2]
-    kw = dict(batch=B, heads=H, head_dim=D, t_cap=t_cap, bits=w.bits, group=w.group, rope=1, n_sink=w.n_sink,
+    kw = dict(batch=B, heads=H, head_dim=D, t_cap=t_cap, bits=w.bits, group=w.group, rope=rope, n_sink=w.n_sink,
               rot=rot, group_heads=w.group_heads)
     tb = TA.make_tables(perm=torch.from_numpy(perm).cuda() if perm is not None else None,
                         rope_cs=TA.rope_table(t_cap, D))
@@ -39,11 +39,12 @@ def build_cache(K, w, x, x_app, perm, rot="fwht_head"):
     return d_pre, tb, pk
 
 
-def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None):
+def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None, rope=1):
     from kv_cache_rotation_b200 import torch_api as TA
     x = W.kv_tensor(w, "k")
     x_app = W.kv_tensor(w, "k_append", T=w.append)
-    d, tb, pk = build_cache(K, w, x, x_app, perm, rot)
+    d, tb, pk = build_cache(K, w, x, x_app, perm, rot, rope)
+    orope = orc.ROPE_STD + (orc.ROPE_HALF if rope == 2 else 0)
     q = W.queries(w)
     n_tok = d.t_cap
     scale = 1.0 / math.sqrt(w.D)
@@ -54,7 +55,7 @@ def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None):
     cache = {"codes": pk.codes.cpu().numpy(), "sz": pk.scale_zero.cpu().numpy().view(np.uint16),
              "sink": pk.sink.cpu().numpy().view(np.uint16) if w.n_sink else None}
     okw = dict(rot={"none": 0, "fwht_head": 1, "fwht_group": 2}[rot], bits=w.bits, group=w.group,
-               group_heads=w.group_heads, rope=1, n_sink=w.n_sink, perm=perm)
+               group_heads=w.group_heads, rope=orope, n_sink=w.n_sink, perm=perm)
     ref = orc.score(q.view(np.uint16), cache, tok, H=w.H, t_cap=n_tok, scale=scale, **okw)
     # attention-space keys (fp64) for the L1 bound
     khat = orc.decode(cache, np.arange(n_tok), (w.B, w.H, n_tok, w.D), **okw)
@@ -64,7 +65,7 @@ def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None):
     for b in range(w.B):
         for qh in range(w.Hq):
             h = qh // gq
-            kk = np.stack([orc.rope_f64(khat[b, h, n], n) for n in tok])
+            kk = np.stack([orc.rope_f64(khat[b, h, n], n, mode=orope) for n in tok])
             bound = SCORE_REL * scale * (np.abs(kk) @ np.abs(q[b, qh].astype(np.float64)))
             err = np.abs(got[b, qh] - ref[b, qh])
             assert np.all(err <= bound), (b, qh, np.max(err / bound))
@@ -107,3 +108,18 @@ def test_score_grouped_cache(K, orc, hg, gq, bits, group, n_sink, T):
     w = W.Workload("score_group", B=2, H=hg, T=T, rot="fwht_group", group_heads=hg, bits=bits, group=group,
                    n_sink=n_sink, Hq=hg * gq, append=1, seed=70 + hg + gq)
     run_score_case(K, orc, w, None, rot="fwht_group")
+
+
+@pytest.mark.parametrize("rot,bits,group,D", [("fwht_head", 2, 128, 128), ("fwht_head", 3, 64, 128),
+                                              ("fwht_head", 2, 32, 64)])
+def test_score_half_split_sinks(K, orc, rot, bits, group, D):
+    """Keys with half-split RoPE pairs: the fp16 sinks are turned on (i, i + D/2)
+    (tensor-core and CUDA-core score kernels)."""
+    w = W.scaled(W.WORKLOADS["decode_score"], B=2, H=2, Hq=4, T=150, D=D, bits=bits, group=group, n_sink=4)
+    run_score_case(K, orc, w, W.random_perm(w.H, D, 12), rot=rot, rope=2)
+
+
+def test_score_grouped_cache_half_split(K, orc):
+    w = W.Workload("score_group_half", B=1, H=8, T=120, rot="fwht_group", group_heads=8, bits=2, group=128,
+                   n_sink=3, Hq=16, append=1, seed=91)
+    run_score_case(K, orc, w, None, rot="fwht_group", rope=2)

@@ -186,6 +186,29 @@ def iso3_tables(D: int, seed: int) -> np.ndarray:
     return g.astype(np.float32)
 
 
+def plant_massive(x: np.ndarray, n_tokens: int, seed: int, lo: float = 2000.0, hi: float = 6000.0,
+                  head_frac: float = 0.25):
+    """Massive activations on a few tokens, in place (the attention-sink tokens
+    of "RotateKV: Accurate and Robust 2-Bit KV Cache Quantization for LLMs via
+    Outlier-Aware Adaptive Rotations", abstract (iii)): per sequence, token 0
+    and n_tokens - 1 other tokens drawn uniformly get, in a random quarter of
+    the heads, one random channel set to +-U[lo, hi] (fp16). Returns the
+    planted token indices per sequence (sorted)."""
+    B, H, T, D = x.shape
+    rng = _rng(seed, 50)
+    planted = []
+    for b in range(B):
+        extra = rng.choice(np.arange(1, T), size=min(n_tokens - 1, T - 1), replace=False) if T > 1 else []
+        toks = sorted({0, *[int(t) for t in extra]})
+        for t in toks:
+            heads = rng.choice(H, size=max(1, int(round(head_frac * H))), replace=False)
+            for h in heads:
+                c = int(rng.integers(D))
+                x[b, h, t, c] = np.float16(rng.uniform(lo, hi) * (1 if rng.random() < 0.5 else -1))
+        planted.append(toks)
+    return planted
+
+
 def random_perm(H: int, D: int, seed: int) -> np.ndarray:
     """[H][D] int16, a seeded random permutation per head (any permutation
     exercises the permutation step; calibrated ones are computed elsewhere)."""
