@@ -99,6 +99,15 @@ def lib():
         L.orc_detect_sinks.argtypes = [ci, ci, ci, ci, i64p, u16p, cd, ci, i32p, i32p]
         L.orc_pair_energy.restype = ci
         L.orc_pair_energy.argtypes = [ci, ci, ci, ci, u16p, ctypes.POINTER(ctypes.c_uint64), i16p]
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        L.orc_dyn_calibrate.restype = ci
+        L.orc_dyn_calibrate.argtypes = [ci, ci, ci, ci, i64p, ci, ci, u16p, f32p, f32p, i32p, f64p, f32p, u32p]
+        L.orc_dyn_encode.restype = ci
+        L.orc_dyn_encode.argtypes = [ci, ci, ci, ci, i64p, ci, ci, ci, u16p, f32p, f32p, f32p, f32p, f32p, u32p,
+                                     u8p, u16p, u16p, f32p, f32p, i32p]
+        L.orc_dyn_decode.restype = ci
+        L.orc_dyn_decode.argtypes = [ci, ci, ci, ci, i64p, ci, ci, ci, u8p, u16p, u16p, f32p, f32p, f32p, f32p,
+                                     f32p, f32p, u32p, f64p, i32p]
         _lib = L
     return _lib
 
@@ -381,3 +390,85 @@ def pair_energy(x):
 def energy_ints(e):
     """(lo, hi) uint64 pairs -> Python ints."""
     return [[int(p[0]) | (int(p[1]) << 64) for p in row] for row in e]
+
+
+# ---------------------------------------------------------------- dynamic codebooks
+def _opt(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype)
+
+
+def dyn_calibrate(x, pos, *, rot, qL, qR=None, n_sink=0, sink_pos=None):
+    """Per-channel statistics of the rotated unit vectors (orc_dyn_calibrate):
+    returns (m2 float64 [H][D], sigma float32 [H][D], wide uint32 [H][D/32])."""
+    x = np.ascontiguousarray(x, np.uint16)
+    B, H, T, D = x.shape
+    pos = np.ascontiguousarray(pos, np.int64)
+    qL = np.ascontiguousarray(qL, np.float32)
+    qR = _opt(qR, np.float32)
+    sp = _opt(sink_pos, np.int32)
+    m2 = np.zeros((H, D), np.float64)
+    sigma = np.zeros((H, D), np.float32)
+    wide = np.zeros((H, D // 32), np.uint32)
+    rc = lib().orc_dyn_calibrate(B, H, T, D, _p(pos, ctypes.c_int64), rot, n_sink, _p(x, ctypes.c_uint16),
+                                 _p(qL, ctypes.c_float), _p(qR, ctypes.c_float) if qR is not None else None,
+                                 _p(sp, ctypes.c_int32) if sp is not None else None, _p(m2, ctypes.c_double),
+                                 _p(sigma, ctypes.c_float), _p(wide, ctypes.c_uint32))
+    if rc:
+        raise ValueError("orc_dyn_calibrate: unsupported arguments")
+    return m2, sigma, wide
+
+
+def dyn_encode(x, pos, *, rot, bits, qL, qR=None, cb, cbw, sigma, wide, n_sink=0, sink_pos=None, want_pre=False):
+    """IsoQuant with per-channel codebooks (orc_dyn_encode): codes [B][H][T][D*bits/8],
+    ext uint16 [B][H][T], sink uint16 [B][H][n_sink][D], norm f32 [B][H][T], pre (optional)."""
+    x = np.ascontiguousarray(x, np.uint16)
+    B, H, T, D = x.shape
+    pos = np.ascontiguousarray(pos, np.int64)
+    out = {"codes": np.zeros((B, H, T, D * bits // 8), np.uint8), "ext": np.zeros((B, H, T), np.uint16),
+           "sink": np.zeros((B, H, max(n_sink, 1), D), np.uint16), "norm": np.zeros((B, H, T), np.float32)}
+    pre = np.zeros((B, H, T, D), np.float32) if want_pre else None
+    qL = np.ascontiguousarray(qL, np.float32)
+    qR = _opt(qR, np.float32)
+    cb, cbw = np.ascontiguousarray(cb, np.float32), np.ascontiguousarray(cbw, np.float32)
+    sigma, wide = np.ascontiguousarray(sigma, np.float32), np.ascontiguousarray(wide, np.uint32)
+    sp = _opt(sink_pos, np.int32)
+    rc = lib().orc_dyn_encode(B, H, T, D, _p(pos, ctypes.c_int64), rot, bits, n_sink, _p(x, ctypes.c_uint16),
+                              _p(qL, ctypes.c_float), _p(qR, ctypes.c_float) if qR is not None else None,
+                              _p(cb, ctypes.c_float), _p(cbw, ctypes.c_float), _p(sigma, ctypes.c_float),
+                              _p(wide, ctypes.c_uint32), _p(out["codes"], ctypes.c_uint8),
+                              _p(out["ext"], ctypes.c_uint16), _p(out["sink"], ctypes.c_uint16),
+                              _p(out["norm"], ctypes.c_float), _p(pre, ctypes.c_float) if pre is not None else None,
+                              _p(sp, ctypes.c_int32) if sp is not None else None)
+    if rc:
+        raise ValueError("orc_dyn_encode: unsupported arguments")
+    if not n_sink:
+        out["sink"] = None
+    if want_pre:
+        out["pre"] = pre
+    return out
+
+
+def dyn_decode(packed, pos, shape, *, rot, bits, qL, qR=None, cb, cbw, sigma, wide, n_sink=0, sink_pos=None):
+    """Inverse of dyn_encode in fp64: float64 [B][H][T][D]."""
+    B, H, T, D = shape
+    pos = np.ascontiguousarray(pos, np.int64)
+    out = np.zeros((B, H, T, D), np.float64)
+    codes = np.ascontiguousarray(packed["codes"], np.uint8)
+    ext = np.ascontiguousarray(packed["ext"], np.uint16)
+    norm = np.ascontiguousarray(packed["norm"], np.float32)
+    sink = packed.get("sink")
+    sink = np.ascontiguousarray(sink, np.uint16) if sink is not None else np.zeros(1, np.uint16)
+    qL = np.ascontiguousarray(qL, np.float32)
+    qR = _opt(qR, np.float32)
+    cb, cbw = np.ascontiguousarray(cb, np.float32), np.ascontiguousarray(cbw, np.float32)
+    sigma, wide = np.ascontiguousarray(sigma, np.float32), np.ascontiguousarray(wide, np.uint32)
+    sp = _opt(sink_pos, np.int32)
+    rc = lib().orc_dyn_decode(B, H, T, D, _p(pos, ctypes.c_int64), rot, bits, n_sink, _p(codes, ctypes.c_uint8),
+                              _p(ext, ctypes.c_uint16), _p(sink, ctypes.c_uint16), _p(norm, ctypes.c_float),
+                              _p(qL, ctypes.c_float), _p(qR, ctypes.c_float) if qR is not None else None,
+                              _p(cb, ctypes.c_float), _p(cbw, ctypes.c_float), _p(sigma, ctypes.c_float),
+                              _p(wide, ctypes.c_uint32), _p(out, ctypes.c_double),
+                              _p(sp, ctypes.c_int32) if sp is not None else None)
+    if rc:
+        raise ValueError("orc_dyn_decode: unsupported arguments")
+    return out

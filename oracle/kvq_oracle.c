@@ -369,7 +369,7 @@ int orc_lloyd_max_normal(int bits, double* levels, double* mse_out) {
    N(0,1) levels scaled by sigma = 1/sqrt(d) (each coordinate of a random unit
    vector has variance 1/d), rounded once to fp32. */
 void orc_codebook(int bits, int d, float* out) {
-  double lv[16];
+  double lv[32];
   orc_lloyd_max_normal(bits, lv, NULL);
   for (int k = 0; k < (1 << bits); ++k) out[k] = (float)(lv[k] / sqrt((double)d));
 }
@@ -492,6 +492,33 @@ static void iso3_unrotate_f64(const double* w, const float* q, int D, double* v)
   }
 }
 
+/* The IsoQuant front end of one vector ([IsoQuant §3.1]): rho = ||x|| (fp64
+   sum of the exact squares in channel order, rounded to fp32), u = x / (rho +
+   1e-8) in fp32, then the rotation of `rot` -- the 4-D sandwich w = qL (x)
+   (u (x) qR) per block ([IsoQuant §2.2, §3.2]) or the 3-D sandwich of
+   iso3_rotate_f32 ([IsoQuant §2.1]). */
+static void iso_front(int rot, const uint16_t* xv, int D, const float* qL, const float* qR, float* w, float* rho_out) {
+  double acc = 0.0;
+  for (int j = 0; j < D; ++j) {
+    float f = orc_half_to_float(xv[j]);
+    acc += (double)f * (double)f;
+  }
+  float rho = (float)sqrt(acc);
+  float den = rho + 1e-8f;
+  float u[256];
+  for (int j = 0; j < D; ++j) u[j] = orc_half_to_float(xv[j]) / den;
+  if (rot == ORC_ROT_ISO3) {
+    iso3_rotate_f32(u, qL, D, w);
+  } else {
+    for (int k = 0; k < D / 4; ++k) {
+      float t4[4];
+      orc_quat_mul_f32(u + 4 * k, qR + 4 * k, t4);
+      orc_quat_mul_f32(qL + 4 * k, t4, w + 4 * k);
+    }
+  }
+  *rho_out = rho;
+}
+
 int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quant, int bits, int group,
                int group_heads, int rope, int n_sink, double base, const uint16_t* x, const int16_t* perm,
                const float* qL, const float* qR, const float* codebook, uint8_t* codes, uint16_t* sz,
@@ -524,48 +551,13 @@ int orc_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int quan
         }
         if (ks >= 0) continue;
 
-        if (rot == ORC_ROT_ISO3) {
-          /* the norm split of [IsoQuant §3.1], then the 3-D sandwich on
-             3-channel blocks ([IsoQuant §2.1]); Lloyd-Max codes */
-          size_t v = ((size_t)(b * H + h0) * T + t);
-          const uint16_t* xv = x + v * D;
-          double acc = 0.0;
-          for (int j = 0; j < D; ++j) {
-            float f = orc_half_to_float(xv[j]);
-            acc += (double)f * (double)f;
-          }
-          float rho = (float)sqrt(acc);
-          float den = rho + 1e-8f;
-          float u[256], w[256];
-          for (int j = 0; j < D; ++j) u[j] = orc_half_to_float(xv[j]) / den;
-          iso3_rotate_f32(u, qL, D, w);
-          uint8_t cds[256];
-          for (int j = 0; j < D; ++j) cds[j] = (uint8_t)codebook_code(w[j], codebook, bits);
-          if (pre) memcpy(pre + v * D, w, sizeof(float) * D);
-          orc_pack(cds, D, bits, codes + v * rb);
-          norm[v] = rho;
-          continue;
-        }
-
-        if (rot == ORC_ROT_ISO) {
+        if (rot == ORC_ROT_ISO || rot == ORC_ROT_ISO3) {
           /* [IsoQuant §3.1]: rho = ||x||, x_hat = x / (rho + eps); 4-D blocks
-             w = qL (x) (v (x) qR) ([IsoQuant §2.2, §3.2]); Lloyd-Max codes. */
+             w = qL (x) (v (x) qR) ([IsoQuant §2.2, §3.2]) or the 3-D sandwich
+             on 3-channel blocks ([IsoQuant §2.1]); Lloyd-Max codes. */
           size_t v = ((size_t)(b * H + h0) * T + t);
-          const uint16_t* xv = x + v * D;
-          double acc = 0.0;
-          for (int j = 0; j < D; ++j) {
-            float f = orc_half_to_float(xv[j]);
-            acc += (double)f * (double)f;
-          }
-          float rho = (float)sqrt(acc);
-          float den = rho + 1e-8f;
-          float u[256], w[256];
-          for (int j = 0; j < D; ++j) u[j] = orc_half_to_float(xv[j]) / den;
-          for (int k = 0; k < D / 4; ++k) {
-            float t4[4];
-            orc_quat_mul_f32(u + 4 * k, qR + 4 * k, t4);
-            orc_quat_mul_f32(qL + 4 * k, t4, w + 4 * k);
-          }
+          float rho, w[256];
+          iso_front(rot, x + v * D, D, qL, qR, w, &rho);
           uint8_t cds[256];
           for (int j = 0; j < D; ++j) cds[j] = (uint8_t)codebook_code(w[j], codebook, bits);
           if (pre) memcpy(pre + v * D, w, sizeof(float) * D);
@@ -655,6 +647,26 @@ static void quat_inv_f64(const float* q, double* o) {
   o[3] = -q[3] / n2;
 }
 
+/* Inverse of iso_front in fp64 ([IsoQuant §3.1] step 3): the inverse
+   rotation -- v = qL^-1 (x) (w (x) qR^-1) per 4-D block, or v = q* (x) (w (x)
+   q) per 3-D block -- then the norm restored, out = v * rho. */
+static void iso_back(int rot, const double* w, int D, const float* qL, const float* qR, float rho, double* out) {
+  if (rot == ORC_ROT_ISO3) {
+    double u[256];
+    iso3_unrotate_f64(w, qL, D, u);
+    for (int j = 0; j < D; ++j) out[j] = u[j] * (double)rho;
+    return;
+  }
+  for (int k = 0; k < D / 4; ++k) {
+    double li[4], ri[4], t4[4], v4[4];
+    quat_inv_f64(qL + 4 * k, li);
+    quat_inv_f64(qR + 4 * k, ri);
+    orc_quat_mul_f64(w + 4 * k, ri, t4);
+    orc_quat_mul_f64(li, t4, v4);
+    for (int e = 0; e < 4; ++e) out[4 * k + e] = v4[e] * (double)rho;
+  }
+}
+
 static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* codes, const uint16_t* sz,
                        const uint16_t* sink, const float* norm, const int16_t* perm, const float* qL,
                        const float* qR, const float* codebook, double* out, int attn_space) {
@@ -681,30 +693,13 @@ static int decode_impl(const orc_shape* s, const int64_t* pos, const uint8_t* co
           }
           continue;
         }
-        if (s->rot == ORC_ROT_ISO3) {
+        if (s->rot == ORC_ROT_ISO || s->rot == ORC_ROT_ISO3) {
           size_t v = ((size_t)(b * H + h0) * T + t);
           uint8_t cds[256];
           orc_unpack(codes + v * rb, D, s->bits, cds);
-          double w[256], u[256];
+          double w[256];
           for (int j = 0; j < D; ++j) w[j] = codebook[cds[j]];
-          iso3_unrotate_f64(w, qL, D, u);
-          for (int j = 0; j < D; ++j) out[v * D + j] = u[j] * (double)norm[v];
-          continue;
-        }
-        if (s->rot == ORC_ROT_ISO) {
-          size_t v = ((size_t)(b * H + h0) * T + t);
-          uint8_t cds[256];
-          orc_unpack(codes + v * rb, D, s->bits, cds);
-          double rho = norm[v];
-          for (int k = 0; k < D / 4; ++k) {
-            double w4[4], li[4], ri[4], t4[4], v4[4];
-            for (int e = 0; e < 4; ++e) w4[e] = codebook[cds[4 * k + e]];
-            quat_inv_f64(qL + 4 * k, li);
-            quat_inv_f64(qR + 4 * k, ri);
-            orc_quat_mul_f64(w4, ri, t4);
-            orc_quat_mul_f64(li, t4, v4);
-            for (int e = 0; e < 4; ++e) out[v * D + 4 * k + e] = v4[e] * rho;
-          }
+          iso_back(s->rot, w, D, qL, qR, norm[v], out + v * D);
           continue;
         }
         if (s->rot == ORC_ROT_FWHT_GROUP) {
@@ -1026,5 +1021,166 @@ int orc_detect_sinks(int B, int H, int T, int D, const int64_t* pos, const uint1
   free(a);
   free(srt);
   free(pick);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Dynamic codebooks for IsoQuant ([IsoQuant §4.2] quantization error
+ * control: per-channel value statistics gathered online, quantization
+ * boundaries set by the KL divergence, codebooks of twice the size for
+ * outlier channels). Readings:
+ *  - the statistics are per head h and channel j of the rotated unit vectors
+ *    w (the quantizer's input, iso_front), over the batches and the
+ *    non-sink positions of the calibration tokens: m2[h][j] = sum w_j^2 / N
+ *    in fp64, sequentially;
+ *  - the candidate codebooks are the Lloyd-Max designs for N(0, sigma^2),
+ *    i.e. the N(0,1) levels l_k scaled by sigma; the KL divergence from the
+ *    channel's distribution to N(0, sigma^2) is
+ *    const + log sigma + m2 / (2 sigma^2), smallest at sigma^2 = m2, so
+ *    sigma[h][j] = (float)sqrt(m2) (fp32(1/sqrt(D)), the fixed codebook's
+ *    scale, when N = 0);
+ *  - outlier channels: sigma_j > 2 * the lower median of the head's sigmas
+ *    (rank floor((D-1)/2)), at most D/8 of them, the largest first, equal
+ *    sigmas to the lower channel; bit j of wide[h][j/32] marks them; they use
+ *    the (bits+1)-bit levels (twice the codebook);
+ *  - channel j's levels are L_k = fp32(sigma_j * l_k) and its boundaries the
+ *    fp32 midpoints 0.5f * (L_k + L_{k+1}); code = number of boundaries
+ *    strictly below w_j (ties to the lower code);
+ *  - storage: the low `bits` bits of every code in the record (LSB-first, as
+ *    the fixed codebook), and the top bit of each outlier channel's code in
+ *    ext[slot] (uint16), in ascending channel order, LSB first.
+ * Pins: sigma against a numerical KL minimisation (scipy) and numpy
+ * moments of the encoder's w; the outlier rule by brute force; codes against
+ * the nearest level by brute force; the fixed-codebook special case
+ * (every sigma equal, no outlier) byte for byte.
+ * ---------------------------------------------------------------------- */
+static int dyn_is_wide(const uint32_t* wide, int h, int D, int j) {
+  return (wide[(size_t)h * (D / 32) + j / 32] >> (j % 32)) & 1u;
+}
+
+static int dyn_code(float w, float sigma, const float* lv, int n) {
+  int c = 0;
+  for (int k = 0; k + 1 < n; ++k) {
+    float a = sigma * lv[k], b = sigma * lv[k + 1];
+    float beta = 0.5f * (a + b);
+    if (w > beta) ++c;
+  }
+  return c;
+}
+
+int orc_dyn_calibrate(int B, int H, int T, int D, const int64_t* pos, int rot, int n_sink, const uint16_t* x,
+                      const float* qL, const float* qR, const int32_t* sink_pos, double* m2, float* sigma,
+                      uint32_t* wide) {
+  if ((rot != ORC_ROT_ISO && rot != ORC_ROT_ISO3) || D < 32 || D > 256 || D % 32) return 1;
+  for (int h = 0; h < H; ++h) {
+    double* s = m2 + (size_t)h * D;
+    for (int j = 0; j < D; ++j) s[j] = 0.0;
+    long long n = 0;
+    for (int b = 0; b < B; ++b)
+      for (int t = 0; t < T; ++t) {
+        if (sink_slot(sink_pos, n_sink, b, pos[t]) >= 0) continue;
+        float w[256], rho;
+        iso_front(rot, x + ((size_t)(b * H + h) * T + t) * D, D, qL, qR, w, &rho);
+        for (int j = 0; j < D; ++j) s[j] += (double)w[j] * (double)w[j];
+        ++n;
+      }
+    float* sg = sigma + (size_t)h * D;
+    for (int j = 0; j < D; ++j) {
+      if (n > 0) s[j] /= (double)n;
+      sg[j] = n > 0 ? (float)sqrt(s[j]) : (float)(1.0 / sqrt((double)D));
+    }
+    /* lower median by counting ranks (ties to the lower channel) */
+    float med = 0.0f;
+    for (int j = 0; j < D; ++j) {
+      int r = 0;
+      for (int k = 0; k < D; ++k) r += sg[k] < sg[j] || (sg[k] == sg[j] && k < j);
+      if (r == (D - 1) / 2) med = sg[j];
+    }
+    uint32_t* wd = wide + (size_t)h * (D / 32);
+    for (int i = 0; i < D / 32; ++i) wd[i] = 0;
+    for (int j = 0; j < D; ++j) {
+      if (!(sg[j] > 2.0f * med)) continue;
+      int above = 0; /* channels ahead of j in the outlier order */
+      for (int k = 0; k < D; ++k) above += sg[k] > sg[j] || (sg[k] == sg[j] && k < j);
+      if (above < D / 8) wd[j / 32] |= 1u << (j % 32);
+    }
+  }
+  return 0;
+}
+
+int orc_dyn_encode(int B, int H, int T, int D, const int64_t* pos, int rot, int bits, int n_sink,
+                   const uint16_t* x, const float* qL, const float* qR, const float* cb, const float* cbw,
+                   const float* sigma, const uint32_t* wide, uint8_t* codes, uint16_t* ext, uint16_t* sink,
+                   float* norm, float* pre, const int32_t* sink_pos) {
+  if ((rot != ORC_ROT_ISO && rot != ORC_ROT_ISO3) || bits < 2 || bits > 4 || D < 32 || D > 256 || D % 32) return 1;
+  size_t rb = (size_t)D * bits / 8;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int t = 0; t < T; ++t) {
+        size_t v = (size_t)(b * H + h) * T + t;
+        const int ks = sink_slot(sink_pos, n_sink, b, pos[t]);
+        if (ks >= 0) {
+          memcpy(sink + ((size_t)(b * H + h) * n_sink + ks) * D, x + v * D, sizeof(uint16_t) * D);
+          memset(codes + v * rb, 0, rb);
+          ext[v] = 0;
+          norm[v] = 0.0f;
+          continue;
+        }
+        float w[256], rho;
+        iso_front(rot, x + v * D, D, qL, qR, w, &rho);
+        uint8_t lo[256];
+        uint16_t e = 0;
+        int nw = 0;
+        for (int j = 0; j < D; ++j) {
+          const float sg = sigma[(size_t)h * D + j];
+          if (dyn_is_wide(wide, h, D, j)) {
+            int c = dyn_code(w[j], sg, cbw, 1 << (bits + 1));
+            lo[j] = (uint8_t)(c & ((1 << bits) - 1));
+            if (nw < 16) e |= (uint16_t)((c >> bits) << nw);
+            ++nw;
+          } else {
+            lo[j] = (uint8_t)dyn_code(w[j], sg, cb, 1 << bits);
+          }
+        }
+        orc_pack(lo, D, bits, codes + v * rb);
+        ext[v] = e;
+        norm[v] = rho;
+        if (pre) memcpy(pre + v * D, w, sizeof(float) * D);
+      }
+  return 0;
+}
+
+int orc_dyn_decode(int B, int H, int T, int D, const int64_t* pos, int rot, int bits, int n_sink,
+                   const uint8_t* codes, const uint16_t* ext, const uint16_t* sink, const float* norm,
+                   const float* qL, const float* qR, const float* cb, const float* cbw, const float* sigma,
+                   const uint32_t* wide, double* out, const int32_t* sink_pos) {
+  if ((rot != ORC_ROT_ISO && rot != ORC_ROT_ISO3) || bits < 2 || bits > 4 || D < 32 || D > 256 || D % 32) return 1;
+  size_t rb = (size_t)D * bits / 8;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int t = 0; t < T; ++t) {
+        size_t v = (size_t)(b * H + h) * T + t;
+        const int ks = sink_slot(sink_pos, n_sink, b, pos[t]);
+        if (ks >= 0) {
+          const uint16_t* sv = sink + ((size_t)(b * H + h) * n_sink + ks) * D;
+          for (int j = 0; j < D; ++j) out[v * D + j] = orc_half_to_float(sv[j]);
+          continue;
+        }
+        uint8_t lo[256];
+        orc_unpack(codes + v * rb, D, bits, lo);
+        double w[256];
+        int nw = 0;
+        for (int j = 0; j < D; ++j) {
+          const float sg = sigma[(size_t)h * D + j];
+          if (dyn_is_wide(wide, h, D, j)) {
+            int c = lo[j] | (nw < 16 ? ((ext[v] >> nw) & 1) << bits : 0);
+            w[j] = (double)(sg * cbw[c]);
+            ++nw;
+          } else {
+            w[j] = (double)(sg * cb[lo[j]]);
+          }
+        }
+        iso_back(rot, w, D, qL, qR, norm[v], out + v * D);
+      }
   return 0;
 }
