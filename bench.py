@@ -411,9 +411,17 @@ class EncDecStep:
             perm = torch.from_numpy(W.random_perm(H, D, w.seed + len(which))).to(device) if w.perm else None
             if iso:
                 qL, qR = W.iso_tables(w) if w.rot == "iso" else (W.iso3_tables(D, w.seed), None)
-                tb = TA.make_tables(qL=torch.from_numpy(qL).to(device),
-                                    qR=torch.from_numpy(qR).to(device) if qR is not None else None,
-                                    codebook=TA.lloyd_max_codebook(w.bits, D, device=device))
+                qLd = torch.from_numpy(qL).to(device)
+                qRd = torch.from_numpy(qR).to(device) if qR is not None else None
+                if w.quant == "codebook_dyn":
+                    # per-channel tables from the same tokens (untimed), then the
+                    # quality of both codebooks on them
+                    tb = TA.make_tables(qL=qLd, qR=qRd, codebook=TA.lloyd_max_codebook(w.bits, 1, device=device),
+                                        codebook_wide=TA.lloyd_max_codebook(w.bits + 1, 1, device=device))
+                    tb.ch_scale, tb.ch_wide = TA.calibrate_codebook(d, x, tb)
+                    self.quality = self._snr(TA, d, x, tb, qLd, qRd, w, device)
+                else:
+                    tb = TA.make_tables(qL=qLd, qR=qRd, codebook=TA.lloyd_max_codebook(w.bits, D, device=device))
             else:
                 tb = TA.make_tables(perm=perm, rope_cs=TA.rope_table(T, D, device=device) if rope else None)
             pk = TA.alloc_packed(d, device)
@@ -421,6 +429,8 @@ class EncDecStep:
             self.items.append((which, d, x, tb, pk, out))
             nvec = B * H * T
             per_vec = D * w.bits // 8 + (4 * (D // w.group) if w.quant == "minmax" else 4)
+            if w.quant == "codebook_dyn":
+                per_vec += 2  # the outlier channels' top bits
             self.alg[f"encode_{which}"] = nvec * (2 * D + per_vec) + (B * H * w.n_sink * D * 2)
             self.alg[f"decode_{which}"] = nvec * (2 * D + per_vec)
             self.fp16_equiv[f"encode_{which}"] = nvec * 2 * D
@@ -433,6 +443,29 @@ class EncDecStep:
                     self.fp32_ops[n] = nvec * D * ops
         self.names = list(self.alg)
         torch.cuda.synchronize(device)
+
+    @staticmethod
+    def _snr(TA, d, x, tb, qL, qR, w, device, rows=1 << 18):
+        """SNR (dB) of the decode against the input on the first `rows` vectors,
+        with the dynamic tables and with the fixed N(0, 1/D) codebook."""
+        import torch
+        n = min(rows, d.batch * d.heads * d.tokens)
+        b = max(1, n // (d.heads * d.tokens))
+        ds = TA.make_desc(batch=b, heads=d.heads, head_dim=d.head_dim, tokens=d.tokens, bits=d.bits, rot=d.rot,
+                          quant=d.quant)
+        xs = x[:b].contiguous()
+        ref = xs.float()
+        out = {}
+        fixed = TA.make_tables(qL=qL, qR=qR, codebook=TA.lloyd_max_codebook(w.bits, d.head_dim, device=device))
+        for name, q, t in (("dynamic", d.quant, tb), ("fixed", TA.QUANT["codebook"], fixed)):
+            ds.quant = q
+            pk = TA.alloc_packed(ds, device)
+            y = torch.empty_like(ref)
+            TA.encode(ds, xs, t, pk)
+            TA.decode(ds, pk, t, y)
+            out[f"snr_db_{name}"] = float(10 * torch.log10((ref ** 2).sum() / ((ref - y) ** 2).sum()))
+        out["snr_sample_vectors"] = b * d.heads * d.tokens
+        return out
 
     def launches(self):
         """One launch per entry of self.names, in the same order (encode then
@@ -761,6 +794,8 @@ def run_ours(args):
             "gpu_launches": getattr(st, "kernels_per_step", nk) * args.steps, "clocks": clocks, "kernels": kernels,
             "status": K.kvq_status_str(status),
         }
+        if hasattr(st, "quality"):
+            line["quality"] = st.quality
         print(json.dumps(line))
     if dist:
         dist.barrier()
@@ -812,6 +847,12 @@ def _other_config(name, n_gpus):
                 "cache": "grouped-head FWHT over 8 heads x 128 before RoPE, 2-bit group 128 (the headline K cache)",
                 "l2": "no flush (the 38 MB cache and 17 MB of scores are read / written once per step)",
                 "parallelism": f"replicas x{n_gpus}"}
+    if name == "llama2_7b_sink_detect":
+        w = W.WORKLOADS["llama2_7b_mha"]
+        return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T,
+                "input": "keys fp16 with massive activations planted on 4 tokens per sequence",
+                "tau": 8.0, "max_sinks": 8,
+                "l2": "no flush (the 268 MB input is larger than L2)", "parallelism": f"replicas x{n_gpus}"}
     if name == "llama3_8b_calibrate":
         w = W.WORKLOADS["llama3_8b_gqa_score"]
         return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T,
@@ -838,7 +879,8 @@ def main():
                     help="token positions (of each of the 4 sequences) per reference-arm step")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--workload", default="llama3_8b_gqa",
-                    choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "isoquant_so3_batch", "decode_score",
+                    choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "isoquant_so3_batch",
+                             "isoquant_dyn_batch", "decode_score",
                              "llama3_8b_gqa_group_score", "llama2_7b_sink_detect",
                              "llama3_8b_gqa_attend", "llama3_8b_calibrate", "llama3_8b_pair_energy", "tiny"],
                     help="which workload a step runs (the headline line is llama3_8b_gqa)")

@@ -62,14 +62,24 @@ enum {
 
 /* Scalar quantizer. */
 enum {
-  KVQ_Q_MINMAX = 0,  /* per-token per-group asymmetric min-max, fp16 (scale, zero); with
-                        rot in {NONE, FWHT_HEAD, FWHT_GROUP} */
-  KVQ_Q_CODEBOOK = 1 /* fixed scalar codebook (Lloyd-Max, [IsoQuant §3.1]); with rot = ISO_SO4
-                        or ISO_SO3 */
+  KVQ_Q_MINMAX = 0,   /* per-token per-group asymmetric min-max, fp16 (scale, zero); with
+                         rot in {NONE, FWHT_HEAD, FWHT_GROUP} */
+  KVQ_Q_CODEBOOK = 1, /* fixed scalar codebook (Lloyd-Max, [IsoQuant §3.1]); with rot = ISO_SO4
+                         or ISO_SO3 */
+  KVQ_Q_CODEBOOK_DYN = 2 /* dynamic codebooks ([IsoQuant §4.2]); with rot = ISO_SO4 or ISO_SO3:
+                         channel j of head h quantizes against the levels fp32(ch_scale[h][j] * l_k)
+                         of the N(0,1) Lloyd-Max design l -- `codebook` (2^bits levels), or
+                         `codebook_wide` (2^(bits+1) levels, twice the codebook) for the channels
+                         marked in ch_wide -- with fp32 midpoints as boundaries (ties to the lower
+                         code). The low `bits` bits of every code go to the record as for
+                         KVQ_Q_CODEBOOK; the top bit of each marked channel's code goes to
+                         ext[slot], in ascending channel order, LSB first (at most 16 marked
+                         channels per head; bits of further ones are dropped). Fill the tables with
+                         kvq_calibrate_codebook and kvq_lloyd_max_codebook(.., head_dim = 1). */
 };
 
 /* Which packed buffer kvq_packed_bytes sizes. */
-enum { KVQ_FIELD_CODES = 0, KVQ_FIELD_SCALE_ZERO = 1, KVQ_FIELD_SINK = 2, KVQ_FIELD_NORM = 3 };
+enum { KVQ_FIELD_CODES = 0, KVQ_FIELD_SCALE_ZERO = 1, KVQ_FIELD_SINK = 2, KVQ_FIELD_NORM = 3, KVQ_FIELD_EXT = 4 };
 
 typedef struct {
   int32_t batch;       /* B > 0 */
@@ -99,13 +109,17 @@ typedef struct {
  *   sink        half [B][H][n_sink][head_dim]          the sink positions, verbatim (row k: position
  *                                                     k, or the list's entry k)
  *   norm        f32  [B][H][t_cap]                      rho; ISO_SO4 and ISO_SO3 only
- * Slots of sink positions hold zero codes, zero scale/zero and zero norm.
- * Alignment: codes, scale_zero and sink 16 bytes; norm 4 bytes. Unused fields may be NULL. */
+ *   ext         u16  [B][H][t_cap]                      KVQ_Q_CODEBOOK_DYN only: the top bits of the
+ *                                                     outlier channels' codes
+ * Slots of sink positions hold zero codes, zero scale/zero, zero norm and zero ext.
+ * Alignment: codes, scale_zero and sink 16 bytes; norm 4 bytes; ext 2 bytes. Unused fields may
+ * be NULL. */
 typedef struct {
   uint8_t* codes;
   void* scale_zero;
   void* sink;
   float* norm;
+  uint16_t* ext;
 } kvq_packed;
 
 /* Read-only tables (device pointers).
@@ -118,7 +132,13 @@ typedef struct {
  *             (ISO_SO4). ISO_SO3 reads qL only: f32 [ceil(head_dim/3)][4], one unit quaternion
  *             per 3-channel block and, when head_dim mod 3 = 2, one for the 2-channel tail whose
  *             i and j parts must be zero (otherwise the tail's output is not a rotation)
- *   codebook  f32 [1 << bits] ascending levels (kvq_lloyd_max_codebook)
+ *   codebook  f32 [1 << bits] ascending levels (kvq_lloyd_max_codebook); for KVQ_Q_CODEBOOK_DYN
+ *             the N(0,1) levels (head_dim 1)
+ *   codebook_wide  f32 [2 << bits] KVQ_Q_CODEBOOK_DYN: the N(0,1) levels of bits + 1
+ *   ch_scale  f32 [H][head_dim] KVQ_Q_CODEBOOK_DYN: per-channel scale (kvq_calibrate_codebook),
+ *             16-byte aligned
+ *   ch_wide   u32 [H][head_dim/32] KVQ_Q_CODEBOOK_DYN: bit j of word j/32 marks channel j as an
+ *             outlier channel (the wide codebook), 4-byte aligned
  *   sink_pos  int32 [B][n_sink] or NULL (the sinks are positions 0..n_sink-1): the list form
  *             of the sink set ([RotateKV] attention sinks found from the activations, e.g. by
  *             kvq_detect_sinks). Entry k of sequence b is the position (cache slot) whose fp16
@@ -135,6 +155,9 @@ typedef struct {
   const float* qR;
   const float* codebook;
   const int32_t* sink_pos;
+  const float* codebook_wide;
+  const float* ch_scale;
+  const uint32_t* ch_wide;
 } kvq_tables;
 
 /* Encode T tokens into cache slots t0..t0+T-1.
@@ -243,6 +266,30 @@ kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables
 /* Workspace bytes kvq_calibrate_perm needs for d; 0 if d is invalid or unsupported. */
 size_t kvq_calibrate_workspace_bytes(const kvq_desc* d);
 
+/* Dynamic codebook tables ([IsoQuant §4.2]: the values of each channel are gathered online, the
+ * quantization boundaries set by the KL divergence, and outlier channels get a codebook twice the
+ * size). For each head h and channel j of the rotated unit vectors w (the quantizer's input of
+ * kvq_encode with d->rot, ISO_SO4 or ISO_SO3, over the B batches and the positions t0..t0+T-1
+ * that are not sinks):
+ *   m2 = mean of w_j^2 (fp64 sums), ch_scale[h][j] = fp32(sqrt(m2)): the sigma of N(0, sigma^2)
+ *        nearest to the channel's values in KL divergence (that divergence is
+ *        const + log sigma + m2 / (2 sigma^2)); fp32(1/sqrt(head_dim)) when no position counts;
+ *   ch_wide[h]: channels with ch_scale > 2 x the lower median of the head's scales, at most
+ *        head_dim/8 of them, the largest first, equal scales to the lower channel.
+ *   x          half [B][H][T][head_dim], 16-byte aligned
+ *   tb         qL (and qR for ISO_SO4) as for kvq_encode; sink_pos optional
+ *   ch_scale_out  f32 [H][head_dim], 16-byte aligned;  ch_wide_out  u32 [H][head_dim/32]
+ *   workspace  device memory of kvq_calibrate_codebook_workspace_bytes(d) bytes, 256-byte aligned
+ * Two kernels: per (sequence, head, 1024-token chunk) sums in a fixed order, then one CTA per head;
+ * the result does not depend on scheduling. KVQ_ERR_UNSUPPORTED for other rotations and for
+ * B*H > 65535. */
+kvq_status kvq_calibrate_codebook(const kvq_desc* d, const void* x, const kvq_tables* tb, float* ch_scale_out,
+                                  uint32_t* ch_wide_out, void* workspace, size_t workspace_bytes,
+                                  kvq_stream_t stream);
+
+/* Workspace bytes kvq_calibrate_codebook needs for d; 0 if d is invalid or unsupported. */
+size_t kvq_calibrate_codebook_workspace_bytes(const kvq_desc* d);
+
 /* Attention sinks by massive activations ([RotateKV] abstract (iii) and 关键设计: the sink
  * tokens carry activations far above the rest and are found from them). Per sequence b of the
  * T tokens x[b][:, t] at positions t0 + t:
@@ -306,7 +353,8 @@ enum {
 kvq_status kvq_rope_table_ex(float* cs_host, int32_t t_max, int32_t head_dim, double base, int32_t freq);
 
 /* Fill a HOST buffer with the 2^bits Lloyd-Max levels of N(0, 1/head_dim), ascending: Lloyd's
- * iteration on N(0,1) in double, scaled by 1/sqrt(head_dim), rounded to fp32 ([IsoQuant §3.1]). */
+ * iteration on N(0,1) in double, scaled by 1/sqrt(head_dim), rounded to fp32 ([IsoQuant §3.1]).
+ * bits 1..5 (5: the wide codebook of 4-bit dynamic codes). */
 kvq_status kvq_lloyd_max_codebook(float* levels_host, int32_t bits, int32_t head_dim);
 
 /* Synchronise `stream` and report (then clear) the device error word of the current device:

@@ -19,12 +19,13 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 KVQ_OK, KVQ_ERR_INVALID, KVQ_ERR_UNSUPPORTED, KVQ_ERR_ALIGN, KVQ_ERR_CUDA, KVQ_ERR_TIMEOUT = range(6)
 KVQ_ROT_NONE, KVQ_ROT_FWHT_HEAD, KVQ_ROT_FWHT_GROUP, KVQ_ROT_ISO_SO4, KVQ_ROT_ISO_SO3 = range(5)
-KVQ_Q_MINMAX, KVQ_Q_CODEBOOK = 0, 1
-KVQ_FIELD_CODES, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_FIELD_NORM = range(4)
+KVQ_Q_MINMAX, KVQ_Q_CODEBOOK, KVQ_Q_CODEBOOK_DYN = 0, 1, 2
+KVQ_FIELD_CODES, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_FIELD_NORM, KVQ_FIELD_EXT = range(5)
 
 EXPORTED = ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_attend_workspace_bytes",
             "kvq_calibrate_perm", "kvq_calibrate_workspace_bytes", "kvq_pair_energy",
             "kvq_detect_sinks", "kvq_detect_sinks_workspace_bytes",
+            "kvq_calibrate_codebook", "kvq_calibrate_codebook_workspace_bytes",
             "kvq_packed_bytes", "kvq_rope_table", "kvq_rope_table_ex", "kvq_lloyd_max_codebook", "kvq_check", "kvq_debug_expire_wait",
             "kvq_status_str", "kvq_version")
 
@@ -37,13 +38,14 @@ class kvq_desc(ctypes.Structure):
 
 class kvq_packed(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scale_zero", ctypes.c_void_p), ("sink", ctypes.c_void_p),
-                ("norm", ctypes.c_void_p)]
+                ("norm", ctypes.c_void_p), ("ext", ctypes.c_void_p)]
 
 
 class kvq_tables(ctypes.Structure):
     _fields_ = [("perm", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p), ("rope_rows", ctypes.c_int32),
                 ("qL", ctypes.c_void_p), ("qR", ctypes.c_void_p), ("codebook", ctypes.c_void_p),
-                ("sink_pos", ctypes.c_void_p)]
+                ("sink_pos", ctypes.c_void_p), ("codebook_wide", ctypes.c_void_p), ("ch_scale", ctypes.c_void_p),
+                ("ch_wide", ctypes.c_void_p)]
 
 
 class KvqError(RuntimeError):
@@ -71,6 +73,9 @@ def _load():
     L.kvq_detect_sinks.argtypes = [P(kvq_desc), vp, ctypes.c_double, i32, vp, vp, vp, ctypes.c_size_t, st]
     L.kvq_detect_sinks_workspace_bytes.argtypes = [P(kvq_desc)]
     L.kvq_detect_sinks_workspace_bytes.restype = ctypes.c_size_t
+    L.kvq_calibrate_codebook.argtypes = [P(kvq_desc), vp, P(kvq_tables), vp, vp, vp, ctypes.c_size_t, st]
+    L.kvq_calibrate_codebook_workspace_bytes.argtypes = [P(kvq_desc)]
+    L.kvq_calibrate_codebook_workspace_bytes.restype = ctypes.c_size_t
     L.kvq_calibrate_workspace_bytes.argtypes = [P(kvq_desc)]
     L.kvq_calibrate_workspace_bytes.restype = ctypes.c_size_t
     L.kvq_attend_workspace_bytes.argtypes = [P(kvq_desc), P(kvq_desc), i32, i32]
@@ -86,7 +91,7 @@ def _load():
     L.kvq_status_str.restype = ctypes.c_char_p
     L.kvq_version.restype = i32
     for n in ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_calibrate_perm",
-              "kvq_pair_energy", "kvq_detect_sinks",
+              "kvq_pair_energy", "kvq_detect_sinks", "kvq_calibrate_codebook",
               "kvq_rope_table", "kvq_rope_table_ex",
               "kvq_lloyd_max_codebook",
               "kvq_check", "kvq_debug_expire_wait"):
@@ -143,6 +148,16 @@ def kvq_detect_sinks(d: kvq_desc, x: int, tau: float, max_sinks: int, sink_pos: 
                      workspace_bytes: int, stream: int = 0) -> int:
     return lib.kvq_detect_sinks(ctypes.byref(d), x, tau, max_sinks, sink_pos, count, workspace, workspace_bytes,
                                 stream)
+
+
+def kvq_calibrate_codebook(d: kvq_desc, x: int, tb: kvq_tables, ch_scale_out: int, ch_wide_out: int,
+                           workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    return lib.kvq_calibrate_codebook(ctypes.byref(d), x, ctypes.byref(tb), ch_scale_out, ch_wide_out, workspace,
+                                      workspace_bytes, stream)
+
+
+def kvq_calibrate_codebook_workspace_bytes(d: kvq_desc) -> int:
+    return lib.kvq_calibrate_codebook_workspace_bytes(ctypes.byref(d))
 
 
 def kvq_detect_sinks_workspace_bytes(d: kvq_desc) -> int:

@@ -62,7 +62,6 @@ kvq_status get_ctx(LaunchCtx* ctx) {
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 
 // Shape / parameter validation common to every entry point.
 kvq_status check_desc(const kvq_desc* d) {
@@ -92,13 +91,14 @@ kvq_status check_desc(const kvq_desc* d) {
       break;
     case KVQ_ROT_ISO_SO4:
     case KVQ_ROT_ISO_SO3:
-      if (d->quant != KVQ_Q_CODEBOOK) return KVQ_ERR_UNSUPPORTED;
+      if (d->quant != KVQ_Q_CODEBOOK && d->quant != KVQ_Q_CODEBOOK_DYN) return KVQ_ERR_UNSUPPORTED;
       if (d->rope) return KVQ_ERR_UNSUPPORTED;
       break;
     default:
       return KVQ_ERR_INVALID;
   }
-  if (d->quant != KVQ_Q_MINMAX && d->quant != KVQ_Q_CODEBOOK) return KVQ_ERR_INVALID;
+  if (d->quant != KVQ_Q_MINMAX && d->quant != KVQ_Q_CODEBOOK && d->quant != KVQ_Q_CODEBOOK_DYN)
+    return KVQ_ERR_INVALID;
   return KVQ_OK;
 }
 
@@ -119,6 +119,11 @@ kvq_status check_tables(const kvq_desc* d, const kvq_tables* tb, int64_t rope_ro
     if (!tb->qL || !tb->codebook) return KVQ_ERR_INVALID;
     if (!aligned(tb->qL, 16) || !aligned(tb->codebook, 4)) return KVQ_ERR_ALIGN;
   }
+  if (d->quant == KVQ_Q_CODEBOOK_DYN) {
+    if (!tb->codebook_wide || !tb->ch_scale || !tb->ch_wide) return KVQ_ERR_INVALID;
+    if (!aligned(tb->codebook_wide, 4) || !aligned(tb->ch_scale, 16) || !aligned(tb->ch_wide, 4))
+      return KVQ_ERR_ALIGN;
+  }
   return KVQ_OK;
 }
 
@@ -132,6 +137,10 @@ kvq_status check_packed(const kvq_desc* d, const kvq_packed* p) {
   if (d->rot == KVQ_ROT_ISO_SO4 || d->rot == KVQ_ROT_ISO_SO3) {
     if (!p->norm) return KVQ_ERR_INVALID;
     if (!aligned(p->norm, 4)) return KVQ_ERR_ALIGN;
+  }
+  if (d->quant == KVQ_Q_CODEBOOK_DYN) {
+    if (!p->ext) return KVQ_ERR_INVALID;
+    if (!aligned(p->ext, 2)) return KVQ_ERR_ALIGN;
   }
   if (d->n_sink > 0) {
     if (!p->sink) return KVQ_ERR_INVALID;
@@ -404,6 +413,30 @@ kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables
   return launch_calibrate(*d, x, *tb, perm_out, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t kvq_calibrate_codebook_workspace_bytes(const kvq_desc* d) {
+  if (check_desc(d) != KVQ_OK || (d->rot != KVQ_ROT_ISO_SO4 && d->rot != KVQ_ROT_ISO_SO3)) return 0;
+  return calibrate_codebook_workspace_bytes(*d);
+}
+
+kvq_status kvq_calibrate_codebook(const kvq_desc* d, const void* x, const kvq_tables* tb, float* ch_scale_out,
+                                  uint32_t* ch_wide_out, void* workspace, size_t workspace_bytes,
+                                  kvq_stream_t stream) {
+  kvq_status s = check_desc(d);
+  if (s != KVQ_OK) return s;
+  if (d->rot != KVQ_ROT_ISO_SO4 && d->rot != KVQ_ROT_ISO_SO3) return KVQ_ERR_UNSUPPORTED;
+  if (!tb || !ch_scale_out || !ch_wide_out || !workspace || (d->tokens > 0 && !x)) return KVQ_ERR_INVALID;
+  if (!tb->qL || (d->rot == KVQ_ROT_ISO_SO4 && !tb->qR)) return KVQ_ERR_INVALID;
+  if ((x && !aligned(x, 16)) || !aligned(tb->qL, 16) || (tb->qR && !aligned(tb->qR, 16)) ||
+      !aligned(ch_scale_out, 16) || !aligned(ch_wide_out, 4) || !aligned(workspace, 256) ||
+      (tb->sink_pos && !aligned(tb->sink_pos, 4)))
+    return KVQ_ERR_ALIGN;
+  if (workspace_bytes < calibrate_codebook_workspace_bytes(*d)) return KVQ_ERR_INVALID;
+  LaunchCtx ctx;
+  if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
+  return launch_calibrate_codebook(*d, x, *tb, ch_scale_out, ch_wide_out, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t kvq_detect_sinks_workspace_bytes(const kvq_desc* d) {
   if (check_desc(d) != KVQ_OK) return 0;
   return detect_sinks_workspace_bytes(*d);
@@ -441,6 +474,8 @@ size_t kvq_packed_bytes(const kvq_desc* d, int32_t field) {
       return static_cast<size_t>(d->batch) * d->heads * d->n_sink * d->head_dim * 2;
     case KVQ_FIELD_NORM:
       return (d->rot == KVQ_ROT_ISO_SO4 || d->rot == KVQ_ROT_ISO_SO3) ? vecs * 4 : 0;
+    case KVQ_FIELD_EXT:
+      return d->quant == KVQ_Q_CODEBOOK_DYN ? vecs * 2 : 0;
     default:
       return 0;
   }
@@ -472,9 +507,9 @@ kvq_status kvq_rope_table_ex(float* cs_host, int32_t t_max, int32_t head_dim, do
 }
 
 kvq_status kvq_lloyd_max_codebook(float* levels_host, int32_t bits, int32_t head_dim) {
-  if (!levels_host || bits < 1 || bits > 4 || head_dim <= 0) return KVQ_ERR_INVALID;
+  if (!levels_host || bits < 1 || bits > 5 || head_dim <= 0) return KVQ_ERR_INVALID;
   const int n = 1 << bits;
-  double lv[16], bd[17];
+  double lv[32], bd[33];
   for (int k = 0; k < n; ++k) lv[k] = -3.0 + 6.0 * (k + 0.5) / n;
   for (int it = 0; it < 200000; ++it) {
     bd[0] = -INFINITY;

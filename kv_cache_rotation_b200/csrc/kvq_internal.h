@@ -55,6 +55,9 @@ size_t calibrate_workspace_bytes(const kvq_desc& d);
 kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& tb, int16_t* perm, void* ws,
                             cudaStream_t st);
 void* attend_scratch();
+size_t calibrate_codebook_workspace_bytes(const kvq_desc& d);
+kvq_status launch_calibrate_codebook(const kvq_desc& d, const void* x, const kvq_tables& tb, float* ch_scale,
+                                     uint32_t* ch_wide, void* ws, cudaStream_t st);
 size_t detect_sinks_workspace_bytes(const kvq_desc& d);
 kvq_status launch_detect_sinks(const kvq_desc& d, const void* x, double tau, int max_sinks, int32_t* sink_pos,
                                int32_t* count, void* ws, cudaStream_t st);

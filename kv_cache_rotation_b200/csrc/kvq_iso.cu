@@ -17,6 +17,18 @@
 // multiplication by its reciprocal. Both reorder fp32 rounding relative to
 // the literal sandwich, so a code can differ by one level where w sits
 // within a few ulps of a decision boundary.
+//
+// Dynamic codebooks (§4.2: per-channel statistics, boundaries set by the KL
+// divergence, twice the codebook for outlier channels): channel j of head h
+// quantizes against the levels fp32(sigma[h][j] * l_k) of the N(0,1)
+// Lloyd-Max design l (2^bits levels, or 2^(bits+1) for the channels marked in
+// ch_wide), with fp32 midpoints as boundaries; the top bit of each outlier
+// channel's code goes to a per-slot 16-bit word. sigma is the square root of
+// the channel's mean square over the calibration tokens, the minimiser of the
+// KL divergence from the channel's values to N(0, sigma^2): k_dyn_stats sums
+// the squares of the rotated values per (sequence, head, 1024-token chunk) in
+// a fixed order, k_dyn_finish adds the chunks in order and marks the outlier
+// channels (sigma > 2 x the lower median, at most D/8).
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -25,16 +37,22 @@ namespace {
 
 struct IsoArgs {
   long long rows;  // B*H*T vectors in this call
-  int T, t0, t_cap, n_sink;
+  int H, T, t0, t_cap, n_sink;
   const float* qL;
   const float* qR;
-  const float* codebook;
+  const float* codebook;  // fixed: the levels; dynamic: the 2^bits N(0,1) levels
+  const float* cb_wide;   // dynamic: the 2^(bits+1) N(0,1) levels
+  const float* ch_scale;  // dynamic: [H][D]
+  const uint32_t* ch_wide;  // dynamic: [H][D/32]
   uint8_t* codes;
   float* norm;
+  uint16_t* ext;  // dynamic: [B][H][t_cap]
   __half* sink;
   uint32_t* err;
   uint64_t wait_ns;
 };
+
+constexpr int kStatChunk = 1024;  // tokens per k_dyn_stats CTA
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
@@ -94,6 +112,88 @@ __device__ __forceinline__ uint32_t cb_code(float w, const float* beta) {
   return c;
 }
 
+// Dynamic codebook: code of w against the levels fp32(s * lv[k]) with fp32
+// midpoints as boundaries (ties to the lower code).
+template <int NL>
+__device__ __forceinline__ uint32_t dyn_code(float w, float s, const float* lv) {
+  uint32_t c = 0;
+#pragma unroll
+  for (int st = NL / 2; st >= 1; st >>= 1) {
+    const float a = __fmul_rn(s, lv[c + st - 1]), b = __fmul_rn(s, lv[c + st]);
+    if (w > __fmul_rn(0.5f, __fadd_rn(a, b))) c += st;
+  }
+  return c;
+}
+
+// The rotated unit vector: w = M_k (x * inv) per block (4-D, or 3-D with its
+// tail), handed to emit(j, w_j) in ascending channel order.
+template <int D, bool SO3, class Emit>
+__device__ __forceinline__ void iso_rotate(const float (&x)[D], float inv, const float* Ms, Emit&& emit) {
+  constexpr int NB = D / 4;
+  constexpr int NB3 = D / 3, TAIL = D % 3;
+  if constexpr (!SO3) {
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+      float u[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) u[e] = __fmul_rn(x[4 * k + e], inv);
+      const float4* Mk = reinterpret_cast<const float4*>(Ms + k * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 row = Mk[i];
+        float wi = __fmul_rn(row.x, u[0]);
+        wi = __fmaf_rn(row.y, u[1], wi);
+        wi = __fmaf_rn(row.z, u[2], wi);
+        wi = __fmaf_rn(row.w, u[3], wi);
+        emit(4 * k + i, wi);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < NB3; ++k) {
+      float u[3];
+#pragma unroll
+      for (int e = 0; e < 3; ++e) u[e] = __fmul_rn(x[3 * k + e], inv);
+      const float* Mk = Ms + k * 9;
+#pragma unroll
+      for (int i = 0; i < 3; ++i) {
+        float wi = __fmul_rn(Mk[3 * i], u[0]);
+        wi = __fmaf_rn(Mk[3 * i + 1], u[1], wi);
+        wi = __fmaf_rn(Mk[3 * i + 2], u[2], wi);
+        emit(3 * k + i, wi);
+      }
+    }
+    if constexpr (TAIL == 2) {  // the tail in its own plane: the matrix's upper-left 2x2 block
+      const float u0 = __fmul_rn(x[D - 2], inv), u1 = __fmul_rn(x[D - 1], inv);
+      const float* Mk = Ms + NB3 * 9;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) emit(D - 2 + i, __fmaf_rn(Mk[3 * i + 1], u1, __fmul_rn(Mk[3 * i], u0)));
+    } else if constexpr (TAIL == 1) {  // a single channel is kept
+      emit(D - 1, __fmul_rn(x[D - 1], inv));
+    }
+  }
+}
+
+// rho = ||x|| from the fp64 sum of squares in channel order (each square is
+// exact in fp64), and the reciprocal of rho + 1e-8.
+template <int D>
+__device__ __forceinline__ float iso_norm(const float (&x)[D], float& inv) {
+  double acc = 0.0;
+#pragma unroll
+  for (int j = 0; j < D; ++j) acc = __fma_rn(static_cast<double>(x[j]), static_cast<double>(x[j]), acc);
+  const float rho = __double2float_rn(__dsqrt_rn(acc));
+  inv = __frcp_rn(__fadd_rn(rho, 1e-8f));
+  return rho;
+}
+
+template <bool SO3>
+__device__ __forceinline__ void build_mats(const IsoArgs& a, float* Ms, int D) {
+  if constexpr (SO3)
+    build_m3(a.qL, Ms, D / 3 + (D % 3 ? 1 : 0));
+  else
+    build_m(a.qL, a.qR, Ms, D / 4);
+}
+
 template <int BITS, int NW>
 __device__ __forceinline__ void put_code(uint32_t (&w)[NW], int j, uint32_t c) {
   const int pos = j * BITS;
@@ -101,17 +201,17 @@ __device__ __forceinline__ void put_code(uint32_t (&w)[NW], int j, uint32_t c) {
   if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= c >> (32 - (pos & 31));
 }
 
-template <int D, int BITS, bool SO3>
+template <int D, int BITS, bool SO3, bool DYN>
 __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUtensorMap xmap, const IsoArgs a) {
   constexpr int NB = D / 4;
-  constexpr int NB3 = D / 3, TAIL = D % 3;  // 3-D sandwich blocks, tail channels
   constexpr int NL = 1 << BITS;
   constexpr int NW = D * BITS / 32;
   constexpr int RB = D * BITS / 8;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar;
   __shared__ __align__(16) float Ms[NB * 16];  // holds the 3x3 matrices too (9 * ceil(D/3) < 4 D)
-  __shared__ float beta[NL];
+  __shared__ float beta[NL];    // fixed: the midpoints; dynamic: the N(0,1) levels
+  __shared__ float lvw[2 * NL];  // dynamic: the wide N(0,1) levels
   uint8_t* xs = align1024(smem_raw);
   const int tid = threadIdx.x;
   const long long r0 = static_cast<long long>(blockIdx.x) * 128;
@@ -126,11 +226,13 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
 #pragma unroll
     for (int hh = 0; hh < D / 64; ++hh) tma_load_2d(xs + hh * 16384, &xmap, hh * 64, static_cast<int>(r0), &bar);
   }
-  if constexpr (SO3)
-    build_m3(a.qL, Ms, NB3 + (TAIL ? 1 : 0));
-  else
-    build_m(a.qL, a.qR, Ms, NB);
-  if (tid < NL - 1) beta[tid] = __fmul_rn(0.5f, __fadd_rn(a.codebook[tid], a.codebook[tid + 1]));
+  build_mats<SO3>(a, Ms, D);
+  if constexpr (DYN) {
+    if (tid < NL) beta[tid] = a.codebook[tid];
+    if (tid < 2 * NL) lvw[tid] = a.cb_wide[tid];
+  } else {
+    if (tid < NL - 1) beta[tid] = __fmul_rn(0.5f, __fadd_rn(a.codebook[tid], a.codebook[tid + 1]));
+  }
   __syncthreads();
   if (!mbar_wait(&bar, 0, a.wait_ns, a.err)) {
     if (tid == 0) mbar_wait(&bar, 0, a.wait_ns, a.err);
@@ -150,63 +252,41 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
 #pragma unroll
     for (int i = 0; i < RB / 8; ++i) reinterpret_cast<uint2*>(a.codes + slot * RB)[i] = make_uint2(0, 0);
     a.norm[slot] = 0.0f;
+    if constexpr (DYN) a.ext[slot] = 0;
     return;
   }
   float x[D];
 #pragma unroll
   for (int c = 0; c < D / 8; ++c) h8_to_f32(lds128(xs_u + (c >> 3) * 16384 + sw128(tid, c & 7)), &x[8 * c]);
-  // rho from the fp64 sum of squares in channel order (each square is exact in fp64)
-  double acc = 0.0;
-#pragma unroll
-  for (int j = 0; j < D; ++j) acc = __fma_rn(static_cast<double>(x[j]), static_cast<double>(x[j]), acc);
-  const float rho = __double2float_rn(__dsqrt_rn(acc));
-  const float inv = __frcp_rn(__fadd_rn(rho, 1e-8f));
+  float inv;
+  const float rho = iso_norm<D>(x, inv);
   uint32_t w[NW];
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
-  if constexpr (!SO3) {
-#pragma unroll
-    for (int k = 0; k < NB; ++k) {
-      float u[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) u[e] = __fmul_rn(x[4 * k + e], inv);
-      const float4* Mk = reinterpret_cast<const float4*>(Ms + k * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 row = Mk[i];
-        float wi = __fmul_rn(row.x, u[0]);
-        wi = __fmaf_rn(row.y, u[1], wi);
-        wi = __fmaf_rn(row.z, u[2], wi);
-        wi = __fmaf_rn(row.w, u[3], wi);
-        put_code<BITS, NW>(w, 4 * k + i, cb_code<NL>(wi, beta));
-      }
-    }
+  if constexpr (!DYN) {
+    iso_rotate<D, SO3>(x, inv, Ms, [&](int j, float wj) { put_code<BITS, NW>(w, j, cb_code<NL>(wj, beta)); });
   } else {
+    const int h = static_cast<int>(bh % a.H);
+    const float* sc = a.ch_scale + static_cast<size_t>(h) * D;
+    uint32_t wd[D / 32];
 #pragma unroll
-    for (int k = 0; k < NB3; ++k) {
-      float u[3];
-#pragma unroll
-      for (int e = 0; e < 3; ++e) u[e] = __fmul_rn(x[3 * k + e], inv);
-      const float* Mk = Ms + k * 9;
-#pragma unroll
-      for (int i = 0; i < 3; ++i) {
-        float wi = __fmul_rn(Mk[3 * i], u[0]);
-        wi = __fmaf_rn(Mk[3 * i + 1], u[1], wi);
-        wi = __fmaf_rn(Mk[3 * i + 2], u[2], wi);
-        put_code<BITS, NW>(w, 3 * k + i, cb_code<NL>(wi, beta));
+    for (int i = 0; i < D / 32; ++i) wd[i] = __ldg(a.ch_wide + static_cast<size_t>(h) * (D / 32) + i);
+    uint32_t ext = 0;
+    int nw = 0;
+    iso_rotate<D, SO3>(x, inv, Ms, [&](int j, float wj) {
+      const float sj = __ldg(sc + j);
+      uint32_t c;
+      if ((wd[j >> 5] >> (j & 31)) & 1u) {
+        c = dyn_code<2 * NL>(wj, sj, lvw);
+        if (nw < 16) ext |= (c >> BITS) << nw;
+        ++nw;
+        c &= NL - 1;
+      } else {
+        c = dyn_code<NL>(wj, sj, beta);
       }
-    }
-    if constexpr (TAIL == 2) {  // the tail in its own plane: the matrix's upper-left 2x2 block
-      const float u0 = __fmul_rn(x[D - 2], inv), u1 = __fmul_rn(x[D - 1], inv);
-      const float* Mk = Ms + NB3 * 9;
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const float wi = __fmaf_rn(Mk[3 * i + 1], u1, __fmul_rn(Mk[3 * i], u0));
-        put_code<BITS, NW>(w, D - 2 + i, cb_code<NL>(wi, beta));
-      }
-    } else if constexpr (TAIL == 1) {  // a single channel is kept
-      put_code<BITS, NW>(w, D - 1, cb_code<NL>(__fmul_rn(x[D - 1], inv), beta));
-    }
+      put_code<BITS, NW>(w, j, c);
+    });
+    a.ext[slot] = static_cast<uint16_t>(ext);
   }
   uint8_t* dst = a.codes + slot * RB;
   if constexpr (RB % 16 == 0) {
@@ -220,7 +300,7 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
   a.norm[slot] = rho;
 }
 
-template <int D, int BITS, bool SO3>
+template <int D, int BITS, bool SO3, bool DYN>
 __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUtensorMap omap, const IsoArgs a,
                                                      int out_fp32) {
   constexpr int NB = D / 4;
@@ -231,14 +311,14 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(16) float Ms[NB * 16];
   __shared__ float lv[NL];
+  __shared__ float lvw[2 * NL];  // dynamic: the wide N(0,1) levels
   uint8_t* os = align1024(smem_raw);
   const int tid = threadIdx.x;
   const long long r0 = static_cast<long long>(blockIdx.x) * 128;
-  if constexpr (SO3)
-    build_m3(a.qL, Ms, NB3 + (TAIL ? 1 : 0));
-  else
-    build_m(a.qL, a.qR, Ms, NB);
+  build_mats<SO3>(a, Ms, D);
   if (tid < NL) lv[tid] = a.codebook[tid];
+  if constexpr (DYN)
+    if (tid < 2 * NL) lvw[tid] = a.cb_wide[tid];
   __syncthreads();
   const long long vid = r0 + tid;
   float x[D];
@@ -268,12 +348,37 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
         }
       }
       const float rho = a.norm[slot];
+      // level of channel j (called in ascending channel order)
+      const float* sc = nullptr;
+      uint32_t wd[D / 32], ext = 0;
+      int nw = 0;
+      if constexpr (DYN) {
+        const int h = static_cast<int>(bh % a.H);
+        sc = a.ch_scale + static_cast<size_t>(h) * D;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) wd[i] = __ldg(a.ch_wide + static_cast<size_t>(h) * (D / 32) + i);
+        ext = a.ext[slot];
+      }
+      auto level = [&](int j) -> float {
+        uint32_t c = unpack_code<BITS, NW>(w, j);
+        if constexpr (!DYN) {
+          return lv[c];
+        } else {
+          const float sj = __ldg(sc + j);
+          if ((wd[j >> 5] >> (j & 31)) & 1u) {
+            if (nw < 16) c |= ((ext >> nw) & 1u) << BITS;
+            ++nw;
+            return __fmul_rn(sj, lvw[c]);
+          }
+          return __fmul_rn(sj, lv[c]);
+        }
+      };
       if constexpr (!SO3) {
 #pragma unroll
         for (int k = 0; k < NB; ++k) {
           float wh[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) wh[e] = lv[unpack_code<BITS, NW>(w, 4 * k + e)];
+          for (int e = 0; e < 4; ++e) wh[e] = level(4 * k + e);
           const float* Mk = Ms + k * 16;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {  // v = M^T w
@@ -289,7 +394,7 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
         for (int k = 0; k < NB3; ++k) {
           float wh[3];
 #pragma unroll
-          for (int e = 0; e < 3; ++e) wh[e] = lv[unpack_code<BITS, NW>(w, 3 * k + e)];
+          for (int e = 0; e < 3; ++e) wh[e] = level(3 * k + e);
           const float* Mk = Ms + k * 9;
 #pragma unroll
           for (int i = 0; i < 3; ++i) {  // v = M^T w
@@ -300,13 +405,14 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
           }
         }
         if constexpr (TAIL == 2) {
-          const float w0 = lv[unpack_code<BITS, NW>(w, D - 2)], w1 = lv[unpack_code<BITS, NW>(w, D - 1)];
+          const float w0 = level(D - 2);
+          const float w1 = level(D - 1);
           const float* Mk = Ms + NB3 * 9;
 #pragma unroll
           for (int i = 0; i < 2; ++i)
             x[D - 2 + i] = __fmul_rn(__fmaf_rn(Mk[3 + i], w1, __fmul_rn(Mk[i], w0)), rho);
         } else if constexpr (TAIL == 1) {
-          x[D - 1] = __fmul_rn(lv[unpack_code<BITS, NW>(w, D - 1)], rho);
+          x[D - 1] = __fmul_rn(level(D - 1), rho);
         }
       }
     }
@@ -333,9 +439,111 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
   }
 }
 
+// ------------------------------------------------------- dynamic statistics
+struct DynStatArgs {
+  int H, T, t0, n_sink, nchunk;
+  const __half* x;
+  const int32_t* sink_pos;  // [B][n_sink] or nullptr (positions < n_sink)
+  const float* qL;
+  const float* qR;
+  double* part;  // [B*H][nchunk][D] sums of squares
+  int* cnt;      // [B*H][nchunk] vectors counted
+};
+
+// Sum over the CTA's tokens of w_j^2 (fp64, token order) for every channel:
+// the rotated rows go through shared memory (pitch D + 1 words, so the row
+// writes and the column reads are both conflict-free); thread j adds column j.
+template <int D, bool SO3>
+__global__ void __launch_bounds__(128) k_dyn_stats(const DynStatArgs a) {
+  extern __shared__ float wsm[];  // [128][D + 1]
+  __shared__ __align__(16) float Ms[D * 4];
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.y, b = bh / a.H;
+  IsoArgs ia{};
+  ia.qL = a.qL;
+  ia.qR = a.qR;
+  build_mats<SO3>(ia, Ms, D);
+  __syncthreads();
+  const int tbeg = blockIdx.x * kStatChunk;
+  const int tend = min(tbeg + kStatChunk, a.T);
+  double acc = 0.0;
+  int cnt = 0;
+  for (int tc = tbeg; tc < tend; tc += 128) {  // the same trip count for every thread
+    const int t = tc + tid;
+    bool live = t < tend;
+    if (live) {
+      const int pos = a.t0 + t;
+      if (!a.sink_pos) {
+        live = pos >= a.n_sink;
+      } else {
+        for (int k = 0; k < a.n_sink; ++k) live &= __ldg(a.sink_pos + static_cast<size_t>(b) * a.n_sink + k) != pos;
+      }
+    }
+    float* row = wsm + tid * (D + 1);
+    if (live) {
+      float x[D];
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + (static_cast<size_t>(bh) * a.T + t) * D);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) h8_to_f32(__ldg(src + c), &x[8 * c]);
+      float inv;
+      (void)iso_norm<D>(x, inv);
+      iso_rotate<D, SO3>(x, inv, Ms, [&](int j, float wj) { row[j] = wj; });
+    } else {
+#pragma unroll 8
+      for (int j = 0; j < D; ++j) row[j] = 0.0f;
+    }
+    cnt += __syncthreads_count(live);
+    if (tid < D)
+      for (int r = 0; r < 128; ++r) {
+        const double v = static_cast<double>(wsm[r * (D + 1) + tid]);
+        acc = __fma_rn(v, v, acc);
+      }
+    __syncthreads();
+  }
+  const size_t pr = static_cast<size_t>(bh) * a.nchunk + blockIdx.x;
+  if (tid < D) a.part[pr * D + tid] = acc;
+  if (tid == 0) a.cnt[pr] = cnt;
+}
+
+// One CTA of D threads per head: the chunk sums in order, sigma, the lower
+// median of the head's sigmas, and the outlier mask (sigma > 2 x median, the
+// D/8 largest at most, equal sigmas to the lower channel).
+template <int D>
+__global__ void __launch_bounds__(D) k_dyn_finish(int B, int H, int nchunk, const double* part, const int* cnt,
+                                                  float* ch_scale, uint32_t* ch_wide) {
+  __shared__ float sg[D];
+  __shared__ float med;
+  const int h = blockIdx.x, j = threadIdx.x;
+  double s = 0.0;
+  long long n = 0;
+  for (int b = 0; b < B; ++b)
+    for (int c = 0; c < nchunk; ++c) {
+      const size_t r = (static_cast<size_t>(b) * H + h) * nchunk + c;
+      s = __dadd_rn(s, part[r * D + j]);
+      n += cnt[r];
+    }
+  const float sigma = n > 0 ? __double2float_rn(__dsqrt_rn(__ddiv_rn(s, static_cast<double>(n))))
+                            : __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(static_cast<double>(D))));
+  sg[j] = sigma;
+  __syncthreads();
+  int below = 0, above = 0;
+  for (int k = 0; k < D; ++k) {
+    const float v = sg[k];
+    below += v < sigma || (v == sigma && k < j);
+    above += v > sigma || (v == sigma && k < j);
+  }
+  if (below == (D - 1) / 2) med = sigma;
+  __syncthreads();
+  const bool wide = sigma > __fmul_rn(2.0f, med) && above < D / 8;
+  const uint32_t word = __ballot_sync(0xffffffffu, wide);
+  ch_scale[static_cast<size_t>(h) * D + j] = sigma;
+  if ((j & 31) == 0) ch_wide[static_cast<size_t>(h) * (D / 32) + (j >> 5)] = word;
+}
+
 IsoArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p, const LaunchCtx& ctx) {
   IsoArgs a{};
   a.rows = static_cast<long long>(d.batch) * d.heads * d.tokens;
+  a.H = d.heads;
   a.T = d.tokens;
   a.t0 = d.t0;
   a.t_cap = d.t_cap;
@@ -343,26 +551,30 @@ IsoArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p, 
   a.qL = tb.qL;
   a.qR = tb.qR;
   a.codebook = tb.codebook;
+  a.cb_wide = tb.codebook_wide;
+  a.ch_scale = tb.ch_scale;
+  a.ch_wide = tb.ch_wide;
   a.codes = p.codes;
   a.norm = p.norm;
+  a.ext = p.ext;
   a.sink = static_cast<__half*>(p.sink);
   a.err = ctx.err;
   a.wait_ns = ctx.wait_ns;
   return a;
 }
 
-template <int D, int BITS, bool SO3>
+template <int D, int BITS, bool SO3, bool DYN>
 kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((a.rows + 127) / 128);
   if (enc) {
     const size_t smem = 1024 + D * 256;
-    auto k = k_encode_iso<D, BITS, SO3>;
+    auto k = k_encode_iso<D, BITS, SO3, DYN>;
     if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
     k<<<grid, 128, smem, st>>>(m0, a);
   } else {
     const size_t smem = 1024 + D * 512;
-    auto k = k_decode_iso<D, BITS, SO3>;
+    auto k = k_decode_iso<D, BITS, SO3, DYN>;
     if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
     k<<<grid, 128, smem, st>>>(m0, a, out_fp32);
@@ -372,10 +584,14 @@ kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, 
 
 kvq_status dispatch(bool enc, const kvq_desc& d, const IsoArgs& a, const CUtensorMap& m0, int out_fp32,
                     cudaStream_t st) {
-#define KVQ_CASE(D_, B_)                                                                  \
-  if (d.head_dim == D_ && d.bits == B_)                                                   \
-    return d.rot == KVQ_ROT_ISO_SO3 ? run<D_, B_, true>(enc, a, m0, out_fp32, st)         \
-                                    : run<D_, B_, false>(enc, a, m0, out_fp32, st);
+#define KVQ_CASE(D_, B_)                                                                              \
+  if (d.head_dim == D_ && d.bits == B_) {                                                             \
+    if (d.quant == KVQ_Q_CODEBOOK_DYN)                                                                \
+      return d.rot == KVQ_ROT_ISO_SO3 ? run<D_, B_, true, true>(enc, a, m0, out_fp32, st)             \
+                                      : run<D_, B_, false, true>(enc, a, m0, out_fp32, st);           \
+    return d.rot == KVQ_ROT_ISO_SO3 ? run<D_, B_, true, false>(enc, a, m0, out_fp32, st)              \
+                                    : run<D_, B_, false, false>(enc, a, m0, out_fp32, st);            \
+  }
   KVQ_CASE(128, 2)
   KVQ_CASE(128, 3)
   KVQ_CASE(128, 4)
@@ -414,6 +630,47 @@ kvq_status launch_decode_iso(const kvq_desc& d, const kvq_packed& in, const kvq_
                 strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
     return KVQ_ERR_CUDA;
   return dispatch(false, d, a, om, out_fp32, st);
+}
+
+size_t dyn_stats_chunks(const kvq_desc& d) {
+  return d.tokens > 0 ? (static_cast<size_t>(d.tokens) + kStatChunk - 1) / kStatChunk : 1;
+}
+
+size_t calibrate_codebook_workspace_bytes(const kvq_desc& d) {
+  const size_t rows = static_cast<size_t>(d.batch) * d.heads * dyn_stats_chunks(d);
+  return rows * d.head_dim * 8 + ((rows * 4 + 255) & ~size_t(255));
+}
+
+kvq_status launch_calibrate_codebook(const kvq_desc& d, const void* x, const kvq_tables& tb, float* ch_scale,
+                                     uint32_t* ch_wide, void* ws, cudaStream_t st) {
+  const size_t nchunk = dyn_stats_chunks(d);
+  const size_t rows = static_cast<size_t>(d.batch) * d.heads * nchunk;
+  if (static_cast<size_t>(d.batch) * d.heads > 65535 || nchunk > 0x7fffffff) return KVQ_ERR_UNSUPPORTED;
+  DynStatArgs a{};
+  a.H = d.heads;
+  a.T = d.tokens;
+  a.t0 = d.t0;
+  a.n_sink = d.n_sink;
+  a.nchunk = static_cast<int>(nchunk);
+  a.x = static_cast<const __half*>(x);
+  a.sink_pos = tb.sink_pos;
+  a.qL = tb.qL;
+  a.qR = tb.qR;
+  a.part = static_cast<double*>(ws);
+  a.cnt = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + rows * d.head_dim * 8);
+  const dim3 grid(static_cast<unsigned>(nchunk), static_cast<unsigned>(d.batch * d.heads));
+  const bool so3 = d.rot == KVQ_ROT_ISO_SO3;
+  auto go = [&](auto kstats, auto kfin, int D) -> kvq_status {
+    const size_t smem = static_cast<size_t>(128) * (D + 1) * 4;
+    if (!set_smem_once(reinterpret_cast<const void*>(kstats), smem)) return KVQ_ERR_CUDA;
+    kstats<<<grid, 128, smem, st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    kfin<<<d.heads, D, 0, st>>>(d.batch, d.heads, a.nchunk, a.part, a.cnt, ch_scale, ch_wide);
+    return launch_status();
+  };
+  if (d.head_dim == 128)
+    return so3 ? go(k_dyn_stats<128, true>, k_dyn_finish<128>, 128) : go(k_dyn_stats<128, false>, k_dyn_finish<128>, 128);
+  return so3 ? go(k_dyn_stats<64, true>, k_dyn_finish<64>, 64) : go(k_dyn_stats<64, false>, k_dyn_finish<64>, 64);
 }
 
 }  // namespace kvq

@@ -206,6 +206,7 @@ struct FixArgs {
   uint8_t* codes;
   uint32_t* sz;  // scale/zero words of a record
   float* norm;
+  uint16_t* ext;  // dynamic codebooks: the outlier channels' top bits
   __half* sink;
   void* out;      // decode output
   float* scores;  // [B][Hq][n_tok]
@@ -229,6 +230,7 @@ __global__ void k_sink_fix_encode(const FixArgs a) {
   if (a.sz)
     for (int i = lane; i < a.sz_words; i += 32) a.sz[slot * a.sz_words + i] = 0u;
   if (a.norm && lane == 0) a.norm[slot] = 0.0f;
+  if (a.ext && lane == 0) a.ext[slot] = 0;
 }
 
 // Decode: the listed positions of this call decode to their fp16 rows.
@@ -301,6 +303,7 @@ FixArgs fix_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p) {
     a.sz_words = d.head_dim / d.group;  // one (scale, zero) half pair per group
   }
   if (d.rot == KVQ_ROT_ISO_SO4 || d.rot == KVQ_ROT_ISO_SO3) a.norm = p.norm;
+  if (d.quant == KVQ_Q_CODEBOOK_DYN) a.ext = p.ext;
   a.sink = static_cast<__half*>(p.sink);
   return a;
 }

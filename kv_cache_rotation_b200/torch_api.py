@@ -13,15 +13,15 @@ from typing import Optional
 
 import torch
 
-from . import (KVQ_FIELD_CODES, KVQ_FIELD_NORM, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_Q_CODEBOOK,
-               KVQ_Q_MINMAX, KVQ_ROT_FWHT_GROUP, KVQ_ROT_FWHT_HEAD, KVQ_ROT_ISO_SO3, KVQ_ROT_ISO_SO4, KVQ_ROT_NONE,
+from . import (KVQ_FIELD_CODES, KVQ_FIELD_EXT, KVQ_FIELD_NORM, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK,
+               KVQ_Q_CODEBOOK, KVQ_Q_CODEBOOK_DYN, KVQ_Q_MINMAX, KVQ_ROT_FWHT_GROUP, KVQ_ROT_FWHT_HEAD, KVQ_ROT_ISO_SO3, KVQ_ROT_ISO_SO4, KVQ_ROT_NONE,
                check,
                kvq_decode, kvq_desc, kvq_encode, kvq_lloyd_max_codebook, kvq_packed, kvq_packed_bytes,
                kvq_rope_table, kvq_score, kvq_tables)
 
 ROT = {"none": KVQ_ROT_NONE, "fwht_head": KVQ_ROT_FWHT_HEAD, "fwht_group": KVQ_ROT_FWHT_GROUP,
        "iso": KVQ_ROT_ISO_SO4, "iso3": KVQ_ROT_ISO_SO3}
-QUANT = {"minmax": KVQ_Q_MINMAX, "codebook": KVQ_Q_CODEBOOK}
+QUANT = {"minmax": KVQ_Q_MINMAX, "codebook": KVQ_Q_CODEBOOK, "codebook_dyn": KVQ_Q_CODEBOOK_DYN}
 
 
 def make_desc(*, batch, heads, head_dim=128, tokens, t0=0, t_cap=None, bits, group=128, group_heads=1, rope=0,
@@ -41,6 +41,7 @@ class Packed:
     scale_zero: Optional[torch.Tensor]
     sink: Optional[torch.Tensor]
     norm: Optional[torch.Tensor]
+    ext: Optional[torch.Tensor] = None
 
     def struct(self) -> kvq_packed:
         p = kvq_packed()
@@ -48,11 +49,12 @@ class Packed:
         p.scale_zero = self.scale_zero.data_ptr() if self.scale_zero is not None else None
         p.sink = self.sink.data_ptr() if self.sink is not None else None
         p.norm = self.norm.data_ptr() if self.norm is not None else None
+        p.ext = self.ext.data_ptr() if self.ext is not None else None
         return p
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in (self.codes, self.scale_zero, self.sink, self.norm)
-                   if t is not None)
+        return sum(t.numel() * t.element_size()
+                   for t in (self.codes, self.scale_zero, self.sink, self.norm, self.ext) if t is not None)
 
 
 def alloc_packed(d: kvq_desc, device="cuda", zero=True) -> Packed:
@@ -72,7 +74,8 @@ def alloc_packed(d: kvq_desc, device="cuda", zero=True) -> Packed:
     sz = buf(KVQ_FIELD_SCALE_ZERO, torch.int16, (B, H, C, ng, 2)) if ng else None
     sink = buf(KVQ_FIELD_SINK, torch.float16, (B, H, d.n_sink, D)) if d.n_sink else None
     norm = buf(KVQ_FIELD_NORM, torch.float32, (B, H, C))
-    return Packed(codes, sz, sink, norm)
+    ext = buf(KVQ_FIELD_EXT, torch.int16, (B, H, C))
+    return Packed(codes, sz, sink, norm, ext)
 
 
 def rope_table(t_max: int, head_dim: int, device="cuda", base: float = 10000.0, freq: int = 0) -> torch.Tensor:
@@ -99,6 +102,9 @@ class Tables:
     qR: Optional[torch.Tensor] = None
     codebook: Optional[torch.Tensor] = None
     sink_pos: Optional[torch.Tensor] = None  # int32 [B][n_sink]: the list form of the sink set
+    codebook_wide: Optional[torch.Tensor] = None  # dynamic codebooks: the (bits+1)-bit N(0,1) levels
+    ch_scale: Optional[torch.Tensor] = None  # dynamic codebooks: f32 [H][D]
+    ch_wide: Optional[torch.Tensor] = None  # dynamic codebooks: int32 [H][D/32] outlier-channel masks
 
     def struct(self) -> kvq_tables:
         tb = kvq_tables()
@@ -111,11 +117,15 @@ class Tables:
         if self.sink_pos is not None:
             _req(self.sink_pos, "sink_pos", (torch.int32,))
             tb.sink_pos = self.sink_pos.data_ptr()
+        tb.codebook_wide = self.codebook_wide.data_ptr() if self.codebook_wide is not None else None
+        tb.ch_scale = self.ch_scale.data_ptr() if self.ch_scale is not None else None
+        tb.ch_wide = self.ch_wide.data_ptr() if self.ch_wide is not None else None
         return tb
 
 
-def make_tables(perm=None, rope_cs=None, qL=None, qR=None, codebook=None, sink_pos=None) -> Tables:
-    return Tables(perm, rope_cs, qL, qR, codebook, sink_pos)
+def make_tables(perm=None, rope_cs=None, qL=None, qR=None, codebook=None, sink_pos=None, codebook_wide=None,
+                ch_scale=None, ch_wide=None) -> Tables:
+    return Tables(perm, rope_cs, qL, qR, codebook, sink_pos, codebook_wide, ch_scale, ch_wide)
 
 
 def _req(t: torch.Tensor, name: str, dtypes, shape=None) -> None:
@@ -221,6 +231,28 @@ def calibrate_perm(d: kvq_desc, x: torch.Tensor, tb: Tables, perm_out: torch.Ten
     check(kvq_calibrate_perm(d, x.data_ptr(), tb.struct(), perm_out.data_ptr(), workspace.data_ptr(),
                              workspace.numel(), _stream(stream)), "kvq_calibrate_perm")
     return perm_out
+
+
+def calibrate_codebook(d: kvq_desc, x: torch.Tensor, tb: Tables, ch_scale: torch.Tensor = None,
+                       ch_wide: torch.Tensor = None, workspace: torch.Tensor = None, stream=None):
+    """Dynamic codebook tables (ch_scale f32 [H][D], ch_wide int32 [H][D/32] bit masks) for
+    Tables.ch_scale / Tables.ch_wide."""
+    from . import kvq_calibrate_codebook, kvq_calibrate_codebook_workspace_bytes
+    _req(x, "x", (torch.float16,), _kv_shape(d))
+    if ch_scale is None:
+        ch_scale = torch.empty((d.heads, d.head_dim), dtype=torch.float32, device=x.device)
+    if ch_wide is None:
+        ch_wide = torch.empty((d.heads, d.head_dim // 32), dtype=torch.int32, device=x.device)
+    if workspace is None:
+        nb = kvq_calibrate_codebook_workspace_bytes(d)
+        if nb == 0:
+            raise ValueError("kvq_calibrate_codebook: invalid or unsupported descriptor")
+        workspace = torch.empty(nb, dtype=torch.uint8, device=x.device)
+    _req(ch_scale, "ch_scale", (torch.float32,), (d.heads, d.head_dim))
+    _req(ch_wide, "ch_wide", (torch.int32,), (d.heads, d.head_dim // 32))
+    check(kvq_calibrate_codebook(d, x.data_ptr(), tb.struct(), ch_scale.data_ptr(), ch_wide.data_ptr(),
+                                 workspace.data_ptr(), workspace.numel(), _stream(stream)), "kvq_calibrate_codebook")
+    return ch_scale, ch_wide
 
 
 def detect_sinks_workspace(d: kvq_desc, device="cuda") -> torch.Tensor:

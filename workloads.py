@@ -73,6 +73,11 @@ WORKLOADS = {
     # 2-channel tail turned in its plane).
     "isoquant_so3_batch": Workload("isoquant_so3_batch", B=8192, H=1, T=2048, rot="iso3", quant="codebook",
                                    bits=3, rope_k=False, dist="student_t", seed=4),
+    # The IsoQuant batch with dynamic codebooks, on keys with outlier
+    # channels (3 % of the channels scaled by U[10, 50], the channel-wise
+    # outliers the per-channel statistics are for): 3-bit, SO(4) blocks.
+    "isoquant_dyn_batch": Workload("isoquant_dyn_batch", B=8192, H=1, T=2048, rot="iso", quant="codebook_dyn",
+                                   bits=3, rope_k=False, outliers=("pairs", 0.03, 10.0, 50.0), seed=5),
     # Decode step: batch 64, 32 heads, 8192-token 2-bit cache encoded as in
     # the Llama-2-7B workload, plus one appended token; fp32 scores.
     "decode_score": Workload("decode_score", B=64, H=32, T=8192, bits=2, group=64, n_sink=4, perm=True,
