@@ -76,3 +76,17 @@ def test_calibration_and_energy_repeat(TA):
     assert torch.equal(p1, p2)
     (e1, e2) = _twice(lambda: tuple(t.cpu() for t in TA.pair_energy(d, x)))
     assert np.array_equal(e1[0].numpy(), e2[0].numpy()) and torch.equal(e1[1], e2[1])
+
+
+def test_sink_detection_and_dynamic_tables_repeat(TA):
+    w = W.Workload("det_sinks", B=3, H=4, T=2500, D=128, outliers=("pairs", 0.03, 10.0, 50.0))
+    xn = W.kv_tensor(w, "k")
+    W.plant_massive(xn, 5, 2)
+    x = torch.from_numpy(xn).cuda()
+    d = TA.make_desc(batch=3, heads=4, head_dim=128, tokens=2500, bits=3, rot="iso", quant="codebook_dyn")
+    (s1, s2) = _twice(lambda: tuple(t.clone() for t in TA.detect_sinks(d, x, tau=4.0, max_sinks=16)))
+    assert torch.equal(s1[0], s2[0]) and torch.equal(s1[1], s2[1])
+    qL, qR = W.unit_quaternions(32, 1, 30), W.unit_quaternions(32, 1, 31)
+    tb = TA.make_tables(qL=torch.from_numpy(qL).cuda(), qR=torch.from_numpy(qR).cuda())
+    (c1, c2) = _twice(lambda: tuple(t.clone() for t in TA.calibrate_codebook(d, x, tb)))
+    assert torch.equal(c1[0], c2[0]) and torch.equal(c1[1], c2[1])

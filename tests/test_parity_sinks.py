@@ -258,8 +258,16 @@ def test_list_score(K, orc, case):
     from kv_cache_rotation_b200 import torch_api as TA
     name, rot, B, H, GQ, T, rope, hg, group = case
     D, bits, n_sink, scale = 128, 2, 4, 0.0884
-    x = _x(B, H, T, D, len(name), planted=3)
-    sp = _lists(B, n_sink, 0, T, 7)
+    # the tokens with massive activations are the sinks (the method keeps them
+    # in fp16), plus one more listed position in even sequences
+    x = _x(B, H, T, D, len(name), planted=0)
+    planted = W.plant_massive(x, 3, len(name))
+    rng = np.random.default_rng(7)
+    sp = np.full((B, n_sink), -1, np.int32)
+    for b in range(B):
+        extra = [] if b % 2 else [int(rng.choice([t for t in range(T) if t not in planted[b]]))]
+        lst = sorted(planted[b] + extra)
+        sp[b, :len(lst)] = lst
     d = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, t_cap=T, bits=bits, group=group, group_heads=hg,
                      rope=rope, n_sink=n_sink, rot=rot)
     tb = TA.make_tables(rope_cs=TA.rope_table(T, D) if rope else None, sink_pos=torch.from_numpy(sp).cuda())
@@ -309,8 +317,12 @@ def test_list_attend_unsupported(K):
     kp, vp = TA.alloc_packed(dk), TA.alloc_packed(dv)
     q = torch.zeros((B, H, D), dtype=torch.float16, device="cuda")
     out = torch.empty((B, H, D), dtype=torch.float32, device="cuda")
+    ws = TA.attend_workspace(dk, dv, H, T)
     with pytest.raises(K.KvqError) as e:
-        TA.attend(dk, dv, q, kp, tk, vp, tv, T, 0.1, out)
+        TA.attend(dk, dv, q, kp, tk, vp, tv, T, 0.1, out, ws)
+    assert e.value.status == K.KVQ_ERR_UNSUPPORTED
+    with pytest.raises(K.KvqError) as e:
+        TA.attend_noalloc(dk, dv, q, kp, tk, vp, tv, T, 0.1, out)
     assert e.value.status == K.KVQ_ERR_UNSUPPORTED
 
 
