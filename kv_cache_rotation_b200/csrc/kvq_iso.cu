@@ -186,6 +186,38 @@ __device__ __forceinline__ float iso_norm(const float (&x)[D], float& inv) {
   return rho;
 }
 
+// Dynamic codebooks: the head shared by all of this CTA's vectors (rows r0 ..
+// r0 + 127, ordered (batch, head, token)), or -1 when they span two heads.
+__device__ __forceinline__ int cta_head(const IsoArgs& a, long long r0) {
+  const long long last = min(r0 + 127, a.rows - 1);
+  const long long bh0 = r0 / a.T, bh1 = last / a.T;
+  return (a.H == 1 || bh0 == bh1) ? static_cast<int>(bh0 % a.H) : -1;
+}
+
+// Per-channel tables of head h in shared memory, row pitch 2 NL floats:
+// encode (LEVELS = false) the boundaries fp32(0.5 (L_k + L_k+1)), decode
+// (LEVELS = true) the levels L_k = fp32(sigma_j l_k) -- the same fp32 values
+// dyn_code and the decode's level() form one by one.
+template <int D, int NL, bool LEVELS>
+__device__ __forceinline__ void dyn_tables(const IsoArgs& a, int h, const float* lv, const float* lvw, float* tab) {
+  const float* sc = a.ch_scale + static_cast<size_t>(h) * D;
+  const uint32_t* wd = a.ch_wide + static_cast<size_t>(h) * (D / 32);
+  for (int e = threadIdx.x; e < D * 2 * NL; e += blockDim.x) {
+    const int j = e / (2 * NL), k = e % (2 * NL);
+    const bool wide = (__ldg(wd + (j >> 5)) >> (j & 31)) & 1u;
+    const int n = wide ? 2 * NL : NL;
+    const float* l = wide ? lvw : lv;
+    const float sj = __ldg(sc + j);
+    float v = 0.0f;
+    if (LEVELS) {
+      if (k < n) v = __fmul_rn(sj, l[k]);
+    } else if (k + 1 < n) {
+      v = __fmul_rn(0.5f, __fadd_rn(__fmul_rn(sj, l[k]), __fmul_rn(sj, l[k + 1])));
+    }
+    tab[e] = v;
+  }
+}
+
 template <bool SO3>
 __device__ __forceinline__ void build_mats(const IsoArgs& a, float* Ms, int D) {
   if constexpr (SO3)
@@ -227,9 +259,14 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
     for (int hh = 0; hh < D / 64; ++hh) tma_load_2d(xs + hh * 16384, &xmap, hh * 64, static_cast<int>(r0), &bar);
   }
   build_mats<SO3>(a, Ms, D);
+  int hc = -1;  // dynamic codebooks: the CTA's head when its channel tables are in shared memory
+  float* tab = reinterpret_cast<float*>(xs + D * 256);
   if constexpr (DYN) {
     if (tid < NL) beta[tid] = a.codebook[tid];
     if (tid < 2 * NL) lvw[tid] = a.cb_wide[tid];
+    hc = cta_head(a, r0);
+    __syncthreads();
+    if (hc >= 0) dyn_tables<D, NL, false>(a, hc, beta, lvw, tab);
   } else {
     if (tid < NL - 1) beta[tid] = __fmul_rn(0.5f, __fadd_rn(a.codebook[tid], a.codebook[tid + 1]));
   }
@@ -274,15 +311,18 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
     uint32_t ext = 0;
     int nw = 0;
     iso_rotate<D, SO3>(x, inv, Ms, [&](int j, float wj) {
-      const float sj = __ldg(sc + j);
       uint32_t c;
-      if ((wd[j >> 5] >> (j & 31)) & 1u) {
-        c = dyn_code<2 * NL>(wj, sj, lvw);
+      const bool wide = (wd[j >> 5] >> (j & 31)) & 1u;
+      if (hc >= 0) {  // the channel's boundaries from shared memory
+        c = wide ? cb_code<2 * NL>(wj, tab + j * 2 * NL) : cb_code<NL>(wj, tab + j * 2 * NL);
+      } else {
+        const float sj = __ldg(sc + j);
+        c = wide ? dyn_code<2 * NL>(wj, sj, lvw) : dyn_code<NL>(wj, sj, beta);
+      }
+      if (wide) {
         if (nw < 16) ext |= (c >> BITS) << nw;
         ++nw;
         c &= NL - 1;
-      } else {
-        c = dyn_code<NL>(wj, sj, beta);
       }
       put_code<BITS, NW>(w, j, c);
     });
@@ -317,8 +357,14 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
   const long long r0 = static_cast<long long>(blockIdx.x) * 128;
   build_mats<SO3>(a, Ms, D);
   if (tid < NL) lv[tid] = a.codebook[tid];
-  if constexpr (DYN)
+  int hc = -1;  // dynamic codebooks: the CTA's head when its channel levels are in shared memory
+  float* tab = reinterpret_cast<float*>(os + D * 512);
+  if constexpr (DYN) {
     if (tid < 2 * NL) lvw[tid] = a.cb_wide[tid];
+    hc = cta_head(a, r0);
+    __syncthreads();
+    if (hc >= 0) dyn_tables<D, NL, true>(a, hc, lv, lvw, tab);
+  }
   __syncthreads();
   const long long vid = r0 + tid;
   float x[D];
@@ -364,13 +410,14 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
         if constexpr (!DYN) {
           return lv[c];
         } else {
-          const float sj = __ldg(sc + j);
-          if ((wd[j >> 5] >> (j & 31)) & 1u) {
+          const bool wide = (wd[j >> 5] >> (j & 31)) & 1u;
+          if (wide) {
             if (nw < 16) c |= ((ext >> nw) & 1u) << BITS;
             ++nw;
-            return __fmul_rn(sj, lvw[c]);
           }
-          return __fmul_rn(sj, lv[c]);
+          if (hc >= 0) return tab[j * 2 * NL + c];
+          const float sj = __ldg(sc + j);
+          return __fmul_rn(sj, wide ? lvw[c] : lv[c]);
         }
       };
       if constexpr (!SO3) {
@@ -566,14 +613,15 @@ IsoArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p, 
 template <int D, int BITS, bool SO3, bool DYN>
 kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((a.rows + 127) / 128);
+  constexpr size_t kTab = DYN ? static_cast<size_t>(D) * (4 << BITS) : 0;  // D x 2^(BITS+1) floats
   if (enc) {
-    const size_t smem = 1024 + D * 256;
+    const size_t smem = 1024 + D * 256 + kTab;
     auto k = k_encode_iso<D, BITS, SO3, DYN>;
     if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
     k<<<grid, 128, smem, st>>>(m0, a);
   } else {
-    const size_t smem = 1024 + D * 512;
+    const size_t smem = 1024 + D * 512 + kTab;
     auto k = k_decode_iso<D, BITS, SO3, DYN>;
     if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
