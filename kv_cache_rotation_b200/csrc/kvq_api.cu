@@ -455,7 +455,7 @@ kvq_status kvq_detect_sinks(const kvq_desc* d, const void* x, double tau, int32_
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
   return launch_detect_sinks(*d, x, tau, max_sinks, sink_pos, count, workspace,
-                             reinterpret_cast<cudaStream_t>(stream));
+                             reinterpret_cast<cudaStream_t>(stream), ctx.num_sms);
 }
 
 size_t kvq_packed_bytes(const kvq_desc* d, int32_t field) {

@@ -60,7 +60,7 @@ kvq_status launch_calibrate_codebook(const kvq_desc& d, const void* x, const kvq
                                      uint32_t* ch_wide, void* ws, cudaStream_t st);
 size_t detect_sinks_workspace_bytes(const kvq_desc& d);
 kvq_status launch_detect_sinks(const kvq_desc& d, const void* x, double tau, int max_sinks, int32_t* sink_pos,
-                               int32_t* count, void* ws, cudaStream_t st);
+                               int32_t* count, void* ws, cudaStream_t st, int num_sms);
 // The list form of the sink set (kvq_tables.sink_pos): run after the kernels of
 // encode / decode / score were launched with n_sink = 0.
 kvq_status launch_sink_fix_encode(const kvq_desc& d, const void* x, const kvq_tables& tb, const kvq_packed& out,

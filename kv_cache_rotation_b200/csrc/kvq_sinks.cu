@@ -42,33 +42,36 @@ __device__ __forceinline__ uint32_t mag_max8(uint4 r) {
 }
 
 // key[b][t] = max over heads and channels of the fp16 magnitude bits of
-// x[b][h][t][:]. A token row is D/8 lanes of 16 bytes; each thread walks the
-// heads with four rows in flight.
+// x[b][h][t][:]. A tile is TPB tokens of one sequence; a token row is D/8
+// lanes of 16 bytes; each thread walks the heads with four rows in flight.
+// Persistent CTAs (one wave) stride over the B * ceil(T / TPB) tiles.
 template <int D>
 __global__ void __launch_bounds__(kAbsThreads) k_token_absmax(const uint4* __restrict__ x, uint16_t* key, int H,
-                                                              int T) {
+                                                              int T, int tiles_per_seq, int n_tiles) {
   constexpr int LPT = D / 8;
   constexpr int TPB = kAbsThreads / LPT;
-  const int b = blockIdx.y;
-  const int t = blockIdx.x * TPB + static_cast<int>(threadIdx.x) / LPT;
   const int c = threadIdx.x % LPT;
-  uint32_t m = 0;
-  if (t < T) {
-    const size_t hs = static_cast<size_t>(T) * LPT;  // uint4 per head slice
-    const uint4* p = x + (static_cast<size_t>(b) * H * T + t) * LPT + c;
-    int h = 0;
-    for (; h + 4 <= H; h += 4) {
-      uint4 r[4];
+  const size_t hs = static_cast<size_t>(T) * LPT;  // uint4 per head slice
+  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const int b = tile / tiles_per_seq;
+    const int t = (tile - b * tiles_per_seq) * TPB + static_cast<int>(threadIdx.x) / LPT;
+    uint32_t m = 0;
+    if (t < T) {
+      const uint4* p = x + (static_cast<size_t>(b) * H * T + t) * LPT + c;
+      int h = 0;
+      for (; h + 4 <= H; h += 4) {
+        uint4 r[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) r[u] = __ldcs(p + (h + u) * hs);
+        for (int u = 0; u < 4; ++u) r[u] = __ldcs(p + (h + u) * hs);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) m = max(m, mag_max8(r[u]));
+        for (int u = 0; u < 4; ++u) m = max(m, mag_max8(r[u]));
+      }
+      for (; h < H; ++h) m = max(m, mag_max8(__ldcs(p + h * hs)));
     }
-    for (; h < H; ++h) m = max(m, mag_max8(__ldcs(p + h * hs)));
-  }
 #pragma unroll
-  for (int o = LPT / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (c == 0 && t < T) key[static_cast<size_t>(b) * T + t] = static_cast<uint16_t>(m);
+    for (int o = LPT / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (c == 0 && t < T) key[static_cast<size_t>(b) * T + t] = static_cast<uint16_t>(m);
+  }
 }
 
 __device__ __forceinline__ double key_value(uint32_t k) {
@@ -317,15 +320,19 @@ size_t detect_sinks_workspace_bytes(const kvq_desc& d) {
 }
 
 kvq_status launch_detect_sinks(const kvq_desc& d, const void* x, double tau, int max_sinks, int32_t* sink_pos,
-                               int32_t* count, void* ws, cudaStream_t st) {
+                               int32_t* count, void* ws, cudaStream_t st, int num_sms) {
   uint16_t* key = static_cast<uint16_t*>(ws);
   const int D = d.head_dim;
   const int tpb = kAbsThreads / (D / 8);
-  const dim3 g1((d.tokens + tpb - 1) / tpb, d.batch);
-  if (D == 128)
-    k_token_absmax<128><<<g1, kAbsThreads, 0, st>>>(static_cast<const uint4*>(x), key, d.heads, d.tokens);
-  else
-    k_token_absmax<64><<<g1, kAbsThreads, 0, st>>>(static_cast<const uint4*>(x), key, d.heads, d.tokens);
+  const long long tiles_per_seq = (d.tokens + tpb - 1) / tpb;
+  const long long n_tiles = tiles_per_seq * d.batch;
+  if (n_tiles >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+  const auto fn = D == 128 ? k_token_absmax<128> : k_token_absmax<64>;
+  const int per_sm = occupancy_once(reinterpret_cast<const void*>(fn), kAbsThreads, 0);
+  const long long wave = static_cast<long long>(num_sms) * per_sm;
+  const unsigned grid = static_cast<unsigned>(n_tiles < wave ? n_tiles : wave);
+  fn<<<grid, kAbsThreads, 0, st>>>(static_cast<const uint4*>(x), key, d.heads, d.tokens,
+                                   static_cast<int>(tiles_per_seq), static_cast<int>(n_tiles));
   if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
   constexpr size_t smem = kBins * sizeof(uint32_t);
   if (!set_smem_once(reinterpret_cast<const void*>(k_sink_select), smem)) return KVQ_ERR_CUDA;
