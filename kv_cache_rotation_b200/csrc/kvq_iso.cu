@@ -613,7 +613,10 @@ IsoArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p, 
 template <int D, int BITS, bool SO3, bool DYN>
 kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((a.rows + 127) / 128);
-  constexpr size_t kTab = DYN ? static_cast<size_t>(D) * (8 << BITS) : 0;  // D x 2^(BITS+1) floats
+  // dynamic codebooks: the channel table after the staging tile, D rows of
+  // 2 NL = 2^(BITS+1) floats (dyn_tables writes entries 0 .. D * 2 NL - 1;
+  // lookups read row j at most entry 2 NL - 1); the 1024 bytes cover align1024
+  constexpr size_t kTab = DYN ? static_cast<size_t>(D) * (2 << BITS) * sizeof(float) : 0;
   if (enc) {
     const size_t smem = 1024 + D * 256 + kTab;
     auto k = k_encode_iso<D, BITS, SO3, DYN>;
