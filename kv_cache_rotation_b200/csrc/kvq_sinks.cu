@@ -12,9 +12,9 @@
 //
 // Two kernels: k_token_absmax streams x once (HBM-bound) and leaves one
 // 16-bit key per token, the fp16 magnitude bits, which order like the values;
-// k_sink_select takes one CTA per sequence, builds a 32768-bin histogram of
-// the keys in shared memory, reads the median and the cut-off key off its
-// prefix sums and writes the list with an ordered block compaction.
+// k_sink_select takes one CTA per sequence, finds the median and the cut-off
+// key by a two-level radix select (256 + 128 bins in shared memory) and
+// writes the list with an ordered block compaction.
 //
 // The list form of the cache (kvq_tables.sink_pos) reuses the prefix-free
 // kernels unchanged: encode, decode and score run on every slot, then the
@@ -31,9 +31,7 @@ namespace kvq {
 namespace {
 
 constexpr int kAbsThreads = 256;
-constexpr int kSelThreads = 1024;
-constexpr int kBins = 32768;  // fp16 magnitude bit patterns
-constexpr int kBinsPerThread = kBins / kSelThreads;
+constexpr int kSelThreads = 256;
 
 __device__ __forceinline__ uint32_t mag_max8(uint4 r) {
   const uint32_t m = __vmaxu2(__vmaxu2(r.x & 0x7fff7fffu, r.y & 0x7fff7fffu),
@@ -78,7 +76,8 @@ __device__ __forceinline__ double key_value(uint32_t k) {
   return static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(k))));
 }
 
-// Exclusive prefix of v over the CTA in thread order, and the CTA total.
+// Exclusive prefix of v over the CTA in thread order (kSelThreads threads),
+// and the CTA total. `wsum` holds kSelThreads / 32 words.
 __device__ __forceinline__ uint32_t cta_exclusive(uint32_t v, uint32_t* wsum, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t inc = v;
@@ -90,7 +89,7 @@ __device__ __forceinline__ uint32_t cta_exclusive(uint32_t v, uint32_t* wsum, ui
   if (lane == 31) wsum[warp] = inc;
   __syncthreads();
   uint32_t off = 0, tot = 0;
-#pragma unroll 8
+#pragma unroll
   for (int w = 0; w < kSelThreads / 32; ++w) {
     const uint32_t s = wsum[w];
     off += w < warp ? s : 0u;
@@ -101,26 +100,61 @@ __device__ __forceinline__ uint32_t cta_exclusive(uint32_t v, uint32_t* wsum, ui
   return off + inc - v;
 }
 
-// The key of ascending rank r (0-based) in the histogram; every thread owns
-// kBinsPerThread consecutive bins.
-__device__ __forceinline__ uint32_t hist_select(const uint32_t* hist, uint32_t r, uint32_t* wsum, uint32_t* out) {
-  const int k0 = threadIdx.x * kBinsPerThread;
-  uint32_t local = 0;
-  for (int i = 0; i < kBinsPerThread; ++i) local += hist[k0 + i];
-  uint32_t total;
-  uint32_t run = cta_exclusive(local, wsum, total);
-  if (r >= run && r < run + local) {
-    for (int i = 0; i < kBinsPerThread; ++i) {
-      run += hist[k0 + i];
-      if (r < run) {
-        *out = static_cast<uint32_t>(k0 + i);
+// Warp 0 finds the bin of ascending rank r in hist[0 .. NB) (NB / 32 bins per
+// lane) and writes (bin, count of keys in the bins below it) to out.
+template <int NB>
+__device__ __forceinline__ void warp_find_rank(const uint32_t* hist, uint32_t r, uint32_t* out) {
+  constexpr int PER = NB / 32;
+  const int lane = threadIdx.x & 31;
+  uint32_t loc[PER], sum = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    loc[j] = hist[lane * PER + j];
+    sum += loc[j];
+  }
+  uint32_t inc = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  uint32_t run = inc - sum;
+  if (r >= run && r < inc) {
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      if (r < run + loc[j]) {
+        out[0] = static_cast<uint32_t>(lane * PER + j);
+        out[1] = run;
         break;
       }
+      run += loc[j];
     }
   }
+}
+
+// The key of ascending rank r (0-based) among key[0 .. T): a two-level radix
+// select, 256 bins on bits 14..7 of the 15-bit key, then 128 bins on bits 6..0
+// of the keys in the chosen bin.
+__device__ uint32_t radix_select(const uint16_t* key, int T, uint32_t r, uint32_t* h1, uint32_t* h2,
+                                 uint32_t* sh) {
+  const int tid = threadIdx.x;
+  for (int i = tid; i < 256; i += kSelThreads) h1[i] = 0;
+  for (int i = tid; i < 128; i += kSelThreads) h2[i] = 0;
   __syncthreads();
-  const uint32_t k = *out;
+  for (int t = tid; t < T; t += kSelThreads) atomicAdd(&h1[(key[t] & 0x7fffu) >> 7], 1u);
   __syncthreads();
+  if (tid < 32) warp_find_rank<256>(h1, r, sh);
+  __syncthreads();
+  const uint32_t hi = sh[0], below = sh[1];
+  for (int t = tid; t < T; t += kSelThreads) {
+    const uint32_t k = key[t] & 0x7fffu;
+    if ((k >> 7) == hi) atomicAdd(&h2[k & 127u], 1u);
+  }
+  __syncthreads();
+  if (tid < 32) warp_find_rank<128>(h2, r - below, sh);
+  __syncthreads();
+  const uint32_t k = (hi << 7) | sh[0];
+  __syncthreads();  // sh is free again
   return k;
 }
 
@@ -132,67 +166,75 @@ struct SelArgs {
   int32_t* count;
 };
 
+// One CTA per sequence. Thread i owns the contiguous token segment
+// [i * S, (i + 1) * S), S = ceil(T / kSelThreads), so the ordered compaction
+// needs one CTA scan for the ranks among equal keys and one for the output
+// slots.
 __global__ void __launch_bounds__(kSelThreads) k_sink_select(const SelArgs a) {
-  extern __shared__ uint32_t hist[];  // kBins counters
-  __shared__ uint32_t wsum[kSelThreads / 32];
-  __shared__ uint32_t sel_key, cnt;
+  __shared__ uint32_t h1[256], h2[128], wsum[kSelThreads / 32], sh[2], cnt;
   const int b = blockIdx.x, tid = threadIdx.x;
   const uint16_t* key = a.key + static_cast<size_t>(b) * a.T;
-  for (int i = tid; i < kBins; i += kSelThreads) hist[i] = 0;
+  const uint32_t T = static_cast<uint32_t>(a.T), M = static_cast<uint32_t>(a.max_sinks);
+  const double thr = a.tau * key_value(radix_select(key, a.T, (T - 1) / 2, h1, h2, sh));
+
+  const int S = (a.T + kSelThreads - 1) / kSelThreads;
+  const int s0 = min(tid * S, a.T), s1 = min(s0 + S, a.T);
+  // C = tokens above the threshold
   if (tid == 0) cnt = 0;
   __syncthreads();
-  for (int t = tid; t < a.T; t += kSelThreads) atomicAdd(&hist[key[t] & (kBins - 1)], 1u);
-  __syncthreads();
-
-  const uint32_t T = static_cast<uint32_t>(a.T), M = static_cast<uint32_t>(a.max_sinks);
-  const double thr = a.tau * key_value(hist_select(hist, (T - 1) / 2, wsum, &sel_key));
-  // C = tokens above the threshold
-  {
-    uint32_t c = 0;
-    const int k0 = tid * kBinsPerThread;
-    for (int i = 0; i < kBinsPerThread; ++i)
-      if (key_value(k0 + i) > thr) c += hist[k0 + i];
-    if (c) atomicAdd(&cnt, c);
-  }
+  uint32_t c = 0;
+  for (int t = s0; t < s1; ++t) c += key_value(key[t] & 0x7fffu) > thr;
+  if (c) atomicAdd(&cnt, c);
   __syncthreads();
   const uint32_t C = cnt;
+  __syncthreads();
   // More candidates than room: keep those above the M-th largest key kc and
   // the earliest `need` tokens equal to it.
   const bool capped = C > M;
   uint32_t kc = 0, need = 0;
   if (capped) {
-    kc = hist_select(hist, T - M, wsum, &sel_key);
-    uint32_t g = 0;
-    const int k0 = tid * kBinsPerThread;
-    for (int i = 0; i < kBinsPerThread; ++i)
-      if (static_cast<uint32_t>(k0 + i) > kc) g += hist[k0 + i];
-    __syncthreads();
+    kc = radix_select(key, a.T, T - M, h1, h2, sh);
     if (tid == 0) cnt = 0;
     __syncthreads();
+    uint32_t g = 0;
+    for (int t = s0; t < s1; ++t) g += (key[t] & 0x7fffu) > kc;
     if (g) atomicAdd(&cnt, g);
     __syncthreads();
     need = M - cnt;
   }
-
-  uint32_t n = 0, eq_seen = 0;
-  int32_t* out = a.sink_pos + static_cast<size_t>(b) * M;
-  for (int t0 = 0; t0 < a.T; t0 += kSelThreads) {  // uniform trip count
-    const int t = t0 + tid;
-    const uint32_t k = t < a.T ? key[t] : 0u;
-    bool sel = false, eq = false;
-    if (t < a.T) {
-      if (!capped) sel = key_value(k) > thr;
-      else if (k > kc) sel = true;
-      else eq = k == kc;
+  auto selected = [&](uint32_t k, uint32_t eq_rank, bool& eq) {
+    eq = capped && k == kc;
+    if (!capped) return key_value(k) > thr;
+    return k > kc || (eq && eq_rank < need);
+  };
+  uint32_t n_eq = 0;
+  if (capped)
+    for (int t = s0; t < s1; ++t) n_eq += (key[t] & 0x7fffu) == kc;
+  uint32_t tot;
+  const uint32_t eq0 = cta_exclusive(n_eq, wsum, tot);
+  uint32_t n_sel = 0;
+  {
+    uint32_t er = eq0;
+    for (int t = s0; t < s1; ++t) {
+      bool eq;
+      n_sel += selected(key[t] & 0x7fffu, er, eq);
+      er += eq;
     }
-    uint32_t eq_tot;
-    const uint32_t eq_rank = eq_seen + cta_exclusive(eq ? 1u : 0u, wsum, eq_tot);
-    eq_seen += eq_tot;
-    sel = sel || (eq && eq_rank < need);
-    uint32_t sel_tot;
-    const uint32_t idx = n + cta_exclusive(sel ? 1u : 0u, wsum, sel_tot);
-    if (sel && idx < M) out[idx] = a.t0 + t;
-    n += sel_tot;
+  }
+  uint32_t n;
+  uint32_t idx = cta_exclusive(n_sel, wsum, n);
+  int32_t* out = a.sink_pos + static_cast<size_t>(b) * M;
+  {
+    uint32_t er = eq0;
+    for (int t = s0; t < s1 && n_sel; ++t) {
+      bool eq;
+      if (selected(key[t] & 0x7fffu, er, eq)) {
+        if (idx < M) out[idx] = a.t0 + t;
+        ++idx;
+        --n_sel;
+      }
+      er += eq;
+    }
   }
   if (n > M) n = M;
   for (uint32_t i = n + tid; i < M; i += kSelThreads) out[i] = -1;
@@ -334,10 +376,8 @@ kvq_status launch_detect_sinks(const kvq_desc& d, const void* x, double tau, int
   fn<<<grid, kAbsThreads, 0, st>>>(static_cast<const uint4*>(x), key, d.heads, d.tokens,
                                    static_cast<int>(tiles_per_seq), static_cast<int>(n_tiles));
   if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
-  constexpr size_t smem = kBins * sizeof(uint32_t);
-  if (!set_smem_once(reinterpret_cast<const void*>(k_sink_select), smem)) return KVQ_ERR_CUDA;
   SelArgs a{d.tokens, d.t0, max_sinks, tau, key, sink_pos, count};
-  k_sink_select<<<d.batch, kSelThreads, smem, st>>>(a);
+  k_sink_select<<<d.batch, kSelThreads, 0, st>>>(a);
   return launch_status();
 }
 
