@@ -43,7 +43,9 @@ __device__ __forceinline__ bool is_sink(const CalArgs& a, int b, int pos) {
   return hit;
 }
 
-template <int D>
+// ROPE: 0 none, 1 interleaved pairs, 2 half-split pairs (the only mode whose
+// threads exchange channels, so the only one that needs a uniform trip count).
+template <int D, int ROPE>
 __global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
   constexpr int TPR = D / 8;           // threads per row
   constexpr int RPI = kThreads / TPR;  // rows in flight per CTA iteration
@@ -56,10 +58,11 @@ __global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = 0.0f;
   constexpr int U = 4;  // rows per thread in flight
-  // the trip count is the same for every thread (rows past r1 are not live),
-  // so the half-split pairs may exchange channels between threads
-  for (int rb = r0; rb < r1; rb += U * RPI) {  // row r = (batch b, token t)
-    const int r = rb + rl;
+  // with half-split pairs the trip count is the same for every thread (rows
+  // past r1 are not live), so the pairs may exchange channels between threads
+  const int rstart = ROPE == 2 ? r0 : r0 + rl;
+  for (int rs = rstart; rs < r1; rs += U * RPI) {  // row r = (batch b, token t)
+    const int r = ROPE == 2 ? rs + rl : rs;
     uint4 raw[U];
     float4 c0[U], c1[U];
     int posu[U];
@@ -75,7 +78,7 @@ __global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
       raw[u] = live[u] ? __ldg(reinterpret_cast<const uint4*>(
                              a.x + ((static_cast<size_t>(b) * a.H + h) * a.T + t) * D) + cg)
                        : make_uint4(0, 0, 0, 0);
-      if (a.rope == 1 && live[u]) {  // pairs 4 cg .. 4 cg + 3 of position pos
+      if (ROPE == 1 && live[u]) {  // pairs 4 cg .. 4 cg + 3 of position pos
         const float4* cs = reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(pos) * D) + 2 * cg;
         c0[u] = __ldg(cs);
         c1[u] = __ldg(cs + 1);
@@ -87,12 +90,12 @@ __global__ void __launch_bounds__(kThreads) k_absmax(const CalArgs a) {
     for (int u = 0; u < U; ++u) {
       float v[8];
       h8_to_f32(raw[u], v);
-      if (a.rope == 1) {
+      if constexpr (ROPE == 1) {
         rope_fwd(v[0], v[1], c0[u].x, c0[u].y);
         rope_fwd(v[2], v[3], c0[u].z, c0[u].w);
         rope_fwd(v[4], v[5], c1[u].x, c1[u].y);
         rope_fwd(v[6], v[7], c1[u].z, c1[u].w);
-      } else if (a.rope == 2) {
+      } else if constexpr (ROPE == 2) {
         // half-split pairs (c, c + D/2): this thread's channel 8 (cg mod TPR/2) + i pairs with the same
         // channel of thread cg ^ TPR/2 (the other half of the row), angle 8 (cg mod TPR/2) + i
         const float4* cs = reinterpret_cast<const float4*>(a.rope_cs + static_cast<size_t>(posu[u]) * D) +
@@ -147,7 +150,13 @@ template <int D>
 kvq_status run(CalArgs& a, int chunks, cudaStream_t st) {
   if (cudaMemsetAsync(a.amax, 0, static_cast<size_t>(a.H) * D * sizeof(uint32_t), st) != cudaSuccess)
     return KVQ_ERR_CUDA;
-  k_absmax<D><<<dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(a.H)), kThreads, 0, st>>>(a);
+  const dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(a.H));
+  if (a.rope == 1)
+    k_absmax<D, 1><<<grid, kThreads, 0, st>>>(a);
+  else if (a.rope == 2)
+    k_absmax<D, 2><<<grid, kThreads, 0, st>>>(a);
+  else
+    k_absmax<D, 0><<<grid, kThreads, 0, st>>>(a);
   kvq_status s = launch_status();
   if (s != KVQ_OK) return s;
   k_perm_rank<D><<<static_cast<unsigned>(a.H), D, 0, st>>>(a);

@@ -233,7 +233,10 @@ __device__ __forceinline__ void put_code(uint32_t (&w)[NW], int j, uint32_t c) {
   if ((pos & 31) + BITS > 32) w[(pos >> 5) + 1] |= c >> (32 - (pos & 31));
 }
 
-template <int D, int BITS, bool SO3, bool DYN>
+// DYN: 0 fixed codebook; 1 dynamic, channel levels formed per element; 2
+// dynamic, the channel boundaries / levels of the CTA's one head in shared
+// memory (the host picks 2 when no CTA spans two heads: H = 1 or T % 128 = 0).
+template <int D, int BITS, bool SO3, int DYN>
 __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUtensorMap xmap, const IsoArgs a) {
   constexpr int NB = D / 4;
   constexpr int NL = 1 << BITS;
@@ -259,14 +262,14 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
     for (int hh = 0; hh < D / 64; ++hh) tma_load_2d(xs + hh * 16384, &xmap, hh * 64, static_cast<int>(r0), &bar);
   }
   build_mats<SO3>(a, Ms, D);
-  int hc = -1;  // dynamic codebooks: the CTA's head when its channel tables are in shared memory
-  float* tab = reinterpret_cast<float*>(xs + D * 256);
-  if constexpr (DYN) {
+  float* tab = reinterpret_cast<float*>(xs + D * 256);  // DYN == 2: the channel boundaries
+  if constexpr (DYN != 0) {
     if (tid < NL) beta[tid] = a.codebook[tid];
     if (tid < 2 * NL) lvw[tid] = a.cb_wide[tid];
-    hc = cta_head(a, r0);
-    __syncthreads();
-    if (hc >= 0) dyn_tables<D, NL, false>(a, hc, beta, lvw, tab);
+    if constexpr (DYN == 2) {
+      __syncthreads();
+      dyn_tables<D, NL, false>(a, cta_head(a, r0), beta, lvw, tab);
+    }
   } else {
     if (tid < NL - 1) beta[tid] = __fmul_rn(0.5f, __fadd_rn(a.codebook[tid], a.codebook[tid + 1]));
   }
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
 #pragma unroll
     for (int i = 0; i < RB / 8; ++i) reinterpret_cast<uint2*>(a.codes + slot * RB)[i] = make_uint2(0, 0);
     a.norm[slot] = 0.0f;
-    if constexpr (DYN) a.ext[slot] = 0;
+    if constexpr (DYN != 0) a.ext[slot] = 0;
     return;
   }
   float x[D];
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
   uint32_t w[NW];
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
-  if constexpr (!DYN) {
+  if constexpr (DYN == 0) {
     iso_rotate<D, SO3>(x, inv, Ms, [&](int j, float wj) { put_code<BITS, NW>(w, j, cb_code<NL>(wj, beta)); });
   } else {
     const int h = static_cast<int>(bh % a.H);
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
     iso_rotate<D, SO3>(x, inv, Ms, [&](int j, float wj) {
       uint32_t c;
       const bool wide = (wd[j >> 5] >> (j & 31)) & 1u;
-      if (hc >= 0) {  // the channel's boundaries from shared memory
+      if constexpr (DYN == 2) {  // the channel's boundaries from shared memory
         c = wide ? cb_code<2 * NL>(wj, tab + j * 2 * NL) : cb_code<NL>(wj, tab + j * 2 * NL);
       } else {
         const float sj = __ldg(sc + j);
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
   a.norm[slot] = rho;
 }
 
-template <int D, int BITS, bool SO3, bool DYN>
+template <int D, int BITS, bool SO3, int DYN>
 __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUtensorMap omap, const IsoArgs a,
                                                      int out_fp32) {
   constexpr int NB = D / 4;
@@ -357,13 +360,13 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
   const long long r0 = static_cast<long long>(blockIdx.x) * 128;
   build_mats<SO3>(a, Ms, D);
   if (tid < NL) lv[tid] = a.codebook[tid];
-  int hc = -1;  // dynamic codebooks: the CTA's head when its channel levels are in shared memory
-  float* tab = reinterpret_cast<float*>(os + D * 512);
-  if constexpr (DYN) {
+  float* tab = reinterpret_cast<float*>(os + D * 512);  // DYN == 2: the channel levels
+  if constexpr (DYN != 0) {
     if (tid < 2 * NL) lvw[tid] = a.cb_wide[tid];
-    hc = cta_head(a, r0);
-    __syncthreads();
-    if (hc >= 0) dyn_tables<D, NL, true>(a, hc, lv, lvw, tab);
+    if constexpr (DYN == 2) {
+      __syncthreads();
+      dyn_tables<D, NL, true>(a, cta_head(a, r0), lv, lvw, tab);
+    }
   }
   __syncthreads();
   const long long vid = r0 + tid;
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
       const float* sc = nullptr;
       uint32_t wd[D / 32], ext = 0;
       int nw = 0;
-      if constexpr (DYN) {
+      if constexpr (DYN != 0) {
         const int h = static_cast<int>(bh % a.H);
         sc = a.ch_scale + static_cast<size_t>(h) * D;
 #pragma unroll
@@ -407,7 +410,7 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
       }
       auto level = [&](int j) -> float {
         uint32_t c = unpack_code<BITS, NW>(w, j);
-        if constexpr (!DYN) {
+        if constexpr (DYN == 0) {
           return lv[c];
         } else {
           const bool wide = (wd[j >> 5] >> (j & 31)) & 1u;
@@ -415,7 +418,7 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
             if (nw < 16) c |= ((ext >> nw) & 1u) << BITS;
             ++nw;
           }
-          if (hc >= 0) return tab[j * 2 * NL + c];
+          if constexpr (DYN == 2) return tab[j * 2 * NL + c];
           const float sj = __ldg(sc + j);
           return __fmul_rn(sj, wide ? lvw[c] : lv[c]);
         }
@@ -610,13 +613,13 @@ IsoArgs make_args(const kvq_desc& d, const kvq_tables& tb, const kvq_packed& p, 
   return a;
 }
 
-template <int D, int BITS, bool SO3, bool DYN>
+template <int D, int BITS, bool SO3, int DYN>
 kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((a.rows + 127) / 128);
   // dynamic codebooks: the channel table after the staging tile, D rows of
   // 2 NL = 2^(BITS+1) floats (dyn_tables writes entries 0 .. D * 2 NL - 1;
   // lookups read row j at most entry 2 NL - 1); the 1024 bytes cover align1024
-  constexpr size_t kTab = DYN ? static_cast<size_t>(D) * (2 << BITS) * sizeof(float) : 0;
+  constexpr size_t kTab = DYN == 2 ? static_cast<size_t>(D) * (2 << BITS) * sizeof(float) : 0;
   if (enc) {
     const size_t smem = 1024 + D * 256 + kTab;
     auto k = k_encode_iso<D, BITS, SO3, DYN>;
@@ -635,13 +638,16 @@ kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, 
 
 kvq_status dispatch(bool enc, const kvq_desc& d, const IsoArgs& a, const CUtensorMap& m0, int out_fp32,
                     cudaStream_t st) {
+  // dynamic codebooks: the shared-memory tables when no 128-vector CTA spans two heads
+  const bool one_head = d.heads == 1 || d.tokens % 128 == 0;
+#define KVQ_RUN(D_, B_, DYN_)                                                                         \
+  return d.rot == KVQ_ROT_ISO_SO3 ? run<D_, B_, true, DYN_>(enc, a, m0, out_fp32, st)                 \
+                                  : run<D_, B_, false, DYN_>(enc, a, m0, out_fp32, st);
 #define KVQ_CASE(D_, B_)                                                                              \
   if (d.head_dim == D_ && d.bits == B_) {                                                             \
-    if (d.quant == KVQ_Q_CODEBOOK_DYN)                                                                \
-      return d.rot == KVQ_ROT_ISO_SO3 ? run<D_, B_, true, true>(enc, a, m0, out_fp32, st)             \
-                                      : run<D_, B_, false, true>(enc, a, m0, out_fp32, st);           \
-    return d.rot == KVQ_ROT_ISO_SO3 ? run<D_, B_, true, false>(enc, a, m0, out_fp32, st)              \
-                                    : run<D_, B_, false, false>(enc, a, m0, out_fp32, st);            \
+    if (d.quant != KVQ_Q_CODEBOOK_DYN) { KVQ_RUN(D_, B_, 0) }                                         \
+    if (one_head) { KVQ_RUN(D_, B_, 2) }                                                              \
+    KVQ_RUN(D_, B_, 1)                                                                                \
   }
   KVQ_CASE(128, 2)
   KVQ_CASE(128, 3)
@@ -650,6 +656,7 @@ kvq_status dispatch(bool enc, const kvq_desc& d, const IsoArgs& a, const CUtenso
   KVQ_CASE(64, 3)
   KVQ_CASE(64, 4)
 #undef KVQ_CASE
+#undef KVQ_RUN
   return KVQ_ERR_UNSUPPORTED;
 }
 

@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kThreads) k_score_simt(const ScoreArgs a) {
 // A block is four m-tiles of 16 tokens.
 constexpr int kMmaThreads = 256;
 constexpr int kMmaWarps = kMmaThreads / 32;
-constexpr int kMmaStages = 3;     // blocks in flight per warp
+constexpr int kMmaStages = 2;     // blocks in flight per warp (2 beat 3 and 4: less shared memory, 4 CTAs per SM)
 constexpr int kMmaCtasPerSm = 4;
 constexpr int kMmaBlk = 64;       // tokens per block
 

@@ -170,10 +170,30 @@ struct SelArgs {
 // [i * S, (i + 1) * S), S = ceil(T / kSelThreads), so the ordered compaction
 // needs one CTA scan for the ranks among equal keys and one for the output
 // slots.
-__global__ void __launch_bounds__(kSelThreads) k_sink_select(const SelArgs a) {
+__global__ void __launch_bounds__(kSelThreads) k_sink_select(const SelArgs a, int staged) {
   __shared__ uint32_t h1[256], h2[128], wsum[kSelThreads / 32], sh[2], cnt;
+  extern __shared__ uint16_t skey[];  // the sequence's keys when they fit (staged != 0)
   const int b = blockIdx.x, tid = threadIdx.x;
-  const uint16_t* key = a.key + static_cast<size_t>(b) * a.T;
+  const uint16_t* gkey = a.key + static_cast<size_t>(b) * a.T;
+  const uint16_t* key = gkey;
+  if (staged) {  // every later pass reads shared memory instead of L2
+    constexpr int U = 8;
+    for (int t0 = 0; t0 < a.T; t0 += U * kSelThreads) {
+      uint16_t v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = t0 + u * kSelThreads + tid;
+        v[u] = t < a.T ? gkey[t] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = t0 + u * kSelThreads + tid;
+        if (t < a.T) skey[t] = v[u];
+      }
+    }
+    __syncthreads();
+    key = skey;
+  }
   const uint32_t T = static_cast<uint32_t>(a.T), M = static_cast<uint32_t>(a.max_sinks);
   const double thr = a.tau * key_value(radix_select(key, a.T, (T - 1) / 2, h1, h2, sh));
 
@@ -377,7 +397,12 @@ kvq_status launch_detect_sinks(const kvq_desc& d, const void* x, double tau, int
                                    static_cast<int>(tiles_per_seq), static_cast<int>(n_tiles));
   if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
   SelArgs a{d.tokens, d.t0, max_sinks, tau, key, sink_pos, count};
-  k_sink_select<<<d.batch, kSelThreads, 0, st>>>(a);
+  // stage a sequence's keys in shared memory when they fit in 96 KB
+  const size_t kbytes = static_cast<size_t>(d.tokens) * sizeof(uint16_t);
+  const int staged = kbytes <= 96 * 1024 ? 1 : 0;
+  const size_t smem = staged ? kbytes : 0;
+  if (smem && !set_smem_once(reinterpret_cast<const void*>(k_sink_select), smem)) return KVQ_ERR_CUDA;
+  k_sink_select<<<d.batch, kSelThreads, smem, st>>>(a, staged);
   return launch_status();
 }
 
