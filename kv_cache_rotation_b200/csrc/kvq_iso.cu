@@ -174,6 +174,93 @@ __device__ __forceinline__ void iso_rotate(const float (&x)[D], float inv, const
   }
 }
 
+// iso_rotate on a row read chunk by chunk (ld(c, v) fills v[0..7] with the
+// channels 8c .. 8c+7): the same operations in the same order, with only the
+// channels of the current blocks live in registers. 4-D blocks take one chunk
+// per two blocks; 3-D blocks take three chunks per eight blocks, then the
+// remaining channels (two or five blocks and the tail).
+template <int D, bool SO3, class Ld, class Emit>
+__device__ __forceinline__ void iso_rotate_chunks(Ld&& ld, float inv, const float* Ms, Emit&& emit) {
+  if constexpr (!SO3) {
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      float v[8];
+      ld(c, v);
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) {
+        const int k = 2 * c + kb;
+        float u[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) u[e] = __fmul_rn(v[4 * kb + e], inv);
+        const float4* Mk = reinterpret_cast<const float4*>(Ms + k * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 row = Mk[i];
+          float wi = __fmul_rn(row.x, u[0]);
+          wi = __fmaf_rn(row.y, u[1], wi);
+          wi = __fmaf_rn(row.z, u[2], wi);
+          wi = __fmaf_rn(row.w, u[3], wi);
+          emit(4 * k + i, wi);
+        }
+      }
+    }
+  } else {
+    constexpr int NG = D / 24;           // groups of 24 channels = 8 blocks
+    constexpr int R0 = 24 * NG, RN = D - R0, RB = RN / 3, TAIL = D % 3;
+    auto block3 = [&](int k, const float* v3) {  // channels 3k .. 3k+2 from v3[0..2]
+      float u[3];
+#pragma unroll
+      for (int e = 0; e < 3; ++e) u[e] = __fmul_rn(v3[e], inv);
+      const float* Mk = Ms + k * 9;
+#pragma unroll
+      for (int i = 0; i < 3; ++i) {
+        float wi = __fmul_rn(Mk[3 * i], u[0]);
+        wi = __fmaf_rn(Mk[3 * i + 1], u[1], wi);
+        wi = __fmaf_rn(Mk[3 * i + 2], u[2], wi);
+        emit(3 * k + i, wi);
+      }
+    };
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      float v[24];
+      ld(3 * g, v);
+      ld(3 * g + 1, v + 8);
+      ld(3 * g + 2, v + 16);
+#pragma unroll
+      for (int kb = 0; kb < 8; ++kb) block3(8 * g + kb, v + 3 * kb);
+    }
+    float v[RN];
+#pragma unroll
+    for (int c = 0; c < RN / 8; ++c) ld(R0 / 8 + c, v + 8 * c);
+#pragma unroll
+    for (int kb = 0; kb < RB; ++kb) block3(8 * NG + kb, v + 3 * kb);
+    if constexpr (TAIL == 2) {  // the tail in its own plane: the matrix's upper-left 2x2 block
+      const float u0 = __fmul_rn(v[RN - 2], inv), u1 = __fmul_rn(v[RN - 1], inv);
+      const float* Mk = Ms + (D / 3) * 9;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) emit(D - 2 + i, __fmaf_rn(Mk[3 * i + 1], u1, __fmul_rn(Mk[3 * i], u0)));
+    } else if constexpr (TAIL == 1) {  // a single channel is kept
+      emit(D - 1, __fmul_rn(v[RN - 1], inv));
+    }
+  }
+}
+
+// iso_norm on a row read chunk by chunk (the same sum in the same order).
+template <int D, class Ld>
+__device__ __forceinline__ float iso_norm_chunks(Ld&& ld, float& inv) {
+  double acc = 0.0;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    float v[8];
+    ld(c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc = __fma_rn(static_cast<double>(v[i]), static_cast<double>(v[i]), acc);
+  }
+  const float rho = __double2float_rn(__dsqrt_rn(acc));
+  inv = __frcp_rn(__fadd_rn(rho, 1e-8f));
+  return rho;
+}
+
 // rho = ||x|| from the fp64 sum of squares in channel order (each square is
 // exact in fp64), and the reciprocal of rho + 1e-8.
 template <int D>
@@ -295,16 +382,16 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
     if constexpr (DYN != 0) a.ext[slot] = 0;
     return;
   }
-  float x[D];
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) h8_to_f32(lds128(xs_u + (c >> 3) * 16384 + sw128(tid, c & 7)), &x[8 * c]);
+  // the staged row is read from shared memory twice (norm, then rotation), so
+  // only a few channels are live in registers at a time
+  auto ld = [&](int c, float* v) { h8_to_f32(lds128(xs_u + (c >> 3) * 16384 + sw128(tid, c & 7)), v); };
   float inv;
-  const float rho = iso_norm<D>(x, inv);
+  const float rho = iso_norm_chunks<D>(ld, inv);
   uint32_t w[NW];
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
   if constexpr (DYN == 0) {
-    iso_rotate<D, SO3>(x, inv, Ms, [&](int j, float wj) { put_code<BITS, NW>(w, j, cb_code<NL>(wj, beta)); });
+    iso_rotate_chunks<D, SO3>(ld, inv, Ms, [&](int j, float wj) { put_code<BITS, NW>(w, j, cb_code<NL>(wj, beta)); });
   } else {
     const int h = static_cast<int>(bh % a.H);
     const float* sc = a.ch_scale + static_cast<size_t>(h) * D;
@@ -313,7 +400,7 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
     for (int i = 0; i < D / 32; ++i) wd[i] = __ldg(a.ch_wide + static_cast<size_t>(h) * (D / 32) + i);
     uint32_t ext = 0;
     int nw = 0;
-    iso_rotate<D, SO3>(x, inv, Ms, [&](int j, float wj) {
+    iso_rotate_chunks<D, SO3>(ld, inv, Ms, [&](int j, float wj) {
       uint32_t c;
       const bool wide = (wd[j >> 5] >> (j & 31)) & 1u;
       if constexpr (DYN == 2) {  // the channel's boundaries from shared memory
@@ -360,7 +447,8 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
   const long long r0 = static_cast<long long>(blockIdx.x) * 128;
   build_mats<SO3>(a, Ms, D);
   if (tid < NL) lv[tid] = a.codebook[tid];
-  float* tab = reinterpret_cast<float*>(os + D * 512);  // DYN == 2: the channel levels
+  // DYN == 2: the channel levels, after the output tile (fp32: D * 512 bytes, fp16: D * 256)
+  float* tab = reinterpret_cast<float*>(os + D * (out_fp32 ? 512 : 256));
   if constexpr (DYN != 0) {
     if (tid < 2 * NL) lvw[tid] = a.cb_wide[tid];
     if constexpr (DYN == 2) {
@@ -370,16 +458,31 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
   }
   __syncthreads();
   const long long vid = r0 + tid;
-  float x[D];
   if (vid < a.rows) {
     const long long bh = vid / a.T;
     const int tt = static_cast<int>(vid - bh * a.T);
     const int m = a.t0 + tt;
     const size_t slot = static_cast<size_t>(bh) * a.t_cap + m;
+    const uint32_t os_u = smem_u32(os);
+    // chunk c = channels 8c .. 8c+7 of this thread's output row, into the tile
+    auto st = [&](int c, const float* v) {
+      if (out_fp32) {
+        sts128(os_u + ((2 * c) >> 3) * 16384 + sw128(tid, (2 * c) & 7),
+               make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3])));
+        sts128(os_u + ((2 * c + 1) >> 3) * 16384 + sw128(tid, (2 * c + 1) & 7),
+               make_uint4(__float_as_uint(v[4]), __float_as_uint(v[5]), __float_as_uint(v[6]), __float_as_uint(v[7])));
+      } else {
+        sts128(os_u + (c >> 3) * 16384 + sw128(tid, c & 7), f32_to_h8(v));
+      }
+    };
     if (m < a.n_sink) {
       const uint4* src = reinterpret_cast<const uint4*>(a.sink + (static_cast<size_t>(bh) * a.n_sink + m) * D);
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) h8_to_f32(__ldg(src + c), &x[8 * c]);
+      for (int c = 0; c < D / 8; ++c) {
+        float v[8];
+        h8_to_f32(__ldg(src + c), v);
+        st(c, v);
+      }
     } else {
       uint32_t w[NW];
       const uint8_t* srcb = a.codes + slot * RB;
@@ -425,23 +528,30 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
       };
       if constexpr (!SO3) {
 #pragma unroll
-        for (int k = 0; k < NB; ++k) {
-          float wh[4];
+        for (int c = 0; c < D / 8; ++c) {  // blocks 2c, 2c+1
+          float x8[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) wh[e] = level(4 * k + e);
-          const float* Mk = Ms + k * 16;
+          for (int kb = 0; kb < 2; ++kb) {
+            const int k = 2 * c + kb;
+            float wh[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {  // v = M^T w
-            float vi = __fmul_rn(Mk[i], wh[0]);
-            vi = __fmaf_rn(Mk[4 + i], wh[1], vi);
-            vi = __fmaf_rn(Mk[8 + i], wh[2], vi);
-            vi = __fmaf_rn(Mk[12 + i], wh[3], vi);
-            x[4 * k + i] = __fmul_rn(vi, rho);
+            for (int e = 0; e < 4; ++e) wh[e] = level(4 * k + e);
+            const float* Mk = Ms + k * 16;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // v = M^T w
+              float vi = __fmul_rn(Mk[i], wh[0]);
+              vi = __fmaf_rn(Mk[4 + i], wh[1], vi);
+              vi = __fmaf_rn(Mk[8 + i], wh[2], vi);
+              vi = __fmaf_rn(Mk[12 + i], wh[3], vi);
+              x8[4 * kb + i] = __fmul_rn(vi, rho);
+            }
           }
+          st(c, x8);
         }
       } else {
-#pragma unroll
-        for (int k = 0; k < NB3; ++k) {
+        constexpr int NG = D / 24;  // groups of 24 channels = 8 blocks
+        constexpr int R0 = 24 * NG, RN = D - R0, RB3 = RN / 3;
+        auto block3 = [&](int k, float* x3) {  // channels 3k .. 3k+2 into x3[0..2]
           float wh[3];
 #pragma unroll
           for (int e = 0; e < 3; ++e) wh[e] = level(3 * k + e);
@@ -451,31 +561,33 @@ __global__ void __launch_bounds__(128) k_decode_iso(const __grid_constant__ CUte
             float vi = __fmul_rn(Mk[i], wh[0]);
             vi = __fmaf_rn(Mk[3 + i], wh[1], vi);
             vi = __fmaf_rn(Mk[6 + i], wh[2], vi);
-            x[3 * k + i] = __fmul_rn(vi, rho);
+            x3[i] = __fmul_rn(vi, rho);
           }
+        };
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          float x24[24];
+#pragma unroll
+          for (int kb = 0; kb < 8; ++kb) block3(8 * g + kb, x24 + 3 * kb);
+          st(3 * g, x24);
+          st(3 * g + 1, x24 + 8);
+          st(3 * g + 2, x24 + 16);
         }
+        float xr[RN];
+#pragma unroll
+        for (int kb = 0; kb < RB3; ++kb) block3(8 * NG + kb, xr + 3 * kb);
         if constexpr (TAIL == 2) {
           const float w0 = level(D - 2);
           const float w1 = level(D - 1);
           const float* Mk = Ms + NB3 * 9;
 #pragma unroll
-          for (int i = 0; i < 2; ++i)
-            x[D - 2 + i] = __fmul_rn(__fmaf_rn(Mk[3 + i], w1, __fmul_rn(Mk[i], w0)), rho);
+          for (int i = 0; i < 2; ++i) xr[RN - 2 + i] = __fmul_rn(__fmaf_rn(Mk[3 + i], w1, __fmul_rn(Mk[i], w0)), rho);
         } else if constexpr (TAIL == 1) {
-          x[D - 1] = __fmul_rn(level(D - 1), rho);
+          xr[RN - 1] = __fmul_rn(level(D - 1), rho);
         }
+#pragma unroll
+        for (int c = 0; c < RN / 8; ++c) st(R0 / 8 + c, xr + 8 * c);
       }
-    }
-    const uint32_t os_u = smem_u32(os);
-    if (out_fp32) {
-#pragma unroll
-      for (int c = 0; c < D / 4; ++c)
-        sts128(os_u + (c >> 3) * 16384 + sw128(tid, c & 7),
-               make_uint4(__float_as_uint(x[4 * c]), __float_as_uint(x[4 * c + 1]), __float_as_uint(x[4 * c + 2]),
-                          __float_as_uint(x[4 * c + 3])));
-    } else {
-#pragma unroll
-      for (int c = 0; c < D / 8; ++c) sts128(os_u + (c >> 3) * 16384 + sw128(tid, c & 7), f32_to_h8(&x[8 * c]));
     }
   }
   fence_async_smem();
@@ -627,7 +739,7 @@ kvq_status run(bool enc, const IsoArgs& a, const CUtensorMap& m0, int out_fp32, 
       return KVQ_ERR_CUDA;
     k<<<grid, 128, smem, st>>>(m0, a);
   } else {
-    const size_t smem = 1024 + D * 512 + kTab;
+    const size_t smem = 1024 + D * (out_fp32 ? 512 : 256) + kTab;
     auto k = k_decode_iso<D, BITS, SO3, DYN>;
     if (!set_smem_once(reinterpret_cast<const void*>(k), smem))
       return KVQ_ERR_CUDA;
