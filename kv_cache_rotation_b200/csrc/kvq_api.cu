@@ -410,7 +410,7 @@ kvq_status kvq_calibrate_perm(const kvq_desc* d, const void* x, const kvq_tables
   if (static_cast<int64_t>(d->batch) * d->tokens >= (int64_t(1) << 31)) return KVQ_ERR_UNSUPPORTED;
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
-  return launch_calibrate(*d, x, *tb, perm_out, workspace, reinterpret_cast<cudaStream_t>(stream));
+  return launch_calibrate(*d, x, *tb, perm_out, workspace, reinterpret_cast<cudaStream_t>(stream), ctx.num_sms);
 }
 
 size_t kvq_calibrate_codebook_workspace_bytes(const kvq_desc* d) {

@@ -140,10 +140,22 @@ __global__ void __launch_bounds__(D) k_perm_rank(const CalArgs a) {
   a.perm[static_cast<size_t>(h) * D + rank] = static_cast<int16_t>(j);
 }
 
-int chunks_for(int64_t rows) {
+// Row chunks per head: at least kMinRows rows each, at most kMaxChunks, and
+// no more than one wave of CTAs over all heads (a second, partial wave would
+// leave most SMs idle for its whole length).
+int chunks_for(int64_t rows, int heads, int wave) {
   int64_t c = (rows + kMinRows - 1) / kMinRows;
-  if (c < 1) c = 1;
-  return static_cast<int>(c < kMaxChunks ? c : kMaxChunks);
+  if (c > kMaxChunks) c = kMaxChunks;
+  const int64_t fit = wave / heads;
+  if (fit >= 1 && c > fit) c = fit;
+  return static_cast<int>(c < 1 ? 1 : c);
+}
+
+template <int D>
+const void* absmax_fn(int rope) {
+  return rope == 1 ? reinterpret_cast<const void*>(k_absmax<D, 1>)
+                   : rope == 2 ? reinterpret_cast<const void*>(k_absmax<D, 2>)
+                               : reinterpret_cast<const void*>(k_absmax<D, 0>);
 }
 
 template <int D>
@@ -172,7 +184,7 @@ bool calibrate_rope(const kvq_desc& d) {
 size_t calibrate_workspace_bytes(const kvq_desc& d) { return static_cast<size_t>(d.heads) * d.head_dim * 4; }
 
 kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& tb, int16_t* perm, void* ws,
-                            cudaStream_t st) {
+                            cudaStream_t st, int num_sms) {
   const int64_t rows = static_cast<int64_t>(d.batch) * d.tokens;
   if (rows >= (int64_t(1) << 31)) return KVQ_ERR_UNSUPPORTED;
   CalArgs a{};
@@ -183,7 +195,9 @@ kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& 
   a.sink_pos = tb.sink_pos;
   a.rope = calibrate_rope(d) ? d.rope : 0;  // 1 interleaved pairs, 2 half-split pairs
   a.rows = static_cast<int>(rows);
-  const int chunks = chunks_for(rows);
+  const int rope = calibrate_rope(d) ? d.rope : 0;
+  const void* fn = d.head_dim == 128 ? absmax_fn<128>(rope) : absmax_fn<64>(rope);
+  const int chunks = chunks_for(rows, d.heads, num_sms * occupancy_once(fn, kThreads, 0));
   a.rows_per_chunk = static_cast<int>((rows + chunks - 1) / chunks);
   a.div_t = FastDiv(static_cast<uint32_t>(d.tokens > 0 ? d.tokens : 1));
   a.x = static_cast<const __half*>(x);

@@ -53,7 +53,7 @@ kvq_status launch_pair_energy(const kvq_desc& d, const void* x, uint64_t* energy
 bool calibrate_rope(const kvq_desc& d);
 size_t calibrate_workspace_bytes(const kvq_desc& d);
 kvq_status launch_calibrate(const kvq_desc& d, const void* x, const kvq_tables& tb, int16_t* perm, void* ws,
-                            cudaStream_t st);
+                            cudaStream_t st, int num_sms);
 void* attend_scratch();
 size_t calibrate_codebook_workspace_bytes(const kvq_desc& d);
 kvq_status launch_calibrate_codebook(const kvq_desc& d, const void* x, const kvq_tables& tb, float* ch_scale,

@@ -387,6 +387,9 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
   auto ld = [&](int c, float* v) { h8_to_f32(lds128(xs_u + (c >> 3) * 16384 + sw128(tid, c & 7)), v); };
   float inv;
   const float rho = iso_norm_chunks<D>(ld, inv);
+  // keep the second pass's shared-memory loads after the norm (they would
+  // otherwise be hoisted and hold the whole row in registers again)
+  asm volatile("" : "+f"(inv));
   uint32_t w[NW];
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
