@@ -112,6 +112,25 @@ __device__ __forceinline__ uint32_t cb_code(float w, const float* beta) {
   return c;
 }
 
+// The same search over boundaries held in registers (NL <= 8): each step's
+// boundary is chosen by selects on the bits found so far, so there is no
+// data-dependent shared-memory load.
+template <int NL>
+__device__ __forceinline__ uint32_t cb_code_reg(float w, const float (&b)[NL > 1 ? NL - 1 : 1]) {
+  static_assert(NL == 4 || NL == 8, "2- or 3-bit codes");
+  if constexpr (NL == 4) {
+    const bool hi = w > b[1];
+    const bool lo = w > (hi ? b[2] : b[0]);
+    return (hi ? 2u : 0u) + (lo ? 1u : 0u);
+  } else {
+    const bool b2 = w > b[3];
+    const bool b1 = w > (b2 ? b[5] : b[1]);
+    const float t = b2 ? (b1 ? b[6] : b[4]) : (b1 ? b[2] : b[0]);
+    const bool b0 = w > t;
+    return (b2 ? 4u : 0u) + (b1 ? 2u : 0u) + (b0 ? 1u : 0u);
+  }
+}
+
 // Dynamic codebook: code of w against the levels fp32(s * lv[k]) with fp32
 // midpoints as boundaries (ties to the lower code).
 template <int NL>
@@ -394,7 +413,15 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
   if constexpr (DYN == 0) {
-    iso_rotate_chunks<D, SO3>(ld, inv, Ms, [&](int j, float wj) { put_code<BITS, NW>(w, j, cb_code<NL>(wj, beta)); });
+    if constexpr (NL <= 8) {  // the boundaries in registers
+      float br[NL - 1];
+#pragma unroll
+      for (int k = 0; k < NL - 1; ++k) br[k] = beta[k];
+      iso_rotate_chunks<D, SO3>(ld, inv, Ms,
+                                [&](int j, float wj) { put_code<BITS, NW>(w, j, cb_code_reg<NL>(wj, br)); });
+    } else {
+      iso_rotate_chunks<D, SO3>(ld, inv, Ms, [&](int j, float wj) { put_code<BITS, NW>(w, j, cb_code<NL>(wj, beta)); });
+    }
   } else {
     const int h = static_cast<int>(bh % a.H);
     const float* sc = a.ch_scale + static_cast<size_t>(h) * D;
