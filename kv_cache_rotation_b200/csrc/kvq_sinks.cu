@@ -40,37 +40,35 @@ __device__ __forceinline__ uint32_t mag_max8(uint4 r) {
 }
 
 // key[b][t] = max over heads and channels of the fp16 magnitude bits of
-// x[b][h][t][:]. The B * T token rows are split into one contiguous, equal
-// range per CTA (one persistent wave, so no CTA gets a whole extra tile); a
-// CTA walks its range TPB tokens at a time, a token row being D/8 lanes of
-// 16 bytes, each thread walking the heads with four rows in flight.
+// x[b][h][t][:]. A tile is TPB tokens of one sequence; a token row is D/8
+// lanes of 16 bytes; each thread walks the heads with four rows in flight.
+// Persistent CTAs (one wave) stride over the B * ceil(T / TPB) tiles.
 template <int D>
 __global__ void __launch_bounds__(kAbsThreads) k_token_absmax(const uint4* __restrict__ x, uint16_t* key, int H,
-                                                              int T, long long rows) {
+                                                              int T, int tiles_per_seq, int n_tiles) {
   constexpr int LPT = D / 8;
   constexpr int TPB = kAbsThreads / LPT;
   const int c = threadIdx.x % LPT;
   const size_t hs = static_cast<size_t>(T) * LPT;  // uint4 per head slice
-  const long long r_beg = rows * blockIdx.x / gridDim.x, r_end = rows * (blockIdx.x + 1) / gridDim.x;
-  for (long long r0 = r_beg; r0 < r_end; r0 += TPB) {  // the same trip count for the CTA's threads
-    const long long r = r0 + static_cast<int>(threadIdx.x) / LPT;
+  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const int b = tile / tiles_per_seq;
+    const int t = (tile - b * tiles_per_seq) * TPB + static_cast<int>(threadIdx.x) / LPT;
     uint32_t m = 0;
-    if (r < r_end) {
-      const int b = static_cast<int>(r / T), t = static_cast<int>(r - static_cast<long long>(b) * T);
+    if (t < T) {
       const uint4* p = x + (static_cast<size_t>(b) * H * T + t) * LPT + c;
       int h = 0;
       for (; h + 4 <= H; h += 4) {
-        uint4 rr[4];
+        uint4 r[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) rr[u] = __ldcs(p + (h + u) * hs);
+        for (int u = 0; u < 4; ++u) r[u] = __ldcs(p + (h + u) * hs);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) m = max(m, mag_max8(rr[u]));
+        for (int u = 0; u < 4; ++u) m = max(m, mag_max8(r[u]));
       }
       for (; h < H; ++h) m = max(m, mag_max8(__ldcs(p + h * hs)));
     }
 #pragma unroll
     for (int o = LPT / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (c == 0 && r < r_end) key[r] = static_cast<uint16_t>(m);
+    if (c == 0 && t < T) key[static_cast<size_t>(b) * T + t] = static_cast<uint16_t>(m);
   }
 }
 
@@ -388,13 +386,15 @@ kvq_status launch_detect_sinks(const kvq_desc& d, const void* x, double tau, int
   uint16_t* key = static_cast<uint16_t*>(ws);
   const int D = d.head_dim;
   const int tpb = kAbsThreads / (D / 8);
-  const long long rows = static_cast<long long>(d.batch) * d.tokens;
-  const long long n_tiles = (rows + tpb - 1) / tpb;
+  const long long tiles_per_seq = (d.tokens + tpb - 1) / tpb;
+  const long long n_tiles = tiles_per_seq * d.batch;
+  if (n_tiles >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
   const auto fn = D == 128 ? k_token_absmax<128> : k_token_absmax<64>;
   const int per_sm = occupancy_once(reinterpret_cast<const void*>(fn), kAbsThreads, 0);
   const long long wave = static_cast<long long>(num_sms) * per_sm;
   const unsigned grid = static_cast<unsigned>(n_tiles < wave ? n_tiles : wave);
-  fn<<<grid, kAbsThreads, 0, st>>>(static_cast<const uint4*>(x), key, d.heads, d.tokens, rows);
+  fn<<<grid, kAbsThreads, 0, st>>>(static_cast<const uint4*>(x), key, d.heads, d.tokens,
+                                   static_cast<int>(tiles_per_seq), static_cast<int>(n_tiles));
   if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
   SelArgs a{d.tokens, d.t0, max_sinks, tau, key, sink_pos, count};
   // stage a sequence's keys in shared memory when they fit in 96 KB
