@@ -116,41 +116,18 @@ __device__ __forceinline__ uint32_t cb_code(float w, const float* beta) {
 // boundary is chosen by selects on the bits found so far, so there is no
 // data-dependent shared-memory load.
 template <int NL>
-__device__ __forceinline__ uint32_t cb_code_reg(float w, const float* b) {
-  static_assert(NL == 4 || NL == 8 || NL == 16, "2-, 3- or 4-bit codes");
+__device__ __forceinline__ uint32_t cb_code_reg(float w, const float (&b)[NL > 1 ? NL - 1 : 1]) {
+  static_assert(NL == 4 || NL == 8, "2- or 3-bit codes");
   if constexpr (NL == 4) {
     const bool hi = w > b[1];
     const bool lo = w > (hi ? b[2] : b[0]);
     return (hi ? 2u : 0u) + (lo ? 1u : 0u);
-  } else if constexpr (NL == 8) {
+  } else {
     const bool b2 = w > b[3];
     const bool b1 = w > (b2 ? b[5] : b[1]);
     const float t = b2 ? (b1 ? b[6] : b[4]) : (b1 ? b[2] : b[0]);
     const bool b0 = w > t;
     return (b2 ? 4u : 0u) + (b1 ? 2u : 0u) + (b0 ? 1u : 0u);
-  } else {
-    const bool b3 = w > b[7];
-    const bool b2 = w > (b3 ? b[11] : b[3]);
-    const float t1 = b3 ? (b2 ? b[13] : b[9]) : (b2 ? b[5] : b[1]);
-    const bool b1 = w > t1;
-    const float t0 = b3 ? (b2 ? (b1 ? b[14] : b[12]) : (b1 ? b[10] : b[8]))
-                        : (b2 ? (b1 ? b[6] : b[4]) : (b1 ? b[2] : b[0]));
-    const bool b0 = w > t0;
-    return (b3 ? 8u : 0u) + (b2 ? 4u : 0u) + (b1 ? 2u : 0u) + (b0 ? 1u : 0u);
-  }
-}
-
-// The channel's boundary row of the shared-memory table (2 NL floats, 16-byte
-// aligned) into registers: the first n - 1 entries are the boundaries.
-template <int N>
-__device__ __forceinline__ void ld_row(const float* row, float (&b)[N]) {
-#pragma unroll
-  for (int i = 0; i < N / 4; ++i) {
-    const float4 v = *reinterpret_cast<const float4*>(row + 4 * i);
-    b[4 * i] = v.x;
-    b[4 * i + 1] = v.y;
-    b[4 * i + 2] = v.z;
-    b[4 * i + 3] = v.w;
   }
 }
 
@@ -456,17 +433,7 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
     iso_rotate_chunks<D, SO3>(ld, inv, Ms, [&](int j, float wj) {
       uint32_t c;
       const bool wide = (wd[j >> 5] >> (j & 31)) & 1u;
-      if constexpr (DYN == 2 && NL <= 8) {  // the channel's boundaries from shared memory, into registers
-        if (wide) {
-          float b[2 * NL];
-          ld_row<2 * NL>(tab + j * 2 * NL, b);
-          c = cb_code_reg<2 * NL>(wj, b);
-        } else {
-          float b[NL];
-          ld_row<NL>(tab + j * 2 * NL, b);
-          c = cb_code_reg<NL>(wj, b);
-        }
-      } else if constexpr (DYN == 2) {
+      if constexpr (DYN == 2) {  // the channel's boundaries from shared memory
         c = wide ? cb_code<2 * NL>(wj, tab + j * 2 * NL) : cb_code<NL>(wj, tab + j * 2 * NL);
       } else {
         const float sj = __ldg(sc + j);
