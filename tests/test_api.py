@@ -213,3 +213,54 @@ def test_freq_aware_rope_table_matches_oracle(orc, d):
     buf = torch.empty(4 * 12).data_ptr()
     assert K.kvq_rope_table_ex(buf, 4, 12, 10000.0, K.KVQ_ROPE_FREQ_AWARE) == K.KVQ_ERR_INVALID  # not a multiple of 8
     assert K.kvq_rope_table_ex(buf, 4, 8, 10000.0, 7) == K.KVQ_ERR_INVALID
+
+
+def test_sink_and_codebook_entry_point_checks():
+    """Argument checks of the detection, sink-list and dynamic-codebook entry
+    points (all host-side: nothing is launched)."""
+    d = _desc(head_dim=64, group=64)
+    ws_need = K.kvq_detect_sinks_workspace_bytes(d)
+    assert ws_need == (2 * 16 * 2 + 15) // 16 * 16
+    assert K.kvq_detect_sinks(d, None, 2.0, 4, 256, 0, 256, ws_need, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_detect_sinks(d, 256, float("nan"), 4, 256, 0, 256, ws_need, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_detect_sinks(d, 256, 2.0, 0, 256, 0, 256, ws_need, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_detect_sinks(d, 256, 2.0, 70000, 256, 0, 256, ws_need, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_detect_sinks(d, 256, 2.0, 4, 256, 0, 256, ws_need - 16, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_detect_sinks(d, 264, 2.0, 4, 256, 0, 256, ws_need, 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_detect_sinks(d, 256, 2.0, 4, 258, 0, 256, ws_need, 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_detect_sinks(_desc(tokens=0), 256, 2.0, 4, 256, 0, 256, 64, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_detect_sinks_workspace_bytes(_desc(batch=0)) == 0
+    # a sink list must be 4-byte aligned
+    tb = K.kvq_tables()
+    tb.sink_pos = 258
+    ds = _desc(n_sink=2)
+    assert K.kvq_encode(ds, 256, tb, _packed(ds, sink=256), 0) == K.KVQ_ERR_ALIGN
+    # dynamic codebooks: IsoQuant rotations only; tables and the ext field required
+    dd = _desc(rot="iso", quant="codebook_dyn", bits=3)
+    assert K.kvq_calibrate_codebook_workspace_bytes(_desc()) == 0  # not an IsoQuant rotation
+    nb = K.kvq_calibrate_codebook_workspace_bytes(dd)
+    assert nb >= 2 * 8 * 1 * 128 * 8
+    t = K.kvq_tables()
+    assert K.kvq_calibrate_codebook(dd, 256, t, 256, 256, 256, nb, 0) == K.KVQ_ERR_INVALID  # no qL/qR
+    t.qL, t.qR = 256, 256
+    assert K.kvq_calibrate_codebook(dd, 256, t, 256, 256, 256, nb - 8, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_calibrate_codebook(dd, 256, t, 260, 256, 256, nb, 0) == K.KVQ_ERR_ALIGN
+    assert K.kvq_calibrate_codebook(_desc(), 256, t, 256, 256, 256, nb, 0) == K.KVQ_ERR_UNSUPPORTED
+    t.codebook = 256
+    p = _packed(dd, norm=256)
+    assert K.kvq_encode(dd, 256, t, p, 0) == K.KVQ_ERR_INVALID  # no wide codebook / scales / masks
+    t.codebook_wide, t.ch_scale, t.ch_wide = 256, 256, 256
+    assert K.kvq_encode(dd, 256, t, p, 0) == K.KVQ_ERR_INVALID  # no ext field
+    assert K.kvq_packed_bytes(dd, K.KVQ_FIELD_EXT) == 2 * 8 * 16 * 2
+    assert K.kvq_packed_bytes(_desc(), K.KVQ_FIELD_EXT) == 0
+    assert K.kvq_lloyd_max_codebook(np.zeros(32, np.float32).ctypes.data, 5, 1) == K.KVQ_OK
+    assert K.kvq_lloyd_max_codebook(np.zeros(64, np.float32).ctypes.data, 6, 1) == K.KVQ_ERR_INVALID
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5])
+def test_unit_normal_codebook_matches_oracle(orc, bits):
+    """The N(0,1) levels (head_dim 1) that the dynamic codebooks scale, up to
+    the 5-bit wide codebook of 4-bit codes, bit-equal to the oracle's."""
+    host = np.zeros(1 << bits, np.float32)
+    assert K.kvq_lloyd_max_codebook(host.ctypes.data, bits, 1) == K.KVQ_OK
+    assert np.array_equal(host, orc.codebook(bits, 1))
