@@ -56,7 +56,7 @@ class KvqError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m kv_cache_rotation_b200.build` "
+        raise ImportError(f"{LIB_PATH} is not built; run `python kv_cache_rotation_b200/build.py` "
                           "(there is no CPU fallback)")
     L = ctypes.CDLL(LIB_PATH)
     P = ctypes.POINTER
