@@ -31,7 +31,7 @@ namespace kvq {
 namespace {
 
 constexpr int kAbsThreads = 256;
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 1024;
 
 __device__ __forceinline__ uint32_t mag_max8(uint4 r) {
   const uint32_t m = __vmaxu2(__vmaxu2(r.x & 0x7fff7fffu, r.y & 0x7fff7fffu),
