@@ -434,7 +434,13 @@ __global__ void __launch_bounds__(128) k_encode_iso(const __grid_constant__ CUte
       uint32_t c;
       const bool wide = (wd[j >> 5] >> (j & 31)) & 1u;
       if constexpr (DYN == 2) {  // the channel's boundaries from shared memory
-        c = wide ? cb_code<2 * NL>(wj, tab + j * 2 * NL) : cb_code<NL>(wj, tab + j * 2 * NL);
+        // one code path for both codebook sizes: the wide channels take the first
+        // step of the 2 NL search (boundary NL - 1), then both run the NL steps
+        const float* row = tab + j * 2 * NL;
+        c = (wide && wj > row[NL - 1]) ? static_cast<uint32_t>(NL) : 0u;
+#pragma unroll
+        for (int st = NL / 2; st >= 1; st >>= 1)
+          if (wj > row[c + st - 1]) c += st;
       } else {
         const float sj = __ldg(sc + j);
         c = wide ? dyn_code<2 * NL>(wj, sj, lvw) : dyn_code<NL>(wj, sj, beta);
