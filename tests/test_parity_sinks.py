@@ -54,6 +54,9 @@ DETECT = [
     ("one_token", 1, 4, 1, 128, 5, 1.0, 2, 1),
     ("two_tokens", 1, 2, 2, 64, 0, 0.5, 4, 1),
     ("heads_not_multiple_of_4", 2, 3, 100, 128, 0, 8.0, 8, 3),
+    # more keys than the selection stages in shared memory (49152): read from global memory
+    ("long_unstaged", 2, 1, 50000, 64, 7, 3.0, 16, 6),
+    ("long_unstaged_capped", 1, 2, 60000, 64, 0, 1.0, 12, 0),
 ]
 
 
