@@ -90,3 +90,33 @@ def test_sink_detection_and_dynamic_tables_repeat(TA):
     tb = TA.make_tables(qL=torch.from_numpy(qL).cuda(), qR=torch.from_numpy(qR).cuda())
     (c1, c2) = _twice(lambda: tuple(t.clone() for t in TA.calibrate_codebook(d, x, tb)))
     assert torch.equal(c1[0], c2[0]) and torch.equal(c1[1], c2[1])
+
+
+def test_isoquant_repeat(TA):
+    """Fixed (SO(4), 3-D) and dynamic codebooks: encode and decode twice, same bytes."""
+    B, H, T, D, bits = 2, 2, 300, 128, 3
+    w = W.Workload("det_iso", B=B, H=H, T=T, D=D, dist="student_t", seed=3)
+    x = torch.from_numpy(W.kv_tensor(w, "k")).cuda()
+    qL4, qR4 = W.unit_quaternions(D // 4, 3, 30), W.unit_quaternions(D // 4, 3, 31)
+    for rot, quant in (("iso", "codebook"), ("iso3", "codebook"), ("iso", "codebook_dyn")):
+        d = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, bits=bits, rot=rot, quant=quant)
+        qL = W.iso3_tables(D, 5) if rot == "iso3" else qL4
+        tb = TA.make_tables(qL=torch.from_numpy(qL).cuda(),
+                            qR=torch.from_numpy(qR4).cuda() if rot == "iso" else None)
+        if quant == "codebook_dyn":
+            tb.codebook = TA.lloyd_max_codebook(bits, 1)
+            tb.codebook_wide = TA.lloyd_max_codebook(bits + 1, 1)
+            tb.ch_scale, tb.ch_wide = TA.calibrate_codebook(d, x, tb)
+        else:
+            tb.codebook = TA.lloyd_max_codebook(bits, D)
+
+        def run():
+            pk = TA.alloc_packed(d, zero=False)
+            TA.encode(d, x, tb, pk)
+            out = torch.empty((B, H, T, D), dtype=torch.float32, device="cuda")
+            TA.decode(d, pk, tb, out)
+            return pk, out
+        (p1, o1), (p2, o2) = _twice(run)
+        assert torch.equal(p1.codes, p2.codes) and torch.equal(p1.norm, p2.norm) and torch.equal(o1, o2)
+        if quant == "codebook_dyn":
+            assert torch.equal(p1.ext, p2.ext)
