@@ -41,6 +41,9 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 512 << 20
 
 
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e specification (context beside the measured copy bandwidth)
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -165,6 +168,7 @@ class Step:
             "encode_k": nvec * 2 * D, "encode_v": nvec * 2 * D, "decode_k": nvec * 2 * D, "decode_v": nvec * 2 * D,
             "append": self.sc.fp16_append, "score": self.sc.fp16_score,
         }
+        self.tokens = {"encode_k": B * T, "encode_v": B * T, "decode_k": B * T, "decode_v": B * T, "append": B}
         self.kernels = {"encode_k": "k_encode_group", "encode_v": "k_encode_group", "decode_k": "k_decode_group",
                         "decode_v": "k_decode_group", "append": "k_encode_head", "score": "k_score_mma"}
         self.fp32_ops = {n: nvec * D * fp32_ops_per_element("fwht_group", n, wg.group_heads, D)
@@ -402,6 +406,7 @@ class EncDecStep:
         tensors = ["k", "v"] if both and not iso else ["k"]
         self.items = []
         self.alg, self.fp16_equiv, self.kernels, self.fp32_ops = {}, {}, {}, {}
+        self.tokens = {}
         kern = {"fwht_head": "head", "none": "head", "fwht_group": "group", "iso": "iso", "iso3": "iso"}[w.rot]
         for which in tensors:
             x = (W.kv_tensor_device(w, which, device) if iso else torch.from_numpy(W.kv_tensor(w, which)).to(device))
@@ -433,6 +438,7 @@ class EncDecStep:
                 per_vec += 2  # the outlier channels' top bits
             self.alg[f"encode_{which}"] = nvec * (2 * D + per_vec) + (B * H * w.n_sink * D * 2)
             self.alg[f"decode_{which}"] = nvec * (2 * D + per_vec)
+            self.tokens[f"encode_{which}"] = self.tokens[f"decode_{which}"] = B * T
             self.fp16_equiv[f"encode_{which}"] = nvec * 2 * D
             self.fp16_equiv[f"decode_{which}"] = nvec * 2 * D
             self.kernels[f"encode_{which}"] = f"k_encode_{kern}"
@@ -756,7 +762,11 @@ def run_ours(args):
         ms = per_kernel[n] / args.steps
         kernels[n] = {"ms": ms, "fp16_gbs": st.fp16_equiv[n] / (ms / 1e3) / 1e9,
                       "alg_gbs": st.alg[n] / (ms / 1e3) / 1e9,
-                      "frac_of_measured_hbm": st.alg[n] / (ms / 1e3) / 1e9 / peak}
+                      "frac_of_measured_hbm": st.alg[n] / (ms / 1e3) / 1e9 / peak,
+                      "frac_of_spec_8tbs": st.alg[n] / (ms / 1e3) / 1e9 / SPEC_HBM_GBS}
+        tok = getattr(st, "tokens", {}).get(n)
+        if tok:  # token positions of one tensor (B x T) processed per second
+            kernels[n]["tokens_per_s"] = tok / (ms / 1e3)
     dom = max(st.names, key=lambda n: per_kernel[n])
     dom_ms = per_kernel[dom] / args.steps
     achieved = st.alg[dom] / (dom_ms / 1e3) / 1e9
