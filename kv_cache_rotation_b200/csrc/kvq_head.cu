@@ -91,10 +91,13 @@ __device__ __forceinline__ void ld_run(const uint8_t* p, uint32_t* w) {
 }
 __host__ __device__ constexpr int pow2_align(int n) { return (n & 15) == 0 ? 16 : (n & 7) == 0 ? 8 : 4; }
 
-// (b * H + h, h, token) of vector v, ordered (batch, head, token) without RoPE
-// and (batch, token, head) with it.
+// (b * H + h, h, token) of vector v, ordered (batch, token, head) for RoPE
+// without a permutation (the heads of a token share one (cos, sin) row in L1)
+// and (batch, head, token) otherwise (a warp's 16 vectors share one
+// permutation, so its gather is conflict-free; with RoPE their 16 rows are
+// staged by stage_rope_rows).
 __device__ __forceinline__ void vec_coords(const HeadArgs& a, uint32_t v, uint32_t& bh, int& h, int& tt) {
-  if (a.rope) {
+  if (a.rope && !a.perm) {
     const uint32_t bt = a.div_h.div(v);
     h = static_cast<int>(a.div_h.mod(v, bt));
     const uint32_t b = a.div_t.div(bt);
@@ -105,6 +108,31 @@ __device__ __forceinline__ void vec_coords(const HeadArgs& a, uint32_t v, uint32
     tt = static_cast<int>(a.div_t.mod(v, bh));
     h = static_cast<int>(a.div_h.mod(bh, a.div_h.div(bh)));
   }
+}
+
+// The (cos, sin) rows of the warp's 16 vectors into its row buffer (row k <-
+// the position of slot k, taken from lane 2k), all lanes loading one row per
+// step so every load is coalesced; 8-byte stores (rows are 8-byte aligned).
+template <int D>
+__device__ __forceinline__ void stage_rope_rows(const HeadArgs& a, uint32_t wbuf, int m, int lane) {
+  constexpr int CH = D * 4 / 16;  // 16-byte chunks of a row: 32 (D = 128) or 16 (D = 64)
+#pragma unroll 4
+  for (int k = 0; k < kVecW; ++k) {
+    const int mk = __shfl_sync(0xffffffffu, m, 2 * k);
+    if (lane < CH) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(mk) * D) + lane);
+      const uint32_t dst = wbuf + k * row_pitch<D>() + 16 * lane;
+      sts64(dst, v.x, v.y);
+      sts64(dst + 8, v.z, v.w);
+    }
+  }
+  __syncwarp();
+}
+
+// 16 bytes of this lane's staged (cos, sin) row at byte offset off.
+__device__ __forceinline__ uint4 staged_cs(uint32_t row, int off) {
+  const uint2 lo = lds64(row + off), hi = lds64(row + off + 8);
+  return make_uint4(lo.x, lo.y, hi.x, hi.y);
 }
 
 template <int D, int BITS, int G, bool ROT>
@@ -151,11 +179,14 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
       P[2 * g] = f2(h01.x, h23.x);
       P[2 * g + 1] = f2(h01.y, h23.y);
     }
+    const bool staged = a.rope && a.perm;  // the warp's (cos, sin) rows in its row buffer
+    if (staged) stage_rope_rows<D>(a, row - slot * row_pitch<D>(), m, lane);
     if (a.rope == 1) {  // pairs (2i, 2i+1): y0 = fma(x0, c, -(x1*s)), y1 = fma(x0, s, x1*c)
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D) + (V / 4) * s;
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
-        const uint4 cv = __ldg(rp + g);  // (c, s) of pairs 2g and 2g+1 of this lane
+        // (c, s) of pairs 2g and 2g+1 of this lane
+        const uint4 cv = staged ? staged_cs(row, 16 * ((V / 4) * s + g)) : __ldg(rp + g);
         const float2 cc = f2(__uint_as_float(cv.x), __uint_as_float(cv.z));
         const float2 ss = f2(__uint_as_float(cv.y), __uint_as_float(cv.w));
         const float2 x0 = P[2 * g], x1 = P[2 * g + 1];
@@ -166,7 +197,9 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D);
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
-        const uint4 c0 = __ldg(rp + 2 * g), c1 = __ldg(rp + 2 * g + 1);  // angles 4g .. 4g+1, 4g+2 .. 4g+3
+        // angles 4g .. 4g+1, 4g+2 .. 4g+3
+        const uint4 c0 = staged ? staged_cs(row, 32 * g) : __ldg(rp + 2 * g);
+        const uint4 c1 = staged ? staged_cs(row, 32 * g + 16) : __ldg(rp + 2 * g + 1);
         // P[2g] holds local channels 4g, 4g+2; P[2g+1] holds 4g+1, 4g+3
         P[2 * g] = rope_half_fwd2(P[2 * g], f2(__uint_as_float(c0.x), __uint_as_float(c1.x)),
                                   f2(__uint_as_float(c0.y), __uint_as_float(c1.y)), s != 0, 1);
@@ -175,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
       }
     }
     if (a.perm) {  // p_j = y_perm[h][j]: stage the row, gather
+      if (staged) __syncwarp();  // every lane has read its (cos, sin) row
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
         sts64(row + 4 * (V * s + 4 * g), __float_as_uint(P[2 * g].x), __float_as_uint(P[2 * g + 1].x));
@@ -375,11 +409,13 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
       }
       __syncwarp();  // the row buffer is free for the next step
     }
+    const bool staged = a.rope && a.perm;  // the warp's (cos, sin) rows in its row buffer
+    if (staged) stage_rope_rows<D>(a, row - slot * row_pitch<D>(), m, lane);
     if (a.rope == 1) {  // inverse pairs: x0 = y0 c + y1 s, x1 = y1 c - y0 s
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D) + (V / 4) * s;
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
-        const uint4 cv = __ldg(rp + g);
+        const uint4 cv = staged ? staged_cs(row, 16 * ((V / 4) * s + g)) : __ldg(rp + g);
         const float2 cc = f2(__uint_as_float(cv.x), __uint_as_float(cv.z));
         const float2 ss = f2(__uint_as_float(cv.y), __uint_as_float(cv.w));
         const float2 y0 = P[2 * g], y1 = P[2 * g + 1];
@@ -390,13 +426,15 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D);
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
-        const uint4 c0 = __ldg(rp + 2 * g), c1 = __ldg(rp + 2 * g + 1);
+        const uint4 c0 = staged ? staged_cs(row, 32 * g) : __ldg(rp + 2 * g);
+        const uint4 c1 = staged ? staged_cs(row, 32 * g + 16) : __ldg(rp + 2 * g + 1);
         P[2 * g] = rope_half_inv2(P[2 * g], f2(__uint_as_float(c0.x), __uint_as_float(c1.x)),
                                   f2(__uint_as_float(c0.y), __uint_as_float(c1.y)), s != 0, 1);
         P[2 * g + 1] = rope_half_inv2(P[2 * g + 1], f2(__uint_as_float(c0.z), __uint_as_float(c1.z)),
                                       f2(__uint_as_float(c0.w), __uint_as_float(c1.w)), s != 0, 1);
       }
     }
+    if (staged) __syncwarp();  // every lane has read its (cos, sin) row: the buffer is free
     // output words of this lane's half row (a sink slot comes back verbatim)
     uint32_t ow[V * ES / 4];
     if (sink_tok) {
