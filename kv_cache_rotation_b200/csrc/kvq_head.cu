@@ -110,29 +110,40 @@ __device__ __forceinline__ void vec_coords(const HeadArgs& a, uint32_t v, uint32
   }
 }
 
-// The (cos, sin) rows of the warp's 16 vectors into its row buffer (row k <-
-// the position of slot k, taken from lane 2k), all lanes loading one row per
-// step so every load is coalesced; 8-byte stores (rows are 8-byte aligned).
+// Staged (cos, sin) rows: 16-byte aligned rows of D floats.
 template <int D>
-__device__ __forceinline__ void stage_rope_rows(const HeadArgs& a, uint32_t wbuf, int m, int lane) {
-  constexpr int CH = D * 4 / 16;  // 16-byte chunks of a row: 32 (D = 128) or 16 (D = 64)
-#pragma unroll 4
-  for (int k = 0; k < kVecW; ++k) {
-    const int mk = __shfl_sync(0xffffffffu, m, 2 * k);
-    if (lane < CH) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(mk) * D) + lane);
-      const uint32_t dst = wbuf + k * row_pitch<D>() + 16 * lane;
-      sts64(dst, v.x, v.y);
-      sts64(dst + 8, v.z, v.w);
-    }
-  }
-  __syncwarp();
+__host__ __device__ constexpr uint32_t cs_pitch() {
+  return D * 4 + 16;
+}
+// Per-warp shared memory: encode keeps the permutation rows and the staged
+// (cos, sin) rows in one buffer (they are used one after the other); decode
+// needs both at once (the rows are staged while the permutation is applied).
+template <int D>
+__host__ __device__ constexpr uint32_t warp_buf(bool enc) {
+  return enc ? kVecW * cs_pitch<D>() : kVecW * (row_pitch<D>() + cs_pitch<D>());
 }
 
-// 16 bytes of this lane's staged (cos, sin) row at byte offset off.
-__device__ __forceinline__ uint4 staged_cs(uint32_t row, int off) {
-  const uint2 lo = lds64(row + off), hi = lds64(row + off + 8);
-  return make_uint4(lo.x, lo.y, hi.x, hi.y);
+// Start copying the (cos, sin) rows of the warp's 16 vectors into cs rows at
+// csbuf (row k <- the position of slot k, taken from lane 2k): every lane
+// copies one 16-byte chunk of every row, so each row is one coalesced
+// transfer; cp.async keeps all 16 in flight without registers.
+template <int D>
+__device__ __forceinline__ void stage_rope_rows(const HeadArgs& a, uint32_t csbuf, int m, int lane) {
+  constexpr int CH = D * 4 / 16;  // 16-byte chunks of a row: 32 (D = 128) or 16 (D = 64)
+#pragma unroll
+  for (int k = 0; k < kVecW; ++k) {
+    const int mk = __shfl_sync(0xffffffffu, m, 2 * k);
+    if (lane < CH)
+      cp_async16(csbuf + k * cs_pitch<D>() + 16 * lane,
+                 reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(mk) * D) + lane, 16);
+  }
+  cp_async_commit();
+}
+
+// The staged rows have landed and every lane sees them.
+__device__ __forceinline__ void staged_rows_ready() {
+  cp_async_wait_all();
+  __syncwarp();
 }
 
 template <int D, int BITS, int G, bool ROT>
@@ -148,9 +159,12 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
   extern __shared__ uint8_t smem_raw[];  // permutation rows: 16 x D floats per warp
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = lane & 1, slot = lane >> 1;
-  const uint32_t row = smem_u32(smem_raw) + (warp * kVecW + slot) * row_pitch<D>();
+  const uint32_t wbuf = smem_u32(smem_raw) + warp * warp_buf<D>(true);
+  const uint32_t row = wbuf + slot * row_pitch<D>();   // permutation staging
+  const uint32_t csrow = wbuf + slot * cs_pitch<D>();  // staged (cos, sin) row, same buffer
   const float r = a.rscale;
   const bool v8 = a.v8 != 0;
+  const bool staged = a.rope && a.perm;  // the warp's (cos, sin) rows in its buffer
   const uint32_t gw = blockIdx.x * (kThreads / 32) + warp, nw = gridDim.x * (kThreads / 32);
 
   for (uint32_t base = gw * kVecW; base < a.n_vec; base += nw * kVecW) {
@@ -162,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
     const int m = a.t0 + tt;
     const size_t vec = bh;
     const bool sink_tok = m < a.n_sink;
+    if (staged) stage_rope_rows<D>(a, wbuf, m, lane);  // in flight while the row loads
 
     uint32_t raw[V / 2];
     ld_row<V / 2>(a.x + (vec * a.T + tt) * D + V * s, v8, raw);
@@ -179,14 +194,13 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
       P[2 * g] = f2(h01.x, h23.x);
       P[2 * g + 1] = f2(h01.y, h23.y);
     }
-    const bool staged = a.rope && a.perm;  // the warp's (cos, sin) rows in its row buffer
-    if (staged) stage_rope_rows<D>(a, row - slot * row_pitch<D>(), m, lane);
+    if (staged) staged_rows_ready();
     if (a.rope == 1) {  // pairs (2i, 2i+1): y0 = fma(x0, c, -(x1*s)), y1 = fma(x0, s, x1*c)
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D) + (V / 4) * s;
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
         // (c, s) of pairs 2g and 2g+1 of this lane
-        const uint4 cv = staged ? staged_cs(row, 16 * ((V / 4) * s + g)) : __ldg(rp + g);
+        const uint4 cv = staged ? lds128(csrow + 16 * ((V / 4) * s + g)) : __ldg(rp + g);
         const float2 cc = f2(__uint_as_float(cv.x), __uint_as_float(cv.z));
         const float2 ss = f2(__uint_as_float(cv.y), __uint_as_float(cv.w));
         const float2 x0 = P[2 * g], x1 = P[2 * g + 1];
@@ -198,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
         // angles 4g .. 4g+1, 4g+2 .. 4g+3
-        const uint4 c0 = staged ? staged_cs(row, 32 * g) : __ldg(rp + 2 * g);
-        const uint4 c1 = staged ? staged_cs(row, 32 * g + 16) : __ldg(rp + 2 * g + 1);
+        const uint4 c0 = staged ? lds128(csrow + 32 * g) : __ldg(rp + 2 * g);
+        const uint4 c1 = staged ? lds128(csrow + 32 * g + 16) : __ldg(rp + 2 * g + 1);
         // P[2g] holds local channels 4g, 4g+2; P[2g+1] holds 4g+1, 4g+3
         P[2 * g] = rope_half_fwd2(P[2 * g], f2(__uint_as_float(c0.x), __uint_as_float(c1.x)),
                                   f2(__uint_as_float(c0.y), __uint_as_float(c1.y)), s != 0, 1);
@@ -332,9 +346,13 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = lane & 1, slot = lane >> 1;
-  const uint32_t row = smem_u32(smem_raw) + (warp * kVecW + slot) * row_pitch<D>();
+  const uint32_t wbuf = smem_u32(smem_raw) + warp * warp_buf<D>(false);
+  const uint32_t row = wbuf + slot * row_pitch<D>();  // permutation staging
+  const uint32_t csbuf = wbuf + kVecW * row_pitch<D>();
+  const uint32_t csrow = csbuf + slot * cs_pitch<D>();  // staged (cos, sin) row
   const float r = a.rscale;
   const bool v8 = a.v8 != 0;
+  const bool staged = a.rope && a.perm;  // the warp's (cos, sin) rows in its buffer
   const uint32_t gw = blockIdx.x * (kThreads / 32) + warp, nw = gridDim.x * (kThreads / 32);
 
   for (uint32_t base = gw * kVecW; base < a.n_vec; base += nw * kVecW) {
@@ -347,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
     const size_t vec = bh;
     const size_t slot_i = vec * a.t_cap + m;
     const bool sink_tok = m < a.n_sink;
+    if (staged) stage_rope_rows<D>(a, csbuf, m, lane);  // in flight while the codes are decoded
 
     uint32_t w[NW];
     ld_run<NBY, pow2_align(NBY)>(a.codes + slot_i * RB + NBY * s, w);
@@ -409,13 +428,12 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
       }
       __syncwarp();  // the row buffer is free for the next step
     }
-    const bool staged = a.rope && a.perm;  // the warp's (cos, sin) rows in its row buffer
-    if (staged) stage_rope_rows<D>(a, row - slot * row_pitch<D>(), m, lane);
+    if (staged) staged_rows_ready();
     if (a.rope == 1) {  // inverse pairs: x0 = y0 c + y1 s, x1 = y1 c - y0 s
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D) + (V / 4) * s;
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
-        const uint4 cv = staged ? staged_cs(row, 16 * ((V / 4) * s + g)) : __ldg(rp + g);
+        const uint4 cv = staged ? lds128(csrow + 16 * ((V / 4) * s + g)) : __ldg(rp + g);
         const float2 cc = f2(__uint_as_float(cv.x), __uint_as_float(cv.z));
         const float2 ss = f2(__uint_as_float(cv.y), __uint_as_float(cv.w));
         const float2 y0 = P[2 * g], y1 = P[2 * g + 1];
@@ -426,8 +444,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
       const uint4* rp = reinterpret_cast<const uint4*>(a.rope_cs + static_cast<size_t>(m) * D);
 #pragma unroll
       for (int g = 0; g < V / 4; ++g) {
-        const uint4 c0 = staged ? staged_cs(row, 32 * g) : __ldg(rp + 2 * g);
-        const uint4 c1 = staged ? staged_cs(row, 32 * g + 16) : __ldg(rp + 2 * g + 1);
+        const uint4 c0 = staged ? lds128(csrow + 32 * g) : __ldg(rp + 2 * g);
+        const uint4 c1 = staged ? lds128(csrow + 32 * g + 16) : __ldg(rp + 2 * g + 1);
         P[2 * g] = rope_half_inv2(P[2 * g], f2(__uint_as_float(c0.x), __uint_as_float(c1.x)),
                                   f2(__uint_as_float(c0.y), __uint_as_float(c1.y)), s != 0, 1);
         P[2 * g + 1] = rope_half_inv2(P[2 * g + 1], f2(__uint_as_float(c0.z), __uint_as_float(c1.z)),
@@ -474,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
 
 template <int D, int BITS, int G, bool ROT>
 kvq_status run(bool enc, const HeadArgs& a, int out_fp32, const LaunchCtx& ctx, cudaStream_t st) {
-  const size_t smem = a.perm ? static_cast<size_t>(kThreads / 32) * kVecW * row_pitch<D>() : 0;
+  const size_t smem = a.perm ? static_cast<size_t>(kThreads / 32) * warp_buf<D>(enc) : 0;
   const void* fn = enc        ? reinterpret_cast<const void*>(k_encode_head<D, BITS, G, ROT>)
                    : out_fp32 ? reinterpret_cast<const void*>(k_decode_head<D, BITS, G, ROT, true>)
                               : reinterpret_cast<const void*>(k_decode_head<D, BITS, G, ROT, false>);
