@@ -503,6 +503,29 @@ class DecodeScoreStep:
         return [self.sc.append, self.sc.score]
 
 
+class LiteralScoreStep:
+    """Both forms of the decode-step score over one prefilled head-variant cache:
+    the query-rotation kernel and the literal form that decodes every key
+    (unpack, dequantize, inverse FWHT) before the dot product."""
+
+    def __init__(self, workload, device):
+        import torch
+        self.workload = workload
+        base = workload[:-len("_literal")]
+        self.sc = ScoreCache(W.WORKLOADS[base], device)
+        self.literal = self.sc.TA.bind_score(self.sc.d_pre, self.sc.q, self.sc.packed, self.sc.tables,
+                                             self.sc.n_tok, self.sc.scale, self.sc.scores, literal=True)
+        self.alg = {"score": self.sc.alg_score, "score_literal": self.sc.alg_score}
+        self.fp16_equiv = {"score": self.sc.fp16_score, "score_literal": self.sc.fp16_score}
+        self.kernels = {"score": "k_score_mma", "score_literal": "k_score_literal"}
+        self.fp32_ops = {}
+        self.names = list(self.alg)
+        torch.cuda.synchronize(device)
+
+    def launches(self):
+        return [self.sc.score, self.literal]
+
+
 def fp32_ops_per_element(rot, step, group_heads, D, rope=None):
     """Algorithmic fp32 operations per element of an encode/decode launch, in
     the oracle's order: FWHT log2(N) add/sub (N = D, or group_heads * D), RoPE
@@ -534,6 +557,8 @@ def make_step(workload, device, batch=None):
         return GroupScoreStep(device)
     if workload == "llama2_7b_sink_detect":
         return SinkDetectStep(device)
+    if workload.endswith("_score_literal"):
+        return LiteralScoreStep(workload, device)
     return EncDecStep(workload, device, batch=batch)
 
 
@@ -896,6 +921,12 @@ def _other_config(name, n_gpus):
         return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T,
                 "input": "keys fp16, RoPE'd before the abs-max (head-dim variant)", "n_sink": w.n_sink,
                 "l2": "no flush (the 268 MB input is larger than L2)", "parallelism": f"replicas x{n_gpus}"}
+    if name.endswith("_score_literal"):
+        c = _other_config(name[:-len("_literal")], n_gpus)
+        c["workload"] = name
+        c["forms"] = ("query rotation (k_score_mma) and the literal per-token decode + inverse FWHT "
+                      "(k_score_literal) over the same cache, timed one after the other")
+        return c
     w = W.WORKLOADS[name]
     return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T, "q_heads": w.Hq,
             "rotation": w.rot, "quant": w.quant, "bits": w.bits, "group": w.group, "n_sink": w.n_sink,
@@ -920,6 +951,7 @@ def main():
                     choices=["llama3_8b_gqa", "llama2_7b_mha", "isoquant_batch", "isoquant_so3_batch",
                              "isoquant_dyn_batch", "decode_score",
                              "llama3_8b_gqa_group_score", "llama2_7b_sink_detect",
+                             "decode_score_literal", "llama3_8b_gqa_score_literal",
                              "llama3_8b_gqa_attend", "llama3_8b_calibrate", "llama3_8b_pair_energy", "tiny"],
                     help="which workload a step runs (the headline line is llama3_8b_gqa)")
     ap.add_argument("--batch", type=int, default=None,

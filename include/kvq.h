@@ -195,6 +195,19 @@ kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kv
                      const kvq_tables* tb, int32_t n_tokens, float scale, float* scores,
                      kvq_stream_t stream);
 
+/* Decode-step score in its literal form ([EliteKV §2.2]; [RotateKV] 关键设计: the inverse
+ * rotation of the head-variant cache): the same scores as kvq_score, with every key decoded on
+ * the fly (unpack, dequantize, inverse FWHT per token) instead of transforming the query once.
+ * The channel permutation is applied to the query (sum_i q_i khat_i = sum_j q_perm[j] p_j).
+ * fp32 throughout (no integer query digits), so it is the reference form the query-rotation
+ * kernel is measured against, at several times its instruction count per element.
+ * Arguments, layouts and sinks (prefix or listed) as kvq_score. Supported for rot in
+ * {NONE, FWHT_HEAD}, head_dim 128, min-max codes, q_heads/H in {1, 2, 4, 8}; other shapes
+ * return KVQ_ERR_UNSUPPORTED. */
+kvq_status kvq_score_literal(const kvq_desc* d, const void* q, int32_t q_heads, const kvq_packed* cache,
+                             const kvq_tables* tb, int32_t n_tokens, float scale, float* scores,
+                             kvq_stream_t stream);
+
 /* Decode-step attention over the compressed cache ([EliteKV §2.2] scores; [EliteKV §7.1] the
  * softmax of the scaled scores weights the values):
  *   out[b][qh] = sum_n p_n vhat[b][h][n],  p = softmax_n(scale * <q[b][qh], khat[b][h][n]>),

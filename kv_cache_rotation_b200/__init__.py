@@ -22,7 +22,7 @@ KVQ_ROT_NONE, KVQ_ROT_FWHT_HEAD, KVQ_ROT_FWHT_GROUP, KVQ_ROT_ISO_SO4, KVQ_ROT_IS
 KVQ_Q_MINMAX, KVQ_Q_CODEBOOK, KVQ_Q_CODEBOOK_DYN = 0, 1, 2
 KVQ_FIELD_CODES, KVQ_FIELD_SCALE_ZERO, KVQ_FIELD_SINK, KVQ_FIELD_NORM, KVQ_FIELD_EXT = range(5)
 
-EXPORTED = ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_attend_workspace_bytes",
+EXPORTED = ("kvq_encode", "kvq_decode", "kvq_score", "kvq_score_literal", "kvq_attend", "kvq_attend_noalloc", "kvq_attend_workspace_bytes",
             "kvq_calibrate_perm", "kvq_calibrate_workspace_bytes", "kvq_pair_energy",
             "kvq_detect_sinks", "kvq_detect_sinks_workspace_bytes",
             "kvq_calibrate_codebook", "kvq_calibrate_codebook_workspace_bytes",
@@ -64,6 +64,7 @@ def _load():
     L.kvq_encode.argtypes = [P(kvq_desc), vp, P(kvq_tables), P(kvq_packed), st]
     L.kvq_decode.argtypes = [P(kvq_desc), P(kvq_packed), P(kvq_tables), vp, i32, st]
     L.kvq_score.argtypes = [P(kvq_desc), vp, i32, P(kvq_packed), P(kvq_tables), i32, ctypes.c_float, vp, st]
+    L.kvq_score_literal.argtypes = L.kvq_score.argtypes
     L.kvq_attend.argtypes = [P(kvq_desc), P(kvq_desc), vp, i32, P(kvq_packed), P(kvq_tables), P(kvq_packed),
                              P(kvq_tables), i32, ctypes.c_float, vp, vp, ctypes.c_size_t, st]
     L.kvq_attend_noalloc.argtypes = [P(kvq_desc), P(kvq_desc), vp, i32, P(kvq_packed), P(kvq_tables),
@@ -90,7 +91,7 @@ def _load():
     L.kvq_status_str.argtypes = [i32]
     L.kvq_status_str.restype = ctypes.c_char_p
     L.kvq_version.restype = i32
-    for n in ("kvq_encode", "kvq_decode", "kvq_score", "kvq_attend", "kvq_attend_noalloc", "kvq_calibrate_perm",
+    for n in ("kvq_encode", "kvq_decode", "kvq_score", "kvq_score_literal", "kvq_attend", "kvq_attend_noalloc", "kvq_calibrate_perm",
               "kvq_pair_energy", "kvq_detect_sinks", "kvq_calibrate_codebook",
               "kvq_rope_table", "kvq_rope_table_ex",
               "kvq_lloyd_max_codebook",
@@ -117,6 +118,12 @@ def kvq_score(desc: kvq_desc, q: int, q_heads: int, cache: kvq_packed, tables: k
               scale: float, scores: int, stream: int = 0) -> int:
     return lib.kvq_score(ctypes.byref(desc), q, q_heads, ctypes.byref(cache), ctypes.byref(tables), n_tokens,
                          scale, scores, stream)
+
+
+def kvq_score_literal(desc: kvq_desc, q: int, q_heads: int, cache: kvq_packed, tables: kvq_tables, n_tokens: int,
+                      scale: float, scores: int, stream: int = 0) -> int:
+    return lib.kvq_score_literal(ctypes.byref(desc), q, q_heads, ctypes.byref(cache), ctypes.byref(tables),
+                                 n_tokens, scale, scores, stream)
 
 
 def kvq_attend(dk: kvq_desc, dv: kvq_desc, q: int, q_heads: int, k_cache: kvq_packed, tk: kvq_tables,

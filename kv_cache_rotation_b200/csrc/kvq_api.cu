@@ -299,6 +299,38 @@ kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kv
   return launch_sink_fix_score(dd, q, q_heads, *cache, *tb, n_tokens, scale, scores, st);
 }
 
+kvq_status kvq_score_literal(const kvq_desc* d, const void* q, int32_t q_heads, const kvq_packed* cache,
+                             const kvq_tables* tb, int32_t n_tokens, float scale, float* scores,
+                             kvq_stream_t stream) {
+  if (!d) return KVQ_ERR_INVALID;
+  kvq_desc dd = *d;
+  dd.tokens = 0;
+  dd.t0 = 0;
+  kvq_status s = check_desc(&dd);
+  if (s != KVQ_OK) return s;
+  if (dd.rot != KVQ_ROT_NONE && dd.rot != KVQ_ROT_FWHT_HEAD) return KVQ_ERR_UNSUPPORTED;
+  if (dd.head_dim != 128 || dd.quant != KVQ_Q_MINMAX) return KVQ_ERR_UNSUPPORTED;
+  if (!q || !scores) return KVQ_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(scores, 16)) return KVQ_ERR_ALIGN;
+  if (q_heads <= 0 || q_heads % dd.heads) return KVQ_ERR_INVALID;
+  const int gq = q_heads / dd.heads;
+  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KVQ_ERR_UNSUPPORTED;
+  if (n_tokens < 0 || n_tokens > dd.t_cap) return KVQ_ERR_INVALID;
+  const bool listed = tb && tb->sink_pos && dd.n_sink > 0;
+  const int64_t rows = listed ? n_tokens : (dd.rope ? (n_tokens < dd.n_sink ? n_tokens : dd.n_sink) : 0);
+  if ((s = check_tables(&dd, tb, rows)) != KVQ_OK) return s;
+  if ((s = check_packed(&dd, cache)) != KVQ_OK) return s;
+  if (n_tokens == 0) return KVQ_OK;
+  LaunchCtx ctx;
+  if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  kvq_desc dm = dd;
+  if (listed) dm.n_sink = 0;  // every slot is scored from its codes first; the listed sinks after
+  s = launch_score_literal(dm, q, q_heads, *cache, *tb, n_tokens, scale, scores, st, ctx);
+  if (s != KVQ_OK || !listed) return s;
+  return launch_sink_fix_score(dd, q, q_heads, *cache, *tb, n_tokens, scale, scores, st);
+}
+
 namespace {
 // Shapes kvq_attend accepts: dk / dv valid, head-variant (or unrotated) min-max
 // caches of the same record shape, head_dim 128, values without RoPE.

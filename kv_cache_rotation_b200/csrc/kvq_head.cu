@@ -22,6 +22,7 @@
 // the 16 rows read at one channel fall on 16 distinct banks.
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
+#include "kvq_qdigits.cuh"
 
 namespace kvq {
 namespace {
@@ -331,6 +332,48 @@ __global__ void __launch_bounds__(kThreads, 4) k_encode_head(const HeadArgs a) {
   }
 }
 
+// This lane's half record back to fp32: dequantize (S, Z per group, already
+// multiplied by the normalisation when ROT) and undo the FWHT. Codes 0 and 2
+// of a quad are masked in place at bit 0, codes 1 and 3 at bit BITS; read
+// through the fp32 pattern 2^23 + v they give code * 2^p, and the power of two
+// 2^p folds exactly into the scale. The transform is its own inverse: stride V
+// across the lane pair, then strides 1 .. V/2 in registers. P ends in the
+// register-pair layout of this lane's V channels of the permuted vector.
+template <int D, int BITS, int G, bool ROT>
+__device__ __forceinline__ void unpack_inverse(const uint32_t* w, const float* Sg, const float* Zg, int s,
+                                               float2 (&P)[D / 4]) {
+  constexpr int V = D / 2;
+  constexpr int GS = G > V ? V : G;
+  constexpr int NW = V * BITS / 32;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+#pragma unroll
+  for (int g = 0; g < V / 4; ++g) {
+    const int gg = (4 * g) / GS;
+    const int pos = 4 * g * BITS;
+    const uint32_t lo = w[pos >> 5] >> (pos & 31);
+    const uint32_t w0 =
+        (32 - (pos & 31) >= 4 * BITS || (pos >> 5) + 1 >= NW) ? lo : (lo | (w[(pos >> 5) + 1] << (32 - (pos & 31))));
+    const uint32_t w1 = w0 >> (2 * BITS);
+    const float2 c02 = f2(__uint_as_float(0x4B000000u | (w0 & MASK)), __uint_as_float(0x4B000000u | (w1 & MASK)));
+    const float2 c13 = f2(__uint_as_float(0x4B000000u | (w0 & (MASK << BITS))),
+                          __uint_as_float(0x4B000000u | (w1 & (MASK << BITS))));
+    const float2 nM = f2(-8388608.0f, -8388608.0f), Z2 = f2(Zg[gg], Zg[gg]);
+    const float S1 = Sg[gg] * (1.0f / (1 << BITS));
+    P[2 * g] = fma2(add2(c02, nM), f2(Sg[gg], Sg[gg]), Z2);
+    P[2 * g + 1] = fma2(add2(c13, nM), f2(S1, S1), Z2);
+  }
+  if constexpr (ROT) {
+    const float sg = s ? -1.0f : 1.0f;
+#pragma unroll
+    for (int k = 0; k < V / 2; ++k) {
+      const float2 o = P[k];
+      const float2 p = f2(__shfl_xor_sync(0xffffffffu, o.x, 1), __shfl_xor_sync(0xffffffffu, o.y, 1));
+      P[k] = fma2(o, f2(sg, sg), p);
+    }
+    fwht_pairs<V>(P);
+  }
+}
+
 template <int D, int BITS, int G, bool ROT, bool F32>
 __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
   constexpr int V = D / 2;
@@ -341,7 +384,6 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
   constexpr int NGT = V / GS;
   constexpr int NBY = V * BITS / 8;
   constexpr int NW = NBY / 4;
-  constexpr uint32_t MASK = (1u << BITS) - 1u;
   constexpr int ES = F32 ? 4 : 2;
   extern __shared__ uint8_t smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -376,36 +418,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
       Sg[gg] = ROT ? __fmul_rn(sz.x, r) : sz.x;  // the normalisation folds into S and Z
       Zg[gg] = ROT ? __fmul_rn(sz.y, r) : sz.y;
     }
-    // dequantize: codes 0 and 2 of a quad are masked in place at bit 0, codes
-    // 1 and 3 at bit BITS; read through the fp32 pattern 2^23 + v they give
-    // code * 2^p, and the power of two 2^p folds exactly into the scale.
     float2 P[V / 2];
-#pragma unroll
-    for (int g = 0; g < V / 4; ++g) {
-      const int gg = (4 * g) / GS;
-      const int pos = 4 * g * BITS;
-      const uint32_t lo = w[pos >> 5] >> (pos & 31);
-      const uint32_t w0 =
-          (32 - (pos & 31) >= 4 * BITS || (pos >> 5) + 1 >= NW) ? lo : (lo | (w[(pos >> 5) + 1] << (32 - (pos & 31))));
-      const uint32_t w1 = w0 >> (2 * BITS);
-      const float2 c02 = f2(__uint_as_float(0x4B000000u | (w0 & MASK)), __uint_as_float(0x4B000000u | (w1 & MASK)));
-      const float2 c13 = f2(__uint_as_float(0x4B000000u | (w0 & (MASK << BITS))),
-                            __uint_as_float(0x4B000000u | (w1 & (MASK << BITS))));
-      const float2 nM = f2(-8388608.0f, -8388608.0f), Z2 = f2(Zg[gg], Zg[gg]);
-      const float S1 = Sg[gg] * (1.0f / (1 << BITS));
-      P[2 * g] = fma2(add2(c02, nM), f2(Sg[gg], Sg[gg]), Z2);
-      P[2 * g + 1] = fma2(add2(c13, nM), f2(S1, S1), Z2);
-    }
-    if constexpr (ROT) {  // the transform is its own inverse: stride V across the pair, then 1 .. V/2
-      const float sg = s ? -1.0f : 1.0f;
-#pragma unroll
-      for (int k = 0; k < V / 2; ++k) {
-        const float2 o = P[k];
-        const float2 p = f2(__shfl_xor_sync(0xffffffffu, o.x, 1), __shfl_xor_sync(0xffffffffu, o.y, 1));
-        P[k] = fma2(o, f2(sg, sg), p);
-      }
-      fwht_pairs<V>(P);
-    }
+    unpack_inverse<D, BITS, G, ROT>(w, Sg, Zg, s, P);
     if (a.perm) {  // x[perm[h][j]] = p_j: scatter into the row, read this lane's half back
       const int16_t* pr = a.perm + static_cast<size_t>(h) * D + V * s;
 #pragma unroll
@@ -490,6 +504,143 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode_head(const HeadArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Literal decode-step score ("EliteKV - RoPE频率选择与低秩投影" §2.2 score over
+// the head-variant cache): every key is decoded on the fly (unpack,
+// dequantize, inverse FWHT per token) and dotted with the GQ query heads of
+// its KV head. The permutation moves onto the query instead of the key
+// (sum_i q_i khat_i = sum_j q_perm[j] p_j, the same products in another
+// order); the transform is applied to every key. This is the reference form
+// that the query-rotation kernels (which transform the query once) are
+// measured against.
+// A CTA owns a contiguous range of 16-token steps of one (batch, KV head)
+// stream; its warps take every 8th step, two lanes per token as in the decode.
+constexpr int kLitThreads = 256;
+constexpr int kLitWarps = kLitThreads / 32;
+
+struct LitArgs {
+  int H, Hq, t_cap, n_tok, n_sink, rope;
+  int splits, n_step;  // CTAs per stream; 16-token steps per stream
+  float scale, rscale;
+  const __half* q;  // [B][Hq][128]
+  const int16_t* perm;
+  const float* rope_cs;
+  const uint8_t* codes;
+  const __half2* sz;
+  const __half* sink;
+  float* scores;  // [B][Hq][n_tok]
+};
+
+// A query row in shared memory: lane half s (channels sV .. sV + V - 1) at
+// s * (V + 4) floats, so the two halves read at once sit on distinct banks.
+template <int D>
+__host__ __device__ constexpr int lit_qpitch() {
+  return 2 * (D / 2 + 4);
+}
+
+template <int BITS, int G, int GQ, bool ROT>
+__global__ void __launch_bounds__(kLitThreads) k_score_literal(const LitArgs a) {
+  constexpr int D = 128, V = D / 2;
+  constexpr int RB = D * BITS / 8;
+  constexpr int NG = D / G;
+  constexpr bool SHARED = G > V;
+  constexpr int GS = SHARED ? V : G;
+  constexpr int NGT = V / GS;
+  constexpr int NBY = V * BITS / 8;
+  constexpr int NW = NBY / 4;
+  constexpr int QP = lit_qpitch<D>();
+  __shared__ __align__(16) float qraw[GQ][D];  // the queries as given (sink keys)
+  __shared__ __align__(16) float qp[GQ][QP];   // q_perm[j] at the lane-half position of channel j
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int s = lane & 1, slot = lane >> 1;
+  const int bh = static_cast<int>(blockIdx.x) / a.splits, part = static_cast<int>(blockIdx.x) % a.splits;
+  const int b = bh / a.H, h = bh - b * a.H;
+  for (int e = tid; e < GQ * D; e += kLitThreads) {
+    const int r = e / D, j = e % D;
+    const __half* qv = a.q + (static_cast<size_t>(b) * a.Hq + h * GQ + r) * D;
+    const int pj = a.perm ? (__ldg(a.perm + static_cast<size_t>(h) * D + j) & (D - 1)) : j;
+    qraw[r][j] = __half2float(qv[j]);
+    qp[r][(j / V) * (V + 4) + (j % V)] = __half2float(qv[pj]);
+  }
+  __syncthreads();
+  float* const out_h = a.scores + (static_cast<size_t>(b) * a.Hq + h * GQ) * a.n_tok;
+  if (part == 0) {  // fp16 sinks: s = scale * q . RoPE_n(sink_n)
+    for (int e = warp; e < min(a.n_sink, a.n_tok) * GQ; e += kLitWarps) {
+      const int n = e / GQ, r = e % GQ;
+      const float acc = sink_dot(qraw[r], a.sink + (static_cast<size_t>(bh) * a.n_sink + n) * D,
+                                 a.rope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane, a.rope == 2);
+      if (lane == 0) out_h[static_cast<size_t>(r) * a.n_tok + n] = acc * a.scale;
+    }
+  }
+  const int st0 = static_cast<int>(static_cast<long long>(a.n_step) * part / a.splits);
+  const int st1 = static_cast<int>(static_cast<long long>(a.n_step) * (part + 1) / a.splits);
+  const size_t rec0 = static_cast<size_t>(bh) * a.t_cap;
+  const uint32_t qbase = smem_u32(&qp[0][0]) + 4 * s * (V + 4);
+  for (int stp = st0 + warp; stp < st1; stp += kLitWarps) {
+    const int n = stp * kVecW + slot;
+    const bool live = n < a.n_tok && n >= a.n_sink;
+    const size_t slot_i = rec0 + (n < a.n_tok ? n : a.n_tok - 1);
+    uint32_t w[NW];
+    ld_run<NBY, pow2_align(NBY)>(a.codes + slot_i * RB + NBY * s, w);
+    float Sg[NGT], Zg[NGT];
+#pragma unroll
+    for (int gg = 0; gg < NGT; ++gg) {
+      const float2 sz = __half22float2(a.sz[slot_i * NG + (SHARED ? 0 : NGT * s + gg)]);
+      Sg[gg] = ROT ? __fmul_rn(sz.x, a.rscale) : sz.x;
+      Zg[gg] = ROT ? __fmul_rn(sz.y, a.rscale) : sz.y;
+    }
+    float2 P[V / 2];
+    unpack_inverse<D, BITS, G, ROT>(w, Sg, Zg, s, P);
+    float acc[GQ];
+#pragma unroll
+    for (int r = 0; r < GQ; ++r) {
+      float2 a2 = f2(0.0f, 0.0f);
+#pragma unroll
+      for (int g = 0; g < V / 4; ++g) {  // channels 4g .. 4g + 3 of this lane's half
+        const uint4 qv = lds128(qbase + 4 * (r * QP + 4 * g));
+        a2 = fma2(P[2 * g], f2(__uint_as_float(qv.x), __uint_as_float(qv.z)), a2);
+        a2 = fma2(P[2 * g + 1], f2(__uint_as_float(qv.y), __uint_as_float(qv.w)), a2);
+      }
+      acc[r] = a2.x + a2.y;
+      acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 1);
+    }
+    if (live) {  // both lanes hold every sum: query head r is written by lane half r mod 2
+#pragma unroll
+      for (int r = 0; r < GQ; ++r)
+        if ((GQ == 1 ? 0 : (r & 1)) == s) out_h[static_cast<size_t>(r) * a.n_tok + n] = acc[r] * a.scale;
+    }
+  }
+}
+
+template <int BITS, int G, int GQ, bool ROT>
+kvq_status run_literal(const kvq_desc& d, const LitArgs& a0, const LaunchCtx& ctx, cudaStream_t st) {
+  LitArgs a = a0;
+  const void* fn = reinterpret_cast<const void*>(k_score_literal<BITS, G, GQ, ROT>);
+  const int per_sm = occupancy_once(fn, kLitThreads, 0);
+  const long long streams = static_cast<long long>(d.batch) * d.heads;
+  a.n_step = (a.n_tok + kVecW - 1) / kVecW;
+  // as many CTAs per stream as one wave holds, each with at least one step per warp
+  long long splits = static_cast<long long>(ctx.num_sms) * per_sm / streams;
+  const long long max_splits = (a.n_step + kLitWarps - 1) / kLitWarps;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  if (streams * splits >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+  a.splits = static_cast<int>(splits);
+  k_score_literal<BITS, G, GQ, ROT><<<static_cast<unsigned>(streams * splits), kLitThreads, 0, st>>>(a);
+  return launch_status();
+}
+
+template <int BITS, int G, bool ROT>
+kvq_status literal_by_gq(const kvq_desc& d, const LitArgs& a, int gq, const LaunchCtx& ctx, cudaStream_t st) {
+  switch (gq) {
+    case 1: return run_literal<BITS, G, 1, ROT>(d, a, ctx, st);
+    case 2: return run_literal<BITS, G, 2, ROT>(d, a, ctx, st);
+    case 4: return run_literal<BITS, G, 4, ROT>(d, a, ctx, st);
+    case 8: return run_literal<BITS, G, 8, ROT>(d, a, ctx, st);
+    default: return KVQ_ERR_UNSUPPORTED;
+  }
+}
+
 template <int D, int BITS, int G, bool ROT>
 kvq_status run(bool enc, const HeadArgs& a, int out_fp32, const LaunchCtx& ctx, cudaStream_t st) {
   const size_t smem = a.perm ? static_cast<size_t>(kThreads / 32) * warp_buf<D>(enc) : 0;
@@ -571,6 +722,40 @@ kvq_status launch_decode_head(const kvq_desc& d, const kvq_packed& in, const kvq
   a.out = x_out;
   a.v8 = aligned32(x_out);
   return dispatch(false, d, a, out_fp32, ctx, st);
+}
+
+kvq_status launch_score_literal(const kvq_desc& d, const void* q, int q_heads, const kvq_packed& cache,
+                                const kvq_tables& tb, int n_tokens, float scale, float* scores, cudaStream_t st,
+                                const LaunchCtx& ctx) {
+  if (d.head_dim != 128 || d.quant != KVQ_Q_MINMAX) return KVQ_ERR_UNSUPPORTED;
+  LitArgs a{};
+  a.H = d.heads;
+  a.Hq = q_heads;
+  a.t_cap = d.t_cap;
+  a.n_tok = n_tokens;
+  a.n_sink = d.n_sink;
+  a.rope = d.rope;
+  a.scale = scale;
+  a.rscale = static_cast<float>(1.0 / sqrt(128.0));
+  a.q = static_cast<const __half*>(q);
+  a.perm = tb.perm;
+  a.rope_cs = tb.rope_cs;
+  a.codes = cache.codes;
+  a.sz = static_cast<const __half2*>(cache.scale_zero);
+  a.sink = static_cast<const __half*>(cache.sink);
+  a.scores = scores;
+  const int gq = q_heads / d.heads;
+  const bool rot = d.rot == KVQ_ROT_FWHT_HEAD;
+#define KVQ_CASE(B_, G_)                                                                   \
+  if (d.bits == B_ && d.group == G_)                                                     \
+    return rot ? literal_by_gq<B_, G_, true>(d, a, gq, ctx, st) : literal_by_gq<B_, G_, false>(d, a, gq, ctx, st);
+#define KVQ_BITS(G_) KVQ_CASE(2, G_) KVQ_CASE(3, G_) KVQ_CASE(4, G_)
+  KVQ_BITS(128)
+  KVQ_BITS(64)
+  KVQ_BITS(32)
+#undef KVQ_BITS
+#undef KVQ_CASE
+  return KVQ_ERR_UNSUPPORTED;
 }
 
 }  // namespace kvq

@@ -43,6 +43,9 @@ kvq_status launch_decode_iso(const kvq_desc& d, const kvq_packed& in, const kvq_
 kvq_status launch_score(const kvq_desc& d, const void* q, int q_heads, const kvq_packed& cache,
                         const kvq_tables& tb, int n_tokens, float scale, float* scores, cudaStream_t st,
                         const LaunchCtx& ctx);
+kvq_status launch_score_literal(const kvq_desc& d, const void* q, int q_heads, const kvq_packed& cache,
+                                const kvq_tables& tb, int n_tokens, float scale, float* scores, cudaStream_t st,
+                                const LaunchCtx& ctx);
 kvq_status launch_score_group(const kvq_desc& d, const void* q, int q_heads, const kvq_packed& cache,
                               const kvq_tables& tb, int n_tokens, float scale, float* scores, cudaStream_t st,
                               const LaunchCtx& ctx);

@@ -17,7 +17,7 @@ from . import (KVQ_FIELD_CODES, KVQ_FIELD_EXT, KVQ_FIELD_NORM, KVQ_FIELD_SCALE_Z
                KVQ_Q_CODEBOOK, KVQ_Q_CODEBOOK_DYN, KVQ_Q_MINMAX, KVQ_ROT_FWHT_GROUP, KVQ_ROT_FWHT_HEAD, KVQ_ROT_ISO_SO3, KVQ_ROT_ISO_SO4, KVQ_ROT_NONE,
                check,
                kvq_decode, kvq_desc, kvq_encode, kvq_lloyd_max_codebook, kvq_packed, kvq_packed_bytes,
-               kvq_rope_table, kvq_score, kvq_tables)
+               kvq_rope_table, kvq_score, kvq_score_literal, kvq_tables)
 
 ROT = {"none": KVQ_ROT_NONE, "fwht_head": KVQ_ROT_FWHT_HEAD, "fwht_group": KVQ_ROT_FWHT_GROUP,
        "iso": KVQ_ROT_ISO_SO4, "iso3": KVQ_ROT_ISO_SO3}
@@ -177,6 +177,15 @@ def score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens
     _req(out, "scores", (torch.float32,), (d.batch, hq, n_tokens))
     check(kvq_score(d, q.data_ptr(), hq, packed.struct(), tables.struct(), n_tokens, scale,
                     out.data_ptr(), _stream(stream)), "kvq_score")
+
+
+def score_literal(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens: int, scale: float,
+                  out: torch.Tensor, stream=None) -> None:
+    """The scores of score(), every key decoded on the fly (the literal per-token form)."""
+    hq = _q_heads(d, q)
+    _req(out, "scores", (torch.float32,), (d.batch, hq, n_tokens))
+    check(kvq_score_literal(d, q.data_ptr(), hq, packed.struct(), tables.struct(), n_tokens, scale,
+                            out.data_ptr(), _stream(stream)), "kvq_score_literal")
 
 
 def attend_workspace(dk: kvq_desc, dv: kvq_desc, q_heads: int, n_tokens: int, device="cuda") -> torch.Tensor:
@@ -394,7 +403,8 @@ def bind_decode(d: kvq_desc, packed: Packed, tables: Tables, out: torch.Tensor, 
 
 
 def bind_score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_tokens: int, scale: float,
-               out: torch.Tensor, stream=None):
+               out: torch.Tensor, stream=None, literal: bool = False):
+    """A prepared kvq_score call (kvq_score_literal with literal=True)."""
     from . import lib
     hq = _q_heads(d, q)
     _req(out, "scores", (torch.float32,), (d.batch, hq, n_tokens))
@@ -403,7 +413,9 @@ def bind_score(d: kvq_desc, q: torch.Tensor, packed: Packed, tables: Tables, n_t
             ctypes.c_float(scale), out.data_ptr(), st)
     keep = (d, q, packed, tables, out, tb, pk)
 
+    fn, name = (lib.kvq_score_literal, "kvq_score_literal") if literal else (lib.kvq_score, "kvq_score")
+
     def call():
-        check(lib.kvq_score(*args), "kvq_score")
+        check(fn(*args), name)
     call.keep = keep
     return call

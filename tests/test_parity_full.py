@@ -134,7 +134,7 @@ def test_full_isoquant_batch(K, orc, name):
     assert np.all(np.abs(got - dec) <= 1e-3 + np.abs(dec) * 2.0 ** -11), np.abs(got - dec).max()
 
 
-def _score_full(K, orc, w, perm, n_tok_sample, seed):
+def _score_full(K, orc, w, perm, n_tok_sample, seed, literal=False):
     from kv_cache_rotation_b200 import torch_api as TA
     D = w.D
     t_cap = w.T + w.append
@@ -150,7 +150,7 @@ def _score_full(K, orc, w, perm, n_tok_sample, seed):
     q = W.queries(w)
     scale = 1.0 / math.sqrt(D)
     out = torch.empty((w.B, w.Hq, t_cap), dtype=torch.float32, device="cuda")
-    TA.score(d_pre, torch.from_numpy(q).cuda(), pk, tb, t_cap, scale, out)
+    (TA.score_literal if literal else TA.score)(d_pre, torch.from_numpy(q).cuda(), pk, tb, t_cap, scale, out)
     assert K.kvq_check(0) == K.KVQ_OK
     assert torch.isfinite(out).all()
     tok = _sample(t_cap, n_tok_sample, seed, always=(0, 1, 2, 3, 4, t_cap - 2, t_cap - 1))
@@ -180,3 +180,13 @@ def test_full_decode_score(K, orc):
 def test_full_llama3_8b_gqa_score(K, orc):
     w = W.WORKLOADS["llama3_8b_gqa_score"]
     _score_full(K, orc, w, None, 32, 12)
+
+
+def test_full_decode_score_literal(K, orc):
+    w = W.WORKLOADS["decode_score"]
+    _score_full(K, orc, w, W.random_perm(w.H, w.D, 23), 24, 13, literal=True)
+
+
+def test_full_llama3_8b_gqa_score_literal(K, orc):
+    w = W.WORKLOADS["llama3_8b_gqa_score"]
+    _score_full(K, orc, w, None, 32, 14, literal=True)

@@ -39,17 +39,17 @@ def build_cache(K, w, x, x_app, perm, rot="fwht_head", rope=1):
     return d_pre, tb, pk
 
 
-def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None, rope=1):
+def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None, rope=1, literal=False):
     from kv_cache_rotation_b200 import torch_api as TA
     x = W.kv_tensor(w, "k")
     x_app = W.kv_tensor(w, "k_append", T=w.append)
     d, tb, pk = build_cache(K, w, x, x_app, perm, rot, rope)
-    orope = orc.ROPE_STD + (orc.ROPE_HALF if rope == 2 else 0)
+    orope = 0 if rope == 0 else orc.ROPE_STD + (orc.ROPE_HALF if rope == 2 else 0)
     q = W.queries(w)
     n_tok = d.t_cap
     scale = 1.0 / math.sqrt(w.D)
     out = torch.full((w.B, w.Hq, n_tok), float("nan"), dtype=torch.float32, device="cuda")
-    TA.score(d, torch.from_numpy(q).cuda(), pk, tb, n_tok, scale, out)
+    (TA.score_literal if literal else TA.score)(d, torch.from_numpy(q).cuda(), pk, tb, n_tok, scale, out)
     assert K.kvq_check(0) == K.KVQ_OK
     tok = np.arange(n_tok) if tokens is None else np.asarray(tokens)
     cache = {"codes": pk.codes.cpu().numpy(), "sz": pk.scale_zero.cpu().numpy().view(np.uint16),
@@ -65,7 +65,7 @@ def run_score_case(K, orc, w, perm, rot="fwht_head", tokens=None, rope=1):
     for b in range(w.B):
         for qh in range(w.Hq):
             h = qh // gq
-            kk = np.stack([orc.rope_f64(khat[b, h, n], n, mode=orope) for n in tok])
+            kk = np.stack([orc.rope_f64(khat[b, h, n], n, mode=orope) for n in tok]) if rope else khat[b, h, tok]
             bound = SCORE_REL * scale * (np.abs(kk) @ np.abs(q[b, qh].astype(np.float64)))
             err = np.abs(got[b, qh] - ref[b, qh])
             assert np.all(err <= bound), (b, qh, np.max(err / bound))
@@ -123,3 +123,54 @@ def test_score_grouped_cache_half_split(K, orc):
     w = W.Workload("score_group_half", B=1, H=8, T=120, rot="fwht_group", group_heads=8, bits=2, group=128,
                    n_sink=3, Hq=16, append=1, seed=91)
     run_score_case(K, orc, w, None, rot="fwht_group", rope=2)
+
+
+LITERAL = [
+    # name, workload, overrides, perm seed (None: no permutation), rot, rope
+    ("mha_perm_sinks_g64", "decode_score", dict(B=2, H=4, Hq=4, T=300), 11, "fwht_head", 1),
+    ("gqa4_g128", "llama3_8b_gqa_score", dict(B=2, H=2, Hq=8, T=257), None, "fwht_head", 1),
+    ("gq2_b3_g32", "decode_score", dict(B=1, H=2, Hq=4, T=130, bits=3, group=32, n_sink=1), 2, "fwht_head", 1),
+    ("gq8_b4_g128", "decode_score", dict(B=1, H=2, Hq=16, T=97, bits=4, group=128, n_sink=2), 5, "fwht_head", 1),
+    ("b3_g64_half_split", "decode_score", dict(B=2, H=2, Hq=4, T=150, bits=3, group=64, n_sink=4), 12,
+     "fwht_head", 2),
+    ("no_rotation", "decode_score", dict(B=1, H=2, Hq=2, T=70, n_sink=0), None, "none", 1),
+    ("no_rope_b4_g32", "decode_score", dict(B=2, H=2, Hq=2, T=45, bits=4, group=32, n_sink=3), 8, "fwht_head", 0),
+]
+
+
+@pytest.mark.parametrize("case", LITERAL, ids=[c[0] for c in LITERAL])
+def test_score_literal(K, orc, case):
+    """The literal per-token form (every key unpacked, dequantized and inverse-
+    transformed before the dot) against the same oracle scores."""
+    name, wl, over, pseed, rot, rope = case
+    w = W.scaled(W.WORKLOADS[wl], **over)
+    perm = W.random_perm(w.H, w.D, pseed) if pseed is not None else None
+    worst = run_score_case(K, orc, w, perm, rot=rot, rope=rope, literal=True)
+    print(f"{name}: worst |err| / S2 bound = {worst:.3g}")
+
+
+def test_score_literal_matches_query_rotation(K):
+    """Both score forms over one cache: equal within the S2 bound's scale (the
+    query-rotation kernel rounds the rotated query to 16-bit digits)."""
+    from kv_cache_rotation_b200 import torch_api as TA
+    w = W.scaled(W.WORKLOADS["llama3_8b_gqa_score"], B=2, H=2, Hq=8, T=513)
+    d, tb, pk = build_cache(K, w, W.kv_tensor(w, "k"), W.kv_tensor(w, "k_append", T=w.append), None)
+    q = torch.from_numpy(W.queries(w)).cuda()
+    n = d.t_cap
+    a = torch.empty((w.B, w.Hq, n), dtype=torch.float32, device="cuda")
+    b = torch.empty_like(a)
+    TA.score(d, q, pk, tb, n, 0.0884, a)
+    TA.score_literal(d, q, pk, tb, n, 0.0884, b)
+    assert K.kvq_check(0) == K.KVQ_OK
+    assert torch.equal(a[:, :, :w.n_sink], b[:, :, :w.n_sink])  # the sinks take the same fp32 path
+    torch.testing.assert_close(a, b, rtol=0, atol=1e-3 * float(b.abs().max()))
+
+
+def test_score_literal_rejects(K):
+    from kv_cache_rotation_b200 import torch_api as TA
+    w = W.scaled(W.WORKLOADS["decode_score"], B=1, H=2, Hq=2, T=32, D=64, group=32)
+    d, tb, pk = build_cache(K, w, W.kv_tensor(w, "k"), W.kv_tensor(w, "k_append", T=w.append), None)
+    q = torch.zeros((1, 2, 64), dtype=torch.float16, device="cuda")
+    out = torch.empty((1, 2, d.t_cap), dtype=torch.float32, device="cuda")
+    assert K.kvq_score_literal(d, q.data_ptr(), 2, pk.struct(), tb.struct(), d.t_cap, 1.0, out.data_ptr(), 0) == \
+        K.KVQ_ERR_UNSUPPORTED  # head_dim 64

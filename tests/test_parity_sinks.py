@@ -256,8 +256,12 @@ SCORE = [
 ]
 
 
-@pytest.mark.parametrize("case", SCORE, ids=[c[0] for c in SCORE])
-def test_list_score(K, orc, case):
+LITERAL = [(c, True) for c in SCORE if c[1] != "fwht_group"]
+
+
+@pytest.mark.parametrize("case,literal", [(c, False) for c in SCORE] + LITERAL,
+                         ids=[c[0] for c in SCORE] + [c[0] + "_literal" for c, _ in LITERAL])
+def test_list_score(K, orc, case, literal):
     from kv_cache_rotation_b200 import torch_api as TA
     name, rot, B, H, GQ, T, rope, hg, group = case
     D, bits, n_sink, scale = 128, 2, 4, 0.0884
@@ -278,7 +282,7 @@ def test_list_score(K, orc, case):
     TA.encode(d, torch.from_numpy(x).cuda(), tb, pk)
     q = np.random.default_rng(3).standard_normal((B, H * GQ, D)).astype(np.float16)
     out = torch.empty((B, H * GQ, T), dtype=torch.float32, device="cuda")
-    TA.score(d, torch.from_numpy(q).cuda(), pk, tb, T, scale, out)
+    (TA.score_literal if literal else TA.score)(d, torch.from_numpy(q).cuda(), pk, tb, T, scale, out)
     assert K.kvq_check(0) == K.KVQ_OK
     okw = dict(rot=ORC_ROT[rot], bits=bits, group=group, group_heads=hg, rope=_orope(orc, rope), n_sink=n_sink)
     cache = {"codes": pk.codes.cpu().numpy(), "sz": pk.scale_zero.cpu().numpy().view(np.uint16),
