@@ -570,16 +570,16 @@ def _kernel_sources_sha(names):
     return h.hexdigest()[:16]
 
 
-def _traffic_for(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+def _traffic_for(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary of this kernel on
+    this workload, if it was taken on the current kernel source; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
-    e = j.get(kernel)
-    if not e:
+    e = j.get(f"{kernel}@{workload}") or j.get(kernel)
+    if not e or e.get("bench_workload") != workload:
         return None
     if e.get("source_sha") != _kernel_sources_sha(e.get("sources", [])):
         return None
@@ -796,7 +796,7 @@ def run_ours(args):
     dom_ms = per_kernel[dom] / args.steps
     achieved = st.alg[dom] / (dom_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": _traffic_for(st.kernels[dom]), "kernel": st.kernels[dom],
+                "traffic": _traffic_for(st.kernels[dom], args.workload), "kernel": st.kernels[dom],
                 "kernel_step": dom, "alg_bytes_per_launch": st.alg[dom], "peak_kind": peak_kind}
     clocks = clk.summary()
     if dom in st.fp32_ops:
