@@ -190,7 +190,12 @@ kvq_status kvq_decode(const kvq_desc* d, const kvq_packed* in, const kvq_tables*
  * (the grouped-head rotation) with rope != 0, no permutation, q_heads/H in {1, 2, 4, 8} and
  * rope_rows >= n_tokens: RoPE comes after the rotation there, so each key is decoded (inverse
  * FWHT over its head group) and turned to its position before the dot product.
- * scores: f32 [B][q_heads][n_tokens]; n_tokens <= t_cap. d->tokens and d->t0 are ignored. */
+ * scores: f32 [B][q_heads][n_tokens]; n_tokens <= t_cap. d->tokens and d->t0 are ignored.
+ * Accuracy: the head-variant tensor-core path rounds the rotated query to 16-bit integer digits,
+ * so a score's error is bounded by scale * max|H P q| / 64000 * sum_j |y_j| over the stored
+ * rotated key y; a key with a massive activation that is neither a sink nor listed spreads it
+ * over all rotated channels and can exceed 1e-3 of sum_j |q_j khat_j|. kvq_score_literal has
+ * no such term (fp32 throughout). */
 kvq_status kvq_score(const kvq_desc* d, const void* q, int32_t q_heads, const kvq_packed* cache,
                      const kvq_tables* tb, int32_t n_tokens, float scale, float* scores,
                      kvq_stream_t stream);

@@ -104,6 +104,27 @@ def test_score_argument_checks():
     assert K.kvq_score(d, 256, 8, p, tb, 0, 1.0, 256, 0) == K.KVQ_OK  # empty: nothing to do
 
 
+def test_score_literal_argument_checks():
+    d = _desc(t_cap=32, tokens=0, head_dim=128)
+    tb = K.kvq_tables()
+    p = _packed(d)
+    f = K.kvq_score_literal
+    assert K.lib.kvq_score_literal(None, 256, 8, ctypes.byref(p), ctypes.byref(tb), 16, ctypes.c_float(1.0), 256,
+                                   None) == K.KVQ_ERR_INVALID
+    assert f(d, 256, 12, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_INVALID  # 12 % 8
+    assert f(d, 256, 24, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_UNSUPPORTED  # 3 query heads per KV head
+    assert f(d, 256, 8, p, tb, 33, 1.0, 256, 0) == K.KVQ_ERR_INVALID  # > t_cap
+    assert f(d, 258, 8, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_ALIGN
+    assert f(d, 256, 8, p, tb, 16, 1.0, 260, 0) == K.KVQ_ERR_ALIGN
+    assert f(_desc(t_cap=32, tokens=0, head_dim=64, group=32), 256, 8, p, tb, 16, 1.0, 256, 0) == \
+        K.KVQ_ERR_UNSUPPORTED
+    dg = _desc(t_cap=32, rot="fwht_group", group_heads=8, group=128)
+    assert f(dg, 256, 8, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_UNSUPPORTED
+    di = _desc(t_cap=32, tokens=0, rot="iso", quant="codebook", bits=3)
+    assert f(di, 256, 8, p, tb, 16, 1.0, 256, 0) == K.KVQ_ERR_UNSUPPORTED
+    assert f(d, 256, 8, p, tb, 0, 1.0, 256, 0) == K.KVQ_OK  # empty: nothing to do
+
+
 def test_attend_argument_checks():
     dk = _desc(t_cap=32, tokens=0, rope=1)
     dv = _desc(t_cap=32, tokens=0, rope=0)
