@@ -24,6 +24,9 @@ CASES = [
     ("half_split_hg8_sinks", 2, 8, 70, 8, 2, 128, 2, False, 2, 0),
     ("half_split_hg4_perm", 1, 4, 90, 4, 2, 128, 2, True, 0, 3),
     ("half_split_hg2_g64", 1, 4, 130, 2, 3, 64, 2, True, 0, 0),
+    # sink positions inside the call (t0 < n_sink < t0 + T), and more sinks than tokens
+    ("sinks_cross_t0", 1, 8, 21, 8, 2, 128, 1, False, 6, 3),
+    ("all_sinks", 2, 8, 3, 8, 2, 128, 1, True, 5, 0),
 ]
 
 

@@ -34,6 +34,9 @@ CASES = [
     ("half_split_perm_sink", 2, 4, 37, 128, 5, 2, 2, 64, 2, True, 4, "fwht_head"),
     ("half_split_d64", 1, 8, 40, 64, 2, 1, 3, 32, 2, True, 1, "fwht_head"),
     ("half_split_no_rotation", 1, 8, 50, 128, 0, 0, 4, 128, 2, False, 2, "none"),
+    # sink positions inside the call (t0 < n_sink < t0 + T), and more sinks than tokens
+    ("sinks_cross_t0", 1, 4, 20, 128, 2, 0, 2, 64, 1, True, 5, "fwht_head"),
+    ("all_sinks", 1, 2, 3, 128, 0, 0, 2, 128, 1, False, 8, "fwht_head"),
 ]
 
 

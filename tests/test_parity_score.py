@@ -135,7 +135,14 @@ LITERAL = [
      "fwht_head", 2),
     ("no_rotation", "decode_score", dict(B=1, H=2, Hq=2, T=70, n_sink=0), None, "none", 1),
     ("no_rope_b4_g32", "decode_score", dict(B=2, H=2, Hq=2, T=45, bits=4, group=32, n_sink=3), 8, "fwht_head", 0),
+    ("only_sinks", "llama3_8b_gqa_score", dict(B=1, H=2, Hq=8, T=2, n_sink=4), None, "fwht_head", 1),
 ]
+
+
+def test_score_only_sinks(K, orc):
+    """Fewer cached slots than sinks: every score is a sink's exact dot."""
+    w = W.scaled(W.WORKLOADS["llama3_8b_gqa_score"], B=1, H=2, Hq=8, T=2, n_sink=4)
+    run_score_case(K, orc, w, None)
 
 
 @pytest.mark.parametrize("case", LITERAL, ids=[c[0] for c in LITERAL])
