@@ -92,7 +92,7 @@ def lib():
                                 u16p, u8p, u16p, u16p, f32p, i16p, f32p, f32p, f32p, i64p, ci, cd, f64p, i32p]
         L.orc_attend.restype = ci
         L.orc_attend.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, cd, u16p,
-                                 u8p, u16p, u16p, i16p, ci, u8p, u16p, u16p, i16p, ci, cd, f64p]
+                                 u8p, u16p, u16p, i16p, ci, u8p, u16p, u16p, i16p, ci, cd, f64p, i32p]
         L.orc_calibrate_perm.restype = ci
         L.orc_calibrate_perm.argtypes = [ci, ci, ci, ci, i64p, ci, ci, cd, u16p, i16p, i32p]
         L.orc_detect_sinks.restype = ci
@@ -321,10 +321,11 @@ def score(q, cache, tokens, *, H, t_cap, rot, quant=Q_MINMAX, bits, group=0, gro
 
 
 def attend(q, kcache, vcache, n_tok, *, H, t_cap, rot, bits, group, n_sink=0, base=10000.0, scale,
-           kperm=None, vperm=None, krope=1, vrope=0):
+           kperm=None, vperm=None, krope=1, vrope=0, sink_pos=None):
     """Decode-step attention (orc_attend). q: uint16 [B][Hq][D] in attention
     space; kcache / vcache: dicts of codes, sz and sink laid out over t_cap
-    slots. Returns float64 [B][Hq][D]."""
+    slots; sink_pos: int32 [B][n_sink] sink list of both caches, or None for
+    the positions < n_sink. Returns float64 [B][Hq][D]."""
     q = np.ascontiguousarray(q, np.uint16)
     B, Hq, D = q.shape
     out = np.zeros((B, Hq, D), np.float64)
@@ -338,11 +339,12 @@ def attend(q, kcache, vcache, n_tok, *, H, t_cap, rot, bits, group, n_sink=0, ba
 
     kc, kz, ks, kp = arrs(kcache, kperm)
     vc, vz, vs, vp = arrs(vcache, vperm)
+    sp = None if sink_pos is None else np.ascontiguousarray(sink_pos, np.int32)
     rc = lib().orc_attend(B, H, Hq, D, t_cap, int(n_tok), rot, bits, group, n_sink, base, _p(q, ctypes.c_uint16),
                           _p(kc, ctypes.c_uint8), _p(kz, ctypes.c_uint16), _p(ks, ctypes.c_uint16),
                           _p(kp, ctypes.c_int16), int(krope), _p(vc, ctypes.c_uint8), _p(vz, ctypes.c_uint16),
                           _p(vs, ctypes.c_uint16), _p(vp, ctypes.c_int16), int(vrope), float(scale),
-                          _p(out, ctypes.c_double))
+                          _p(out, ctypes.c_double), _p(sp, ctypes.c_int32))
     if rc:
         raise ValueError("oracle attend: unsupported parameters")
     return out

@@ -829,13 +829,15 @@ int orc_score(int B, int H, int Hq, int D, int t_cap, int rot, int quant, int bi
  *   p_n   = exp(s_n - max s) / sum exp(s - max s)
  *   out   = sum_n p_n * vhat_n          (vhat_n: decoded V slot n; sinks verbatim)
  * K and V caches share the record shape (rot, bits, group, n_sink) and have
- * their own RoPE flag and permutation. fp64 throughout.
+ * their own RoPE flag and permutation. sink_pos: NULL (the sinks are the
+ * positions < n_sink) or the sink list [B][n_sink] of both caches, as
+ * orc_score and orc_decode take it. fp64 throughout.
  * ---------------------------------------------------------------------- */
 int orc_attend(int B, int H, int Hq, int D, int t_cap, int n_tok, int rot, int bits, int group, int n_sink,
                double base, const uint16_t* q, const uint8_t* kcodes, const uint16_t* ksz,
                const uint16_t* ksink, const int16_t* kperm, int krope, const uint8_t* vcodes,
                const uint16_t* vsz, const uint16_t* vsink, const int16_t* vperm, int vrope, double scale,
-               double* out) {
+               double* out, const int32_t* sink_pos) {
   if (Hq % H || n_tok < 1 || n_tok > t_cap) return 1;
   if (rot != ORC_ROT_NONE && rot != ORC_ROT_FWHT_HEAD) return 1;
   int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)t_cap);
@@ -843,10 +845,10 @@ int orc_attend(int B, int H, int Hq, int D, int t_cap, int n_tok, int rot, int b
   double* s = (double*)malloc(sizeof(double) * (size_t)B * Hq * n_tok);
   double* vh = (double*)malloc(sizeof(double) * (size_t)B * H * t_cap * D);
   int rc = orc_score(B, H, Hq, D, t_cap, rot, ORC_Q_MINMAX, bits, group, 1, krope, n_sink, base, q, kcodes, ksz,
-                     ksink, NULL, kperm, NULL, NULL, NULL, tok, n_tok, scale, s, NULL);
+                     ksink, NULL, kperm, NULL, NULL, NULL, tok, n_tok, scale, s, sink_pos);
   if (!rc)
     rc = orc_decode(B, H, t_cap, D, tok, rot, ORC_Q_MINMAX, bits, group, 1, vrope, n_sink, base, vcodes, vsz,
-                    vsink, NULL, vperm, NULL, NULL, NULL, vh, NULL);
+                    vsink, NULL, vperm, NULL, NULL, NULL, vh, sink_pos);
   if (!rc) {
     for (int b = 0; b < B; ++b)
       for (int qh = 0; qh < Hq; ++qh) {

@@ -89,3 +89,35 @@ def test_query_heads_share_their_kv_head(orc, caches):
                      vperm=caches["vp"], **caches["common"])
     assert np.array_equal(out[:, 1], out[:, 0])
     assert not np.allclose(out[:, HQ // H], out[:, 0])  # a different cache gives a different result
+
+
+def test_listed_prefix_is_the_prefix_form(orc, caches):
+    # a sink list naming positions 0 .. n_sink-1 is the prefix form
+    sp = np.tile(np.arange(3, dtype=np.int32), (B, 1))
+    a = _attend(orc, caches, T, 1.0 / np.sqrt(D))
+    b = orc.attend(caches["q"], caches["kc"], caches["vc"], T, H=H, t_cap=T, scale=1.0 / np.sqrt(D),
+                   kperm=caches["kp"], vperm=caches["vp"], sink_pos=sp, **caches["common"])
+    assert np.array_equal(a, b)
+
+
+def test_listed_sinks_zero_scale_mean(orc):
+    # caches whose sinks are listed positions: with a zero scale the output is the plain mean over the
+    # slots, each listed slot contributing its fp16 row and every other slot its decoded codes
+    w = W.Workload("attn_list", B=B, H=H, Hq=HQ, T=T, D=D, bits=2, group=64, n_sink=3)
+    k = W.kv_tensor(w, "k").view(np.uint16)
+    v = W.kv_tensor(w, "v").view(np.uint16)
+    pos = np.arange(T)
+    sp = np.array([[4, 11, -1], [0, 17, 23]], np.int32)
+    common = dict(rot=orc.ROT_FWHT_HEAD, bits=2, group=64, n_sink=3, sink_pos=sp)
+    kc = orc.encode(k, pos, rope=1, **common)
+    vc = orc.encode(v, pos, rope=0, **common)
+    out = orc.attend(W.queries(w).view(np.uint16), kc, vc, T, H=H, t_cap=T, scale=0.0, **common)
+    plain = orc.decode(vc, pos, (B, H, T, D), rope=0, rot=orc.ROT_FWHT_HEAD, bits=2, group=64)  # no sinks
+    rows = v.view(np.float16).astype(np.float64)
+    for b in range(B):
+        vals = plain[b].copy()  # [H][T][D]
+        for p in sp[b]:
+            if p >= 0:
+                vals[:, p] = rows[b, :, p]
+        for qh in range(HQ):
+            np.testing.assert_allclose(out[b, qh], vals[qh // (HQ // H)].mean(axis=0), rtol=0, atol=1e-12)
