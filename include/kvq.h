@@ -143,10 +143,11 @@ typedef struct {
  *             of the sink set ([RotateKV] attention sinks found from the activations, e.g. by
  *             kvq_detect_sinks). Entry k of sequence b is the position (cache slot) whose fp16
  *             row is sink row k, or -1 for an unused entry; entries must be distinct. 4-byte
- *             aligned. Read by kvq_encode, kvq_decode, kvq_score and kvq_calibrate_perm;
- *             kvq_attend returns KVQ_ERR_UNSUPPORTED for it. With a list, encode, decode and
- *             score run their kernels on every slot and one more small kernel then writes the
- *             sink entries; kvq_score then needs rope_rows >= n_tokens when rope != 0. */
+ *             aligned. Read by kvq_encode, kvq_decode, kvq_score, kvq_score_literal,
+ *             kvq_calibrate_perm and kvq_attend (which needs it in both caches' tables). With a
+ *             list, encode, decode and score run their kernels on every slot and one more small
+ *             kernel then writes the sink entries; kvq_score and kvq_attend then need
+ *             rope_rows >= n_tokens when rope != 0. */
 typedef struct {
   const int16_t* perm;
   const float* rope_cs;
@@ -232,7 +233,10 @@ kvq_status kvq_score_literal(const kvq_desc* d, const void* q, int32_t q_heads, 
  * records (scores, running softmax and value sums on the tensor cores) and a merge launched as
  * its programmatic dependent; other shapes run three (scores, chunked softmax-weighted sums,
  * merge). Results agree with kvq_score's scores through an exact fp64 softmax within
- * 2e-5 * max|vhat|. */
+ * 2e-5 * max|vhat|. Sinks given as a list (tk->sink_pos and tv->sink_pos, the list both caches
+ * were encoded with; one without the other is KVQ_ERR_INVALID) enter with their exact fp16
+ * scores and rows; the fused form masks the listed slots and takes up to 32 entries, longer
+ * lists run the three-kernel form. */
 kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int32_t q_heads,
                       const kvq_packed* k_cache, const kvq_tables* tk, const kvq_packed* v_cache,
                       const kvq_tables* tv, int32_t n_tokens, float scale, float* out, void* workspace,

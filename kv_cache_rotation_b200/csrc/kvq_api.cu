@@ -359,6 +359,19 @@ kvq_status check_attend(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads,
 }
 }  // namespace
 
+// The tables of an attention call: a sink list goes with both caches (they were
+// encoded with it) and needs RoPE rows up to n_tokens for the keys.
+static kvq_status check_attend_tables(const kvq_desc& k, const kvq_desc& v, const kvq_tables* tk, const kvq_tables* tv,
+                               int32_t n_tokens) {
+  if (!tk || !tv) return KVQ_ERR_INVALID;
+  const bool listed = k.n_sink > 0 && tk->sink_pos;
+  if (k.n_sink > 0 && (!tk->sink_pos != !tv->sink_pos)) return KVQ_ERR_INVALID;
+  const int64_t rows = k.rope ? (listed ? n_tokens : (n_tokens < k.n_sink ? n_tokens : k.n_sink)) : 0;
+  kvq_status s = check_tables(&k, tk, rows);
+  if (s != KVQ_OK) return s;
+  return check_tables(&v, tv, 0);
+}
+
 size_t kvq_attend_workspace_bytes(const kvq_desc* dk, const kvq_desc* dv, int32_t q_heads, int32_t n_tokens) {
   kvq_desc k, v;
   if (check_attend(dk, dv, q_heads, n_tokens, &k, &v) != KVQ_OK) return 0;
@@ -375,9 +388,7 @@ kvq_status kvq_attend(const kvq_desc* dk, const kvq_desc* dv, const void* q, int
   if (!q || !out || !workspace) return KVQ_ERR_INVALID;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_ALIGN;
   if (workspace_bytes < attend_workspace_bytes(k, q_heads, n_tokens)) return KVQ_ERR_INVALID;
-  if ((s = check_tables(&k, tk, k.rope ? (n_tokens < k.n_sink ? n_tokens : k.n_sink) : 0)) != KVQ_OK) return s;
-  if ((s = check_tables(&v, tv, 0)) != KVQ_OK) return s;
-  if (tk->sink_pos || tv->sink_pos) return KVQ_ERR_UNSUPPORTED;  // sinks as a prefix only
+  if ((s = check_attend_tables(k, v, tk, tv, n_tokens)) != KVQ_OK) return s;
   if ((s = check_packed(&k, k_cache)) != KVQ_OK || (s = check_packed(&v, v_cache)) != KVQ_OK) return s;
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;
@@ -395,9 +406,7 @@ kvq_status kvq_attend_noalloc(const kvq_desc* dk, const kvq_desc* dv, const void
   if (!q || !out) return KVQ_ERR_INVALID;
   if (!aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_ALIGN;
   if (attend_workspace_bytes(k, q_heads, n_tokens) > attend_scratch_bytes()) return KVQ_ERR_UNSUPPORTED;
-  if ((s = check_tables(&k, tk, k.rope ? (n_tokens < k.n_sink ? n_tokens : k.n_sink) : 0)) != KVQ_OK) return s;
-  if ((s = check_tables(&v, tv, 0)) != KVQ_OK) return s;
-  if (tk->sink_pos || tv->sink_pos) return KVQ_ERR_UNSUPPORTED;  // sinks as a prefix only
+  if ((s = check_attend_tables(k, v, tk, tv, n_tokens)) != KVQ_OK) return s;
   if ((s = check_packed(&k, k_cache)) != KVQ_OK || (s = check_packed(&v, v_cache)) != KVQ_OK) return s;
   LaunchCtx ctx;
   if ((s = get_ctx(&ctx)) != KVQ_OK) return s;

@@ -34,6 +34,7 @@ constexpr int kThreads = 128;  // part: one token each, then 32 channel quads x 
 
 struct AttnArgs {
   int B, H, Hq, GQ, t_cap, n_tok, n_chunks, n_sink, rot;
+  const int32_t* list;  // sink positions [B][n_sink] (-1 unused), or nullptr: the positions < n_sink
   float rscale;  // fp32(1/sqrt(D))
   const float* scores;  // [B][Hq][n_tok]
   const uint8_t* vcodes;
@@ -218,11 +219,14 @@ __global__ void __launch_bounds__(kThreads) k_attend_combine(const AttnArgs a) {
   nat[a.vperm ? a.vperm[static_cast<size_t>(h) * D + j] & (D - 1) : j] = y;
   __syncthreads();
   float o = nat[j];
-  // sink rows, verbatim values weighted by their softmax probability
-  const int ns = min(a.n_sink, a.n_tok);
+  // sink rows, verbatim values weighted by their softmax probability (their
+  // scores are in the score array and their weights in L; their codes decode to 0)
+  const int ns = a.list ? a.n_sink : min(a.n_sink, a.n_tok);
   const float* sv = a.scores + static_cast<size_t>(bq) * a.n_tok;
   for (int n = 0; n < ns; ++n) {
-    const float p = __expf(sv[n] - M) * invL;
+    const int m = a.list ? a.list[static_cast<size_t>(b) * a.n_sink + n] : n;
+    if (m < 0 || m >= a.n_tok) continue;
+    const float p = __expf(sv[m] - M) * invL;
     o = fmaf(p, __half2float(a.vsink[((static_cast<size_t>(b) * a.H + h) * a.n_sink + n) * D + j]), o);
   }
   a.out[static_cast<size_t>(bq) * D + j] = o;
@@ -311,6 +315,8 @@ struct FusedCfg {
 
 struct FusedArgs {
   int B, H, Hq, t_cap, n_tok, n_sink, rot, blocks, blocks_per_chunk, n_chunks;
+  const int32_t* list;  // listed sinks [B][n_list] (n_sink is then 0), or nullptr
+  int n_list;           // <= 32: lane k holds entry k
   float scale, rscale;
   const __half* q;
   const int16_t* kperm;
@@ -386,6 +392,12 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend
   const int my_n = nk > warp ? (nk - warp + kFWarps - 1) / kFWarps : 0;  // blocks k_begin + warp + 8 i
   const size_t rec0 = static_cast<size_t>(bh) * a.t_cap;
   const uint32_t wbase = smem_u32(fdyn) + warp * (S * C::STAGE);
+  // listed sinks: lane k holds position k of this sequence's list (INT_MAX for none)
+  int my_list = 0x7fffffff;
+  if (a.list && lane < a.n_list) {
+    const int m = __ldg(a.list + static_cast<size_t>(b) * a.n_list + lane);
+    my_list = m >= 0 ? m : 0x7fffffff;
+  }
   // The merge kernel may launch once every CTA of this grid has started (all are resident by then, so its
   // CTAs never hold slots this grid still needs); it runs its input-only prologue beside this grid and
   // waits for this grid's completion before reading any partial.
@@ -466,10 +478,11 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend
   const int srcA = 8 * tig + (g >> 1), srcB = srcA + 4;
   const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;  // column g: digit hi (low halves) or lo
 
-  // one 16-token block; INTERIOR: no sink and no position past n_tok in it
+  // one 16-token block; INTERIOR: no sink and no position past n_tok in it;
+  // lbits: the block's listed positions (bit t: position n0 + t)
   // shared-memory reads as plain loads, so the compiler may schedule them around the products
   auto ld4 = [](const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); };
-  auto block = [&](auto interior, int n0, const uint8_t* kcb) {
+  auto block = [&](auto interior, int n0, const uint8_t* kcb, uint32_t lbits) {
     constexpr bool INTERIOR = decltype(interior)::value;
     const uint8_t* vcb = kcb + kFBlock * RB;
     const uint8_t* kzb = vcb + kFBlock * RB;
@@ -501,8 +514,8 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend
       for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
     bool va = true, vb = true;
     if constexpr (!INTERIOR) {
-      va = n0 + g >= a.n_sink && n0 + g < a.n_tok;
-      vb = n0 + g + 8 >= a.n_sink && n0 + g + 8 < a.n_tok;
+      va = n0 + g >= a.n_sink && n0 + g < a.n_tok && !((lbits >> g) & 1u);
+      vb = n0 + g + 8 >= a.n_sink && n0 + g + 8 < a.n_tok && !((lbits >> (g + 8)) & 1u);
     }
     const float2 kza = h2f(ld4(kzb + 4 * g)), kzb2 = h2f(ld4(kzb + 4 * (g + 8)));
     float2 vza = h2f(ld4(vzb + 4 * g)), vzb2 = h2f(ld4(vzb + 4 * (g + 8)));
@@ -603,8 +616,13 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend
     __syncwarp();                  // ... and every other lane's
     const int n0 = n_first + i * static_cast<int>(kStep);
     const uint8_t* kcb = fdyn + (warp * S + st) * C::STAGE;
-    if (n0 >= a.n_sink && n0 + kFBlock <= a.n_tok) block(std::true_type{}, n0, kcb);
-    else block(std::false_type{}, n0, kcb);
+    uint32_t lbits = 0;
+    if (a.list) {  // uniform over the grid
+      const bool in = my_list >= n0 && my_list < n0 + kFBlock;
+      lbits = __reduce_or_sync(0xffffffffu, in ? 1u << (my_list - n0) : 0u);
+    }
+    if (lbits == 0 && n0 >= a.n_sink && n0 + kFBlock <= a.n_tok) block(std::true_type{}, n0, kcb, 0u);
+    else block(std::false_type{}, n0, kcb, lbits);
     __syncwarp();  // every lane has read the stage
     if (i + S < my_n) issue(i + S, st);
     cp_async_commit();
@@ -680,6 +698,7 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend
 
 struct MergeArgs {
   int B, H, Hq, GQ, n_tok, n_sink, n_chunks, rot, krope;
+  const int32_t* list;  // sink positions [B][n_sink] (-1 unused), or nullptr: the positions < n_sink
   float scale, rscale;
   const __half* q;
   const __half* ksink;
@@ -706,15 +725,23 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
   const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
   const int bq = blockIdx.x;
   const int b = bq / a.Hq, qh = bq % a.Hq, h = qh / a.GQ;
-  const int ns = min(a.n_sink, a.n_tok);
+  // sink n sits at position n, or at list entry n (skipped when -1 or past n_tok: score -inf)
+  const int ns = a.list ? a.n_sink : min(a.n_sink, a.n_tok);
+  const int32_t* lst = a.list ? a.list + static_cast<size_t>(b) * a.n_sink : nullptr;
+  auto sink_at = [&](int n) { return lst ? lst[n] : n; };
   const size_t vh = static_cast<size_t>(b) * a.H + h;
   const int pj = a.vperm ? a.vperm[static_cast<size_t>(h) * D + j] & (D - 1) : j;
   qraw[j] = __half2float(a.q[static_cast<size_t>(bq) * D + j]);
   __syncthreads();
   float mloc = -INFINITY;
   for (int n = warp; n < ns; n += kThreads / 32) {
+    const int m = sink_at(n);
+    if (m < 0 || m >= a.n_tok) {
+      if (lane == 0) ts[n] = -INFINITY;
+      continue;
+    }
     const float s = sink_dot(qraw, a.ksink + (vh * a.n_sink + n) * D,
-                             a.krope ? a.rope_cs + static_cast<size_t>(n) * D : nullptr, lane, a.krope == 2) *
+                             a.krope ? a.rope_cs + static_cast<size_t>(m) * D : nullptr, lane, a.krope == 2) *
                     a.scale;
     if (lane == 0) ts[n] = s;
     mloc = fmaxf(mloc, s * kLog2e);
@@ -722,8 +749,10 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
   constexpr int kPre = 4;  // sink values held in registers from before the wait
   float sv[kPre];
 #pragma unroll
-  for (int n = 0; n < kPre; ++n)
-    sv[n] = n < ns ? __half2float(a.vsink[(vh * a.n_sink + n) * D + j]) : 0.0f;
+  for (int n = 0; n < kPre; ++n) {
+    const int m = n < ns ? sink_at(n) : -1;
+    sv[n] = m >= 0 && m < a.n_tok ? __half2float(a.vsink[(vh * a.n_sink + n) * D + j]) : 0.0f;
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the fused kernel's partials are complete
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + static_cast<size_t>(bq) * a.n_chunks;
   const float* pa = a.part_acc + static_cast<size_t>(bq) * a.n_chunks * D;
@@ -751,7 +780,8 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
       acc = __fmaf_rn(v[u], f, acc);
     }
   }
-  for (int n = 0; n < ns; ++n) L += ex2_approx(__fmaf_rn(ts[n], kLog2e, -M));
+  for (int n = 0; n < ns; ++n)
+    if (ts[n] > -INFINITY) L += ex2_approx(__fmaf_rn(ts[n], kLog2e, -M));
   const float invL = 1.0f / L;
   float y = acc * invL;  // sum_n p_n y_n, channel j of the rotated basis
   if (a.rot == KVQ_ROT_FWHT_HEAD) {  // x = H y / sqrt(D), Sylvester order, strides 1 .. 64
@@ -772,8 +802,9 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
   float o = nat[j];
 #pragma unroll
   for (int n = 0; n < kPre; ++n)
-    if (n < ns) o = __fmaf_rn(ex2_approx(__fmaf_rn(ts[n], kLog2e, -M)) * invL, sv[n], o);
+    if (n < ns && ts[n] > -INFINITY) o = __fmaf_rn(ex2_approx(__fmaf_rn(ts[n], kLog2e, -M)) * invL, sv[n], o);
   for (int n = kPre; n < ns; ++n) {
+    if (!(ts[n] > -INFINITY)) continue;
     const float p = ex2_approx(__fmaf_rn(ts[n], kLog2e, -M)) * invL;
     o = __fmaf_rn(p, __half2float(a.vsink[(vh * a.n_sink + n) * D + j]), o);
   }
@@ -823,8 +854,10 @@ kvq_status launch_merge(const MergeArgs& ma, unsigned grid, cudaStream_t st) {
   return launch_status();
 }
 
-bool fused_path(int bits, int group, int n_sink) {
-  return (bits == 2 || bits == 4) && group == 128 && n_sink <= kFMaxSinks;
+// Listed sinks take the fused path up to 32 entries (one per lane of a warp).
+constexpr int kFMaxListed = 32;
+bool fused_path(int bits, int group, int n_sink, bool listed) {
+  return (bits == 2 || bits == 4) && group == 128 && n_sink <= (listed ? kFMaxListed : kFMaxSinks);
 }
 
 int fused_tiles(int n_tokens) { return (n_tokens + kFBlock - 1) / kFBlock; }
@@ -861,21 +894,27 @@ void* attend_scratch() {
 }
 
 size_t attend_workspace_bytes(const kvq_desc& dk, int q_heads, int n_tokens) {
+  // enough for the prefix and the list form of these sinks (they take different paths above 32 sinks)
   const size_t bq = static_cast<size_t>(dk.batch) * q_heads;
-  if (fused_path(dk.bits, dk.group, dk.n_sink)) {  // chunk partials only; chunks <= min(tiles, kFMaxChunks)
+  size_t fused = 0, other = 0;
+  if (fused_path(dk.bits, dk.group, dk.n_sink, false)) {  // chunk partials only; chunks <= min(tiles, kFMaxChunks)
     const int tiles = fused_tiles(n_tokens);
     const size_t n_chunks = static_cast<size_t>(tiles < kFMaxChunks ? tiles : kFMaxChunks);
-    return align256(bq * n_chunks * D * 4) + align256(bq * n_chunks * 2 * 4);
+    fused = align256(bq * n_chunks * D * 4) + align256(bq * n_chunks * 2 * 4);
   }
-  const size_t n_chunks = (static_cast<size_t>(n_tokens) + kCh * kSub - 1) / (kCh * kSub);
-  return align256(bq * n_tokens * 4) + align256(bq * n_chunks * D * 4) + align256(bq * n_chunks * 2 * 4);
+  if (!fused_path(dk.bits, dk.group, dk.n_sink, true)) {
+    const size_t n_chunks = (static_cast<size_t>(n_tokens) + kCh * kSub - 1) / (kCh * kSub);
+    other = align256(bq * n_tokens * 4) + align256(bq * n_chunks * D * 4) + align256(bq * n_chunks * 2 * 4);
+  }
+  return fused > other ? fused : other;
 }
 
 kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, int q_heads,
                          const kvq_packed& kc, const kvq_tables& tk, const kvq_packed& vc, const kvq_tables& tv,
                          int n_tokens, float scale, float* out, void* ws, cudaStream_t st, const LaunchCtx& ctx) {
   const size_t bq = static_cast<size_t>(dk.batch) * q_heads;
-  if (fused_path(dk.bits, dk.group, dk.n_sink)) {
+  const int32_t* list = dk.n_sink > 0 ? tk.sink_pos : nullptr;  // listed sinks (both caches' list)
+  if (fused_path(dk.bits, dk.group, dk.n_sink, list != nullptr)) {
     const int tiles = fused_tiles(n_tokens);
     const int max_chunks = tiles < kFMaxChunks ? tiles : kFMaxChunks;
     FusedArgs fa{};
@@ -884,7 +923,9 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
     fa.Hq = q_heads;
     fa.t_cap = dk.t_cap;
     fa.n_tok = n_tokens;
-    fa.n_sink = dk.n_sink;
+    fa.n_sink = list ? 0 : dk.n_sink;
+    fa.list = list;
+    fa.n_list = list ? dk.n_sink : 0;
     fa.rot = dk.rot;
     fa.blocks = tiles;
     fa.scale = scale;
@@ -908,6 +949,7 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
     ma.GQ = gq;
     ma.n_tok = n_tokens;
     ma.n_sink = dk.n_sink;
+    ma.list = list;
     ma.n_chunks = fa.n_chunks;
     ma.rot = dv.rot;
     ma.krope = dk.rope;
@@ -932,6 +974,7 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
   a.n_tok = n_tokens;
   a.n_chunks = (n_tokens + kCh * kSub - 1) / (kCh * kSub);
   a.n_sink = dv.n_sink;
+  a.list = list;
   a.rot = dv.rot;
   a.rscale = static_cast<float>(1.0 / sqrt(static_cast<double>(D)));
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -946,8 +989,13 @@ kvq_status launch_attend(const kvq_desc& dk, const kvq_desc& dv, const void* q, 
   a.vsink = static_cast<const __half*>(vc.sink);
   a.vperm = tv.perm;
   a.out = out;
-  kvq_status s = launch_score(dk, q, q_heads, kc, tk, n_tokens, scale, scores, st, ctx);
+  // scores of every slot from its codes; with a list, the listed slots' exact scores
+  // over them (their codes are zero, so their values enter only through the combine)
+  kvq_desc dm = dk;
+  if (list) dm.n_sink = 0;
+  kvq_status s = launch_score(dm, q, q_heads, kc, tk, n_tokens, scale, scores, st, ctx);
   if (s != KVQ_OK) return s;
+  if (list && (s = launch_sink_fix_score(dk, q, q_heads, kc, tk, n_tokens, scale, scores, st)) != KVQ_OK) return s;
   if ((s = dispatch_part(dv.bits, dv.group, a, st)) != KVQ_OK) return s;
   k_attend_combine<<<static_cast<unsigned>(bq), kThreads, 0, st>>>(a);
   return launch_status();

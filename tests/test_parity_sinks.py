@@ -313,7 +313,8 @@ def test_list_calibrate(K, orc):
         assert np.array_equal(perm, ref), rope
 
 
-def test_list_attend_unsupported(K):
+def test_list_attend_needs_both_tables(K):
+    """A sink list goes with both caches; naming it for the keys only is an error."""
     from kv_cache_rotation_b200 import torch_api as TA
     B, H, T, D = 1, 2, 16, 128
     dk = TA.make_desc(batch=B, heads=H, head_dim=D, tokens=T, t_cap=T, bits=2, group=128, rope=1, n_sink=2)
@@ -327,10 +328,14 @@ def test_list_attend_unsupported(K):
     ws = TA.attend_workspace(dk, dv, H, T)
     with pytest.raises(K.KvqError) as e:
         TA.attend(dk, dv, q, kp, tk, vp, tv, T, 0.1, out, ws)
-    assert e.value.status == K.KVQ_ERR_UNSUPPORTED
+    assert e.value.status == K.KVQ_ERR_INVALID
     with pytest.raises(K.KvqError) as e:
         TA.attend_noalloc(dk, dv, q, kp, tk, vp, tv, T, 0.1, out)
-    assert e.value.status == K.KVQ_ERR_UNSUPPORTED
+    assert e.value.status == K.KVQ_ERR_INVALID
+    tr = TA.make_tables(rope_cs=TA.rope_table(8, D), sink_pos=sp)  # RoPE rows must reach n_tokens
+    with pytest.raises(K.KvqError) as e:
+        TA.attend(dk, dv, q, kp, tr, vp, TA.make_tables(sink_pos=sp), T, 0.1, out, ws)
+    assert e.value.status == K.KVQ_ERR_INVALID
 
 
 def test_detect_then_encode_end_to_end(K, orc):
