@@ -31,6 +31,8 @@ CASES = [
     ("no_rotation", 1, 2, 2, 64, 64, 2, 64, 2, True, "none"),
     ("single_token", 2, 2, 8, 16, 1, 2, 128, 0, False, "fwht_head"),
     ("sinks_only", 1, 2, 4, 16, 3, 2, 64, 4, True, "fwht_head"),
+    ("gqa4_bits4_g32", 1, 2, 8, 100, 97, 4, 32, 2, True, "fwht_head"),
+    ("gqa1_bits2_g32", 2, 2, 2, 150, 150, 2, 32, 0, False, "fwht_head"),
     # one group per record, 2 or 4 bits: the fused single-pass kernel
     ("fused_gqa4_perm_40_chunks", 1, 1, 4, 5000, 4999, 2, 128, 4, True, "fwht_head"),
     ("fused_gqa2_9_tiles_per_chunk", 2, 16, 32, 10000, 9990, 2, 128, 4, False, "fwht_head"),

@@ -90,6 +90,13 @@ def test_score_bits(K, orc, bits, group):
     run_score_case(K, orc, w, W.random_perm(w.H, w.D, 2))
 
 
+@pytest.mark.parametrize("bits,group,gq", [(2, 32, 2), (4, 32, 1), (4, 64, 8), (2, 64, 4)])
+def test_score_mma_groups(K, orc, bits, group, gq):
+    """The tensor-core score with 2 and 4 quantization groups per record (head_dim 128)."""
+    w = W.scaled(W.WORKLOADS["decode_score"], B=2, H=2, Hq=2 * gq, T=161, bits=bits, group=group, n_sink=3)
+    run_score_case(K, orc, w, W.random_perm(w.H, w.D, 9))
+
+
 def test_score_no_rotation(K, orc):
     w = W.scaled(W.WORKLOADS["decode_score"], B=1, H=2, Hq=2, T=70, n_sink=0)
     run_score_case(K, orc, w, None, rot="none")
