@@ -103,22 +103,10 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 // Pull a tensor tile into L2 ahead of its TMA load (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
                "r"(smem_u32(src)), "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int y, int z, const void* src) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, int x, int y, int z, int w, const void* src) {
@@ -164,11 +152,6 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
 
 // ---------------------------------------------------------------- smem access
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -198,14 +181,6 @@ __device__ __forceinline__ float lds32f(uint32_t addr) {
 }
 __device__ __forceinline__ void sts32f(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void sts16(uint32_t addr, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
-}
-__device__ __forceinline__ uint16_t lds16(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
 }
 
 // Byte offset of 16-byte chunk c of row r in a TMA tile written with
@@ -302,22 +277,6 @@ __device__ __forceinline__ void fwht_pairs(float2 (&P)[V / 2]) {
   }
 }
 
-// Strides 4 .. V/2 of the FWHT on the register-pair layout above (strides 1
-// and 2 already applied).
-template <int V>
-__device__ __forceinline__ void fwht_pairs_from4(float2 (&P)[V / 2]) {
-#pragma unroll
-  for (int hs = 1; hs < V / 4; hs <<= 1) {
-#pragma unroll
-    for (int g = 0; g < V / 4; ++g) {
-      if ((g & hs) == 0) {
-        bfly(P[2 * g], P[2 * (g + hs)]);
-        bfly(P[2 * g + 1], P[2 * (g + hs) + 1]);
-      }
-    }
-  }
-}
-
 // N words (N a multiple of 8) of global memory <-> registers: 256-bit accesses
 // when the address is 32-byte aligned, 128-bit ones otherwise. Loads use the
 // read-only path and do not allocate in L1.
@@ -394,14 +353,6 @@ __device__ __forceinline__ float2 rope_half_inv2(float2 own, float2 cc, float2 s
   return upper ? fma2(own, cc, mul2(oth, f2(-ss.x, -ss.y))) : fma2(own, cc, mul2(oth, ss));
 }
 
-// Inverse rotation (decode; tolerance-checked, any rounding order is fine).
-__device__ __forceinline__ void rope_inv(float& y0, float& y1, float c, float s) {
-  const float x0 = __fmaf_rn(y0, c, __fmul_rn(y1, s));
-  const float x1 = __fmaf_rn(y1, c, -__fmul_rn(y0, s));
-  y0 = x0;
-  y1 = x1;
-}
-
 // ---------------------------------------------------------------- min/max
 __device__ __forceinline__ float min3f(float a, float b, float c) {
   float d;
@@ -412,17 +363,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-// Min and max of v[off .. off+n) (n even, n >= 2).
-template <int N>
-__device__ __forceinline__ void minmax_range(const float (&v)[N], int off, int n, float& mn, float& mx) {
-  mn = fminf(v[off], v[off + 1]);
-  mx = fmaxf(v[off], v[off + 1]);
-#pragma unroll
-  for (int j = 2; j + 1 < n; j += 2) {
-    mn = min3f(mn, v[off + j], v[off + j + 1]);
-    mx = max3f(mx, v[off + j], v[off + j + 1]);
-  }
 }
 
 // Scale / zero of one min-max group from its (canonicalised) min and max:
@@ -447,26 +387,8 @@ __device__ __forceinline__ QParams minmax_params(float mn, float mx) {
   p.sz = __halves2half2(sh, zh);
   return p;
 }
-// code = round-half-even of the exact product fp32(p - Z) * R; the result's
-// fp32 bit pattern is kMagicBits + code (code in [0, 2^BITS - 1]).
-__device__ __forceinline__ uint32_t quant_code(float p, float Z, float R) {
-  const float d = __fsub_rn(p, Z);
-  return __float_as_uint(__fmaf_rn(d, R, kMagicRound)) - kMagicBits;
-}
 
 // ---------------------------------------------------------------- packing
-// Pack N codes (each < 2^BITS) LSB-first into N*BITS/32 words.
-template <int N, int BITS>
-__device__ __forceinline__ void pack_codes(const uint32_t (&c)[N], uint32_t (&w)[N * BITS / 32]) {
-#pragma unroll
-  for (int i = 0; i < N * BITS / 32; ++i) w[i] = 0u;
-#pragma unroll
-  for (int j = 0; j < N; ++j) {
-    const int p = j * BITS;
-    w[p >> 5] |= c[j] << (p & 31);
-    if ((p & 31) + BITS > 32) w[(p >> 5) + 1] |= c[j] >> (32 - (p & 31));
-  }
-}
 // Code j of a packed word array.
 template <int BITS, int NW>
 __device__ __forceinline__ uint32_t unpack_code(const uint32_t (&w)[NW], int j) {
