@@ -234,18 +234,21 @@ class ScoreCache:
 
 
 class AttendStep:
-    """Decode-step attention at the Llama-3-8B shape: append one token to the
-    K and the V cache, then out = softmax(q . k) . v over every slot."""
+    """Decode-step attention: append one token to the K and the V cache, then
+    out = softmax(q . k) . v over every slot (the Llama-3-8B shape by default;
+    the Llama-2-7B shape runs the three-kernel form)."""
 
-    workload = "llama3_8b_gqa_attend"
-    kernels_per_step = 4  # two appends, the fused attention kernel and its merge
-    # K and V caches are 75 MB, less than the 126 MB L2: flush it before every step
+    # K and V caches are 75 MB (Llama-3-8B) or 84 MB (Llama-2-7B), less than the 126 MB L2: flush it before every step
     l2_flush = True
 
-    def __init__(self, device):
+    def __init__(self, device, workload="llama3_8b_gqa_attend"):
         import torch
         from kv_cache_rotation_b200 import torch_api as TA
+        self.workload = workload
         ws = W.WORKLOADS[self.workload]
+        fused = ws.group == 128 and ws.bits in (2, 4)
+        # two appends, then the fused attention kernel and its merge, or the scores, the chunk sums and the merge
+        self.kernels_per_step = 4 if fused else 5
         self.k = ScoreCache(ws, device, "k")
         self.v = ScoreCache(ws, device, "v")
         n = self.k.n_tok
@@ -258,7 +261,8 @@ class AttendStep:
                     "attend": self.k.alg_cache + self.v.alg_cache + q_out}
         self.fp16_equiv = {"append_k": self.k.fp16_append, "append_v": self.v.fp16_append,
                            "attend": 2 * self.k.fp16_score}
-        self.kernels = {"append_k": "k_encode_head", "append_v": "k_encode_head", "attend": "k_attend_fused"}
+        self.kernels = {"append_k": "k_encode_head", "append_v": "k_encode_head",
+                        "attend": "k_attend_fused" if fused else "k_attend_part"}
         self.fp32_ops = {}
         self.names = list(self.alg)
         torch.cuda.synchronize(device)
@@ -547,8 +551,8 @@ def make_step(workload, device, batch=None):
         return Step(device)
     if workload == "decode_score":
         return DecodeScoreStep(device)
-    if workload == "llama3_8b_gqa_attend":
-        return AttendStep(device)
+    if workload in ("llama3_8b_gqa_attend", "llama2_7b_mha_attend"):
+        return AttendStep(device, workload)
     if workload == "llama3_8b_calibrate":
         return CalibrateStep(device)
     if workload == "llama3_8b_pair_energy":
@@ -931,7 +935,7 @@ def _other_config(name, n_gpus):
     return {"workload": name, "batch": w.B, "kv_heads": w.H, "head_dim": w.D, "tokens": w.T, "q_heads": w.Hq,
             "rotation": w.rot, "quant": w.quant, "bits": w.bits, "group": w.group, "n_sink": w.n_sink,
             "perm": w.perm, "l2": ("flushed before every step by a 512 MB read (outside the timed steps)"
-                                   if name == "llama3_8b_gqa_attend" else
+                                   if name in ("llama3_8b_gqa_attend", "llama2_7b_mha_attend") else
                                    "no flush (inputs larger than L2)" if name != "tiny" else "L2-resident"),
             "parallelism": f"replicas x{n_gpus}"}
 
@@ -952,7 +956,8 @@ def main():
                              "isoquant_dyn_batch", "decode_score",
                              "llama3_8b_gqa_group_score", "llama2_7b_sink_detect",
                              "decode_score_literal", "llama3_8b_gqa_score_literal",
-                             "llama3_8b_gqa_attend", "llama3_8b_calibrate", "llama3_8b_pair_energy", "tiny"],
+                             "llama3_8b_gqa_attend", "llama2_7b_mha_attend", "llama3_8b_calibrate",
+                             "llama3_8b_pair_energy", "tiny"],
                     help="which workload a step runs (the headline line is llama3_8b_gqa)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch of an encode/decode workload (small profiling captures)")

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kThreads) k_attend_part(const AttnArgs a) {
   constexpr int RB = D * BITS / 8;
   constexpr uint32_t MASK = (1u << BITS) - 1u;
   __shared__ __align__(16) float wsm[kCh][NG][GQ];  // p_n * S_ng of the sub-chunk
-  __shared__ __align__(16) uint32_t csm[kCh][RB / 4];
+  __shared__ __align__(16) uint32_t csm[2][kCh][RB / 4];  // value records: this sub-chunk's and the next one's
   __shared__ float red[4][GQ * (1 + NG)];
   __shared__ float mx_s[4][GQ];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -85,24 +85,50 @@ __global__ void __launch_bounds__(kThreads) k_attend_part(const AttnArgs a) {
     for (int e = 0; e < 4; ++e) acc[r][e] = 0.0f;
   }
 
+  // one sub-chunk ahead: its value records by cp.async into the other csm
+  // buffer (zero past the last token), this thread's token's scores and
+  // scale / zero words into registers
+  float sv_n[GQ];
+  float2 sz_n[NG];
+  auto prefetch = [&](int sub) {
+    const int n0 = (c * kSub + sub) * kCh;
+    const int nn = min(kCh, a.n_tok - n0);
+    const uint8_t* vsrc = a.vcodes + (static_cast<size_t>(bh) * a.t_cap + n0) * RB;
+    const uint32_t dst = smem_u32(&csm[sub & 1][0][0]);
+    for (int i = tid; i < kCh * RB / 16; i += kThreads) {
+      const bool live = i / (RB / 16) < nn;
+      cp_async16(dst + 16 * i, live ? vsrc + 16 * i : vsrc, live ? 16u : 0u);
+    }
+#pragma unroll
+    for (int r = 0; r < GQ; ++r)
+      sv_n[r] = tid < nn ? __ldg(a.scores + (static_cast<size_t>(b) * a.Hq + h * GQ + r) * a.n_tok + n0 + tid)
+                         : -INFINITY;
+#pragma unroll
+    for (int gg = 0; gg < NG; ++gg)
+      sz_n[gg] = tid < nn ? __half22float2(a.vsz[(static_cast<size_t>(bh) * a.t_cap + n0 + tid) * NG + gg])
+                          : make_float2(0.0f, 0.0f);
+  };
+  if (c * kSub * kCh < a.n_tok) prefetch(0);
+  cp_async_commit();
+
   for (int sub = 0; sub < kSub; ++sub) {
     const int n0 = (c * kSub + sub) * kCh;
     if (n0 >= a.n_tok) break;  // uniform over the CTA
     const int nn = min(kCh, a.n_tok - n0);
-    __syncthreads();  // the previous sub-chunk's csm / wsm / red readers are done
-
-    // packed value records (zero past the last token)
-    const uint4* vsrc = reinterpret_cast<const uint4*>(a.vcodes + (static_cast<size_t>(bh) * a.t_cap + n0) * RB);
-    for (int i = tid; i < kCh * RB / 16; i += kThreads) {
-      const int n = i / (RB / 16);
-      reinterpret_cast<uint4*>(&csm[0][0])[i] = n < nn ? __ldg(vsrc + i) : make_uint4(0, 0, 0, 0);
-    }
-    // scores (thread = token), the sub-chunk max per query head
     float sv[GQ];
+    float2 sz[NG];
+#pragma unroll
+    for (int r = 0; r < GQ; ++r) sv[r] = sv_n[r];
+#pragma unroll
+    for (int gg = 0; gg < NG; ++gg) sz[gg] = sz_n[gg];
+    __syncthreads();  // the previous sub-chunk's csm / wsm / red readers are done
+    if (sub + 1 < kSub && n0 + kCh < a.n_tok) prefetch(sub + 1);
+    cp_async_commit();  // one group per sub-chunk (empty at the end)
+    const uint32_t(*cs)[RB / 4] = csm[sub & 1];
+
+    // scores (thread = token), the sub-chunk max per query head
 #pragma unroll
     for (int r = 0; r < GQ; ++r) {
-      const float* sp = a.scores + (static_cast<size_t>(b) * a.Hq + h * GQ + r) * a.n_tok + n0;
-      sv[r] = tid < nn ? __ldg(sp + tid) : -INFINITY;
       const float v = warp_max(sv[r]);
       if (lane == 0) mx_s[warp][r] = v;
     }
@@ -115,11 +141,6 @@ __global__ void __launch_bounds__(kThreads) k_attend_part(const AttnArgs a) {
     }
     // p_n = e^(s_n - m); w_n = p_n S_g; sub-chunk sums of p_n and p_n Z_g
     {
-      float2 sz[NG];
-#pragma unroll
-      for (int gg = 0; gg < NG; ++gg)
-        sz[gg] = tid < nn ? __half22float2(a.vsz[(static_cast<size_t>(bh) * a.t_cap + n0 + tid) * NG + gg])
-                          : make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int r = 0; r < GQ; ++r) {
         const float p = tid < nn ? __expf(sv[r] - m_new[r]) : 0.0f;
@@ -133,6 +154,7 @@ __global__ void __launch_bounds__(kThreads) k_attend_part(const AttnArgs a) {
         }
       }
     }
+    cp_async_wait_group<1>();  // this sub-chunk's records (the next one's may still be in flight)
     __syncthreads();
 #pragma unroll
     for (int r = 0; r < GQ; ++r) {
@@ -145,9 +167,9 @@ __global__ void __launch_bounds__(kThreads) k_attend_part(const AttnArgs a) {
     }
     // sum_n w_n c_n for this thread's channels and token phase
     for (int n = ph; n < nn; n += 4) {
-      uint32_t v = csm[n][wi] >> sh;
+      uint32_t v = cs[n][wi] >> sh;
       if constexpr ((4 * BITS) % 8 != 0 || 32 % (4 * BITS) != 0) {
-        if (sh + 4 * BITS > 32) v |= csm[n][wi + 1] << (32 - sh);
+        if (sh + 4 * BITS > 32) v |= cs[n][wi + 1] << (32 - sh);
       }
       float cf[4];
 #pragma unroll

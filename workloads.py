@@ -90,6 +90,11 @@ WORKLOADS = {
     # RoPE), one token appended to each, then softmax(q . k) . v.
     "llama3_8b_gqa_attend": Workload("llama3_8b_gqa_attend", B=4, H=8, T=32768, bits=2, group=128, n_sink=4,
                                      seed=7, Hq=32, append=1),
+    # Decode-step attention at the Llama-2-7B shape (32 heads, MHA, 4096 cached
+    # tokens + 1, 2-bit group 64, permutation, 4 sinks): two groups per record,
+    # so the three-kernel form (scores, chunked sums, merge).
+    "llama2_7b_mha_attend": Workload("llama2_7b_mha_attend", B=8, H=32, T=4096, bits=2, group=64, n_sink=4,
+                                     perm=True, seed=8, Hq=32, append=1),
 }
 
 
