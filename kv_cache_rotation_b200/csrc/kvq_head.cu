@@ -4,7 +4,9 @@
 // attention sinks):
 //   RoPE (keys) -> channel permutation -> normalised FWHT over head_dim
 //   -> per-group min-max quantization with fp16 (scale, zero) -> LSB-first packing.
-// Decode is the inverse.
+// Decode is the inverse. The literal per-token score over the same cache
+// (k_score_literal, at the end of this file) reuses the decode's unpacking
+// and inverse transform.
 //
 // Two lanes of a warp share one token-head vector: lane 2i + s holds channels
 // [sV, sV + V), V = D/2, loaded straight from global memory (256-bit loads).
