@@ -387,7 +387,9 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t y, uint32_t msk) {
 
 __device__ __forceinline__ float2 h2f(uint32_t w) { return __half22float2(*reinterpret_cast<const __half2*>(&w)); }
 
-template <int BITS, int GQ>
+// LIST: the sinks are a list (a.list), masked block by block; without it the
+// kernel has no per-block list test at all.
+template <int BITS, int GQ, bool LIST>
 __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend_fused(const FusedArgs a) {
   using C = FusedCfg<BITS>;
   constexpr int D = 128;
@@ -416,7 +418,7 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend
   const uint32_t wbase = smem_u32(fdyn) + warp * (S * C::STAGE);
   // listed sinks: lane k holds position k of this sequence's list (INT_MAX for none)
   int my_list = 0x7fffffff;
-  if (a.list && lane < a.n_list) {
+  if (LIST && lane < a.n_list) {
     const int m = __ldg(a.list + static_cast<size_t>(b) * a.n_list + lane);
     my_list = m >= 0 ? m : 0x7fffffff;
   }
@@ -639,7 +641,7 @@ __global__ void __launch_bounds__(kFThreads, GQ <= 4 ? kFMinBlocks : 1) k_attend
     const int n0 = n_first + i * static_cast<int>(kStep);
     const uint8_t* kcb = fdyn + (warp * S + st) * C::STAGE;
     uint32_t lbits = 0;
-    if (a.list) {  // uniform over the grid
+    if constexpr (LIST) {
       const bool in = my_list >= n0 && my_list < n0 + kFBlock;
       lbits = __reduce_or_sync(0xffffffffu, in ? 1u << (my_list - n0) : 0u);
     }
@@ -833,10 +835,10 @@ __global__ void __launch_bounds__(kThreads) k_attend_merge(const MergeArgs a) {
   a.out[static_cast<size_t>(bq) * D + j] = o;
 }
 
-template <int BITS, int GQ>
+template <int BITS, int GQ, bool LIST>
 kvq_status run_fused(FusedArgs& fa, const LaunchCtx& ctx, cudaStream_t st) {
   constexpr size_t smem = FusedCfg<BITS>::SMEM;
-  const void* fn = reinterpret_cast<const void*>(k_attend_fused<BITS, GQ>);
+  const void* fn = reinterpret_cast<const void*>(k_attend_fused<BITS, GQ, LIST>);
   if (!set_smem_once(fn, smem)) return KVQ_ERR_CUDA;
   const int per_sm = occupancy_once(fn, kFThreads, smem);
   const int bh = fa.B * fa.H;
@@ -844,7 +846,7 @@ kvq_status run_fused(FusedArgs& fa, const LaunchCtx& ctx, cudaStream_t st) {
   want = want < 1 ? 1 : (want > kFMaxChunks ? kFMaxChunks : want);
   fa.blocks_per_chunk = (fa.blocks + want - 1) / want;
   fa.n_chunks = (fa.blocks + fa.blocks_per_chunk - 1) / fa.blocks_per_chunk;
-  k_attend_fused<BITS, GQ><<<dim3(static_cast<unsigned>(fa.n_chunks), static_cast<unsigned>(bh)), kFThreads,
+  k_attend_fused<BITS, GQ, LIST><<<dim3(static_cast<unsigned>(fa.n_chunks), static_cast<unsigned>(bh)), kFThreads,
                              smem, st>>>(fa);
   return launch_status();
 }
@@ -852,10 +854,10 @@ kvq_status run_fused(FusedArgs& fa, const LaunchCtx& ctx, cudaStream_t st) {
 template <int BITS>
 kvq_status fused_by_gq(FusedArgs& fa, int gq, const LaunchCtx& ctx, cudaStream_t st) {
   switch (gq) {
-    case 1: return run_fused<BITS, 1>(fa, ctx, st);
-    case 2: return run_fused<BITS, 2>(fa, ctx, st);
-    case 4: return run_fused<BITS, 4>(fa, ctx, st);
-    case 8: return run_fused<BITS, 8>(fa, ctx, st);
+    case 1: return fa.list ? run_fused<BITS, 1, true>(fa, ctx, st) : run_fused<BITS, 1, false>(fa, ctx, st);
+    case 2: return fa.list ? run_fused<BITS, 2, true>(fa, ctx, st) : run_fused<BITS, 2, false>(fa, ctx, st);
+    case 4: return fa.list ? run_fused<BITS, 4, true>(fa, ctx, st) : run_fused<BITS, 4, false>(fa, ctx, st);
+    case 8: return fa.list ? run_fused<BITS, 8, true>(fa, ctx, st) : run_fused<BITS, 8, false>(fa, ctx, st);
     default: return KVQ_ERR_UNSUPPORTED;
   }
 }
