@@ -144,6 +144,26 @@ def test_attend_argument_checks():
     assert K.kvq_attend(dk, dv4, 256, 16, p, tb, p, tb, 20, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_INVALID
 
 
+def test_attend_workspace_covers_both_sink_forms():
+    """Up to 32 sinks both forms take the same path; above that a list runs the
+    three-kernel form, so the workspace covers the larger of the two layouts."""
+    def ws(n_sink, group=128, n=4097):
+        dk = _desc(batch=4, heads=8, t_cap=n, tokens=0, rope=1, group=group, n_sink=n_sink)
+        dv = _desc(batch=4, heads=8, t_cap=n, tokens=0, rope=0, group=group, n_sink=n_sink)
+        return K.kvq_attend_workspace_bytes(dk, dv, 32, n)
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+    bq, n, d = 4 * 32, 4097, 128
+    chunks_f = min((n + 15) // 16, 256)  # fused: 16-token tiles, at most 256 chunks per query head
+    fused = a256(bq * chunks_f * d * 4) + a256(bq * chunks_f * 2 * 4)
+    chunks_u = (n + 511) // 512  # three kernels: scores, then 512-token chunks
+    three = a256(bq * n * 4) + a256(bq * chunks_u * d * 4) + a256(bq * chunks_u * 2 * 4)
+    assert ws(4) == fused and ws(32) == fused
+    assert ws(40) == max(fused, three)
+    assert ws(4, group=64) == three and ws(40, group=64) == three
+
+
 def test_attend_noalloc_rejects_oversize():
     # 8 sequences x 64 query heads x 32768 tokens: 67 MB of scores alone, more than the 40 MiB scratch
     dk = _desc(batch=8, heads=8, t_cap=32768, tokens=0, rope=0)
