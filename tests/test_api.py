@@ -164,6 +164,24 @@ def test_attend_workspace_covers_both_sink_forms():
     assert ws(4, group=64) == three and ws(40, group=64) == three
 
 
+def test_attend_sink_list_in_both_tables():
+    dk = _desc(t_cap=32, tokens=0, rope=1, n_sink=2)
+    dv = _desc(t_cap=32, tokens=0, rope=0, n_sink=2)
+    p = _packed(dk, sink=4096)
+    ws = K.kvq_attend_workspace_bytes(dk, dv, 16, 20)
+    tk, tv = K.kvq_tables(), K.kvq_tables()
+    tk.rope_cs, tk.rope_rows = 256, 32
+    tk.sink_pos = 1024  # keys listed, values not
+    assert K.kvq_attend(dk, dv, 256, 16, p, tk, p, tv, 20, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_INVALID
+    assert K.kvq_attend_noalloc(dk, dv, 256, 16, p, tk, p, tv, 20, 1.0, 256, 0) == K.KVQ_ERR_INVALID
+    tv.sink_pos = 1024
+    tk.rope_rows = 8  # a list needs RoPE rows up to n_tokens
+    assert K.kvq_attend(dk, dv, 256, 16, p, tk, p, tv, 20, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_INVALID
+    tk.sink_pos = 1026  # 4-byte alignment
+    tk.rope_rows = 32
+    assert K.kvq_attend(dk, dv, 256, 16, p, tk, p, tv, 20, 1.0, 256, 256, ws, 0) == K.KVQ_ERR_ALIGN
+
+
 def test_attend_noalloc_rejects_oversize():
     # 8 sequences x 64 query heads x 32768 tokens: 67 MB of scores alone, more than the 40 MiB scratch
     dk = _desc(batch=8, heads=8, t_cap=32768, tokens=0, rope=0)
